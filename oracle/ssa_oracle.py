@@ -1,0 +1,379 @@
+"""Plain, slow, fp64 CPU oracle of spatial sparse attention (SSA).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+bench's CPU-baseline leg may import this module.  It shares no code with the
+CUDA library and must never be used as a fallback for it.
+
+What it follows (all citations are to the pages as titled):
+
+* Direct3D-S2 (hyper.ai/cn/papers/2505.17412), section "方法", the SSA
+  paragraph: tokens are grouped into m_cmp^3 blocks by their 3D coordinates
+  (not by 1D index); "sparse 3D compression" mean-pools each block's keys and
+  values; "spatial block selection" picks the top-k blocks by the
+  query/compressed-block attention score and runs a second, full attention over
+  every token of the selected blocks; "sparse 3D window" attends only inside
+  non-overlapping m_win^3 windows; the three module outputs are summed with
+  predicted gate weights.
+* LSRM (shuwu5.cn/article/2502.html), "空间块划分与键值压缩": in-block average
+  pooling for the compressed keys/values; "阶段一" for GQA with 32 query and 2
+  KV heads and a Linear+Sigmoid gate.
+
+Readings where the pages are silent (each is also listed in the design notes):
+
+* block / window ids: floor(coord / m), per sequence, numbered in
+  lexicographic (x, y, z) order of the block coordinate, offset by the number
+  of blocks of earlier sequences; members ordered by token index.
+* compression is the mean only (no learned convolution); the stored Kc/Vc is
+  computed as fp32(sum) / fp32(n), then rounded to the storage dtype (bf16
+  round-to-nearest-even) -- "pool_rounding".
+* selection score: softmax probability over the sequence's compressed blocks,
+  summed over the query heads of a GQA group; top-k with ties to the lower
+  block id; k_eff = min(k, blocks in sequence); sel stored ascending, padded -1.
+* all three branches are outputs (cmp, slc, win), combined with per
+  (token, head, branch) gates: the gate value itself (mode 0) or its sigmoid
+  (mode 1).  softmax scale 1/sqrt(d) everywhere; no causal mask; a query's own
+  token is in its window; selection is a constant for the backward; the
+  rounding of Kc/Vc passes the gradient straight through (dKc/dK_i = 1/n_b).
+
+Everything is computed in float64 from the exact input values.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# step 1: binning (Direct3D-S2, "方法": spatially coherent block partition)
+# ----------------------------------------------------------------------------
+
+
+def bin_tokens(coords: np.ndarray, cu_seqlens: np.ndarray, m: int) -> dict:
+    """Partition each sequence's tokens into m^3 cells of the integer grid.
+
+    Returns id [N] (global, compacted), perm [N] (tokens sorted by (id, index)),
+    ptr [B+1] (CSR into perm), cu [S+1] (first id of each sequence) and
+    key [B, 3] (the cell coordinate of each id).
+    """
+    coords = np.asarray(coords, dtype=np.int64)
+    cu_seqlens = np.asarray(cu_seqlens, dtype=np.int64)
+    n = coords.shape[0]
+    ids = np.empty(n, dtype=np.int64)
+    cu = [0]
+    keys = []
+    for s in range(len(cu_seqlens) - 1):
+        a, b = int(cu_seqlens[s]), int(cu_seqlens[s + 1])
+        if b == a:
+            cu.append(cu[-1])
+            continue
+        cell = np.floor_divide(coords[a:b], m)
+        uniq, inv = np.unique(cell, axis=0, return_inverse=True)  # rows sorted lexicographically
+        ids[a:b] = cu[-1] + inv.reshape(-1)
+        cu.append(cu[-1] + len(uniq))
+        keys.append(uniq)
+    total = cu[-1]
+    perm = np.argsort(ids, kind="stable")
+    counts = np.bincount(ids, minlength=total) if n else np.zeros(0, np.int64)
+    ptr = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    key = np.concatenate(keys) if keys else np.zeros((0, 3), np.int64)
+    return {"id": ids, "perm": perm, "ptr": ptr, "cu": np.array(cu, np.int64), "key": key,
+            "count": total}
+
+
+# ----------------------------------------------------------------------------
+# step 2: sparse 3D compression by mean pooling
+# ----------------------------------------------------------------------------
+
+
+def _round_bf16(x32: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 (round to nearest, ties to even) -> value as float64."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def mean_pool(x: np.ndarray, blk: dict, pool_rounding: str) -> np.ndarray:
+    """Per block and KV head, the mean of its members' vectors.
+
+    x: [N, Hkv, d] float64 (exact input values).  Returns [B, Hkv, d] float64.
+    pool_rounding: "bf16" -> bf16(fp32(sum) / fp32(n)); "f32" -> fp32(sum) / fp32(n);
+    "none" -> exact mean (used by derivative checks).
+    """
+    nb = blk["count"]
+    sums = np.zeros((nb,) + x.shape[1:], dtype=np.float64)
+    np.add.at(sums, blk["id"], x)  # members in ascending token order
+    cnt = np.diff(blk["ptr"]).astype(np.float64)
+    if pool_rounding == "none":
+        return sums / cnt[:, None, None]
+    q = sums.astype(np.float32) / cnt.astype(np.float32)[:, None, None]
+    if pool_rounding == "f32":
+        return q.astype(np.float64)
+    if pool_rounding == "bf16":
+        return _round_bf16(q)
+    raise ValueError(pool_rounding)
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+
+def _logsumexp(s: np.ndarray, axis: int = -1) -> np.ndarray:
+    m = np.max(s, axis=axis, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    return (m + np.log(np.sum(np.exp(s - m), axis=axis, keepdims=True))).squeeze(axis)
+
+
+def _seq_of_tokens(cu_seqlens: np.ndarray, n: int) -> np.ndarray:
+    return np.repeat(np.arange(len(cu_seqlens) - 1), np.diff(cu_seqlens))
+
+
+def gate_weights(gates: np.ndarray, gate_mode: int) -> np.ndarray:
+    g = np.asarray(gates, dtype=np.float64)
+    if gate_mode == 0:
+        return g
+    return 1.0 / (1.0 + np.exp(-g))
+
+
+# ----------------------------------------------------------------------------
+# step 3: compressed attention + top-k block selection
+# ----------------------------------------------------------------------------
+
+
+def cmp_attention(q_rows: np.ndarray, kc: np.ndarray, vc: np.ndarray, scale: float):
+    """q_rows [n, G, d] against all compressed blocks kc/vc [B_s, d] of one group.
+
+    Returns lse [n, G], o [n, G, d], p [n, G, B_s] (softmax probabilities)."""
+    s = scale * (q_rows @ kc.T)  # [n, G, B]
+    lse = _logsumexp(s, -1)
+    p = np.exp(s - lse[..., None])
+    o = p @ vc
+    return lse, o, p
+
+
+def topk_blocks(importance: np.ndarray, k: int) -> np.ndarray:
+    """importance [n, B_s] -> local ids of the k_eff largest (ties: lower id),
+    ascending, padded with -1 to k."""
+    n, b = importance.shape
+    keff = min(k, b)
+    order = np.argsort(-importance, axis=1, kind="stable")[:, :keff]
+    order = np.sort(order, axis=1)
+    out = np.full((n, k), -1, dtype=np.int64)
+    out[:, :keff] = order
+    return out
+
+
+# ----------------------------------------------------------------------------
+# steps 4/5: selected-block attention and window attention
+# ----------------------------------------------------------------------------
+
+
+def _attend(q: np.ndarray, kk: np.ndarray, vv: np.ndarray, scale: float):
+    """q [G, d] against keys kk [L, d]; returns lse [G], o [G, d], p [G, L]."""
+    s = scale * (q @ kk.T)
+    lse = _logsumexp(s, -1)
+    p = np.exp(s - lse[:, None])
+    return lse, p @ vv, p
+
+
+def selected_tokens(sel_row: np.ndarray, blk: dict) -> np.ndarray:
+    """Token indices of all members of the selected (global) block ids."""
+    parts = [blk["perm"][blk["ptr"][b]:blk["ptr"][b + 1]] for b in sel_row if b >= 0]
+    return np.concatenate(parts) if parts else np.zeros(0, np.int64)
+
+
+# ----------------------------------------------------------------------------
+# full forward
+# ----------------------------------------------------------------------------
+
+
+class State(dict):
+    pass
+
+
+def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
+            gate_mode, scale=None, pool_rounding="bf16", tokens=None, chunk=256) -> State:
+    """SSA forward.  q [N, Hq, d], k/v [N, Hkv, d] (any float type; converted to
+    float64), gates [N, Hq, 3].
+
+    `tokens` restricts the per-query outputs (lse, o_*, sel, O) to a subset of
+    query tokens (all other rows are NaN / -2); binning and compression are
+    always complete.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    n, _, d = q.shape
+    assert hq % hkv == 0
+    G = hq // hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    cu_seqlens = np.asarray(cu_seqlens, dtype=np.int64)
+    blk = bin_tokens(coords, cu_seqlens, m_cmp)
+    win = bin_tokens(coords, cu_seqlens, m_win)
+    kc = mean_pool(k, blk, pool_rounding)
+    vc = mean_pool(v, blk, pool_rounding)
+    seq = _seq_of_tokens(cu_seqlens, n)
+    if tokens is None:
+        tokens = np.arange(n)
+    tokens = np.asarray(tokens, dtype=np.int64)
+
+    lse = np.full((3, n, hq), np.nan)
+    o = np.full((3, n, hq, d), np.nan)
+    sel = np.full((n, hkv, topk), -2, dtype=np.int64)
+
+    # --- compressed branch + selection, per sequence and group, chunked over tokens
+    for s in range(len(cu_seqlens) - 1):
+        toks = tokens[seq[tokens] == s] if len(tokens) else tokens
+        if len(toks) == 0:
+            continue
+        b0, b1 = int(blk["cu"][s]), int(blk["cu"][s + 1])
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            kcg = kc[b0:b1, g, :]
+            vcg = vc[b0:b1, g, :]
+            for c0 in range(0, len(toks), chunk):
+                tt = toks[c0:c0 + chunk]
+                l_, o_, p_ = cmp_attention(q[tt, hs, :], kcg, vcg, scale)
+                lse[0, tt, hs] = l_
+                o[0, tt, hs, :] = o_
+                imp = p_.sum(axis=1)  # [n, B_s]: probabilities summed over the group's heads
+                loc = topk_blocks(imp, topk)
+                sel[tt, g, :] = np.where(loc >= 0, loc + b0, -1)
+
+    # --- selected-block attention and window attention, per query token and group
+    for t in tokens:
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            js = selected_tokens(sel[t, g], blk)
+            l_, o_, _ = _attend(q[t, hs, :], k[js, g, :], v[js, g, :], scale)
+            lse[1, t, hs] = l_
+            o[1, t, hs, :] = o_
+            w = win["id"][t]
+            jw = win["perm"][win["ptr"][w]:win["ptr"][w + 1]]
+            l_, o_, _ = _attend(q[t, hs, :], k[jw, g, :], v[jw, g, :], scale)
+            lse[2, t, hs] = l_
+            o[2, t, hs, :] = o_
+
+    gw = gate_weights(gates, gate_mode)  # [N, Hq, 3]
+    out = np.einsum("nhc,cnhd->nhd", gw, np.nan_to_num(o))
+    out[np.isnan(o[0, :, :, 0])] = np.nan
+    st = State(blk=blk, win=win, kc=kc, vc=vc, lse=lse, o=o, sel=sel, out=out, scale=scale,
+               q=q, k=k, v=v, gates=np.asarray(gates, np.float64), gate_mode=gate_mode,
+               hq=hq, hkv=hkv, G=G, topk=topk, cu_seqlens=cu_seqlens, tokens=tokens)
+    return st
+
+
+def importance(st: State, t: int, g: int) -> np.ndarray:
+    """fp64 selection score of every block of t's sequence for group g (local ids)."""
+    cu = st["cu_seqlens"]
+    s = int(np.searchsorted(cu, t, side="right") - 1)
+    b0, b1 = int(st["blk"]["cu"][s]), int(st["blk"]["cu"][s + 1])
+    G = st["G"]
+    hs = slice(g * G, (g + 1) * G)
+    _, _, p = cmp_attention(st["q"][t:t + 1, hs, :], st["kc"][b0:b1, g, :], st["vc"][b0:b1, g, :],
+                            st["scale"])
+    return p[0].sum(axis=0)
+
+
+def attend_with_sel(st: State, t: int, g: int, sel_row: np.ndarray):
+    """Selected-branch output of (t, g) for a given selection (used to check the
+    attention itself when a certified near-tie flipped the selection)."""
+    G = st["G"]
+    hs = slice(g * G, (g + 1) * G)
+    js = selected_tokens(np.asarray(sel_row), st["blk"])
+    l_, o_, _ = _attend(st["q"][t, hs, :], st["k"][js, g, :], st["v"][js, g, :], st["scale"])
+    return l_, o_
+
+
+# ----------------------------------------------------------------------------
+# step 7: backward (analytic chain rule of the forward, selection held fixed)
+# ----------------------------------------------------------------------------
+
+
+def backward(st: State, dout: np.ndarray, chunk: int = 256) -> dict:
+    """Gradients of sum(dout * O) w.r.t. q, k, v and gates.  Requires a forward
+    over all tokens.  Returns dq, dk, dv, dgates and the per-branch parts."""
+    q, k, v = st["q"], st["k"], st["v"]
+    n, hq, d = q.shape
+    hkv, G, scale = st["hkv"], st["G"], st["scale"]
+    assert len(st["tokens"]) == n, "backward needs the full forward"
+    blk, win = st["blk"], st["win"]
+    dout = np.asarray(dout, dtype=np.float64)
+    gw = gate_weights(st["gates"], st["gate_mode"])  # [N, Hq, 3]
+    o = st["o"]
+
+    # gates: O = sum_c w_c o_c
+    dots = np.einsum("nhd,cnhd->nhc", dout, o)
+    if st["gate_mode"] == 0:
+        dgates = dots
+    else:
+        dgates = dots * gw * (1.0 - gw)
+
+    dq = {c: np.zeros_like(q) for c in ("cmp", "slc", "win")}
+    dk = {c: np.zeros_like(k) for c in ("cmp", "slc", "win")}
+    dv = {c: np.zeros_like(v) for c in ("cmp", "slc", "win")}
+    nb = blk["count"]
+    dkc = np.zeros((nb, hkv, d))
+    dvc = np.zeros((nb, hkv, d))
+    seq = _seq_of_tokens(st["cu_seqlens"], n)
+
+    def attn_bwd(qr, kk, vv, dor, lse_r):
+        # qr [G, d], kk/vv [L, d], dor [G, d] (gate-weighted), lse_r [G]
+        s = scale * (qr @ kk.T)
+        p = np.exp(s - lse_r[:, None])
+        dp = dor @ vv.T
+        dsum = np.sum(p * dp, axis=1, keepdims=True)
+        ds = p * (dp - dsum)
+        return scale * (ds @ kk), scale * (ds.T @ qr), p.T @ dor
+
+    # compressed branch
+    for s in range(len(st["cu_seqlens"]) - 1):
+        toks = np.nonzero(seq == s)[0]
+        if len(toks) == 0:
+            continue
+        b0, b1 = int(blk["cu"][s]), int(blk["cu"][s + 1])
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            kcg, vcg = st["kc"][b0:b1, g, :], st["vc"][b0:b1, g, :]
+            for c0 in range(0, len(toks), chunk):
+                tt = toks[c0:c0 + chunk]
+                qr = q[tt, hs, :]
+                dor = dout[tt, hs, :] * gw[tt, hs, 0][..., None]
+                sc = scale * (qr @ kcg.T)
+                p = np.exp(sc - st["lse"][0, tt, hs][..., None])
+                dp = dor @ vcg.T
+                dsum = np.sum(p * dp, axis=-1, keepdims=True)
+                ds = p * (dp - dsum)
+                dq["cmp"][tt, hs, :] = scale * (ds @ kcg)
+                dkc[b0:b1, g, :] += scale * np.einsum("ngb,ngd->bd", ds, qr)
+                dvc[b0:b1, g, :] += np.einsum("ngb,ngd->bd", p, dor)
+    cnt = np.diff(blk["ptr"]).astype(np.float64)
+    dk["cmp"] = dkc[blk["id"]] / cnt[blk["id"]][:, None, None]
+    dv["cmp"] = dvc[blk["id"]] / cnt[blk["id"]][:, None, None]
+
+    # selected-block and window branches
+    for t in range(n):
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            js = selected_tokens(st["sel"][t, g], blk)
+            a, b_, c_ = attn_bwd(q[t, hs, :], k[js, g, :], v[js, g, :],
+                                 dout[t, hs, :] * gw[t, hs, 1][:, None], st["lse"][1, t, hs])
+            dq["slc"][t, hs, :] = a
+            np.add.at(dk["slc"][:, g, :], js, b_)
+            np.add.at(dv["slc"][:, g, :], js, c_)
+            w = win["id"][t]
+            jw = win["perm"][win["ptr"][w]:win["ptr"][w + 1]]
+            a, b_, c_ = attn_bwd(q[t, hs, :], k[jw, g, :], v[jw, g, :],
+                                 dout[t, hs, :] * gw[t, hs, 2][:, None], st["lse"][2, t, hs])
+            dq["win"][t, hs, :] = a
+            np.add.at(dk["win"][:, g, :], jw, b_)
+            np.add.at(dv["win"][:, g, :], jw, c_)
+
+    return {
+        "dq": dq["cmp"] + dq["slc"] + dq["win"],
+        "dk": dk["cmp"] + dk["slc"] + dk["win"],
+        "dv": dv["cmp"] + dv["slc"] + dv["win"],
+        "dgates": dgates,
+        "parts": {"dq": dq, "dk": dk, "dv": dv, "dkc": dkc, "dvc": dvc},
+    }
