@@ -1,0 +1,176 @@
+/*
+ * ssa.h -- C ABI of the spatial sparse attention (SSA) library, libssa.so.
+ *
+ * SSA is the attention of Direct3D-S2 (hyper.ai/cn/papers/2505.17412, section
+ * "方法", the SSA paragraph) over the variable-length set of occupied sparse
+ * voxels near a 3D surface.  Three modules run side by side and their outputs
+ * are summed with per-token gate weights:
+ *   - sparse 3D compression: tokens are grouped into m_cmp^3 blocks by their
+ *     integer (x, y, z) and each block's keys/values are mean-pooled;
+ *   - spatial block selection: every query attends to all compressed blocks
+ *     of its sequence, the top-k blocks by that attention score are picked and
+ *     a second, full attention runs over every token of the picked blocks;
+ *   - sparse 3D window: attention only inside non-overlapping m_win^3 windows.
+ * GQA (several query heads per KV head) follows LSRM (shuwu5.cn/article/2502.html,
+ * "阶段一": 32 query heads, 2 KV heads).
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers unless stated; the caller owns
+ *     and allocates every buffer, including the workspace.  The library never
+ *     allocates or frees device memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).  Only ssa_bin and ssa_get_device_status
+ *     synchronise that stream.
+ *   - Errors are returned as ssa_status codes; nothing aborts or throws across
+ *     the ABI.  Argument errors are detected on the host before any launch.
+ *   - N = number of tokens (all sequences), S = number of sequences,
+ *     cu_seqlens = int32 [S+1] prefix offsets (cu_seqlens[0] = 0,
+ *     non-decreasing, cu_seqlens[S] = N); sequence s owns tokens
+ *     cu_seqlens[s] .. cu_seqlens[s+1]-1.  Tokens never attend across sequences.
+ *   - Tensors are token-major and contiguous: Q, O [N, Hq, d]; K, V [N, Hkv, d];
+ *     query head h belongs to KV head (group) h / (Hq/Hkv).
+ *   - Results do not depend on the order of tokens inside a sequence (block,
+ *     window and selected ids are functions of the coordinates only).
+ */
+#ifndef SSA_H
+#define SSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSA_API __attribute__((visibility("default")))
+
+typedef enum ssa_status {
+  SSA_OK = 0,
+  SSA_ERR_INVALID_ARG = 1, /* null pointer, bad size or head layout, m < 1, topk < 1 ... */
+  SSA_ERR_UNSUPPORTED = 2, /* head dim / group size / key width this build does not handle */
+  SSA_ERR_WORKSPACE = 3,   /* ws_bytes smaller than ssa_workspace_size() */
+  SSA_ERR_COORD_RANGE = 4, /* a coordinate outside [0, R) or malformed cu_seqlens (device check) */
+  SSA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  SSA_ERR_TIMEOUT = 6      /* a bounded device wait gave up */
+} ssa_status;
+
+enum { SSA_DTYPE_BF16 = 0, SSA_DTYPE_F32 = 1 };
+enum { SSA_GATE_WEIGHTS = 0, SSA_GATE_LOGITS = 1 };
+enum { SSA_OP_BIN = 0, SSA_OP_FORWARD = 1, SSA_OP_BACKWARD = 2 };
+
+/* Shape and method parameters shared by forward and backward. */
+typedef struct ssa_params {
+  int32_t hq;        /* query heads */
+  int32_t hkv;       /* key/value heads; hq % hkv == 0, G = hq / hkv in {1,2,4,8,16} */
+  int32_t d;         /* head dim: 32 or 64 */
+  int32_t m_cmp;     /* compression block edge (voxels), >= 1 */
+  int32_t m_win;     /* window edge (voxels), >= 1 */
+  int32_t topk;      /* selected blocks per (token, KV head), 1..32 */
+  float scale;       /* softmax scale; 0 means 1/sqrt(d) */
+  int32_t dtype;     /* SSA_DTYPE_BF16 (bf16 storage, fp32 math) or SSA_DTYPE_F32 */
+  int32_t gate_mode; /* SSA_GATE_WEIGHTS: gates are the weights; SSA_GATE_LOGITS: weight = sigmoid(gate) */
+} ssa_params;
+
+/*
+ * One partition of the tokens into cells of edge m (compression blocks or
+ * windows).  Direct3D-S2 "方法": the partition is by 3D coordinate, not by 1D
+ * index.  Cells are numbered per sequence in lexicographic (x, y, z) order of
+ * the cell coordinate floor(coord / m), offset by the cells of earlier
+ * sequences.  Caller-allocated device arrays, filled by ssa_bin:
+ */
+typedef struct ssa_partition {
+  int32_t* id;   /* [N]      cell id of every token */
+  int32_t* perm; /* [N]      tokens sorted by (cell id, token index) */
+  int32_t* ptr;  /* [N+1]    members of cell c are perm[ptr[c] .. ptr[c+1]-1]; count+1 entries used */
+  int32_t* cu;   /* [S+1]    cells of sequence s are cu[s] .. cu[s+1]-1 */
+  int32_t* key;  /* [N, 3]   cell coordinate of cell c (rows 0 .. count-1 used) */
+  int64_t count; /* out: number of cells (B_tot or W_tot) */
+} ssa_partition;
+
+/*
+ * Buffers the forward writes and the backward reads (caller-allocated, device).
+ * B = blk.count.  Layouts are head-major so that one block's rows are contiguous.
+ */
+typedef struct ssa_saved {
+  void* kc;       /* [Hkv, B, d] dtype: mean-pooled keys, fp32(sum)/fp32(n) rounded to dtype */
+  void* vc;       /* [Hkv, B, d] dtype: mean-pooled values */
+  void* ks;       /* [Hkv, N, d] dtype: keys gathered in blk.perm order */
+  void* vs;       /* [Hkv, N, d] dtype: values gathered in blk.perm order */
+  float* o_branch; /* [3, N, Hq, d] fp32: branch outputs (0 compressed, 1 selected, 2 window) */
+  float* lse;     /* [3, N, Hq] natural-log softmax normalisers of the three branches */
+  int32_t* sel;   /* [N, Hkv, topk] selected block ids (global), ascending, padded with -1 */
+} ssa_saved;
+
+/*
+ * ssa_bin -- step 1, coordinate binning (Direct3D-S2 "方法": spatially coherent
+ * block partition into m_cmp^3 blocks and m_win^3 windows).
+ *   coords   int32 [N, 3], 0 <= x, y, z < R
+ *   R        grid resolution, 1 <= R <= 2^20
+ * Fills `blk` (edge m_cmp) and `win` (edge m_win), including their counts.
+ * Bit-exact integer work.  Synchronises `stream` once to return the counts and
+ * the device check (SSA_ERR_COORD_RANGE if a coordinate is outside [0, R) or
+ * cu_seqlens is malformed; outputs are then unspecified but in bounds).
+ * SSA_ERR_UNSUPPORTED if the sort key (sequence bits + 3 x cell bits) exceeds 64 bits.
+ */
+SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                           int32_t R, int32_t m_cmp, int32_t m_win, ssa_partition* blk,
+                           ssa_partition* win, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ssa_forward -- steps 2-6: mean-pool compression; compressed attention of every
+ * query against all blocks of its sequence; top-k block selection by the
+ * softmax probability summed over the query heads of a GQA group (ties go to
+ * the lower block id; k_eff = min(topk, blocks in the sequence)); full
+ * attention over the tokens of the selected blocks; attention inside the
+ * query's window; out = sum_c w_c * o_c with w = gates or sigmoid(gates).
+ *   q [N, Hq, d], k/v [N, Hkv, d] in params->dtype; gates fp32 [N, Hq, 3]
+ *   (branch order: compressed, selected, window); out [N, Hq, d] dtype.
+ *   blk/win: partitions from ssa_bin with the same m_cmp / m_win.
+ * Asynchronous.  Writes every buffer of `saved`.
+ */
+SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                               const ssa_partition* blk, const ssa_partition* win, const void* q,
+                               const void* k, const void* v, const float* gates, void* out,
+                               const ssa_saved* saved, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ssa_backward -- step 7: gradients of sum(dout * out) with the selection held
+ * fixed.  The mean pooling passes gradients through as dK_i += dKc_b / n_b
+ * (its rounding is treated as the identity).
+ *   dout [N, Hq, d] dtype; outputs fp32: dq [N, Hq, d], dk/dv [N, Hkv, d],
+ *   dgates [N, Hq, 3] (w.r.t. the gate inputs, including the sigmoid in
+ *   SSA_GATE_LOGITS mode).  `saved` must come from ssa_forward on the same inputs.
+ * Asynchronous.  Every output element is written (no accumulation into caller data).
+ */
+SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S,
+                                int64_t N, const ssa_partition* blk, const ssa_partition* win,
+                                const void* q, const void* k, const void* v, const float* gates,
+                                const ssa_saved* saved, const void* dout, float* dq, float* dk,
+                                float* dv, float* dgates, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Workspace bytes needed by `op` (SSA_OP_BIN / _FORWARD / _BACKWARD) for the
+ * given sizes; B_tot and W_tot are the partition counts (pass N as an upper
+ * bound before binning).  The workspace must be 256-byte aligned.  Returns 0
+ * for invalid arguments.
+ */
+SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, int64_t N,
+                                  int64_t B_tot, int64_t W_tot);
+
+/* Static, human-readable text of a status code. */
+SSA_API const char* ssa_error_string(ssa_status status);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device check word
+ * for the current device: SSA_OK, or the status a kernel recorded.
+ */
+SSA_API ssa_status ssa_get_device_status(void* stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+SSA_API int32_t ssa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H */

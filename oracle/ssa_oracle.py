@@ -377,3 +377,36 @@ def backward(st: State, dout: np.ndarray, chunk: int = 256) -> dict:
         "dgates": dgates,
         "parts": {"dq": dq, "dk": dk, "dv": dv, "dkc": dkc, "dvc": dvc},
     }
+
+
+def dq_rows(st: State, dout: np.ndarray, tokens) -> np.ndarray:
+    """dQ of the given query tokens only ([len(tokens), Hq, d]).  The gradient of a
+    query row needs only that row's own softmax quantities, so this works on a
+    forward restricted to those tokens; same arithmetic as `backward`."""
+    q, k, v = st["q"], st["k"], st["v"]
+    hkv, G, scale = st["hkv"], st["G"], st["scale"]
+    blk, win = st["blk"], st["win"]
+    gw = gate_weights(st["gates"], st["gate_mode"])
+    cu = st["cu_seqlens"]
+    out = np.zeros((len(tokens), q.shape[1], q.shape[2]))
+    for i, t in enumerate(tokens):
+        s = int(np.searchsorted(cu, t, side="right") - 1)
+        b0, b1 = int(blk["cu"][s]), int(blk["cu"][s + 1])
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            do = np.asarray(dout[t, hs, :], np.float64)
+            w = win["id"][t]
+            keysets = (
+                (st["kc"][b0:b1, g, :], st["vc"][b0:b1, g, :]),
+                (k[selected_tokens(st["sel"][t, g], blk), g, :], v[selected_tokens(st["sel"][t, g], blk), g, :]),
+                (k[win["perm"][win["ptr"][w]:win["ptr"][w + 1]], g, :],
+                 v[win["perm"][win["ptr"][w]:win["ptr"][w + 1]], g, :]),
+            )
+            for c, (kk, vv) in enumerate(keysets):
+                dor = do * gw[t, hs, c][:, None]
+                sc = scale * (q[t, hs, :] @ kk.T)
+                p = np.exp(sc - st["lse"][c, t, hs][:, None])
+                dp = dor @ vv.T
+                ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+                out[i, hs, :] += scale * (ds @ kk)
+    return out

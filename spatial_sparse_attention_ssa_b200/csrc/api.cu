@@ -1,0 +1,315 @@
+// C ABI of libssa: argument checks, workspace layout and launch order.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+// Device check word (or of ssa::kStatus* bits), read and cleared by the host.
+__device__ int g_ssa_status;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Carver {
+  char* p;
+  size_t used = 0;
+  explicit Carver(void* base) : p(static_cast<char*>(base)) {}
+  template <typename T>
+  T* take(size_t count) {
+    T* r = reinterpret_cast<T*>(p ? p + used : nullptr);
+    used += align256(sizeof(T) * (count > 0 ? count : 1));
+    return r;
+  }
+};
+
+int* status_ptr() {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_ssa_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(ptr);
+}
+
+ssa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
+
+ssa_status check_params(const ssa_params* p) {
+  if (!p) return SSA_ERR_INVALID_ARG;
+  if (p->hq < 1 || p->hkv < 1 || p->hq % p->hkv != 0) return SSA_ERR_INVALID_ARG;
+  if (p->m_cmp < 1 || p->m_win < 1 || p->topk < 1) return SSA_ERR_INVALID_ARG;
+  if (p->dtype != SSA_DTYPE_BF16 && p->dtype != SSA_DTYPE_F32) return SSA_ERR_INVALID_ARG;
+  if (p->gate_mode != SSA_GATE_WEIGHTS && p->gate_mode != SSA_GATE_LOGITS) return SSA_ERR_INVALID_ARG;
+  if (!(p->scale >= 0.f) || isinf(p->scale)) return SSA_ERR_INVALID_ARG;
+  if (p->d != 32 && p->d != 64) return SSA_ERR_UNSUPPORTED;
+  if (p->topk > 32) return SSA_ERR_UNSUPPORTED;
+  const int G = p->hq / p->hkv;
+  if (G & (G - 1)) return SSA_ERR_UNSUPPORTED;  // power of two
+  if (G * (p->d / 32) > 32) return SSA_ERR_UNSUPPORTED;
+  return SSA_OK;
+}
+
+bool partition_ok(const ssa_partition* x) {
+  return x && x->id && x->perm && x->ptr && x->cu && x->key && x->count >= 0;
+}
+
+float eff_scale(const ssa_params* p) { return p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->d); }
+
+// Workspace of the forward (after `ws` base): plan arrays.
+void carve_plan(Carver& c, int32_t S, int32_t** tc, int32_t** tp, int32_t** ic, int32_t** ip, int32_t** st) {
+  *tc = c.take<int32_t>(S + 1);
+  *tp = c.take<int32_t>(S + 1);
+  *ic = c.take<int32_t>(S + 1);
+  *ip = c.take<int32_t>(S + 1);
+  *st = c.take<int32_t>(ssa::scan_tmp_ints(S + 1));
+}
+
+size_t bin_bytes(int32_t S, int64_t N) { return ssa::bin_ws_bytes(S, N) + 256; }
+
+size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W) {
+  (void)p;
+  (void)N;
+  (void)B;
+  (void)W;
+  Carver c(nullptr);
+  int32_t *a, *b, *d, *e, *f;
+  carve_plan(c, S, &a, &b, &d, &e, &f);
+  return c.used;
+}
+
+struct BwdWs {
+  float* Dc;
+  float *dkc, *dvc;
+  uint64_t *ka, *kb;
+  int32_t *va, *vb, *inv_ptr, *radix_tmp;
+  int32_t *tc, *tp, *ic, *ip, *st;
+};
+
+size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t B, BwdWs* w) {
+  Carver c(base);
+  const int64_t nsel = N * p->hkv * p->topk;
+  w->Dc = c.take<float>(3 * N * p->hq);
+  w->dkc = c.take<float>(p->hkv * B * p->d);
+  w->dvc = c.take<float>(p->hkv * B * p->d);
+  w->ka = c.take<uint64_t>(nsel);
+  w->kb = c.take<uint64_t>(nsel);
+  w->va = c.take<int32_t>(nsel);
+  w->vb = c.take<int32_t>(nsel);
+  w->inv_ptr = c.take<int32_t>(p->hkv * B + 1);
+  w->radix_tmp = c.take<int32_t>(ssa::radix_tmp_ints(nsel));
+  carve_plan(c, S, &w->tc, &w->tp, &w->ic, &w->ip, &w->st);
+  return c.used;
+}
+
+}  // namespace
+
+extern "C" {
+
+SSA_API int32_t ssa_version(void) { return 100; }
+
+SSA_API const char* ssa_error_string(ssa_status s) {
+  switch (s) {
+    case SSA_OK: return "ok";
+    case SSA_ERR_INVALID_ARG: return "invalid argument";
+    case SSA_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case SSA_ERR_WORKSPACE: return "workspace too small";
+    case SSA_ERR_COORD_RANGE: return "coordinate outside [0, R) or malformed cu_seqlens";
+    case SSA_ERR_CUDA: return "CUDA error";
+    case SSA_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, int64_t N, int64_t B_tot,
+                                  int64_t W_tot) {
+  if (S < 0 || N < 0 || B_tot < 0 || W_tot < 0) return 0;
+  if (op == SSA_OP_BIN) return bin_bytes(S, N);
+  if (check_params(p) != SSA_OK) return 0;
+  if (op == SSA_OP_FORWARD) return fwd_bytes(p, S, N, B_tot, W_tot);
+  if (op == SSA_OP_BACKWARD) {
+    BwdWs w;
+    return carve_bwd(nullptr, p, S, N, B_tot, &w);
+  }
+  return 0;
+}
+
+SSA_API ssa_status ssa_get_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* sp = status_ptr();
+  if (!sp) return SSA_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyAsync(&h, sp, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSA_ERR_CUDA;
+  if (h) {
+    cudaMemsetAsync(sp, 0, sizeof(int), st);
+    cudaStreamSynchronize(st);
+  }
+  if (h & ssa::kStatusTimeout) return SSA_ERR_TIMEOUT;
+  if (h & (ssa::kStatusCoordRange | ssa::kStatusSeqlens)) return SSA_ERR_COORD_RANGE;
+  return SSA_OK;
+}
+
+SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N, int32_t R,
+                           int32_t m_cmp, int32_t m_win, ssa_partition* blk, ssa_partition* win, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || R < 1 || R > (1 << 20) || m_cmp < 1 || m_win < 1)
+    return SSA_ERR_INVALID_ARG;
+  if (!cu_seqlens || (N > 0 && !coords) || !partition_ok(blk) || !partition_ok(win) || !ws)
+    return SSA_ERR_INVALID_ARG;
+  if (ws_bytes < bin_bytes(S, N)) return SSA_ERR_WORKSPACE;
+  int sbits = 0;
+  while ((1ll << sbits) < S) ++sbits;
+  for (int m : {m_cmp, m_win}) {
+    int cbits = 1;
+    while ((1ll << cbits) < (R + m - 1) / m) ++cbits;
+    if (sbits + 3 * cbits > 64) return SSA_ERR_UNSUPPORTED;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* sp = status_ptr();
+  if (!sp) return SSA_ERR_CUDA;
+  int32_t* d_counts = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + ssa::bin_ws_bytes(S, N));
+  cudaError_t e = ssa::bin_partition(coords, cu_seqlens, S, N, R, m_cmp, blk, d_counts, ws, sp, st);
+  if (e != cudaSuccess) return SSA_ERR_CUDA;
+  if (m_win == m_cmp) {
+    e = cudaMemcpyAsync(win->id, blk->id, sizeof(int32_t) * N, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(win->perm, blk->perm, sizeof(int32_t) * N, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(win->ptr, blk->ptr, sizeof(int32_t) * (N + 1), cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(win->cu, blk->cu, sizeof(int32_t) * (S + 1), cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess && N > 0)
+      e = cudaMemcpyAsync(win->key, blk->key, sizeof(int32_t) * 3 * N, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_counts + 1, d_counts, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+  } else {
+    e = ssa::bin_partition(coords, cu_seqlens, S, N, R, m_win, win, d_counts + 1, ws, sp, st);
+  }
+  if (e != cudaSuccess) return SSA_ERR_CUDA;
+  int32_t h_counts[2] = {0, 0};
+  int h_status = 0;
+  e = cudaMemcpyAsync(h_counts, d_counts, sizeof(h_counts), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h_status, sp, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return SSA_ERR_CUDA;
+  blk->count = h_counts[0];
+  win->count = h_counts[1];
+  if (h_status) {
+    cudaMemsetAsync(sp, 0, sizeof(int), st);
+    cudaStreamSynchronize(st);
+    return (h_status & ssa::kStatusTimeout) ? SSA_ERR_TIMEOUT : SSA_ERR_COORD_RANGE;
+  }
+  return SSA_OK;
+}
+
+SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                               const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
+                               const void* v, const float* gates, void* out, const ssa_saved* saved, void* ws,
+                               size_t ws_bytes, void* stream) {
+  ssa_status ps = check_params(p);
+  if (ps != SSA_OK) return ps;
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
+    return SSA_ERR_INVALID_ARG;
+  if (N == 0) return SSA_OK;
+  if (!q || !k || !v || !gates || !out || !saved->kc || !saved->vc || !saved->ks || !saved->vs ||
+      !saved->o_branch || !saved->lse || !saved->sel || !ws)
+    return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
+  if (ws_bytes < fwd_bytes(p, S, N, blk->count, win->count)) return SSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = ssa::launch_pool(p->dtype, k, v, blk, N, p->hkv, p->d, saved->ks, saved->vs, saved->kc, saved->vc,
+                                   st);
+  if (e != cudaSuccess) return SSA_ERR_CUDA;
+  ssa::FwdArgs a;
+  a.dtype = p->dtype;
+  a.d = p->d;
+  a.hq = p->hq;
+  a.hkv = p->hkv;
+  a.topk = p->topk;
+  a.gate_mode = p->gate_mode;
+  a.scale = eff_scale(p);
+  a.S = S;
+  a.N = N;
+  a.cu_seqlens = cu_seqlens;
+  a.blk = blk;
+  a.win = win;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.gates = gates;
+  a.out = out;
+  a.kc = saved->kc;
+  a.vc = saved->vc;
+  a.ks = saved->ks;
+  a.vs = saved->vs;
+  a.o_branch = saved->o_branch;
+  a.lse = saved->lse;
+  a.sel = saved->sel;
+  Carver c(ws);
+  carve_plan(c, S, &a.tiles_cnt, &a.tiles_pre, &a.items_cnt, &a.items_pre, &a.scan_tmp);
+  return cuda_status(ssa::simt_forward(a, st));
+}
+
+SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                                const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
+                                const void* v, const float* gates, const ssa_saved* saved, const void* dout,
+                                float* dq, float* dk, float* dv, float* dgates, void* ws, size_t ws_bytes,
+                                void* stream) {
+  ssa_status ps = check_params(p);
+  if (ps != SSA_OK) return ps;
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
+    return SSA_ERR_INVALID_ARG;
+  if (N == 0) return SSA_OK;
+  if (!q || !k || !v || !gates || !dout || !dq || !dk || !dv || !dgates || !saved->kc || !saved->vc ||
+      !saved->ks || !saved->vs || !saved->o_branch || !saved->lse || !saved->sel || !ws)
+    return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
+  if ((int64_t)N * p->hkv * p->topk > INT32_MAX) return SSA_ERR_UNSUPPORTED;
+  BwdWs w;
+  if (ws_bytes < carve_bwd(nullptr, p, S, N, blk->count, &w)) return SSA_ERR_WORKSPACE;
+  carve_bwd(ws, p, S, N, blk->count, &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ssa::BwdArgs a;
+  a.dtype = p->dtype;
+  a.d = p->d;
+  a.hq = p->hq;
+  a.hkv = p->hkv;
+  a.topk = p->topk;
+  a.gate_mode = p->gate_mode;
+  a.scale = eff_scale(p);
+  a.S = S;
+  a.N = N;
+  a.cu_seqlens = cu_seqlens;
+  a.blk = blk;
+  a.win = win;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.gates = gates;
+  a.kc = saved->kc;
+  a.vc = saved->vc;
+  a.ks = saved->ks;
+  a.vs = saved->vs;
+  a.o_branch = saved->o_branch;
+  a.lse = saved->lse;
+  a.sel = saved->sel;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dgates = dgates;
+  a.Dc = w.Dc;
+  a.dkc = w.dkc;
+  a.dvc = w.dvc;
+  a.inv_keys_a = w.ka;
+  a.inv_keys_b = w.kb;
+  a.inv_vals_a = w.va;
+  a.inv_vals_b = w.vb;
+  a.inv_ptr = w.inv_ptr;
+  a.radix_tmp = w.radix_tmp;
+  a.tiles_cnt = w.tc;
+  a.tiles_pre = w.tp;
+  a.items_cnt = w.ic;
+  a.items_pre = w.ip;
+  a.scan_tmp = w.st;
+  return cuda_status(ssa::simt_backward(a, st));
+}
+
+}  // extern "C"

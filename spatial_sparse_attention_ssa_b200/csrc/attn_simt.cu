@@ -1,0 +1,1043 @@
+// Steps 3-7 of SSA as fp32 SIMT kernels (FFMA): compressed attention + top-k
+// selection, selected-block attention, window attention, gated combine and the
+// backward of all three branches.
+//
+// Direct3D-S2 (hyper.ai, "方法"): queries attend to the compressed blocks; the
+// top-k blocks by that attention score get a second, full attention over their
+// tokens; a third attention runs inside non-overlapping m_win^3 windows; the
+// three outputs are summed with predicted gate weights.  The selection score of
+// a block is its softmax probability summed over the query heads of a GQA group
+// (LSRM, shuwu5.cn, "阶段一": grouped-query attention with 2 KV heads).
+//
+// These kernels serve the fp32 configuration (which needs true fp32 math) and
+// every shape the tensor-core kernels do not cover.  Layout: NT = D/32 adjacent
+// lanes own one query row (32 dims each); keys/values are staged in shared
+// memory as fp32 with a 4-float pad between 32-dim sub-rows (no bank conflicts
+// between the NT sub-lanes).  Softmax runs in the log2 domain (q pre-scaled by
+// scale * log2(e)); stored lse values are natural logs.
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ssa {
+namespace {
+
+template <int D>
+struct Cfg {
+  static constexpr int NT = D / 32;          // lanes per row
+  static constexpr int THREADS = 128;
+  static constexpr int ROWS = THREADS / NT;  // rows per CTA
+  static constexpr int KSTR = NT * 36;       // floats per staged row
+};
+
+__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xffff0000u));
+}
+
+// Stage n rows of D elements into shared memory (fp32, padded sub-rows).
+template <typename T, int D, typename F>
+__device__ __forceinline__ void stage_rows(float* dst, int n, F src, float mul = 1.f) {
+  constexpr int QPR = D / 4;
+  for (int idx = threadIdx.x; idx < n * QPR; idx += blockDim.x) {
+    const int j = idx / QPR, qd = idx % QPR;
+    float4 v = load4(src(j) + qd * 4);
+    v.x *= mul;
+    v.y *= mul;
+    v.z *= mul;
+    v.w *= mul;
+    *reinterpret_cast<float4*>(dst + j * Cfg<D>::KSTR + (qd >> 3) * 36 + (qd & 7) * 4) = v;
+  }
+}
+
+__device__ __forceinline__ float dot32(const float* a, const float* row) {
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 k = r4[i];
+    acc = fmaf(a[4 * i + 0], k.x, acc);
+    acc = fmaf(a[4 * i + 1], k.y, acc);
+    acc = fmaf(a[4 * i + 2], k.z, acc);
+    acc = fmaf(a[4 * i + 3], k.w, acc);
+  }
+  return acc;
+}
+
+__device__ __forceinline__ float dot32r(const float* a, const float* b) {
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc = fmaf(a[i], b[i], acc);
+  return acc;
+}
+
+__device__ __forceinline__ void axpy32(float* y, float a, const float* row) {
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 k = r4[i];
+    y[4 * i + 0] = fmaf(a, k.x, y[4 * i + 0]);
+    y[4 * i + 1] = fmaf(a, k.y, y[4 * i + 1]);
+    y[4 * i + 2] = fmaf(a, k.z, y[4 * i + 2]);
+    y[4 * i + 3] = fmaf(a, k.w, y[4 * i + 3]);
+  }
+}
+
+template <int NT>
+__device__ __forceinline__ float row_sum(float x, unsigned mask) {
+  if (NT >= 2) x += __shfl_xor_sync(mask, x, 1);
+  if (NT >= 4) x += __shfl_xor_sync(mask, x, 2);
+  return x;
+}
+
+__device__ __forceinline__ float gate_weight(const float* gates, int64_t idx, int mode) {
+  const float x = gates[idx];
+  return mode == SSA_GATE_LOGITS ? 1.f / (1.f + expf(-x)) : x;
+}
+
+// ---------------------------------------------------------------------------
+// compressed branch, pass 1: lse over all blocks of the query's sequence
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) cmp_lse_kernel(const T* __restrict__ q, const T* __restrict__ kc,
+                                                      const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
+                                                      const int32_t* __restrict__ tpre, int S, int hq, int hkv,
+                                                      int64_t btot, float qs2, float* __restrict__ lse_out) {
+  using C = Cfg<D>;
+  constexpr int KT = 64;
+  __shared__ __align__(16) float sk[KT * C::KSTR];
+  const int g = blockIdx.y, G = hq / hkv;
+  const int r = threadIdx.x / C::NT, sub = threadIdx.x % C::NT;
+  const int ntiles = tpre[S];
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int s = find_segment(tpre, S, tile);
+    const int64_t nrows = (int64_t)(cu[s + 1] - cu[s]) * G;
+    const int64_t gr = (int64_t)(tile - tpre[s]) * C::ROWS + r;
+    const bool valid = gr < nrows;
+    const int64_t t = cu[s] + (valid ? gr / G : 0);
+    const int h = g * G + (valid ? (int)(gr % G) : 0);
+    float qv[32];
+    load32(q + (t * hq + h) * D + sub * 32, qv);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) qv[i] *= qs2;
+    float m = -CUDART_INF_F, l = 0.f;
+    const int b0 = bcu[s], nb = bcu[s + 1] - b0;
+    for (int c0 = 0; c0 < nb; c0 += KT) {
+      const int kn = min(KT, nb - c0);
+      __syncthreads();
+      stage_rows<T, D>(sk, kn, [&](int j) { return kc + ((int64_t)g * btot + b0 + c0 + j) * D; });
+      __syncthreads();
+      for (int j0 = 0; j0 < kn; j0 += 16) {
+        float sc[16];
+        float cm = -CUDART_INF_F;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          float x = -CUDART_INF_F;
+          if (j0 + jj < kn) x = row_sum<C::NT>(dot32(qv, sk + (j0 + jj) * C::KSTR + sub * 36), 0xffffffffu);
+          sc[jj] = x;
+          cm = fmaxf(cm, x);
+        }
+        const float mn = fmaxf(m, cm);
+        l *= exp2f(m - mn);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) l += exp2f(sc[jj] - mn);
+        m = mn;
+      }
+    }
+    if (valid && sub == 0) lse_out[t * hq + h] = (m + log2f(l)) * kLn2;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// compressed branch, pass 2: output with the final lse + top-k block selection
+// ---------------------------------------------------------------------------
+constexpr int kTopkMax = 32;
+
+__device__ __forceinline__ int find_worst(const float* v, const int* id, int n) {
+  int w = 0;
+  for (int i = 1; i < n; ++i)
+    if (v[i] < v[w] || (v[i] == v[w] && id[i] > id[w])) w = i;
+  return w;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) cmp_out_topk_kernel(
+    const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc, const int32_t* __restrict__ cu,
+    const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S, int hq, int hkv, int64_t btot,
+    float qs2, const float* __restrict__ lse_in, float* __restrict__ o_out, int topk, int32_t* __restrict__ sel) {
+  using C = Cfg<D>;
+  constexpr int KT = 32;
+  __shared__ __align__(16) float sk[KT * C::KSTR];
+  __shared__ __align__(16) float sv[KT * C::KSTR];
+  __shared__ float tv[C::ROWS][kTopkMax];
+  __shared__ int ti[C::ROWS][kTopkMax];
+  const int g = blockIdx.y, G = hq / hkv;
+  const int r = threadIdx.x / C::NT, sub = threadIdx.x % C::NT;
+  const int tok = r / G;
+  const bool leader = (r % G == 0) && sub == 0;
+  const int ntiles = tpre[S];
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int s = find_segment(tpre, S, tile);
+    const int64_t nrows = (int64_t)(cu[s + 1] - cu[s]) * G;
+    const int64_t gr = (int64_t)(tile - tpre[s]) * C::ROWS + r;
+    const bool valid = gr < nrows;
+    const int64_t t = cu[s] + (valid ? gr / G : 0);
+    const int h = g * G + (valid ? (int)(gr % G) : 0);
+    float qv[32], o[32];
+    load32(q + (t * hq + h) * D + sub * 32, qv);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      qv[i] *= qs2;
+      o[i] = 0.f;
+    }
+    const float lse2 = lse_in[t * hq + h] * kLog2e;
+    const int b0 = bcu[s], nb = bcu[s + 1] - b0;
+    const int keff = min(topk, nb);
+    int cnt = 0, worst = 0;
+    for (int c0 = 0; c0 < nb; c0 += KT) {
+      const int kn = min(KT, nb - c0);
+      __syncthreads();
+      stage_rows<T, D>(sk, kn, [&](int j) { return kc + ((int64_t)g * btot + b0 + c0 + j) * D; });
+      stage_rows<T, D>(sv, kn, [&](int j) { return vc + ((int64_t)g * btot + b0 + c0 + j) * D; });
+      __syncthreads();
+      for (int j = 0; j < kn; ++j) {
+        const float s2 = row_sum<C::NT>(dot32(qv, sk + j * C::KSTR + sub * 36), 0xffffffffu);
+        const float p = exp2f(s2 - lse2);
+        axpy32(o, p, sv + j * C::KSTR + sub * 36);
+        float imp = p;
+        for (int off = C::NT; off < G * C::NT; off <<= 1) imp += __shfl_xor_sync(0xffffffffu, imp, off);
+        if (leader && valid) {
+          const int bid = b0 + c0 + j;
+          if (cnt < keff) {
+            tv[tok][cnt] = imp;
+            ti[tok][cnt] = bid;
+            ++cnt;
+            if (cnt == keff) worst = find_worst(tv[tok], ti[tok], keff);
+          } else if (imp > tv[tok][worst]) {
+            tv[tok][worst] = imp;
+            ti[tok][worst] = bid;
+            worst = find_worst(tv[tok], ti[tok], keff);
+          }
+        }
+      }
+    }
+    if (valid) {
+      store32(o_out + (t * hq + h) * D + sub * 32, o);
+      if (leader) {
+        int* ids = ti[tok];
+        for (int i = 1; i < keff; ++i) {  // insertion sort, ascending ids
+          const int x = ids[i];
+          int j = i - 1;
+          while (j >= 0 && ids[j] > x) {
+            ids[j + 1] = ids[j];
+            --j;
+          }
+          ids[j + 1] = x;
+        }
+        int32_t* out = sel + (t * hkv + g) * topk;
+        for (int i = 0; i < topk; ++i) out[i] = i < keff ? ids[i] : -1;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// selected-block attention: per (token, group), all tokens of the selected blocks
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) slc_fwd_kernel(const T* __restrict__ q, const T* __restrict__ ks,
+                                                      const T* __restrict__ vs, const int32_t* __restrict__ bptr,
+                                                      const int32_t* __restrict__ sel, int64_t N, int hq, int hkv,
+                                                      int topk, float qs2, float* __restrict__ o_out,
+                                                      float* __restrict__ lse_out) {
+  constexpr int NT = D / 32;
+  const int G = hq / hkv, GT = G * NT, PPC = 128 / GT;
+  const int lane = threadIdx.x & 31;
+  const unsigned gmask = GT >= 32 ? 0xffffffffu : (((1u << GT) - 1u) << (lane & ~(GT - 1)));
+  const int r = (threadIdx.x % GT) / NT, sub = threadIdx.x % NT;
+  const int64_t npairs = N * hkv;
+  for (int64_t pair = (int64_t)blockIdx.x * PPC + threadIdx.x / GT; pair < npairs; pair += (int64_t)gridDim.x * PPC) {
+    const int64_t t = pair / hkv;
+    const int g = (int)(pair % hkv), h = g * G + r;
+    float qv[32], o[32];
+    load32(q + (t * hq + h) * D + sub * 32, qv);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      qv[i] *= qs2;
+      o[i] = 0.f;
+    }
+    float m = -CUDART_INF_F, l = 0.f;
+    const int32_t* srow = sel + pair * topk;
+    for (int si = 0; si < topk; ++si) {
+      const int b = srow[si];
+      if (b < 0) continue;
+      const int p1 = bptr[b + 1];
+      for (int j0 = bptr[b]; j0 < p1; j0 += 8) {
+        float sc[8];
+        float cm = -CUDART_INF_F;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          float x = -CUDART_INF_F;
+          if (j0 + jj < p1) {
+            float kv[32];
+            load32(ks + ((int64_t)g * N + j0 + jj) * D + sub * 32, kv);
+            x = row_sum<NT>(dot32r(qv, kv), gmask);
+          }
+          sc[jj] = x;
+          cm = fmaxf(cm, x);
+        }
+        const float mn = fmaxf(m, cm);
+        const float corr = exp2f(m - mn);
+        l *= corr;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= corr;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          if (j0 + jj < p1) {
+            const float p = exp2f(sc[jj] - mn);
+            l += p;
+            float vv[32];
+            load32(vs + ((int64_t)g * N + j0 + jj) * D + sub * 32, vv);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = fmaf(p, vv[i], o[i]);
+          }
+        }
+        m = mn;
+      }
+    }
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] *= inv;
+    store32(o_out + (t * hq + h) * D + sub * 32, o);
+    if (sub == 0) lse_out[t * hq + h] = (m + log2f(l)) * kLn2;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// window attention: per (window, group), every token of the window
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) win_fwd_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                      const T* __restrict__ v, const int32_t* __restrict__ wperm,
+                                                      const int32_t* __restrict__ wptr, int64_t wtot, int hq, int hkv,
+                                                      float qs2, float* __restrict__ o_out, float* __restrict__ lse_out) {
+  using C = Cfg<D>;
+  constexpr int KT = 64;
+  __shared__ __align__(16) float sk[KT * C::KSTR];
+  __shared__ __align__(16) float sv[KT * C::KSTR];
+  const int g = blockIdx.y, G = hq / hkv;
+  const int r = threadIdx.x / C::NT, sub = threadIdx.x % C::NT;
+  for (int64_t w = blockIdx.x; w < wtot; w += gridDim.x) {
+    const int p0 = wptr[w], nw = wptr[w + 1] - p0;
+    const int nrows = nw * G;
+    const int nchunks = (nw + KT - 1) / KT;
+    for (int row0 = 0; row0 < nrows; row0 += C::ROWS) {
+      const int rr = row0 + r;
+      const bool valid = rr < nrows;
+      const int64_t t = wperm[p0 + (valid ? rr / G : 0)];
+      const int h = g * G + (valid ? rr % G : 0);
+      float qv[32], o[32];
+      load32(q + (t * hq + h) * D + sub * 32, qv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        qv[i] *= qs2;
+        o[i] = 0.f;
+      }
+      float m = -CUDART_INF_F, l = 0.f;
+      for (int c = 0; c < nchunks; ++c) {
+        const int kn = min(KT, nw - c * KT);
+        if (nchunks > 1 || row0 == 0) {
+          __syncthreads();
+          stage_rows<T, D>(sk, kn, [&](int j) { return k + ((int64_t)wperm[p0 + c * KT + j] * hkv + g) * D; });
+          stage_rows<T, D>(sv, kn, [&](int j) { return v + ((int64_t)wperm[p0 + c * KT + j] * hkv + g) * D; });
+          __syncthreads();
+        }
+        for (int j0 = 0; j0 < kn; j0 += 16) {
+          float sc[16];
+          float cm = -CUDART_INF_F;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            float x = -CUDART_INF_F;
+            if (j0 + jj < kn) x = row_sum<C::NT>(dot32(qv, sk + (j0 + jj) * C::KSTR + sub * 36), 0xffffffffu);
+            sc[jj] = x;
+            cm = fmaxf(cm, x);
+          }
+          const float mn = fmaxf(m, cm);
+          const float corr = exp2f(m - mn);
+          l *= corr;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= corr;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            if (j0 + jj < kn) {
+              const float p = exp2f(sc[jj] - mn);
+              l += p;
+              axpy32(o, p, sv + (j0 + jj) * C::KSTR + sub * 36);
+            }
+          }
+          m = mn;
+        }
+      }
+      if (valid) {
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= inv;
+        store32(o_out + (t * hq + h) * D + sub * 32, o);
+        if (sub == 0) lse_out[t * hq + h] = (m + log2f(l)) * kLn2;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gated combine: out = sum_c w_c * o_c
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void combine_kernel(const float* __restrict__ ob, const float* __restrict__ gates, int64_t rows, int mode,
+                               T* __restrict__ out) {
+  constexpr int NT = D / 32;
+  const int64_t total = rows * NT;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / NT;
+    const int sub = (int)(i % NT);
+    float acc[32], x[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      const float w = gate_weight(gates, row * 3 + c, mode);
+      load32(ob + ((int64_t)c * rows + row) * D + sub * 32, x);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) acc[e] = fmaf(w, x[e], acc[e]);
+    }
+    store32(out + row * D + sub * 32, acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// backward: per-row dot products <dO, o_c>, the softmax correction D_c and dgates
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict__ dout, const float* __restrict__ gates,
+                               int64_t rows, int mode, float* __restrict__ Dc, float* __restrict__ dgates) {
+  constexpr int NT = D / 32;
+  const int64_t total = rows * NT;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t iters = (total + stride - 1) / stride;
+  for (int64_t it = 0; it < iters; ++it) {
+    const int64_t i = it * stride + blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const bool valid = i < total;
+    const int64_t row = valid ? i / NT : 0;
+    const int sub = (int)(i % NT);
+    float dov[32], x[32];
+    load32(dout + row * D + sub * 32, dov);
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      load32(ob + ((int64_t)c * rows + row) * D + sub * 32, x);
+      const float dot = row_sum<NT>(dot32r(dov, x), 0xffffffffu);
+      if (valid && sub == 0) {
+        const float w = gate_weight(gates, row * 3 + c, mode);
+        Dc[(int64_t)c * rows + row] = w * dot;
+        dgates[row * 3 + c] = mode == SSA_GATE_LOGITS ? dot * w * (1.f - w) : dot;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// compressed branch backward: dQ (query-major)
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) cmp_bwd_dq_kernel(
+    const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc, const T* __restrict__ dout,
+    const float* __restrict__ gates, int mode, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
+    const int32_t* __restrict__ tpre, int S, int hq, int hkv, int64_t btot, float qs2, float scale,
+    const float* __restrict__ lse_in, const float* __restrict__ Dc, float* __restrict__ dq_out) {
+  using C = Cfg<D>;
+  constexpr int KT = 32;
+  __shared__ __align__(16) float sk[KT * C::KSTR];
+  __shared__ __align__(16) float sv[KT * C::KSTR];
+  const int g = blockIdx.y, G = hq / hkv;
+  const int r = threadIdx.x / C::NT, sub = threadIdx.x % C::NT;
+  const int ntiles = tpre[S];
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int s = find_segment(tpre, S, tile);
+    const int64_t nrows = (int64_t)(cu[s + 1] - cu[s]) * G;
+    const int64_t gr = (int64_t)(tile - tpre[s]) * C::ROWS + r;
+    const bool valid = gr < nrows;
+    const int64_t t = cu[s] + (valid ? gr / G : 0);
+    const int h = g * G + (valid ? (int)(gr % G) : 0);
+    const int64_t row = t * hq + h;
+    float qv[32], dov[32], dq[32];
+    load32(q + row * D + sub * 32, qv);
+    load32(dout + row * D + sub * 32, dov);
+    const float wg = gate_weight(gates, row * 3 + 0, mode);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      qv[i] *= qs2;
+      dov[i] *= wg;
+      dq[i] = 0.f;
+    }
+    const float lse2 = lse_in[row] * kLog2e;
+    const float Dr = Dc[row];
+    const int b0 = bcu[s], nb = bcu[s + 1] - b0;
+    for (int c0 = 0; c0 < nb; c0 += KT) {
+      const int kn = min(KT, nb - c0);
+      __syncthreads();
+      stage_rows<T, D>(sk, kn, [&](int j) { return kc + ((int64_t)g * btot + b0 + c0 + j) * D; });
+      stage_rows<T, D>(sv, kn, [&](int j) { return vc + ((int64_t)g * btot + b0 + c0 + j) * D; });
+      __syncthreads();
+      for (int j = 0; j < kn; ++j) {
+        const float* krow = sk + j * C::KSTR + sub * 36;
+        const float s2 = row_sum<C::NT>(dot32(qv, krow), 0xffffffffu);
+        const float p = exp2f(s2 - lse2);
+        const float dp = row_sum<C::NT>(dot32(dov, sv + j * C::KSTR + sub * 36), 0xffffffffu);
+        axpy32(dq, p * (dp - Dr), krow);
+      }
+    }
+    if (valid) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dq[i] *= scale;
+      store32(dq_out + row * D + sub * 32, dq);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Shared key-major backward core: a CTA owns KPC keys (k, v rows in registers)
+// and streams query rows through shared memory, accumulating dk, dv.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+struct RowStage {
+  static constexpr int RT = 16;  // rows per stage
+  float q[RT * Cfg<D>::KSTR];
+  float dO[RT * Cfg<D>::KSTR];
+  float lse2[RT];
+  float Dr[RT];
+};
+
+// Stage rows [r0, r0+n) where row index -> (global q/dO row, lse index) via `map`.
+// map(i, &row, &ok): row = token*hq + head of staged row i.
+template <typename T, int D, typename MAP>
+__device__ __forceinline__ void stage_query_rows(RowStage<T, D>& st, int n, MAP map, const T* q, const T* dout,
+                                                 const float* gates, int mode, int branch, const float* lse_b,
+                                                 const float* Dc_b) {
+  constexpr int QPR = D / 4;
+  for (int idx = threadIdx.x; idx < RowStage<T, D>::RT * QPR; idx += blockDim.x) {
+    const int i = idx / QPR, qd = idx % QPR;
+    int64_t row = 0;
+    bool ok = i < n && map(i, &row);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (ok) {
+      a = load4(q + row * D + qd * 4);
+      b = load4(dout + row * D + qd * 4);
+      const float w = gate_weight(gates, row * 3 + branch, mode);
+      b.x *= w;
+      b.y *= w;
+      b.z *= w;
+      b.w *= w;
+    }
+    const int off = i * Cfg<D>::KSTR + (qd >> 3) * 36 + (qd & 7) * 4;
+    *reinterpret_cast<float4*>(st.q + off) = a;
+    *reinterpret_cast<float4*>(st.dO + off) = b;
+    if (qd == 0) {
+      st.lse2[i] = ok ? lse_b[row] * kLog2e : CUDART_INF_F;
+      st.Dr[i] = ok ? Dc_b[row] : 0.f;
+    }
+  }
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void accumulate_rows(const RowStage<T, D>& st, const float* kv, const float* vv, float qs2,
+                                                float* dk, float* dv) {
+  constexpr int NT = D / 32;
+  const int sub = threadIdx.x % NT;
+#pragma unroll 2
+  for (int i = 0; i < RowStage<T, D>::RT; ++i) {
+    const float* qrow = st.q + i * Cfg<D>::KSTR + sub * 36;
+    const float* drow = st.dO + i * Cfg<D>::KSTR + sub * 36;
+    const float s2 = row_sum<NT>(dot32(kv, qrow), 0xffffffffu) * qs2;
+    const float p = exp2f(s2 - st.lse2[i]);
+    const float dp = row_sum<NT>(dot32(vv, drow), 0xffffffffu);
+    const float ds = p * (dp - st.Dr[i]);
+    axpy32(dk, ds, qrow);
+    axpy32(dv, p, drow);
+  }
+}
+
+// compressed branch: dKc, dVc (atomic fp32 accumulation across row chunks)
+template <typename T, int D>
+__global__ void __launch_bounds__(128) cmp_bwd_dkv_kernel(
+    const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc, const T* __restrict__ dout,
+    const float* __restrict__ gates, int mode, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
+    const int32_t* __restrict__ ipre, int S, int hq, int hkv, int64_t btot, float qs2, float scale, int rc_rows,
+    const float* __restrict__ lse_in, const float* __restrict__ Dc, float* __restrict__ dkc, float* __restrict__ dvc) {
+  using C = Cfg<D>;
+  __shared__ __align__(16) RowStage<T, D> st;
+  const int g = blockIdx.y, G = hq / hkv;
+  const int sub = threadIdx.x % C::NT;
+  const int nitems = ipre[S];
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int s = find_segment(ipre, S, item);
+    const int b0 = bcu[s], nb = bcu[s + 1] - b0;
+    const int nbt = (nb + C::ROWS - 1) / C::ROWS;
+    const int local = item - ipre[s];
+    const int bt = local % nbt, rc = local / nbt;
+    const int j = bt * C::ROWS + threadIdx.x / C::NT;
+    const bool validb = j < nb;
+    const int64_t bidx = (int64_t)g * btot + b0 + (validb ? j : 0);
+    float kv[32], vv[32], dk[32], dv[32];
+    load32(kc + bidx * D + sub * 32, kv);
+    load32(vc + bidx * D + sub * 32, vv);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) dk[i] = dv[i] = 0.f;
+    const int64_t nrows = (int64_t)(cu[s + 1] - cu[s]) * G;
+    const int64_t r0 = (int64_t)rc * rc_rows;
+    const int64_t r1 = min(nrows, r0 + rc_rows);
+    for (int64_t rs = r0; rs < r1; rs += RowStage<T, D>::RT) {
+      const int n = (int)min((int64_t)RowStage<T, D>::RT, r1 - rs);
+      __syncthreads();
+      stage_query_rows<T, D>(
+          st, n,
+          [&](int i, int64_t* row) {
+            const int64_t gr = rs + i;
+            *row = (cu[s] + gr / G) * hq + g * G + gr % G;
+            return true;
+          },
+          q, dout, gates, mode, 0, lse_in, Dc);
+      __syncthreads();
+      accumulate_rows<T, D>(st, kv, vv, qs2, dk, dv);
+    }
+    if (validb) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        atomicAdd(dkc + bidx * D + sub * 32 + i, dk[i] * scale);
+        atomicAdd(dvc + bidx * D + sub * 32 + i, dv[i]);
+      }
+    }
+  }
+}
+
+// selected branch: dQ (query-major, like the forward)
+template <typename T, int D>
+__global__ void __launch_bounds__(128) slc_bwd_dq_kernel(
+    const T* __restrict__ q, const T* __restrict__ ks, const T* __restrict__ vs, const T* __restrict__ dout,
+    const float* __restrict__ gates, int mode, const int32_t* __restrict__ bptr, const int32_t* __restrict__ sel,
+    int64_t N, int hq, int hkv, int topk, float qs2, float scale, const float* __restrict__ lse_in,
+    const float* __restrict__ Dc, float* __restrict__ dq_out) {
+  constexpr int NT = D / 32;
+  const int G = hq / hkv, GT = G * NT, PPC = 128 / GT;
+  const int lane = threadIdx.x & 31;
+  const unsigned gmask = GT >= 32 ? 0xffffffffu : (((1u << GT) - 1u) << (lane & ~(GT - 1)));
+  const int r = (threadIdx.x % GT) / NT, sub = threadIdx.x % NT;
+  const int64_t npairs = N * hkv;
+  for (int64_t pair = (int64_t)blockIdx.x * PPC + threadIdx.x / GT; pair < npairs; pair += (int64_t)gridDim.x * PPC) {
+    const int64_t t = pair / hkv;
+    const int g = (int)(pair % hkv), h = g * G + r;
+    const int64_t row = t * hq + h;
+    float qv[32], dov[32], dq[32];
+    load32(q + row * D + sub * 32, qv);
+    load32(dout + row * D + sub * 32, dov);
+    const float wg = gate_weight(gates, row * 3 + 1, mode);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      qv[i] *= qs2;
+      dov[i] *= wg;
+      dq[i] = 0.f;
+    }
+    const float lse2 = lse_in[row] * kLog2e;
+    const float Dr = Dc[row];
+    const int32_t* srow = sel + pair * topk;
+    for (int si = 0; si < topk; ++si) {
+      const int b = srow[si];
+      if (b < 0) continue;
+      const int p1 = bptr[b + 1];
+      for (int j = bptr[b]; j < p1; ++j) {
+        float kv[32], vv[32];
+        load32(ks + ((int64_t)g * N + j) * D + sub * 32, kv);
+        load32(vs + ((int64_t)g * N + j) * D + sub * 32, vv);
+        const float s2 = row_sum<NT>(dot32r(qv, kv), gmask);
+        const float p = exp2f(s2 - lse2);
+        const float dp = row_sum<NT>(dot32r(dov, vv), gmask);
+        const float ds = p * (dp - Dr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dq[i] = fmaf(ds, kv[i], dq[i]);
+      }
+    }
+    float* dst = dq_out + row * D + sub * 32;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) dst[i] += dq[i] * scale;
+  }
+}
+
+// selected branch: dK, dV per block, over the (token, group) pairs that selected it
+template <typename T, int D>
+__global__ void __launch_bounds__(128) slc_bwd_dkv_kernel(
+    const T* __restrict__ q, const T* __restrict__ ks, const T* __restrict__ vs, const T* __restrict__ dout,
+    const float* __restrict__ gates, int mode, const int32_t* __restrict__ bptr, const int32_t* __restrict__ bperm,
+    const int32_t* __restrict__ inv_ptr, const int32_t* __restrict__ inv_tok, int64_t N, int64_t btot, int hq, int hkv,
+    float qs2, float scale, const float* __restrict__ lse_in, const float* __restrict__ Dc, float* __restrict__ dk_out,
+    float* __restrict__ dv_out) {
+  using C = Cfg<D>;
+  __shared__ __align__(16) RowStage<T, D> st;
+  const int g = blockIdx.y, G = hq / hkv;
+  const int sub = threadIdx.x % C::NT;
+  for (int64_t b = blockIdx.x; b < btot; b += gridDim.x) {
+    const int p0 = bptr[b], nb = bptr[b + 1] - p0;
+    const int l0 = inv_ptr[g * btot + b], l1 = inv_ptr[g * btot + b + 1];
+    const int64_t nrows = (int64_t)(l1 - l0) * G;
+    for (int kp = 0; kp < nb; kp += C::ROWS) {
+      const int j = kp + threadIdx.x / C::NT;
+      const bool validk = j < nb;
+      const int64_t kidx = (int64_t)g * N + p0 + (validk ? j : 0);
+      float kv[32], vv[32], dk[32], dv[32];
+      load32(ks + kidx * D + sub * 32, kv);
+      load32(vs + kidx * D + sub * 32, vv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dk[i] = dv[i] = 0.f;
+      for (int64_t rs = 0; rs < nrows; rs += RowStage<T, D>::RT) {
+        const int n = (int)min((int64_t)RowStage<T, D>::RT, nrows - rs);
+        __syncthreads();
+        stage_query_rows<T, D>(
+            st, n,
+            [&](int i, int64_t* row) {
+              const int64_t gr = rs + i;
+              *row = (int64_t)inv_tok[l0 + gr / G] * hq + g * G + gr % G;
+              return true;
+            },
+            q, dout, gates, mode, 1, lse_in, Dc);
+        __syncthreads();
+        accumulate_rows<T, D>(st, kv, vv, qs2, dk, dv);
+      }
+      if (validk) {
+        const int64_t tok = bperm[p0 + j];
+        float* a = dk_out + (tok * hkv + g) * D + sub * 32;
+        float* c = dv_out + (tok * hkv + g) * D + sub * 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          a[i] = dk[i] * scale;
+          c[i] = dv[i];
+        }
+      }
+    }
+  }
+}
+
+// window branch: dQ
+template <typename T, int D>
+__global__ void __launch_bounds__(128) win_bwd_dq_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ dout,
+    const float* __restrict__ gates, int mode, const int32_t* __restrict__ wperm, const int32_t* __restrict__ wptr,
+    int64_t wtot, int hq, int hkv, float qs2, float scale, const float* __restrict__ lse_in,
+    const float* __restrict__ Dc, float* __restrict__ dq_out) {
+  using C = Cfg<D>;
+  constexpr int KT = 32;
+  __shared__ __align__(16) float sk[KT * C::KSTR];
+  __shared__ __align__(16) float sv[KT * C::KSTR];
+  const int g = blockIdx.y, G = hq / hkv;
+  const int r = threadIdx.x / C::NT, sub = threadIdx.x % C::NT;
+  for (int64_t w = blockIdx.x; w < wtot; w += gridDim.x) {
+    const int p0 = wptr[w], nw = wptr[w + 1] - p0;
+    const int nrows = nw * G;
+    const int nchunks = (nw + KT - 1) / KT;
+    for (int row0 = 0; row0 < nrows; row0 += C::ROWS) {
+      const int rr = row0 + r;
+      const bool valid = rr < nrows;
+      const int64_t t = wperm[p0 + (valid ? rr / G : 0)];
+      const int h = g * G + (valid ? rr % G : 0);
+      const int64_t row = t * hq + h;
+      float qv[32], dov[32], dq[32];
+      load32(q + row * D + sub * 32, qv);
+      load32(dout + row * D + sub * 32, dov);
+      const float wg = gate_weight(gates, row * 3 + 2, mode);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        qv[i] *= qs2;
+        dov[i] *= wg;
+        dq[i] = 0.f;
+      }
+      const float lse2 = lse_in[row] * kLog2e;
+      const float Dr = Dc[row];
+      for (int c = 0; c < nchunks; ++c) {
+        const int kn = min(KT, nw - c * KT);
+        if (nchunks > 1 || row0 == 0) {
+          __syncthreads();
+          stage_rows<T, D>(sk, kn, [&](int j) { return k + ((int64_t)wperm[p0 + c * KT + j] * hkv + g) * D; });
+          stage_rows<T, D>(sv, kn, [&](int j) { return v + ((int64_t)wperm[p0 + c * KT + j] * hkv + g) * D; });
+          __syncthreads();
+        }
+        for (int j = 0; j < kn; ++j) {
+          const float* krow = sk + j * C::KSTR + sub * 36;
+          const float s2 = row_sum<C::NT>(dot32(qv, krow), 0xffffffffu);
+          const float p = exp2f(s2 - lse2);
+          const float dp = row_sum<C::NT>(dot32(dov, sv + j * C::KSTR + sub * 36), 0xffffffffu);
+          axpy32(dq, p * (dp - Dr), krow);
+        }
+      }
+      if (valid) {
+        float* dst = dq_out + row * D + sub * 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dst[i] += dq[i] * scale;
+      }
+    }
+  }
+}
+
+// window branch: dK, dV (added onto the selected branch's values)
+template <typename T, int D>
+__global__ void __launch_bounds__(128) win_bwd_dkv_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ dout,
+    const float* __restrict__ gates, int mode, const int32_t* __restrict__ wperm, const int32_t* __restrict__ wptr,
+    int64_t wtot, int hq, int hkv, float qs2, float scale, const float* __restrict__ lse_in,
+    const float* __restrict__ Dc, float* __restrict__ dk_out, float* __restrict__ dv_out) {
+  using C = Cfg<D>;
+  __shared__ __align__(16) RowStage<T, D> st;
+  const int g = blockIdx.y, G = hq / hkv;
+  const int sub = threadIdx.x % C::NT;
+  for (int64_t w = blockIdx.x; w < wtot; w += gridDim.x) {
+    const int p0 = wptr[w], nw = wptr[w + 1] - p0;
+    const int64_t nrows = (int64_t)nw * G;
+    for (int kp = 0; kp < nw; kp += C::ROWS) {
+      const int j = kp + threadIdx.x / C::NT;
+      const bool validk = j < nw;
+      const int64_t tok = wperm[p0 + (validk ? j : 0)];
+      float kv[32], vv[32], dk[32], dv[32];
+      load32(k + (tok * hkv + g) * D + sub * 32, kv);
+      load32(v + (tok * hkv + g) * D + sub * 32, vv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dk[i] = dv[i] = 0.f;
+      for (int64_t rs = 0; rs < nrows; rs += RowStage<T, D>::RT) {
+        const int n = (int)min((int64_t)RowStage<T, D>::RT, nrows - rs);
+        __syncthreads();
+        stage_query_rows<T, D>(
+            st, n,
+            [&](int i, int64_t* row) {
+              const int64_t gr = rs + i;
+              *row = (int64_t)wperm[p0 + gr / G] * hq + g * G + gr % G;
+              return true;
+            },
+            q, dout, gates, mode, 2, lse_in, Dc);
+        __syncthreads();
+        accumulate_rows<T, D>(st, kv, vv, qs2, dk, dv);
+      }
+      if (validk) {
+        float* a = dk_out + (tok * hkv + g) * D + sub * 32;
+        float* c = dv_out + (tok * hkv + g) * D + sub * 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          a[i] += dk[i] * scale;
+          c[i] += dv[i];
+        }
+      }
+    }
+  }
+}
+
+// compression gradient back to tokens: dK_i += dKc_b / n_b (likewise V)
+__global__ void cmp_scatter_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
+                                   const int32_t* __restrict__ bid, const int32_t* __restrict__ bptr, int64_t N,
+                                   int64_t btot, int hkv, int d, float* __restrict__ dk, float* __restrict__ dv) {
+  const int q4 = d / 4;
+  const int64_t total = N * hkv * q4;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int qd = (int)(i % q4);
+    const int64_t tg = i / q4;
+    const int g = (int)(tg % hkv);
+    const int64_t t = tg / hkv;
+    const int b = bid[t];
+    const float n = (float)(bptr[b + 1] - bptr[b]);
+    const int64_t src = ((int64_t)g * btot + b) * d + qd * 4;
+    const float4 a = *reinterpret_cast<const float4*>(dkc + src);
+    const float4 c = *reinterpret_cast<const float4*>(dvc + src);
+    float4* pk = reinterpret_cast<float4*>(dk + tg * d + qd * 4);
+    float4* pv = reinterpret_cast<float4*>(dv + tg * d + qd * 4);
+    float4 x = *pk, y = *pv;
+    x.x += __fdiv_rn(a.x, n);
+    x.y += __fdiv_rn(a.y, n);
+    x.z += __fdiv_rn(a.z, n);
+    x.w += __fdiv_rn(a.w, n);
+    y.x += __fdiv_rn(c.x, n);
+    y.y += __fdiv_rn(c.y, n);
+    y.z += __fdiv_rn(c.z, n);
+    y.w += __fdiv_rn(c.w, n);
+    *pk = x;
+    *pv = y;
+  }
+}
+
+// inverted selection: key (g * btot + b) per (token, group, slot), sentinel for -1
+__global__ void sel_keys_kernel(const int32_t* __restrict__ sel, int64_t N, int hkv, int topk, int64_t btot,
+                                uint64_t* __restrict__ keys, int32_t* __restrict__ vals) {
+  const int64_t total = N * hkv * topk;
+  const uint64_t sentinel = (uint64_t)hkv * btot;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t pair = i / topk;
+    const int g = (int)(pair % hkv);
+    const int b = sel[i];
+    keys[i] = b >= 0 ? (uint64_t)g * btot + b : sentinel;
+    vals[i] = (int32_t)(pair / hkv);
+  }
+}
+
+// CSR pointers from sorted keys: ptr[key] = first position with that key (or later)
+__global__ void keys_to_ptr_kernel(const uint64_t* __restrict__ keys, int64_t n, int64_t nkeys,
+                                   int32_t* __restrict__ ptr) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i <= n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t lo = i == 0 ? 0 : (int64_t)keys[i - 1] + 1;
+    const int64_t hi = i == n ? nkeys : (int64_t)keys[i];
+    for (int64_t k = lo; k <= hi && k <= nkeys; ++k) ptr[k] = (int32_t)i;
+  }
+}
+
+// per-sequence work counts for the tiled kernels
+__global__ void plan_counts_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, int S, int G,
+                                   int rows_per_tile, int blocks_per_item, int rc_rows, int32_t* __restrict__ tiles,
+                                   int32_t* __restrict__ items) {
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s <= S; s += gridDim.x * blockDim.x) {
+    if (s == S) {
+      tiles[s] = 0;
+      items[s] = 0;
+      continue;
+    }
+    const int64_t nrows = (int64_t)(cu[s + 1] - cu[s]) * G;
+    const int nb = bcu[s + 1] - bcu[s];
+    tiles[s] = (int32_t)((nrows + rows_per_tile - 1) / rows_per_tile);
+    items[s] = (int32_t)(((nb + blocks_per_item - 1) / blocks_per_item) * ((nrows + rc_rows - 1) / rc_rows));
+  }
+}
+
+inline int grid_1d(int64_t n, int threads, int cap = 148 * 16) {
+  int64_t b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > cap) b = cap;
+  return (int)b;
+}
+
+template <typename T, int D>
+cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
+  using C = Cfg<D>;
+  const int G = a.hq / a.hkv;
+  const float qs2 = a.scale * kLog2e;
+  const int64_t rows = a.N * a.hq;
+  const T* q = static_cast<const T*>(a.q);
+  const T* kc = static_cast<const T*>(a.kc);
+  const T* vc = static_cast<const T*>(a.vc);
+  float* ob = static_cast<float*>(a.o_branch);
+  // plan
+  plan_counts_kernel<<<grid_1d(a.S + 1, 256), 256, 0, st>>>(a.cu_seqlens, a.blk->cu, a.S, G, C::ROWS, C::ROWS,
+                                                            kCmpRowChunk, a.tiles_cnt, a.items_cnt);
+  cudaError_t e = exclusive_scan(a.tiles_cnt, a.tiles_pre, a.S + 1, a.scan_tmp, st);
+  if (e != cudaSuccess) return e;
+  const int tile_grid = grid_1d(rows, C::ROWS, 148 * 8);
+  const dim3 g2(tile_grid, a.hkv);
+  cmp_lse_kernel<T, D><<<g2, 128, 0, st>>>(q, kc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
+                                           a.blk->count, qs2, a.lse);
+  cmp_out_topk_kernel<T, D><<<g2, 128, 0, st>>>(q, kc, vc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
+                                                a.blk->count, qs2, a.lse, ob, a.topk, a.sel);
+  const int pairs_per_cta = 128 / (G * C::NT);
+  slc_fwd_kernel<T, D><<<grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st>>>(
+      q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2,
+      ob + rows * D, a.lse + rows);
+  const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
+  win_fwd_kernel<T, D><<<gw, 128, 0, st>>>(q, static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.win->perm,
+                                           a.win->ptr, a.win->count, a.hq, a.hkv, qs2, ob + 2 * rows * D,
+                                           a.lse + 2 * rows);
+  combine_kernel<T, D><<<grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st>>>(ob, a.gates, rows, a.gate_mode,
+                                                                             static_cast<T*>(a.out));
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
+  using C = Cfg<D>;
+  const int G = a.hq / a.hkv;
+  const float qs2 = a.scale * kLog2e;
+  const int64_t rows = a.N * a.hq;
+  const int64_t btot = a.blk->count;
+  const T* q = static_cast<const T*>(a.q);
+  const T* k = static_cast<const T*>(a.k);
+  const T* v = static_cast<const T*>(a.v);
+  const T* kc = static_cast<const T*>(a.kc);
+  const T* vc = static_cast<const T*>(a.vc);
+  const T* ks = static_cast<const T*>(a.ks);
+  const T* vs = static_cast<const T*>(a.vs);
+  const float* ob = static_cast<const float*>(a.o_branch);
+  const T* dout = static_cast<const T*>(a.dout);
+
+  plan_counts_kernel<<<grid_1d(a.S + 1, 256), 256, 0, st>>>(a.cu_seqlens, a.blk->cu, a.S, G, C::ROWS, C::ROWS,
+                                                            kCmpRowChunk, a.tiles_cnt, a.items_cnt);
+  cudaError_t e = exclusive_scan(a.tiles_cnt, a.tiles_pre, a.S + 1, a.scan_tmp, st);
+  if (e != cudaSuccess) return e;
+  e = exclusive_scan(a.items_cnt, a.items_pre, a.S + 1, a.scan_tmp, st);
+  if (e != cudaSuccess) return e;
+
+  bwd_pre_kernel<T, D><<<grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st>>>(ob, dout, a.gates, rows, a.gate_mode,
+                                                                             a.Dc, a.dgates);
+  const dim3 g2(grid_1d(rows, C::ROWS, 148 * 8), a.hkv);
+  cmp_bwd_dq_kernel<T, D><<<g2, 128, 0, st>>>(q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu,
+                                              a.tiles_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.dq);
+  cudaMemsetAsync(a.dkc, 0, sizeof(float) * a.hkv * btot * D, st);
+  cudaMemsetAsync(a.dvc, 0, sizeof(float) * a.hkv * btot * D, st);
+  cmp_bwd_dkv_kernel<T, D><<<dim3(148 * 8, a.hkv), 128, 0, st>>>(
+      q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu, a.items_pre, a.S, a.hq, a.hkv, btot, qs2,
+      a.scale, kCmpRowChunk, a.lse, a.Dc, a.dkc, a.dvc);
+  const int pairs_per_cta = 128 / (G * C::NT);
+  slc_bwd_dq_kernel<T, D><<<grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st>>>(
+      q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
+      a.Dc + rows, a.dq);
+  // inverted selection CSR: for (g, b), the tokens whose group g selected b, ascending
+  const int64_t nsel = a.N * a.hkv * a.topk;
+  const int64_t nkeys = a.hkv * btot;
+  sel_keys_kernel<<<grid_1d(nsel, 256, 148 * 32), 256, 0, st>>>(a.sel, a.N, a.hkv, a.topk, btot, a.inv_keys_a,
+                                                                a.inv_vals_a);
+  int bits = 1;
+  while ((1ll << bits) <= nkeys) ++bits;
+  bool in_b = false;
+  e = radix_sort_pairs(a.inv_keys_a, a.inv_vals_a, a.inv_keys_b, a.inv_vals_b, nsel, bits, a.radix_tmp, &in_b, st);
+  if (e != cudaSuccess) return e;
+  const uint64_t* sk = in_b ? a.inv_keys_b : a.inv_keys_a;
+  const int32_t* sv = in_b ? a.inv_vals_b : a.inv_vals_a;
+  keys_to_ptr_kernel<<<grid_1d(nsel + 1, 256, 148 * 32), 256, 0, st>>>(sk, nsel, nkeys, a.inv_ptr);
+  slc_bwd_dkv_kernel<T, D><<<dim3(grid_1d(btot, 1, 148 * 16), a.hkv), 128, 0, st>>>(
+      q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.N, btot, a.hq, a.hkv, qs2,
+      a.scale, a.lse + rows, a.Dc + rows, a.dk, a.dv);
+  const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
+  win_bwd_dq_kernel<T, D><<<gw, 128, 0, st>>>(q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
+                                              a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
+                                              a.Dc + 2 * rows, a.dq);
+  win_bwd_dkv_kernel<T, D><<<gw, 128, 0, st>>>(q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
+                                               a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
+                                               a.Dc + 2 * rows, a.dk, a.dv);
+  cmp_scatter_kernel<<<grid_1d(a.N * a.hkv * D / 4, 256, 148 * 32), 256, 0, st>>>(
+      a.dkc, a.dvc, a.blk->id, a.blk->ptr, a.N, btot, a.hkv, D, a.dk, a.dv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st) {
+  if (a.dtype == SSA_DTYPE_BF16) {
+    if (a.d == 32) return forward_impl<__nv_bfloat16, 32>(a, st);
+    if (a.d == 64) return forward_impl<__nv_bfloat16, 64>(a, st);
+  } else {
+    if (a.d == 32) return forward_impl<float, 32>(a, st);
+    if (a.d == 64) return forward_impl<float, 64>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st) {
+  if (a.dtype == SSA_DTYPE_BF16) {
+    if (a.d == 32) return backward_impl<__nv_bfloat16, 32>(a, st);
+    if (a.d == 64) return backward_impl<__nv_bfloat16, 64>(a, st);
+  } else {
+    if (a.d == 32) return backward_impl<float, 32>(a, st);
+    if (a.d == 64) return backward_impl<float, 64>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ssa

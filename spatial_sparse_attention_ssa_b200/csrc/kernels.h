@@ -1,0 +1,65 @@
+// Argument bundles passed from the C ABI layer to the kernel launchers (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssa.h"
+
+namespace ssa {
+
+// Query rows per work item of the compressed-branch dKc/dVc kernel.
+constexpr int kCmpRowChunk = 2048;
+
+struct FwdArgs {
+  int dtype, d, hq, hkv, topk, gate_mode;
+  float scale;
+  int32_t S;
+  int64_t N;
+  const int32_t* cu_seqlens;
+  const ssa_partition* blk;
+  const ssa_partition* win;
+  const void *q, *k, *v;
+  const float* gates;
+  void* out;
+  // saved
+  void *kc, *vc, *ks, *vs;
+  float* o_branch;
+  float* lse;
+  int32_t* sel;
+  // workspace
+  int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
+};
+
+struct BwdArgs {
+  int dtype, d, hq, hkv, topk, gate_mode;
+  float scale;
+  int32_t S;
+  int64_t N;
+  const int32_t* cu_seqlens;
+  const ssa_partition* blk;
+  const ssa_partition* win;
+  const void *q, *k, *v;
+  const float* gates;
+  const void *kc, *vc, *ks, *vs;
+  const float* o_branch;
+  const float* lse;
+  const int32_t* sel;
+  const void* dout;
+  float *dq, *dk, *dv, *dgates;
+  // workspace
+  float* Dc;          // [3, N, Hq]
+  float *dkc, *dvc;   // [Hkv, B, d]
+  uint64_t *inv_keys_a, *inv_keys_b;
+  int32_t *inv_vals_a, *inv_vals_b;
+  int32_t* inv_ptr;   // [Hkv * B + 1]
+  int32_t* radix_tmp;
+  int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
+};
+
+cudaError_t launch_pool(int dtype, const void* k, const void* v, const ssa_partition* blk, int64_t N, int hkv,
+                        int d, void* ks, void* vs, void* kc, void* vc, cudaStream_t st);
+cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st);
+cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st);
+
+}  // namespace ssa

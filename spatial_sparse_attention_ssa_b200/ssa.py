@@ -1,0 +1,254 @@
+"""ctypes binding of libssa.so (argument marshalling only).
+
+Each call here converts torch tensors to device pointers, sizes and the
+current CUDA stream, allocates the caller-owned outputs and workspace with
+torch, and calls the C ABI of include/ssa.h.  Every step of the attention
+runs in the library's CUDA kernels; there is no CPU path.  A missing or
+unloadable library raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssa.so")
+
+SSA_OK = 0
+STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED", 3: "SSA_ERR_WORKSPACE",
+                4: "SSA_ERR_COORD_RANGE", 5: "SSA_ERR_CUDA", 6: "SSA_ERR_TIMEOUT"}
+DTYPE_BF16, DTYPE_F32 = 0, 1
+GATE_WEIGHTS, GATE_LOGITS = 0, 1
+OP_BIN, OP_FORWARD, OP_BACKWARD = 0, 1, 2
+
+EXPORTS = ("ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size", "ssa_error_string",
+           "ssa_get_device_status", "ssa_version")
+
+
+class SSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s (%s)" % (where, STATUS_NAMES.get(status, status),
+                                                 _lib().ssa_error_string(status).decode()))
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("hq", ctypes.c_int32), ("hkv", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("m_cmp", ctypes.c_int32), ("m_win", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("gate_mode", ctypes.c_int32)]
+
+
+class Partition(ctypes.Structure):
+    _fields_ = [("id", ctypes.c_void_p), ("perm", ctypes.c_void_p), ("ptr", ctypes.c_void_p),
+                ("cu", ctypes.c_void_p), ("key", ctypes.c_void_p), ("count", ctypes.c_int64)]
+
+
+class Saved(ctypes.Structure):
+    _fields_ = [("kc", ctypes.c_void_p), ("vc", ctypes.c_void_p), ("ks", ctypes.c_void_p),
+                ("vs", ctypes.c_void_p), ("o_branch", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("sel", ctypes.c_void_p)]
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libssa.so is not built (python -m spatial_sparse_attention_ssa_b200.build)")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        pp = ctypes.POINTER(Partition)
+        lib.ssa_bin.argtypes = [vp, vp, i32, i64, i32, i32, i32, pp, pp, vp, sz, vp]
+        lib.ssa_bin.restype = ctypes.c_int
+        lib.ssa_forward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, pp, pp, vp, vp, vp, vp, vp,
+                                    ctypes.POINTER(Saved), vp, sz, vp]
+        lib.ssa_forward.restype = ctypes.c_int
+        lib.ssa_backward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, pp, pp, vp, vp, vp, vp,
+                                     ctypes.POINTER(Saved), vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.ssa_backward.restype = ctypes.c_int
+        lib.ssa_workspace_size.argtypes = [i32, ctypes.POINTER(Params), i32, i64, i64, i64]
+        lib.ssa_workspace_size.restype = sz
+        lib.ssa_error_string.argtypes = [ctypes.c_int]
+        lib.ssa_error_string.restype = ctypes.c_char_p
+        lib.ssa_get_device_status.argtypes = [vp]
+        lib.ssa_get_device_status.restype = ctypes.c_int
+        lib.ssa_version.argtypes = []
+        lib.ssa_version.restype = i32
+        _LIB = lib
+    return _LIB
+
+
+def lib():
+    """The loaded ctypes library (raises if it is not built)."""
+    return _lib()
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(device: torch.device | None = None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != SSA_OK:
+        raise SSAError(status, where)
+
+
+def _require_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("SSA tensors must be contiguous CUDA tensors")
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------
+# binning
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class Bins:
+    """One partition (blocks or windows): device int32 tensors + count."""
+    id: torch.Tensor
+    perm: torch.Tensor
+    ptr: torch.Tensor
+    cu: torch.Tensor
+    key: torch.Tensor
+    count: int
+
+    @staticmethod
+    def empty(n: int, s: int, device) -> "Bins":
+        z = lambda *shape: torch.empty(*shape, dtype=torch.int32, device=device)  # noqa: E731
+        return Bins(z(n), z(n), z(n + 1), z(s + 1), z(max(n, 1), 3), 0)
+
+    def c(self) -> Partition:
+        return Partition(_ptr(self.id), _ptr(self.perm), _ptr(self.ptr), _ptr(self.cu), _ptr(self.key),
+                         self.count)
+
+
+def ssa_bin(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cmp: int, m_win: int,
+            out: tuple[Bins, Bins] | None = None, workspace: torch.Tensor | None = None):
+    """Step 1: block and window partitions of the tokens.  Returns (blk, win)."""
+    _require_cuda(coords, cu_seqlens)
+    n = int(coords.shape[0])
+    s = int(cu_seqlens.shape[0]) - 1
+    dev = coords.device
+    blk, win = out if out is not None else (Bins.empty(n, s, dev), Bins.empty(n, s, dev))
+    L = _lib()
+    need = L.ssa_workspace_size(OP_BIN, None, s, n, n, n)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb, pw = blk.c(), win.c()
+    st = L.ssa_bin(_ptr(coords), _ptr(cu_seqlens), s, n, int(R), int(m_cmp), int(m_win),
+                   ctypes.byref(pb), ctypes.byref(pw), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ssa_bin")
+    blk.count = int(pb.count)
+    win.count = int(pw.count)
+    return blk, win
+
+
+# ---------------------------------------------------------------------------
+# forward / backward
+# ---------------------------------------------------------------------------
+
+
+def make_params(hq, hkv, d, m_cmp, m_win, topk, dtype: torch.dtype, gate_mode: int,
+                scale: float = 0.0) -> Params:
+    dt = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32 if dtype == torch.float32 else None
+    if dt is None:
+        raise ValueError("dtype must be torch.bfloat16 or torch.float32")
+    return Params(hq, hkv, d, m_cmp, m_win, topk, scale, dt, gate_mode)
+
+
+@dataclass
+class SavedTensors:
+    kc: torch.Tensor
+    vc: torch.Tensor
+    ks: torch.Tensor
+    vs: torch.Tensor
+    o_branch: torch.Tensor
+    lse: torch.Tensor
+    sel: torch.Tensor
+
+    @staticmethod
+    def empty(p: Params, n: int, btot: int, dtype, device) -> "SavedTensors":
+        return SavedTensors(
+            torch.empty(p.hkv, max(btot, 1), p.d, dtype=dtype, device=device),
+            torch.empty(p.hkv, max(btot, 1), p.d, dtype=dtype, device=device),
+            torch.empty(p.hkv, n, p.d, dtype=dtype, device=device),
+            torch.empty(p.hkv, n, p.d, dtype=dtype, device=device),
+            torch.empty(3, n, p.hq, p.d, dtype=torch.float32, device=device),
+            torch.empty(3, n, p.hq, dtype=torch.float32, device=device),
+            torch.empty(n, p.hkv, p.topk, dtype=torch.int32, device=device))
+
+    def c(self) -> Saved:
+        return Saved(_ptr(self.kc), _ptr(self.vc), _ptr(self.ks), _ptr(self.vs), _ptr(self.o_branch),
+                     _ptr(self.lse), _ptr(self.sel))
+
+
+def workspace_size(op: int, p: Params, s: int, n: int, btot: int, wtot: int) -> int:
+    return int(_lib().ssa_workspace_size(op, ctypes.byref(p), s, n, btot, wtot))
+
+
+def ssa_forward(p: Params, cu_seqlens: torch.Tensor, blk: Bins, win: Bins, q: torch.Tensor,
+                k: torch.Tensor, v: torch.Tensor, gates: torch.Tensor, out: torch.Tensor | None = None,
+                saved: SavedTensors | None = None, workspace: torch.Tensor | None = None):
+    """Steps 2-6.  Returns (out [N, Hq, d], saved)."""
+    _require_cuda(cu_seqlens, q, k, v, gates)
+    n = int(q.shape[0])
+    s = int(cu_seqlens.shape[0]) - 1
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if saved is None:
+        saved = SavedTensors.empty(p, n, blk.count, q.dtype, dev)
+    need = workspace_size(OP_FORWARD, p, s, n, blk.count, win.count)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb, pw, sv = blk.c(), win.c(), saved.c()
+    st = _lib().ssa_forward(ctypes.byref(p), _ptr(cu_seqlens), s, n, ctypes.byref(pb), ctypes.byref(pw),
+                            _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), ctypes.byref(sv), _ptr(ws),
+                            ws.numel(), _stream(dev))
+    _check(st, "ssa_forward")
+    return out, saved
+
+
+def ssa_backward(p: Params, cu_seqlens: torch.Tensor, blk: Bins, win: Bins, q, k, v, gates,
+                 saved: SavedTensors, dout: torch.Tensor, grads=None, workspace: torch.Tensor | None = None):
+    """Step 7.  Returns (dq, dk, dv, dgates), all fp32."""
+    _require_cuda(cu_seqlens, q, k, v, gates, dout)
+    n = int(q.shape[0])
+    s = int(cu_seqlens.shape[0]) - 1
+    dev = q.device
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = (torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32),
+                 torch.empty(gates.shape, **f32))
+    dq, dk, dv, dg = grads
+    need = workspace_size(OP_BACKWARD, p, s, n, blk.count, win.count)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb, pw, sv = blk.c(), win.c(), saved.c()
+    st = _lib().ssa_backward(ctypes.byref(p), _ptr(cu_seqlens), s, n, ctypes.byref(pb), ctypes.byref(pw),
+                             _ptr(q), _ptr(k), _ptr(v), _ptr(gates), ctypes.byref(sv), _ptr(dout), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ssa_backward")
+    return dq, dk, dv, dg
+
+
+def device_status(stream: int | None = None) -> int:
+    return int(_lib().ssa_get_device_status(stream if stream is not None else _stream()))
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,75 @@
+"""The C-ABI library loads and exports every entry point the header declares.
+
+Runs without a GPU: only host-side calls (sizes, error strings, argument checks
+that return before any CUDA work) are made.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from spatial_sparse_attention_ssa_b200 import ssa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"SSA_API\s+[\w\s\*]+?\b(ssa_\w+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ssa.lib()
+    declared = _declared()
+    assert {"ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(ssa.EXPORTS) <= declared
+
+
+def test_host_side_calls():
+    lib = ssa.lib()
+    assert lib.ssa_version() >= 100
+    for code in range(7):
+        assert lib.ssa_error_string(code)
+    p = ssa.Params(32, 2, 64, 8, 8, 16, 0.0, ssa.DTYPE_BF16, ssa.GATE_LOGITS)
+    n, b = 131072, 2322
+    fw = ssa.workspace_size(ssa.OP_FORWARD, p, 1, n, b, b)
+    bw = ssa.workspace_size(ssa.OP_BACKWARD, p, 1, n, b, b)
+    assert fw > 0 and bw > 3 * n * 32 * 4
+    assert lib.ssa_workspace_size(ssa.OP_BIN, None, 1, n, n, n) > 16 * n
+    bad = ssa.Params(30, 4, 64, 8, 8, 16, 0.0, ssa.DTYPE_BF16, ssa.GATE_LOGITS)  # 30 % 4 != 0
+    assert ssa.workspace_size(ssa.OP_FORWARD, bad, 1, n, b, b) == 0
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("hq", 31, 1), ("hq", 30, 2), ("d", 48, 2), ("topk", 0, 1), ("topk", 33, 2), ("m_cmp", 0, 1), ("dtype", 7, 1),
+    ("gate_mode", 3, 1), ("scale", -1.0, 1), ("hkv", 1, 2),  # G = 32 with d = 64 is not handled
+])
+def test_argument_errors_are_status_codes(field, value, code):
+    lib = ssa.lib()
+    p = ssa.Params(32, 2, 64, 8, 8, 16, 0.0, ssa.DTYPE_BF16, ssa.GATE_LOGITS)
+    setattr(p, field, value)
+    part = ssa.Partition(1, 1, 1, 1, 1, 10)
+    saved = ssa.Saved(1, 1, 1, 1, 1, 1, 1)
+    st = lib.ssa_forward(ctypes.byref(p), 1, 1, 100, ctypes.byref(part), ctypes.byref(part), 1, 1, 1, 1, 1,
+                         ctypes.byref(saved), 1, 1 << 30, None)
+    assert st == code
+
+
+def test_bin_rejects_bad_arguments_before_launching():
+    lib = ssa.lib()
+    part = ssa.Partition(1, 1, 1, 1, 1, 0)
+    null = ssa.Partition(None, 1, 1, 1, 1, 0)
+    assert lib.ssa_bin(1, 1, 1, 10, 64, 0, 4, ctypes.byref(part), ctypes.byref(part), 1, 1 << 20, None) == 1
+    assert lib.ssa_bin(1, 1, 1, 10, 64, 4, 4, ctypes.byref(null), ctypes.byref(part), 1, 1 << 20, None) == 1
+    assert lib.ssa_bin(1, 1, 1, 10, 1 << 21, 4, 4, ctypes.byref(part), ctypes.byref(part), 1, 1 << 20, None) == 1
+    assert lib.ssa_bin(1, 1, 1, 10, 64, 4, 4, ctypes.byref(part), ctypes.byref(part), 1, 16, None) == 3
+    # sequence bits + 3 x cell bits above 64: 2^20 grid with unit cells and 2^5 sequences
+    assert lib.ssa_bin(1, 1, 32, 10, 1 << 20, 1, 1, ctypes.byref(part), ctypes.byref(part), 1, 1 << 30,
+                       None) == 2

@@ -448,3 +448,13 @@ def test_subset_forward_matches_full():
     st2 = _run(w, t, tokens=toks)
     np.testing.assert_array_equal(st2["out"][toks], st["out"][toks])
     np.testing.assert_array_equal(st2["sel"][toks], st["sel"][toks])
+
+
+def test_dq_rows_matches_full_backward():
+    w, t = _small_workload(seed=6, n_seqs=2)
+    st = _run(w, t)
+    do = t.as_f32("do").astype(np.float64)
+    g = O.backward(st, do)
+    toks = np.array([0, 3, w.n - 1, int(w.cu_seqlens[1])])
+    st2 = _run(w, t, tokens=toks)
+    np.testing.assert_allclose(O.dq_rows(st2, do, toks), g["dq"][toks], rtol=1e-10, atol=1e-12)
