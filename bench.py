@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""SSA forward + backward throughput on one B200 per rank.
+
+A step is one pass of the whole SSA hot path -- binning (ssa_bin), compression,
+compressed attention + top-k selection, selected-block and window attention,
+the gated combine (ssa_forward) and the backward of all of it (ssa_backward) --
+over the 1024^3 surface-shell workload with exactly 131072 voxel tokens
+(32 query / 2 KV heads, d = 64, m_cmp = m_win = 8, top-k = 16, bf16 inputs,
+fp32 accumulation, gate logits).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch with torch.distributed.run: every rank runs its own
+independent workload (seeded by rank; no data-path collective) and the time is
+the max over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSA fwd+bwd voxel tokens/s at 128k tokens; % of bf16 tensor / HBM peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=131072,
+                    help="tokens of the 1024^3 workload (131072 is the benchmark; smaller only for ncu captures)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def _workload(seed: int, tokens: int = 131072):
+    from spatial_sparse_attention_ssa_b200 import workloads as W
+    return W.gigascale1024(seed, n_keep=tokens, backward=True)
+
+
+def _workload_desc(w, nb, nw):
+    return {"workload": "1024^3 surface shell of 5 ellipsoids + 2 slabs (semi-axes U(20,50)), subsampled to "
+                        "%d voxel tokens; SSA fwd+bwd, 32 query / 2 KV heads, d=64, m_cmp=m_win=8, "
+                        "top-k=16, bf16 in / fp32 accumulate, sigmoid gate logits" % w.n,
+            "tokens": w.n, "blocks": nb, "windows": nw, "sequences": w.s}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+               "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.th = threading.Thread(target=self._read, daemon=True)
+        self.th.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per kernel (flops / bytes per launch)
+# ---------------------------------------------------------------------------
+
+def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
+    """Per kernel name: (bound, algorithmic units per launch, unit).
+
+    Scores: compressed = sum over sequences of n_s * Hq * B_s; selected = sum
+    over (token, group) of G * (tokens in the selected blocks); window = Hq *
+    sum over windows of n_w^2.  Contraction flops per score: 2d for each
+    q.k / p.v / dO.v / ds.k / ds^T.q / p^T.dO the kernel performs.
+    """
+    d, hq, hkv = w.d, w.hq, w.hkv
+    G = hq // hkv
+    nb_s = np.diff(blk_cu)
+    n_s = np.diff(w.cu_seqlens)
+    sc_cmp = float(np.sum(n_s.astype(np.float64) * hq * nb_s))
+    bsize = np.diff(blk_ptr).astype(np.float64)
+    selv = sel.reshape(-1)
+    sc_slc = float(G * np.sum(bsize[selv[selv >= 0]]))
+    wsize = np.diff(win_ptr).astype(np.float64)
+    sc_win = float(hq * np.sum(wsize ** 2))
+    e = 2  # bf16 bytes
+    N, B = w.n, len(bsize)
+    work = {
+        "cmp_lse_kernel": ("flops", 2 * d * sc_cmp),
+        "cmp_out_topk_kernel": ("flops", 4 * d * sc_cmp),
+        "slc_fwd_kernel": ("flops", 4 * d * sc_slc),
+        "win_fwd_kernel": ("flops", 4 * d * sc_win),
+        "cmp_bwd_dq_kernel": ("flops", 6 * d * sc_cmp),
+        "cmp_bwd_dkv_kernel": ("flops", 8 * d * sc_cmp),
+        "slc_bwd_dq_kernel": ("flops", 6 * d * sc_slc),
+        "slc_bwd_dkv_kernel": ("flops", 8 * d * sc_slc),
+        "win_bwd_dq_kernel": ("flops", 6 * d * sc_win),
+        "win_bwd_dkv_kernel": ("flops", 8 * d * sc_win),
+        "pool_kernel": ("bytes", 4.0 * N * hkv * d * e + 2.0 * B * hkv * d * e),
+        "combine_kernel": ("bytes", 3.0 * N * hq * d * 4 + N * hq * 3 * 4 + N * hq * d * e),
+        "bwd_pre_kernel": ("bytes", 3.0 * N * hq * d * 4 + N * hq * d * e + N * hq * 3 * 4 * 3),
+    }
+    scores = {"cmp": sc_cmp, "slc": sc_slc, "win": sc_win}
+    return work, scores
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+
+    from spatial_sparse_attention_ssa_b200 import ssa
+    from spatial_sparse_attention_ssa_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    w = _workload(a.seed + rank, a.tokens)
+    t = W.make_tensors(w)
+
+    def to_dev(x, bf=True):
+        if bf and x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+
+    coords = to_dev(w.coords.astype(np.int32), False)
+    cu = to_dev(w.cu_seqlens.astype(np.int32), False)
+    q, k, v, do = to_dev(t.q), to_dev(t.k), to_dev(t.v), to_dev(t.do)
+    gates = to_dev(t.gates, False)
+    p = ssa.make_params(w.hq, w.hkv, w.d, w.m_cmp, w.m_win, w.topk, torch.bfloat16, w.gate_mode)
+    n, s = w.n, w.s
+    bins = (ssa.Bins.empty(n, s, dev), ssa.Bins.empty(n, s, dev))
+    ws_bin = torch.empty(ssa.lib().ssa_workspace_size(ssa.OP_BIN, None, s, n, n, n), dtype=torch.uint8, device=dev)
+    blk, win = ssa.ssa_bin(coords, cu, w.R, w.m_cmp, w.m_win, out=bins, workspace=ws_bin)
+    saved = ssa.SavedTensors.empty(p, n, blk.count, torch.bfloat16, dev)
+    out = torch.empty_like(q)
+    grads = (torch.empty(q.shape, dtype=torch.float32, device=dev), torch.empty(k.shape, dtype=torch.float32, device=dev),
+             torch.empty(v.shape, dtype=torch.float32, device=dev),
+             torch.empty(gates.shape, dtype=torch.float32, device=dev))
+    ws_f = torch.empty(max(256, ssa.workspace_size(ssa.OP_FORWARD, p, s, n, blk.count, win.count)), dtype=torch.uint8,
+                       device=dev)
+    ws_b = torch.empty(max(256, ssa.workspace_size(ssa.OP_BACKWARD, p, s, n, blk.count, win.count)),
+                       dtype=torch.uint8, device=dev)
+
+    def step(cx=coords, cux=cu, qx=q, kx=k, vx=v, gx=gates, dx=do):
+        b_, w_ = ssa.ssa_bin(cx, cux, w.R, w.m_cmp, w.m_win, out=bins, workspace=ws_bin)
+        ssa.ssa_forward(p, cux, b_, w_, qx, kx, vx, gx, out=out, saved=saved, workspace=ws_f)
+        ssa.ssa_backward(p, cux, b_, w_, qx, kx, vx, gx, saved, dx, grads=grads, workspace=ws_b)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, device-timed per step, L2 flushed between steps
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", ""))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = ssa.launch_count()
+    ssa.profile_read()
+    ssa.profile_enable(True)
+    sampler.start()
+    wall0 = time.perf_counter()
+    for i in range(a.steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    ssa.profile_enable(False)
+    launches = ssa.launch_count() - launches0
+    prof = ssa.profile_read()
+    ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / a.steps
+    ms_max = ms
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+    total_tokens = n * world
+
+    # ---- end to end through host buffers (pinned), same metric
+    e2e = None
+    if not a.no_e2e:
+        host_in = {"coords": coords.cpu().pin_memory(), "cu": cu.cpu().pin_memory(), "q": q.cpu().pin_memory(),
+                   "k": k.cpu().pin_memory(), "v": v.cpu().pin_memory(), "gates": gates.cpu().pin_memory(),
+                   "do": do.cpu().pin_memory()}
+        dev_in = {kk: torch.empty_like(vv, device=dev) for kk, vv in host_in.items()}
+        host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory()] + \
+                   [torch.empty(g_.shape, dtype=g_.dtype).pin_memory() for g_ in grads]
+        h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+        d2h = sum(x.numel() * x.element_size() for x in host_out)
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(a.steps):
+            flush.zero_()
+            ee[i][0].record()
+            for kk in host_in:
+                dev_in[kk].copy_(host_in[kk], non_blocking=True)
+            step(dev_in["coords"], dev_in["cu"], dev_in["q"], dev_in["k"], dev_in["v"], dev_in["gates"],
+                 dev_in["do"])
+            for src, dst in zip([out, *grads], host_out):
+                dst.copy_(src, non_blocking=True)
+            ee[i][1].record()
+        torch.cuda.synchronize()
+        e_ms = sum(a_.elapsed_time(b_) for a_, b_ in ee) / a.steps
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": total_tokens / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---- roofline of the dominant kernel
+    peaks = _peaks()
+    blk_ptr = blk.ptr[:blk.count + 1].cpu().numpy()
+    blk_cu = blk.cu.cpu().numpy()
+    win_ptr = win.ptr[:win.count + 1].cpu().numpy()
+    sel = saved.sel.cpu().numpy()
+    work, scores = kernel_work(w, blk_ptr, blk_cu, win_ptr, sel)
+    per_kernel = {}
+    step_ms_kernels = 0.0
+    for name, (tot, cnt) in prof.items():
+        per_kernel[name] = {"ms_per_step": tot / a.steps, "launches": cnt, "ms_per_launch": tot / max(cnt, 1)}
+        step_ms_kernels += tot / a.steps
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
+    roof = None
+    if dom is not None:
+        avg_ms = prof[dom][0] / max(prof[dom][1], 1)
+        kind, units = work.get(dom, ("bytes", None))
+        mhz = peaks.get("sm_max_mhz", 1965.0)
+        if kind == "flops" and units is not None:
+            achieved = units / (avg_ms / 1e3) / 1e12
+            # the attention kernels in this build are fp32 SIMT (FFMA): ALU-bound
+            peak = SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+            roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "peak_source": "derived: %d SMs x %d FP32 lanes x 2 flop x %.0f MHz" % (SMS, FP32_LANES_PER_SM, mhz),
+                    "algorithmic_per_launch": units, "ms_per_launch": avg_ms}
+        elif units is not None:
+            achieved = units / (avg_ms / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": None, "peak_source": peaks["_source"],
+                    "algorithmic_per_launch": units, "ms_per_launch": avg_ms}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(w, t, a.cpu_seconds)
+
+    if rank == 0:
+        cfg = _workload_desc(w, blk.count, win.count)
+        cfg.update({"global_batch": world, "parallelism": "dp%d" % world,
+                    "l2": "256 MB buffer written between timed steps (L2 is 126 MB); step working set ~6 GB",
+                    "scores": scores})
+        line = {"metric": METRIC, "value": total_tokens / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+                "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded surface-shell voxels, N(0,1) bf16 Q/K/V/dO, N(0,1) gate logits)",
+                "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+                "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel,
+                "peaks_source": peaks["_source"]}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle leg
+# ---------------------------------------------------------------------------
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def _oracle_sample(w, t, tokens):
+    from oracle import ssa_oracle as O
+    st = O.forward(w.coords, w.cu_seqlens, t.as_f32("q"), t.as_f32("k"), t.as_f32("v"), t.gates, hq=w.hq,
+                   hkv=w.hkv, m_cmp=w.m_cmp, m_win=w.m_win, topk=w.topk, gate_mode=w.gate_mode,
+                   pool_rounding="bf16", tokens=tokens)
+    O.dq_rows(st, t.as_f32("do"), tokens)
+
+
+def _sample_tokens(w, n):
+    return np.linspace(0, w.n - 1, num=max(1, n)).astype(np.int64)
+
+
+def cpu_baseline(w, t, seconds: float) -> dict:
+    """The oracle as it stands, on a bounded sample: binning + pooling of all
+    tokens, then every forward branch and the dQ rows for T sampled query tokens."""
+    t0 = time.perf_counter()
+    _oracle_sample(w, t, _sample_tokens(w, 16))
+    t1 = time.perf_counter() - t0
+    T = int(max(16, min(w.n, 16 * seconds / max(t1, 1e-3))))
+    t0 = time.perf_counter()
+    _oracle_sample(w, t, _sample_tokens(w, T))
+    el = time.perf_counter() - t0
+    return {"value": T / el, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": "numpy fp64 oracle: binning + mean pooling of all %d tokens, then compressed attention + "
+                      "top-k, selected and window attention and the dQ rows of %d evenly spaced query tokens "
+                      "(dK/dV, which need every query, not included); %.1f s" % (w.n, T, el),
+            "seconds": el}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from spatial_sparse_attention_ssa_b200 import workloads as W
+    w = _workload(a.seed)
+    t = W.make_tensors(w)
+    budget = max(2.0, 150.0 / max(1, a.steps + a.warmup))  # whole run within a few minutes
+    t0 = time.perf_counter()
+    _oracle_sample(w, t, _sample_tokens(w, 8))
+    t1 = time.perf_counter() - t0
+    T = int(max(8, min(w.n, 8 * budget / max(t1, 1e-3))))
+    for _ in range(a.warmup):
+        _oracle_sample(w, t, _sample_tokens(w, T))
+    times = []
+    for _ in range(a.steps):
+        t0 = time.perf_counter()
+        _oracle_sample(w, t, _sample_tokens(w, T))
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = T / (ms / 1e3)
+    cores = _blas_threads()
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded workload as the GPU arm)",
+            "config": _workload_desc(w, None, None), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "per step: binning + pooling of all tokens, then forward branches and dQ "
+                                       "rows of %d evenly spaced query tokens" % T},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = _args()
+    if a.warmup < 0 or a.steps < 1:
+        raise SystemExit("bad --steps / --warmup")
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

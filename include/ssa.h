@@ -166,6 +166,22 @@ SSA_API const char* ssa_error_string(ssa_status status);
  */
 SSA_API ssa_status ssa_get_device_status(void* stream);
 
+/*
+ * Tracing (no counterpart on the pages; used by the benchmark to time kernels).
+ * ssa_launch_count: number of kernels this library has launched in this
+ * process (all devices, all streams).  ssa_profile_enable(1): from now on,
+ * record a CUDA event pair on the launching stream around every launch;
+ * ssa_profile_enable(0) stops recording.  ssa_profile_read synchronises the
+ * recorded events, writes per kernel name (at most max_entries rows, names
+ * truncated to name_len-1 chars, NUL-terminated, row i at names + i*name_len)
+ * the summed milliseconds and launch counts, clears the records and returns
+ * the number of distinct names.  Any output pointer may be NULL.
+ */
+SSA_API uint64_t ssa_launch_count(void);
+SSA_API void ssa_profile_enable(int32_t on);
+SSA_API int32_t ssa_profile_read(char* names, int32_t name_len, float* total_ms, int32_t* launches,
+                                 int32_t max_entries);
+
 /* Library version as major*10000 + minor*100 + patch. */
 SSA_API int32_t ssa_version(void);
 

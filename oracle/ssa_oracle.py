@@ -200,7 +200,6 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
     query tokens (all other rows are NaN / -2); binning and compression are
     always complete.
     """
-    q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     n, _, d = q.shape
@@ -218,8 +217,12 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
         tokens = np.arange(n)
     tokens = np.asarray(tokens, dtype=np.int64)
 
+    def qrows(idx, hs):  # exact float64 copies of the needed query rows only
+        return np.asarray(q[idx, hs, :], dtype=np.float64)
+
+    # rows of tokens outside `tokens` are left unset (lse NaN, sel -2, o/out undefined)
     lse = np.full((3, n, hq), np.nan)
-    o = np.full((3, n, hq, d), np.nan)
+    o = np.empty((3, n, hq, d))
     sel = np.full((n, hkv, topk), -2, dtype=np.int64)
 
     # --- compressed branch + selection, per sequence and group, chunked over tokens
@@ -234,7 +237,7 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
             vcg = vc[b0:b1, g, :]
             for c0 in range(0, len(toks), chunk):
                 tt = toks[c0:c0 + chunk]
-                l_, o_, p_ = cmp_attention(q[tt, hs, :], kcg, vcg, scale)
+                l_, o_, p_ = cmp_attention(qrows(tt, hs), kcg, vcg, scale)
                 lse[0, tt, hs] = l_
                 o[0, tt, hs, :] = o_
                 imp = p_.sum(axis=1)  # [n, B_s]: probabilities summed over the group's heads
@@ -245,19 +248,20 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
     for t in tokens:
         for g in range(hkv):
             hs = slice(g * G, (g + 1) * G)
+            qt = qrows(t, hs)
             js = selected_tokens(sel[t, g], blk)
-            l_, o_, _ = _attend(q[t, hs, :], k[js, g, :], v[js, g, :], scale)
+            l_, o_, _ = _attend(qt, k[js, g, :], v[js, g, :], scale)
             lse[1, t, hs] = l_
             o[1, t, hs, :] = o_
             w = win["id"][t]
             jw = win["perm"][win["ptr"][w]:win["ptr"][w + 1]]
-            l_, o_, _ = _attend(q[t, hs, :], k[jw, g, :], v[jw, g, :], scale)
+            l_, o_, _ = _attend(qt, k[jw, g, :], v[jw, g, :], scale)
             lse[2, t, hs] = l_
             o[2, t, hs, :] = o_
 
-    gw = gate_weights(gates, gate_mode)  # [N, Hq, 3]
-    out = np.einsum("nhc,cnhd->nhd", gw, np.nan_to_num(o))
-    out[np.isnan(o[0, :, :, 0])] = np.nan
+    gw = gate_weights(gates[tokens], gate_mode)  # [T, Hq, 3]
+    out = np.empty((n, hq, d))
+    out[tokens] = np.einsum("nhc,cnhd->nhd", gw, o[:, tokens])
     st = State(blk=blk, win=win, kc=kc, vc=vc, lse=lse, o=o, sel=sel, out=out, scale=scale,
                q=q, k=k, v=v, gates=np.asarray(gates, np.float64), gate_mode=gate_mode,
                hq=hq, hkv=hkv, G=G, topk=topk, cu_seqlens=cu_seqlens, tokens=tokens)
@@ -271,7 +275,8 @@ def importance(st: State, t: int, g: int) -> np.ndarray:
     b0, b1 = int(st["blk"]["cu"][s]), int(st["blk"]["cu"][s + 1])
     G = st["G"]
     hs = slice(g * G, (g + 1) * G)
-    _, _, p = cmp_attention(st["q"][t:t + 1, hs, :], st["kc"][b0:b1, g, :], st["vc"][b0:b1, g, :],
+    _, _, p = cmp_attention(np.asarray(st["q"][t:t + 1, hs, :], np.float64), st["kc"][b0:b1, g, :],
+                            st["vc"][b0:b1, g, :],
                             st["scale"])
     return p[0].sum(axis=0)
 
@@ -282,7 +287,8 @@ def attend_with_sel(st: State, t: int, g: int, sel_row: np.ndarray):
     G = st["G"]
     hs = slice(g * G, (g + 1) * G)
     js = selected_tokens(np.asarray(sel_row), st["blk"])
-    l_, o_, _ = _attend(st["q"][t, hs, :], st["k"][js, g, :], st["v"][js, g, :], st["scale"])
+    l_, o_, _ = _attend(np.asarray(st["q"][t, hs, :], np.float64), st["k"][js, g, :], st["v"][js, g, :],
+                        st["scale"])
     return l_, o_
 
 
@@ -294,7 +300,7 @@ def attend_with_sel(st: State, t: int, g: int, sel_row: np.ndarray):
 def backward(st: State, dout: np.ndarray, chunk: int = 256) -> dict:
     """Gradients of sum(dout * O) w.r.t. q, k, v and gates.  Requires a forward
     over all tokens.  Returns dq, dk, dv, dgates and the per-branch parts."""
-    q, k, v = st["q"], st["k"], st["v"]
+    q, k, v = np.asarray(st["q"], np.float64), st["k"], st["v"]
     n, hq, d = q.shape
     hkv, G, scale = st["hkv"], st["G"], st["scale"]
     assert len(st["tokens"]) == n, "backward needs the full forward"
@@ -404,7 +410,7 @@ def dq_rows(st: State, dout: np.ndarray, tokens) -> np.ndarray:
             )
             for c, (kk, vv) in enumerate(keysets):
                 dor = do * gw[t, hs, c][:, None]
-                sc = scale * (q[t, hs, :] @ kk.T)
+                sc = scale * (np.asarray(q[t, hs, :], np.float64) @ kk.T)
                 p = np.exp(sc - st["lse"][c, t, hs][:, None])
                 dp = dor @ vv.T
                 ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))

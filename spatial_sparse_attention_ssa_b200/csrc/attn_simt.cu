@@ -927,25 +927,25 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   const T* vc = static_cast<const T*>(a.vc);
   float* ob = static_cast<float*>(a.o_branch);
   // plan
-  plan_counts_kernel<<<grid_1d(a.S + 1, 256), 256, 0, st>>>(a.cu_seqlens, a.blk->cu, a.S, G, C::ROWS, C::ROWS,
+  SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu, a.S, G, C::ROWS, C::ROWS,
                                                             kCmpRowChunk, a.tiles_cnt, a.items_cnt);
   cudaError_t e = exclusive_scan(a.tiles_cnt, a.tiles_pre, a.S + 1, a.scan_tmp, st);
   if (e != cudaSuccess) return e;
   const int tile_grid = grid_1d(rows, C::ROWS, 148 * 8);
   const dim3 g2(tile_grid, a.hkv);
-  cmp_lse_kernel<T, D><<<g2, 128, 0, st>>>(q, kc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
+  SSA_LAUNCH("cmp_lse_kernel", (cmp_lse_kernel<T, D>), g2, 128, 0, st, q, kc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
                                            a.blk->count, qs2, a.lse);
-  cmp_out_topk_kernel<T, D><<<g2, 128, 0, st>>>(q, kc, vc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
+  SSA_LAUNCH("cmp_out_topk_kernel", (cmp_out_topk_kernel<T, D>), g2, 128, 0, st, q, kc, vc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
                                                 a.blk->count, qs2, a.lse, ob, a.topk, a.sel);
   const int pairs_per_cta = 128 / (G * C::NT);
-  slc_fwd_kernel<T, D><<<grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st>>>(
+  SSA_LAUNCH("slc_fwd_kernel", (slc_fwd_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
       q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2,
       ob + rows * D, a.lse + rows);
   const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
-  win_fwd_kernel<T, D><<<gw, 128, 0, st>>>(q, static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.win->perm,
+  SSA_LAUNCH("win_fwd_kernel", (win_fwd_kernel<T, D>), gw, 128, 0, st, q, static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.win->perm,
                                            a.win->ptr, a.win->count, a.hq, a.hkv, qs2, ob + 2 * rows * D,
                                            a.lse + 2 * rows);
-  combine_kernel<T, D><<<grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st>>>(ob, a.gates, rows, a.gate_mode,
+  SSA_LAUNCH("combine_kernel", (combine_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, a.gates, rows, a.gate_mode,
                                                                              static_cast<T*>(a.out));
   return cudaGetLastError();
 }
@@ -967,31 +967,31 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   const float* ob = static_cast<const float*>(a.o_branch);
   const T* dout = static_cast<const T*>(a.dout);
 
-  plan_counts_kernel<<<grid_1d(a.S + 1, 256), 256, 0, st>>>(a.cu_seqlens, a.blk->cu, a.S, G, C::ROWS, C::ROWS,
+  SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu, a.S, G, C::ROWS, C::ROWS,
                                                             kCmpRowChunk, a.tiles_cnt, a.items_cnt);
   cudaError_t e = exclusive_scan(a.tiles_cnt, a.tiles_pre, a.S + 1, a.scan_tmp, st);
   if (e != cudaSuccess) return e;
   e = exclusive_scan(a.items_cnt, a.items_pre, a.S + 1, a.scan_tmp, st);
   if (e != cudaSuccess) return e;
 
-  bwd_pre_kernel<T, D><<<grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st>>>(ob, dout, a.gates, rows, a.gate_mode,
+  SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout, a.gates, rows, a.gate_mode,
                                                                              a.Dc, a.dgates);
   const dim3 g2(grid_1d(rows, C::ROWS, 148 * 8), a.hkv);
-  cmp_bwd_dq_kernel<T, D><<<g2, 128, 0, st>>>(q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu,
+  SSA_LAUNCH("cmp_bwd_dq_kernel", (cmp_bwd_dq_kernel<T, D>), g2, 128, 0, st, q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu,
                                               a.tiles_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.dq);
   cudaMemsetAsync(a.dkc, 0, sizeof(float) * a.hkv * btot * D, st);
   cudaMemsetAsync(a.dvc, 0, sizeof(float) * a.hkv * btot * D, st);
-  cmp_bwd_dkv_kernel<T, D><<<dim3(148 * 8, a.hkv), 128, 0, st>>>(
+  SSA_LAUNCH("cmp_bwd_dkv_kernel", (cmp_bwd_dkv_kernel<T, D>), dim3(148 * 8, a.hkv), 128, 0, st, 
       q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu, a.items_pre, a.S, a.hq, a.hkv, btot, qs2,
       a.scale, kCmpRowChunk, a.lse, a.Dc, a.dkc, a.dvc);
   const int pairs_per_cta = 128 / (G * C::NT);
-  slc_bwd_dq_kernel<T, D><<<grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st>>>(
+  SSA_LAUNCH("slc_bwd_dq_kernel", (slc_bwd_dq_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
       q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
       a.Dc + rows, a.dq);
   // inverted selection CSR: for (g, b), the tokens whose group g selected b, ascending
   const int64_t nsel = a.N * a.hkv * a.topk;
   const int64_t nkeys = a.hkv * btot;
-  sel_keys_kernel<<<grid_1d(nsel, 256, 148 * 32), 256, 0, st>>>(a.sel, a.N, a.hkv, a.topk, btot, a.inv_keys_a,
+  SSA_LAUNCH("sel_keys_kernel", sel_keys_kernel, grid_1d(nsel, 256, 148 * 32), 256, 0, st, a.sel, a.N, a.hkv, a.topk, btot, a.inv_keys_a,
                                                                 a.inv_vals_a);
   int bits = 1;
   while ((1ll << bits) <= nkeys) ++bits;
@@ -1000,18 +1000,18 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const uint64_t* sk = in_b ? a.inv_keys_b : a.inv_keys_a;
   const int32_t* sv = in_b ? a.inv_vals_b : a.inv_vals_a;
-  keys_to_ptr_kernel<<<grid_1d(nsel + 1, 256, 148 * 32), 256, 0, st>>>(sk, nsel, nkeys, a.inv_ptr);
-  slc_bwd_dkv_kernel<T, D><<<dim3(grid_1d(btot, 1, 148 * 16), a.hkv), 128, 0, st>>>(
+  SSA_LAUNCH("keys_to_ptr_kernel", keys_to_ptr_kernel, grid_1d(nsel + 1, 256, 148 * 32), 256, 0, st, sk, nsel, nkeys, a.inv_ptr);
+  SSA_LAUNCH("slc_bwd_dkv_kernel", (slc_bwd_dkv_kernel<T, D>), dim3(grid_1d(btot, 1, 148 * 16), a.hkv), 128, 0, st, 
       q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.N, btot, a.hq, a.hkv, qs2,
       a.scale, a.lse + rows, a.Dc + rows, a.dk, a.dv);
   const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
-  win_bwd_dq_kernel<T, D><<<gw, 128, 0, st>>>(q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
+  SSA_LAUNCH("win_bwd_dq_kernel", (win_bwd_dq_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
                                               a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
                                               a.Dc + 2 * rows, a.dq);
-  win_bwd_dkv_kernel<T, D><<<gw, 128, 0, st>>>(q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
+  SSA_LAUNCH("win_bwd_dkv_kernel", (win_bwd_dkv_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
                                                a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
                                                a.Dc + 2 * rows, a.dk, a.dv);
-  cmp_scatter_kernel<<<grid_1d(a.N * a.hkv * D / 4, 256, 148 * 32), 256, 0, st>>>(
+  SSA_LAUNCH("cmp_scatter_kernel", cmp_scatter_kernel, grid_1d(a.N * a.hkv * D / 4, 256, 148 * 32), 256, 0, st, 
       a.dkc, a.dvc, a.blk->id, a.blk->ptr, a.N, btot, a.hkv, D, a.dk, a.dv);
   return cudaGetLastError();
 }

@@ -269,9 +269,9 @@ size_t scan_tmp_ints(int64_t n) { return (size_t)cdiv(n, kScanChunk) + 64; }
 cudaError_t exclusive_scan(const int32_t* in, int32_t* out, int64_t n, int32_t* tmp, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const int64_t nc = cdiv(n, kScanChunk);
-  scan_reduce_kernel<<<(unsigned)nc, kScanThreads, 0, st>>>(in, n, tmp);
-  scan_sums_kernel<<<1, kScanThreads, 0, st>>>(tmp, nc);
-  scan_apply_kernel<<<(unsigned)nc, kScanThreads, 0, st>>>(in, out, n, tmp);
+  SSA_LAUNCH("scan_reduce_kernel", scan_reduce_kernel, (unsigned)nc, kScanThreads, 0, st, in, n, tmp);
+  SSA_LAUNCH("scan_sums_kernel", scan_sums_kernel, 1, kScanThreads, 0, st, tmp, nc);
+  SSA_LAUNCH("scan_apply_kernel", scan_apply_kernel, (unsigned)nc, kScanThreads, 0, st, in, out, n, tmp);
   return cudaGetLastError();
 }
 
@@ -293,10 +293,10 @@ cudaError_t radix_sort_pairs(uint64_t* keys_a, int32_t* vals_a, uint64_t* keys_b
   uint64_t *ki = keys_a, *ko = keys_b;
   int32_t *vi = vals_a, *vo = vals_b;
   for (int shift = 0; shift < bits; shift += 8) {
-    radix_hist_kernel<<<num_tiles, kRadixThreads, 0, st>>>(ki, n, shift, num_tiles, counts);
+    SSA_LAUNCH("radix_hist_kernel", radix_hist_kernel, num_tiles, kRadixThreads, 0, st, ki, n, shift, num_tiles, counts);
     cudaError_t e = exclusive_scan(counts, offsets, m, scratch, st);
     if (e != cudaSuccess) return e;
-    radix_scatter_kernel<<<num_tiles, kRadixThreads, 0, st>>>(ki, vi, ko, vo, n, shift, num_tiles, offsets);
+    SSA_LAUNCH("radix_scatter_kernel", radix_scatter_kernel, num_tiles, kRadixThreads, 0, st, ki, vi, ko, vo, n, shift, num_tiles, offsets);
     std::swap(ki, ko);
     std::swap(vi, vo);
     *result_in_b = !*result_in_b;
@@ -337,26 +337,26 @@ cudaError_t bin_partition(const int32_t* coords, const int32_t* cu_seqlens, int3
   int32_t* excl = reinterpret_cast<int32_t*>(p); p += align256(sizeof(int32_t) * n);
   int32_t* tmp = reinterpret_cast<int32_t*>(p);
 
-  check_seqlens_kernel<<<grid_for(S + 1, 256), 256, 0, st>>>(cu_seqlens, S, N, d_status);
+  SSA_LAUNCH("check_seqlens_kernel", check_seqlens_kernel, grid_for(S + 1, 256), 256, 0, st, cu_seqlens, S, N, d_status);
   if (N == 0) {
     cudaMemsetAsync(out->cu, 0, sizeof(int32_t) * (S + 1), st);
     cudaMemsetAsync(out->ptr, 0, sizeof(int32_t), st);
     cudaMemsetAsync(d_count, 0, sizeof(int32_t), st);
     return cudaGetLastError();
   }
-  make_keys_kernel<<<grid_for(N, 256), 256, 0, st>>>(coords, cu_seqlens, S, N, R, m, cbits, keys_a, vals_a,
+  SSA_LAUNCH("make_keys_kernel", make_keys_kernel, grid_for(N, 256), 256, 0, st, coords, cu_seqlens, S, N, R, m, cbits, keys_a, vals_a,
                                                      d_status);
   bool in_b = false;
   cudaError_t e = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, N, bits, tmp, &in_b, st);
   if (e != cudaSuccess) return e;
   const uint64_t* ks = in_b ? keys_b : keys_a;
   const int32_t* vs = in_b ? vals_b : vals_a;
-  head_flags_kernel<<<grid_for(N, 256), 256, 0, st>>>(ks, N, flags);
+  SSA_LAUNCH("head_flags_kernel", head_flags_kernel, grid_for(N, 256), 256, 0, st, ks, N, flags);
   e = exclusive_scan(flags, excl, N, tmp, st);
   if (e != cudaSuccess) return e;
-  finalize_kernel<<<grid_for(N, 256), 256, 0, st>>>(ks, vs, flags, excl, N, cbits, out->id, out->perm, out->ptr,
+  SSA_LAUNCH("finalize_kernel", finalize_kernel, grid_for(N, 256), 256, 0, st, ks, vs, flags, excl, N, cbits, out->id, out->perm, out->ptr,
                                                     out->key, d_count);
-  seq_offsets_kernel<<<grid_for(S + 1, 256), 256, 0, st>>>(cu_seqlens, S, N, excl, d_count, out->cu);
+  SSA_LAUNCH("seq_offsets_kernel", seq_offsets_kernel, grid_for(S + 1, 256), 256, 0, st, cu_seqlens, S, N, excl, d_count, out->cu);
   return cudaGetLastError();
 }
 

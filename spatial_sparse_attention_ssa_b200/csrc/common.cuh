@@ -118,3 +118,18 @@ cudaError_t bin_partition(const int32_t* coords, const int32_t* cu_seqlens, int3
                           int* d_status, cudaStream_t st);
 
 }  // namespace ssa
+
+namespace ssa {
+// Tracing hooks (profile.cu): every library kernel launch is wrapped by these.
+void prof_begin(const char* name, cudaStream_t st);
+void prof_end(cudaStream_t st);
+}  // namespace ssa
+
+// Launch `kernel<<<grid, block, smem, st>>>(args...)` with launch counting and,
+// when enabled, per-kernel CUDA-event timing under `name`.
+#define SSA_LAUNCH(name, kernel, grid, block, smem, st, ...)  \
+  do {                                                       \
+    ::ssa::prof_begin(name, st);                             \
+    kernel<<<grid, block, smem, st>>>(__VA_ARGS__);          \
+    ::ssa::prof_end(st);                                     \
+  } while (0)

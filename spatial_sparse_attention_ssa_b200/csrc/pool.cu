@@ -61,11 +61,11 @@ cudaError_t launch_pool(int dtype, const void* k, const void* v, const ssa_parti
   const int threads = ((hkv * d + 31) / 32) * 32;
   const int grid = (int)(count_host < 148 * 64 ? count_host : 148 * 64);
   if (dtype == SSA_DTYPE_BF16) {
-    pool_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
+    SSA_LAUNCH("pool_kernel", (pool_kernel<__nv_bfloat16>), grid, threads, 0, st, 
         (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, blk->perm, blk->ptr, (int)count_host, N, hkv, d,
         (__nv_bfloat16*)ks, (__nv_bfloat16*)vs, (__nv_bfloat16*)kc, (__nv_bfloat16*)vc);
   } else {
-    pool_kernel<float><<<grid, threads, 0, st>>>((const float*)k, (const float*)v, blk->perm, blk->ptr,
+    SSA_LAUNCH("pool_kernel", (pool_kernel<float>), grid, threads, 0, st, (const float*)k, (const float*)v, blk->perm, blk->ptr,
                                                   (int)count_host, N, hkv, d, (float*)ks, (float*)vs, (float*)kc, (float*)vc);
   }
   return cudaGetLastError();

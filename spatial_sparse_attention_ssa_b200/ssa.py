@@ -26,7 +26,8 @@ GATE_WEIGHTS, GATE_LOGITS = 0, 1
 OP_BIN, OP_FORWARD, OP_BACKWARD = 0, 1, 2
 
 EXPORTS = ("ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size", "ssa_error_string",
-           "ssa_get_device_status", "ssa_version")
+           "ssa_get_device_status", "ssa_version", "ssa_launch_count", "ssa_profile_enable",
+           "ssa_profile_read")
 
 
 class SSAError(RuntimeError):
@@ -80,6 +81,13 @@ def _lib():
         lib.ssa_get_device_status.restype = ctypes.c_int
         lib.ssa_version.argtypes = []
         lib.ssa_version.restype = i32
+        lib.ssa_launch_count.argtypes = []
+        lib.ssa_launch_count.restype = ctypes.c_uint64
+        lib.ssa_profile_enable.argtypes = [i32]
+        lib.ssa_profile_enable.restype = None
+        lib.ssa_profile_read.argtypes = [ctypes.c_char_p, i32, ctypes.POINTER(ctypes.c_float),
+                                         ctypes.POINTER(ctypes.c_int32), i32]
+        lib.ssa_profile_read.restype = i32
         _LIB = lib
     return _LIB
 
@@ -248,6 +256,30 @@ def ssa_backward(p: Params, cu_seqlens: torch.Tensor, blk: Bins, win: Bins, q, k
 
 def device_status(stream: int | None = None) -> int:
     return int(_lib().ssa_get_device_status(stream if stream is not None else _stream()))
+
+
+def launch_count() -> int:
+    """Kernels this library has launched in this process."""
+    return int(_lib().ssa_launch_count())
+
+
+def profile_enable(on: bool) -> None:
+    _lib().ssa_profile_enable(1 if on else 0)
+
+
+def profile_read(max_entries: int = 128) -> dict:
+    """{kernel name: (total ms, launches)} recorded since the last read."""
+    L = _lib()
+    name_len = 64
+    names = ctypes.create_string_buffer(name_len * max_entries)
+    ms = (ctypes.c_float * max_entries)()
+    cnt = (ctypes.c_int32 * max_entries)()
+    n = min(L.ssa_profile_read(names, name_len, ms, cnt, max_entries), max_entries)
+    out = {}
+    for i in range(n):
+        nm = names.raw[i * name_len:(i + 1) * name_len].split(b"\0", 1)[0].decode()
+        out[nm] = (float(ms[i]), int(cnt[i]))
+    return out
 
 
 def default_scale(d: int) -> float:
