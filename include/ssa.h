@@ -117,6 +117,32 @@ SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int
                            ssa_partition* win, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ssa_bin_noalloc -- ssa_bin without a workspace argument, for callers that
+ * cannot allocate device memory when they bin (the pages have no counterpart:
+ * this is a property of the library, not of the method).  Examples: a plugin
+ * whose host application owns all device memory through its own pool, a
+ * latency-critical loop where cudaMalloc / cudaFree would synchronise the
+ * device, a process that reserved nearly all memory up front.
+ * The scratch is a fixed array in the library's device memory (about 11 MB on
+ * every GPU that loads the library, held until the process exits), so:
+ *   - N must be <= SSA_BIN_NOALLOC_MAX_TOKENS, else SSA_ERR_WORKSPACE and
+ *     nothing is enqueued;
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing any stream into a CUDA graph;
+ *   - all calls on a device share the array: calls whose GPU work overlaps
+ *     (other streams, other host threads) race and corrupt each other; the
+ *     array keeps the last call's contents, and each call clears the parts
+ *     that must start at zero.
+ * Arguments, outputs, synchronisation and error codes are those of ssa_bin.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define SSA_BIN_NOALLOC_MAX_TOKENS 262144
+SSA_API ssa_status ssa_bin_noalloc(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                                   int32_t R, int32_t m_cmp, int32_t m_win, ssa_partition* blk,
+                                   ssa_partition* win, void* stream);
+
+/*
  * ssa_forward -- steps 2-6: mean-pool compression; compressed attention of every
  * query against all blocks of its sequence; top-k block selection by the
  * softmax probability summed over the query heads of a GQA group (ties go to

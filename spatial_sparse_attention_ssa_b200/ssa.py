@@ -167,6 +167,33 @@ def ssa_bin(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cmp: int, 
     return blk, win
 
 
+def ssa_bin_noalloc(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cmp: int, m_win: int,
+                    out: tuple[Bins, Bins] | None = None):
+    """ssa_bin with the library's fixed internal scratch instead of a workspace,
+    for callers that cannot allocate device memory at binning time (up to
+    SSA_BIN_NOALLOC_MAX_TOKENS tokens; calls that overlap on the GPU race).
+    `out` must be preallocated by such callers; without it this wrapper
+    allocates the output tensors itself with torch."""
+    _require_cuda(coords, cu_seqlens)
+    n = int(coords.shape[0])
+    s = int(cu_seqlens.shape[0]) - 1
+    dev = coords.device
+    blk, win = out if out is not None else (Bins.empty(n, s, dev), Bins.empty(n, s, dev))
+    L = _lib()
+    fn = L.ssa_bin_noalloc
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                   ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(Partition), ctypes.POINTER(Partition),
+                   ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    pb, pw = blk.c(), win.c()
+    st = fn(_ptr(coords), _ptr(cu_seqlens), s, n, int(R), int(m_cmp), int(m_win), ctypes.byref(pb),
+            ctypes.byref(pw), _stream(dev))
+    _check(st, "ssa_bin_noalloc")
+    blk.count = int(pb.count)
+    win.count = int(pw.count)
+    return blk, win
+
+
 # ---------------------------------------------------------------------------
 # forward / backward
 # ---------------------------------------------------------------------------
