@@ -80,7 +80,7 @@ struct BwdWs {
   float* Dc;
   float *dkc, *dvc;
   uint64_t *ka, *kb;
-  int32_t *va, *vb, *inv_ptr, *radix_tmp;
+  int32_t *va, *vb, *inv_ptr, *radix_tmp, *slc_cnt, *slc_pre;
   int32_t *tc, *tp, *ic, *ip, *st;
 };
 
@@ -96,7 +96,11 @@ size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t 
   w->vb = c.take<int32_t>(nsel);
   w->inv_ptr = c.take<int32_t>(p->hkv * B + 1);
   w->radix_tmp = c.take<int32_t>(ssa::radix_tmp_ints(nsel));
-  carve_plan(c, S, &w->tc, &w->tp, &w->ic, &w->ip, &w->st);
+  w->slc_cnt = c.take<int32_t>(p->hkv * B + 1);
+  w->slc_pre = c.take<int32_t>(p->hkv * B + 1);
+  w->st = c.take<int32_t>(ssa::scan_tmp_ints(p->hkv * B + 1 > S + 1 ? p->hkv * B + 1 : S + 1));
+  int32_t* unused_st;
+  carve_plan(c, S, &w->tc, &w->tp, &w->ic, &w->ip, &unused_st);
   return c.used;
 }
 
@@ -304,6 +308,8 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.inv_vals_b = w.vb;
   a.inv_ptr = w.inv_ptr;
   a.radix_tmp = w.radix_tmp;
+  a.slc_cnt = w.slc_cnt;
+  a.slc_pre = w.slc_pre;
   a.tiles_cnt = w.tc;
   a.tiles_pre = w.tp;
   a.items_cnt = w.ic;

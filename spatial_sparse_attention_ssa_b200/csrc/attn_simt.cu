@@ -673,24 +673,67 @@ __global__ void __launch_bounds__(128) slc_bwd_dq_kernel(
   }
 }
 
-// selected branch: dK, dV per block, over the (token, group) pairs that selected it
+// selected branch: dK, dV per block, over the (token, group) pairs that selected it.
+// A work item is (group g, block b, chunk of kSlcRowChunk rows of the pairs that
+// selected b).  Threads split as (key slot, row slice): small blocks (the common
+// case, 1-2 tokens) use many row slices, large blocks many key slots.  Partial
+// dk/dv are reduced over row slices in shared memory and added to dK/dV (zeroed
+// beforehand) with fp32 atomics.
+constexpr int kSlcRowChunk = 1024;
+constexpr int kSlcStageRows = 64;
+
+template <typename T, int D>
+struct SlcStage {
+  float q[kSlcStageRows * Cfg<D>::KSTR];
+  float dO[kSlcStageRows * Cfg<D>::KSTR];
+  float lse2[kSlcStageRows];
+  float Dr[kSlcStageRows];
+};
+
+__global__ void slc_items_kernel(const int32_t* __restrict__ inv_ptr, int64_t nkeys, int G, int32_t* __restrict__ cnt) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i <= nkeys; i += (int64_t)gridDim.x * blockDim.x) {
+    if (i == nkeys) {
+      cnt[i] = 0;
+      continue;
+    }
+    const int64_t rows = (int64_t)(inv_ptr[i + 1] - inv_ptr[i]) * G;
+    cnt[i] = (int32_t)((rows + kSlcRowChunk - 1) / kSlcRowChunk);
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) slc_bwd_dkv_kernel(
     const T* __restrict__ q, const T* __restrict__ ks, const T* __restrict__ vs, const T* __restrict__ dout,
     const float* __restrict__ gates, int mode, const int32_t* __restrict__ bptr, const int32_t* __restrict__ bperm,
-    const int32_t* __restrict__ inv_ptr, const int32_t* __restrict__ inv_tok, int64_t N, int64_t btot, int hq, int hkv,
-    float qs2, float scale, const float* __restrict__ lse_in, const float* __restrict__ Dc, float* __restrict__ dk_out,
-    float* __restrict__ dv_out) {
-  using C = Cfg<D>;
-  __shared__ __align__(16) RowStage<T, D> st;
-  const int g = blockIdx.y, G = hq / hkv;
-  const int sub = threadIdx.x % C::NT;
-  for (int64_t b = blockIdx.x; b < btot; b += gridDim.x) {
+    const int32_t* __restrict__ inv_ptr, const int32_t* __restrict__ inv_tok, const int32_t* __restrict__ ipre,
+    int64_t N, int64_t btot, int hq, int hkv, float qs2, float scale, const float* __restrict__ lse_in,
+    const float* __restrict__ Dc, float* __restrict__ dk_out, float* __restrict__ dv_out) {
+  constexpr int NT = D / 32;
+  constexpr int SLOTS = 128 / NT;  // (key slot, row slice) pairs
+  __shared__ __align__(16) SlcStage<T, D> st;
+  constexpr int KMAX = 64;  // key slots per pass (the reduction buffers hold KMAX * D floats each)
+  static_assert(kSlcStageRows * Cfg<D>::KSTR >= KMAX * D, "reduction buffers must fit in the staging area");
+  const int G = hq / hkv;
+  const int sub = threadIdx.x % NT;
+  const int pair_id = threadIdx.x / NT;
+  const int64_t nkeys = (int64_t)hkv * btot;
+  const int nitems = ipre[nkeys];
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int64_t key = find_segment(ipre, (int)nkeys, item);  // g * btot + b
+    const int g = (int)(key / btot);
+    const int64_t b = key % btot;
+    const int chunk = item - ipre[key];
+    const int l0 = inv_ptr[key];
+    const int64_t nrows_all = (int64_t)(inv_ptr[key + 1] - l0) * G;
+    const int64_t r0 = (int64_t)chunk * kSlcRowChunk;
+    const int64_t r1 = min(nrows_all, r0 + kSlcRowChunk);
     const int p0 = bptr[b], nb = bptr[b + 1] - p0;
-    const int l0 = inv_ptr[g * btot + b], l1 = inv_ptr[g * btot + b + 1];
-    const int64_t nrows = (int64_t)(l1 - l0) * G;
-    for (int kp = 0; kp < nb; kp += C::ROWS) {
-      const int j = kp + threadIdx.x / C::NT;
+    int kpc = 1;
+    while (kpc < nb && kpc < KMAX) kpc <<= 1;
+    const int rs = SLOTS / kpc;
+    const int kslot = pair_id % kpc, rslice = pair_id / kpc;
+    for (int kp = 0; kp < nb; kp += kpc) {
+      const int j = kp + kslot;
       const bool validk = j < nb;
       const int64_t kidx = (int64_t)g * N + p0 + (validk ? j : 0);
       float kv[32], vv[32], dk[32], dv[32];
@@ -698,28 +741,70 @@ __global__ void __launch_bounds__(128) slc_bwd_dkv_kernel(
       load32(vs + kidx * D + sub * 32, vv);
 #pragma unroll
       for (int i = 0; i < 32; ++i) dk[i] = dv[i] = 0.f;
-      for (int64_t rs = 0; rs < nrows; rs += RowStage<T, D>::RT) {
-        const int n = (int)min((int64_t)RowStage<T, D>::RT, nrows - rs);
+      for (int64_t rsb = r0; rsb < r1; rsb += kSlcStageRows) {
+        const int n = (int)min((int64_t)kSlcStageRows, r1 - rsb);
         __syncthreads();
-        stage_query_rows<T, D>(
-            st, n,
-            [&](int i, int64_t* row) {
-              const int64_t gr = rs + i;
-              *row = (int64_t)inv_tok[l0 + gr / G] * hq + g * G + gr % G;
-              return true;
-            },
-            q, dout, gates, mode, 1, lse_in, Dc);
+        constexpr int QPR = D / 4;
+        for (int idx = threadIdx.x; idx < kSlcStageRows * QPR; idx += blockDim.x) {
+          const int i = idx / QPR, qd = idx % QPR;
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
+          int64_t row = 0;
+          const bool ok = i < n;
+          if (ok) {
+            const int64_t gr = rsb + i;
+            row = (int64_t)inv_tok[l0 + gr / G] * hq + g * G + gr % G;
+            a = load4(q + row * D + qd * 4);
+            c = load4(dout + row * D + qd * 4);
+            const float w = gate_weight(gates, row * 3 + 1, mode);
+            c.x *= w;
+            c.y *= w;
+            c.z *= w;
+            c.w *= w;
+          }
+          const int off = i * Cfg<D>::KSTR + (qd >> 3) * 36 + (qd & 7) * 4;
+          *reinterpret_cast<float4*>(st.q + off) = a;
+          *reinterpret_cast<float4*>(st.dO + off) = c;
+          if (qd == 0) {
+            st.lse2[i] = ok ? lse_in[row] * kLog2e : CUDART_INF_F;
+            st.Dr[i] = ok ? Dc[row] : 0.f;
+          }
+        }
         __syncthreads();
-        accumulate_rows<T, D>(st, kv, vv, qs2, dk, dv);
+        for (int i = rslice; i < kSlcStageRows; i += rs) {
+          const float* qrow = st.q + i * Cfg<D>::KSTR + sub * 36;
+          const float* drow = st.dO + i * Cfg<D>::KSTR + sub * 36;
+          const float s2 = row_sum<NT>(dot32(kv, qrow), 0xffffffffu) * qs2;
+          const float p = exp2f(s2 - st.lse2[i]);
+          const float dp = row_sum<NT>(dot32(vv, drow), 0xffffffffu);
+          const float ds = p * (dp - st.Dr[i]);
+          axpy32(dk, ds, qrow);
+          axpy32(dv, p, drow);
+        }
       }
+      // reduce over row slices (in the staging area, now free), then one atomic
+      // add per (key, dim)
+      float* red_k = st.q;
+      float* red_v = st.dO;
+      __syncthreads();
+      for (int i = threadIdx.x; i < kpc * D; i += blockDim.x) {
+        red_k[i] = 0.f;
+        red_v[i] = 0.f;
+      }
+      __syncthreads();
       if (validk) {
-        const int64_t tok = bperm[p0 + j];
-        float* a = dk_out + (tok * hkv + g) * D + sub * 32;
-        float* c = dv_out + (tok * hkv + g) * D + sub * 32;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          a[i] = dk[i] * scale;
-          c[i] = dv[i];
+          atomicAdd(&red_k[kslot * D + sub * 32 + i], dk[i]);
+          atomicAdd(&red_v[kslot * D + sub * 32 + i], dv[i]);
+        }
+      }
+      __syncthreads();
+      for (int i = threadIdx.x; i < kpc * D; i += blockDim.x) {
+        const int jj = kp + i / D;
+        if (jj < nb) {
+          const int64_t tok = bperm[p0 + jj];
+          atomicAdd(dk_out + (tok * hkv + g) * D + i % D, red_k[i] * scale);
+          atomicAdd(dv_out + (tok * hkv + g) * D + i % D, red_v[i]);
         }
       }
     }
@@ -1001,9 +1086,15 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   const uint64_t* sk = in_b ? a.inv_keys_b : a.inv_keys_a;
   const int32_t* sv = in_b ? a.inv_vals_b : a.inv_vals_a;
   SSA_LAUNCH("keys_to_ptr_kernel", keys_to_ptr_kernel, grid_1d(nsel + 1, 256, 148 * 32), 256, 0, st, sk, nsel, nkeys, a.inv_ptr);
-  SSA_LAUNCH("slc_bwd_dkv_kernel", (slc_bwd_dkv_kernel<T, D>), dim3(grid_1d(btot, 1, 148 * 16), a.hkv), 128, 0, st, 
-      q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.N, btot, a.hq, a.hkv, qs2,
-      a.scale, a.lse + rows, a.Dc + rows, a.dk, a.dv);
+  SSA_LAUNCH("slc_items_kernel", slc_items_kernel, grid_1d(nkeys + 1, 256, 148 * 32), 256, 0, st, a.inv_ptr, nkeys,
+             G, a.slc_cnt);
+  e = exclusive_scan(a.slc_cnt, a.slc_pre, nkeys + 1, a.scan_tmp, st);
+  if (e != cudaSuccess) return e;
+  cudaMemsetAsync(a.dk, 0, sizeof(float) * a.N * a.hkv * D, st);
+  cudaMemsetAsync(a.dv, 0, sizeof(float) * a.N * a.hkv * D, st);
+  SSA_LAUNCH("slc_bwd_dkv_kernel", (slc_bwd_dkv_kernel<T, D>), 148 * 8, 128, 0, st, q, ks, vs, dout, a.gates,
+             a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.slc_pre, a.N, btot, a.hq, a.hkv, qs2, a.scale,
+             a.lse + rows, a.Dc + rows, a.dk, a.dv);
   const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
   SSA_LAUNCH("win_bwd_dq_kernel", (win_bwd_dq_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
                                               a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,

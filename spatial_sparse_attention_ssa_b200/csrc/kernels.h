@@ -54,6 +54,7 @@ struct BwdArgs {
   int32_t *inv_vals_a, *inv_vals_b;
   int32_t* inv_ptr;   // [Hkv * B + 1]
   int32_t* radix_tmp;
+  int32_t *slc_cnt, *slc_pre;  // [Hkv * B + 1] work items of the selected-branch dK/dV kernel
   int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
 };
 
