@@ -1,5 +1,6 @@
 // C ABI of libssa: argument checks, workspace layout and launch order.
 #include <math.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -54,6 +55,16 @@ bool partition_ok(const ssa_partition* x) {
 
 float eff_scale(const ssa_params* p) { return p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->d); }
 
+// SSA_DISABLE_TC=1 selects the fp32 SIMT kernels for every shape (cross-checks).
+bool tc_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("SSA_DISABLE_TC");
+    v = (e && e[0] == '1') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 // Workspace of the forward (after `ws` base): plan arrays.
 void carve_plan(Carver& c, int32_t S, int32_t** tc, int32_t** tp, int32_t** ic, int32_t** ip, int32_t** st) {
   *tc = c.take<int32_t>(S + 1);
@@ -65,14 +76,15 @@ void carve_plan(Carver& c, int32_t S, int32_t** tc, int32_t** tp, int32_t** ic, 
 
 size_t bin_bytes(int32_t S, int64_t N) { return ssa::bin_ws_bytes(S, N) + 256; }
 
-size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W) {
-  (void)p;
+size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W, float** imp = nullptr,
+                 void* base = nullptr) {
   (void)N;
-  (void)B;
   (void)W;
-  Carver c(nullptr);
+  Carver c(base);
   int32_t *a, *b, *d, *e, *f;
   carve_plan(c, S, &a, &b, &d, &e, &f);
+  float* x = c.take<float>(ssa::cmp_tc_scratch_floats(p->hq, p->hkv, B));
+  if (imp) *imp = x;
   return c.used;
 }
 
@@ -228,6 +240,9 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   a.hkv = p->hkv;
   a.topk = p->topk;
   a.gate_mode = p->gate_mode;
+  a.use_tc = tc_enabled();
+  a.status = status_ptr();
+  if (!a.status) return SSA_ERR_CUDA;
   a.scale = eff_scale(p);
   a.S = S;
   a.N = N;
@@ -248,6 +263,7 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   a.sel = saved->sel;
   Carver c(ws);
   carve_plan(c, S, &a.tiles_cnt, &a.tiles_pre, &a.items_cnt, &a.items_pre, &a.scan_tmp);
+  fwd_bytes(p, S, N, blk->count, win->count, &a.imp_scratch, ws);
   return cuda_status(ssa::simt_forward(a, st));
 }
 
@@ -277,6 +293,9 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.hkv = p->hkv;
   a.topk = p->topk;
   a.gate_mode = p->gate_mode;
+  a.use_tc = tc_enabled();
+  a.status = status_ptr();
+  if (!a.status) return SSA_ERR_CUDA;
   a.scale = eff_scale(p);
   a.S = S;
   a.N = N;

@@ -1016,12 +1016,22 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
                                                             kCmpRowChunk, a.tiles_cnt, a.items_cnt);
   cudaError_t e = exclusive_scan(a.tiles_cnt, a.tiles_pre, a.S + 1, a.scan_tmp, st);
   if (e != cudaSuccess) return e;
-  const int tile_grid = grid_1d(rows, C::ROWS, 148 * 8);
-  const dim3 g2(tile_grid, a.hkv);
-  SSA_LAUNCH("cmp_lse_kernel", (cmp_lse_kernel<T, D>), g2, 128, 0, st, q, kc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
-                                           a.blk->count, qs2, a.lse);
-  SSA_LAUNCH("cmp_out_topk_kernel", (cmp_out_topk_kernel<T, D>), g2, 128, 0, st, q, kc, vc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
-                                                a.blk->count, qs2, a.lse, ob, a.topk, a.sel);
+  if (a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
+    // 128-row tiles for the tensor-core kernels
+    SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu,
+               a.S, G, 128, 128, kCmpRowChunk, a.items_cnt, a.tiles_cnt);
+    e = exclusive_scan(a.items_cnt, a.items_pre, a.S + 1, a.scan_tmp, st);
+    if (e != cudaSuccess) return e;
+    e = cmp_fwd_tc(a, a.items_pre, (a.N * G + 127) / 128 + a.S, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    const int tile_grid = grid_1d(rows, C::ROWS, 148 * 8);
+    const dim3 g2(tile_grid, a.hkv);
+    SSA_LAUNCH("cmp_lse_kernel", (cmp_lse_kernel<T, D>), g2, 128, 0, st, q, kc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
+                                             a.blk->count, qs2, a.lse);
+    SSA_LAUNCH("cmp_out_topk_kernel", (cmp_out_topk_kernel<T, D>), g2, 128, 0, st, q, kc, vc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
+                                                  a.blk->count, qs2, a.lse, ob, a.topk, a.sel);
+  }
   const int pairs_per_cta = 128 / (G * C::NT);
   SSA_LAUNCH("slc_fwd_kernel", (slc_fwd_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
       q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2,

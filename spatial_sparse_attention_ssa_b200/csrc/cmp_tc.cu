@@ -1,0 +1,841 @@
+// Compressed branch of SSA on the tcgen05 tensor cores (bf16 inputs, fp32
+// accumulation in TMEM), head dim 64.
+//
+// Direct3D-S2 (hyper.ai, "方法"): every query attends to all compressed blocks
+// of its sequence; the top-k blocks by that attention score are selected.  The
+// selection score of a block is its softmax probability summed over the query
+// heads of a GQA group (LSRM, shuwu5.cn, "阶段一").
+//
+// A row tile is 128 query rows = (128/G tokens) x (G heads of one KV group),
+// loaded by one 3D TMA box from Q [N, Hq, 64].  A key tile is 128 compressed
+// blocks of Kc/Vc [Hkv, B, 64] (2D TMA, 128-byte swizzle).
+//
+//   pass 1 (cmp_lse_tc):  S = Q Kc^T in TMEM, one thread per row keeps the
+//                         online max / sum of exp2 -> lse.
+//   pass 2 (cmp_out_tc):  S^T = Kc Q^T (one thread per block), p = exp2(s - lse)
+//                         with the final lse; the block's score for a token is
+//                         the sum of its G heads' p (registers); P^T goes to
+//                         shared memory as the MN-major A operand of
+//                         O += P Vc (TMEM accumulator); per-token top-k by
+//                         threshold filtering + insertion.
+//
+// Roles per CTA: warps 0-3 compute (thread i <-> TMEM lane i), warp 4 issues
+// TMA loads, warp 5 issues tcgen05.mma.  Every wait is bounded; on a timeout the
+// kernel records kStatusTimeout, drains what it issued (bounded) and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace ssa {
+namespace {
+
+using namespace tc;
+
+constexpr int kRows = 128;           // query rows per tile
+constexpr int kBN = 128;             // compressed blocks per key tile
+constexpr int kTile = 128 * 128;     // bytes of a 128 x 64 bf16 tile
+constexpr int kStages = 4;           // key-tile ring depth
+constexpr int kThreads = 192;        // 4 compute warps + TMA warp + MMA warp
+
+struct TileInfo {
+  int g, s, t0, t_end, b0, nb;
+};
+
+__device__ __forceinline__ TileInfo tile_info(int it, int ntiles, const int32_t* tpre, int S, const int32_t* cu,
+                                              const int32_t* bcu, int G) {
+  TileInfo ti;
+  ti.g = it / ntiles;
+  const int tile = it % ntiles;
+  ti.s = find_segment(tpre, S, tile);
+  ti.t0 = cu[ti.s] + (tile - tpre[ti.s]) * (kRows / G);
+  ti.t_end = cu[ti.s + 1];
+  ti.b0 = bcu[ti.s];
+  ti.nb = bcu[ti.s + 1] - ti.b0;
+  return ti;
+}
+
+__device__ __forceinline__ void record_timeout(int* status, int* abort_flag) {
+  atomicOr(status, kStatusTimeout);
+  *reinterpret_cast<volatile int*>(abort_flag) = 1;
+}
+
+__device__ __forceinline__ bool aborted(const int* abort_flag) {
+  return *reinterpret_cast<const volatile int*>(abort_flag) != 0;
+}
+
+// ---------------------------------------------------------------------------
+// pass 1: lse
+// ---------------------------------------------------------------------------
+struct LseSmem {
+  uint8_t q[2][kTile];
+  uint8_t kc[kStages][kTile];
+  uint64_t q_full[2], q_empty[2], mma_done;
+  uint64_t kc_full[kStages], kc_empty[kStages];
+  uint64_t s_full[2], s_empty[2];
+  uint32_t tmem;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) cmp_lse_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap, const int32_t* __restrict__ cu,
+    const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S, int hq, int hkv, int btot, float qs2,
+    float* __restrict__ lse_out, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  LseSmem& sm = *reinterpret_cast<LseSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = hq / hkv;
+  const int ntiles = tpre[S];
+  const int total = ntiles * hkv;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+    }
+    mbar_init(&sm.mma_done, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.kc_full[i], 1);
+      mbar_init(&sm.kc_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_empty[i], 4);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+
+  if (warp == 4) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&qmap);
+      prefetch_tmap(&kcmap);
+      uint32_t kc_count = 0, q_count = 0;
+      int last_par[kStages];
+      for (int i = 0; i < kStages; ++i) last_par[i] = -1;
+      for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+        mbar_expect_tx(&sm.q_full[qb], kTile);
+        tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kc_count % kStages;
+          const uint32_t ph = (kc_count / kStages) & 1;
+          if (!mbar_wait(&sm.kc_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+          mbar_expect_tx(&sm.kc_full[st], kTile);
+          tma_load_2d(sm.kc[st], &kcmap, &sm.kc_full[st], 0, ti.g * btot + ti.b0 + j * kBN);
+          last_par[st] = (int)ph;
+          ++kc_count;
+        }
+      }
+      // drain: every issued load has landed before the CTA may exit
+      for (int i = 0; i < kStages; ++i)
+        if (last_par[i] >= 0) mbar_wait(&sm.kc_full[i], (uint32_t)last_par[i]);
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kRows, kBN);
+      uint32_t kc_count = 0, q_count = 0, s_count = 0;
+      for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { record_timeout(status, &sm.abort_flag); break; }
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        bool ok = true;
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kc_count % kStages;
+          const int sb = s_count % 2;
+          if (!mbar_wait(&sm.kc_full[st], (kc_count / kStages) & 1) ||
+              !mbar_wait(&sm.s_empty[sb], ((s_count / 2) & 1) ^ 1)) {
+            record_timeout(status, &sm.abort_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(tmem + sb * kBN, sdesc_kmajor_sw128(sm.q[qb], 32 * k), sdesc_kmajor_sw128(sm.kc[st], 32 * k),
+                        idesc, k > 0);
+          mma_commit(&sm.s_full[sb]);
+          mma_commit(&sm.kc_empty[st]);
+          ++kc_count;
+          ++s_count;
+        }
+        mma_commit(&sm.q_empty[qb]);
+        if (!ok) break;
+      }
+      mma_commit(&sm.mma_done);
+      mbar_wait(&sm.mma_done, 0);
+    }
+  } else {
+    // ---------------- compute warps: thread = row
+    const int r = threadIdx.x;  // 0..127
+    uint32_t s_count = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+      const int64_t t = ti.t0 + r / G;
+      const int h = ti.g * G + r % G;
+      const bool valid = t < ti.t_end;
+      float m = -CUDART_INF_F, l = 0.f;
+      const int nbt = (ti.nb + kBN - 1) / kBN;
+      bool ok = true;
+      for (int j = 0; j < nbt; ++j) {
+        const int sb = s_count % 2;
+        if (!mbar_wait(&sm.s_full[sb], (s_count / 2) & 1)) { record_timeout(status, &sm.abort_flag); ok = false; break; }
+        tc_fence_after();
+        float sv[kBN];
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + sb * kBN;
+#pragma unroll
+        for (int c = 0; c < kBN; c += 32) tmem_ld32(taddr + c, sv + c);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+        ++s_count;
+        const int vc = min(kBN, ti.nb - j * kBN);
+        float cm = -CUDART_INF_F;
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          sv[c] = c < vc ? sv[c] * qs2 : -CUDART_INF_F;
+          cm = fmaxf(cm, sv[c]);
+        }
+        const float mn = fmaxf(m, cm);
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) acc += exp2f(sv[c] - mn);
+        l = l * exp2f(m - mn) + acc;
+        m = mn;
+      }
+      if (!ok) break;
+      if (valid) lse_out[t * hq + h] = (m + log2f(l)) * kLn2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// pass 2: output + top-k (transposed: thread = block)
+// ---------------------------------------------------------------------------
+constexpr int kTopkMax = 32;
+constexpr int kOutStages = 3;
+constexpr int kCandMax = 128;  // top-k candidates per token kept for exact ranking
+constexpr int kComputeWarps = 8;  // pass 2: two warpgroups of compute warps
+constexpr int kOutThreads = 32 * (kComputeWarps + 2);  // + TMA warp + MMA warp
+
+struct OutSmem {
+  uint8_t q[2][kTile];
+  uint8_t kc[kOutStages][kTile];
+  uint8_t vc[kOutStages][kTile];
+  uint8_t pt_hi[2 * kTile];  // P^T (bf16 high part) as the MN-major A operand: [2 row atoms][128 blocks][64 rows]
+  uint8_t pt_lo[2 * kTile];  // p - bf16(p), same layout: O += (P_hi + P_lo) Vc keeps fp32-level accuracy
+  __align__(16) float lse2[kRows];
+  float candv[kComputeWarps][kCandMax];
+  int candi[kComputeWarps][kCandMax];
+  uint64_t q_full[2], q_empty[2], mma_done, o_full, o_empty, cw;
+  uint64_t kv_full[kOutStages], kv_empty[kOutStages];
+  uint64_t s_full, s_empty, pt_full, pt_empty;
+  uint32_t tmem;
+  int abort_flag;
+};
+
+// Store rows [8c, 8c+8) of block `b` into a P^T tile (MN-major A operand,
+// 128-byte swizzle): row atom a = row / 64 holds 64 rows of one block in a
+// 128-byte line; the 16-byte chunks of line b are XOR-swizzled with b % 8.
+__device__ __forceinline__ void store_pt_chunk(uint8_t* pt, int b, int c, uint4 v) {
+  const int a = c / 8;
+  const int chunk = c % 8;
+  *reinterpret_cast<uint4*>(pt + a * kTile + b * 128 + ((chunk ^ (b & 7)) * 16)) = v;
+}
+
+// (v, id) ranks above (v2, id2): higher score, or equal score and lower id.
+__device__ __forceinline__ bool beats(float v, int id, float v2, int id2) { return v > v2 || (v == v2 && id < id2); }
+
+// Sync of the 4 compute warps through an mbarrier (bounded wait, unlike bar.sync).
+__device__ __forceinline__ bool cw_sync(uint64_t* bar, uint32_t& phase) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase & 1);
+  ++phase;
+  return ok;
+}
+
+// Top-k of imp[0..nb) (scores of the sequence's blocks for one token) by one
+// warp.  Each lane keeps a sorted list of its KL best entries in registers (one
+// coalesced pass over the scores), then k rounds of a warp-wide arg-max over the
+// list heads pick the winners.  Writes b0 + local id of the picks, ascending,
+// padded with -1, to out[0..topk).  Requires topk <= KL.
+template <int KL>
+__device__ void warp_topk(const float* __restrict__ imp, int nb, int topk, int b0, int32_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int keff = min(topk, nb);
+  float lv[KL];
+  int li[KL];
+#pragma unroll
+  for (int k = 0; k < KL; ++k) {
+    lv[k] = -CUDART_INF_F;
+    li[k] = 0x7fffffff;
+  }
+  // imp is 16-byte aligned; each lane reads 4 consecutive scores per float4, 4 float4 in flight
+  for (int base = 0; base < nb; base += 512) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i0 = base + u * 128 + lane * 4;
+      if (i0 + 3 < nb) {
+        v[u] = *reinterpret_cast<const float4*>(imp + i0);
+      } else {
+        v[u].x = i0 + 0 < nb ? imp[i0 + 0] : -CUDART_INF_F;
+        v[u].y = i0 + 1 < nb ? imp[i0 + 1] : -CUDART_INF_F;
+        v[u].z = i0 + 2 < nb ? imp[i0 + 2] : -CUDART_INF_F;
+        v[u].w = -CUDART_INF_F;
+        if (i0 + 3 < nb) v[u].w = imp[i0 + 3];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = base + u * 128 + lane * 4 + e;
+        const float x = e == 0 ? v[u].x : e == 1 ? v[u].y : e == 2 ? v[u].z : v[u].w;
+        if (i >= nb || !beats(x, i, lv[KL - 1], li[KL - 1])) continue;
+#pragma unroll
+        for (int k = KL - 1; k >= 1; --k) {
+          const bool above_prev = beats(x, i, lv[k - 1], li[k - 1]);
+          const bool above_cur = beats(x, i, lv[k], li[k]);
+          if (above_prev) {
+            lv[k] = lv[k - 1];
+            li[k] = li[k - 1];
+          } else if (above_cur) {
+            lv[k] = x;
+            li[k] = i;
+          }
+        }
+        if (beats(x, i, lv[0], li[0])) {
+          lv[0] = x;
+          li[0] = i;
+        }
+      }
+    }
+  }
+  int chosen = 0x7fffffff;  // lane r keeps the r-th pick (r < keff)
+  for (int r = 0; r < keff; ++r) {
+    float v = lv[0];
+    int id = li[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+      const int id2 = __shfl_xor_sync(0xffffffffu, id, o);
+      if (beats(v2, id2, v, id)) {
+        v = v2;
+        id = id2;
+      }
+    }
+    if (lane == r) chosen = id;
+    if (id == li[0]) {  // this lane owned the winner: pop its head
+#pragma unroll
+      for (int k = 0; k < KL - 1; ++k) {
+        lv[k] = lv[k + 1];
+        li[k] = li[k + 1];
+      }
+      lv[KL - 1] = -CUDART_INF_F;
+      li[KL - 1] = 0x7fffffff;
+    }
+  }
+  int rank = 0;  // ascending ids: rank of each pick among the picks
+  for (int r = 0; r < keff; ++r) {
+    const int other = __shfl_sync(0xffffffffu, chosen, r);
+    if (other < chosen) ++rank;
+  }
+  if (lane < keff) out[rank] = b0 + chosen;
+  for (int i = keff + lane; i < topk; i += 32) out[i] = -1;
+}
+
+// Fast exact top-k of imp[0..nb) by one warp (same result as warp_topk):
+//  1. each lane's best entry (one pass of float4 loads);
+//  2. tau = the keff-th best of the 32 lane bests -- at least keff entries rank
+//     at or above tau, so every top-keff entry does;
+//  3. entries ranking at or above tau (typically a few dozen) are collected in
+//     shared memory and ranked exactly against each other.
+// Falls back to warp_topk when more than kCandMax entries pass the threshold.
+template <int KL>
+__device__ void warp_topk_fast(const float* __restrict__ imp, int nb, int topk, int b0, int32_t* __restrict__ out,
+                               float* cv, int* ci) {
+  const int lane = threadIdx.x & 31;
+  const int keff = min(topk, nb);
+  // 1. lane best
+  float bv = -CUDART_INF_F;
+  int bi = 0x7fffffff;
+  for (int base = 0; base < nb; base += 512) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i0 = base + u * 128 + lane * 4;
+      if (i0 + 3 < nb) {
+        v[u] = *reinterpret_cast<const float4*>(imp + i0);
+      } else {
+        v[u].x = i0 + 0 < nb ? imp[i0 + 0] : -CUDART_INF_F;
+        v[u].y = i0 + 1 < nb ? imp[i0 + 1] : -CUDART_INF_F;
+        v[u].z = i0 + 2 < nb ? imp[i0 + 2] : -CUDART_INF_F;
+        v[u].w = -CUDART_INF_F;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i0 = base + u * 128 + lane * 4;
+      if (i0 < nb && beats(v[u].x, i0, bv, bi)) { bv = v[u].x; bi = i0; }
+      if (i0 + 1 < nb && beats(v[u].y, i0 + 1, bv, bi)) { bv = v[u].y; bi = i0 + 1; }
+      if (i0 + 2 < nb && beats(v[u].z, i0 + 2, bv, bi)) { bv = v[u].z; bi = i0 + 2; }
+      if (i0 + 3 < nb && beats(v[u].w, i0 + 3, bv, bi)) { bv = v[u].w; bi = i0 + 3; }
+    }
+  }
+  // 2. rank of each lane best among the 32; tau = the one of rank keff-1
+  int rank = 0;
+#pragma unroll
+  for (int o = 0; o < 32; ++o) {
+    const float v2 = __shfl_sync(0xffffffffu, bv, o);
+    const int i2 = __shfl_sync(0xffffffffu, bi, o);
+    if (beats(v2, i2, bv, bi)) ++rank;
+  }
+  const unsigned own = __ballot_sync(0xffffffffu, rank == keff - 1);
+  if (keff > 32 || own == 0u) {  // fewer than keff lanes hold entries: exact path
+    warp_topk<KL>(imp, nb, topk, b0, out);
+    return;
+  }
+  const int src = __ffs(own) - 1;
+  const float tv = __shfl_sync(0xffffffffu, bv, src);
+  const int ti = __shfl_sync(0xffffffffu, bi, src);
+  // 3. collect entries at or above (tv, ti)
+  int n = 0;
+  bool overflow = false;
+  for (int base = 0; base < nb && !overflow; base += 32) {
+    const int i = base + lane;
+    const float x = i < nb ? imp[i] : -CUDART_INF_F;
+    const bool take = i < nb && (x == tv ? i <= ti : x > tv);
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    const int slot = n + __popc(m & ((1u << lane) - 1u));
+    if (take && slot < kCandMax) {
+      cv[slot] = x;
+      ci[slot] = i;
+    }
+    n += __popc(m);
+    overflow = n > kCandMax;
+  }
+  if (overflow) {
+    __syncwarp();
+    warp_topk<KL>(imp, nb, topk, b0, out);
+    return;
+  }
+  __syncwarp();
+  // exact ranks among the candidates; picks are those with rank < keff
+  int picked_id[kCandMax / 32];
+  bool picked[kCandMax / 32];
+#pragma unroll
+  for (int u = 0; u < kCandMax / 32; ++u) {
+    const int c = u * 32 + lane;
+    picked[u] = false;
+    picked_id[u] = 0x7fffffff;
+    if (c < n) {
+      const float x = cv[c];
+      const int id = ci[c];
+      int r = 0;
+      for (int j = 0; j < n; ++j) r += beats(cv[j], ci[j], x, id) ? 1 : 0;
+      picked[u] = r < keff;
+      picked_id[u] = id;
+    }
+  }
+  __syncwarp();
+  // write picks in ascending id order: position = number of picks with a lower id
+#pragma unroll
+  for (int u = 0; u < kCandMax / 32; ++u) {
+    const int c = u * 32 + lane;
+    if (c < n) ci[c] = picked[u] ? picked_id[u] : 0x7fffffff;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < kCandMax / 32; ++u) {
+    if (picked[u]) {
+      int pos = 0;
+      for (int j = 0; j < n; ++j) pos += ci[j] < picked_id[u] ? 1 : 0;
+      out[pos] = b0 + picked_id[u];
+    }
+  }
+  for (int i = keff + lane; i < topk; i += 32) out[i] = -1;
+  __syncwarp();
+}
+
+template <int G>
+__global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap,
+    const __grid_constant__ CUtensorMap vcmap, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
+    const int32_t* __restrict__ tpre, int S, int hq, int hkv, int btot, float qs2, const float* __restrict__ lse_in,
+    float* __restrict__ o_out, int topk, int32_t* __restrict__ sel, float* __restrict__ imp_scratch,
+    int64_t imp_stride, int* status) {
+  constexpr int TPT = kRows / G;  // tokens per tile
+  extern __shared__ uint8_t smem_raw[];
+  OutSmem& sm = *reinterpret_cast<OutSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int ntiles = tpre[S];
+  const int total = ntiles * hkv;
+  // this CTA's scores: [TPT tokens][imp_stride blocks]
+  float* imp_base = imp_scratch + (int64_t)blockIdx.x * TPT * imp_stride;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+    }
+    mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.o_empty, kComputeWarps);
+    mbar_init(&sm.cw, kComputeWarps);
+    for (int i = 0; i < kOutStages; ++i) {
+      mbar_init(&sm.kv_full[i], 1);
+      mbar_init(&sm.kv_empty[i], 1);
+    }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_empty, kComputeWarps);
+    mbar_init(&sm.pt_full, kComputeWarps);
+    mbar_init(&sm.pt_empty, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  const uint32_t tm_s = tmem, tm_o = tmem + 128;  // S^T: columns [0,128); O: [128,192)
+
+  if (warp == kComputeWarps) {
+    // ---------------- TMA producer: Q per tile; (Kc, Vc) per key tile
+    if (lane == 0) {
+      prefetch_tmap(&qmap);
+      prefetch_tmap(&kcmap);
+      prefetch_tmap(&vcmap);
+      uint32_t kv_count = 0, q_count = 0;
+      int last_par[kOutStages];
+      for (int i = 0; i < kOutStages; ++i) last_par[i] = -1;
+      for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+        mbar_expect_tx(&sm.q_full[qb], kTile);
+        tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kv_count % kOutStages;
+          const uint32_t ph = (kv_count / kOutStages) & 1;
+          if (!mbar_wait(&sm.kv_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+          mbar_expect_tx(&sm.kv_full[st], 2 * kTile);
+          const int row = ti.g * btot + ti.b0 + j * kBN;
+          tma_load_2d(sm.kc[st], &kcmap, &sm.kv_full[st], 0, row);
+          tma_load_2d(sm.vc[st], &vcmap, &sm.kv_full[st], 0, row);
+          last_par[st] = (int)ph;
+          ++kv_count;
+        }
+      }
+      for (int i = 0; i < kOutStages; ++i)
+        if (last_par[i] >= 0) mbar_wait(&sm.kv_full[i], (uint32_t)last_par[i]);
+    }
+  } else if (warp == kComputeWarps + 1) {
+    // ---------------- MMA issuer: S^T(j+1) is issued as soon as S^T(j) has been read,
+    // so it overlaps with the exps of tile j; O += P(j) Vc(j) follows when P^T(j) is ready.
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(kBN, kRows);            // S^T[blocks, rows] = Kc Q^T
+      const uint32_t id_o = idesc_bf16(kRows, 64, true, true);  // O[rows, 64] += P[rows, blocks] Vc
+      uint32_t kv_count = 0, q_count = 0, s_count = 0, pt_count = 0, o_count = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        auto issue_s = [&](uint32_t kv_idx) -> bool {
+          const int st = kv_idx % kOutStages;
+          if (!mbar_wait(&sm.kv_full[st], (kv_idx / kOutStages) & 1) || !mbar_wait(&sm.s_empty, (s_count & 1) ^ 1))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(tm_s, sdesc_kmajor_sw128(sm.kc[st], 32 * k), sdesc_kmajor_sw128(sm.q[qb], 32 * k), id_s,
+                        k > 0);
+          mma_commit(&sm.s_full);
+          ++s_count;
+          return true;
+        };
+        if (nbt > 0 && !issue_s(kv_count)) { ok = false; break; }
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kv_count % kOutStages;
+          if (j + 1 < nbt && !issue_s(kv_count + 1)) { ok = false; break; }
+          // O is overwritten by the first P Vc of a tile: the previous tile's O must have been read
+          if ((j == 0 && !mbar_wait(&sm.o_empty, (o_count & 1) ^ 1)) || !mbar_wait(&sm.pt_full, pt_count & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            const uint64_t bdesc = sdesc_mnmajor_sw128(sm.vc[st], 2048 * k, kTile);
+            mma_bf16_ss(tm_o, sdesc_mnmajor_sw128(sm.pt_hi, 2048 * k, kTile), bdesc, id_o, j > 0 || k > 0);
+            mma_bf16_ss(tm_o, sdesc_mnmajor_sw128(sm.pt_lo, 2048 * k, kTile), bdesc, id_o, true);
+          }
+          mma_commit(&sm.pt_empty);
+          mma_commit(&sm.kv_empty[st]);
+          ++pt_count;
+          ++kv_count;
+        }
+        if (!ok) break;
+        mma_commit(&sm.q_empty[qb]);
+        mma_commit(&sm.o_full);
+        ++o_count;
+      }
+      if (!ok) record_timeout(status, &sm.abort_flag);
+      mma_commit(&sm.mma_done);
+      mbar_wait(&sm.mma_done, 0);
+    }
+  } else {
+    // ---------------- compute warps (two warpgroups): thread = block of the key tile;
+    // warpgroup wg handles query rows [64 wg, 64 wg + 64) of the tile.
+    const int b = threadIdx.x % 128;
+    const int wg = warp / 4;
+    const int r0 = 64 * wg;
+    uint32_t s_count = 0, pt_count = 0, o_count = 0, cw_phase = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+      if (wg == 0) {
+        const int r = threadIdx.x;
+        const int64_t t = min((int64_t)ti.t0 + r / G, (int64_t)ti.t_end - 1);
+        sm.lse2[r] = lse_in[t * hq + ti.g * G + r % G] * kLog2e;
+      }
+      if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
+      const int nbt = (ti.nb + kBN - 1) / kBN;
+      bool ok = true;
+      for (int j = 0; j < nbt; ++j) {
+        if (!mbar_wait(&sm.s_full, s_count & 1)) { ok = false; break; }
+        tc_fence_after();
+        float p[64];
+        const uint32_t taddr = tm_s + ((uint32_t)((warp % 4) * 32) << 16) + r0;
+        tmem_ld32(taddr, p);
+        tmem_ld32(taddr + 32, p + 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_empty);
+        ++s_count;
+        const int bidx = j * kBN + b;  // block index inside the sequence
+        const bool bvalid = bidx < ti.nb;
+#pragma unroll
+        for (int r = 0; r < 64; r += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[r0 + r]);
+          p[r + 0] = bvalid ? exp2f(p[r + 0] * qs2 - l4.x) : 0.f;
+          p[r + 1] = bvalid ? exp2f(p[r + 1] * qs2 - l4.y) : 0.f;
+          p[r + 2] = bvalid ? exp2f(p[r + 2] * qs2 - l4.z) : 0.f;
+          p[r + 3] = bvalid ? exp2f(p[r + 3] * qs2 - l4.w) : 0.f;
+        }
+        if (!mbar_wait(&sm.pt_empty, (pt_count & 1) ^ 1)) { ok = false; break; }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = p[8 * c + 2 * e], x1 = p[8 * c + 2 * e + 1];
+            const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+            const float2 hf = __bfloat1622float2(h);
+            hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+            lo[e] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+          }
+          store_pt_chunk(sm.pt_hi, b, 8 * wg + c, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+          store_pt_chunk(sm.pt_lo, b, 8 * wg + c, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.pt_full);
+        ++pt_count;
+        // selection score of this block for each of the warpgroup's tokens:
+        // probability summed over the group's heads
+        if (bvalid) {
+#pragma unroll
+          for (int tl = 0; tl < 64 / G; ++tl) {
+            float imp = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) imp += p[tl * G + hh];
+            imp_base[(int64_t)(wg * (64 / G) + tl) * imp_stride + bidx] = imp;
+          }
+        }
+      }
+      if (!ok) {
+        record_timeout(status, &sm.abort_flag);
+        break;
+      }
+      // O of this tile: wait for the last P Vc; warpgroup wg writes columns [32 wg, 32 wg + 32)
+      if (!mbar_wait(&sm.o_full, o_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      ++o_count;
+      tc_fence_after();
+      {
+        const int r = b;  // TMEM lane = query row
+        const int64_t t = ti.t0 + r / G;
+        const int h = ti.g * G + r % G;
+        float o[32];
+        tmem_ld32(tm_o + ((uint32_t)((warp % 4) * 32) << 16) + 32 * wg, o);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.o_empty);
+        if (t < ti.t_end) {
+          float4* dst = reinterpret_cast<float4*>(o_out + (t * hq + h) * 64 + 32 * wg);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
+      }
+      // top-k per token from the scores of all blocks (one warp per token)
+      __threadfence_block();
+      if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
+      for (int tk = warp; tk < TPT; tk += kComputeWarps) {
+        const int64_t t = ti.t0 + tk;
+        if (t < ti.t_end) {
+          if (topk <= 16)
+            warp_topk_fast<16>(imp_base + (int64_t)tk * imp_stride, ti.nb, topk, ti.b0,
+                               sel + (t * hkv + ti.g) * topk, sm.candv[warp], sm.candi[warp]);
+          else
+            warp_topk_fast<kTopkMax>(imp_base + (int64_t)tk * imp_stride, ti.nb, topk, ti.b0,
+                                     sel + (t * hkv + ti.g) * topk, sm.candv[warp], sm.candi[warp]);
+        }
+      }
+      __threadfence_block();
+      if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D map over [rows, 64] bf16 with a box of 128 rows, 128-byte swizzle.
+bool map_rows64(CUtensorMap* m, const void* base, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {64, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D map over Q [N, Hq, 64] bf16 with a box of (64, G heads, 128/G tokens).
+bool map_q(CUtensorMap* m, const void* base, int64_t n, int hq, int G) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)hq, (cuuint64_t)n};
+  cuuint64_t strides[2] = {128, (cuuint64_t)hq * 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(kRows / G)};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t smem_bytes_lse() { return sizeof(LseSmem) + 1024; }
+size_t smem_bytes_out() { return sizeof(OutSmem) + 1024; }
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int G>
+cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st) {
+  CUtensorMap qm, km, vm;
+  if (!map_q(&qm, a.q, a.N, a.hq, G) || !map_rows64(&km, a.kc, (int64_t)a.hkv * a.blk->count) ||
+      !map_rows64(&vm, a.vc, (int64_t)a.hkv * a.blk->count))
+    return cudaErrorInvalidValue;
+  const float qs2 = a.scale * kLog2e;
+  const int btot = (int)a.blk->count;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(cmp_lse_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_lse());
+    cudaFuncSetAttribute(cmp_out_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_out());
+    cudaFuncSetAttribute(cmp_out_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_out());
+    attr_done = true;
+  }
+  const int sms = num_sms() < kCmpOutCtas ? num_sms() : kCmpOutCtas;
+  const int64_t tiles = total_tiles_bound * a.hkv;
+  const int g1 = (int)(tiles < 2 * sms ? (tiles > 0 ? tiles : 1) : 2 * sms);
+  const int g2 = (int)(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);  // at most kCmpOutCtas (scratch size)
+  SSA_LAUNCH("cmp_lse_tc_kernel", cmp_lse_tc_kernel, g1, kThreads, smem_bytes_lse(), st, qm, km, a.cu_seqlens,
+             a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.status);
+  SSA_LAUNCH("cmp_out_tc_kernel", cmp_out_tc_kernel<G>, g2, kOutThreads, smem_bytes_out(), st, qm, km, vm,
+             a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.o_branch, a.topk, a.sel,
+             a.imp_scratch, (int64_t)((btot + 3) & ~3), a.status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t cmp_tc_scratch_floats(int hq, int hkv, int64_t btot) {
+  const int G = hkv > 0 ? hq / hkv : 1;
+  return (size_t)kCmpOutCtas * (kRows / (G > 0 ? G : 1)) * (size_t)((btot + 3) & ~int64_t(3)) + 4;
+}
+
+bool cmp_tc_supported(int dtype, int d, int hq, int hkv, int topk) {
+  const int G = hkv > 0 ? hq / hkv : 0;
+  return dtype == SSA_DTYPE_BF16 && d == 64 && (G == 8 || G == 16) && topk <= kTopkMax && encode_fn() != nullptr;
+}
+
+// Compressed branch forward (lse, o_cmp, sel) on the tensor cores; `tpre` is the
+// per-sequence prefix of 128-row tiles (per group).
+cudaError_t cmp_fwd_tc(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st) {
+  const int G = a.hq / a.hkv;
+  if (G == 16) return cmp_fwd_tc_g<16>(a, tpre, total_tiles_bound, st);
+  if (G == 8) return cmp_fwd_tc_g<8>(a, tpre, total_tiles_bound, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ssa

@@ -10,9 +10,13 @@ namespace ssa {
 
 // Query rows per work item of the compressed-branch dKc/dVc kernel.
 constexpr int kCmpRowChunk = 2048;
+// Upper bound on the CTAs of the tensor-core compressed-output kernel (sizes its score scratch).
+constexpr int kCmpOutCtas = 160;
 
 struct FwdArgs {
   int dtype, d, hq, hkv, topk, gate_mode;
+  int use_tc;   // run the tensor-core kernels where they cover the shape
+  int* status;  // device check word
   float scale;
   int32_t S;
   int64_t N;
@@ -29,10 +33,13 @@ struct FwdArgs {
   int32_t* sel;
   // workspace
   int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
+  float* imp_scratch;  // [kCmpOutCtas, 128/G, B] selection scores (tensor-core path)
 };
 
 struct BwdArgs {
   int dtype, d, hq, hkv, topk, gate_mode;
+  int use_tc;
+  int* status;
   float scale;
   int32_t S;
   int64_t N;
@@ -61,6 +68,11 @@ struct BwdArgs {
 cudaError_t launch_pool(int dtype, const void* k, const void* v, const ssa_partition* blk, int64_t N, int hkv,
                         int d, void* ks, void* vs, void* kc, void* vc, cudaStream_t st);
 cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st);
+
+// Tensor-core (tcgen05) kernels of the compressed branch, bf16, head dim 64.
+bool cmp_tc_supported(int dtype, int d, int hq, int hkv, int topk);
+size_t cmp_tc_scratch_floats(int hq, int hkv, int64_t btot);
+cudaError_t cmp_fwd_tc(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st);
 cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st);
 
 }  // namespace ssa
