@@ -387,10 +387,16 @@ def _sample_tokens(w, n):
 def cpu_baseline(w, t, seconds: float) -> dict:
     """The oracle as it stands, on a bounded sample: binning + pooling of all
     tokens, then every forward branch and the dQ rows for T sampled query tokens."""
+    # two calibration points separate the fixed cost (binning, pooling) from the per-token cost
     t0 = time.perf_counter()
     _oracle_sample(w, t, _sample_tokens(w, 16))
-    t1 = time.perf_counter() - t0
-    T = int(max(16, min(w.n, 16 * seconds / max(t1, 1e-3))))
+    ta = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    _oracle_sample(w, t, _sample_tokens(w, 80))
+    tb = time.perf_counter() - t0
+    per_tok = max((tb - ta) / 64.0, 1e-4)
+    fixed = max(ta - 16 * per_tok, 0.0)
+    T = int(max(16, min(w.n, (seconds - fixed) / per_tok)))
     t0 = time.perf_counter()
     _oracle_sample(w, t, _sample_tokens(w, T))
     el = time.perf_counter() - t0

@@ -1071,14 +1071,24 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
 
   SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout, a.gates, rows, a.gate_mode,
                                                                              a.Dc, a.dgates);
-  const dim3 g2(grid_1d(rows, C::ROWS, 148 * 8), a.hkv);
-  SSA_LAUNCH("cmp_bwd_dq_kernel", (cmp_bwd_dq_kernel<T, D>), g2, 128, 0, st, q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu,
-                                              a.tiles_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.dq);
-  cudaMemsetAsync(a.dkc, 0, sizeof(float) * a.hkv * btot * D, st);
-  cudaMemsetAsync(a.dvc, 0, sizeof(float) * a.hkv * btot * D, st);
-  SSA_LAUNCH("cmp_bwd_dkv_kernel", (cmp_bwd_dkv_kernel<T, D>), dim3(148 * 8, a.hkv), 128, 0, st, 
-      q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu, a.items_pre, a.S, a.hq, a.hkv, btot, qs2,
-      a.scale, kCmpRowChunk, a.lse, a.Dc, a.dkc, a.dvc);
+  if (a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
+    // 128-row tiles for the tensor-core kernels (tiles_cnt / tiles_pre are free again here)
+    SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu,
+               a.S, G, 128, 128, kCmpRowChunk, a.tiles_cnt, a.items_cnt);
+    e = exclusive_scan(a.tiles_cnt, a.tiles_pre, a.S + 1, a.scan_tmp, st);
+    if (e != cudaSuccess) return e;
+    e = cmp_bwd_tc(a, a.tiles_pre, a.items_cnt, a.items_pre, a.scan_tmp, (a.N * G + 127) / 128 + a.S, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    const dim3 g2(grid_1d(rows, C::ROWS, 148 * 8), a.hkv);
+    SSA_LAUNCH("cmp_bwd_dq_kernel", (cmp_bwd_dq_kernel<T, D>), g2, 128, 0, st, q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu,
+                                                a.tiles_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.dq);
+    cudaMemsetAsync(a.dkc, 0, sizeof(float) * a.hkv * btot * D, st);
+    cudaMemsetAsync(a.dvc, 0, sizeof(float) * a.hkv * btot * D, st);
+    SSA_LAUNCH("cmp_bwd_dkv_kernel", (cmp_bwd_dkv_kernel<T, D>), dim3(148 * 8, a.hkv), 128, 0, st, 
+        q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu, a.items_pre, a.S, a.hq, a.hkv, btot, qs2,
+        a.scale, kCmpRowChunk, a.lse, a.Dc, a.dkc, a.dvc);
+  }
   const int pairs_per_cta = 128 / (G * C::NT);
   SSA_LAUNCH("slc_bwd_dq_kernel", (slc_bwd_dq_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
       q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,

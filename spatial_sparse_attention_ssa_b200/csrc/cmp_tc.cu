@@ -735,6 +735,508 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// backward, dQ (thread = row): S = Q Kc^T, dP = dO Vc^T in TMEM; dS = P (w dP - D)
+// in registers; dQ += dS Kc with dS (bf16 hi + lo) as the TMEM A operand.
+// ---------------------------------------------------------------------------
+constexpr int kBwdStages = 3;
+
+struct DqSmem {
+  uint8_t q[2][kTile];
+  uint8_t dout[2][kTile];
+  uint8_t kc[kBwdStages][kTile];
+  uint8_t vc[kBwdStages][kTile];
+  uint64_t q_full[2], q_empty[2], kv_full[kBwdStages], kv_empty[kBwdStages];
+  uint64_t sdp_full, sdp_empty, ds_full, ds_empty, dq_full, dq_empty, mma_done;
+  uint32_t tmem;
+  int abort_flag;
+};
+
+template <int G>
+__global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
+    const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
+    const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S, int hq,
+    int hkv, int btot, float qs2, float scale, const float* __restrict__ lse_in, const float* __restrict__ Dc,
+    const float* __restrict__ gates, int gate_mode, float* __restrict__ dq_out, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  DqSmem& sm = *reinterpret_cast<DqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int ntiles = tpre[S];
+  const int total = ntiles * hkv;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+    }
+    for (int i = 0; i < kBwdStages; ++i) {
+      mbar_init(&sm.kv_full[i], 1);
+      mbar_init(&sm.kv_empty[i], 1);
+    }
+    mbar_init(&sm.sdp_full, 1);
+    mbar_init(&sm.sdp_empty, kComputeWarps);
+    mbar_init(&sm.ds_full, kComputeWarps);
+    mbar_init(&sm.ds_empty, 1);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.dq_empty, kComputeWarps);
+    mbar_init(&sm.mma_done, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  // TMEM columns: S [0,128), dP [128,256), dS hi [256,320), dS lo [320,384), dQ [384,448)
+  const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dsh = tmem + 256, tm_dsl = tmem + 320, tm_dq = tmem + 384;
+
+  if (warp == kComputeWarps) {
+    // ---------------- TMA producer: (Q, dO) per row tile; (Kc, Vc) per key tile
+    if (lane == 0) {
+      uint32_t kv_count = 0, q_count = 0;
+      int last_par[kBwdStages];
+      for (int i = 0; i < kBwdStages; ++i) last_par[i] = -1;
+      for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+        mbar_expect_tx(&sm.q_full[qb], 2 * kTile);
+        tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
+        tma_load_3d(sm.dout[qb], &dmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kv_count % kBwdStages;
+          const uint32_t ph = (kv_count / kBwdStages) & 1;
+          if (!mbar_wait(&sm.kv_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+          mbar_expect_tx(&sm.kv_full[st], 2 * kTile);
+          const int row = ti.g * btot + ti.b0 + j * kBN;
+          tma_load_2d(sm.kc[st], &kcmap, &sm.kv_full[st], 0, row);
+          tma_load_2d(sm.vc[st], &vcmap, &sm.kv_full[st], 0, row);
+          last_par[st] = (int)ph;
+          ++kv_count;
+        }
+      }
+      for (int i = 0; i < kBwdStages; ++i)
+        if (last_par[i] >= 0) mbar_wait(&sm.kv_full[i], (uint32_t)last_par[i]);
+    }
+  } else if (warp == kComputeWarps + 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(kRows, kBN);              // S, dP [rows, blocks]
+      const uint32_t id_q = idesc_bf16(kRows, 64, false, true);   // dQ[rows, 64] += dS[rows, blocks] Kc
+      uint32_t kv_count = 0, q_count = 0, sdp_count = 0, ds_count = 0, dq_count = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        auto issue_sdp = [&](uint32_t kv_idx) -> bool {
+          const int st = kv_idx % kBwdStages;
+          if (!mbar_wait(&sm.kv_full[st], (kv_idx / kBwdStages) & 1) ||
+              !mbar_wait(&sm.sdp_empty, (sdp_count & 1) ^ 1))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            mma_bf16_ss(tm_s, sdesc_kmajor_sw128(sm.q[qb], 32 * k), sdesc_kmajor_sw128(sm.kc[st], 32 * k), id_s, k > 0);
+            mma_bf16_ss(tm_dp, sdesc_kmajor_sw128(sm.dout[qb], 32 * k), sdesc_kmajor_sw128(sm.vc[st], 32 * k), id_s,
+                        k > 0);
+          }
+          mma_commit(&sm.sdp_full);
+          ++sdp_count;
+          return true;
+        };
+        if (nbt > 0 && !issue_sdp(kv_count)) { ok = false; break; }
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kv_count % kBwdStages;
+          if (j + 1 < nbt && !issue_sdp(kv_count + 1)) { ok = false; break; }
+          if ((j == 0 && !mbar_wait(&sm.dq_empty, (dq_count & 1) ^ 1)) || !mbar_wait(&sm.ds_full, ds_count & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            const uint64_t bdesc = sdesc_mnmajor_sw128(sm.kc[st], 2048 * k, kTile);
+            mma_bf16_ts(tm_dq, tm_dsh + 8 * k, bdesc, id_q, j > 0 || k > 0);
+            mma_bf16_ts(tm_dq, tm_dsl + 8 * k, bdesc, id_q, true);
+          }
+          mma_commit(&sm.ds_empty);
+          mma_commit(&sm.kv_empty[st]);
+          ++ds_count;
+          ++kv_count;
+        }
+        if (!ok) break;
+        mma_commit(&sm.q_empty[qb]);
+        mma_commit(&sm.dq_full);
+        ++dq_count;
+      }
+      if (!ok) record_timeout(status, &sm.abort_flag);
+      mma_commit(&sm.mma_done);
+      mbar_wait(&sm.mma_done, 0);
+    }
+  } else {
+    // ---------------- compute warps: thread = row; warpgroup wg owns blocks [64 wg, 64 wg + 64) of a key tile
+    const int r = threadIdx.x % 128;
+    const int wg = warp / 4;
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    uint32_t sdp_count = 0, ds_count = 0, dq_count = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+      const int64_t t = ti.t0 + r / G;
+      const bool valid = t < ti.t_end;
+      const int64_t row = min(t, (int64_t)ti.t_end - 1) * hq + ti.g * G + r % G;
+      const float lse2 = lse_in[row] * kLog2e;
+      const float Dr = Dc[row];
+      const float gx = gates[row * 3 + 0];
+      const float wr = gate_mode == SSA_GATE_LOGITS ? 1.f / (1.f + expf(-gx)) : gx;
+      const int nbt = (ti.nb + kBN - 1) / kBN;
+      bool ok = true;
+      for (int j = 0; j < nbt; ++j) {
+        if (!mbar_wait(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
+        tc_fence_after();
+        float sv[64], dp[64];
+        tmem_ld32(tm_s + lane_off + 64 * wg, sv);
+        tmem_ld32(tm_s + lane_off + 64 * wg + 32, sv + 32);
+        tmem_ld32(tm_dp + lane_off + 64 * wg, dp);
+        tmem_ld32(tm_dp + lane_off + 64 * wg + 32, dp + 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sdp_empty);
+        ++sdp_count;
+        const int nvalid = ti.nb - (j * kBN + 64 * wg);  // valid blocks of this warpgroup's half
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float d0 = 0.f, d1 = 0.f;
+          if (c < nvalid) d0 = exp2f(sv[c] * qs2 - lse2) * (wr * dp[c] - Dr);
+          if (c + 1 < nvalid) d1 = exp2f(sv[c + 1] * qs2 - lse2) * (wr * dp[c + 1] - Dr);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
+          const float2 hf = __bfloat1622float2(h);
+          hi[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[c / 2] = pack_bf16x2(d0 - hf.x, d1 - hf.y);
+        }
+        if (!mbar_wait(&sm.ds_empty, (ds_count & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st16(tm_dsh + lane_off + 32 * wg, hi);
+        tmem_st16(tm_dsh + lane_off + 32 * wg + 16, hi + 16);
+        tmem_st16(tm_dsl + lane_off + 32 * wg, lo);
+        tmem_st16(tm_dsl + lane_off + 32 * wg + 16, lo + 16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.ds_full);
+        ++ds_count;
+      }
+      if (!ok) {
+        record_timeout(status, &sm.abort_flag);
+        break;
+      }
+      if (!mbar_wait(&sm.dq_full, dq_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      ++dq_count;
+      tc_fence_after();
+      float g32[32];
+      tmem_ld32(tm_dq + lane_off + 32 * wg, g32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.dq_empty);
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(dq_out + row * 64 + 32 * wg);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(g32[4 * i] * scale, g32[4 * i + 1] * scale, g32[4 * i + 2] * scale,
+                               g32[4 * i + 3] * scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// backward, dKc / dVc (thread = block): S^T = Kc Q^T, dP^T = Vc dO^T in TMEM;
+// P^T w and dS^T (bf16) as TMEM A operands of dVc += (P^T w) dO and
+// dKc += dS^T Q.  A work item is (group, key tile, chunk of row tiles); its
+// partial dKc / dVc are added to the fp32 workspace with vector atomics.
+// ---------------------------------------------------------------------------
+constexpr int kDkvRowTilesPerItem = 128;
+
+struct DkvSmem {
+  uint8_t kc[kTile];
+  uint8_t vc[kTile];
+  uint8_t q[2][kTile];
+  uint8_t dout[2][kTile];
+  __align__(16) float lse2[2][kRows];
+  __align__(16) float Dr[2][kRows];
+  __align__(16) float wr[2][kRows];
+  uint64_t kv_full, kv_empty, q_full[2], q_empty[2];
+  uint64_t sdp_full, sdp_empty, pds_full, pds_empty, acc_full, acc_empty, mma_done;
+  uint32_t tmem;
+  int abort_flag;
+};
+
+template <int G>
+__global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
+    const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
+    const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ ipre, int S, int hq,
+    int hkv, int btot, float qs2, float scale, const float* __restrict__ lse_in, const float* __restrict__ Dc,
+    const float* __restrict__ gates, int gate_mode, float* __restrict__ dkc, float* __restrict__ dvc, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  DkvSmem& sm = *reinterpret_cast<DkvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  constexpr int TPT = kRows / G;
+  const int nitems_g = ipre[S];
+  const int total = nitems_g * hkv;
+  // item -> (g, s, key tile, row-tile range); items of a sequence: nkt x nchunks, key tile fastest
+  auto item_of = [&](int it, int& g, int& s, int& kt, int& rt0, int& rt1, int& t_beg, int& t_end, int& b0, int& nb) {
+    g = it / nitems_g;
+    const int local = it % nitems_g;
+    s = find_segment(ipre, S, local);
+    const int k = local - ipre[s];
+    b0 = bcu[s];
+    nb = bcu[s + 1] - b0;
+    const int nkt = (nb + kBN - 1) / kBN;
+    kt = k % nkt;
+    const int chunk = k / nkt;
+    t_beg = cu[s];
+    t_end = cu[s + 1];
+    const int nrt = (t_end - t_beg + TPT - 1) / TPT;
+    rt0 = chunk * kDkvRowTilesPerItem;
+    rt1 = min(nrt, rt0 + kDkvRowTilesPerItem);
+  };
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.kv_full, 1);
+    mbar_init(&sm.kv_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+    }
+    mbar_init(&sm.sdp_full, 1);
+    mbar_init(&sm.sdp_empty, kComputeWarps);
+    mbar_init(&sm.pds_full, kComputeWarps);
+    mbar_init(&sm.pds_empty, 1);
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.acc_empty, kComputeWarps);
+    mbar_init(&sm.mma_done, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  // TMEM columns: S^T [0,128), dP^T [128,256), P^T w [256,320), dS^T [320,384), dKc [384,448), dVc [448,512)
+  const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_p = tmem + 256, tm_ds = tmem + 320, tm_dk = tmem + 384,
+                 tm_dv = tmem + 448;
+
+  if (warp == kComputeWarps) {
+    // ---------------- producer warp: (Kc, Vc) per item; (Q, dO) + row scalars per row tile
+    uint32_t kv_count = 0, q_count = 0;
+    bool kv_issued = false;
+    uint32_t kv_last_par = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+      int g, s, kt, rt0, rt1, t_beg, t_end, b0, nb;
+      item_of(it, g, s, kt, rt0, rt1, t_beg, t_end, b0, nb);
+      bool okk = true;
+      if (lane == 0) {
+        okk = mbar_wait(&sm.kv_empty, (kv_count & 1) ^ 1);
+        if (okk) {
+          mbar_expect_tx(&sm.kv_full, 2 * kTile);
+          const int row = g * btot + b0 + kt * kBN;
+          tma_load_2d(sm.kc, &kcmap, &sm.kv_full, 0, row);
+          tma_load_2d(sm.vc, &vcmap, &sm.kv_full, 0, row);
+          kv_last_par = kv_count & 1;
+          kv_issued = true;
+        }
+      }
+      okk = __shfl_sync(0xffffffffu, okk ? 1 : 0, 0) != 0;
+      if (!okk) { record_timeout(status, &sm.abort_flag); break; }
+      ++kv_count;
+      for (int rt = rt0; rt < rt1; ++rt) {
+        const int qb = q_count % 2;
+        bool okw = true;
+        if (lane == 0) okw = mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1);
+        okw = __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
+        if (!okw) { record_timeout(status, &sm.abort_flag); break; }
+        const int t0 = t_beg + rt * TPT;
+        // row scalars of this row tile (lse in the log2 domain, D, gate weight)
+        for (int rr = lane; rr < kRows; rr += 32) {
+          const int64_t t = t0 + rr / G;
+          const bool v = t < t_end;
+          const int64_t row = (v ? t : t_end - 1) * hq + g * G + rr % G;
+          const float gx = gates[row * 3 + 0];
+          sm.lse2[qb][rr] = v ? lse_in[row] * kLog2e : CUDART_INF_F;
+          sm.Dr[qb][rr] = v ? Dc[row] : 0.f;
+          sm.wr[qb][rr] = v ? (gate_mode == SSA_GATE_LOGITS ? 1.f / (1.f + expf(-gx)) : gx) : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(&sm.q_full[qb], 2 * kTile);
+          tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, g * G, t0);
+          tma_load_3d(sm.dout[qb], &dmap, &sm.q_full[qb], 0, g * G, t0);
+        }
+        ++q_count;
+      }
+    }
+    if (lane == 0 && kv_issued) mbar_wait(&sm.kv_full, kv_last_par);
+    (void)kv_last_par;
+  } else if (warp == kComputeWarps + 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(kBN, kRows);              // S^T, dP^T [blocks, rows]
+      const uint32_t id_a = idesc_bf16(kBN, 64, false, true);     // dKc / dVc [blocks, 64] += X^T[blocks, rows] Y
+      uint32_t kv_count = 0, q_count = 0, sdp_count = 0, pds_count = 0, acc_count = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
+        int g, s, kt, rt0, rt1, t_beg, t_end, b0, nb;
+        item_of(it, g, s, kt, rt0, rt1, t_beg, t_end, b0, nb);
+        if (!mbar_wait(&sm.kv_full, kv_count & 1)) { ok = false; break; }
+        ++kv_count;
+        const int nrt = rt1 - rt0;
+        auto issue_sdp = [&](uint32_t qi) -> bool {
+          const int qb = qi % 2;
+          if (!mbar_wait(&sm.q_full[qb], (qi / 2) & 1) || !mbar_wait(&sm.sdp_empty, (sdp_count & 1) ^ 1))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            mma_bf16_ss(tm_s, sdesc_kmajor_sw128(sm.kc, 32 * k), sdesc_kmajor_sw128(sm.q[qb], 32 * k), id_s, k > 0);
+            mma_bf16_ss(tm_dp, sdesc_kmajor_sw128(sm.vc, 32 * k), sdesc_kmajor_sw128(sm.dout[qb], 32 * k), id_s,
+                        k > 0);
+          }
+          mma_commit(&sm.sdp_full);
+          ++sdp_count;
+          return true;
+        };
+        if (nrt > 0 && !issue_sdp(q_count)) { ok = false; break; }
+        for (int i = 0; i < nrt; ++i) {
+          const int qb = q_count % 2;
+          if (i + 1 < nrt && !issue_sdp(q_count + 1)) { ok = false; break; }
+          if ((i == 0 && !mbar_wait(&sm.acc_empty, (acc_count & 1) ^ 1)) || !mbar_wait(&sm.pds_full, pds_count & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kRows / 16; ++k) {
+            mma_bf16_ts(tm_dv, tm_p + 8 * k, sdesc_mnmajor_sw128(sm.dout[qb], 2048 * k, kTile), id_a, i > 0 || k > 0);
+            mma_bf16_ts(tm_dk, tm_ds + 8 * k, sdesc_mnmajor_sw128(sm.q[qb], 2048 * k, kTile), id_a, i > 0 || k > 0);
+          }
+          mma_commit(&sm.pds_empty);
+          mma_commit(&sm.q_empty[qb]);
+          ++pds_count;
+          ++q_count;
+        }
+        if (!ok) break;
+        mma_commit(&sm.kv_empty);
+        mma_commit(&sm.acc_full);
+        ++acc_count;
+      }
+      if (!ok) record_timeout(status, &sm.abort_flag);
+      mma_commit(&sm.mma_done);
+      mbar_wait(&sm.mma_done, 0);
+    }
+  } else {
+    // ---------------- compute warps: thread = block; warpgroup wg owns rows [64 wg, 64 wg + 64)
+    const int b = threadIdx.x % 128;
+    const int wg = warp / 4;
+    const int r0 = 64 * wg;
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    uint32_t sdp_count = 0, pds_count = 0, acc_count = 0, q_count = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+      int g, s, kt, rt0, rt1, t_beg, t_end, b0, nb;
+      item_of(it, g, s, kt, rt0, rt1, t_beg, t_end, b0, nb);
+      const int nrt = rt1 - rt0;
+      bool ok = true;
+      for (int i = 0; i < nrt; ++i) {
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
+        tc_fence_after();
+        float sv[64], dp[64];
+        tmem_ld32(tm_s + lane_off + r0, sv);
+        tmem_ld32(tm_s + lane_off + r0 + 32, sv + 32);
+        tmem_ld32(tm_dp + lane_off + r0, dp);
+        tmem_ld32(tm_dp + lane_off + r0 + 32, dp + 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sdp_empty);
+        ++sdp_count;
+        // the row scalars of this row tile were stored before q_full[qb] was armed
+        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        uint32_t pw[32], dsv[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[qb][r0 + c]);
+          const float4 d4 = *reinterpret_cast<const float4*>(&sm.Dr[qb][r0 + c]);
+          const float4 w4 = *reinterpret_cast<const float4*>(&sm.wr[qb][r0 + c]);
+          const float p0 = exp2f(sv[c] * qs2 - l4.x), p1 = exp2f(sv[c + 1] * qs2 - l4.y);
+          const float p2 = exp2f(sv[c + 2] * qs2 - l4.z), p3 = exp2f(sv[c + 3] * qs2 - l4.w);
+          pw[c / 2] = pack_bf16x2(p0 * w4.x, p1 * w4.y);
+          pw[c / 2 + 1] = pack_bf16x2(p2 * w4.z, p3 * w4.w);
+          dsv[c / 2] = pack_bf16x2(p0 * (w4.x * dp[c] - d4.x), p1 * (w4.y * dp[c + 1] - d4.y));
+          dsv[c / 2 + 1] = pack_bf16x2(p2 * (w4.z * dp[c + 2] - d4.z), p3 * (w4.w * dp[c + 3] - d4.w));
+        }
+        if (!mbar_wait(&sm.pds_empty, (pds_count & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st16(tm_p + lane_off + 32 * wg, pw);
+        tmem_st16(tm_p + lane_off + 32 * wg + 16, pw + 16);
+        tmem_st16(tm_ds + lane_off + 32 * wg, dsv);
+        tmem_st16(tm_ds + lane_off + 32 * wg + 16, dsv + 16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.pds_full);
+        ++pds_count;
+        ++q_count;
+      }
+      if (!ok) {
+        record_timeout(status, &sm.abort_flag);
+        break;
+      }
+      if (!mbar_wait(&sm.acc_full, acc_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      ++acc_count;
+      tc_fence_after();
+      // warpgroup 0 adds dKc, warpgroup 1 adds dVc (lane = block)
+      float acc[64];
+      const uint32_t src = (wg == 0 ? tm_dk : tm_dv) + lane_off;
+      tmem_ld32(src, acc);
+      tmem_ld32(src + 32, acc + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty);
+      const int bidx = kt * kBN + b;
+      if (bidx < nb && nrt > 0) {
+        float* dst = (wg == 0 ? dkc : dvc) + ((int64_t)g * btot + b0 + bidx) * 64;
+        const float mul = wg == 0 ? scale : 1.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          atomicAdd(reinterpret_cast<float4*>(dst) + i,
+                    make_float4(acc[4 * i] * mul, acc[4 * i + 1] * mul, acc[4 * i + 2] * mul, acc[4 * i + 3] * mul));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -817,6 +1319,62 @@ cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_ti
   return cudaGetLastError();
 }
 
+
+__global__ void dkv_plan_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, int S, int G,
+                                int32_t* __restrict__ cnt) {
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s <= S; s += gridDim.x * blockDim.x) {
+    if (s == S) {
+      cnt[s] = 0;
+      continue;
+    }
+    const int nb = bcu[s + 1] - bcu[s];
+    const int64_t rows = (int64_t)(cu[s + 1] - cu[s]) * G;
+    const int64_t nrt = (rows + kRows - 1) / kRows;
+    const int64_t nch = (nrt + kDkvRowTilesPerItem - 1) / kDkvRowTilesPerItem;
+    cnt[s] = (int32_t)(((nb + kBN - 1) / kBN) * nch);
+  }
+}
+
+size_t smem_bytes_dq() { return sizeof(DqSmem) + 1024; }
+size_t smem_bytes_dkv() { return sizeof(DkvSmem) + 1024; }
+
+template <int G>
+cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, int32_t* dkv_pre,
+                         int32_t* scan_tmp, int64_t tiles_bound, cudaStream_t st) {
+  CUtensorMap qm, dm, km, vm;
+  const int64_t rows_kv = (int64_t)a.hkv * a.blk->count;
+  if (!map_q(&qm, a.q, a.N, a.hq, G) || !map_q(&dm, a.dout, a.N, a.hq, G) || !map_rows64(&km, a.kc, rows_kv) ||
+      !map_rows64(&vm, a.vc, rows_kv))
+    return cudaErrorInvalidValue;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(cmp_bwd_dq_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_dq());
+    cudaFuncSetAttribute(cmp_bwd_dq_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_dq());
+    cudaFuncSetAttribute(cmp_bwd_dkv_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes_dkv());
+    cudaFuncSetAttribute(cmp_bwd_dkv_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes_dkv());
+    attr_done = true;
+  }
+  const float qs2 = a.scale * kLog2e;
+  const int btot = (int)a.blk->count;
+  const int sms = num_sms();
+  const int64_t tiles = tiles_bound * a.hkv;
+  const int gq = (int)(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);
+  SSA_LAUNCH("cmp_bwd_dq_tc_kernel", cmp_bwd_dq_tc_kernel<G>, gq, kOutThreads, smem_bytes_dq(), st, qm, dm, km, vm,
+             a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.gates, a.gate_mode,
+             a.dq, a.status);
+  SSA_LAUNCH("dkv_plan_kernel", dkv_plan_kernel, (a.S + 256) / 256, 256, 0, st, a.cu_seqlens, a.blk->cu, a.S, G,
+             dkv_cnt);
+  cudaError_t e = exclusive_scan(dkv_cnt, dkv_pre, a.S + 1, scan_tmp, st);
+  if (e != cudaSuccess) return e;
+  cudaMemsetAsync(a.dkc, 0, sizeof(float) * rows_kv * 64, st);
+  cudaMemsetAsync(a.dvc, 0, sizeof(float) * rows_kv * 64, st);
+  SSA_LAUNCH("cmp_bwd_dkv_tc_kernel", cmp_bwd_dkv_tc_kernel<G>, sms, kOutThreads, smem_bytes_dkv(), st, qm, dm, km,
+             vm, a.cu_seqlens, a.blk->cu, dkv_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.gates,
+             a.gate_mode, a.dkc, a.dvc, a.status);
+  return cudaGetLastError();
+}
 }  // namespace
 
 size_t cmp_tc_scratch_floats(int hq, int hkv, int64_t btot) {
@@ -838,4 +1396,16 @@ cudaError_t cmp_fwd_tc(const FwdArgs& a, const int32_t* tpre, int64_t total_tile
   return cudaErrorInvalidValue;
 }
 
+}  // namespace ssa
+
+namespace ssa {
+// Compressed branch backward on the tensor cores: dQ (written), dKc / dVc (fp32
+// workspace, accumulated).  `tpre` is the per-sequence prefix of 128-row tiles.
+cudaError_t cmp_bwd_tc(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, int32_t* dkv_pre, int32_t* scan_tmp,
+                       int64_t tiles_bound, cudaStream_t st) {
+  const int G = a.hq / a.hkv;
+  if (G == 16) return cmp_bwd_tc_g<16>(a, tpre, dkv_cnt, dkv_pre, scan_tmp, tiles_bound, st);
+  if (G == 8) return cmp_bwd_tc_g<8>(a, tpre, dkv_cnt, dkv_pre, scan_tmp, tiles_bound, st);
+  return cudaErrorInvalidValue;
+}
 }  // namespace ssa

@@ -73,6 +73,8 @@ cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st);
 bool cmp_tc_supported(int dtype, int d, int hq, int hkv, int topk);
 size_t cmp_tc_scratch_floats(int hq, int hkv, int64_t btot);
 cudaError_t cmp_fwd_tc(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st);
+cudaError_t cmp_bwd_tc(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, int32_t* dkv_pre, int32_t* scan_tmp,
+                       int64_t tiles_bound, cudaStream_t st);
 cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st);
 
 }  // namespace ssa

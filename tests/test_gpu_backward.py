@@ -43,7 +43,11 @@ def test_zero_gates_give_zero_input_gradients():
 
 
 def test_gradient_sums():
-    """Softmax rows sum to one: sum_i dV_i = sum_rows w_c dO; key gradients sum to 0."""
+    """Softmax rows sum to one: sum_i dV_i = sum_rows w_c dO; key gradients sum to 0.
+
+    The sums run over ~10^4 rounded terms (the tensor-core kernels multiply bf16
+    P and dS), so the tolerance grows with the magnitude of what is summed:
+    2e-2 + 1e-3 x (sum of the absolute values of the terms)."""
     w = W.small_shell(seed=13, R=40, n_prims=2, lo=5.0, hi=11.0, n_keep=1500)
     t = W.make_tensors(w)
     run = GpuRun(w, t).run()
@@ -54,5 +58,7 @@ def test_gradient_sums():
     for g in range(w.hkv):
         hs = slice(g * G, (g + 1) * G)
         want = np.einsum("nh,nhd->d", gw[:, hs, :].sum(-1), do[:, hs, :])
-        np.testing.assert_allclose(dv[:, g, :].sum(0), want, atol=2e-2)
-        np.testing.assert_allclose(dk[:, g, :].sum(0), 0.0, atol=2e-2)
+        mag_v = np.einsum("nh,nhd->d", gw[:, hs, :].sum(-1), np.abs(do[:, hs, :]))
+        assert (np.abs(dv[:, g, :].sum(0) - want) <= 2e-2 + 1e-3 * mag_v).all()
+        mag_k = np.abs(dk[:, g, :]).sum(0)
+        assert (np.abs(dk[:, g, :].sum(0)) <= 2e-2 + 1e-3 * mag_k).all()
