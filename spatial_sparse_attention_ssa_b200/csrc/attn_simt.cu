@@ -811,6 +811,136 @@ __global__ void __launch_bounds__(128) slc_bwd_dkv_kernel(
   }
 }
 
+// selected branch backward, query-centric and fused (head dim 64, G in {8, 16}):
+// one warp per (token, group); lane l owns dims {2l, 2l+1} of every head of the
+// group.  For each key of the selected blocks the per-head dot products are
+// reduced across the warp by a transpose-reduction (G values, G shuffles), each
+// lane finishes the softmax gradient of its head, the results are broadcast,
+// and the warp accumulates dQ in registers and adds dK, dV rows of the key with
+// fp32 vector atomics.  Q and dO are read once per pair.
+template <typename T>
+__device__ __forceinline__ float2 load2(const T* p);
+template <>
+__device__ __forceinline__ float2 load2<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+template <>
+__device__ __forceinline__ float2 load2<float>(const float* p) {
+  return __ldg(reinterpret_cast<const float2*>(p));
+}
+
+// Sum over the 32 lanes of each of the G values a[0..G); on return the 32/G
+// lanes [h * 32/G, (h+1) * 32/G) hold the total of value h (G in {8, 16}).
+template <int G>
+__device__ __forceinline__ float warp_transpose_reduce(float (&a)[G]) {
+  const int lane = threadIdx.x & 31;
+  float v[G];
+#pragma unroll
+  for (int i = 0; i < G; ++i) v[i] = a[i];
+  // offsets 16, 8, 4, 2 halve the number of values per lane (head bits 3..0 <- lane bits 4..1)
+  int n = G;
+#pragma unroll
+  for (int off = 16; off >= 2; off >>= 1) {
+    if (n == 1) {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+      continue;
+    }
+    const bool up = (lane & off) != 0;
+    const int h = n / 2;
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) {
+      if (i < h) {
+        const float send = up ? v[i] : v[i + h];
+        const float keep = up ? v[i + h] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+    }
+    n = h;
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(256) slc_bwd_fused_kernel(
+    const T* __restrict__ q, const T* __restrict__ ks, const T* __restrict__ vs, const T* __restrict__ dout,
+    const float* __restrict__ gates, int mode, const int32_t* __restrict__ bptr, const int32_t* __restrict__ bperm,
+    const int32_t* __restrict__ sel, int64_t N, int hq, int hkv, int topk, float qs2, float scale,
+    const float* __restrict__ lse_in, const float* __restrict__ Dc, float* __restrict__ dq_out,
+    float* __restrict__ dk_out, float* __restrict__ dv_out) {
+  constexpr int D = 64;
+  const int lane = threadIdx.x & 31;
+  const int wpc = blockDim.x / 32;
+  const int64_t npairs = N * hkv;
+  // head whose softmax this lane finishes after the reduction: lanes [h LPH, (h+1) LPH) -> head h
+  constexpr int LPH = 32 / G;
+  const int myh = lane / LPH;
+  for (int64_t pair = (int64_t)blockIdx.x * wpc + threadIdx.x / 32; pair < npairs; pair += (int64_t)gridDim.x * wpc) {
+    const int64_t t = pair / hkv;
+    const int g = (int)(pair % hkv);
+    float q2[G][2], d2[G][2], dq2[G][2];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const int64_t row = t * hq + g * G + h;
+      const float2 a = load2<T>(q + row * D + 2 * lane);
+      const float2 b = load2<T>(dout + row * D + 2 * lane);
+      const float w = gate_weight(gates, row * 3 + 1, mode);
+      q2[h][0] = a.x;
+      q2[h][1] = a.y;
+      d2[h][0] = b.x * w;
+      d2[h][1] = b.y * w;
+      dq2[h][0] = dq2[h][1] = 0.f;
+    }
+    const int64_t my_row = t * hq + g * G + myh;
+    const float lse2 = lse_in[my_row] * kLog2e;
+    const float Dm = Dc[my_row];
+    const int32_t* srow = sel + pair * topk;
+    for (int si = 0; si < topk; ++si) {
+      const int b = srow[si];
+      if (b < 0) continue;
+      const int p1 = bptr[b + 1];
+      for (int j = bptr[b]; j < p1; ++j) {
+        const int64_t kidx = (int64_t)g * N + j;
+        const float2 kk = load2<T>(ks + kidx * D + 2 * lane);
+        const float2 vv = load2<T>(vs + kidx * D + 2 * lane);
+        float ps[G], pd[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          ps[h] = q2[h][0] * kk.x + q2[h][1] * kk.y;
+          pd[h] = d2[h][0] * vv.x + d2[h][1] * vv.y;
+        }
+        const float s2 = warp_transpose_reduce<G>(ps) * qs2;
+        const float dp = warp_transpose_reduce<G>(pd);
+        const float pm = exp2f(s2 - lse2);
+        const float dsm = pm * (dp - Dm);
+        float dk0 = 0.f, dk1 = 0.f, dv0 = 0.f, dv1 = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float ph = __shfl_sync(0xffffffffu, pm, h * LPH);
+          const float dsh = __shfl_sync(0xffffffffu, dsm, h * LPH);
+          dq2[h][0] = fmaf(dsh, kk.x, dq2[h][0]);
+          dq2[h][1] = fmaf(dsh, kk.y, dq2[h][1]);
+          dk0 = fmaf(dsh, q2[h][0], dk0);
+          dk1 = fmaf(dsh, q2[h][1], dk1);
+          dv0 = fmaf(ph, d2[h][0], dv0);
+          dv1 = fmaf(ph, d2[h][1], dv1);
+        }
+        const int64_t tok = bperm[j];
+        atomicAdd(reinterpret_cast<float2*>(dk_out + (tok * hkv + g) * D + 2 * lane), make_float2(dk0 * scale, dk1 * scale));
+        atomicAdd(reinterpret_cast<float2*>(dv_out + (tok * hkv + g) * D + 2 * lane), make_float2(dv0, dv1));
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float2* dst = reinterpret_cast<float2*>(dq_out + (t * hq + g * G + h) * D + 2 * lane);
+      float2 cur = *dst;
+      cur.x += dq2[h][0] * scale;
+      cur.y += dq2[h][1] * scale;
+      *dst = cur;
+    }
+  }
+}
+
 // window branch: dQ
 template <typename T, int D>
 __global__ void __launch_bounds__(128) win_bwd_dq_kernel(
@@ -1089,32 +1219,46 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
         q, kc, vc, dout, a.gates, a.gate_mode, a.cu_seqlens, a.blk->cu, a.items_pre, a.S, a.hq, a.hkv, btot, qs2,
         a.scale, kCmpRowChunk, a.lse, a.Dc, a.dkc, a.dvc);
   }
-  const int pairs_per_cta = 128 / (G * C::NT);
-  SSA_LAUNCH("slc_bwd_dq_kernel", (slc_bwd_dq_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
-      q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
-      a.Dc + rows, a.dq);
-  // inverted selection CSR: for (g, b), the tokens whose group g selected b, ascending
-  const int64_t nsel = a.N * a.hkv * a.topk;
-  const int64_t nkeys = a.hkv * btot;
-  SSA_LAUNCH("sel_keys_kernel", sel_keys_kernel, grid_1d(nsel, 256, 148 * 32), 256, 0, st, a.sel, a.N, a.hkv, a.topk, btot, a.inv_keys_a,
-                                                                a.inv_vals_a);
-  int bits = 1;
-  while ((1ll << bits) <= nkeys) ++bits;
-  bool in_b = false;
-  e = radix_sort_pairs(a.inv_keys_a, a.inv_vals_a, a.inv_keys_b, a.inv_vals_b, nsel, bits, a.radix_tmp, &in_b, st);
-  if (e != cudaSuccess) return e;
-  const uint64_t* sk = in_b ? a.inv_keys_b : a.inv_keys_a;
-  const int32_t* sv = in_b ? a.inv_vals_b : a.inv_vals_a;
-  SSA_LAUNCH("keys_to_ptr_kernel", keys_to_ptr_kernel, grid_1d(nsel + 1, 256, 148 * 32), 256, 0, st, sk, nsel, nkeys, a.inv_ptr);
-  SSA_LAUNCH("slc_items_kernel", slc_items_kernel, grid_1d(nkeys + 1, 256, 148 * 32), 256, 0, st, a.inv_ptr, nkeys,
-             G, a.slc_cnt);
-  e = exclusive_scan(a.slc_cnt, a.slc_pre, nkeys + 1, a.scan_tmp, st);
-  if (e != cudaSuccess) return e;
-  cudaMemsetAsync(a.dk, 0, sizeof(float) * a.N * a.hkv * D, st);
-  cudaMemsetAsync(a.dv, 0, sizeof(float) * a.N * a.hkv * D, st);
-  SSA_LAUNCH("slc_bwd_dkv_kernel", (slc_bwd_dkv_kernel<T, D>), 148 * 8, 128, 0, st, q, ks, vs, dout, a.gates,
-             a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.slc_pre, a.N, btot, a.hq, a.hkv, qs2, a.scale,
-             a.lse + rows, a.Dc + rows, a.dk, a.dv);
+  if (D == 64 && (G == 8 || G == 16)) {
+    cudaMemsetAsync(a.dk, 0, sizeof(float) * a.N * a.hkv * D, st);
+    cudaMemsetAsync(a.dv, 0, sizeof(float) * a.N * a.hkv * D, st);
+    const int g_slc = grid_1d(a.N * a.hkv, 8, 148 * 16);
+    if (G == 16)
+      SSA_LAUNCH("slc_bwd_fused_kernel", (slc_bwd_fused_kernel<T, 16>), g_slc, 256, 0, st, q, ks, vs, dout, a.gates,
+                 a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
+                 a.Dc + rows, a.dq, a.dk, a.dv);
+    else
+      SSA_LAUNCH("slc_bwd_fused_kernel", (slc_bwd_fused_kernel<T, 8>), g_slc, 256, 0, st, q, ks, vs, dout, a.gates,
+                 a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
+                 a.Dc + rows, a.dq, a.dk, a.dv);
+  } else {
+    const int pairs_per_cta = 128 / (G * C::NT);
+    SSA_LAUNCH("slc_bwd_dq_kernel", (slc_bwd_dq_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
+        q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
+        a.Dc + rows, a.dq);
+    // inverted selection CSR: for (g, b), the tokens whose group g selected b, ascending
+    const int64_t nsel = a.N * a.hkv * a.topk;
+    const int64_t nkeys = a.hkv * btot;
+    SSA_LAUNCH("sel_keys_kernel", sel_keys_kernel, grid_1d(nsel, 256, 148 * 32), 256, 0, st, a.sel, a.N, a.hkv, a.topk, btot, a.inv_keys_a,
+                                                                  a.inv_vals_a);
+    int bits = 1;
+    while ((1ll << bits) <= nkeys) ++bits;
+    bool in_b = false;
+    e = radix_sort_pairs(a.inv_keys_a, a.inv_vals_a, a.inv_keys_b, a.inv_vals_b, nsel, bits, a.radix_tmp, &in_b, st);
+    if (e != cudaSuccess) return e;
+    const uint64_t* sk = in_b ? a.inv_keys_b : a.inv_keys_a;
+    const int32_t* sv = in_b ? a.inv_vals_b : a.inv_vals_a;
+    SSA_LAUNCH("keys_to_ptr_kernel", keys_to_ptr_kernel, grid_1d(nsel + 1, 256, 148 * 32), 256, 0, st, sk, nsel, nkeys, a.inv_ptr);
+    SSA_LAUNCH("slc_items_kernel", slc_items_kernel, grid_1d(nkeys + 1, 256, 148 * 32), 256, 0, st, a.inv_ptr, nkeys,
+               G, a.slc_cnt);
+    e = exclusive_scan(a.slc_cnt, a.slc_pre, nkeys + 1, a.scan_tmp, st);
+    if (e != cudaSuccess) return e;
+    cudaMemsetAsync(a.dk, 0, sizeof(float) * a.N * a.hkv * D, st);
+    cudaMemsetAsync(a.dv, 0, sizeof(float) * a.N * a.hkv * D, st);
+    SSA_LAUNCH("slc_bwd_dkv_kernel", (slc_bwd_dkv_kernel<T, D>), 148 * 8, 128, 0, st, q, ks, vs, dout, a.gates,
+               a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.slc_pre, a.N, btot, a.hq, a.hkv, qs2, a.scale,
+               a.lse + rows, a.Dc + rows, a.dk, a.dv);
+  }
   const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
   SSA_LAUNCH("win_bwd_dq_kernel", (win_bwd_dq_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
                                               a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
