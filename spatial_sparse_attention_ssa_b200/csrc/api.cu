@@ -90,6 +90,7 @@ size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W
 
 struct BwdWs {
   float* Dc;
+  float* wcmp;
   float *dkc, *dvc;
   uint64_t *ka, *kb;
   int32_t *va, *vb, *inv_ptr, *radix_tmp, *slc_cnt, *slc_pre;
@@ -100,6 +101,7 @@ size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t 
   Carver c(base);
   const int64_t nsel = N * p->hkv * p->topk;
   w->Dc = c.take<float>(3 * N * p->hq);
+  w->wcmp = c.take<float>(N * p->hq);
   w->dkc = c.take<float>(p->hkv * B * p->d);
   w->dvc = c.take<float>(p->hkv * B * p->d);
   w->ka = c.take<uint64_t>(nsel);
@@ -319,6 +321,7 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.dv = dv;
   a.dgates = dgates;
   a.Dc = w.Dc;
+  a.wcmp = w.wcmp;
   a.dkc = w.dkc;
   a.dvc = w.dvc;
   a.inv_keys_a = w.ka;

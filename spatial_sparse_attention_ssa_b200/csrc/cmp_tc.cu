@@ -975,9 +975,9 @@ struct DkvSmem {
   uint8_t vc[kTile];
   uint8_t q[2][kTile];
   uint8_t dout[2][kTile];
-  __align__(16) float lse2[2][kRows];
-  __align__(16) float Dr[2][kRows];
-  __align__(16) float wr[2][kRows];
+  __align__(128) float lse2[2][kRows];  // TMA destinations: 128-byte aligned
+  __align__(128) float Dr[2][kRows];
+  __align__(128) float wr[2][kRows];
   uint64_t kv_full, kv_empty, q_full[2], q_empty[2];
   uint64_t sdp_full, sdp_empty, pds_full, pds_empty, acc_full, acc_empty, mma_done;
   uint32_t tmem;
@@ -988,9 +988,10 @@ template <int G>
 __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
     const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
-    const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ ipre, int S, int hq,
-    int hkv, int btot, float qs2, float scale, const float* __restrict__ lse_in, const float* __restrict__ Dc,
-    const float* __restrict__ gates, int gate_mode, float* __restrict__ dkc, float* __restrict__ dvc, int* status) {
+    const __grid_constant__ CUtensorMap lsemap, const __grid_constant__ CUtensorMap dcmap,
+    const __grid_constant__ CUtensorMap wmap, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
+    const int32_t* __restrict__ ipre, int S, int hq, int hkv, int btot, float qs2, float scale,
+    float* __restrict__ dkc, float* __restrict__ dvc, int* status) {
   extern __shared__ uint8_t smem_raw[];
   DkvSmem& sm = *reinterpret_cast<DkvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -1073,21 +1074,14 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
         okw = __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
         if (!okw) { record_timeout(status, &sm.abort_flag); break; }
         const int t0 = t_beg + rt * TPT;
-        // row scalars of this row tile (lse in the log2 domain, D, gate weight)
-        for (int rr = lane; rr < kRows; rr += 32) {
-          const int64_t t = t0 + rr / G;
-          const bool v = t < t_end;
-          const int64_t row = (v ? t : t_end - 1) * hq + g * G + rr % G;
-          const float gx = gates[row * 3 + 0];
-          sm.lse2[qb][rr] = v ? lse_in[row] * kLog2e : CUDART_INF_F;
-          sm.Dr[qb][rr] = v ? Dc[row] : 0.f;
-          sm.wr[qb][rr] = v ? (gate_mode == SSA_GATE_LOGITS ? 1.f / (1.f + expf(-gx)) : gx) : 0.f;
-        }
-        __syncwarp();
         if (lane == 0) {
-          mbar_expect_tx(&sm.q_full[qb], 2 * kTile);
+          // Q, dO tiles and the row scalars (lse, D, gate weight) of the row tile
+          mbar_expect_tx(&sm.q_full[qb], 2 * kTile + 3 * kRows * 4);
           tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, g * G, t0);
           tma_load_3d(sm.dout[qb], &dmap, &sm.q_full[qb], 0, g * G, t0);
+          tma_load_2d(sm.lse2[qb], &lsemap, &sm.q_full[qb], g * G, t0);
+          tma_load_2d(sm.Dr[qb], &dcmap, &sm.q_full[qb], g * G, t0);
+          tma_load_2d(sm.wr[qb], &wmap, &sm.q_full[qb], g * G, t0);
         }
         ++q_count;
       }
@@ -1176,14 +1170,20 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.sdp_empty);
         ++sdp_count;
-        // the row scalars of this row tile were stored before q_full[qb] was armed
+        // row scalars of this row tile arrived with q_full[qb] (already complete for the MMA)
         if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        const int t_first = t_beg + (rt0 + i) * TPT;  // rows of tokens >= t_end contribute nothing
         uint32_t pw[32], dsv[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[qb][r0 + c]);
+          float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[qb][r0 + c]);
           const float4 d4 = *reinterpret_cast<const float4*>(&sm.Dr[qb][r0 + c]);
           const float4 w4 = *reinterpret_cast<const float4*>(&sm.wr[qb][r0 + c]);
+          const bool vrow = t_first + (r0 + c) / G < t_end;  // the 4 rows share a token (G >= 4)
+          l4.x = vrow ? l4.x * kLog2e : CUDART_INF_F;
+          l4.y = vrow ? l4.y * kLog2e : CUDART_INF_F;
+          l4.z = vrow ? l4.z * kLog2e : CUDART_INF_F;
+          l4.w = vrow ? l4.w * kLog2e : CUDART_INF_F;
           const float p0 = exp2f(sv[c] * qs2 - l4.x), p1 = exp2f(sv[c + 1] * qs2 - l4.y);
           const float p2 = exp2f(sv[c + 2] * qs2 - l4.z), p3 = exp2f(sv[c + 3] * qs2 - l4.w);
           pw[c / 2] = pack_bf16x2(p0 * w4.x, p1 * w4.y);
@@ -1275,6 +1275,20 @@ bool map_q(CUtensorMap* m, const void* base, int64_t n, int hq, int G) {
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D map over per-row fp32 scalars [N, Hq] with a box of (G heads, 128/G tokens), no swizzle:
+// one box is the 128 row scalars of a row tile in row order.
+bool map_rowscalars(CUtensorMap* m, const float* base, int64_t n, int hq, int G) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)hq, (cuuint64_t)n};
+  cuuint64_t strides[1] = {(cuuint64_t)hq * 4};
+  cuuint32_t box[2] = {(cuuint32_t)G, (cuuint32_t)(kRows / G)};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1370,9 +1384,13 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
   if (e != cudaSuccess) return e;
   cudaMemsetAsync(a.dkc, 0, sizeof(float) * rows_kv * 64, st);
   cudaMemsetAsync(a.dvc, 0, sizeof(float) * rows_kv * 64, st);
+  CUtensorMap lm, dcm, wm;
+  if (!map_rowscalars(&lm, a.lse, a.N, a.hq, G) || !map_rowscalars(&dcm, a.Dc, a.N, a.hq, G) ||
+      !map_rowscalars(&wm, a.wcmp, a.N, a.hq, G))
+    return cudaErrorInvalidValue;
   SSA_LAUNCH("cmp_bwd_dkv_tc_kernel", cmp_bwd_dkv_tc_kernel<G>, sms, kOutThreads, smem_bytes_dkv(), st, qm, dm, km,
-             vm, a.cu_seqlens, a.blk->cu, dkv_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.gates,
-             a.gate_mode, a.dkc, a.dvc, a.status);
+             vm, lm, dcm, wm, a.cu_seqlens, a.blk->cu, dkv_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.dkc, a.dvc,
+             a.status);
   return cudaGetLastError();
 }
 }  // namespace

@@ -56,6 +56,7 @@ struct BwdArgs {
   float *dq, *dk, *dv, *dgates;
   // workspace
   float* Dc;          // [3, N, Hq]
+  float* wcmp;        // [N, Hq] gate weights of the compressed branch
   float *dkc, *dvc;   // [Hkv, B, d]
   uint64_t *inv_keys_a, *inv_keys_b;
   int32_t *inv_vals_a, *inv_vals_b;
