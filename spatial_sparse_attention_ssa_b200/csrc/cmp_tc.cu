@@ -220,8 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1) cmp_lse_tc_kernel(
         const float mn = fmaxf(m, cm);
         float acc = 0.f;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) acc += exp2f(sv[c] - mn);
-        l = l * exp2f(m - mn) + acc;
+        for (int c = 0; c < kBN; ++c) acc += ex2(sv[c] - mn);
+        l = l * ex2(m - mn) + acc;
         m = mn;
       }
       if (!ok) break;
@@ -424,20 +424,55 @@ __device__ void warp_topk_fast(const float* __restrict__ imp, int nb, int topk, 
   const int src = __ffs(own) - 1;
   const float tv = __shfl_sync(0xffffffffu, bv, src);
   const int ti = __shfl_sync(0xffffffffu, bi, src);
-  // 3. collect entries at or above (tv, ti)
+  // 3. collect entries at or above (tv, ti): 512 entries per round, 4 float4 loads per lane in flight
   int n = 0;
   bool overflow = false;
-  for (int base = 0; base < nb && !overflow; base += 32) {
-    const int i = base + lane;
-    const float x = i < nb ? imp[i] : -CUDART_INF_F;
-    const bool take = i < nb && (x == tv ? i <= ti : x > tv);
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    const int slot = n + __popc(m & ((1u << lane) - 1u));
-    if (take && slot < kCandMax) {
-      cv[slot] = x;
-      ci[slot] = i;
+  for (int base = 0; base < nb && !overflow; base += 512) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i0 = base + u * 128 + lane * 4;
+      if (i0 + 3 < nb) {
+        v[u] = *reinterpret_cast<const float4*>(imp + i0);
+      } else {
+        v[u].x = i0 + 0 < nb ? imp[i0 + 0] : -CUDART_INF_F;
+        v[u].y = i0 + 1 < nb ? imp[i0 + 1] : -CUDART_INF_F;
+        v[u].z = i0 + 2 < nb ? imp[i0 + 2] : -CUDART_INF_F;
+        v[u].w = -CUDART_INF_F;
+      }
     }
-    n += __popc(m);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i0 = base + u * 128 + lane * 4;
+      const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      bool tk[4];
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + e;
+        tk[e] = i < nb && (xs[e] == tv ? i <= ti : xs[e] > tv);
+        c += tk[e] ? 1 : 0;
+      }
+      // exclusive prefix of c over the lanes
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int slot = n + incl - c;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (tk[e]) {
+          if (slot < kCandMax) {
+            cv[slot] = xs[e];
+            ci[slot] = i0 + e;
+          }
+          ++slot;
+        }
+      }
+      n += __shfl_sync(0xffffffffu, incl, 31);
+    }
     overflow = n > kCandMax;
   }
   if (overflow) {
@@ -651,10 +686,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
 #pragma unroll
         for (int r = 0; r < 64; r += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[r0 + r]);
-          p[r + 0] = bvalid ? exp2f(p[r + 0] * qs2 - l4.x) : 0.f;
-          p[r + 1] = bvalid ? exp2f(p[r + 1] * qs2 - l4.y) : 0.f;
-          p[r + 2] = bvalid ? exp2f(p[r + 2] * qs2 - l4.z) : 0.f;
-          p[r + 3] = bvalid ? exp2f(p[r + 3] * qs2 - l4.w) : 0.f;
+          p[r + 0] = bvalid ? ex2(p[r + 0] * qs2 - l4.x) : 0.f;
+          p[r + 1] = bvalid ? ex2(p[r + 1] * qs2 - l4.y) : 0.f;
+          p[r + 2] = bvalid ? ex2(p[r + 2] * qs2 - l4.z) : 0.f;
+          p[r + 3] = bvalid ? ex2(p[r + 3] * qs2 - l4.w) : 0.f;
         }
         if (!mbar_wait(&sm.pt_empty, (pt_count & 1) ^ 1)) { ok = false; break; }
 #pragma unroll
@@ -916,8 +951,8 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           float d0 = 0.f, d1 = 0.f;
-          if (c < nvalid) d0 = exp2f(sv[c] * qs2 - lse2) * (wr * dp[c] - Dr);
-          if (c + 1 < nvalid) d1 = exp2f(sv[c + 1] * qs2 - lse2) * (wr * dp[c + 1] - Dr);
+          if (c < nvalid) d0 = ex2(sv[c] * qs2 - lse2) * (wr * dp[c] - Dr);
+          if (c + 1 < nvalid) d1 = ex2(sv[c + 1] * qs2 - lse2) * (wr * dp[c + 1] - Dr);
           const __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
           const float2 hf = __bfloat1622float2(h);
           hi[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
@@ -1184,8 +1219,8 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
           l4.y = vrow ? l4.y * kLog2e : CUDART_INF_F;
           l4.z = vrow ? l4.z * kLog2e : CUDART_INF_F;
           l4.w = vrow ? l4.w * kLog2e : CUDART_INF_F;
-          const float p0 = exp2f(sv[c] * qs2 - l4.x), p1 = exp2f(sv[c + 1] * qs2 - l4.y);
-          const float p2 = exp2f(sv[c + 2] * qs2 - l4.z), p3 = exp2f(sv[c + 3] * qs2 - l4.w);
+          const float p0 = ex2(sv[c] * qs2 - l4.x), p1 = ex2(sv[c + 1] * qs2 - l4.y);
+          const float p2 = ex2(sv[c + 2] * qs2 - l4.z), p3 = ex2(sv[c + 3] * qs2 - l4.w);
           pw[c / 2] = pack_bf16x2(p0 * w4.x, p1 * w4.y);
           pw[c / 2 + 1] = pack_bf16x2(p2 * w4.z, p3 * w4.w);
           dsv[c / 2] = pack_bf16x2(p0 * (w4.x * dp[c] - d4.x), p1 * (w4.y * dp[c + 1] - d4.y));
