@@ -158,6 +158,15 @@ def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
     e = 2  # bf16 bytes
     N, B = w.n, len(bsize)
     work = {
+        # tensor-core kernels: (kind, contraction flops, exps) -- the exps bound them at d = 64
+        "cmp_lse_tc_kernel": ("tc", 2 * d * sc_cmp, sc_cmp),
+        "cmp_out_tc_kernel": ("tc", 4 * d * sc_cmp, sc_cmp),
+        "cmp_bwd_dq_tc_kernel": ("tc", 6 * d * sc_cmp, sc_cmp),
+        "cmp_bwd_dkv_tc_kernel": ("tc", 8 * d * sc_cmp, sc_cmp),
+        "win_fwd_tc_kernel": ("tc", 4 * d * sc_win, 2 * sc_win),
+        "win_bwd_dq_tc_kernel": ("tc", 6 * d * sc_win, sc_win),
+        "win_bwd_dkv_tc_kernel": ("tc", 8 * d * sc_win, sc_win),
+        "slc_bwd_fused_kernel": ("flops", 10 * d * sc_slc),
         "cmp_lse_kernel": ("flops", 2 * d * sc_cmp),
         "cmp_out_topk_kernel": ("flops", 4 * d * sc_cmp),
         "slc_fwd_kernel": ("flops", 4 * d * sc_slc),
@@ -231,9 +240,18 @@ def run_ours(a):
         ssa.ssa_backward(p, cux, b_, w_, qx, kx, vx, gx, saved, dx, grads=grads, workspace=ws_b)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
-    for _ in range(a.warmup):
+
+    def check_device(where):
+        torch.cuda.synchronize()
+        code = ssa.device_status()
+        if code != 0:
+            raise SystemExit("device check word after %s: %s" % (where, ssa.STATUS_NAMES.get(code, code)))
+
+    for i in range(a.warmup):
         step()
-    torch.cuda.synchronize()
+        if i == 0:
+            check_device("the first step")
+    check_device("warm-up")
 
     # ---- timed region: K steps, device-timed per step, L2 flushed between steps
     sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", ""))
@@ -259,6 +277,7 @@ def run_ours(a):
     ssa.profile_enable(False)
     launches = ssa.launch_count() - launches0
     prof = ssa.profile_read()
+    check_device("the timed steps")
     ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / a.steps
     ms_max = ms
     if world > 1:
@@ -315,11 +334,26 @@ def run_ours(a):
         step_ms_kernels += tot / a.steps
     dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
     roof = None
+    exp_roof = None
     if dom is not None:
         avg_ms = prof[dom][0] / max(prof[dom][1], 1)
-        kind, units = work.get(dom, ("bytes", None))
+        entry = work.get(dom, ("bytes", None))
+        kind, units = entry[0], entry[1]
         mhz = peaks.get("sm_max_mhz", 1965.0)
-        if kind == "flops" and units is not None:
+        if kind == "tc":
+            achieved = units / (avg_ms / 1e3) / 1e12
+            peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+            roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "peak_source": "%s bf16 dense, sustained (kernel timed inside the step)" % peaks["_source"],
+                    "algorithmic_per_launch": units, "ms_per_launch": avg_ms}
+            exps = entry[2]
+            mufu_peak = SMS * 16 * mhz * 1e6 / 1e12  # 16 ex2 per clock per SM
+            exp_roof = {"kernel": dom, "bound": "mufu", "achieved": exps / (avg_ms / 1e3) / 1e12,
+                        "peak": mufu_peak, "unit": "Texp/s", "frac": exps / (avg_ms / 1e3) / 1e12 / mufu_peak,
+                        "peak_source": "derived: %d SMs x 16 ex2/clock x %.0f MHz" % (SMS, mhz),
+                        "exps_per_launch": exps}
+        elif kind == "flops" and units is not None:
             achieved = units / (avg_ms / 1e3) / 1e12
             # the attention kernels in this build are fp32 SIMT (FFMA): ALU-bound
             peak = SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
@@ -348,7 +382,8 @@ def run_ours(a):
                 "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded surface-shell voxels, N(0,1) bf16 Q/K/V/dO, N(0,1) gate logits)",
-                "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+                "config": cfg, "roofline": roof, "roofline_exp": exp_roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": int(launches),
                 "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel,
                 "peaks_source": peaks["_source"]}
         print(json.dumps(line), flush=True)

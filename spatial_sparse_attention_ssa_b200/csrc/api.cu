@@ -77,14 +77,19 @@ void carve_plan(Carver& c, int32_t S, int32_t** tc, int32_t** tp, int32_t** ic, 
 size_t bin_bytes(int32_t S, int64_t N) { return ssa::bin_ws_bytes(S, N) + 256; }
 
 size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W, float** imp = nullptr,
-                 void* base = nullptr) {
+                 int32_t** wc = nullptr, int32_t** wp = nullptr, int32_t** wst = nullptr, void* base = nullptr) {
   (void)N;
-  (void)W;
   Carver c(base);
   int32_t *a, *b, *d, *e, *f;
   carve_plan(c, S, &a, &b, &d, &e, &f);
   float* x = c.take<float>(ssa::cmp_tc_scratch_floats(p->hq, p->hkv, B));
+  int32_t* y0 = c.take<int32_t>(W + 1);
+  int32_t* y1 = c.take<int32_t>(W + 1);
+  int32_t* y2 = c.take<int32_t>(ssa::scan_tmp_ints(W + 1));
   if (imp) *imp = x;
+  if (wc) *wc = y0;
+  if (wp) *wp = y1;
+  if (wst) *wst = y2;
   return c.used;
 }
 
@@ -93,11 +98,12 @@ struct BwdWs {
   float* wcmp;
   float *dkc, *dvc;
   uint64_t *ka, *kb;
-  int32_t *va, *vb, *inv_ptr, *radix_tmp, *slc_cnt, *slc_pre;
+  int32_t *va, *vb, *inv_ptr, *radix_tmp, *slc_cnt, *slc_pre, *win_cnt, *win_pre;
+  float* wwin;
   int32_t *tc, *tp, *ic, *ip, *st;
 };
 
-size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t B, BwdWs* w) {
+size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W, BwdWs* w) {
   Carver c(base);
   const int64_t nsel = N * p->hkv * p->topk;
   w->Dc = c.take<float>(3 * N * p->hq);
@@ -112,7 +118,12 @@ size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t 
   w->radix_tmp = c.take<int32_t>(ssa::radix_tmp_ints(nsel));
   w->slc_cnt = c.take<int32_t>(p->hkv * B + 1);
   w->slc_pre = c.take<int32_t>(p->hkv * B + 1);
-  w->st = c.take<int32_t>(ssa::scan_tmp_ints(p->hkv * B + 1 > S + 1 ? p->hkv * B + 1 : S + 1));
+  w->wwin = c.take<float>(N * p->hq);
+  w->win_cnt = c.take<int32_t>(W + 1);
+  w->win_pre = c.take<int32_t>(W + 1);
+  int64_t mx = p->hkv * B + 1 > S + 1 ? p->hkv * B + 1 : S + 1;
+  mx = mx > W + 1 ? mx : W + 1;
+  w->st = c.take<int32_t>(ssa::scan_tmp_ints(mx));
   int32_t* unused_st;
   carve_plan(c, S, &w->tc, &w->tp, &w->ic, &w->ip, &unused_st);
   return c.used;
@@ -145,7 +156,7 @@ SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, in
   if (op == SSA_OP_FORWARD) return fwd_bytes(p, S, N, B_tot, W_tot);
   if (op == SSA_OP_BACKWARD) {
     BwdWs w;
-    return carve_bwd(nullptr, p, S, N, B_tot, &w);
+    return carve_bwd(nullptr, p, S, N, B_tot, W_tot, &w);
   }
   return 0;
 }
@@ -242,6 +253,8 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   a.hkv = p->hkv;
   a.topk = p->topk;
   a.gate_mode = p->gate_mode;
+  a.m_cmp = p->m_cmp;
+  a.m_win = p->m_win;
   a.use_tc = tc_enabled();
   a.status = status_ptr();
   if (!a.status) return SSA_ERR_CUDA;
@@ -265,7 +278,9 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   a.sel = saved->sel;
   Carver c(ws);
   carve_plan(c, S, &a.tiles_cnt, &a.tiles_pre, &a.items_cnt, &a.items_pre, &a.scan_tmp);
-  fwd_bytes(p, S, N, blk->count, win->count, &a.imp_scratch, ws);
+  int32_t* win_scan = nullptr;
+  fwd_bytes(p, S, N, blk->count, win->count, &a.imp_scratch, &a.win_cnt, &a.win_pre, &win_scan, ws);
+  a.win_scan = win_scan;
   return cuda_status(ssa::simt_forward(a, st));
 }
 
@@ -285,8 +300,8 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
   if ((int64_t)N * p->hkv * p->topk > INT32_MAX) return SSA_ERR_UNSUPPORTED;
   BwdWs w;
-  if (ws_bytes < carve_bwd(nullptr, p, S, N, blk->count, &w)) return SSA_ERR_WORKSPACE;
-  carve_bwd(ws, p, S, N, blk->count, &w);
+  if (ws_bytes < carve_bwd(nullptr, p, S, N, blk->count, win->count, &w)) return SSA_ERR_WORKSPACE;
+  carve_bwd(ws, p, S, N, blk->count, win->count, &w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ssa::BwdArgs a;
   a.dtype = p->dtype;
@@ -295,6 +310,8 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.hkv = p->hkv;
   a.topk = p->topk;
   a.gate_mode = p->gate_mode;
+  a.m_cmp = p->m_cmp;
+  a.m_win = p->m_win;
   a.use_tc = tc_enabled();
   a.status = status_ptr();
   if (!a.status) return SSA_ERR_CUDA;
@@ -322,6 +339,9 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.dgates = dgates;
   a.Dc = w.Dc;
   a.wcmp = w.wcmp;
+  a.wwin = w.wwin;
+  a.win_cnt = w.win_cnt;
+  a.win_pre = w.win_pre;
   a.dkc = w.dkc;
   a.dvc = w.dvc;
   a.inv_keys_a = w.ka;

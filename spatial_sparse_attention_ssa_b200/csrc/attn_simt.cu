@@ -423,7 +423,7 @@ __global__ void combine_kernel(const float* __restrict__ ob, const float* __rest
 template <typename T, int D>
 __global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict__ dout, const float* __restrict__ gates,
                                int64_t rows, int mode, float* __restrict__ Dc, float* __restrict__ dgates,
-                               float* __restrict__ wcmp) {
+                               float* __restrict__ wcmp, float* __restrict__ wwin) {
   constexpr int NT = D / 32;
   const int64_t total = rows * NT;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -444,6 +444,7 @@ __global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict
         Dc[(int64_t)c * rows + row] = w * dot;
         dgates[row * 3 + c] = mode == SSA_GATE_LOGITS ? dot * w * (1.f - w) : dot;
         if (c == 0) wcmp[row] = w;
+        if (c == 2) wwin[row] = w;
       }
     }
   }
@@ -1169,6 +1170,10 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
       q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2,
       ob + rows * D, a.lse + rows);
   const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
+  if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
+    e = win_fwd_tc(a, a.win_cnt, a.win_pre, a.win_scan, st);
+    if (e != cudaSuccess) return e;
+  } else
   SSA_LAUNCH("win_fwd_kernel", (win_fwd_kernel<T, D>), gw, 128, 0, st, q, static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.win->perm,
                                            a.win->ptr, a.win->count, a.hq, a.hkv, qs2, ob + 2 * rows * D,
                                            a.lse + 2 * rows);
@@ -1202,7 +1207,7 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
 
   SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout, a.gates, rows, a.gate_mode,
-                                                                             a.Dc, a.dgates, a.wcmp);
+                                                                             a.Dc, a.dgates, a.wcmp, a.wwin);
   if (a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
     // 128-row tiles for the tensor-core kernels (tiles_cnt / tiles_pre are free again here)
     SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu,
@@ -1261,13 +1266,18 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.slc_pre, a.N, btot, a.hq, a.hkv, qs2, a.scale,
                a.lse + rows, a.Dc + rows, a.dk, a.dv);
   }
-  const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
-  SSA_LAUNCH("win_bwd_dq_kernel", (win_bwd_dq_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
-                                              a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
-                                              a.Dc + 2 * rows, a.dq);
-  SSA_LAUNCH("win_bwd_dkv_kernel", (win_bwd_dkv_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
-                                               a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
-                                               a.Dc + 2 * rows, a.dk, a.dv);
+  if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
+    e = win_bwd_tc(a, a.win_cnt, a.win_pre, a.scan_tmp, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
+    SSA_LAUNCH("win_bwd_dq_kernel", (win_bwd_dq_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
+                                                a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
+                                                a.Dc + 2 * rows, a.dq);
+    SSA_LAUNCH("win_bwd_dkv_kernel", (win_bwd_dkv_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
+                                                 a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
+                                                 a.Dc + 2 * rows, a.dk, a.dv);
+  }
   SSA_LAUNCH("cmp_scatter_kernel", cmp_scatter_kernel, grid_1d(a.N * a.hkv * D / 4, 256, 148 * 32), 256, 0, st, 
       a.dkc, a.dvc, a.blk->id, a.blk->ptr, a.N, btot, a.hkv, D, a.dk, a.dv);
   return cudaGetLastError();

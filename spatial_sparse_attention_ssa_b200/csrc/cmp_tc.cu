@@ -31,13 +31,14 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
+#include "tc_host.cuh"
 
 namespace ssa {
 namespace {
 
 using namespace tc;
+using namespace tch;
 
-constexpr int kRows = 128;           // query rows per tile
 constexpr int kBN = 128;             // compressed blocks per key tile
 constexpr int kTile = 128 * 128;     // bytes of a 128 x 64 bf16 tile
 constexpr int kStages = 4;           // key-tile ring depth
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) cmp_lse_tc_kernel(
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
         const int sb = s_count % 2;
-        if (!mbar_wait(&sm.s_full[sb], (s_count / 2) & 1)) { record_timeout(status, &sm.abort_flag); ok = false; break; }
+        if (!mbar_wait_warp(&sm.s_full[sb], (s_count / 2) & 1)) { record_timeout(status, &sm.abort_flag); ok = false; break; }
         tc_fence_after();
         float sv[kBN];
         const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + sb * kBN;
@@ -274,7 +275,7 @@ __device__ __forceinline__ bool beats(float v, int id, float v2, int id2) { retu
 __device__ __forceinline__ bool cw_sync(uint64_t* bar, uint32_t& phase) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase & 1);
+  const bool ok = mbar_wait_warp(bar, phase & 1);
   ++phase;
   return ok;
 }
@@ -670,7 +671,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
       const int nbt = (ti.nb + kBN - 1) / kBN;
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
-        if (!mbar_wait(&sm.s_full, s_count & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.s_full, s_count & 1)) { ok = false; break; }
         tc_fence_after();
         float p[64];
         const uint32_t taddr = tm_s + ((uint32_t)((warp % 4) * 32) << 16) + r0;
@@ -691,7 +692,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
           p[r + 2] = bvalid ? ex2(p[r + 2] * qs2 - l4.z) : 0.f;
           p[r + 3] = bvalid ? ex2(p[r + 3] * qs2 - l4.w) : 0.f;
         }
-        if (!mbar_wait(&sm.pt_empty, (pt_count & 1) ^ 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.pt_empty, (pt_count & 1) ^ 1)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t hi[4], lo[4];
@@ -727,7 +728,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
         break;
       }
       // O of this tile: wait for the last P Vc; warpgroup wg writes columns [32 wg, 32 wg + 32)
-      if (!mbar_wait(&sm.o_full, o_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      if (!mbar_wait_warp(&sm.o_full, o_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++o_count;
       tc_fence_after();
       {
@@ -934,7 +935,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
       const int nbt = (ti.nb + kBN - 1) / kBN;
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
-        if (!mbar_wait(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
         tc_fence_after();
         float sv[64], dp[64];
         tmem_ld32(tm_s + lane_off + 64 * wg, sv);
@@ -958,7 +959,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
           hi[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
           lo[c / 2] = pack_bf16x2(d0 - hf.x, d1 - hf.y);
         }
-        if (!mbar_wait(&sm.ds_empty, (ds_count & 1) ^ 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.ds_empty, (ds_count & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
         tmem_st16(tm_dsh + lane_off + 32 * wg, hi);
         tmem_st16(tm_dsh + lane_off + 32 * wg + 16, hi + 16);
@@ -974,7 +975,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
         record_timeout(status, &sm.abort_flag);
         break;
       }
-      if (!mbar_wait(&sm.dq_full, dq_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      if (!mbar_wait_warp(&sm.dq_full, dq_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++dq_count;
       tc_fence_after();
       float g32[32];
@@ -1010,6 +1011,10 @@ struct DkvSmem {
   uint8_t vc[kTile];
   uint8_t q[2][kTile];
   uint8_t dout[2][kTile];
+  // low bf16 parts of P^T w and dS^T [blocks, 128 rows] (K-major A operands, two
+  // 64-row atoms each); the high parts are TMEM operands
+  uint8_t plo[2 * kTile];
+  uint8_t dslo[2 * kTile];
   __align__(128) float lse2[2][kRows];  // TMA destinations: 128-byte aligned
   __align__(128) float Dr[2][kRows];
   __align__(128) float wr[2][kRows];
@@ -1162,8 +1167,13 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kRows / 16; ++k) {
-            mma_bf16_ts(tm_dv, tm_p + 8 * k, sdesc_mnmajor_sw128(sm.dout[qb], 2048 * k, kTile), id_a, i > 0 || k > 0);
-            mma_bf16_ts(tm_dk, tm_ds + 8 * k, sdesc_mnmajor_sw128(sm.q[qb], 2048 * k, kTile), id_a, i > 0 || k > 0);
+            const uint64_t bdo = sdesc_mnmajor_sw128(sm.dout[qb], 2048 * k, kTile);
+            const uint64_t bq = sdesc_mnmajor_sw128(sm.q[qb], 2048 * k, kTile);
+            const uint32_t lo_off = (k / 4) * kTile;
+            mma_bf16_ts(tm_dv, tm_p + 8 * k, bdo, id_a, i > 0 || k > 0);
+            mma_bf16_ss(tm_dv, sdesc_kmajor_sw128(sm.plo + lo_off, 32 * (k % 4)), bdo, id_a, true);
+            mma_bf16_ts(tm_dk, tm_ds + 8 * k, bq, id_a, i > 0 || k > 0);
+            mma_bf16_ss(tm_dk, sdesc_kmajor_sw128(sm.dslo + lo_off, 32 * (k % 4)), bq, id_a, true);
           }
           mma_commit(&sm.pds_empty);
           mma_commit(&sm.q_empty[qb]);
@@ -1193,7 +1203,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
       bool ok = true;
       for (int i = 0; i < nrt; ++i) {
         const int qb = q_count % 2;
-        if (!mbar_wait(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
         tc_fence_after();
         float sv[64], dp[64];
         tmem_ld32(tm_s + lane_off + r0, sv);
@@ -1206,9 +1216,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
         if (lane == 0) mbar_arrive(&sm.sdp_empty);
         ++sdp_count;
         // row scalars of this row tile arrived with q_full[qb] (already complete for the MMA)
-        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
         const int t_first = t_beg + (rt0 + i) * TPT;  // rows of tokens >= t_end contribute nothing
-        uint32_t pw[32], dsv[32];
+        // P^T w and dS^T as bf16 high + low parts: the sums over many rows of
+        // near-equal probabilities would otherwise carry the bf16 rounding of
+        // each term coherently (a 2^-9 relative bias)
+        uint32_t pw[32], dsv[32], pwl[32], dsl[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
           float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[qb][r0 + c]);
@@ -1221,17 +1234,24 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
           l4.w = vrow ? l4.w * kLog2e : CUDART_INF_F;
           const float p0 = ex2(sv[c] * qs2 - l4.x), p1 = ex2(sv[c + 1] * qs2 - l4.y);
           const float p2 = ex2(sv[c + 2] * qs2 - l4.z), p3 = ex2(sv[c + 3] * qs2 - l4.w);
-          pw[c / 2] = pack_bf16x2(p0 * w4.x, p1 * w4.y);
-          pw[c / 2 + 1] = pack_bf16x2(p2 * w4.z, p3 * w4.w);
-          dsv[c / 2] = pack_bf16x2(p0 * (w4.x * dp[c] - d4.x), p1 * (w4.y * dp[c + 1] - d4.y));
-          dsv[c / 2 + 1] = pack_bf16x2(p2 * (w4.z * dp[c + 2] - d4.z), p3 * (w4.w * dp[c + 3] - d4.w));
+          split_bf16x2(p0 * w4.x, p1 * w4.y, pw[c / 2], pwl[c / 2]);
+          split_bf16x2(p2 * w4.z, p3 * w4.w, pw[c / 2 + 1], pwl[c / 2 + 1]);
+          split_bf16x2(p0 * (w4.x * dp[c] - d4.x), p1 * (w4.y * dp[c + 1] - d4.y), dsv[c / 2], dsl[c / 2]);
+          split_bf16x2(p2 * (w4.z * dp[c + 2] - d4.z), p3 * (w4.w * dp[c + 3] - d4.w), dsv[c / 2 + 1],
+                       dsl[c / 2 + 1]);
         }
-        if (!mbar_wait(&sm.pds_empty, (pds_count & 1) ^ 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.pds_empty, (pds_count & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
         tmem_st16(tm_p + lane_off + 32 * wg, pw);
         tmem_st16(tm_p + lane_off + 32 * wg + 16, pw + 16);
         tmem_st16(tm_ds + lane_off + 32 * wg, dsv);
         tmem_st16(tm_ds + lane_off + 32 * wg + 16, dsv + 16);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          store_pt_chunk(sm.plo, b, 8 * wg + c, make_uint4(pwl[4 * c], pwl[4 * c + 1], pwl[4 * c + 2], pwl[4 * c + 3]));
+          store_pt_chunk(sm.dslo, b, 8 * wg + c, make_uint4(dsl[4 * c], dsl[4 * c + 1], dsl[4 * c + 2], dsl[4 * c + 3]));
+        }
+        fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -1243,7 +1263,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
         record_timeout(status, &sm.abort_flag);
         break;
       }
-      if (!mbar_wait(&sm.acc_full, acc_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      if (!mbar_wait_warp(&sm.acc_full, acc_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++acc_count;
       tc_fence_after();
       // warpgroup 0 adds dKc, warpgroup 1 adds dVc (lane = block)
@@ -1274,72 +1294,9 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2D map over [rows, 64] bf16 with a box of 128 rows, 128-byte swizzle.
-bool map_rows64(CUtensorMap* m, const void* base, int64_t rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {64, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 3D map over Q [N, Hq, 64] bf16 with a box of (64, G heads, 128/G tokens).
-bool map_q(CUtensorMap* m, const void* base, int64_t n, int hq, int G) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {64, (cuuint64_t)hq, (cuuint64_t)n};
-  cuuint64_t strides[2] = {128, (cuuint64_t)hq * 128};
-  cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(kRows / G)};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 2D map over per-row fp32 scalars [N, Hq] with a box of (G heads, 128/G tokens), no swizzle:
-// one box is the 128 row scalars of a row tile in row order.
-bool map_rowscalars(CUtensorMap* m, const float* base, int64_t n, int hq, int G) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)hq, (cuuint64_t)n};
-  cuuint64_t strides[1] = {(cuuint64_t)hq * 4};
-  cuuint32_t box[2] = {(cuuint32_t)G, (cuuint32_t)(kRows / G)};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 size_t smem_bytes_lse() { return sizeof(LseSmem) + 1024; }
 size_t smem_bytes_out() { return sizeof(OutSmem) + 1024; }
 
-int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 template <int G>
 cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st) {

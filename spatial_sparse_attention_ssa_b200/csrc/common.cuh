@@ -71,6 +71,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// (x0, x1) = hi + lo with hi the bf16 rounding and lo the bf16 rounding of the
+// remainder: hi + lo carries about 16 significant bits.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+}
+
 __device__ __forceinline__ void store32(__nv_bfloat16* p, const float* v) {
   uint4* p4 = reinterpret_cast<uint4*>(p);
 #pragma unroll

@@ -14,7 +14,7 @@ constexpr int kCmpRowChunk = 2048;
 constexpr int kCmpOutCtas = 160;
 
 struct FwdArgs {
-  int dtype, d, hq, hkv, topk, gate_mode;
+  int dtype, d, hq, hkv, topk, gate_mode, m_cmp, m_win;
   int use_tc;   // run the tensor-core kernels where they cover the shape
   int* status;  // device check word
   float scale;
@@ -34,10 +34,11 @@ struct FwdArgs {
   // workspace
   int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
   float* imp_scratch;  // [kCmpOutCtas, 128/G, B] selection scores (tensor-core path)
+  int32_t *win_cnt, *win_pre, *win_scan;  // [W + 1] window work plan
 };
 
 struct BwdArgs {
-  int dtype, d, hq, hkv, topk, gate_mode;
+  int dtype, d, hq, hkv, topk, gate_mode, m_cmp, m_win;
   int use_tc;
   int* status;
   float scale;
@@ -57,6 +58,8 @@ struct BwdArgs {
   // workspace
   float* Dc;          // [3, N, Hq]
   float* wcmp;        // [N, Hq] gate weights of the compressed branch
+  float* wwin;        // [N, Hq] gate weights of the window branch
+  int32_t *win_cnt, *win_pre;  // [W + 1] window work plan
   float *dkc, *dvc;   // [Hkv, B, d]
   uint64_t *inv_keys_a, *inv_keys_b;
   int32_t *inv_vals_a, *inv_vals_b;
@@ -74,6 +77,9 @@ cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st);
 bool cmp_tc_supported(int dtype, int d, int hq, int hkv, int topk);
 size_t cmp_tc_scratch_floats(int hq, int hkv, int64_t btot);
 cudaError_t cmp_fwd_tc(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st);
+bool win_tc_supported(int dtype, int d, int hq, int hkv, int m_cmp, int m_win);
+cudaError_t win_fwd_tc(const FwdArgs& a, int32_t* cnt, int32_t* pre, int32_t* scan_tmp, cudaStream_t st);
+cudaError_t win_bwd_tc(const BwdArgs& a, int32_t* cnt, int32_t* pre, int32_t* scan_tmp, cudaStream_t st);
 cudaError_t cmp_bwd_tc(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, int32_t* dkv_pre, int32_t* scan_tmp,
                        int64_t tiles_bound, cudaStream_t st);
 cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st);

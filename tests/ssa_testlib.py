@@ -60,6 +60,8 @@ class GpuRun:
             self.grads = ssa.ssa_backward(self.p, self.cu, self.blk, self.win, self.q, self.k, self.v,
                                           self.gates, self.saved, self.dout)
         torch.cuda.synchronize()
+        status = ssa.device_status()
+        assert status == 0, "device check word: %s" % ssa.STATUS_NAMES.get(status, status)
         return self
 
 

@@ -32,6 +32,23 @@ def test_small_shell_backward_parity(kw):
     print(w.n, errs)
 
 
+@pytest.mark.parametrize("kw", [
+    # 16 heads per KV head, windows and blocks of 16^3 voxels: windows of more than
+    # 128 tokens span several key tiles of the tensor-core kernels
+    dict(hq=32, hkv=2, d=64, m_cmp=16, m_win=16, topk=4, dtype="bf16", gate_mode=1),
+    dict(hq=16, hkv=2, d=64, m_cmp=16, m_win=16, topk=4, dtype="bf16", gate_mode=1),
+    dict(hq=32, hkv=2, d=64, m_cmp=4, m_win=4, topk=8, dtype="bf16", gate_mode=1),
+])
+def test_large_windows_and_16_head_groups(kw):
+    w = W.small_shell(seed=21, R=40, n_prims=2, lo=6.0, hi=12.0, n_keep=None, **kw)
+    t = W.make_tensors(w)
+    sizes = np.bincount(O.bin_tokens(w.coords, w.cu_seqlens, w.m_win)["id"])
+    if w.m_win == 16:
+        assert sizes.max() > 128  # the case these shapes are for
+    _, _, _, errs = _bwd_parity(w, t)
+    print(w.n, sizes.max(), errs)
+
+
 def test_zero_gates_give_zero_input_gradients():
     w = W.small_shell(seed=12, R=32, n_prims=2, lo=4.0, hi=9.0, n_keep=600, gate_mode=0)
     t = W.make_tensors(w)
