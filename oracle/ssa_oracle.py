@@ -416,3 +416,47 @@ def dq_rows(st: State, dout: np.ndarray, tokens) -> np.ndarray:
                 ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
                 out[i, hs, :] += scale * (ds @ kk)
     return out
+
+
+def dgates_rows(st: State, dout: np.ndarray, tokens) -> np.ndarray:
+    """dgates of the given tokens only ([len(tokens), Hq, 3]); needs the forward
+    rows of those tokens.  Same arithmetic as `backward`."""
+    tokens = np.asarray(tokens)
+    o = st["o"][:, tokens]
+    do = np.asarray(dout[tokens], np.float64)
+    dots = np.einsum("nhd,cnhd->nhc", do, o)
+    if st["gate_mode"] == 0:
+        return dots
+    gw = gate_weights(st["gates"][tokens], st["gate_mode"])
+    return dots * gw * (1.0 - gw)
+
+
+def window_kv_grads(st: State, dout: np.ndarray, windows) -> tuple:
+    """Window-branch dK, dV of every token of the given windows: (tokens,
+    dk [len, Hkv, d], dv [len, Hkv, d]).  A key's window gradient comes only from
+    the queries of its own window, so a forward restricted to those windows'
+    tokens suffices.  Same arithmetic as `backward`."""
+    q, k, v = st["q"], st["k"], st["v"]
+    hkv, G, scale = st["hkv"], st["G"], st["scale"]
+    win = st["win"]
+    gw = gate_weights(st["gates"], st["gate_mode"])
+    toks, dks, dvs = [], [], []
+    for w in windows:
+        jw = win["perm"][win["ptr"][w]:win["ptr"][w + 1]]
+        dk = np.zeros((len(jw), hkv, k.shape[2]))
+        dv = np.zeros_like(dk)
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            kk, vv = k[jw, g, :], v[jw, g, :]
+            for t in jw:
+                qr = np.asarray(q[t, hs, :], np.float64)
+                dor = np.asarray(dout[t, hs, :], np.float64) * gw[t, hs, 2][:, None]
+                p = np.exp(scale * (qr @ kk.T) - st["lse"][2, t, hs][:, None])
+                dp = dor @ vv.T
+                ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+                dk[:, g, :] += scale * (ds.T @ qr)
+                dv[:, g, :] += p.T @ dor
+        toks.append(jw)
+        dks.append(dk)
+        dvs.append(dv)
+    return np.concatenate(toks), np.concatenate(dks), np.concatenate(dvs)

@@ -1,0 +1,113 @@
+"""Parity at the full benchmark sizes, on outputs the oracle can compute one by one.
+
+Each test runs the whole path through the C ABI at the configuration's real size
+(the launch configuration the bench times for config 5) and checks:
+  * Kc / Vc of every block bit-exact, and the id arrays bit-exact (test_gpu_bin);
+  * for sampled query tokens: selection (near-tie rule), the three branch outputs,
+    their lse and the combined output; in backward, dQ and dgates of those rows;
+  * window-branch dK / dV of sampled windows (window gates one-hot, so the other
+    branches contribute exactly zero to dK / dV);
+  * properties that hold at any size: sum_i dV_i = sum over rows of (sum_c w_c) dO
+    and sum_i dK_i = 0 per KV head.
+"""
+import dataclasses
+import functools
+
+import numpy as np
+import pytest
+
+from oracle import ssa_oracle as O
+from spatial_sparse_attention_ssa_b200 import workloads as W
+from tests.ssa_testlib import ATOL, GpuRun, compare_forward, f64, max_abs, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@functools.lru_cache(maxsize=2)
+def _load(cfg: int):
+    """Workload and tensors of a configuration, generated once per module.
+    Configs 3 and 5 share geometry, heads and seeded tensors (5 adds dO, which
+    make_tensors always draws), so 3 reuses 5's."""
+    if cfg == 3:
+        return _load(5)
+    w = W.config(cfg)
+    return w, W.make_tensors(w)
+
+
+def _sample_tokens(w, n_per_seq: int, seed: int) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    out = []
+    for s in range(w.s):
+        a, b = int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1])
+        if b <= a:
+            continue
+        pick = rng.choice(np.arange(a, b), size=min(n_per_seq, b - a), replace=False)
+        out.append(np.concatenate([[a, b - 1], pick]))
+    return np.unique(np.concatenate(out))
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_forward_sampled_rows_at_full_size(cfg):
+    w, t = _load(cfg)
+    run = GpuRun(w, t, backward=False).run(backward=False)
+    toks = _sample_tokens(w, 48 if w.s == 1 else 16, seed=cfg)
+    st = run_oracle(w, t, tokens=toks)
+    errs, flips = compare_forward(run, st, toks, ATOL[w.dtype])
+    print(cfg, w.n, len(toks), errs, "flips", len(flips))
+
+
+def test_backward_sampled_rows_and_sums_at_full_size():
+    w, t = _load(5)
+    run = GpuRun(w, t).run()
+    toks = _sample_tokens(w, 32, seed=55)
+    st = run_oracle(w, t, tokens=toks)
+    _, flips = compare_forward(run, st, toks, ATOL[w.dtype])
+    flipped = {tt for tt, _ in flips}
+    keep = np.array([tt for tt in toks if tt not in flipped])
+    do = t.as_f32("do").astype(np.float64)
+    dq, dk, dv, dg = (f64(x) for x in run.grads)
+    e_dq = max_abs(dq[keep], O.dq_rows(st, do, keep))
+    e_dg = max_abs(dg[keep], O.dgates_rows(st, do, keep))
+    assert e_dq <= ATOL[w.dtype] and e_dg <= ATOL[w.dtype], (e_dq, e_dg)
+
+    # sums over all tokens.  Softmax rows sum to one in every branch, so
+    # sum_i dV_i = sum_rows (sum_c w_c) dO and sum_i dK_i = 0 (the compressed
+    # branch included: sum_i dKc_b(i)/n_b = sum_b dKc_b).  The GPU multiplies
+    # bf16-rounded P and dS in some tiles; each term then carries a relative
+    # error below 2^-9 with independent signs, and sum_j p_j^2 <= 1 per row, so
+    # 4 sigma of the rounding noise is below 4 * 2^-9 / sqrt(3) * sqrt(sum_rows
+    # |w dO|^2) for dV; dK gets the same bound in terms of its own rows.
+    gw = O.gate_weights(t.gates, w.gate_mode)
+    G = w.hq // w.hkv
+    for g in range(w.hkv):
+        hs = slice(g * G, (g + 1) * G)
+        wsum = gw[:, hs, :].sum(-1)
+        want = np.einsum("nh,nhd->d", wsum, do[:, hs, :])
+        noise = np.sqrt(np.einsum("nh,nhd->d", wsum ** 2, do[:, hs, :] ** 2))
+        tol_v = 2e-2 + 4 * 2.0 ** -9 / np.sqrt(3) * noise
+        assert (np.abs(dv[:, g, :].sum(0) - want) <= tol_v).all(), (g, np.abs(dv[:, g, :].sum(0) - want).max())
+        tol_k = 2e-2 + 4 * 2.0 ** -9 / np.sqrt(3) * np.sqrt((dk[:, g, :] ** 2).sum(0))
+        assert (np.abs(dk[:, g, :].sum(0)) <= tol_k).all(), (g, np.abs(dk[:, g, :].sum(0)).max())
+
+
+def test_window_gradients_of_sampled_windows_at_full_size():
+    w, t = _load(5)
+    w = dataclasses.replace(w, gate_mode=0)
+    gates = np.zeros_like(t.gates)
+    gates[:, :, 2] = 1.0  # window branch only: the other branches add exact zeros to dK / dV
+    t = dataclasses.replace(t, gates=gates)
+    run = GpuRun(w, t).run()
+    wb = O.bin_tokens(w.coords, w.cu_seqlens, w.m_win)
+    sizes = np.diff(wb["ptr"])
+    rng = np.random.default_rng(7)
+    wins = np.unique(np.concatenate([np.argsort(-sizes, kind="stable")[:4], rng.choice(len(sizes), 12, replace=False)]))
+    members = np.concatenate([wb["perm"][wb["ptr"][x]:wb["ptr"][x + 1]] for x in wins])
+    st = run_oracle(w, t, tokens=np.unique(members))
+    do = t.as_f32("do").astype(np.float64)
+    tk, dk_ref, dv_ref = O.window_kv_grads(st, do, wins)
+    dq, dk, dv, _ = (f64(x) for x in run.grads)
+    e = {"dk": max_abs(dk[tk], dk_ref), "dv": max_abs(dv[tk], dv_ref),
+         "dq": max_abs(dq[tk], O.dq_rows(st, do, tk))}
+    print(len(wins), sizes[wins].max(), e)
+    for key, val in e.items():
+        assert val <= ATOL[w.dtype], (key, val)

@@ -458,3 +458,21 @@ def test_dq_rows_matches_full_backward():
     toks = np.array([0, 3, w.n - 1, int(w.cu_seqlens[1])])
     st2 = _run(w, t, tokens=toks)
     np.testing.assert_allclose(O.dq_rows(st2, do, toks), g["dq"][toks], rtol=1e-10, atol=1e-12)
+
+
+def test_dgates_rows_and_window_grads_match_full_backward():
+    """The row- and window-restricted gradients used by the full-size GPU tests
+    equal the full backward (itself pinned by autograd and central differences)."""
+    w, t = _small_workload(seed=7, n_seqs=2)
+    st = _run(w, t)
+    do = t.as_f32("do").astype(np.float64)
+    g = O.backward(st, do)
+    wins = np.array([0, 3, st["win"]["count"] - 1])
+    members = np.concatenate([st["win"]["perm"][st["win"]["ptr"][x]:st["win"]["ptr"][x + 1]] for x in wins])
+    toks = np.unique(np.concatenate([members, [0, w.n - 1]]))
+    st2 = _run(w, t, tokens=toks)
+    np.testing.assert_allclose(O.dgates_rows(st2, do, toks), g["dgates"][toks], rtol=1e-12, atol=1e-14)
+    tk, dk, dv = O.window_kv_grads(st2, do, wins)
+    np.testing.assert_array_equal(np.sort(tk), np.sort(members))
+    np.testing.assert_allclose(dk, g["parts"]["dk"]["win"][tk], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, g["parts"]["dv"]["win"][tk], rtol=1e-10, atol=1e-12)
