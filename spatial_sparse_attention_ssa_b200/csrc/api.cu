@@ -95,11 +95,10 @@ size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W
 
 struct BwdWs {
   float* Dc;
-  float* wcmp;
+  float* rc;
   float *dkc, *dvc;
   uint64_t *ka, *kb;
   int32_t *va, *vb, *inv_ptr, *radix_tmp, *slc_cnt, *slc_pre, *win_cnt, *win_pre;
-  float* wwin;
   int32_t *tc, *tp, *ic, *ip, *st;
 };
 
@@ -107,7 +106,7 @@ size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t 
   Carver c(base);
   const int64_t nsel = N * p->hkv * p->topk;
   w->Dc = c.take<float>(3 * N * p->hq);
-  w->wcmp = c.take<float>(N * p->hq);
+  w->rc = c.take<float>(6 * N * p->hq);
   w->dkc = c.take<float>(p->hkv * B * p->d);
   w->dvc = c.take<float>(p->hkv * B * p->d);
   w->ka = c.take<uint64_t>(nsel);
@@ -118,7 +117,6 @@ size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t 
   w->radix_tmp = c.take<int32_t>(ssa::radix_tmp_ints(nsel));
   w->slc_cnt = c.take<int32_t>(p->hkv * B + 1);
   w->slc_pre = c.take<int32_t>(p->hkv * B + 1);
-  w->wwin = c.take<float>(N * p->hq);
   w->win_cnt = c.take<int32_t>(W + 1);
   w->win_pre = c.take<int32_t>(W + 1);
   int64_t mx = p->hkv * B + 1 > S + 1 ? p->hkv * B + 1 : S + 1;
@@ -338,8 +336,7 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.dv = dv;
   a.dgates = dgates;
   a.Dc = w.Dc;
-  a.wcmp = w.wcmp;
-  a.wwin = w.wwin;
+  a.rc = w.rc;
   a.win_cnt = w.win_cnt;
   a.win_pre = w.win_pre;
   a.dkc = w.dkc;

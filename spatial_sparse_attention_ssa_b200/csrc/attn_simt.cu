@@ -420,10 +420,12 @@ __global__ void combine_kernel(const float* __restrict__ ob, const float* __rest
 // ---------------------------------------------------------------------------
 // backward: per-row dot products <dO, o_c>, the softmax correction D_c and dgates
 // ---------------------------------------------------------------------------
+// Also writes the per-row constants of the tensor-core kernels (rc, [2][3][rows]):
+// for the compressed (c = 0) and window (c = 2) branches, -lse * log2(e), w and -D.
 template <typename T, int D>
 __global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict__ dout, const float* __restrict__ gates,
-                               int64_t rows, int mode, float* __restrict__ Dc, float* __restrict__ dgates,
-                               float* __restrict__ wcmp, float* __restrict__ wwin) {
+                               const float* __restrict__ lse, int64_t rows, int mode, float* __restrict__ Dc,
+                               float* __restrict__ dgates, float* __restrict__ rc) {
   constexpr int NT = D / 32;
   const int64_t total = rows * NT;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -443,8 +445,12 @@ __global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict
         const float w = gate_weight(gates, row * 3 + c, mode);
         Dc[(int64_t)c * rows + row] = w * dot;
         dgates[row * 3 + c] = mode == SSA_GATE_LOGITS ? dot * w * (1.f - w) : dot;
-        if (c == 0) wcmp[row] = w;
-        if (c == 2) wwin[row] = w;
+        if (c != 1) {
+          float* r = rc + (c == 0 ? 0 : 3 * rows);
+          r[row] = -lse[(int64_t)c * rows + row] * kLog2e;
+          r[rows + row] = w;
+          r[2 * rows + row] = -(w * dot);
+        }
       }
     }
   }
@@ -1206,8 +1212,8 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   e = exclusive_scan(a.items_cnt, a.items_pre, a.S + 1, a.scan_tmp, st);
   if (e != cudaSuccess) return e;
 
-  SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout, a.gates, rows, a.gate_mode,
-                                                                             a.Dc, a.dgates, a.wcmp, a.wwin);
+  SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout, a.gates, a.lse, rows, a.gate_mode,
+                                                                             a.Dc, a.dgates, a.rc);
   if (a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
     // 128-row tiles for the tensor-core kernels (tiles_cnt / tiles_pre are free again here)
     SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu,

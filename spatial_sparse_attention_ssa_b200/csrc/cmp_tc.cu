@@ -212,17 +212,19 @@ __global__ void __launch_bounds__(kThreads, 1) cmp_lse_tc_kernel(
         if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
         ++s_count;
         const int vc = min(kBN, ti.nb - j * kBN);
-        float cm = -CUDART_INF_F;
+        if (vc < kBN) {  // ragged last key tile
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          sv[c] = c < vc ? sv[c] * qs2 : -CUDART_INF_F;
-          cm = fmaxf(cm, sv[c]);
+          for (int c = 0; c < kBN; ++c) sv[c] = c < vc ? sv[c] : -CUDART_INF_F;
         }
-        const float mn = fmaxf(m, cm);
-        float acc = 0.f;
+        float cm = sv[0];
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) acc += ex2(sv[c] - mn);
-        l = l * ex2(m - mn) + acc;
+        for (int c = 1; c < kBN; ++c) cm = fmaxf(cm, sv[c]);
+        const float mn = fmaxf(m, cm * qs2);  // qs2 > 0
+        const float2 qs = make_float2(qs2, qs2), nm = make_float2(-mn, -mn);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kBN; c += 2) acc = fadd2(acc, ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nm)));
+        l = l * ex2(m - mn) + (acc.x + acc.y);
         m = mn;
       }
       if (!ok) break;
@@ -665,7 +667,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
       if (wg == 0) {
         const int r = threadIdx.x;
         const int64_t t = min((int64_t)ti.t0 + r / G, (int64_t)ti.t_end - 1);
-        sm.lse2[r] = lse_in[t * hq + ti.g * G + r % G] * kLog2e;
+        sm.lse2[r] = -lse_in[t * hq + ti.g * G + r % G] * kLog2e;  // -lse log2(e)
       }
       if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
       const int nbt = (ti.nb + kBN - 1) / kBN;
@@ -684,26 +686,27 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
         ++s_count;
         const int bidx = j * kBN + b;  // block index inside the sequence
         const bool bvalid = bidx < ti.nb;
+        if (!bvalid) {  // ragged last key tile: blocks past the sequence get p = 0
+#pragma unroll
+          for (int r = 0; r < 64; ++r) p[r] = -CUDART_INF_F;
+        }
+        const float2 qs = make_float2(qs2, qs2);
 #pragma unroll
         for (int r = 0; r < 64; r += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[r0 + r]);
-          p[r + 0] = bvalid ? ex2(p[r + 0] * qs2 - l4.x) : 0.f;
-          p[r + 1] = bvalid ? ex2(p[r + 1] * qs2 - l4.y) : 0.f;
-          p[r + 2] = bvalid ? ex2(p[r + 2] * qs2 - l4.z) : 0.f;
-          p[r + 3] = bvalid ? ex2(p[r + 3] * qs2 - l4.w) : 0.f;
+          const float2 pa = ex2x2(ffma2(make_float2(p[r], p[r + 1]), qs, make_float2(l4.x, l4.y)));
+          const float2 pb = ex2x2(ffma2(make_float2(p[r + 2], p[r + 3]), qs, make_float2(l4.z, l4.w)));
+          p[r] = pa.x;
+          p[r + 1] = pa.y;
+          p[r + 2] = pb.x;
+          p[r + 3] = pb.y;
         }
         if (!mbar_wait_warp(&sm.pt_empty, (pt_count & 1) ^ 1)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = p[8 * c + 2 * e], x1 = p[8 * c + 2 * e + 1];
-            const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-            const float2 hf = __bfloat1622float2(h);
-            hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-            lo[e] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
-          }
+          for (int e = 0; e < 4; ++e) split2(make_float2(p[8 * c + 2 * e], p[8 * c + 2 * e + 1]), hi[e], lo[e]);
           store_pt_chunk(sm.pt_hi, b, 8 * wg + c, make_uint4(hi[0], hi[1], hi[2], hi[3]));
           store_pt_chunk(sm.pt_lo, b, 8 * wg + c, make_uint4(lo[0], lo[1], lo[2], lo[3]));
         }
@@ -716,10 +719,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
         if (bvalid) {
 #pragma unroll
           for (int tl = 0; tl < 64 / G; ++tl) {
-            float imp = 0.f;
+            float2 acc = make_float2(p[tl * G], p[tl * G + 1]);
 #pragma unroll
-            for (int hh = 0; hh < G; ++hh) imp += p[tl * G + hh];
-            imp_base[(int64_t)(wg * (64 / G) + tl) * imp_stride + bidx] = imp;
+            for (int hh = 2; hh < G; hh += 2) acc = fadd2(acc, make_float2(p[tl * G + hh], p[tl * G + hh + 1]));
+            imp_base[(int64_t)(wg * (64 / G) + tl) * imp_stride + bidx] = acc.x + acc.y;
           }
         }
       }
@@ -775,6 +778,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
 // in registers; dQ += dS Kc with dS (bf16 hi + lo) as the TMEM A operand.
 // ---------------------------------------------------------------------------
 constexpr int kBwdStages = 3;
+// four compute warpgroups, each owning 32 of a key tile's 128 blocks: twice the
+// warps of a two-warpgroup split, to hide the latency of TMEM loads and MUFU
+constexpr int kDqWarpgroups = 4;
+constexpr int kDqComputeWarps = 4 * kDqWarpgroups;
+constexpr int kDqThreads = 32 * (kDqComputeWarps + 2);  // + TMA warp + MMA warp
+constexpr int kDqCols = kBN / kDqWarpgroups;
 
 struct DqSmem {
   uint8_t q[2][kTile];
@@ -788,12 +797,12 @@ struct DqSmem {
 };
 
 template <int G>
-__global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
+__global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
     const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
     const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S, int hq,
-    int hkv, int btot, float qs2, float scale, const float* __restrict__ lse_in, const float* __restrict__ Dc,
-    const float* __restrict__ gates, int gate_mode, float* __restrict__ dq_out, int* status) {
+    int hkv, int btot, float qs2, float scale, const float* __restrict__ rc, int64_t rows,
+    float* __restrict__ dq_out, int* status) {
   extern __shared__ uint8_t smem_raw[];
   DqSmem& sm = *reinterpret_cast<DqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -809,11 +818,11 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
       mbar_init(&sm.kv_empty[i], 1);
     }
     mbar_init(&sm.sdp_full, 1);
-    mbar_init(&sm.sdp_empty, kComputeWarps);
-    mbar_init(&sm.ds_full, kComputeWarps);
+    mbar_init(&sm.sdp_empty, kDqComputeWarps);
+    mbar_init(&sm.ds_full, kDqComputeWarps);
     mbar_init(&sm.ds_empty, 1);
     mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_empty, kComputeWarps);
+    mbar_init(&sm.dq_empty, kDqComputeWarps);
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -829,7 +838,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
   // TMEM columns: S [0,128), dP [128,256), dS hi [256,320), dS lo [320,384), dQ [384,448)
   const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dsh = tmem + 256, tm_dsl = tmem + 320, tm_dq = tmem + 384;
 
-  if (warp == kComputeWarps) {
+  if (warp == kDqComputeWarps) {
     // ---------------- TMA producer: (Q, dO) per row tile; (Kc, Vc) per key tile
     if (lane == 0) {
       uint32_t kv_count = 0, q_count = 0;
@@ -859,7 +868,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
       for (int i = 0; i < kBwdStages; ++i)
         if (last_par[i] >= 0) mbar_wait(&sm.kv_full[i], (uint32_t)last_par[i]);
     }
-  } else if (warp == kComputeWarps + 1) {
+  } else if (warp == kDqComputeWarps + 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(kRows, kBN);              // S, dP [rows, blocks]
@@ -918,9 +927,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
       mbar_wait(&sm.mma_done, 0);
     }
   } else {
-    // ---------------- compute warps: thread = row; warpgroup wg owns blocks [64 wg, 64 wg + 64) of a key tile
+    // ---------------- compute warps: thread = row; warpgroup wg owns blocks [32 wg, 32 wg + 32) of a key tile
     const int r = threadIdx.x % 128;
     const int wg = warp / 4;
+    const int c0 = kDqCols * wg;
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
     uint32_t sdp_count = 0, ds_count = 0, dq_count = 0;
     for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
@@ -928,43 +938,41 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
       const int64_t t = ti.t0 + r / G;
       const bool valid = t < ti.t_end;
       const int64_t row = min(t, (int64_t)ti.t_end - 1) * hq + ti.g * G + r % G;
-      const float lse2 = lse_in[row] * kLog2e;
-      const float Dr = Dc[row];
-      const float gx = gates[row * 3 + 0];
-      const float wr = gate_mode == SSA_GATE_LOGITS ? 1.f / (1.f + expf(-gx)) : gx;
+      // row constants: -lse log2(e), w, -D
+      const float2 nl2 = make_float2(rc[row], rc[row]);
+      const float2 w2 = make_float2(rc[rows + row], rc[rows + row]);
+      const float2 nd2 = make_float2(rc[2 * rows + row], rc[2 * rows + row]);
+      const float2 qs = make_float2(qs2, qs2);
       const int nbt = (ti.nb + kBN - 1) / kBN;
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
         if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
         tc_fence_after();
-        float sv[64], dp[64];
-        tmem_ld32(tm_s + lane_off + 64 * wg, sv);
-        tmem_ld32(tm_s + lane_off + 64 * wg + 32, sv + 32);
-        tmem_ld32(tm_dp + lane_off + 64 * wg, dp);
-        tmem_ld32(tm_dp + lane_off + 64 * wg + 32, dp + 32);
+        float sv[kDqCols], dp[kDqCols];
+        tmem_ld32(tm_s + lane_off + c0, sv);
+        tmem_ld32(tm_dp + lane_off + c0, dp);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.sdp_empty);
         ++sdp_count;
-        const int nvalid = ti.nb - (j * kBN + 64 * wg);  // valid blocks of this warpgroup's half
-        uint32_t hi[32], lo[32];
+        const int nvalid = ti.nb - (j * kBN + c0);  // valid blocks of this warpgroup's columns
+        if (nvalid < kDqCols) {  // ragged last key tile: blocks past the sequence get p = 0
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float d0 = 0.f, d1 = 0.f;
-          if (c < nvalid) d0 = ex2(sv[c] * qs2 - lse2) * (wr * dp[c] - Dr);
-          if (c + 1 < nvalid) d1 = ex2(sv[c + 1] * qs2 - lse2) * (wr * dp[c + 1] - Dr);
-          const __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
-          const float2 hf = __bfloat1622float2(h);
-          hi[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[c / 2] = pack_bf16x2(d0 - hf.x, d1 - hf.y);
+          for (int c = 0; c < kDqCols; ++c) sv[c] = c < nvalid ? sv[c] : -CUDART_INF_F;
+        }
+        // dS = p (w dP - D), p = 2^(s qs2 - lse log2 e)
+        uint32_t hi[kDqCols / 2], lo[kDqCols / 2];
+#pragma unroll
+        for (int c = 0; c < kDqCols; c += 2) {
+          const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
+          const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
+          split2(d, hi[c / 2], lo[c / 2]);
         }
         if (!mbar_wait_warp(&sm.ds_empty, (ds_count & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        tmem_st16(tm_dsh + lane_off + 32 * wg, hi);
-        tmem_st16(tm_dsh + lane_off + 32 * wg + 16, hi + 16);
-        tmem_st16(tm_dsl + lane_off + 32 * wg, lo);
-        tmem_st16(tm_dsl + lane_off + 32 * wg + 16, lo + 16);
+        tmem_st16(tm_dsh + lane_off + c0 / 2, hi);
+        tmem_st16(tm_dsl + lane_off + c0 / 2, lo);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -978,18 +986,18 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
       if (!mbar_wait_warp(&sm.dq_full, dq_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++dq_count;
       tc_fence_after();
-      float g32[32];
-      tmem_ld32(tm_dq + lane_off + 32 * wg, g32);
+      float g16[16];  // warpgroup wg writes dQ columns [16 wg, 16 wg + 16)
+      tmem_ld16(tm_dq + lane_off + 16 * wg, g16);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.dq_empty);
       if (valid) {
-        float4* dst = reinterpret_cast<float4*>(dq_out + row * 64 + 32 * wg);
+        float4* dst = reinterpret_cast<float4*>(dq_out + row * 64 + 16 * wg);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(g32[4 * i] * scale, g32[4 * i + 1] * scale, g32[4 * i + 2] * scale,
-                               g32[4 * i + 3] * scale);
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_float4(g16[4 * i] * scale, g16[4 * i + 1] * scale, g16[4 * i + 2] * scale,
+                               g16[4 * i + 3] * scale);
       }
     }
   }
@@ -1005,27 +1013,33 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dq_tc_kernel(
 // partial dKc / dVc are added to the fp32 workspace with vector atomics.
 // ---------------------------------------------------------------------------
 constexpr int kDkvRowTilesPerItem = 128;
+constexpr int kDkvQStages = 3;  // Q / dO / row-constant stages: each row tile is used once per item
+// four compute warpgroups of 32 rows each (thread = block): enough warps to hide
+// the latency of the per-score arithmetic
+constexpr int kDkvComputeWarps = 16;
+constexpr int kDkvThreads = 32 * (kDkvComputeWarps + 2);
 
 struct DkvSmem {
   uint8_t kc[kTile];
   uint8_t vc[kTile];
-  uint8_t q[2][kTile];
-  uint8_t dout[2][kTile];
+  uint8_t q[kDkvQStages][kTile];
+  uint8_t dout[kDkvQStages][kTile];
   // low bf16 parts of P^T w and dS^T [blocks, 128 rows] (K-major A operands, two
   // 64-row atoms each); the high parts are TMEM operands
   uint8_t plo[2 * kTile];
   uint8_t dslo[2 * kTile];
-  __align__(128) float lse2[2][kRows];  // TMA destinations: 128-byte aligned
-  __align__(128) float Dr[2][kRows];
-  __align__(128) float wr[2][kRows];
-  uint64_t kv_full, kv_empty, q_full[2], q_empty[2];
+  // row constants, TMA destinations (128-byte aligned): -lse log2(e), -D, w
+  __align__(128) float lse2[kDkvQStages][kRows];
+  __align__(128) float Dr[kDkvQStages][kRows];
+  __align__(128) float wr[kDkvQStages][kRows];
+  uint64_t kv_full, kv_empty, q_full[kDkvQStages], q_empty[kDkvQStages];
   uint64_t sdp_full, sdp_empty, pds_full, pds_empty, acc_full, acc_empty, mma_done;
   uint32_t tmem;
   int abort_flag;
 };
 
 template <int G>
-__global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
+__global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
     const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
     const __grid_constant__ CUtensorMap lsemap, const __grid_constant__ CUtensorMap dcmap,
@@ -1058,16 +1072,16 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
   if (threadIdx.x == 0) {
     mbar_init(&sm.kv_full, 1);
     mbar_init(&sm.kv_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kDkvQStages; ++i) {
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
     }
     mbar_init(&sm.sdp_full, 1);
-    mbar_init(&sm.sdp_empty, kComputeWarps);
-    mbar_init(&sm.pds_full, kComputeWarps);
+    mbar_init(&sm.sdp_empty, kDkvComputeWarps);
+    mbar_init(&sm.pds_full, kDkvComputeWarps);
     mbar_init(&sm.pds_empty, 1);
     mbar_init(&sm.acc_full, 1);
-    mbar_init(&sm.acc_empty, kComputeWarps);
+    mbar_init(&sm.acc_empty, kDkvComputeWarps);
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -1084,7 +1098,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
   const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_p = tmem + 256, tm_ds = tmem + 320, tm_dk = tmem + 384,
                  tm_dv = tmem + 448;
 
-  if (warp == kComputeWarps) {
+  if (warp == kDkvComputeWarps) {
     // ---------------- producer warp: (Kc, Vc) per item; (Q, dO) + row scalars per row tile
     uint32_t kv_count = 0, q_count = 0;
     bool kv_issued = false;
@@ -1108,9 +1122,9 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
       if (!okk) { record_timeout(status, &sm.abort_flag); break; }
       ++kv_count;
       for (int rt = rt0; rt < rt1; ++rt) {
-        const int qb = q_count % 2;
+        const int qb = q_count % kDkvQStages;
         bool okw = true;
-        if (lane == 0) okw = mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1);
+        if (lane == 0) okw = mbar_wait(&sm.q_empty[qb], ((q_count / kDkvQStages) & 1) ^ 1);
         okw = __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
         if (!okw) { record_timeout(status, &sm.abort_flag); break; }
         const int t0 = t_beg + rt * TPT;
@@ -1128,7 +1142,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
     }
     if (lane == 0 && kv_issued) mbar_wait(&sm.kv_full, kv_last_par);
     (void)kv_last_par;
-  } else if (warp == kComputeWarps + 1) {
+  } else if (warp == kDkvComputeWarps + 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(kBN, kRows);              // S^T, dP^T [blocks, rows]
@@ -1141,10 +1155,8 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
         if (!mbar_wait(&sm.kv_full, kv_count & 1)) { ok = false; break; }
         ++kv_count;
         const int nrt = rt1 - rt0;
-        auto issue_sdp = [&](uint32_t qi) -> bool {
-          const int qb = qi % 2;
-          if (!mbar_wait(&sm.q_full[qb], (qi / 2) & 1) || !mbar_wait(&sm.sdp_empty, (sdp_count & 1) ^ 1))
-            return false;
+        auto issue_sdp_now = [&](uint32_t qi) {
+          const int qb = qi % kDkvQStages;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -1154,15 +1166,42 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
           }
           mma_commit(&sm.sdp_full);
           ++sdp_count;
+        };
+        // S^T / dP^T of row tile qi may go once its Q / dO tiles landed and the
+        // compute warps released the previous S^T / dP^T
+        auto sdp_ready = [&](uint32_t qi) -> bool {
+          return mbar_test(&sm.q_full[qi % kDkvQStages], (qi / kDkvQStages) & 1) &&
+                 mbar_test(&sm.sdp_empty, (sdp_count & 1) ^ 1);
+        };
+        auto issue_sdp = [&](uint32_t qi) -> bool {
+          if (!mbar_wait(&sm.q_full[qi % kDkvQStages], (qi / kDkvQStages) & 1) ||
+              !mbar_wait(&sm.sdp_empty, (sdp_count & 1) ^ 1))
+            return false;
+          issue_sdp_now(qi);
           return true;
         };
         if (nrt > 0 && !issue_sdp(q_count)) { ok = false; break; }
         for (int i = 0; i < nrt; ++i) {
-          const int qb = q_count % 2;
-          if (i + 1 < nrt && !issue_sdp(q_count + 1)) { ok = false; break; }
-          if ((i == 0 && !mbar_wait(&sm.acc_empty, (acc_count & 1) ^ 1)) || !mbar_wait(&sm.pds_full, pds_count & 1)) {
-            ok = false;
-            break;
+          const int qb = q_count % kDkvQStages;
+          bool next_pending = i + 1 < nrt;
+          if (i == 0 && !mbar_wait(&sm.acc_empty, (acc_count & 1) ^ 1)) { ok = false; break; }
+          // wait for P^T w / dS^T of this tile; the next tile's S^T / dP^T goes out as
+          // soon as it can, so that the tensor pipe works while the compute warps do
+          {
+            bool got = false;
+            const uint64_t t0 = global_ns();
+            for (uint32_t spin = 1;; ++spin) {
+              if (next_pending && sdp_ready(q_count + 1)) {
+                issue_sdp_now(q_count + 1);
+                next_pending = false;
+              }
+              if (mbar_test(&sm.pds_full, pds_count & 1)) {
+                got = true;
+                break;
+              }
+              if ((spin & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) break;
+            }
+            if (!got) { ok = false; break; }
           }
           tc_fence_after();
 #pragma unroll
@@ -1179,6 +1218,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
           mma_commit(&sm.q_empty[qb]);
           ++pds_count;
           ++q_count;
+          if (next_pending && !issue_sdp(q_count)) { ok = false; break; }
         }
         if (!ok) break;
         mma_commit(&sm.kv_empty);
@@ -1190,10 +1230,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
       mbar_wait(&sm.mma_done, 0);
     }
   } else {
-    // ---------------- compute warps: thread = block; warpgroup wg owns rows [64 wg, 64 wg + 64)
+    // ---------------- compute warps: thread = block; warpgroup wg owns rows [32 wg, 32 wg + 32)
     const int b = threadIdx.x % 128;
     const int wg = warp / 4;
-    const int r0 = 64 * wg;
+    const int r0 = 32 * wg;
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
     uint32_t sdp_count = 0, pds_count = 0, acc_count = 0, q_count = 0;
     for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
@@ -1202,55 +1242,79 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
       const int nrt = rt1 - rt0;
       bool ok = true;
       for (int i = 0; i < nrt; ++i) {
-        const int qb = q_count % 2;
-        if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
+        const int qb = q_count % kDkvQStages;
+        // S^T / dP^T of this tile, and its row constants (-lse log2 e, -D, w), which
+        // arrived with q_full[qb]
+        if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1) ||
+            !mbar_wait_warp(&sm.q_full[qb], (q_count / kDkvQStages) & 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        float sv[64], dp[64];
-        tmem_ld32(tm_s + lane_off + r0, sv);
-        tmem_ld32(tm_s + lane_off + r0 + 32, sv + 32);
-        tmem_ld32(tm_dp + lane_off + r0, dp);
-        tmem_ld32(tm_dp + lane_off + r0 + 32, dp + 32);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sdp_empty);
+        const int t_first = t_beg + (rt0 + i) * TPT;
+        const int nvr = (int)min((int64_t)kRows, (int64_t)(t_end - t_first) * G) - r0;  // valid rows of this warpgroup
+        const float2 qs = make_float2(qs2, qs2);
+        // the warpgroup's 32 rows in two passes of 16; S^T / dP^T are released after
+        // the second read, P^T w / dS^T written once the MMAs of the previous tile
+        // consumed them.  P^T w and dS^T go out as bf16 high + low parts: sums over
+        // many rows of near-equal probabilities would otherwise carry the bf16
+        // rounding of each term coherently (a 2^-9 relative bias).
+        bool ok_half = true;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float sv[16], dp[16];
+          tmem_ld16(tm_s + lane_off + r0 + 16 * hh, sv);
+          tmem_ld16(tm_dp + lane_off + r0 + 16 * hh, dp);
+          tmem_ld_wait();
+          if (hh == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sdp_empty);
+          }
+          const int nvh = nvr - 16 * hh;
+          if (nvh < 16) {  // rows of tokens past the sequence get p = 0
+#pragma unroll
+            for (int c = 0; c < 16; ++c) sv[c] = c < nvh ? sv[c] : -CUDART_INF_F;
+          }
+          uint32_t pw[8], dsv[8], pwl[8], dsl[8];
+#pragma unroll
+          for (int c = 0; c < 16; c += 4) {
+            const int rr = r0 + 16 * hh + c;
+            const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[qb][rr]);
+            const float4 d4 = *reinterpret_cast<const float4*>(&sm.Dr[qb][rr]);
+            const float4 w4 = *reinterpret_cast<const float4*>(&sm.wr[qb][rr]);
+            const float2 wa = make_float2(w4.x, w4.y), wb = make_float2(w4.z, w4.w);
+            const float2 pa = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, make_float2(l4.x, l4.y)));
+            const float2 pb = ex2x2(ffma2(make_float2(sv[c + 2], sv[c + 3]), qs, make_float2(l4.z, l4.w)));
+            split2(fmul2(pa, wa), pw[c / 2], pwl[c / 2]);
+            split2(fmul2(pb, wb), pw[c / 2 + 1], pwl[c / 2 + 1]);
+            split2(fmul2(pa, ffma2(wa, make_float2(dp[c], dp[c + 1]), make_float2(d4.x, d4.y))), dsv[c / 2],
+                   dsl[c / 2]);
+            split2(fmul2(pb, ffma2(wb, make_float2(dp[c + 2], dp[c + 3]), make_float2(d4.z, d4.w))),
+                   dsv[c / 2 + 1], dsl[c / 2 + 1]);
+          }
+          if (hh == 0) {
+            if (!mbar_wait_warp(&sm.pds_empty, (pds_count & 1) ^ 1)) {
+              ok_half = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          // rows [r0 + 16 hh, +16): packed TMEM columns [r0/2 + 8 hh, +8), SMEM 8-row chunks 2 (r0/16 + hh) + {0, 1}
+          tmem_st8(tm_p + lane_off + r0 / 2 + 8 * hh, pw);
+          tmem_st8(tm_ds + lane_off + r0 / 2 + 8 * hh, dsv);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int ch = r0 / 8 + 2 * hh + c;
+            store_pt_chunk(sm.plo, b, ch, make_uint4(pwl[4 * c], pwl[4 * c + 1], pwl[4 * c + 2], pwl[4 * c + 3]));
+            store_pt_chunk(sm.dslo, b, ch, make_uint4(dsl[4 * c], dsl[4 * c + 1], dsl[4 * c + 2], dsl[4 * c + 3]));
+          }
+        }
+        if (!ok_half) {
+          ok = false;
+          break;
+        }
         ++sdp_count;
-        // row scalars of this row tile arrived with q_full[qb] (already complete for the MMA)
-        if (!mbar_wait_warp(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
-        const int t_first = t_beg + (rt0 + i) * TPT;  // rows of tokens >= t_end contribute nothing
-        // P^T w and dS^T as bf16 high + low parts: the sums over many rows of
-        // near-equal probabilities would otherwise carry the bf16 rounding of
-        // each term coherently (a 2^-9 relative bias)
-        uint32_t pw[32], dsv[32], pwl[32], dsl[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[qb][r0 + c]);
-          const float4 d4 = *reinterpret_cast<const float4*>(&sm.Dr[qb][r0 + c]);
-          const float4 w4 = *reinterpret_cast<const float4*>(&sm.wr[qb][r0 + c]);
-          const bool vrow = t_first + (r0 + c) / G < t_end;  // the 4 rows share a token (G >= 4)
-          l4.x = vrow ? l4.x * kLog2e : CUDART_INF_F;
-          l4.y = vrow ? l4.y * kLog2e : CUDART_INF_F;
-          l4.z = vrow ? l4.z * kLog2e : CUDART_INF_F;
-          l4.w = vrow ? l4.w * kLog2e : CUDART_INF_F;
-          const float p0 = ex2(sv[c] * qs2 - l4.x), p1 = ex2(sv[c + 1] * qs2 - l4.y);
-          const float p2 = ex2(sv[c + 2] * qs2 - l4.z), p3 = ex2(sv[c + 3] * qs2 - l4.w);
-          split_bf16x2(p0 * w4.x, p1 * w4.y, pw[c / 2], pwl[c / 2]);
-          split_bf16x2(p2 * w4.z, p3 * w4.w, pw[c / 2 + 1], pwl[c / 2 + 1]);
-          split_bf16x2(p0 * (w4.x * dp[c] - d4.x), p1 * (w4.y * dp[c + 1] - d4.y), dsv[c / 2], dsl[c / 2]);
-          split_bf16x2(p2 * (w4.z * dp[c + 2] - d4.z), p3 * (w4.w * dp[c + 3] - d4.w), dsv[c / 2 + 1],
-                       dsl[c / 2 + 1]);
-        }
-        if (!mbar_wait_warp(&sm.pds_empty, (pds_count & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        tmem_st16(tm_p + lane_off + 32 * wg, pw);
-        tmem_st16(tm_p + lane_off + 32 * wg + 16, pw + 16);
-        tmem_st16(tm_ds + lane_off + 32 * wg, dsv);
-        tmem_st16(tm_ds + lane_off + 32 * wg + 16, dsv + 16);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          store_pt_chunk(sm.plo, b, 8 * wg + c, make_uint4(pwl[4 * c], pwl[4 * c + 1], pwl[4 * c + 2], pwl[4 * c + 3]));
-          store_pt_chunk(sm.dslo, b, 8 * wg + c, make_uint4(dsl[4 * c], dsl[4 * c + 1], dsl[4 * c + 2], dsl[4 * c + 3]));
-        }
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
@@ -1266,21 +1330,20 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_bwd_dkv_tc_kernel(
       if (!mbar_wait_warp(&sm.acc_full, acc_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++acc_count;
       tc_fence_after();
-      // warpgroup 0 adds dKc, warpgroup 1 adds dVc (lane = block)
-      float acc[64];
-      const uint32_t src = (wg == 0 ? tm_dk : tm_dv) + lane_off;
+      // warpgroups 0, 1 add dKc columns [0, 32), [32, 64); warpgroups 2, 3 the same of dVc (lane = block)
+      float acc[32];
+      const uint32_t src = (wg < 2 ? tm_dk : tm_dv) + lane_off + 32 * (wg & 1);
       tmem_ld32(src, acc);
-      tmem_ld32(src + 32, acc + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty);
       const int bidx = kt * kBN + b;
       if (bidx < nb && nrt > 0) {
-        float* dst = (wg == 0 ? dkc : dvc) + ((int64_t)g * btot + b0 + bidx) * 64;
-        const float mul = wg == 0 ? scale : 1.f;
+        float* dst = (wg < 2 ? dkc : dvc) + ((int64_t)g * btot + b0 + bidx) * 64 + 32 * (wg & 1);
+        const float mul = wg < 2 ? scale : 1.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 8; ++i)
           atomicAdd(reinterpret_cast<float4*>(dst) + i,
                     make_float4(acc[4 * i] * mul, acc[4 * i + 1] * mul, acc[4 * i + 2] * mul, acc[4 * i + 3] * mul));
       }
@@ -1367,20 +1430,21 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
   const int sms = num_sms();
   const int64_t tiles = tiles_bound * a.hkv;
   const int gq = (int)(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);
-  SSA_LAUNCH("cmp_bwd_dq_tc_kernel", cmp_bwd_dq_tc_kernel<G>, gq, kOutThreads, smem_bytes_dq(), st, qm, dm, km, vm,
-             a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.lse, a.Dc, a.gates, a.gate_mode,
-             a.dq, a.status);
+  const int64_t rows = a.N * a.hq;
+  SSA_LAUNCH("cmp_bwd_dq_tc_kernel", cmp_bwd_dq_tc_kernel<G>, gq, kDqThreads, smem_bytes_dq(), st, qm, dm, km, vm,
+             a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.rc, rows, a.dq, a.status);
   SSA_LAUNCH("dkv_plan_kernel", dkv_plan_kernel, (a.S + 256) / 256, 256, 0, st, a.cu_seqlens, a.blk->cu, a.S, G,
              dkv_cnt);
   cudaError_t e = exclusive_scan(dkv_cnt, dkv_pre, a.S + 1, scan_tmp, st);
   if (e != cudaSuccess) return e;
   cudaMemsetAsync(a.dkc, 0, sizeof(float) * rows_kv * 64, st);
   cudaMemsetAsync(a.dvc, 0, sizeof(float) * rows_kv * 64, st);
+  // row constants of the compressed branch: -lse log2(e), -D, w
   CUtensorMap lm, dcm, wm;
-  if (!map_rowscalars(&lm, a.lse, a.N, a.hq, G) || !map_rowscalars(&dcm, a.Dc, a.N, a.hq, G) ||
-      !map_rowscalars(&wm, a.wcmp, a.N, a.hq, G))
+  if (!map_rowscalars(&lm, a.rc, a.N, a.hq, G) || !map_rowscalars(&dcm, a.rc + 2 * rows, a.N, a.hq, G) ||
+      !map_rowscalars(&wm, a.rc + rows, a.N, a.hq, G))
     return cudaErrorInvalidValue;
-  SSA_LAUNCH("cmp_bwd_dkv_tc_kernel", cmp_bwd_dkv_tc_kernel<G>, sms, kOutThreads, smem_bytes_dkv(), st, qm, dm, km,
+  SSA_LAUNCH("cmp_bwd_dkv_tc_kernel", cmp_bwd_dkv_tc_kernel<G>, sms, kDkvThreads, smem_bytes_dkv(), st, qm, dm, km,
              vm, lm, dcm, wm, a.cu_seqlens, a.blk->cu, dkv_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.dkc, a.dvc,
              a.status);
   return cudaGetLastError();

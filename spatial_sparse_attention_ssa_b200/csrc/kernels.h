@@ -57,8 +57,9 @@ struct BwdArgs {
   float *dq, *dk, *dv, *dgates;
   // workspace
   float* Dc;          // [3, N, Hq]
-  float* wcmp;        // [N, Hq] gate weights of the compressed branch
-  float* wwin;        // [N, Hq] gate weights of the window branch
+  // per-row constants of the tensor-core backward kernels, [2 branches (cmp, win)]
+  // x [3][N, Hq]: -lse * log2(e), the gate weight w, and -D (D = w <dO, o>)
+  float* rc;
   int32_t *win_cnt, *win_pre;  // [W + 1] window work plan
   float *dkc, *dvc;   // [Hkv, B, d]
   uint64_t *inv_keys_a, *inv_keys_b;

@@ -252,13 +252,14 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
         if (lane == 0) mbar_arrive(&sm.s_empty);
         ++s_count;
         const int vc = min(kKT, x.nw - kt * kKT);
-        float cm = -CUDART_INF_F;
+        if (vc < kKT) {  // keys past the window
 #pragma unroll
-        for (int c = 0; c < kKT; ++c) {
-          sv[c] = c < vc ? sv[c] * qs2 : -CUDART_INF_F;
-          cm = fmaxf(cm, sv[c]);
+          for (int c = 0; c < kKT; ++c) sv[c] = c < vc ? sv[c] : -CUDART_INF_F;
         }
-        const float mn = fmaxf(m, cm);
+        float cm = sv[0];
+#pragma unroll
+        for (int c = 1; c < kKT; ++c) cm = fmaxf(cm, sv[c]);
+        const float mn = fmaxf(m, cm * qs2);  // qs2 > 0
         // the previous P V must be done before P is overwritten (and before O is rescaled)
         if (kt > 0 && !mbar_wait_warp(&sm.pv_done, (p_count - 1) & 1)) { ok = false; break; }
         // rescale the partial O by 2^(m - mn) (1 where the max did not grow); the
@@ -279,16 +280,16 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
           l *= corr;
         }
         m = mn;
+        const float2 qs = make_float2(qs2, qs2), nm = make_float2(-m, -m);
+        float2 lsum = make_float2(0.f, 0.f);
         uint32_t hi[64], lo[64];
 #pragma unroll
         for (int c = 0; c < kKT; c += 2) {
-          const float p0 = ex2(sv[c] - m), p1 = ex2(sv[c + 1] - m);
-          l += p0 + p1;
-          const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-          const float2 hf = __bfloat1622float2(h);
-          hi[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[c / 2] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
+          const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nm));
+          lsum = fadd2(lsum, p);
+          split2(p, hi[c / 2], lo[c / 2]);
         }
+        l += lsum.x + lsum.y;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 64; c += 16) {
@@ -501,9 +502,11 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
       const int qb = q_count % 2;
       if (!mbar_wait_warp(&sm.q_full[qb], (q_count / 2) & 1)) { timeout_exit(status, &sm.abort_flag); break; }
       ++q_count;
-      const float lse2 = sm.lse[qb][scalar_idx(r, G)] * kLog2e;
-      const float Dr = sm.Dr[qb][scalar_idx(r, G)];
-      const float wr = sm.wr[qb][scalar_idx(r, G)];
+      // row constants: -lse log2(e), -D, w
+      const float2 nl2 = make_float2(sm.lse[qb][scalar_idx(r, G)], sm.lse[qb][scalar_idx(r, G)]);
+      const float2 nd2 = make_float2(sm.Dr[qb][scalar_idx(r, G)], sm.Dr[qb][scalar_idx(r, G)]);
+      const float2 w2 = make_float2(sm.wr[qb][scalar_idx(r, G)], sm.wr[qb][scalar_idx(r, G)]);
+      const float2 qs = make_float2(qs2, qs2);
       const int tk = x.rt * TPT + r / G;
       const bool valid = tk < x.nw;
       const int nkt = (x.nw + kKT - 1) / kKT;
@@ -521,16 +524,16 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
           tmem_ld32(tm_dp + lane_off + 64 * half, dp);
           tmem_ld32(tm_dp + lane_off + 64 * half + 32, dp + 32);
           tmem_ld_wait();
+          const int nvh = vc - 64 * half;
+          if (nvh < 64) {  // keys past the window
+#pragma unroll
+            for (int c = 0; c < 64; ++c) sv[c] = c < nvh ? sv[c] : -CUDART_INF_F;
+          }
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
-            const int cc = 64 * half + c;
-            float d0 = 0.f, d1 = 0.f;
-            if (cc < vc) d0 = ex2(sv[c] * qs2 - lse2) * (wr * dp[c] - Dr);
-            if (cc + 1 < vc) d1 = ex2(sv[c + 1] * qs2 - lse2) * (wr * dp[c + 1] - Dr);
-            const __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
-            const float2 hf = __bfloat1622float2(h);
-            hi[cc / 2] = *reinterpret_cast<const uint32_t*>(&h);
-            lo[cc / 2] = pack_bf16x2(d0 - hf.x, d1 - hf.y);
+            const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
+            const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
+            split2(d, hi[(64 * half + c) / 2], lo[(64 * half + c) / 2]);
           }
         }
         tc_fence_before();
@@ -770,21 +773,24 @@ __global__ void __launch_bounds__(32 * (kCW + 2), 1) win_bwd_dkv_tc_kernel(
         if (lane == 0) mbar_arrive(&sm.sdp_empty);
         ++sdp_count;
         if (!mbar_wait_warp(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        const float2 qs = make_float2(qs2, qs2);
         uint32_t pw[32], dsv[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-          // 4 consecutive rows share a token (G >= 8): one float4 of its scalar slot
+          // 4 consecutive rows share a token (G >= 8): one float4 of its slot of row
+          // constants (-lse log2 e, -D, w); rows of tokens past the window were loaded
+          // as zeros: w = D = 0 there, so they add nothing
           const int si = scalar_idx(r0 + c, G);
           const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse[qb][si]);
           const float4 d4 = *reinterpret_cast<const float4*>(&sm.Dr[qb][si]);
           const float4 w4 = *reinterpret_cast<const float4*>(&sm.wr[qb][si]);
-          // rows of tokens past the window were loaded as zeros: w = D = 0 there, so they add nothing
-          const float p0 = ex2(sv[c] * qs2 - l4.x * kLog2e), p1 = ex2(sv[c + 1] * qs2 - l4.y * kLog2e);
-          const float p2 = ex2(sv[c + 2] * qs2 - l4.z * kLog2e), p3 = ex2(sv[c + 3] * qs2 - l4.w * kLog2e);
-          pw[c / 2] = pack_bf16x2(p0 * w4.x, p1 * w4.y);
-          pw[c / 2 + 1] = pack_bf16x2(p2 * w4.z, p3 * w4.w);
-          dsv[c / 2] = pack_bf16x2(p0 * (w4.x * dp[c] - d4.x), p1 * (w4.y * dp[c + 1] - d4.y));
-          dsv[c / 2 + 1] = pack_bf16x2(p2 * (w4.z * dp[c + 2] - d4.z), p3 * (w4.w * dp[c + 3] - d4.w));
+          const float2 wa = make_float2(w4.x, w4.y), wb = make_float2(w4.z, w4.w);
+          const float2 pa = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, make_float2(l4.x, l4.y)));
+          const float2 pb = ex2x2(ffma2(make_float2(sv[c + 2], sv[c + 3]), qs, make_float2(l4.z, l4.w)));
+          pw[c / 2] = pack2(fmul2(pa, wa));
+          pw[c / 2 + 1] = pack2(fmul2(pb, wb));
+          dsv[c / 2] = pack2(fmul2(pa, ffma2(wa, make_float2(dp[c], dp[c + 1]), make_float2(d4.x, d4.y))));
+          dsv[c / 2 + 1] = pack2(fmul2(pb, ffma2(wb, make_float2(dp[c + 2], dp[c + 3]), make_float2(d4.z, d4.w))));
         }
         if (!mbar_wait_warp(&sm.pds_empty, (pds_count & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
@@ -871,9 +877,9 @@ cudaError_t win_bwd_tc_g(const BwdArgs& a, int32_t* cnt, int32_t* pre, int32_t* 
   CUtensorMap qm, dm, km, vm, lm, cm, wm;
   if (!map_q_token(&qm, a.q, N, a.hq, G) || !map_q_token(&dm, a.dout, N, a.hq, G) ||
       !map_rows64(&km, a.ks, (int64_t)a.hkv * N) || !map_rows64(&vm, a.vs, (int64_t)a.hkv * N) ||
-      !map_rowscalars_token(&lm, a.lse + 2 * rows, N, a.hq, G) ||
-      !map_rowscalars_token(&cm, a.Dc + 2 * rows, N, a.hq, G) ||
-      !map_rowscalars_token(&wm, a.wwin, N, a.hq, G))
+      !map_rowscalars_token(&lm, a.rc + 3 * rows, N, a.hq, G) ||  // -lse log2(e) of the window branch
+      !map_rowscalars_token(&cm, a.rc + 5 * rows, N, a.hq, G) ||  // -D
+      !map_rowscalars_token(&wm, a.rc + 4 * rows, N, a.hq, G))    // w
     return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
