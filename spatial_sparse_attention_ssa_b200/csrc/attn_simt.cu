@@ -1171,10 +1171,15 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     SSA_LAUNCH("cmp_out_topk_kernel", (cmp_out_topk_kernel<T, D>), g2, 128, 0, st, q, kc, vc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
                                                   a.blk->count, qs2, a.lse, ob, a.topk, a.sel);
   }
-  const int pairs_per_cta = 128 / (G * C::NT);
-  SSA_LAUNCH("slc_fwd_kernel", (slc_fwd_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
-      q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2,
-      ob + rows * D, a.lse + rows);
+  if (a.use_tc && D == 64 && slc_mma_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
+    e = slc_fwd_mma(a, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    const int pairs_per_cta = 128 / (G * C::NT);
+    SSA_LAUNCH("slc_fwd_kernel", (slc_fwd_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st,
+               q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.hq, a.hkv,
+               a.topk, qs2, ob + rows * D, a.lse + rows);
+  }
   const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
   if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
     e = win_fwd_tc(a, a.win_cnt, a.win_pre, a.win_scan, st);
@@ -1236,7 +1241,10 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
     cudaMemsetAsync(a.dk, 0, sizeof(float) * a.N * a.hkv * D, st);
     cudaMemsetAsync(a.dv, 0, sizeof(float) * a.N * a.hkv * D, st);
     const int g_slc = grid_1d(a.N * a.hkv, 8, 148 * 16);
-    if (G == 16)
+    if (a.use_tc && slc_mma_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
+      e = slc_bwd_mma(a, st);
+      if (e != cudaSuccess) return e;
+    } else if (G == 16)
       SSA_LAUNCH("slc_bwd_fused_kernel", (slc_bwd_fused_kernel<T, 16>), g_slc, 256, 0, st, q, ks, vs, dout, a.gates,
                  a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
                  a.Dc + rows, a.dq, a.dk, a.dv);

@@ -85,4 +85,9 @@ cudaError_t cmp_bwd_tc(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, 
                        int64_t tiles_bound, cudaStream_t st);
 cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st);
 
+// Selected-block branch on warp-level MMAs (bf16, head dim 64, G in {8, 16}, top-k <= 32).
+bool slc_mma_supported(int dtype, int d, int hq, int hkv, int topk);
+cudaError_t slc_fwd_mma(const FwdArgs& a, cudaStream_t st);
+cudaError_t slc_bwd_mma(const BwdArgs& a, cudaStream_t st);
+
 }  // namespace ssa
