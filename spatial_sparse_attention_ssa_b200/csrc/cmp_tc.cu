@@ -244,6 +244,12 @@ constexpr int kOutStages = 3;
 constexpr int kCandMax = 128;  // top-k candidates per token kept for exact ranking
 constexpr int kComputeWarps = 8;  // pass 2: two warpgroups of compute warps
 constexpr int kOutThreads = 32 * (kComputeWarps + 2);  // + TMA warp + MMA warp
+// pass 2 adds a warpgroup that picks the top-k of the previous row tile while the
+// compute warps work on the next one (the importance scratch is double-buffered)
+constexpr int kOutTopkWarps = 4;
+constexpr int kOutTmaWarp = kComputeWarps + kOutTopkWarps;
+constexpr int kOutMmaWarp = kOutTmaWarp + 1;
+constexpr int kOutThreadsTk = 32 * (kOutMmaWarp + 1);
 
 struct OutSmem {
   uint8_t q[2][kTile];
@@ -251,10 +257,10 @@ struct OutSmem {
   uint8_t vc[kOutStages][kTile];
   uint8_t pt_hi[2 * kTile];  // P^T (bf16 high part) as the MN-major A operand: [2 row atoms][128 blocks][64 rows]
   uint8_t pt_lo[2 * kTile];  // p - bf16(p), same layout: O += (P_hi + P_lo) Vc keeps fp32-level accuracy
-  __align__(16) float lse2[kRows];
-  float candv[kComputeWarps][kCandMax];
-  int candi[kComputeWarps][kCandMax];
-  uint64_t q_full[2], q_empty[2], mma_done, o_full, o_empty, cw;
+  __align__(16) float lse2[2][kRows];  // -lse log2(e) of the tile's rows, double-buffered by tile
+  float candv[kOutTopkWarps][kCandMax];
+  int candi[kOutTopkWarps][kCandMax];
+  uint64_t q_full[2], q_empty[2], mma_done, o_full, o_empty, cw, imp_full[2], imp_empty[2];
   uint64_t kv_full[kOutStages], kv_empty[kOutStages];
   uint64_t s_full, s_empty, pt_full, pt_empty;
   uint32_t tmem;
@@ -288,7 +294,7 @@ __device__ __forceinline__ bool cw_sync(uint64_t* bar, uint32_t& phase) {
 // list heads pick the winners.  Writes b0 + local id of the picks, ascending,
 // padded with -1, to out[0..topk).  Requires topk <= KL.
 template <int KL>
-__device__ void warp_topk(const float* __restrict__ imp, int nb, int topk, int b0, int32_t* __restrict__ out) {
+__device__ void warp_topk(const float* imp, int nb, int topk, int b0, int32_t* __restrict__ out) {
   const int lane = threadIdx.x & 31;
   const int keff = min(topk, nb);
   float lv[KL];
@@ -381,7 +387,7 @@ __device__ void warp_topk(const float* __restrict__ imp, int nb, int topk, int b
 //     shared memory and ranked exactly against each other.
 // Falls back to warp_topk when more than kCandMax entries pass the threshold.
 template <int KL>
-__device__ void warp_topk_fast(const float* __restrict__ imp, int nb, int topk, int b0, int32_t* __restrict__ out,
+__device__ void warp_topk_fast(const float* imp, int nb, int topk, int b0, int32_t* __restrict__ out,
                                float* cv, int* ci) {
   const int lane = threadIdx.x & 31;
   const int keff = min(topk, nb);
@@ -521,8 +527,137 @@ __device__ void warp_topk_fast(const float* __restrict__ imp, int nb, int topk, 
   __syncwarp();
 }
 
+// Exact top-k as warp_topk_fast for nb <= 256 * NF4, built for short dependency
+// chains: the scores are read in two batches of NF4 float4 per lane (each batch's
+// loads in flight together) for the lane bests, then read again (mostly L1 hits)
+// while candidates are compacted with warp votes, skipping the 4-entry groups that
+// hold none (typically all but a few).
+template <int NF4>
+__device__ __forceinline__ void load_batch(const float* imp, int nb, int base, int lane, float4* v) {
+#pragma unroll
+  for (int u = 0; u < NF4; ++u) {
+    const int i0 = base + 128 * u + 4 * lane;
+    if (i0 + 3 < nb) {
+      v[u] = *reinterpret_cast<const float4*>(imp + i0);
+    } else {
+      v[u].x = i0 + 0 < nb ? imp[i0 + 0] : -CUDART_INF_F;
+      v[u].y = i0 + 1 < nb ? imp[i0 + 1] : -CUDART_INF_F;
+      v[u].z = i0 + 2 < nb ? imp[i0 + 2] : -CUDART_INF_F;
+      v[u].w = -CUDART_INF_F;
+    }
+  }
+}
+template <int NF4, int KL>
+__device__ void warp_topk_regs(const float* imp, int nb, int topk, int b0, int32_t* __restrict__ out, float* cv,
+                               int* ci) {
+  const int lane = threadIdx.x & 31;
+  const int keff = min(topk, nb);
+  // 1. lane best (ties to the lower index); entries past nb are -inf and never win
+  float bv = -CUDART_INF_F;
+  int bi = 0x7fffffff;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float4 v[NF4];
+    load_batch<NF4>(imp, nb, h * 128 * NF4, lane, v);
+#pragma unroll
+    for (int u = 0; u < NF4; ++u) {
+      const int i0 = h * 128 * NF4 + 128 * u + 4 * lane;
+      if (i0 < nb && v[u].x > bv) { bv = v[u].x; bi = i0; }
+      if (i0 + 1 < nb && v[u].y > bv) { bv = v[u].y; bi = i0 + 1; }
+      if (i0 + 2 < nb && v[u].z > bv) { bv = v[u].z; bi = i0 + 2; }
+      if (i0 + 3 < nb && v[u].w > bv) { bv = v[u].w; bi = i0 + 3; }
+    }
+  }
+  // 2. tau = the lane best of rank keff - 1 among the 32
+  int rank = 0;
+#pragma unroll
+  for (int o = 0; o < 32; ++o) {
+    const float v2 = __shfl_sync(0xffffffffu, bv, o);
+    const int i2 = __shfl_sync(0xffffffffu, bi, o);
+    if (beats(v2, i2, bv, bi)) ++rank;
+  }
+  const unsigned own = __ballot_sync(0xffffffffu, rank == keff - 1);
+  if (keff > 32 || own == 0u) {
+    warp_topk<KL>(imp, nb, topk, b0, out);
+    return;
+  }
+  const int src = __ffs(own) - 1;
+  const float tv = __shfl_sync(0xffffffffu, bv, src);
+  const int ti = __shfl_sync(0xffffffffu, bi, src);
+  // 3. entries at or above (tv, ti), compacted in index order by warp votes
+  const unsigned lt = (1u << lane) - 1u;
+  int n = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float4 v[NF4];
+    load_batch<NF4>(imp, nb, h * 128 * NF4, lane, v);
+#pragma unroll
+    for (int u = 0; u < NF4; ++u) {
+      const int i0 = h * 128 * NF4 + 128 * u + 4 * lane;
+      const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      bool tk[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tk[e] = i0 + e < nb && (xs[e] == tv ? i0 + e <= ti : xs[e] > tv);
+      if (__ballot_sync(0xffffffffu, tk[0] || tk[1] || tk[2] || tk[3]) == 0u) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const unsigned m = __ballot_sync(0xffffffffu, tk[e]);
+        if (tk[e]) {
+          const int slot = n + __popc(m & lt);
+          if (slot < kCandMax) {
+            cv[slot] = xs[e];
+            ci[slot] = i0 + e;
+          }
+        }
+        n += __popc(m);
+      }
+    }
+  }
+  if (n > kCandMax) {
+    __syncwarp();
+    warp_topk<KL>(imp, nb, topk, b0, out);
+    return;
+  }
+  __syncwarp();
+  // exact ranks among the candidates; picks are those with rank < keff
+  int picked_id[kCandMax / 32];
+  bool picked[kCandMax / 32];
+#pragma unroll
+  for (int u = 0; u < kCandMax / 32; ++u) {
+    const int c = u * 32 + lane;
+    picked[u] = false;
+    picked_id[u] = 0x7fffffff;
+    if (c < n) {
+      const float x = cv[c];
+      const int id = ci[c];
+      int r = 0;
+      for (int j = 0; j < n; ++j) r += beats(cv[j], ci[j], x, id) ? 1 : 0;
+      picked[u] = r < keff;
+      picked_id[u] = id;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < kCandMax / 32; ++u) {
+    const int c = u * 32 + lane;
+    if (c < n) ci[c] = picked[u] ? picked_id[u] : 0x7fffffff;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < kCandMax / 32; ++u) {
+    if (picked[u]) {
+      int pos = 0;
+      for (int j = 0; j < n; ++j) pos += ci[j] < picked_id[u] ? 1 : 0;
+      out[pos] = b0 + picked_id[u];
+    }
+  }
+  for (int i = keff + lane; i < topk; i += 32) out[i] = -1;
+  __syncwarp();
+}
+constexpr int kTopkRegF4 = 10;  // float4 per lane per batch: two batches cover sequences of up to 2560 blocks
+
 template <int G>
-__global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
+__global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_out_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap,
     const __grid_constant__ CUtensorMap vcmap, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
     const int32_t* __restrict__ tpre, int S, int hq, int hkv, int btot, float qs2, const float* __restrict__ lse_in,
@@ -534,8 +669,8 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntiles = tpre[S];
   const int total = ntiles * hkv;
-  // this CTA's scores: [TPT tokens][imp_stride blocks]
-  float* imp_base = imp_scratch + (int64_t)blockIdx.x * TPT * imp_stride;
+  // this CTA's scores, two buffers of [TPT tokens][imp_stride blocks]
+  float* imp_cta = imp_scratch + (int64_t)blockIdx.x * 2 * TPT * imp_stride;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.q_full[i], 1);
@@ -545,6 +680,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_empty, kComputeWarps);
     mbar_init(&sm.cw, kComputeWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.imp_full[i], kComputeWarps);
+      mbar_init(&sm.imp_empty[i], kOutTopkWarps);
+    }
     for (int i = 0; i < kOutStages; ++i) {
       mbar_init(&sm.kv_full[i], 1);
       mbar_init(&sm.kv_empty[i], 1);
@@ -566,7 +705,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
   const uint32_t tmem = sm.tmem;
   const uint32_t tm_s = tmem, tm_o = tmem + 128;  // S^T: columns [0,128); O: [128,192)
 
-  if (warp == kComputeWarps) {
+  if (warp == kOutTmaWarp) {
     // ---------------- TMA producer: Q per tile; (Kc, Vc) per key tile
     if (lane == 0) {
       prefetch_tmap(&qmap);
@@ -598,7 +737,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
       for (int i = 0; i < kOutStages; ++i)
         if (last_par[i] >= 0) mbar_wait(&sm.kv_full[i], (uint32_t)last_par[i]);
     }
-  } else if (warp == kComputeWarps + 1) {
+  } else if (warp == kOutMmaWarp) {
     // ---------------- MMA issuer: S^T(j+1) is issued as soon as S^T(j) has been read,
     // so it overlaps with the exps of tile j; O += P(j) Vc(j) follows when P^T(j) is ready.
     if (lane == 0) {
@@ -655,81 +794,102 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
       mma_commit(&sm.mma_done);
       mbar_wait(&sm.mma_done, 0);
     }
-  } else {
+  } else if (warp < kComputeWarps) {
     // ---------------- compute warps (two warpgroups): thread = block of the key tile;
-    // warpgroup wg handles query rows [64 wg, 64 wg + 64) of the tile.
+    // warpgroup wg handles query rows [64 wg, 64 wg + 64) of the tile, in two passes of 32.
     const int b = threadIdx.x % 128;
     const int wg = warp / 4;
     const int r0 = 64 * wg;
-    uint32_t s_count = 0, pt_count = 0, o_count = 0, cw_phase = 0;
-    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+    uint32_t s_count = 0, pt_count = 0, o_count = 0, cw_phase = 0, n_tile = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x, ++n_tile) {
       const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+      const int lb = n_tile & 1;
       if (wg == 0) {
         const int r = threadIdx.x;
         const int64_t t = min((int64_t)ti.t0 + r / G, (int64_t)ti.t_end - 1);
-        sm.lse2[r] = -lse_in[t * hq + ti.g * G + r % G] * kLog2e;  // -lse log2(e)
+        sm.lse2[lb][r] = -lse_in[t * hq + ti.g * G + r % G] * kLog2e;  // -lse log2(e)
       }
       if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
+      // the top-k warps have released this tile's importance buffer
+      if (!mbar_wait_warp(&sm.imp_empty[lb], ((n_tile >> 1) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+      float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
       const int nbt = (ti.nb + kBN - 1) / kBN;
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
         if (!mbar_wait_warp(&sm.s_full, s_count & 1)) { ok = false; break; }
         tc_fence_after();
-        float p[64];
-        const uint32_t taddr = tm_s + ((uint32_t)((warp % 4) * 32) << 16) + r0;
-        tmem_ld32(taddr, p);
-        tmem_ld32(taddr + 32, p + 32);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_empty);
-        ++s_count;
         const int bidx = j * kBN + b;  // block index inside the sequence
         const bool bvalid = bidx < ti.nb;
-        if (!bvalid) {  // ragged last key tile: blocks past the sequence get p = 0
-#pragma unroll
-          for (int r = 0; r < 64; ++r) p[r] = -CUDART_INF_F;
-        }
+        const uint32_t taddr = tm_s + ((uint32_t)((warp % 4) * 32) << 16) + r0;
         const float2 qs = make_float2(qs2, qs2);
+        bool ok_half = true;
 #pragma unroll
-        for (int r = 0; r < 64; r += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[r0 + r]);
-          const float2 pa = ex2x2(ffma2(make_float2(p[r], p[r + 1]), qs, make_float2(l4.x, l4.y)));
-          const float2 pb = ex2x2(ffma2(make_float2(p[r + 2], p[r + 3]), qs, make_float2(l4.z, l4.w)));
-          p[r] = pa.x;
-          p[r + 1] = pa.y;
-          p[r + 2] = pb.x;
-          p[r + 3] = pb.y;
+        for (int hh = 0; hh < 2; ++hh) {
+          float p[32];
+          tmem_ld32(taddr + 32 * hh, p);
+          tmem_ld_wait();
+          if (hh == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_empty);
+          }
+          if (!bvalid) {  // ragged last key tile: blocks past the sequence get p = 0
+#pragma unroll
+            for (int r = 0; r < 32; ++r) p[r] = -CUDART_INF_F;
+          }
+#pragma unroll
+          for (int r = 0; r < 32; r += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[lb][r0 + 32 * hh + r]);
+            const float2 pa = ex2x2(ffma2(make_float2(p[r], p[r + 1]), qs, make_float2(l4.x, l4.y)));
+            const float2 pb = ex2x2(ffma2(make_float2(p[r + 2], p[r + 3]), qs, make_float2(l4.z, l4.w)));
+            p[r] = pa.x;
+            p[r + 1] = pa.y;
+            p[r + 2] = pb.x;
+            p[r + 3] = pb.y;
+          }
+          if (hh == 0) {
+            if (!mbar_wait_warp(&sm.pt_empty, (pt_count & 1) ^ 1)) {
+              ok_half = false;
+              break;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) split2(make_float2(p[8 * c + 2 * e], p[8 * c + 2 * e + 1]), hi[e], lo[e]);
+            store_pt_chunk(sm.pt_hi, b, 8 * wg + 4 * hh + c, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+            store_pt_chunk(sm.pt_lo, b, 8 * wg + 4 * hh + c, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+          }
+          // selection score of this block for the pass's tokens: probability summed over the group's heads
+          if (bvalid) {
+#pragma unroll
+            for (int tl = 0; tl < 32 / G; ++tl) {
+              float2 acc = make_float2(p[tl * G], p[tl * G + 1]);
+#pragma unroll
+              for (int hh2 = 2; hh2 < G; hh2 += 2) acc = fadd2(acc, make_float2(p[tl * G + hh2], p[tl * G + hh2 + 1]));
+              imp_base[(int64_t)((r0 + 32 * hh) / G + tl) * imp_stride + bidx] = acc.x + acc.y;
+            }
+          }
         }
-        if (!mbar_wait_warp(&sm.pt_empty, (pt_count & 1) ^ 1)) { ok = false; break; }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) split2(make_float2(p[8 * c + 2 * e], p[8 * c + 2 * e + 1]), hi[e], lo[e]);
-          store_pt_chunk(sm.pt_hi, b, 8 * wg + c, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-          store_pt_chunk(sm.pt_lo, b, 8 * wg + c, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+        if (!ok_half) {
+          ok = false;
+          break;
         }
+        ++s_count;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.pt_full);
         ++pt_count;
-        // selection score of this block for each of the warpgroup's tokens:
-        // probability summed over the group's heads
-        if (bvalid) {
-#pragma unroll
-          for (int tl = 0; tl < 64 / G; ++tl) {
-            float2 acc = make_float2(p[tl * G], p[tl * G + 1]);
-#pragma unroll
-            for (int hh = 2; hh < G; hh += 2) acc = fadd2(acc, make_float2(p[tl * G + hh], p[tl * G + hh + 1]));
-            imp_base[(int64_t)(wg * (64 / G) + tl) * imp_stride + bidx] = acc.x + acc.y;
-          }
-        }
       }
       if (!ok) {
         record_timeout(status, &sm.abort_flag);
         break;
       }
+      // this tile's importances are complete: hand them to the top-k warps
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.imp_full[lb]);
       // O of this tile: wait for the last P Vc; warpgroup wg writes columns [32 wg, 32 wg + 32)
       if (!mbar_wait_warp(&sm.o_full, o_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++o_count;
@@ -750,22 +910,35 @@ __global__ void __launch_bounds__(kOutThreads, 1) cmp_out_tc_kernel(
           for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
       }
-      // top-k per token from the scores of all blocks (one warp per token)
-      __threadfence_block();
-      if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
-      for (int tk = warp; tk < TPT; tk += kComputeWarps) {
+    }
+  } else {
+    // ---------------- top-k warps: the selection of each tile's tokens (one warp per token)
+    const int tw = warp - kComputeWarps;
+    uint32_t n_tile = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x, ++n_tile) {
+      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+      const int lb = n_tile & 1;
+      if (!mbar_wait_warp(&sm.imp_full[lb], (n_tile >> 1) & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      const float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
+      for (int tk = tw; tk < TPT; tk += kOutTopkWarps) {
         const int64_t t = ti.t0 + tk;
         if (t < ti.t_end) {
-          if (topk <= 16)
-            warp_topk_fast<16>(imp_base + (int64_t)tk * imp_stride, ti.nb, topk, ti.b0,
-                               sel + (t * hkv + ti.g) * topk, sm.candv[warp], sm.candi[warp]);
-          else
-            warp_topk_fast<kTopkMax>(imp_base + (int64_t)tk * imp_stride, ti.nb, topk, ti.b0,
-                                     sel + (t * hkv + ti.g) * topk, sm.candv[warp], sm.candi[warp]);
+          const float* imp = imp_base + (int64_t)tk * imp_stride;
+          int32_t* dst = sel + (t * hkv + ti.g) * topk;
+          if (ti.nb <= 256 * kTopkRegF4) {
+            if (topk <= 16)
+              warp_topk_regs<kTopkRegF4, 16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+            else
+              warp_topk_regs<kTopkRegF4, kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+          } else if (topk <= 16) {
+            warp_topk_fast<16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+          } else {
+            warp_topk_fast<kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+          }
         }
       }
-      __threadfence_block();
-      if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.imp_empty[lb]);
     }
   }
   tc_fence_before();
@@ -1382,7 +1555,7 @@ cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_ti
   const int g2 = (int)(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);  // at most kCmpOutCtas (scratch size)
   SSA_LAUNCH("cmp_lse_tc_kernel", cmp_lse_tc_kernel, g1, kThreads, smem_bytes_lse(), st, qm, km, a.cu_seqlens,
              a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.status);
-  SSA_LAUNCH("cmp_out_tc_kernel", cmp_out_tc_kernel<G>, g2, kOutThreads, smem_bytes_out(), st, qm, km, vm,
+  SSA_LAUNCH("cmp_out_tc_kernel", cmp_out_tc_kernel<G>, g2, kOutThreadsTk, smem_bytes_out(), st, qm, km, vm,
              a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.o_branch, a.topk, a.sel,
              a.imp_scratch, (int64_t)((btot + 3) & ~3), a.status);
   return cudaGetLastError();
@@ -1453,7 +1626,7 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
 
 size_t cmp_tc_scratch_floats(int hq, int hkv, int64_t btot) {
   const int G = hkv > 0 ? hq / hkv : 1;
-  return (size_t)kCmpOutCtas * (kRows / (G > 0 ? G : 1)) * (size_t)((btot + 3) & ~int64_t(3)) + 4;
+  return (size_t)kCmpOutCtas * 2 * (kRows / (G > 0 ? G : 1)) * (size_t)((btot + 3) & ~int64_t(3)) + 4;
 }
 
 bool cmp_tc_supported(int dtype, int d, int hq, int hkv, int topk) {
