@@ -209,8 +209,9 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
             break;
           }
           tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < kKT / 16; ++k) {
+          // only the 16-key steps that hold keys of the window (P is zero past them)
+          const int nks = (min(kKT, x.nw - kt * kKT) + 15) / 16;
+          for (int k = 0; k < nks; ++k) {
             const uint64_t bdesc = sdesc_mnmajor_sw128(sm.v[st], 2048 * k, kTile);
             mma_bf16_ts(tm_o, tm_ph + 8 * k, bdesc, id_o, kt > 0 || k > 0);
             mma_bf16_ts(tm_o, tm_pl + 8 * k, bdesc, id_o, true);
@@ -472,8 +473,9 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
             break;
           }
           tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < kKT / 16; ++k) {
+          // only the 16-key steps that hold keys of the window (dS is zero past them)
+          const int nks = (min(kKT, x.nw - kt * kKT) + 15) / 16;
+          for (int k = 0; k < nks; ++k) {
             const uint64_t bdesc = sdesc_mnmajor_sw128(sm.k[st], 2048 * k, kTile);
             mma_bf16_ts(tm_dq, tm_dsh + 8 * k, bdesc, id_q, kt > 0 || k > 0);
             mma_bf16_ts(tm_dq, tm_dsl + 8 * k, bdesc, id_q, true);
@@ -514,26 +516,28 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
       for (int kt = 0; kt < nkt; ++kt) {
         if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
         tc_fence_after();
+        // only the 32-key chunks that hold keys of the window take part (vc keys)
         const int vc = min(kKT, x.nw - kt * kKT);
+        const int nch = (vc + 31) / 32;
         uint32_t hi[64], lo[64];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float sv[64], dp[64];
-          tmem_ld32(tm_s + lane_off + 64 * half, sv);
-          tmem_ld32(tm_s + lane_off + 64 * half + 32, sv + 32);
-          tmem_ld32(tm_dp + lane_off + 64 * half, dp);
-          tmem_ld32(tm_dp + lane_off + 64 * half + 32, dp + 32);
-          tmem_ld_wait();
-          const int nvh = vc - 64 * half;
-          if (nvh < 64) {  // keys past the window
+        for (int ch = 0; ch < kKT / 32; ++ch) {
+          if (ch < nch) {
+            float sv[32], dp[32];
+            tmem_ld32(tm_s + lane_off + 32 * ch, sv);
+            tmem_ld32(tm_dp + lane_off + 32 * ch, dp);
+            tmem_ld_wait();
+            const int nvh = vc - 32 * ch;
+            if (nvh < 32) {  // keys past the window
 #pragma unroll
-            for (int c = 0; c < 64; ++c) sv[c] = c < nvh ? sv[c] : -CUDART_INF_F;
-          }
+              for (int c = 0; c < 32; ++c) sv[c] = c < nvh ? sv[c] : -CUDART_INF_F;
+            }
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
-            const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
-            split2(d, hi[(64 * half + c) / 2], lo[(64 * half + c) / 2]);
+            for (int c = 0; c < 32; c += 2) {
+              const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
+              const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
+              split2(d, hi[(32 * ch + c) / 2], lo[(32 * ch + c) / 2]);
+            }
           }
         }
         tc_fence_before();
@@ -543,9 +547,11 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
         if (!mbar_wait_warp(&sm.ds_empty, (ds_count & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 64; c += 16) {
-          tmem_st16(tm_dsh + lane_off + c, hi + c);
-          tmem_st16(tm_dsl + lane_off + c, lo + c);
+        for (int ch = 0; ch < kKT / 32; ++ch) {
+          if (ch < nch) {
+            tmem_st16(tm_dsh + lane_off + 16 * ch, hi + 16 * ch);
+            tmem_st16(tm_dsl + lane_off + 16 * ch, lo + 16 * ch);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -757,11 +763,26 @@ __global__ void __launch_bounds__(32 * (kCW + 2), 1) win_bwd_dkv_tc_kernel(
     for (int it = blockIdx.x; it < total && !is_aborted(&sm.abort_flag); it += gridDim.x) {
       const WinItem x = win_kitem(it, nitems_g, wkpre, W, wptr);
       const int nrt = (x.nw + TPT - 1) / TPT;
+      // a warp whose 32 keys all lie past the window skips the arithmetic (its rows of
+      // dK / dV are discarded) but keeps the barrier protocol
+      const bool active = 32 * (warp % 4) < x.nw - x.rt * kKT;
       bool ok = true;
       for (int i = 0; i < nrt; ++i) {
         const int qb = q_count % 2;
         if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
         tc_fence_after();
+        if (!active) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.sdp_empty);
+          ++sdp_count;
+          if (!mbar_wait_warp(&sm.pds_empty, (pds_count & 1) ^ 1)) { ok = false; break; }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.pds_full);
+          ++pds_count;
+          ++q_count;
+          continue;
+        }
         float sv[64], dp[64];
         tmem_ld32(tm_s + lane_off + r0, sv);
         tmem_ld32(tm_s + lane_off + r0 + 32, sv + 32);
