@@ -947,30 +947,29 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_out_tc_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// backward, dQ (thread = row): S = Q Kc^T, dP = dO Vc^T in TMEM; dS = P (w dP - D)
-// in registers; dQ += dS Kc with dS (bf16 hi + lo) as the TMEM A operand.
+// backward, dQ (thread = row): S = Q Kc^T, dP = dO Vc^T in TMEM over 64-block key
+// tiles; dS = P (w dP - D) in registers; dQ += dS Kc with dS (bf16 hi + lo) as the
+// TMEM A operand.  A CTA holds 256 TMEM columns and ~80 KB of shared memory, so two
+// CTAs share an SM and one's exponentials overlap the other's MMAs.
 // ---------------------------------------------------------------------------
 constexpr int kBwdStages = 3;
-// four compute warpgroups, each owning 32 of a key tile's 128 blocks: twice the
-// warps of a two-warpgroup split, to hide the latency of TMEM loads and MUFU
-constexpr int kDqWarpgroups = 4;
-constexpr int kDqComputeWarps = 4 * kDqWarpgroups;
-constexpr int kDqThreads = 32 * (kDqComputeWarps + 2);  // + TMA warp + MMA warp
-constexpr int kDqCols = kBN / kDqWarpgroups;
+constexpr int kDqBN = 64;                 // compressed blocks per key tile
+constexpr int kDqThreads = 32 * (4 + 2);  // one compute warpgroup + TMA warp + MMA warp
+constexpr int kDqCtasPerSm = 2;
 
 struct DqSmem {
-  uint8_t q[2][kTile];
-  uint8_t dout[2][kTile];
-  uint8_t kc[kBwdStages][kTile];
-  uint8_t vc[kBwdStages][kTile];
-  uint64_t q_full[2], q_empty[2], kv_full[kBwdStages], kv_empty[kBwdStages];
+  uint8_t q[kTile];
+  uint8_t dout[kTile];
+  uint8_t kc[kBwdStages][kTile / 2];  // 64 blocks x 64 bf16
+  uint8_t vc[kBwdStages][kTile / 2];
+  uint64_t q_full, q_empty, kv_full[kBwdStages], kv_empty[kBwdStages];
   uint64_t sdp_full, sdp_empty, ds_full, ds_empty, dq_full, dq_empty, mma_done;
   uint32_t tmem;
   int abort_flag;
 };
 
 template <int G>
-__global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
+__global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) cmp_bwd_dq_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap dmap,
     const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
     const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S, int hq,
@@ -982,36 +981,34 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
   const int ntiles = tpre[S];
   const int total = ntiles * hkv;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.q_full[i], 1);
-      mbar_init(&sm.q_empty[i], 1);
-    }
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
     for (int i = 0; i < kBwdStages; ++i) {
       mbar_init(&sm.kv_full[i], 1);
       mbar_init(&sm.kv_empty[i], 1);
     }
     mbar_init(&sm.sdp_full, 1);
-    mbar_init(&sm.sdp_empty, kDqComputeWarps);
-    mbar_init(&sm.ds_full, kDqComputeWarps);
+    mbar_init(&sm.sdp_empty, 4);
+    mbar_init(&sm.ds_full, 4);
     mbar_init(&sm.ds_empty, 1);
     mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_empty, kDqComputeWarps);
+    mbar_init(&sm.dq_empty, 4);
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&sm.tmem, 512);
+    tmem_alloc(&sm.tmem, 256);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  // TMEM columns: S [0,128), dP [128,256), dS hi [256,320), dS lo [320,384), dQ [384,448)
-  const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dsh = tmem + 256, tm_dsl = tmem + 320, tm_dq = tmem + 384;
+  // TMEM columns: S [0,64), dP [64,128), dS hi [128,160), dS lo [160,192), dQ [192,256)
+  const uint32_t tm_s = tmem, tm_dp = tmem + 64, tm_dsh = tmem + 128, tm_dsl = tmem + 160, tm_dq = tmem + 192;
 
-  if (warp == kDqComputeWarps) {
+  if (warp == 4) {
     // ---------------- TMA producer: (Q, dO) per row tile; (Kc, Vc) per key tile
     if (lane == 0) {
       uint32_t kv_count = 0, q_count = 0;
@@ -1019,19 +1016,18 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
       for (int i = 0; i < kBwdStages; ++i) last_par[i] = -1;
       for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
         const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
-        const int qb = q_count % 2;
-        if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
-        mbar_expect_tx(&sm.q_full[qb], 2 * kTile);
-        tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
-        tma_load_3d(sm.dout[qb], &dmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
+        if (!mbar_wait(&sm.q_empty, (q_count & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+        mbar_expect_tx(&sm.q_full, 2 * kTile);
+        tma_load_3d(sm.q, &qmap, &sm.q_full, 0, ti.g * G, ti.t0);
+        tma_load_3d(sm.dout, &dmap, &sm.q_full, 0, ti.g * G, ti.t0);
         ++q_count;
-        const int nbt = (ti.nb + kBN - 1) / kBN;
+        const int nbt = (ti.nb + kDqBN - 1) / kDqBN;
         for (int j = 0; j < nbt; ++j) {
           const int st = kv_count % kBwdStages;
           const uint32_t ph = (kv_count / kBwdStages) & 1;
           if (!mbar_wait(&sm.kv_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
-          mbar_expect_tx(&sm.kv_full[st], 2 * kTile);
-          const int row = ti.g * btot + ti.b0 + j * kBN;
+          mbar_expect_tx(&sm.kv_full[st], kTile);
+          const int row = ti.g * btot + ti.b0 + j * kDqBN;
           tma_load_2d(sm.kc[st], &kcmap, &sm.kv_full[st], 0, row);
           tma_load_2d(sm.vc[st], &vcmap, &sm.kv_full[st], 0, row);
           last_par[st] = (int)ph;
@@ -1041,19 +1037,18 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
       for (int i = 0; i < kBwdStages; ++i)
         if (last_par[i] >= 0) mbar_wait(&sm.kv_full[i], (uint32_t)last_par[i]);
     }
-  } else if (warp == kDqComputeWarps + 1) {
+  } else if (warp == 5) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      const uint32_t id_s = idesc_bf16(kRows, kBN);              // S, dP [rows, blocks]
+      const uint32_t id_s = idesc_bf16(kRows, kDqBN);             // S, dP [rows, blocks]
       const uint32_t id_q = idesc_bf16(kRows, 64, false, true);   // dQ[rows, 64] += dS[rows, blocks] Kc
       uint32_t kv_count = 0, q_count = 0, sdp_count = 0, ds_count = 0, dq_count = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
         const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
-        const int qb = q_count % 2;
-        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        if (!mbar_wait(&sm.q_full, q_count & 1)) { ok = false; break; }
         ++q_count;
-        const int nbt = (ti.nb + kBN - 1) / kBN;
+        const int nbt = (ti.nb + kDqBN - 1) / kDqBN;
         auto issue_sdp = [&](uint32_t kv_idx) -> bool {
           const int st = kv_idx % kBwdStages;
           if (!mbar_wait(&sm.kv_full[st], (kv_idx / kBwdStages) & 1) ||
@@ -1062,8 +1057,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            mma_bf16_ss(tm_s, sdesc_kmajor_sw128(sm.q[qb], 32 * k), sdesc_kmajor_sw128(sm.kc[st], 32 * k), id_s, k > 0);
-            mma_bf16_ss(tm_dp, sdesc_kmajor_sw128(sm.dout[qb], 32 * k), sdesc_kmajor_sw128(sm.vc[st], 32 * k), id_s,
+            mma_bf16_ss(tm_s, sdesc_kmajor_sw128(sm.q, 32 * k), sdesc_kmajor_sw128(sm.kc[st], 32 * k), id_s, k > 0);
+            mma_bf16_ss(tm_dp, sdesc_kmajor_sw128(sm.dout, 32 * k), sdesc_kmajor_sw128(sm.vc[st], 32 * k), id_s,
                         k > 0);
           }
           mma_commit(&sm.sdp_full);
@@ -1080,7 +1075,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
           }
           tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {
+          for (int k = 0; k < kDqBN / 16; ++k) {
             const uint64_t bdesc = sdesc_mnmajor_sw128(sm.kc[st], 2048 * k, kTile);
             mma_bf16_ts(tm_dq, tm_dsh + 8 * k, bdesc, id_q, j > 0 || k > 0);
             mma_bf16_ts(tm_dq, tm_dsl + 8 * k, bdesc, id_q, true);
@@ -1091,7 +1086,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
           ++kv_count;
         }
         if (!ok) break;
-        mma_commit(&sm.q_empty[qb]);
+        mma_commit(&sm.q_empty);
         mma_commit(&sm.dq_full);
         ++dq_count;
       }
@@ -1100,11 +1095,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
       mbar_wait(&sm.mma_done, 0);
     }
   } else {
-    // ---------------- compute warps: thread = row; warpgroup wg owns blocks [32 wg, 32 wg + 32) of a key tile
-    const int r = threadIdx.x % 128;
-    const int wg = warp / 4;
-    const int c0 = kDqCols * wg;
-    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    // ---------------- compute warpgroup: thread = row; the key tile's 64 blocks in two passes of 32
+    const int r = threadIdx.x;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     uint32_t sdp_count = 0, ds_count = 0, dq_count = 0;
     for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
       const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
@@ -1116,36 +1109,52 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
       const float2 w2 = make_float2(rc[rows + row], rc[rows + row]);
       const float2 nd2 = make_float2(rc[2 * rows + row], rc[2 * rows + row]);
       const float2 qs = make_float2(qs2, qs2);
-      const int nbt = (ti.nb + kBN - 1) / kBN;
+      const int nbt = (ti.nb + kDqBN - 1) / kDqBN;
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
         if (!mbar_wait_warp(&sm.sdp_full, sdp_count & 1)) { ok = false; break; }
         tc_fence_after();
-        float sv[kDqCols], dp[kDqCols];
-        tmem_ld32(tm_s + lane_off + c0, sv);
-        tmem_ld32(tm_dp + lane_off + c0, dp);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sdp_empty);
+        const int nvalid = ti.nb - j * kDqBN;  // valid blocks of this key tile
+        bool ok_half = true;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float sv[32], dp[32];
+          tmem_ld32(tm_s + lane_off + 32 * hh, sv);
+          tmem_ld32(tm_dp + lane_off + 32 * hh, dp);
+          tmem_ld_wait();
+          if (hh == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sdp_empty);
+          }
+          const int nvh = nvalid - 32 * hh;
+          if (nvh < 32) {  // ragged last key tile: blocks past the sequence get p = 0
+#pragma unroll
+            for (int c = 0; c < 32; ++c) sv[c] = c < nvh ? sv[c] : -CUDART_INF_F;
+          }
+          // dS = p (w dP - D), p = 2^(s qs2 - lse log2 e)
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
+            const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
+            split2(d, hi[c / 2], lo[c / 2]);
+          }
+          if (hh == 0) {
+            if (!mbar_wait_warp(&sm.ds_empty, (ds_count & 1) ^ 1)) {
+              ok_half = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          tmem_st16(tm_dsh + lane_off + 16 * hh, hi);
+          tmem_st16(tm_dsl + lane_off + 16 * hh, lo);
+        }
+        if (!ok_half) {
+          ok = false;
+          break;
+        }
         ++sdp_count;
-        const int nvalid = ti.nb - (j * kBN + c0);  // valid blocks of this warpgroup's columns
-        if (nvalid < kDqCols) {  // ragged last key tile: blocks past the sequence get p = 0
-#pragma unroll
-          for (int c = 0; c < kDqCols; ++c) sv[c] = c < nvalid ? sv[c] : -CUDART_INF_F;
-        }
-        // dS = p (w dP - D), p = 2^(s qs2 - lse log2 e)
-        uint32_t hi[kDqCols / 2], lo[kDqCols / 2];
-#pragma unroll
-        for (int c = 0; c < kDqCols; c += 2) {
-          const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
-          const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
-          split2(d, hi[c / 2], lo[c / 2]);
-        }
-        if (!mbar_wait_warp(&sm.ds_empty, (ds_count & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        tmem_st16(tm_dsh + lane_off + c0 / 2, hi);
-        tmem_st16(tm_dsl + lane_off + c0 / 2, lo);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -1159,32 +1168,26 @@ __global__ void __launch_bounds__(kDqThreads, 1) cmp_bwd_dq_tc_kernel(
       if (!mbar_wait_warp(&sm.dq_full, dq_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++dq_count;
       tc_fence_after();
-      float g16[16];  // warpgroup wg writes dQ columns [16 wg, 16 wg + 16)
-      tmem_ld16(tm_dq + lane_off + 16 * wg, g16);
+      float g[64];
+      tmem_ld32(tm_dq + lane_off, g);
+      tmem_ld32(tm_dq + lane_off + 32, g + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.dq_empty);
       if (valid) {
-        float4* dst = reinterpret_cast<float4*>(dq_out + row * 64 + 16 * wg);
+        float4* dst = reinterpret_cast<float4*>(dq_out + row * 64);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_float4(g16[4 * i] * scale, g16[4 * i + 1] * scale, g16[4 * i + 2] * scale,
-                               g16[4 * i + 3] * scale);
+        for (int i = 0; i < 16; ++i)
+          dst[i] = make_float4(g[4 * i] * scale, g[4 * i + 1] * scale, g[4 * i + 2] * scale, g[4 * i + 3] * scale);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
-// ---------------------------------------------------------------------------
-// backward, dKc / dVc (thread = block): S^T = Kc Q^T, dP^T = Vc dO^T in TMEM;
-// P^T w and dS^T (bf16) as TMEM A operands of dVc += (P^T w) dO and
-// dKc += dS^T Q.  A work item is (group, key tile, chunk of row tiles); its
-// partial dKc / dVc are added to the fp32 workspace with vector atomics.
-// ---------------------------------------------------------------------------
 constexpr int kDkvRowTilesPerItem = 128;
 constexpr int kDkvQStages = 3;  // Q / dO / row-constant stages: each row tile is used once per item
 // four compute warpgroups of 32 rows each (thread = block): enough warps to hide
@@ -1585,8 +1588,10 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
                          int32_t* scan_tmp, int64_t tiles_bound, cudaStream_t st) {
   CUtensorMap qm, dm, km, vm;
   const int64_t rows_kv = (int64_t)a.hkv * a.blk->count;
+  CUtensorMap km64, vm64;  // 64-block key tiles of the dQ kernel
   if (!map_q(&qm, a.q, a.N, a.hq, G) || !map_q(&dm, a.dout, a.N, a.hq, G) || !map_rows64(&km, a.kc, rows_kv) ||
-      !map_rows64(&vm, a.vc, rows_kv))
+      !map_rows64(&vm, a.vc, rows_kv) || !map_rows64(&km64, a.kc, rows_kv, kDqBN) ||
+      !map_rows64(&vm64, a.vc, rows_kv, kDqBN))
     return cudaErrorInvalidValue;
   static bool attr_done = false;
   if (!attr_done) {
@@ -1602,9 +1607,9 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
   const int btot = (int)a.blk->count;
   const int sms = num_sms();
   const int64_t tiles = tiles_bound * a.hkv;
-  const int gq = (int)(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);
+  const int gq = (int)(tiles < kDqCtasPerSm * sms ? (tiles > 0 ? tiles : 1) : kDqCtasPerSm * sms);
   const int64_t rows = a.N * a.hq;
-  SSA_LAUNCH("cmp_bwd_dq_tc_kernel", cmp_bwd_dq_tc_kernel<G>, gq, kDqThreads, smem_bytes_dq(), st, qm, dm, km, vm,
+  SSA_LAUNCH("cmp_bwd_dq_tc_kernel", cmp_bwd_dq_tc_kernel<G>, gq, kDqThreads, smem_bytes_dq(), st, qm, dm, km64, vm64,
              a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.rc, rows, a.dq, a.status);
   SSA_LAUNCH("dkv_plan_kernel", dkv_plan_kernel, (a.S + 256) / 256, 256, 0, st, a.cu_seqlens, a.blk->cu, a.S, G,
              dkv_cnt);

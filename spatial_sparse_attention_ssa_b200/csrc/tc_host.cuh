@@ -26,13 +26,13 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D map over [rows, 64] bf16 with a box of 128 rows, 128-byte swizzle.
-inline bool map_rows64(CUtensorMap* m, const void* base, int64_t rows) {
+// 2D map over [rows, 64] bf16 with a box of `box_rows` rows (128 by default), 128-byte swizzle.
+inline bool map_rows64(CUtensorMap* m, const void* base, int64_t rows, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {64, (cuuint64_t)rows};
   cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
