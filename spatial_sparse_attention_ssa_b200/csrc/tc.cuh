@@ -282,6 +282,27 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 ex2x2(float2 x) { return make_float2(ex2(x.x), ex2(x.y)); }
 
+// 2^x for x <= 0 on the FMA and integer pipes, leaving the MUFU to other elements:
+// x is clamped at -127 (the exponent field stays non-negative; smaller values read
+// as at most 2^-126), split as x = j + f with j = round(x) (via the 1.5 * 2^23
+// rounding constant) and |f| <= 1/2; 2^f is the degree-5 polynomial through 2^f at
+// the six Chebyshev nodes of [-1/2, 1/2] (relative error <= 2.5e-7 evaluated in fp32,
+// about that of ex2.approx); 2^j is added to the exponent field.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
+  const float2 j = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ffma2(j, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(1.339086331e-03f, 1.339086331e-03f), f, make_float2(9.676031768e-03f, 9.676031768e-03f));
+  p = ffma2(p, f, make_float2(5.550356954e-02f, 5.550356954e-02f));
+  p = ffma2(p, f, make_float2(2.402210683e-01f, 2.402210683e-01f));
+  p = ffma2(p, f, make_float2(6.931471825e-01f, 6.931471825e-01f));
+  p = ffma2(p, f, make_float2(1.000000119e+00f, 1.000000119e+00f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // x = hi + lo as two bf16 pairs, with integer and FMA-pipe instructions only (the
 // fp32 -> bf16 conversion instructions issue at a quarter of the FMA rate): hi is x
 // truncated to its upper 16 bits, lo = x - hi exactly in fp32, then rounded to bf16
