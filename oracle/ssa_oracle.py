@@ -460,3 +460,37 @@ def window_kv_grads(st: State, dout: np.ndarray, windows) -> tuple:
         dks.append(dk)
         dvs.append(dv)
     return np.concatenate(toks), np.concatenate(dks), np.concatenate(dvs)
+
+
+# ----------------------------------------------------------------------------
+# 3D-aware block routing (selection by geometric distance instead of scores)
+# ----------------------------------------------------------------------------
+
+
+def geo_topk(coords: np.ndarray, cu_seqlens: np.ndarray, m_cmp: int, k: int, tokens=None) -> np.ndarray:
+    """Selection by explicit geometric distance (LSRM, shuwu5.cn/article/2502.html,
+    "3D 感知空间块路由机制", voxel-only case): a voxel token's point is the centre of
+    its voxel; the distance of a query token to a block is the shortest Euclidean
+    distance to the points of the block's tokens; each token selects the k blocks of
+    its sequence nearest to it (ties: lower block id), stored ascending, padded -1.
+
+    Voxel centres differ by integer vectors, so squared distances are exact integers.
+    Returns global block ids [len(tokens), k] (all tokens by default)."""
+    coords = np.asarray(coords, np.int64)
+    cu = np.asarray(cu_seqlens, np.int64)
+    blk = bin_tokens(coords, cu, m_cmp)
+    n = len(coords)
+    tokens = np.arange(n) if tokens is None else np.asarray(tokens, np.int64)
+    seq = _seq_of_tokens(cu, n)
+    out = np.full((len(tokens), k), -1, np.int64)
+    for row, t in enumerate(tokens):
+        s = seq[t]
+        b0, b1 = int(blk["cu"][s]), int(blk["cu"][s + 1])
+        members = np.arange(cu[s], cu[s + 1])
+        d2 = np.sum((coords[members] - coords[t]) ** 2, axis=1)
+        best = np.full(b1 - b0, np.iinfo(np.int64).max)
+        np.minimum.at(best, blk["id"][members] - b0, d2)
+        keff = min(k, b1 - b0)
+        order = np.lexsort((np.arange(b1 - b0), best))[:keff]  # by distance, then by id
+        out[row, :keff] = np.sort(order) + b0
+    return out

@@ -476,3 +476,59 @@ def test_dgates_rows_and_window_grads_match_full_backward():
     np.testing.assert_array_equal(np.sort(tk), np.sort(members))
     np.testing.assert_allclose(dk, g["parts"]["dk"]["win"][tk], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(dv, g["parts"]["dv"]["win"][tk], rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# geometric block routing
+# ----------------------------------------------------------------------------
+
+def _geo_brute(coords, cu, m, k):
+    """Python loops over every (token, block, member) triple."""
+    out = []
+    cells = {}
+    for s in range(len(cu) - 1):
+        keys = sorted({tuple(int(c) // m for c in coords[i]) for i in range(cu[s], cu[s + 1])})
+        cells[s] = keys
+    base = 0
+    for s in range(len(cu) - 1):
+        keys = cells[s]
+        for t in range(cu[s], cu[s + 1]):
+            dist = []
+            for j, key in enumerate(keys):
+                dmin = min(sum((int(coords[i][a]) - int(coords[t][a])) ** 2 for a in range(3))
+                           for i in range(cu[s], cu[s + 1]) if tuple(int(c) // m for c in coords[i]) == key)
+                dist.append((dmin, j))
+            picks = sorted(j for _, j in sorted(dist)[:k])
+            out.append([base + j for j in picks] + [-1] * (k - len(picks)))
+        base += len(keys)
+    return np.array(out)
+
+
+def test_geo_topk_matches_brute_force_with_ties_and_short_sequences():
+    rng = np.random.default_rng(4)
+    pts = np.unique(rng.integers(0, 12, size=(120, 3)), axis=0)[:90]
+    coords = np.concatenate([pts, pts[:7] + 1])  # a short second sequence
+    cu = np.array([0, 90, 97])
+    for k in (1, 3, 40):
+        np.testing.assert_array_equal(O.geo_topk(coords, cu, 4, k), _geo_brute(coords, cu, 4, k))
+
+
+def test_geo_topk_hand_example():
+    # blocks of edge 2 along x: {0,1} | {2,3} | {4,5} | {8,9}; query at x = 3
+    coords = np.array([[0, 0, 0], [3, 0, 0], [5, 0, 0], [9, 0, 0], [1, 1, 0]])
+    cu = np.array([0, 5])
+    # distances^2 from token 1 (3,0,0): block0 min(9, 5)=5, block1 0, block2 4, block4 36
+    np.testing.assert_array_equal(O.geo_topk(coords, cu, 2, 2, tokens=[1]), [[1, 2]])
+    np.testing.assert_array_equal(O.geo_topk(coords, cu, 2, 3, tokens=[1]), [[0, 1, 2]])
+    # a tie (token 4 at (1,1,0): block0 0, block1 (3,0,0): 4+1=5, block2 16+1=17 ... ) and k=1
+    np.testing.assert_array_equal(O.geo_topk(coords, cu, 2, 1, tokens=[4]), [[0]])
+
+
+def test_geo_topk_own_block_always_selected_and_permutation_invariant():
+    w, t = _small_workload(seed=8, n_seqs=2)
+    sel = O.geo_topk(w.coords, w.cu_seqlens, w.m_cmp, w.topk)
+    blk = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)
+    assert all(blk["id"][i] in sel[i] for i in range(w.n))
+    w2, _, src = W.permute_workload(w, t, seed=3)
+    sel2 = O.geo_topk(w2.coords, w2.cu_seqlens, w2.m_cmp, w2.topk)
+    np.testing.assert_array_equal(sel2, sel[src])
