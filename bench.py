@@ -70,6 +70,7 @@ def _args():
                     help="tokens of the 1024^3 workload (131072 is the benchmark; smaller only for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-geo", action="store_true", help="skip the separate timing of geometric block routing")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -390,6 +391,27 @@ def run_ours(a):
                     "frac": achieved / peak, "traffic": None, "peak_source": peaks["_source"],
                     "algorithmic_per_launch": units, "ms_per_launch": avg_ms}
 
+    # ---- geometric block routing (selection by voxel distance), timed on its own
+    geo = None
+    if not a.no_geo:
+        sel_geo = torch.empty((n, w.hkv, w.topk), dtype=torch.int32, device=dev)
+        ws_geo = torch.empty(ssa.lib().ssa_workspace_size(ssa.OP_GEO_SELECT, None, s, n, blk.count, 0),
+                             dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            ssa.ssa_geo_select(coords, cu, w.R, blk, w.m_cmp, w.topk, w.hkv, out=sel_geo, workspace=ws_geo)
+        check_device("geometric routing warm-up")
+        eg = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+        for i in range(a.steps):
+            flush.zero_()
+            eg[i][0].record()
+            ssa.ssa_geo_select(coords, cu, w.R, blk, w.m_cmp, w.topk, w.hkv, out=sel_geo, workspace=ws_geo)
+            eg[i][1].record()
+        torch.cuda.synchronize()
+        check_device("geometric routing")
+        g_ms = sum(a_.elapsed_time(b_) for a_, b_ in eg) / a.steps
+        geo = {"ms_per_call": g_ms, "tokens_per_s": n / (g_ms / 1e3), "blocks": int(blk.count),
+               "topk": int(w.topk), "launches_per_call": 2}
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -406,7 +428,7 @@ def run_ours(a):
                 "data": "synthetic (seeded surface-shell voxels, N(0,1) bf16 Q/K/V/dO, N(0,1) gate logits)",
                 "config": cfg, "roofline": roof, "roofline_exp": exp_roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(launches),
-                "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel,
+                "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel, "geo_routing": geo,
                 "peaks_source": peaks["_source"]}
         print(json.dumps(line), flush=True)
     if world > 1:

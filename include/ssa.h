@@ -56,7 +56,7 @@ typedef enum ssa_status {
 
 enum { SSA_DTYPE_BF16 = 0, SSA_DTYPE_F32 = 1 };
 enum { SSA_GATE_WEIGHTS = 0, SSA_GATE_LOGITS = 1 };
-enum { SSA_OP_BIN = 0, SSA_OP_FORWARD = 1, SSA_OP_BACKWARD = 2 };
+enum { SSA_OP_BIN = 0, SSA_OP_FORWARD = 1, SSA_OP_BACKWARD = 2, SSA_OP_GEO_SELECT = 3 };
 
 /* Shape and method parameters shared by forward and backward. */
 typedef struct ssa_params {
@@ -141,6 +141,27 @@ SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int
 SSA_API ssa_status ssa_bin_noalloc(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N,
                                    int32_t R, int32_t m_cmp, int32_t m_win, ssa_partition* blk,
                                    ssa_partition* win, void* stream);
+
+/*
+ * ssa_geo_select -- 3D-aware block routing (LSRM "3D 感知空间块路由机制", voxel-only
+ * case: no camera projection): every token selects the topk blocks of its
+ * sequence nearest to it, the distance to a block being the shortest Euclidean
+ * distance between the token's voxel centre and the voxel centres of the block's
+ * tokens; ties go to the lower block id; k_eff = min(topk, blocks in the
+ * sequence).  Squared distances are exact integers: bit-exact integer work.
+ *   coords   int32 [N, 3] device, 0 <= x, y, z < R, R <= 32768
+ *   blk      block partition from ssa_bin with edge m_cmp (device arrays)
+ *   sel      int32 [N, hkv, topk] device, caller-owned: global block ids,
+ *            ascending, padded with -1; the same selection for every KV group
+ *            (the layout of ssa_saved.sel)
+ *   ws       device workspace of ssa_workspace_size(SSA_OP_GEO_SELECT, ...) bytes
+ * Asynchronous.  SSA_ERR_INVALID_ARG for null pointers or bad sizes (topk must be
+ * in 1..32), SSA_ERR_UNSUPPORTED for R > 32768, SSA_ERR_WORKSPACE if ws_bytes is
+ * too small; all are found on the host before anything is enqueued.
+ */
+SSA_API ssa_status ssa_geo_select(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                                  int32_t R, const ssa_partition* blk, int32_t m_cmp, int32_t topk,
+                                  int32_t hkv, int32_t* sel, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * ssa_forward -- steps 2-6: mean-pool compression; compressed attention of every

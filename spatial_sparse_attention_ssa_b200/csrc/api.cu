@@ -150,6 +150,7 @@ SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, in
                                   int64_t W_tot) {
   if (S < 0 || N < 0 || B_tot < 0 || W_tot < 0) return 0;
   if (op == SSA_OP_BIN) return bin_bytes(S, N);
+  if (op == SSA_OP_GEO_SELECT) return ssa::geo_ws_bytes(N);
   if (check_params(p) != SSA_OK) return 0;
   if (op == SSA_OP_FORWARD) return fwd_bytes(p, S, N, B_tot, W_tot);
   if (op == SSA_OP_BACKWARD) {
@@ -157,6 +158,20 @@ SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, in
     return carve_bwd(nullptr, p, S, N, B_tot, W_tot, &w);
   }
   return 0;
+}
+
+SSA_API ssa_status ssa_geo_select(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N, int32_t R,
+                                  const ssa_partition* blk, int32_t m_cmp, int32_t topk, int32_t hkv, int32_t* sel,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || R < 1 || m_cmp < 1 || topk < 1 || topk > 32 || hkv < 1)
+    return SSA_ERR_INVALID_ARG;
+  if (R > 32768) return SSA_ERR_UNSUPPORTED;  // squared distances must fit 32 bits
+  if (N == 0) return SSA_OK;
+  if (!coords || !cu_seqlens || !partition_ok(blk) || !sel || !ws) return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > N) return SSA_ERR_INVALID_ARG;
+  if (ws_bytes < ssa::geo_ws_bytes(N)) return SSA_ERR_WORKSPACE;
+  return cuda_status(ssa::geo_select(coords, cu_seqlens, S, N, blk, m_cmp, topk, hkv, sel, ws,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 SSA_API ssa_status ssa_get_device_status(void* stream) {

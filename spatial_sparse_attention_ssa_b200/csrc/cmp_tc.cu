@@ -248,7 +248,6 @@ constexpr int kTopkMax = 32;
 constexpr int kOutStages = 3;
 constexpr int kCandMax = 128;  // top-k candidates per token kept for exact ranking
 constexpr int kComputeWarps = 8;  // pass 2: two warpgroups of compute warps
-constexpr int kOutThreads = 32 * (kComputeWarps + 2);  // + TMA warp + MMA warp
 // pass 2 adds a warpgroup that picks the top-k of the previous row tile while the
 // compute warps work on the next one (the importance scratch is double-buffered)
 constexpr int kOutTopkWarps = 4;

@@ -85,6 +85,11 @@ cudaError_t cmp_bwd_tc(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, 
                        int64_t tiles_bound, cudaStream_t st);
 cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st);
 
+// 3D-aware block routing: selection by the shortest distance to a block's voxels.
+size_t geo_ws_bytes(int64_t N);
+cudaError_t geo_select(const int32_t* coords, const int32_t* cu_seqlens, int S, int64_t N, const ssa_partition* blk,
+                       int m, int topk, int hkv, int32_t* sel, void* ws, cudaStream_t st);
+
 // Selected-block branch on warp-level MMAs (bf16, head dim 64, G in {8, 16}, top-k <= 32).
 bool slc_mma_supported(int dtype, int d, int hq, int hkv, int topk);
 cudaError_t slc_fwd_mma(const FwdArgs& a, cudaStream_t st);

@@ -23,11 +23,11 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
                 4: "SSA_ERR_COORD_RANGE", 5: "SSA_ERR_CUDA", 6: "SSA_ERR_TIMEOUT"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 GATE_WEIGHTS, GATE_LOGITS = 0, 1
-OP_BIN, OP_FORWARD, OP_BACKWARD = 0, 1, 2
+OP_BIN, OP_FORWARD, OP_BACKWARD, OP_GEO_SELECT = 0, 1, 2, 3
 
 EXPORTS = ("ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size", "ssa_error_string",
            "ssa_get_device_status", "ssa_version", "ssa_launch_count", "ssa_profile_enable",
-           "ssa_profile_read")
+           "ssa_profile_read", "ssa_geo_select")
 
 
 class SSAError(RuntimeError):
@@ -73,6 +73,8 @@ def _lib():
         lib.ssa_backward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, pp, pp, vp, vp, vp, vp,
                                      ctypes.POINTER(Saved), vp, vp, vp, vp, vp, vp, sz, vp]
         lib.ssa_backward.restype = ctypes.c_int
+        lib.ssa_geo_select.argtypes = [vp, vp, i32, i64, i32, pp, i32, i32, i32, vp, vp, sz, vp]
+        lib.ssa_geo_select.restype = ctypes.c_int
         lib.ssa_workspace_size.argtypes = [i32, ctypes.POINTER(Params), i32, i64, i64, i64]
         lib.ssa_workspace_size.restype = sz
         lib.ssa_error_string.argtypes = [ctypes.c_int]
@@ -165,6 +167,26 @@ def ssa_bin(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cmp: int, 
     blk.count = int(pb.count)
     win.count = int(pw.count)
     return blk, win
+
+
+def ssa_geo_select(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, blk: "Bins", m_cmp: int, topk: int,
+                   hkv: int, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """3D-aware block routing: the topk blocks nearest to each token (shortest
+    distance between voxel centres; ties to the lower id), int32 [N, hkv, topk]
+    global block ids, ascending, padded with -1, the same for every KV group."""
+    _require_cuda(coords, cu_seqlens)
+    n = int(coords.shape[0])
+    s = int(cu_seqlens.shape[0]) - 1
+    dev = coords.device
+    sel = out if out is not None else torch.empty((n, hkv, topk), dtype=torch.int32, device=dev)
+    L = _lib()
+    need = L.ssa_workspace_size(OP_GEO_SELECT, None, s, n, blk.count, 0)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb = blk.c()
+    st = L.ssa_geo_select(_ptr(coords), _ptr(cu_seqlens), s, n, int(R), ctypes.byref(pb), int(m_cmp), int(topk),
+                          int(hkv), _ptr(sel), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ssa_geo_select")
+    return sel
 
 
 def ssa_bin_noalloc(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cmp: int, m_win: int,

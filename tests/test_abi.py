@@ -73,3 +73,20 @@ def test_bin_rejects_bad_arguments_before_launching():
     # sequence bits + 3 x cell bits above 64: 2^20 grid with unit cells and 2^5 sequences
     assert lib.ssa_bin(1, 1, 32, 10, 1 << 20, 1, 1, ctypes.byref(part), ctypes.byref(part), 1, 1 << 30,
                        None) == 2
+
+
+def test_geo_select_argument_errors_are_found_on_the_host():
+    lib = ssa.lib()
+    part = ssa.Partition(1, 1, 1, 1, 1, 10)
+    assert lib.ssa_workspace_size(ssa.OP_GEO_SELECT, None, 1, 1000, 100, 0) >= 16 * 1000
+    ok = dict(coords=1, cu=1, S=1, N=100, R=64, m=4, topk=8, hkv=2, sel=1, ws=1, ws_bytes=1 << 20)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.ssa_geo_select(a["coords"], a["cu"], a["S"], a["N"], a["R"], ctypes.byref(part), a["m"],
+                                  a["topk"], a["hkv"], a["sel"], a["ws"], a["ws_bytes"], None)
+    assert call(topk=0) == 1 and call(topk=33) == 1 and call(hkv=0) == 1 and call(m=0) == 1
+    assert call(S=0) == 1 and call(N=-1) == 1 and call(sel=None) == 1
+    assert call(R=40000) == 2                    # squared distances must fit 32 bits
+    assert call(ws_bytes=100) == 3               # workspace too small
+    assert call(N=0) == 0                        # nothing to do

@@ -1,0 +1,80 @@
+"""3D-aware geometric block routing on the GPU against the oracle, bit-exact.
+
+The selection is decided by integer squared distances between voxel centres, so
+the CUDA path and the oracle must agree exactly, ties included (lower block id):
+  * every token of small multi-sequence shells, topk 1 / 4 / 16 / 32, blocks of
+    4^3 and 8^3, fewer blocks than topk in the short sequences;
+  * an empty sequence between two others, and a one-token sequence;
+  * a token whose 696 nearest blocks tie (lattice points on one sphere, one voxel
+    per block): more candidates than the kernel keeps in shared memory, so the
+    exhaustive path runs, and the tie order decides all but one pick;
+  * sampled tokens of the 131072-token benchmark shape.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import ssa_oracle as O
+from spatial_sparse_attention_ssa_b200 import ssa
+from spatial_sparse_attention_ssa_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_select(coords, cu, R, m, topk, hkv=2):
+    c = torch.from_numpy(np.ascontiguousarray(coords, np.int32)).cuda()
+    s = torch.from_numpy(np.asarray(cu, np.int32)).cuda()
+    blk, _ = ssa.ssa_bin(c, s, R, m, m)
+    sel = ssa.ssa_geo_select(c, s, R, blk, m, topk, hkv)
+    torch.cuda.synchronize()
+    assert ssa.device_status() == 0
+    out = sel.cpu().numpy()
+    for g in range(1, hkv):
+        np.testing.assert_array_equal(out[:, g], out[:, 0])
+    return out[:, 0]
+
+
+@pytest.mark.parametrize("m,topk", [(4, 1), (4, 4), (4, 16), (8, 32), (4, 32)])
+def test_every_token_of_small_shells(m, topk):
+    w = W.small_shell(seed=11 + topk, R=48, n_prims=2, lo=4.0, hi=11.0, n_keep=900, n_seqs=3, m_cmp=m)
+    got = _gpu_select(w.coords, w.cu_seqlens, w.R, m, topk)
+    want = O.geo_topk(w.coords, w.cu_seqlens, m, topk)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_empty_and_single_token_sequences():
+    w = W.small_shell(seed=5, R=40, n_prims=1, lo=4.0, hi=9.0, n_keep=400, n_seqs=2, m_cmp=4)
+    a = int(w.cu_seqlens[1])
+    coords = np.concatenate([w.coords, np.array([[3, 7, 9]], np.int32)])
+    cu = np.array([0, a, a, len(w.coords), len(coords)], np.int32)  # sequence 1 empty, 3 has one token
+    got = _gpu_select(coords, cu, w.R, 4, 8)
+    want = O.geo_topk(coords, cu, 4, 8)
+    np.testing.assert_array_equal(got, want)
+    assert (got[-1, 1:] == -1).all()
+
+
+def test_ties_beyond_the_shared_memory_candidate_list():
+    g = np.arange(-36, 37)
+    x, y, z = np.meshgrid(g, g, g, indexing="ij")
+    on = (x * x + y * y + z * z) == 1286
+    ring = np.stack([x[on], y[on], z[on]], 1) + 36
+    coords = np.concatenate([np.array([[36, 36, 36]]), ring]).astype(np.int32)
+    assert len(coords) == 697
+    cu = np.array([0, len(coords)], np.int32)
+    for topk in (16, 32):
+        got = _gpu_select(coords, cu, 73, 1, topk, hkv=1)
+        want = O.geo_topk(coords, cu, 1, topk)
+        np.testing.assert_array_equal(got, want)
+
+
+def test_sampled_tokens_at_benchmark_size():
+    w = W.config(5)
+    got = _gpu_select(w.coords, w.cu_seqlens, w.R, w.m_cmp, w.topk, hkv=w.hkv)
+    rng = np.random.default_rng(17)
+    toks = np.unique(np.concatenate([[0, w.n - 1], rng.choice(w.n, 160, replace=False)]))
+    want = O.geo_topk(w.coords, w.cu_seqlens, w.m_cmp, w.topk, tokens=toks)
+    np.testing.assert_array_equal(got[toks], want)
+    # at any size: a token's own block is always picked, ids ascend within a row
+    b = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)
+    assert (got == b["id"][:, None]).any(1).all()
+    assert (np.diff(got, axis=1) > 0).all()
