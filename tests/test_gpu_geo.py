@@ -5,9 +5,10 @@ the CUDA path and the oracle must agree exactly, ties included (lower block id):
   * every token of small multi-sequence shells, topk 1 / 4 / 16 / 32, blocks of
     4^3 and 8^3, fewer blocks than topk in the short sequences;
   * an empty sequence between two others, and a one-token sequence;
-  * a token whose 696 nearest blocks tie (lattice points on one sphere, one voxel
-    per block): more candidates than the kernel keeps in shared memory, so the
-    exhaustive path runs, and the tie order decides all but one pick;
+  * a token whose 696 or 4368 nearest blocks tie (lattice points on one sphere,
+    one voxel per block): more candidates than the kernel keeps in shared memory
+    for one token, or for one query block, so the exhaustive paths run, and the tie
+    order decides all but one pick;
   * sampled tokens of the 131072-token benchmark shape.
 """
 import numpy as np
@@ -53,16 +54,31 @@ def test_empty_and_single_token_sequences():
     assert (got[-1, 1:] == -1).all()
 
 
-def test_ties_beyond_the_shared_memory_candidate_list():
-    g = np.arange(-36, 37)
-    x, y, z = np.meshgrid(g, g, g, indexing="ij")
-    on = (x * x + y * y + z * z) == 1286
-    ring = np.stack([x[on], y[on], z[on]], 1) + 36
-    coords = np.concatenate([np.array([[36, 36, 36]]), ring]).astype(np.int32)
-    assert len(coords) == 697
+def _sphere(n2: int) -> np.ndarray:
+    """Integer points (x, y, z) with x^2 + y^2 + z^2 = n2."""
+    r = int(np.sqrt(n2))
+    g = np.arange(-r, r + 1)
+    x, y = np.meshgrid(g, g, indexing="ij")
+    z2 = n2 - x * x - y * y
+    ok = z2 >= 0
+    z = np.rint(np.sqrt(np.where(ok, z2, 0))).astype(np.int64)
+    ok &= z * z == z2
+    pos = np.stack([x[ok], y[ok], z[ok]], 1)
+    neg = pos[pos[:, 2] > 0] * np.array([1, 1, -1])
+    return np.concatenate([pos, neg])
+
+
+@pytest.mark.parametrize("n2,npts", [(1286, 696), (38246, 4368)])
+def test_ties_beyond_the_shared_memory_candidate_lists(n2, npts):
+    """A token at the centre of a lattice sphere, one voxel per block: all sphere
+    blocks tie.  696 ties overflow the per-token list, 4368 the per-query-block list."""
+    ring = _sphere(n2)
+    assert len(ring) == npts
+    c = int(np.sqrt(n2)) + 1
+    coords = (np.concatenate([np.zeros((1, 3), np.int64), ring]) + c).astype(np.int32)
     cu = np.array([0, len(coords)], np.int32)
     for topk in (16, 32):
-        got = _gpu_select(coords, cu, 73, 1, topk, hkv=1)
+        got = _gpu_select(coords, cu, 2 * c + 1, 1, topk, hkv=1)
         want = O.geo_topk(coords, cu, 1, topk)
         np.testing.assert_array_equal(got, want)
 
