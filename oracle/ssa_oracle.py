@@ -192,9 +192,13 @@ class State(dict):
 
 
 def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
-            gate_mode, scale=None, pool_rounding="bf16", tokens=None, chunk=256) -> State:
+            gate_mode, scale=None, pool_rounding="bf16", tokens=None, chunk=256, sel_given=None) -> State:
     """SSA forward.  q [N, Hq, d], k/v [N, Hkv, d] (any float type; converted to
     float64), gates [N, Hq, 3].
+
+    `sel_given` ([N, Hkv, topk] global block ids or -1) replaces the score top-k:
+    the selected branch attends the tokens of those blocks instead (a routing by
+    geometry, LSRM "3D 感知空间块路由机制", is one source of such a selection).
 
     `tokens` restricts the per-query outputs (lse, o_*, sel, O) to a subset of
     query tokens (all other rows are NaN / -2); binning and compression are
@@ -240,9 +244,12 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
                 l_, o_, p_ = cmp_attention(qrows(tt, hs), kcg, vcg, scale)
                 lse[0, tt, hs] = l_
                 o[0, tt, hs, :] = o_
-                imp = p_.sum(axis=1)  # [n, B_s]: probabilities summed over the group's heads
-                loc = topk_blocks(imp, topk)
-                sel[tt, g, :] = np.where(loc >= 0, loc + b0, -1)
+                if sel_given is None:
+                    imp = p_.sum(axis=1)  # [n, B_s]: probabilities summed over the group's heads
+                    loc = topk_blocks(imp, topk)
+                    sel[tt, g, :] = np.where(loc >= 0, loc + b0, -1)
+    if sel_given is not None:
+        sel[tokens] = np.asarray(sel_given, np.int64)[tokens]
 
     # --- selected-block attention and window attention, per query token and group
     for t in tokens:

@@ -532,3 +532,42 @@ def test_geo_topk_own_block_always_selected_and_permutation_invariant():
     w2, _, src = W.permute_workload(w, t, seed=3)
     sel2 = O.geo_topk(w2.coords, w2.cu_seqlens, w2.m_cmp, w2.topk)
     np.testing.assert_array_equal(sel2, sel[src])
+
+
+def test_given_selection_of_every_block_is_full_attention():
+    """A given selection listing every block of the token's sequence (in descending
+    order, padding first) makes the selected branch full attention."""
+    coords, cu, q, k, v, gates = _rand_case(13)
+    b = O.bin_tokens(coords, cu, 4)
+    nb = np.diff(b["cu"])
+    k_sel = int(nb.max()) + 2
+    sel = np.full((len(coords), 2, k_sel), -1, np.int64)
+    for t in range(len(coords)):
+        s = int(np.searchsorted(cu, t, side="right") - 1)
+        ids = np.arange(b["cu"][s], b["cu"][s + 1])[::-1]
+        sel[t, :, k_sel - len(ids):] = ids
+    st = O.forward(coords, cu, q, k, v, gates, hq=4, hkv=2, m_cmp=4, m_win=4, topk=k_sel, gate_mode=1,
+                   sel_given=sel)
+    np.testing.assert_allclose(st["o"][1], _sdpa_full(q, k, v, cu, 4, 2), rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(st["sel"], sel)
+
+
+def test_geometric_selection_backward_matches_autograd():
+    """The geometric routing as the selection: the forward and its backward against
+    autograd of the dense re-expression built from that selection."""
+    coords, cu, q, k, v, gates = _rand_case(17, n_per_seq=(48, 30), R=8, hq=4, hkv=2, d=8, unique=False)
+    geo = O.geo_topk(coords, cu, 2, 3)
+    sel = np.repeat(geo[:, None, :], 2, axis=1)
+    st = O.forward(coords, cu, q, k, v, gates, hq=4, hkv=2, m_cmp=2, m_win=4, topk=3, gate_mode=1,
+                   pool_rounding="none", sel_given=sel)
+    ref = O.forward(coords, cu, q, k, v, gates, hq=4, hkv=2, m_cmp=2, m_win=4, topk=3, gate_mode=1,
+                    pool_rounding="none")
+    assert (st["sel"] != ref["sel"]).any()  # the two routings differ on this case
+    np.testing.assert_array_equal(st["o"][0], ref["o"][0])  # the compressed branch does not depend on it
+    out, (qt, kt, vt, gt) = _torch_reexpression(coords, cu, q, k, v, gates, st, 1, st["scale"])
+    np.testing.assert_allclose(out.detach().numpy(), st["out"], rtol=1e-12, atol=1e-12)
+    do = np.random.default_rng(5).standard_normal(q.shape)
+    (out * torch.from_numpy(do)).sum().backward()
+    g = O.backward(st, do)
+    for key, tt in (("dq", qt), ("dk", kt), ("dv", vt), ("dgates", gt)):
+        np.testing.assert_allclose(g[key], tt.grad.numpy(), rtol=1e-10, atol=1e-12)
