@@ -56,6 +56,8 @@ typedef enum ssa_status {
 
 enum { SSA_DTYPE_BF16 = 0, SSA_DTYPE_F32 = 1 };
 enum { SSA_GATE_WEIGHTS = 0, SSA_GATE_LOGITS = 1 };
+/* where the selected branch's blocks come from (ssa_params.selection) */
+enum { SSA_SEL_SCORES = 0, SSA_SEL_GIVEN = 1 };
 enum { SSA_OP_BIN = 0, SSA_OP_FORWARD = 1, SSA_OP_BACKWARD = 2, SSA_OP_GEO_SELECT = 3 };
 
 /* Shape and method parameters shared by forward and backward. */
@@ -69,6 +71,9 @@ typedef struct ssa_params {
   float scale;       /* softmax scale; 0 means 1/sqrt(d) */
   int32_t dtype;     /* SSA_DTYPE_BF16 (bf16 storage, fp32 math) or SSA_DTYPE_F32 */
   int32_t gate_mode; /* SSA_GATE_WEIGHTS: gates are the weights; SSA_GATE_LOGITS: weight = sigmoid(gate) */
+  int32_t selection; /* SSA_SEL_SCORES: the forward selects by compressed-attention score (top-k) and writes
+                        saved->sel; SSA_SEL_GIVEN: saved->sel is an input the caller filled (for instance by
+                        ssa_geo_select), read by the selected branch and the backward, see ssa_forward */
 } ssa_params;
 
 /*
@@ -174,6 +179,15 @@ SSA_API ssa_status ssa_geo_select(const int32_t* coords, const int32_t* cu_seqle
  *   (branch order: compressed, selected, window); out [N, Hq, d] dtype.
  *   blk/win: partitions from ssa_bin with the same m_cmp / m_win.
  * Asynchronous.  Writes every buffer of `saved`.
+ * With params->selection == SSA_SEL_GIVEN the top-k step is skipped and
+ * saved->sel is read instead: [N, Hkv, topk] int32, each entry a global id of
+ * a block of the token's own sequence or -1 (any order, any padding position;
+ * a block listed twice is attended twice).  This is how a routing other than
+ * the score top-k (LSRM "3D 感知空间块路由机制": ssa_geo_select) replaces the
+ * selection; the backward then holds that selection fixed as usual.  Every
+ * entry is checked on the device before use: an id outside the token's
+ * sequence is replaced by -1 and ssa_get_device_status then reports
+ * SSA_ERR_INVALID_ARG.
  */
 SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
                                const ssa_partition* blk, const ssa_partition* win, const void* q,

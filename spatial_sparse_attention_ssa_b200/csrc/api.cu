@@ -40,6 +40,7 @@ ssa_status check_params(const ssa_params* p) {
   if (p->m_cmp < 1 || p->m_win < 1 || p->topk < 1) return SSA_ERR_INVALID_ARG;
   if (p->dtype != SSA_DTYPE_BF16 && p->dtype != SSA_DTYPE_F32) return SSA_ERR_INVALID_ARG;
   if (p->gate_mode != SSA_GATE_WEIGHTS && p->gate_mode != SSA_GATE_LOGITS) return SSA_ERR_INVALID_ARG;
+  if (p->selection != SSA_SEL_SCORES && p->selection != SSA_SEL_GIVEN) return SSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.f) || isinf(p->scale)) return SSA_ERR_INVALID_ARG;
   if (p->d != 32 && p->d != 64) return SSA_ERR_UNSUPPORTED;
   if (p->topk > 32) return SSA_ERR_UNSUPPORTED;
@@ -187,6 +188,7 @@ SSA_API ssa_status ssa_get_device_status(void* stream) {
   }
   if (h & ssa::kStatusTimeout) return SSA_ERR_TIMEOUT;
   if (h & (ssa::kStatusCoordRange | ssa::kStatusSeqlens)) return SSA_ERR_COORD_RANGE;
+  if (h & ssa::kStatusSelection) return SSA_ERR_INVALID_ARG;
   return SSA_OK;
 }
 
@@ -266,6 +268,7 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   a.hkv = p->hkv;
   a.topk = p->topk;
   a.gate_mode = p->gate_mode;
+  a.sel_given = p->selection == SSA_SEL_GIVEN;
   a.m_cmp = p->m_cmp;
   a.m_win = p->m_win;
   a.use_tc = tc_enabled();

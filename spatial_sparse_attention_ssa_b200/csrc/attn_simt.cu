@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(128) cmp_out_topk_kernel(
         axpy32(o, p, sv + j * C::KSTR + sub * 36);
         float imp = p;
         for (int off = C::NT; off < G * C::NT; off <<= 1) imp += __shfl_xor_sync(0xffffffffu, imp, off);
-        if (leader && valid) {
+        if (leader && valid && sel) {
           const int bid = b0 + c0 + j;
           if (cnt < keff) {
             tv[tok][cnt] = imp;
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(128) cmp_out_topk_kernel(
     }
     if (valid) {
       store32(o_out + (t * hq + h) * D + sub * 32, o);
-      if (leader) {
+      if (leader && sel) {
         int* ids = ti[tok];
         for (int i = 1; i < keff; ++i) {  // insertion sort, ascending ids
           const int x = ids[i];
@@ -1093,6 +1093,25 @@ __global__ void cmp_scatter_kernel(const float* __restrict__ dkc, const float* _
 }
 
 // inverted selection: key (g * btot + b) per (token, group, slot), sentinel for -1
+// A selection given by the caller: every entry must be -1 or a block of the token's
+// own sequence; anything else becomes -1 and is reported in the device check word.
+__global__ void sel_check_kernel(int32_t* __restrict__ sel, int64_t N, int hkv, int topk,
+                                 const int32_t* __restrict__ cu, int S, const int32_t* __restrict__ bcu,
+                                 int* __restrict__ status) {
+  const int64_t total = N * hkv * topk;
+  bool bad = false;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t b = sel[i];
+    if (b == -1) continue;
+    const int s = find_segment(cu, S, i / ((int64_t)hkv * topk));
+    if (b < bcu[s] || b >= bcu[s + 1]) {
+      sel[i] = -1;
+      bad = true;
+    }
+  }
+  if (bad) atomicOr(status, kStatusSelection);
+}
+
 __global__ void sel_keys_kernel(const int32_t* __restrict__ sel, int64_t N, int hkv, int topk, int64_t btot,
                                 uint64_t* __restrict__ keys, int32_t* __restrict__ vals) {
   const int64_t total = N * hkv * topk;
@@ -1150,6 +1169,9 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   const T* kc = static_cast<const T*>(a.kc);
   const T* vc = static_cast<const T*>(a.vc);
   float* ob = static_cast<float*>(a.o_branch);
+  if (a.sel_given)
+    SSA_LAUNCH("sel_check_kernel", sel_check_kernel, grid_1d(a.N * a.hkv * a.topk, 256, 148 * 32), 256, 0, st, a.sel,
+               a.N, a.hkv, a.topk, a.cu_seqlens, a.S, a.blk->cu, a.status);
   // plan
   SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu, a.S, G, C::ROWS, C::ROWS,
                                                             kCmpRowChunk, a.tiles_cnt, a.items_cnt);
@@ -1169,7 +1191,8 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     SSA_LAUNCH("cmp_lse_kernel", (cmp_lse_kernel<T, D>), g2, 128, 0, st, q, kc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
                                              a.blk->count, qs2, a.lse);
     SSA_LAUNCH("cmp_out_topk_kernel", (cmp_out_topk_kernel<T, D>), g2, 128, 0, st, q, kc, vc, a.cu_seqlens, a.blk->cu, a.tiles_pre, a.S, a.hq, a.hkv,
-                                                  a.blk->count, qs2, a.lse, ob, a.topk, a.sel);
+                                                  a.blk->count, qs2, a.lse, ob, a.topk,
+                                                  a.sel_given ? nullptr : a.sel);
   }
   if (a.use_tc && D == 64 && slc_mma_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
     e = slc_fwd_mma(a, st);

@@ -926,7 +926,7 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_out_tc_kernel(
       const float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
       for (int tk = tw; tk < TPT; tk += kOutTopkWarps) {
         const int64_t t = ti.t0 + tk;
-        if (t < ti.t_end) {
+        if (t < ti.t_end && sel) {  // no sel: the selection is given, only the protocol runs
           const float* imp = imp_base + (int64_t)tk * imp_stride;
           int32_t* dst = sel + (t * hkv + ti.g) * topk;
           if (ti.nb <= 256 * kTopkRegF4) {
@@ -1563,8 +1563,8 @@ cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_ti
   SSA_LAUNCH("cmp_lse_tc_kernel", cmp_lse_tc_kernel, g1, kThreads, smem_bytes_lse(), st, qm, km, a.cu_seqlens,
              a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.status);
   SSA_LAUNCH("cmp_out_tc_kernel", cmp_out_tc_kernel<G>, g2, kOutThreadsTk, smem_bytes_out(), st, qm, km, vm,
-             a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.o_branch, a.topk, a.sel,
-             a.imp_scratch, (int64_t)((btot + 3) & ~3), a.status);
+             a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.o_branch, a.topk,
+             a.sel_given ? nullptr : a.sel, a.imp_scratch, (int64_t)((btot + 3) & ~3), a.status);
   return cudaGetLastError();
 }
 

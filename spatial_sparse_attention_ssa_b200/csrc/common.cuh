@@ -10,7 +10,7 @@
 namespace ssa {
 
 // Device check bits recorded by kernels (or-ed into the status word).
-enum : int { kStatusCoordRange = 1, kStatusSeqlens = 2, kStatusTimeout = 4 };
+enum : int { kStatusCoordRange = 1, kStatusSeqlens = 2, kStatusTimeout = 4, kStatusSelection = 8 };
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

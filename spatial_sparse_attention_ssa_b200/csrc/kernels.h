@@ -15,6 +15,7 @@ constexpr int kCmpOutCtas = 160;
 
 struct FwdArgs {
   int dtype, d, hq, hkv, topk, gate_mode, m_cmp, m_win;
+  int sel_given;  // sel is an input (checked, not computed)
   int use_tc;   // run the tensor-core kernels where they cover the shape
   int* status;  // device check word
   float scale;

@@ -9,6 +9,7 @@ unloadable library raises immediately.
 from __future__ import annotations
 
 import ctypes
+import dataclasses
 import math
 import os
 from dataclasses import dataclass
@@ -24,6 +25,7 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
 DTYPE_BF16, DTYPE_F32 = 0, 1
 GATE_WEIGHTS, GATE_LOGITS = 0, 1
 OP_BIN, OP_FORWARD, OP_BACKWARD, OP_GEO_SELECT = 0, 1, 2, 3
+SEL_SCORES, SEL_GIVEN = 0, 1
 
 EXPORTS = ("ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size", "ssa_error_string",
            "ssa_get_device_status", "ssa_version", "ssa_launch_count", "ssa_profile_enable",
@@ -40,7 +42,8 @@ class SSAError(RuntimeError):
 class Params(ctypes.Structure):
     _fields_ = [("hq", ctypes.c_int32), ("hkv", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("m_cmp", ctypes.c_int32), ("m_win", ctypes.c_int32), ("topk", ctypes.c_int32),
-                ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("gate_mode", ctypes.c_int32)]
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("gate_mode", ctypes.c_int32),
+                ("selection", ctypes.c_int32)]
 
 
 class Partition(ctypes.Structure):
@@ -222,11 +225,11 @@ def ssa_bin_noalloc(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cm
 
 
 def make_params(hq, hkv, d, m_cmp, m_win, topk, dtype: torch.dtype, gate_mode: int,
-                scale: float = 0.0) -> Params:
+                scale: float = 0.0, selection: int = SEL_SCORES) -> Params:
     dt = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32 if dtype == torch.float32 else None
     if dt is None:
         raise ValueError("dtype must be torch.bfloat16 or torch.float32")
-    return Params(hq, hkv, d, m_cmp, m_win, topk, scale, dt, gate_mode)
+    return Params(hq, hkv, d, m_cmp, m_win, topk, scale, dt, gate_mode, selection)
 
 
 @dataclass
@@ -261,8 +264,12 @@ def workspace_size(op: int, p: Params, s: int, n: int, btot: int, wtot: int) -> 
 
 def ssa_forward(p: Params, cu_seqlens: torch.Tensor, blk: Bins, win: Bins, q: torch.Tensor,
                 k: torch.Tensor, v: torch.Tensor, gates: torch.Tensor, out: torch.Tensor | None = None,
-                saved: SavedTensors | None = None, workspace: torch.Tensor | None = None):
-    """Steps 2-6.  Returns (out [N, Hq, d], saved)."""
+                saved: SavedTensors | None = None, workspace: torch.Tensor | None = None,
+                sel: torch.Tensor | None = None):
+    """Steps 2-6.  Returns (out [N, Hq, d], saved).  With p.selection == SEL_GIVEN,
+    `sel` (int32 [N, Hkv, topk], e.g. from ssa_geo_select) becomes saved.sel and is
+    read instead of the score top-k; entries outside the token's sequence are set
+    to -1 on the device and reported by device_status()."""
     _require_cuda(cu_seqlens, q, k, v, gates)
     n = int(q.shape[0])
     s = int(cu_seqlens.shape[0]) - 1
@@ -271,6 +278,13 @@ def ssa_forward(p: Params, cu_seqlens: torch.Tensor, blk: Bins, win: Bins, q: to
         out = torch.empty_like(q)
     if saved is None:
         saved = SavedTensors.empty(p, n, blk.count, q.dtype, dev)
+    if p.selection == SEL_GIVEN:
+        if sel is not None:
+            if sel.dtype != torch.int32 or not sel.is_contiguous() or tuple(sel.shape) != (n, p.hkv, p.topk):
+                raise ValueError("sel must be a contiguous int32 tensor [N, Hkv, topk]")
+            saved = dataclasses.replace(saved, sel=sel)
+    elif sel is not None:
+        raise ValueError("sel is only read with selection=SEL_GIVEN")
     need = workspace_size(OP_FORWARD, p, s, n, blk.count, win.count)
     ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
     pb, pw, sv = blk.c(), win.c(), saved.c()

@@ -9,7 +9,11 @@ the CUDA path and the oracle must agree exactly, ties included (lower block id):
     one voxel per block): more candidates than the kernel keeps in shared memory
     for one token, or for one query block, so the exhaustive paths run, and the tie
     order decides all but one pick;
-  * sampled tokens of the 131072-token benchmark shape.
+  * sampled tokens of the 131072-token benchmark shape;
+  * the routing as the selection of the selected branch (selection = SEL_GIVEN):
+    forward and backward against the oracle given the same selection, on the
+    tensor-core (G = 8, 16) and SIMT (fp32, d = 32) paths; entries of a given
+    selection outside the token's sequence are dropped and reported.
 """
 import numpy as np
 import pytest
@@ -18,6 +22,7 @@ import torch
 from oracle import ssa_oracle as O
 from spatial_sparse_attention_ssa_b200 import ssa
 from spatial_sparse_attention_ssa_b200 import workloads as W
+from tests.ssa_testlib import ATOL, GpuRun, compare_backward, compare_forward, pool_rounding
 
 pytestmark = pytest.mark.gpu
 
@@ -94,3 +99,75 @@ def test_sampled_tokens_at_benchmark_size():
     b = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)
     assert (got == b["id"][:, None]).any(1).all()
     assert (np.diff(got, axis=1) > 0).all()
+
+
+# ---------------------------------------------------------------------------
+# the geometric routing as the selection of the selected branch (SEL_GIVEN)
+# ---------------------------------------------------------------------------
+
+def _run_given(w, t, sel=None):
+    """bin -> geometric routing -> forward with the given selection -> backward."""
+    run = GpuRun(w, t)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    run.p = ssa.make_params(w.hq, w.hkv, w.d, w.m_cmp, w.m_win, w.topk, tdt, w.gate_mode,
+                            selection=ssa.SEL_GIVEN)
+    run.blk, run.win = ssa.ssa_bin(run.coords, run.cu, w.R, w.m_cmp, w.m_win)
+    if sel is None:
+        sel = ssa.ssa_geo_select(run.coords, run.cu, w.R, run.blk, w.m_cmp, w.topk, w.hkv)
+    run.out, run.saved = ssa.ssa_forward(run.p, run.cu, run.blk, run.win, run.q, run.k, run.v, run.gates, sel=sel)
+    run.grads = ssa.ssa_backward(run.p, run.cu, run.blk, run.win, run.q, run.k, run.v, run.gates, run.saved,
+                                 run.dout)
+    torch.cuda.synchronize()
+    return run
+
+
+def _oracle_given(w, t, sel):
+    st = O.forward(w.coords, w.cu_seqlens, t.as_f32("q"), t.as_f32("k"), t.as_f32("v"), t.gates, hq=w.hq,
+                   hkv=w.hkv, m_cmp=w.m_cmp, m_win=w.m_win, topk=w.topk, gate_mode=w.gate_mode,
+                   pool_rounding=pool_rounding(w), sel_given=sel)
+    return st, O.backward(st, t.as_f32("do").astype(np.float64))
+
+
+@pytest.mark.parametrize("hq,d,dtype", [(16, 64, "bf16"), (32, 64, "bf16"), (4, 32, "f32")])
+def test_forward_and_backward_with_geometric_selection(hq, d, dtype):
+    w = W.small_shell(seed=23, R=40, n_prims=2, lo=4.0, hi=9.0, n_keep=700, n_seqs=2, hq=hq, hkv=2, d=d,
+                      m_cmp=4, m_win=4, topk=8, dtype=dtype)
+    t = W.make_tensors(w)
+    run = _run_given(w, t)
+    assert ssa.device_status() == 0
+    geo = O.geo_topk(w.coords, w.cu_seqlens, w.m_cmp, w.topk)
+    np.testing.assert_array_equal(run.saved.sel.cpu().numpy(), np.repeat(geo[:, None, :], w.hkv, axis=1))
+    st, g = _oracle_given(w, t, np.repeat(geo[:, None, :], w.hkv, axis=1))
+    toks = np.arange(w.n)
+    _, flips = compare_forward(run, st, toks, ATOL[w.dtype])
+    assert not flips
+    compare_backward(run, st, g, ATOL[w.dtype], flips)
+
+
+def test_given_selection_entries_outside_the_sequence_are_dropped_and_reported():
+    w = W.small_shell(seed=29, R=40, n_prims=2, lo=4.0, hi=9.0, n_keep=500, n_seqs=2, m_cmp=4, m_win=4, topk=8)
+    t = W.make_tensors(w)
+    b = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)
+    geo = np.repeat(O.geo_topk(w.coords, w.cu_seqlens, w.m_cmp, w.topk)[:, None, :], w.hkv, axis=1)
+    bad = geo.copy()
+    t0 = 3                                  # a token of sequence 0
+    bad[t0, 0, 0] = int(b["cu"][1])         # a block of sequence 1
+    bad[t0, 1, 1] = 1 << 20                 # past the last block
+    bad[w.n - 1, 0, 2] = -7                 # a negative id other than -1
+    sel = torch.from_numpy(bad.astype(np.int32)).cuda()
+    run = _run_given(w, t, sel=sel)
+    assert ssa.device_status() == 1         # SSA_ERR_INVALID_ARG
+    assert ssa.device_status() == 0         # read and cleared
+    want = bad.copy()
+    want[t0, 0, 0] = want[t0, 1, 1] = want[w.n - 1, 0, 2] = -1
+    np.testing.assert_array_equal(run.saved.sel.cpu().numpy(), want)
+    st, g = _oracle_given(w, t, want)
+    # rows t0 and n-1 now hold -1 between ids, which the score-selection checks of
+    # compare_forward reject: compare their branch outputs directly
+    rest = np.setdiff1d(np.arange(w.n), [t0, w.n - 1])
+    compare_forward(run, st, rest, ATOL[w.dtype])
+    ob = run.saved.o_branch.float().cpu().numpy().astype(np.float64)
+    for tt in (t0, w.n - 1):
+        for c in range(3):
+            assert np.abs(ob[c, tt] - st["o"][c][tt]).max() <= ATOL[w.dtype], (tt, c)
+    compare_backward(run, st, g, ATOL[w.dtype], [])
