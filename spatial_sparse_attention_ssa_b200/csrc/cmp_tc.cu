@@ -1335,8 +1335,10 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
         if (!mbar_wait(&sm.kv_full, kv_count & 1)) { ok = false; break; }
         ++kv_count;
         const int nrt = rt1 - rt0;
-        auto issue_sdp_now = [&](uint32_t qi) {
+        auto issue_sdp = [&](uint32_t qi) -> bool {
           const int qb = qi % kDkvQStages;
+          if (!mbar_wait(&sm.q_full[qb], (qi / kDkvQStages) & 1) || !mbar_wait(&sm.sdp_empty, (sdp_count & 1) ^ 1))
+            return false;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -1346,43 +1348,18 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
           }
           mma_commit(&sm.sdp_full);
           ++sdp_count;
-        };
-        // S^T / dP^T of row tile qi may go once its Q / dO tiles landed and the
-        // compute warps released the previous S^T / dP^T
-        auto sdp_ready = [&](uint32_t qi) -> bool {
-          return mbar_test(&sm.q_full[qi % kDkvQStages], (qi / kDkvQStages) & 1) &&
-                 mbar_test(&sm.sdp_empty, (sdp_count & 1) ^ 1);
-        };
-        auto issue_sdp = [&](uint32_t qi) -> bool {
-          if (!mbar_wait(&sm.q_full[qi % kDkvQStages], (qi / kDkvQStages) & 1) ||
-              !mbar_wait(&sm.sdp_empty, (sdp_count & 1) ^ 1))
-            return false;
-          issue_sdp_now(qi);
           return true;
         };
         if (nrt > 0 && !issue_sdp(q_count)) { ok = false; break; }
         for (int i = 0; i < nrt; ++i) {
           const int qb = q_count % kDkvQStages;
-          bool next_pending = i + 1 < nrt;
           if (i == 0 && !mbar_wait(&sm.acc_empty, (acc_count & 1) ^ 1)) { ok = false; break; }
-          // wait for P^T w / dS^T of this tile; the next tile's S^T / dP^T goes out as
-          // soon as it can, so that the tensor pipe works while the compute warps do
-          {
-            bool got = false;
-            const uint64_t t0 = global_ns();
-            for (uint32_t spin = 1;; ++spin) {
-              if (next_pending && sdp_ready(q_count + 1)) {
-                issue_sdp_now(q_count + 1);
-                next_pending = false;
-              }
-              if (mbar_test(&sm.pds_full, pds_count & 1)) {
-                got = true;
-                break;
-              }
-              if ((spin & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) break;
-            }
-            if (!got) { ok = false; break; }
-          }
+          // S^T / dP^T of the next tile first: the compute warps release this tile's
+          // S^T / dP^T before they hand over its P^T w / dS^T, so the next products
+          // queue on the tensor pipe ahead of this tile's dKc / dVc and run while the
+          // compute warps finish
+          if (i + 1 < nrt && !issue_sdp(q_count + 1)) { ok = false; break; }
+          if (!mbar_wait(&sm.pds_full, pds_count & 1)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kRows / 16; ++k) {
@@ -1398,7 +1375,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
           mma_commit(&sm.q_empty[qb]);
           ++pds_count;
           ++q_count;
-          if (next_pending && !issue_sdp(q_count)) { ok = false; break; }
         }
         if (!ok) break;
         mma_commit(&sm.kv_empty);
