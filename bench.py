@@ -256,10 +256,10 @@ def run_ours(a):
     ws_b = torch.empty(max(256, ssa.workspace_size(ssa.OP_BACKWARD, p, s, n, blk.count, win.count)),
                        dtype=torch.uint8, device=dev)
 
-    def step(cx=coords, cux=cu, qx=q, kx=k, vx=v, gx=gates, dx=do):
+    def step(cx=coords, cux=cu, qx=q, kx=k, vx=v, gx=gates, dx=do, outx=out, gradsx=grads):
         b_, w_ = ssa.ssa_bin(cx, cux, w.R, w.m_cmp, w.m_win, out=bins, workspace=ws_bin)
-        ssa.ssa_forward(p, cux, b_, w_, qx, kx, vx, gx, out=out, saved=saved, workspace=ws_f)
-        ssa.ssa_backward(p, cux, b_, w_, qx, kx, vx, gx, saved, dx, grads=grads, workspace=ws_b)
+        ssa.ssa_forward(p, cux, b_, w_, qx, kx, vx, gx, out=outx, saved=saved, workspace=ws_f)
+        ssa.ssa_backward(p, cux, b_, w_, qx, kx, vx, gx, saved, dx, grads=gradsx, workspace=ws_b)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
 
@@ -314,11 +314,21 @@ def run_ours(a):
         host_in = {"coords": coords.cpu().pin_memory(), "cu": cu.cpu().pin_memory(), "q": q.cpu().pin_memory(),
                    "k": k.cpu().pin_memory(), "v": v.cpu().pin_memory(), "gates": gates.cpu().pin_memory(),
                    "do": do.cpu().pin_memory()}
-        dev_in = {kk: torch.empty_like(vv, device=dev) for kk, vv in host_in.items()}
-        host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory()] + \
-                   [torch.empty(g_.shape, dtype=g_.dtype).pin_memory() for g_ in grads]
         h2d = sum(x.numel() * x.element_size() for x in host_in.values())
-        d2h = sum(x.numel() * x.element_size() for x in host_out)
+        d2h = sum(x.numel() * x.element_size() for x in [out, *grads])
+
+        def reduce_max(ms_):
+            if world > 1:
+                tt = torch.tensor([ms_], device=dev, dtype=torch.float64)
+                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+                ms_ = float(tt.item())
+            return ms_
+
+        # (1) serial: copy in, step, copy out, one step after the other
+        nset = 3  # buffer sets of the pipelined run (3 x ~3 GB on the device)
+        dev_in = [{kk: torch.empty_like(vv, device=dev) for kk, vv in host_in.items()} for _ in range(nset)]
+        dev_out = [[torch.empty_like(out)] + [torch.empty_like(g_) for g_ in grads] for _ in range(nset)]
+        host_out = [[torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in [out, *grads]] for _ in range(nset)]
         ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
         if world > 1:
             dist.barrier()
@@ -327,20 +337,71 @@ def run_ours(a):
             flush.zero_()
             ee[i][0].record()
             for kk in host_in:
-                dev_in[kk].copy_(host_in[kk], non_blocking=True)
-            step(dev_in["coords"], dev_in["cu"], dev_in["q"], dev_in["k"], dev_in["v"], dev_in["gates"],
-                 dev_in["do"])
-            for src, dst in zip([out, *grads], host_out):
+                dev_in[0][kk].copy_(host_in[kk], non_blocking=True)
+            di = dev_in[0]
+            step(di["coords"], di["cu"], di["q"], di["k"], di["v"], di["gates"], di["do"], dev_out[0][0],
+                 tuple(dev_out[0][1:]))
+            for src, dst in zip(dev_out[0], host_out[0]):
                 dst.copy_(src, non_blocking=True)
             ee[i][1].record()
         torch.cuda.synchronize()
-        e_ms = sum(a_.elapsed_time(b_) for a_, b_ in ee) / a.steps
+        serial_ms = reduce_max(sum(a_.elapsed_time(b_) for a_, b_ in ee) / a.steps)
+
+        # (2) pipelined: step i's inputs go up on one copy stream while earlier steps
+        # compute, its results come down on another while later steps compute; three
+        # device buffer sets.  Every step still moves all of its inputs and results.
+        comp = torch.cuda.current_stream(dev)
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_ready = [torch.cuda.Event() for _ in range(nset)]
+        in_free = [torch.cuda.Event() for _ in range(nset)]
+        out_ready = [torch.cuda.Event() for _ in range(nset)]
+        out_free = [torch.cuda.Event() for _ in range(nset)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def upload(j):
+            with torch.cuda.stream(up):
+                for kk in host_in:
+                    dev_in[j][kk].copy_(host_in[kk], non_blocking=True)
+                in_ready[j].record(up)
+
         if world > 1:
-            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start.record(comp)
+        up.wait_stream(comp)
+        down.wait_stream(comp)
+        upload(0)
+        for i in range(a.steps):
+            j = i % nset
+            if i + 1 < a.steps:
+                jn = (i + 1) % nset
+                if i + 1 >= nset:
+                    up.wait_event(in_free[jn])  # step i+1-nset is done with that input set
+                upload(jn)
+            comp.wait_event(in_ready[j])
+            if i >= nset:
+                comp.wait_event(out_free[j])  # step i-nset's results are down
+            flush.zero_()
+            di = dev_in[j]
+            step(di["coords"], di["cu"], di["q"], di["k"], di["v"], di["gates"], di["do"], dev_out[j][0],
+                 tuple(dev_out[j][1:]))
+            in_free[j].record(comp)
+            out_ready[j].record(comp)
+            down.wait_event(out_ready[j])
+            with torch.cuda.stream(down):
+                for src, dst in zip(dev_out[j], host_out[j]):
+                    dst.copy_(src, non_blocking=True)
+                out_free[j].record(down)
+        comp.wait_stream(down)
+        comp.wait_stream(up)
+        t_end.record(comp)
+        torch.cuda.synchronize()
+        e_ms = reduce_max(t_start.elapsed_time(t_end) / a.steps)
         e2e = {"value": total_tokens / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "mode": "pipelined: step i+1's inputs up and earlier steps' results down while step i computes "
+                       "(three buffer sets, two copy streams); timed from the first upload to the last download",
+               "serial": {"value": total_tokens / (serial_ms / 1e3), "ms_per_step": serial_ms}}
 
     # ---- roofline of the dominant kernel
     peaks = _peaks()
