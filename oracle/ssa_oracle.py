@@ -275,6 +275,126 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
     return st
 
 
+# ----------------------------------------------------------------------------
+# cross-attention SSA: queries of another token set attend the voxel tokens
+# ----------------------------------------------------------------------------
+
+
+def cross_forward(q_cu, kv_coords, kv_cu, q, k, v, gates, *, hq, hkv, m_cmp, topk, gate_mode, scale=None,
+                  pool_rounding="bf16", chunk=256, sel_given=None) -> State:
+    """Cross-attention SSA (LSRM, shuwu5.cn/article/2502.html: the NSA attention is
+    also used as cross attention between image tokens and voxel tokens).  The
+    queries q [Nq, Hq, d] of sequence s are rows q_cu[s] .. q_cu[s+1]-1; the keys
+    and values k/v [Nkv, Hkv, d] of sequence s are the voxel tokens kv_cu[s] ..
+    kv_cu[s+1]-1 at kv_coords, grouped into m_cmp^3 blocks and mean-pooled as in
+    the self-attention path.  Two branches: compressed attention over all blocks
+    of the sequence (with the group-summed top-k selection) and full attention
+    over the tokens of the selected blocks.  The queries have no voxel, so there
+    is no window branch; gates [Nq, Hq, 2] weight (compressed, selected)."""
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    nq, _, d = q.shape
+    G = hq // hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    q_cu = np.asarray(q_cu, dtype=np.int64)
+    kv_cu = np.asarray(kv_cu, dtype=np.int64)
+    blk = bin_tokens(kv_coords, kv_cu, m_cmp)
+    kc = mean_pool(k, blk, pool_rounding)
+    vc = mean_pool(v, blk, pool_rounding)
+    lse = np.full((2, nq, hq), np.nan)
+    o = np.zeros((2, nq, hq, d))
+    sel = np.full((nq, hkv, topk), -1, dtype=np.int64)
+    for s in range(len(q_cu) - 1):
+        toks = np.arange(q_cu[s], q_cu[s + 1])
+        b0, b1 = int(blk["cu"][s]), int(blk["cu"][s + 1])
+        if len(toks) == 0 or b1 == b0:
+            continue
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            for c0 in range(0, len(toks), chunk):
+                tt = toks[c0:c0 + chunk]
+                l_, o_, p_ = cmp_attention(np.asarray(q[tt, hs, :], np.float64), kc[b0:b1, g, :], vc[b0:b1, g, :],
+                                           scale)
+                lse[0, tt, hs] = l_
+                o[0, tt, hs, :] = o_
+                if sel_given is None:
+                    loc = topk_blocks(p_.sum(axis=1), topk)
+                    sel[tt, g, :] = np.where(loc >= 0, loc + b0, -1)
+    if sel_given is not None:
+        sel = np.asarray(sel_given, np.int64).copy()
+    for t in range(nq):
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            js = selected_tokens(sel[t, g], blk)
+            if len(js) == 0:
+                continue
+            l_, o_, _ = _attend(np.asarray(q[t, hs, :], np.float64), k[js, g, :], v[js, g, :], scale)
+            lse[1, t, hs] = l_
+            o[1, t, hs, :] = o_
+    gw = gate_weights(gates, gate_mode)  # [Nq, Hq, 2]
+    out = np.einsum("nhc,cnhd->nhd", gw, o)
+    return State(blk=blk, kc=kc, vc=vc, lse=lse, o=o, sel=sel, out=out, scale=scale, q=q, k=k, v=v,
+                 gates=np.asarray(gates, np.float64), gate_mode=gate_mode, hq=hq, hkv=hkv, G=G, topk=topk,
+                 q_cu=q_cu, kv_cu=kv_cu)
+
+
+def cross_backward(st: State, dout: np.ndarray, chunk: int = 256) -> dict:
+    """Gradients of sum(dout * O) of `cross_forward` w.r.t. q, k, v and gates, by
+    the chain rule of its two branches (selection held fixed, the Kc/Vc rounding
+    passed straight through, dKc/dK_i = 1/n_b)."""
+    q, k, v = np.asarray(st["q"], np.float64), st["k"], st["v"]
+    nq, hq, d = q.shape
+    hkv, G, scale = st["hkv"], st["G"], st["scale"]
+    blk = st["blk"]
+    dout = np.asarray(dout, dtype=np.float64)
+    gw = gate_weights(st["gates"], st["gate_mode"])
+    dots = np.einsum("nhd,cnhd->nhc", dout, st["o"])
+    dgates = dots if st["gate_mode"] == 0 else dots * gw * (1.0 - gw)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dkc = np.zeros((blk["count"], hkv, d))
+    dvc = np.zeros((blk["count"], hkv, d))
+    q_cu = st["q_cu"]
+    for s in range(len(q_cu) - 1):
+        toks = np.arange(q_cu[s], q_cu[s + 1])
+        b0, b1 = int(blk["cu"][s]), int(blk["cu"][s + 1])
+        if len(toks) == 0 or b1 == b0:
+            continue
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            kcg, vcg = st["kc"][b0:b1, g, :], st["vc"][b0:b1, g, :]
+            for c0 in range(0, len(toks), chunk):
+                tt = toks[c0:c0 + chunk]
+                qr = q[tt, hs, :]
+                dor = dout[tt, hs, :] * gw[tt, hs, 0][..., None]
+                p = np.exp(scale * (qr @ kcg.T) - st["lse"][0, tt, hs][..., None])
+                dp = dor @ vcg.T
+                ds = p * (dp - np.sum(p * dp, axis=-1, keepdims=True))
+                dq[tt, hs, :] += scale * (ds @ kcg)
+                dkc[b0:b1, g, :] += scale * np.einsum("ngb,ngd->bd", ds, qr)
+                dvc[b0:b1, g, :] += np.einsum("ngb,ngd->bd", p, dor)
+    cnt = np.diff(blk["ptr"]).astype(np.float64)
+    dk += dkc[blk["id"]] / cnt[blk["id"]][:, None, None]
+    dv += dvc[blk["id"]] / cnt[blk["id"]][:, None, None]
+    for t in range(nq):
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            js = selected_tokens(st["sel"][t, g], blk)
+            if len(js) == 0:
+                continue
+            qr = q[t, hs, :]
+            dor = dout[t, hs, :] * gw[t, hs, 1][:, None]
+            p = np.exp(scale * (qr @ k[js, g, :].T) - st["lse"][1, t, hs][:, None])
+            dp = dor @ v[js, g, :].T
+            ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+            dq[t, hs, :] += scale * (ds @ k[js, g, :])
+            np.add.at(dk[:, g, :], js, scale * (ds.T @ qr))
+            np.add.at(dv[:, g, :], js, p.T @ dor)
+    return {"dq": dq, "dk": dk, "dv": dv, "dgates": dgates, "dkc": dkc, "dvc": dvc}
+
+
 def importance(st: State, t: int, g: int) -> np.ndarray:
     """fp64 selection score of every block of t's sequence for group g (local ids)."""
     cu = st["cu_seqlens"]

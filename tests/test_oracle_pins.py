@@ -571,3 +571,105 @@ def test_geometric_selection_backward_matches_autograd():
     g = O.backward(st, do)
     for key, tt in (("dq", qt), ("dk", kt), ("dv", vt), ("dgates", gt)):
         np.testing.assert_allclose(g[key], tt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# cross-attention SSA (queries from another token set)
+# ----------------------------------------------------------------------------
+
+
+def _cross_case(seed, nq=(40, 0, 23), nkv=(90, 12, 57), R=16, hq=4, hkv=2, d=16):
+    rng = np.random.default_rng(seed)
+    coords, _, _, k, v, _ = _rand_case(seed, n_per_seq=nkv, R=R, hq=hq, hkv=hkv, d=d)
+    q_cu = np.concatenate([[0], np.cumsum(nq)]).astype(np.int64)
+    kv_cu = np.concatenate([[0], np.cumsum(nkv)]).astype(np.int64)
+    q = rng.standard_normal((int(q_cu[-1]), hq, d))
+    gates = rng.standard_normal((int(q_cu[-1]), hq, 2))
+    return q_cu, coords, kv_cu, q, k, v, gates
+
+
+def _sdpa_cross(q, k, v, q_cu, kv_cu, hq, hkv):
+    out = np.zeros_like(q)
+    G = hq // hkv
+    for s in range(len(q_cu) - 1):
+        a, b = int(q_cu[s]), int(q_cu[s + 1])
+        c, e = int(kv_cu[s]), int(kv_cu[s + 1])
+        if a == b:
+            continue
+        qt = torch.from_numpy(q[a:b]).transpose(0, 1)
+        kt = torch.from_numpy(k[c:e]).transpose(0, 1).repeat_interleave(G, 0)
+        vt = torch.from_numpy(v[c:e]).transpose(0, 1).repeat_interleave(G, 0)
+        out[a:b] = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).transpose(0, 1).numpy()
+    return out
+
+
+def test_cross_selection_covering_everything_is_full_cross_attention():
+    q_cu, coords, kv_cu, q, k, v, gates = _cross_case(31)
+    st = O.cross_forward(q_cu, coords, kv_cu, q, k, v, gates, hq=4, hkv=2, m_cmp=4, topk=10_000, gate_mode=1)
+    np.testing.assert_allclose(st["o"][1], _sdpa_cross(q, k, v, q_cu, kv_cu, 4, 2), rtol=1e-12, atol=1e-12)
+
+
+def test_cross_unit_blocks_make_compression_full_cross_attention():
+    q_cu, coords, kv_cu, q, k, v, gates = _cross_case(32)
+    st = O.cross_forward(q_cu, coords, kv_cu, q, k, v, gates, hq=4, hkv=2, m_cmp=1, topk=3, gate_mode=0,
+                         pool_rounding="none")
+    np.testing.assert_allclose(st["o"][0], _sdpa_cross(q, k, v, q_cu, kv_cu, 4, 2), rtol=1e-12, atol=1e-12)
+
+
+def test_cross_with_the_voxel_tokens_as_queries_matches_self_attention_branches():
+    """Queries = the voxel tokens themselves: the two cross branches, the selection
+    and (window gate 0) every gradient equal those of the self-attention oracle."""
+    coords, cu, q, k, v, gates = _rand_case(33, n_per_seq=(60, 0, 41), R=8, hq=4, hkv=2, d=8, unique=False)
+    g3 = np.abs(gates)
+    g3[..., 2] = 0.0
+    st = O.forward(coords, cu, q, k, v, g3, hq=4, hkv=2, m_cmp=2, m_win=4, topk=3, gate_mode=0,
+                   pool_rounding="none")
+    cr = O.cross_forward(cu, coords, cu, q, k, v, g3[..., :2], hq=4, hkv=2, m_cmp=2, topk=3, gate_mode=0,
+                         pool_rounding="none")
+    np.testing.assert_array_equal(cr["sel"], st["sel"])
+    np.testing.assert_allclose(cr["o"], st["o"][:2], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(cr["out"], st["out"], rtol=1e-12, atol=1e-12)
+    do = np.random.default_rng(4).standard_normal(q.shape)
+    gs, gc = O.backward(st, do), O.cross_backward(cr, do)
+    for key in ("dq", "dk", "dv"):
+        np.testing.assert_allclose(gc[key], gs[key], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(gc["dgates"], gs["dgates"][..., :2], rtol=1e-10, atol=1e-12)
+
+
+def test_cross_backward_matches_autograd():
+    """Independent dense-mask expression in torch (fp64) of the two cross branches,
+    with the oracle's bins and selection as constants, differentiated by autograd."""
+    q_cu, coords, kv_cu, q, k, v, gates = _cross_case(34, nq=(21, 9), nkv=(40, 25), R=8, hq=4, hkv=2, d=8)
+    for gate_mode in (0, 1):
+        st = O.cross_forward(q_cu, coords, kv_cu, q, k, v, gates, hq=4, hkv=2, m_cmp=2, topk=3,
+                             gate_mode=gate_mode, pool_rounding="none")
+        blk = st["blk"]
+        nb = int(blk["count"])
+        qt, kt, vt, gt = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v, gates))
+        onehot = torch.nn.functional.one_hot(torch.from_numpy(blk["id"]), nb).to(torch.float64)
+        kc = torch.einsum("nb,ngd->bgd", onehot, kt) / onehot.sum(0)[:, None, None]
+        vc = torch.einsum("nb,ngd->bgd", onehot, vt) / onehot.sum(0)[:, None, None]
+        qseq = torch.from_numpy(np.repeat(np.arange(len(q_cu) - 1), np.diff(q_cu)))
+        bseq = torch.from_numpy(np.repeat(np.arange(len(kv_cu) - 1), np.diff(blk["cu"])))
+        sel = torch.from_numpy(st["sel"])
+        gw = gt if gate_mode == 0 else torch.sigmoid(gt)
+        scale = st["scale"]
+        out = torch.zeros(q.shape, dtype=torch.float64)
+        for h in range(4):
+            g = h // 2
+            s_c = (scale * qt[:, h] @ kc[:, g].T).masked_fill(qseq[:, None] != bseq[None, :], -math.inf)
+            o_c = torch.softmax(s_c, -1) @ vc[:, g]
+            allowed = torch.zeros(q.shape[0], nb, dtype=torch.bool)
+            for slot in range(sel.shape[2]):
+                b = sel[:, g, slot]
+                ok = b >= 0
+                allowed[torch.nonzero(ok)[:, 0], b[ok]] = True
+            mask = allowed[:, torch.from_numpy(blk["id"])]
+            o_s = torch.softmax((scale * qt[:, h] @ kt[:, g].T).masked_fill(~mask, -math.inf), -1) @ vt[:, g]
+            out[:, h] = gw[:, h, 0:1] * o_c + gw[:, h, 1:2] * o_s
+        np.testing.assert_allclose(out.detach().numpy(), st["out"], rtol=1e-12, atol=1e-12)
+        do = np.random.default_rng(6).standard_normal(q.shape)
+        (out * torch.from_numpy(do)).sum().backward()
+        gr = O.cross_backward(st, do)
+        for key, tt in (("dq", qt), ("dk", kt), ("dv", vt), ("dgates", gt)):
+            np.testing.assert_allclose(gr[key], tt.grad.numpy(), rtol=1e-10, atol=1e-12)
