@@ -58,7 +58,14 @@ enum { SSA_DTYPE_BF16 = 0, SSA_DTYPE_F32 = 1 };
 enum { SSA_GATE_WEIGHTS = 0, SSA_GATE_LOGITS = 1 };
 /* where the selected branch's blocks come from (ssa_params.selection) */
 enum { SSA_SEL_SCORES = 0, SSA_SEL_GIVEN = 1 };
-enum { SSA_OP_BIN = 0, SSA_OP_FORWARD = 1, SSA_OP_BACKWARD = 2, SSA_OP_GEO_SELECT = 3 };
+enum {
+  SSA_OP_BIN = 0,
+  SSA_OP_FORWARD = 1,
+  SSA_OP_BACKWARD = 2,
+  SSA_OP_GEO_SELECT = 3,
+  SSA_OP_CROSS_FORWARD = 4,
+  SSA_OP_CROSS_BACKWARD = 5
+};
 
 /* Shape and method parameters shared by forward and backward. */
 typedef struct ssa_params {
@@ -210,10 +217,48 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
                                 float* dv, float* dgates, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Workspace bytes needed by `op` (SSA_OP_BIN / _FORWARD / _BACKWARD) for the
- * given sizes; B_tot and W_tot are the partition counts (pass N as an upper
- * bound before binning).  The workspace must be 256-byte aligned.  Returns 0
- * for invalid arguments.
+ * ssa_cross_forward -- cross-attention SSA (LSRM: the NSA attention also serves as
+ * cross attention between image tokens and voxel tokens): queries of another token
+ * set attend the voxel tokens of the same sequence through two branches, the
+ * compressed attention over all blocks (with the group-summed top-k selection, or a
+ * given selection, as in ssa_forward) and full attention over the tokens of the
+ * selected blocks.  The queries have no voxel, so there is no window branch.
+ *   q [Nq, Hq, d] dtype, rows of sequence s are q_cu[s] .. q_cu[s+1]-1 (q_cu int32
+ *   [S+1], device); k/v [Nkv, Hkv, d] dtype, the voxel tokens; blk: the block
+ *   partition from ssa_bin over the voxel tokens (their coordinates and cu_seqlens,
+ *   same S; the window partition is not used); gates fp32 [Nq, Hq, 2] (compressed,
+ *   selected), weights or logits as params->gate_mode; out [Nq, Hq, d] dtype.
+ *   saved: kc/vc [Hkv, B, d], ks/vs [Hkv, Nkv, d], o_branch fp32 [2, Nq, Hq, d],
+ *   lse fp32 [2, Nq, Hq], sel int32 [Nq, Hkv, topk].
+ *   ws: ssa_workspace_size(SSA_OP_CROSS_FORWARD, p, S, Nq, B, 0) bytes.
+ * Every sequence with queries must have voxel tokens: the call checks this on the
+ * device and synchronises the stream once to read the check (SSA_ERR_INVALID_ARG
+ * if it fails, before any attention kernel runs).  Otherwise asynchronous.
+ */
+SSA_API ssa_status ssa_cross_forward(const ssa_params* p, const int32_t* q_cu, int32_t S, int64_t Nq,
+                                     int64_t Nkv, const ssa_partition* blk, const void* q, const void* k,
+                                     const void* v, const float* gates, void* out, const ssa_saved* saved,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ssa_cross_backward -- gradients of sum(dout * out) of ssa_cross_forward with the
+ * selection held fixed: dq [Nq, Hq, d], dk/dv [Nkv, Hkv, d], dgates [Nq, Hq, 2], all
+ * fp32 and all written.  dout [Nq, Hq, d] dtype; `saved` from ssa_cross_forward on
+ * the same inputs; ws: ssa_workspace_size(SSA_OP_CROSS_BACKWARD, p, S, Nq, B, 0)
+ * bytes.  Same check and single stream synchronisation as the forward.
+ */
+SSA_API ssa_status ssa_cross_backward(const ssa_params* p, const int32_t* q_cu, int32_t S, int64_t Nq,
+                                      int64_t Nkv, const ssa_partition* blk, const void* q, const void* k,
+                                      const void* v, const float* gates, const ssa_saved* saved,
+                                      const void* dout, float* dq, float* dk, float* dv, float* dgates,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Workspace bytes needed by `op` (SSA_OP_BIN / _FORWARD / _BACKWARD / _GEO_SELECT /
+ * _CROSS_FORWARD / _CROSS_BACKWARD) for the given sizes; B_tot and W_tot are the
+ * partition counts (pass N as an upper bound before binning); for the cross ops N
+ * is the number of query tokens and W_tot is ignored.  The workspace must be
+ * 256-byte aligned.  Returns 0 for invalid arguments.
  */
 SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, int64_t N,
                                   int64_t B_tot, int64_t W_tot);

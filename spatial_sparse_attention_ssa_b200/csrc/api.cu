@@ -94,6 +94,10 @@ size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W
   return c.used;
 }
 
+// Cross-attention extras after the regular workspace: the gates widened to three
+// columns (the kernels read gates with a row stride of 3) and one check word.
+size_t cross_extra_bytes(int64_t Nq, int hq) { return align256(sizeof(float) * 3 * (size_t)Nq * hq) + 256; }
+
 struct BwdWs {
   float* Dc;
   float* rc;
@@ -157,6 +161,12 @@ SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, in
   if (op == SSA_OP_BACKWARD) {
     BwdWs w;
     return carve_bwd(nullptr, p, S, N, B_tot, W_tot, &w);
+  }
+  // cross attention: N = query tokens, W_tot unused (no window branch)
+  if (op == SSA_OP_CROSS_FORWARD) return fwd_bytes(p, S, N, B_tot, 0) + cross_extra_bytes(N, p->hq);
+  if (op == SSA_OP_CROSS_BACKWARD) {
+    BwdWs w;
+    return carve_bwd(nullptr, p, S, N, B_tot, 0, &w) + cross_extra_bytes(N, p->hq);
   }
   return 0;
 }
@@ -243,23 +253,20 @@ SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int
   return SSA_OK;
 }
 
-SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
-                               const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
-                               const void* v, const float* gates, void* out, const ssa_saved* saved, void* ws,
-                               size_t ws_bytes, void* stream) {
-  ssa_status ps = check_params(p);
-  if (ps != SSA_OK) return ps;
-  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
-    return SSA_ERR_INVALID_ARG;
-  if (N == 0) return SSA_OK;
-  if (!q || !k || !v || !gates || !out || !saved->kc || !saved->vc || !saved->ks || !saved->vs ||
-      !saved->o_branch || !saved->lse || !saved->sel || !ws)
-    return SSA_ERR_INVALID_ARG;
-  if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
-  if (ws_bytes < fwd_bytes(p, S, N, blk->count, win->count)) return SSA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = ssa::launch_pool(p->dtype, k, v, blk, N, p->hkv, p->d, saved->ks, saved->vs, saved->kc, saved->vc,
-                                   st);
+}  // extern "C"
+
+namespace {
+
+// The forward of the self-attention path (cross == 0: queries are the voxel tokens,
+// Nkv == N, three branches) and of the cross-attention path (cross == 1: queries of
+// another token set, keys / values the Nkv voxel tokens, no window branch, gates
+// already widened to 3 columns).
+ssa_status forward_common(const ssa_params* p, const int32_t* cu, int32_t S, int64_t N, int64_t Nkv, int cross,
+                          const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
+                          const void* v, const float* gates, void* out, const ssa_saved* saved, void* ws,
+                          cudaStream_t st) {
+  cudaError_t e = ssa::launch_pool(p->dtype, k, v, blk, Nkv, p->hkv, p->d, saved->ks, saved->vs, saved->kc,
+                                   saved->vc, st);
   if (e != cudaSuccess) return SSA_ERR_CUDA;
   ssa::FwdArgs a;
   a.dtype = p->dtype;
@@ -269,6 +276,8 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   a.topk = p->topk;
   a.gate_mode = p->gate_mode;
   a.sel_given = p->selection == SSA_SEL_GIVEN;
+  a.cross = cross;
+  a.Nkv = Nkv;
   a.m_cmp = p->m_cmp;
   a.m_win = p->m_win;
   a.use_tc = tc_enabled();
@@ -277,7 +286,7 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   a.scale = eff_scale(p);
   a.S = S;
   a.N = N;
-  a.cu_seqlens = cu_seqlens;
+  a.cu_seqlens = cu;
   a.blk = blk;
   a.win = win;
   a.q = q;
@@ -295,30 +304,17 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   Carver c(ws);
   carve_plan(c, S, &a.tiles_cnt, &a.tiles_pre, &a.items_cnt, &a.items_pre, &a.scan_tmp);
   int32_t* win_scan = nullptr;
-  fwd_bytes(p, S, N, blk->count, win->count, &a.imp_scratch, &a.win_cnt, &a.win_pre, &win_scan, ws);
+  fwd_bytes(p, S, N, blk->count, win ? win->count : 0, &a.imp_scratch, &a.win_cnt, &a.win_pre, &win_scan, ws);
   a.win_scan = win_scan;
   return cuda_status(ssa::simt_forward(a, st));
 }
 
-SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
-                                const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
-                                const void* v, const float* gates, const ssa_saved* saved, const void* dout,
-                                float* dq, float* dk, float* dv, float* dgates, void* ws, size_t ws_bytes,
-                                void* stream) {
-  ssa_status ps = check_params(p);
-  if (ps != SSA_OK) return ps;
-  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
-    return SSA_ERR_INVALID_ARG;
-  if (N == 0) return SSA_OK;
-  if (!q || !k || !v || !gates || !dout || !dq || !dk || !dv || !dgates || !saved->kc || !saved->vc ||
-      !saved->ks || !saved->vs || !saved->o_branch || !saved->lse || !saved->sel || !ws)
-    return SSA_ERR_INVALID_ARG;
-  if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
-  if ((int64_t)N * p->hkv * p->topk > INT32_MAX) return SSA_ERR_UNSUPPORTED;
+ssa_status backward_common(const ssa_params* p, const int32_t* cu, int32_t S, int64_t N, int64_t Nkv, int cross,
+                           const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
+                           const void* v, const float* gates, const ssa_saved* saved, const void* dout, float* dq,
+                           float* dk, float* dv, float* dgates, void* ws, cudaStream_t st) {
   BwdWs w;
-  if (ws_bytes < carve_bwd(nullptr, p, S, N, blk->count, win->count, &w)) return SSA_ERR_WORKSPACE;
-  carve_bwd(ws, p, S, N, blk->count, win->count, &w);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  carve_bwd(ws, p, S, N, blk->count, win ? win->count : 0, &w);
   ssa::BwdArgs a;
   a.dtype = p->dtype;
   a.d = p->d;
@@ -326,6 +322,8 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.hkv = p->hkv;
   a.topk = p->topk;
   a.gate_mode = p->gate_mode;
+  a.cross = cross;
+  a.Nkv = Nkv;
   a.m_cmp = p->m_cmp;
   a.m_win = p->m_win;
   a.use_tc = tc_enabled();
@@ -334,7 +332,7 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.scale = eff_scale(p);
   a.S = S;
   a.N = N;
-  a.cu_seqlens = cu_seqlens;
+  a.cu_seqlens = cu;
   a.blk = blk;
   a.win = win;
   a.q = q;
@@ -373,6 +371,118 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   a.items_pre = w.ip;
   a.scan_tmp = w.st;
   return cuda_status(ssa::simt_backward(a, st));
+}
+
+bool saved_ok(const ssa_saved* s) {
+  return s && s->kc && s->vc && s->ks && s->vs && s->o_branch && s->lse && s->sel;
+}
+
+// Widen the gates and check that every sequence with queries has voxel tokens;
+// synchronises the stream once to read the check.
+ssa_status cross_prepare(const ssa_params* p, const int32_t* q_cu, int32_t S, int64_t Nq, const ssa_partition* blk,
+                         const float* gates, void* extra, float** gates3, cudaStream_t st) {
+  *gates3 = static_cast<float*>(extra);
+  int* bad = reinterpret_cast<int*>(static_cast<char*>(extra) + align256(sizeof(float) * 3 * (size_t)Nq * p->hq));
+  if (cudaMemsetAsync(bad, 0, sizeof(int), st) != cudaSuccess) return SSA_ERR_CUDA;
+  if (ssa::cross_prep(gates, Nq * p->hq, *gates3, q_cu, blk->cu, S, bad, st) != cudaSuccess) return SSA_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyAsync(&h, bad, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSA_ERR_CUDA;
+  return h ? SSA_ERR_INVALID_ARG : SSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                               const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
+                               const void* v, const float* gates, void* out, const ssa_saved* saved, void* ws,
+                               size_t ws_bytes, void* stream) {
+  ssa_status ps = check_params(p);
+  if (ps != SSA_OK) return ps;
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
+    return SSA_ERR_INVALID_ARG;
+  if (N == 0) return SSA_OK;
+  if (!q || !k || !v || !gates || !out || !saved_ok(saved) || !ws) return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
+  if (ws_bytes < fwd_bytes(p, S, N, blk->count, win->count)) return SSA_ERR_WORKSPACE;
+  return forward_common(p, cu_seqlens, S, N, N, 0, blk, win, q, k, v, gates, out, saved, ws,
+                        static_cast<cudaStream_t>(stream));
+}
+
+SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, int32_t S, int64_t N,
+                                const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
+                                const void* v, const float* gates, const ssa_saved* saved, const void* dout,
+                                float* dq, float* dk, float* dv, float* dgates, void* ws, size_t ws_bytes,
+                                void* stream) {
+  ssa_status ps = check_params(p);
+  if (ps != SSA_OK) return ps;
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
+    return SSA_ERR_INVALID_ARG;
+  if (N == 0) return SSA_OK;
+  if (!q || !k || !v || !gates || !dout || !dq || !dk || !dv || !dgates || !saved_ok(saved) || !ws)
+    return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
+  if ((int64_t)N * p->hkv * p->topk > INT32_MAX) return SSA_ERR_UNSUPPORTED;
+  BwdWs w;
+  if (ws_bytes < carve_bwd(nullptr, p, S, N, blk->count, win->count, &w)) return SSA_ERR_WORKSPACE;
+  return backward_common(p, cu_seqlens, S, N, N, 0, blk, win, q, k, v, gates, saved, dout, dq, dk, dv, dgates, ws,
+                         static_cast<cudaStream_t>(stream));
+}
+
+SSA_API ssa_status ssa_cross_forward(const ssa_params* p, const int32_t* q_cu, int32_t S, int64_t Nq, int64_t Nkv,
+                                     const ssa_partition* blk, const void* q, const void* k, const void* v,
+                                     const float* gates, void* out, const ssa_saved* saved, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  ssa_status ps = check_params(p);
+  if (ps != SSA_OK) return ps;
+  if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk) ||
+      !saved)
+    return SSA_ERR_INVALID_ARG;
+  if (Nq == 0) return SSA_OK;
+  if (Nkv < 1 || !q || !k || !v || !gates || !out || !saved_ok(saved) || !ws) return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > Nkv) return SSA_ERR_INVALID_ARG;
+  const size_t base = fwd_bytes(p, S, Nq, blk->count, 0);
+  if (ws_bytes < base + cross_extra_bytes(Nq, p->hq)) return SSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* gates3 = nullptr;
+  ps = cross_prepare(p, q_cu, S, Nq, blk, gates, static_cast<char*>(ws) + base, &gates3, st);
+  if (ps != SSA_OK) return ps;
+  return forward_common(p, q_cu, S, Nq, Nkv, 1, blk, nullptr, q, k, v, gates3, out, saved, ws, st);
+}
+
+SSA_API ssa_status ssa_cross_backward(const ssa_params* p, const int32_t* q_cu, int32_t S, int64_t Nq, int64_t Nkv,
+                                      const ssa_partition* blk, const void* q, const void* k, const void* v,
+                                      const float* gates, const ssa_saved* saved, const void* dout, float* dq,
+                                      float* dk, float* dv, float* dgates, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  ssa_status ps = check_params(p);
+  if (ps != SSA_OK) return ps;
+  if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk) ||
+      !saved)
+    return SSA_ERR_INVALID_ARG;
+  if (Nkv > 0 && dk && dv && Nq == 0) {  // no queries: the key gradients are zero
+    cudaStream_t st0 = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(dk, 0, sizeof(float) * Nkv * p->hkv * p->d, st0) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, sizeof(float) * Nkv * p->hkv * p->d, st0) != cudaSuccess)
+      return SSA_ERR_CUDA;
+    return SSA_OK;
+  }
+  if (Nq == 0) return SSA_OK;
+  if (Nkv < 1 || !q || !k || !v || !gates || !dout || !dq || !dk || !dv || !dgates || !saved_ok(saved) || !ws)
+    return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > Nkv) return SSA_ERR_INVALID_ARG;
+  if ((int64_t)Nq * p->hkv * p->topk > INT32_MAX) return SSA_ERR_UNSUPPORTED;
+  BwdWs w;
+  const size_t base = carve_bwd(nullptr, p, S, Nq, blk->count, 0, &w);
+  if (ws_bytes < base + cross_extra_bytes(Nq, p->hq)) return SSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* gates3 = nullptr;
+  ps = cross_prepare(p, q_cu, S, Nq, blk, gates, static_cast<char*>(ws) + base, &gates3, st);
+  if (ps != SSA_OK) return ps;
+  return backward_common(p, q_cu, S, Nq, Nkv, 1, blk, nullptr, q, k, v, gates3, saved, dout, dq, dk, dv, dgates,
+                         ws, st);
 }
 
 }  // extern "C"

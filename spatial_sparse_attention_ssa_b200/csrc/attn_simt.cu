@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(128) cmp_out_topk_kernel(
 template <typename T, int D>
 __global__ void __launch_bounds__(128) slc_fwd_kernel(const T* __restrict__ q, const T* __restrict__ ks,
                                                       const T* __restrict__ vs, const int32_t* __restrict__ bptr,
-                                                      const int32_t* __restrict__ sel, int64_t N, int hq, int hkv,
-                                                      int topk, float qs2, float* __restrict__ o_out,
+                                                      const int32_t* __restrict__ sel, int64_t N, int64_t ldk,
+                                                      int hq, int hkv, int topk, float qs2, float* __restrict__ o_out,
                                                       float* __restrict__ lse_out) {
   constexpr int NT = D / 32;
   const int G = hq / hkv, GT = G * NT, PPC = 128 / GT;
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(128) slc_fwd_kernel(const T* __restrict__ q, c
           float x = -CUDART_INF_F;
           if (j0 + jj < p1) {
             float kv[32];
-            load32(ks + ((int64_t)g * N + j0 + jj) * D + sub * 32, kv);
+            load32(ks + ((int64_t)g * ldk + j0 + jj) * D + sub * 32, kv);
             x = row_sum<NT>(dot32r(qv, kv), gmask);
           }
           sc[jj] = x;
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(128) slc_fwd_kernel(const T* __restrict__ q, c
             const float p = exp2f(sc[jj] - mn);
             l += p;
             float vv[32];
-            load32(vs + ((int64_t)g * N + j0 + jj) * D + sub * 32, vv);
+            load32(vs + ((int64_t)g * ldk + j0 + jj) * D + sub * 32, vv);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = fmaf(p, vv[i], o[i]);
           }
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(128) win_fwd_kernel(const T* __restrict__ q, c
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void combine_kernel(const float* __restrict__ ob, const float* __restrict__ gates, int64_t rows, int mode,
-                               T* __restrict__ out) {
+                               int nbr, T* __restrict__ out) {
   constexpr int NT = D / 32;
   const int64_t total = rows * NT;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
@@ -408,6 +408,7 @@ __global__ void combine_kernel(const float* __restrict__ ob, const float* __rest
     for (int e = 0; e < 32; ++e) acc[e] = 0.f;
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
+      if (c >= nbr) break;
       const float w = gate_weight(gates, row * 3 + c, mode);
       load32(ob + ((int64_t)c * rows + row) * D + sub * 32, x);
 #pragma unroll
@@ -424,7 +425,7 @@ __global__ void combine_kernel(const float* __restrict__ ob, const float* __rest
 // for the compressed (c = 0) and window (c = 2) branches, -lse * log2(e), w and -D.
 template <typename T, int D>
 __global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict__ dout, const float* __restrict__ gates,
-                               const float* __restrict__ lse, int64_t rows, int mode, float* __restrict__ Dc,
+                               const float* __restrict__ lse, int64_t rows, int mode, int nbr, float* __restrict__ Dc,
                                float* __restrict__ dgates, float* __restrict__ rc) {
   constexpr int NT = D / 32;
   const int64_t total = rows * NT;
@@ -439,12 +440,13 @@ __global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict
     load32(dout + row * D + sub * 32, dov);
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
+      if (c >= nbr) break;
       load32(ob + ((int64_t)c * rows + row) * D + sub * 32, x);
       const float dot = row_sum<NT>(dot32r(dov, x), 0xffffffffu);
       if (valid && sub == 0) {
         const float w = gate_weight(gates, row * 3 + c, mode);
         Dc[(int64_t)c * rows + row] = w * dot;
-        dgates[row * 3 + c] = mode == SSA_GATE_LOGITS ? dot * w * (1.f - w) : dot;
+        dgates[row * nbr + c] = mode == SSA_GATE_LOGITS ? dot * w * (1.f - w) : dot;
         if (c != 1) {
           float* r = rc + (c == 0 ? 0 : 3 * rows);
           r[row] = -lse[(int64_t)c * rows + row] * kLog2e;
@@ -635,7 +637,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) slc_bwd_dq_kernel(
     const T* __restrict__ q, const T* __restrict__ ks, const T* __restrict__ vs, const T* __restrict__ dout,
     const float* __restrict__ gates, int mode, const int32_t* __restrict__ bptr, const int32_t* __restrict__ sel,
-    int64_t N, int hq, int hkv, int topk, float qs2, float scale, const float* __restrict__ lse_in,
+    int64_t N, int64_t ldk, int hq, int hkv, int topk, float qs2, float scale, const float* __restrict__ lse_in,
     const float* __restrict__ Dc, float* __restrict__ dq_out) {
   constexpr int NT = D / 32;
   const int G = hq / hkv, GT = G * NT, PPC = 128 / GT;
@@ -666,8 +668,8 @@ __global__ void __launch_bounds__(128) slc_bwd_dq_kernel(
       const int p1 = bptr[b + 1];
       for (int j = bptr[b]; j < p1; ++j) {
         float kv[32], vv[32];
-        load32(ks + ((int64_t)g * N + j) * D + sub * 32, kv);
-        load32(vs + ((int64_t)g * N + j) * D + sub * 32, vv);
+        load32(ks + ((int64_t)g * ldk + j) * D + sub * 32, kv);
+        load32(vs + ((int64_t)g * ldk + j) * D + sub * 32, vv);
         const float s2 = row_sum<NT>(dot32r(qv, kv), gmask);
         const float p = exp2f(s2 - lse2);
         const float dp = row_sum<NT>(dot32r(dov, vv), gmask);
@@ -715,7 +717,7 @@ __global__ void __launch_bounds__(128) slc_bwd_dkv_kernel(
     const T* __restrict__ q, const T* __restrict__ ks, const T* __restrict__ vs, const T* __restrict__ dout,
     const float* __restrict__ gates, int mode, const int32_t* __restrict__ bptr, const int32_t* __restrict__ bperm,
     const int32_t* __restrict__ inv_ptr, const int32_t* __restrict__ inv_tok, const int32_t* __restrict__ ipre,
-    int64_t N, int64_t btot, int hq, int hkv, float qs2, float scale, const float* __restrict__ lse_in,
+    int64_t ldk, int64_t btot, int hq, int hkv, float qs2, float scale, const float* __restrict__ lse_in,
     const float* __restrict__ Dc, float* __restrict__ dk_out, float* __restrict__ dv_out) {
   constexpr int NT = D / 32;
   constexpr int SLOTS = 128 / NT;  // (key slot, row slice) pairs
@@ -744,7 +746,7 @@ __global__ void __launch_bounds__(128) slc_bwd_dkv_kernel(
     for (int kp = 0; kp < nb; kp += kpc) {
       const int j = kp + kslot;
       const bool validk = j < nb;
-      const int64_t kidx = (int64_t)g * N + p0 + (validk ? j : 0);
+      const int64_t kidx = (int64_t)g * ldk + p0 + (validk ? j : 0);
       float kv[32], vv[32], dk[32], dv[32];
       load32(ks + kidx * D + sub * 32, kv);
       load32(vs + kidx * D + sub * 32, vv);
@@ -874,7 +876,7 @@ template <typename T, int G>
 __global__ void __launch_bounds__(256) slc_bwd_fused_kernel(
     const T* __restrict__ q, const T* __restrict__ ks, const T* __restrict__ vs, const T* __restrict__ dout,
     const float* __restrict__ gates, int mode, const int32_t* __restrict__ bptr, const int32_t* __restrict__ bperm,
-    const int32_t* __restrict__ sel, int64_t N, int hq, int hkv, int topk, float qs2, float scale,
+    const int32_t* __restrict__ sel, int64_t N, int64_t ldk, int hq, int hkv, int topk, float qs2, float scale,
     const float* __restrict__ lse_in, const float* __restrict__ Dc, float* __restrict__ dq_out,
     float* __restrict__ dk_out, float* __restrict__ dv_out) {
   constexpr int D = 64;
@@ -909,7 +911,7 @@ __global__ void __launch_bounds__(256) slc_bwd_fused_kernel(
       if (b < 0) continue;
       const int p1 = bptr[b + 1];
       for (int j = bptr[b]; j < p1; ++j) {
-        const int64_t kidx = (int64_t)g * N + j;
+        const int64_t kidx = (int64_t)g * ldk + j;
         const float2 kk = load2<T>(ks + kidx * D + 2 * lane);
         const float2 vv = load2<T>(vs + kidx * D + 2 * lane);
         float ps[G], pd[G];
@@ -1112,6 +1114,21 @@ __global__ void sel_check_kernel(int32_t* __restrict__ sel, int64_t N, int hkv, 
   if (bad) atomicOr(status, kStatusSelection);
 }
 
+// Cross attention: gates [rows, 2] widened to the [rows, 3] layout the kernels read
+// (column 2 unused), and a check that every sequence with queries has blocks.
+__global__ void cross_prep_kernel(const float* __restrict__ g2, int64_t rows, float* __restrict__ g3,
+                                  const int32_t* __restrict__ q_cu, const int32_t* __restrict__ bcu, int S,
+                                  int* __restrict__ bad) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows; r += stride) {
+    g3[3 * r] = g2[2 * r];
+    g3[3 * r + 1] = g2[2 * r + 1];
+    g3[3 * r + 2] = 0.f;
+  }
+  for (int64_t s = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; s < S; s += stride)
+    if (q_cu[s + 1] > q_cu[s] && bcu[s + 1] == bcu[s]) atomicOr(bad, 1);
+}
+
 __global__ void sel_keys_kernel(const int32_t* __restrict__ sel, int64_t N, int hkv, int topk, int64_t btot,
                                 uint64_t* __restrict__ keys, int32_t* __restrict__ vals) {
   const int64_t total = N * hkv * topk;
@@ -1200,19 +1217,21 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   } else {
     const int pairs_per_cta = 128 / (G * C::NT);
     SSA_LAUNCH("slc_fwd_kernel", (slc_fwd_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st,
-               q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.hq, a.hkv,
-               a.topk, qs2, ob + rows * D, a.lse + rows);
+               q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.Nkv, a.hq,
+               a.hkv, a.topk, qs2, ob + rows * D, a.lse + rows);
   }
-  const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
-  if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
-    e = win_fwd_tc(a, a.win_cnt, a.win_pre, a.win_scan, st);
-    if (e != cudaSuccess) return e;
-  } else
-  SSA_LAUNCH("win_fwd_kernel", (win_fwd_kernel<T, D>), gw, 128, 0, st, q, static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.win->perm,
-                                           a.win->ptr, a.win->count, a.hq, a.hkv, qs2, ob + 2 * rows * D,
-                                           a.lse + 2 * rows);
-  SSA_LAUNCH("combine_kernel", (combine_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, a.gates, rows, a.gate_mode,
-                                                                             static_cast<T*>(a.out));
+  if (!a.cross) {  // cross attention has no window branch (the queries have no voxel)
+    const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
+    if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
+      e = win_fwd_tc(a, a.win_cnt, a.win_pre, a.win_scan, st);
+      if (e != cudaSuccess) return e;
+    } else
+      SSA_LAUNCH("win_fwd_kernel", (win_fwd_kernel<T, D>), gw, 128, 0, st, q, static_cast<const T*>(a.k),
+                 static_cast<const T*>(a.v), a.win->perm, a.win->ptr, a.win->count, a.hq, a.hkv, qs2,
+                 ob + 2 * rows * D, a.lse + 2 * rows);
+  }
+  SSA_LAUNCH("combine_kernel", (combine_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, a.gates,
+             rows, a.gate_mode, a.cross ? 2 : 3, static_cast<T*>(a.out));
   return cudaGetLastError();
 }
 
@@ -1240,8 +1259,8 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   e = exclusive_scan(a.items_cnt, a.items_pre, a.S + 1, a.scan_tmp, st);
   if (e != cudaSuccess) return e;
 
-  SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout, a.gates, a.lse, rows, a.gate_mode,
-                                                                             a.Dc, a.dgates, a.rc);
+  SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout,
+             a.gates, a.lse, rows, a.gate_mode, a.cross ? 2 : 3, a.Dc, a.dgates, a.rc);
   if (a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
     // 128-row tiles for the tensor-core kernels (tiles_cnt / tiles_pre are free again here)
     SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu,
@@ -1261,24 +1280,27 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
         a.scale, kCmpRowChunk, a.lse, a.Dc, a.dkc, a.dvc);
   }
   if (D == 64 && (G == 8 || G == 16)) {
-    cudaMemsetAsync(a.dk, 0, sizeof(float) * a.N * a.hkv * D, st);
-    cudaMemsetAsync(a.dv, 0, sizeof(float) * a.N * a.hkv * D, st);
+    cudaMemsetAsync(a.dk, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
+    cudaMemsetAsync(a.dv, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
     const int g_slc = grid_1d(a.N * a.hkv, 8, 148 * 16);
     if (a.use_tc && slc_mma_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
       e = slc_bwd_mma(a, st);
       if (e != cudaSuccess) return e;
     } else if (G == 16)
       SSA_LAUNCH("slc_bwd_fused_kernel", (slc_bwd_fused_kernel<T, 16>), g_slc, 256, 0, st, q, ks, vs, dout, a.gates,
-                 a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
+                 a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
+                 a.lse + rows,
                  a.Dc + rows, a.dq, a.dk, a.dv);
     else
       SSA_LAUNCH("slc_bwd_fused_kernel", (slc_bwd_fused_kernel<T, 8>), g_slc, 256, 0, st, q, ks, vs, dout, a.gates,
-                 a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
+                 a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
+                 a.lse + rows,
                  a.Dc + rows, a.dq, a.dk, a.dv);
   } else {
     const int pairs_per_cta = 128 / (G * C::NT);
     SSA_LAUNCH("slc_bwd_dq_kernel", (slc_bwd_dq_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
-        q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale, a.lse + rows,
+        q, ks, vs, dout, a.gates, a.gate_mode, a.blk->ptr, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
+        a.lse + rows,
         a.Dc + rows, a.dq);
     // inverted selection CSR: for (g, b), the tokens whose group g selected b, ascending
     const int64_t nsel = a.N * a.hkv * a.topk;
@@ -1297,13 +1319,15 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                G, a.slc_cnt);
     e = exclusive_scan(a.slc_cnt, a.slc_pre, nkeys + 1, a.scan_tmp, st);
     if (e != cudaSuccess) return e;
-    cudaMemsetAsync(a.dk, 0, sizeof(float) * a.N * a.hkv * D, st);
-    cudaMemsetAsync(a.dv, 0, sizeof(float) * a.N * a.hkv * D, st);
+    cudaMemsetAsync(a.dk, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
+    cudaMemsetAsync(a.dv, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
     SSA_LAUNCH("slc_bwd_dkv_kernel", (slc_bwd_dkv_kernel<T, D>), 148 * 8, 128, 0, st, q, ks, vs, dout, a.gates,
-               a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.slc_pre, a.N, btot, a.hq, a.hkv, qs2, a.scale,
+               a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.slc_pre, a.Nkv, btot, a.hq, a.hkv, qs2, a.scale,
                a.lse + rows, a.Dc + rows, a.dk, a.dv);
   }
-  if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
+  if (a.cross) {
+    // no window branch
+  } else if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
     e = win_bwd_tc(a, a.win_cnt, a.win_pre, a.scan_tmp, st);
     if (e != cudaSuccess) return e;
   } else {
@@ -1315,12 +1339,19 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                                                  a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
                                                  a.Dc + 2 * rows, a.dk, a.dv);
   }
-  SSA_LAUNCH("cmp_scatter_kernel", cmp_scatter_kernel, grid_1d(a.N * a.hkv * D / 4, 256, 148 * 32), 256, 0, st, 
-      a.dkc, a.dvc, a.blk->id, a.blk->ptr, a.N, btot, a.hkv, D, a.dk, a.dv);
+  SSA_LAUNCH("cmp_scatter_kernel", cmp_scatter_kernel, grid_1d(a.Nkv * a.hkv * D / 4, 256, 148 * 32), 256, 0, st,
+             a.dkc, a.dvc, a.blk->id, a.blk->ptr, a.Nkv, btot, a.hkv, D, a.dk, a.dv);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t cross_prep(const float* gates2, int64_t rows, float* gates3, const int32_t* q_cu, const int32_t* bcu,
+                       int S, int* bad, cudaStream_t st) {
+  SSA_LAUNCH("cross_prep_kernel", cross_prep_kernel, grid_1d(rows > S ? rows : S, 256, 148 * 32), 256, 0, st, gates2,
+             rows, gates3, q_cu, bcu, S, bad);
+  return cudaGetLastError();
+}
 
 cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st) {
   if (a.dtype == SSA_DTYPE_BF16) {

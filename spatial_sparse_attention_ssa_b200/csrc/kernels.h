@@ -16,6 +16,8 @@ constexpr int kCmpOutCtas = 160;
 struct FwdArgs {
   int dtype, d, hq, hkv, topk, gate_mode, m_cmp, m_win;
   int sel_given;  // sel is an input (checked, not computed)
+  int cross;      // queries from another token set: no window branch, gates hold 2 live columns
+  int64_t Nkv;    // key / value tokens (= N unless cross)
   int use_tc;   // run the tensor-core kernels where they cover the shape
   int* status;  // device check word
   float scale;
@@ -40,6 +42,8 @@ struct FwdArgs {
 
 struct BwdArgs {
   int dtype, d, hq, hkv, topk, gate_mode, m_cmp, m_win;
+  int cross;    // as in FwdArgs
+  int64_t Nkv;  // key / value tokens (= N unless cross)
   int use_tc;
   int* status;
   float scale;
@@ -74,6 +78,8 @@ struct BwdArgs {
 cudaError_t launch_pool(int dtype, const void* k, const void* v, const ssa_partition* blk, int64_t N, int hkv,
                         int d, void* ks, void* vs, void* kc, void* vc, cudaStream_t st);
 cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st);
+cudaError_t cross_prep(const float* gates2, int64_t rows, float* gates3, const int32_t* q_cu, const int32_t* bcu,
+                       int S, int* bad, cudaStream_t st);
 
 // Tensor-core (tcgen05) kernels of the compressed branch, bf16, head dim 64.
 bool cmp_tc_supported(int dtype, int d, int hq, int hkv, int topk);

@@ -177,8 +177,8 @@ struct SlcFwdSmem {
 template <int G>
 __global__ void __launch_bounds__(32 * kSlcWarps) slc_fwd_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ ks, const __nv_bfloat16* __restrict__ vs,
-    const int32_t* __restrict__ bptr, const int32_t* __restrict__ sel, int64_t N, int hq, int hkv, int topk,
-    float qs2, float* __restrict__ o_out, float* __restrict__ lse_out) {
+    const int32_t* __restrict__ bptr, const int32_t* __restrict__ sel, int64_t N, int64_t ldk, int hq, int hkv,
+    int topk, float qs2, float* __restrict__ o_out, float* __restrict__ lse_out) {
   __shared__ SlcFwdSmem sm;
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gid = lane / 4, tig = lane % 4;
@@ -189,8 +189,8 @@ __global__ void __launch_bounds__(32 * kSlcWarps) slc_fwd_mma_kernel(
   for (int64_t pair = (int64_t)blockIdx.x * kSlcWarps + w; pair < npairs; pair += (int64_t)gridDim.x * kSlcWarps) {
     const int64_t t = pair / hkv;
     const int g = (int)(pair % hkv);
-    const __nv_bfloat16* kg = ks + (int64_t)g * N * 64;
-    const __nv_bfloat16* vg = vs + (int64_t)g * N * 64;
+    const __nv_bfloat16* kg = ks + (int64_t)g * ldk * 64;
+    const __nv_bfloat16* vg = vs + (int64_t)g * ldk * 64;
     stage_heads(qs_t, q + (t * hq + (int64_t)g * G) * 64, G, lane);
     const KeyList kl = key_list(sel + pair * topk, bptr, topk, lane);
     __syncwarp();
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(32 * kSlcWarps) slc_bwd_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ ks, const __nv_bfloat16* __restrict__ vs,
     const __nv_bfloat16* __restrict__ dout, const float* __restrict__ gates, int mode,
     const int32_t* __restrict__ bptr, const int32_t* __restrict__ bperm, const int32_t* __restrict__ sel, int64_t N,
-    int hq, int hkv, int topk, float qs2, float scale, const float* __restrict__ lse_in,
+    int64_t ldk, int hq, int hkv, int topk, float qs2, float scale, const float* __restrict__ lse_in,
     const float* __restrict__ Dc, float* __restrict__ dq_out, float* __restrict__ dk_out,
     float* __restrict__ dv_out) {
   extern __shared__ uint8_t smem_raw[];
@@ -322,8 +322,8 @@ __global__ void __launch_bounds__(32 * kSlcWarps) slc_bwd_mma_kernel(
   for (int64_t pair = (int64_t)blockIdx.x * kSlcWarps + w; pair < npairs; pair += (int64_t)gridDim.x * kSlcWarps) {
     const int64_t t = pair / hkv;
     const int g = (int)(pair % hkv);
-    const __nv_bfloat16* kg = ks + (int64_t)g * N * 64;
-    const __nv_bfloat16* vg = vs + (int64_t)g * N * 64;
+    const __nv_bfloat16* kg = ks + (int64_t)g * ldk * 64;
+    const __nv_bfloat16* vg = vs + (int64_t)g * ldk * 64;
     const int64_t row0 = t * hq + (int64_t)g * G;
     __syncwarp();  // the previous pair's reads of the staged tiles are done
     stage_heads(qs_t, q + row0 * 64, G, lane);
@@ -463,10 +463,10 @@ cudaError_t slc_fwd_mma(const FwdArgs& a, cudaStream_t st) {
   const float qs2 = a.scale * kLog2e;
   if (G == 16)
     SSA_LAUNCH("slc_fwd_mma_kernel", slc_fwd_mma_kernel<16>, grid, 32 * kSlcWarps, 0, st, q, ksp, vsp, a.blk->ptr,
-               a.sel, a.N, a.hq, a.hkv, a.topk, qs2, o, a.lse + rows);
+               a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, o, a.lse + rows);
   else
     SSA_LAUNCH("slc_fwd_mma_kernel", slc_fwd_mma_kernel<8>, grid, 32 * kSlcWarps, 0, st, q, ksp, vsp, a.blk->ptr,
-               a.sel, a.N, a.hq, a.hkv, a.topk, qs2, o, a.lse + rows);
+               a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, o, a.lse + rows);
   return cudaGetLastError();
 }
 
@@ -488,11 +488,11 @@ cudaError_t slc_bwd_mma(const BwdArgs& a, cudaStream_t st) {
   }
   if (G == 16)
     SSA_LAUNCH("slc_bwd_mma_kernel", slc_bwd_mma_kernel<16>, grid, 32 * kSlcWarps, smem, st, q, ksp, vsp, dO,
-               a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale,
+               a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
                a.lse + rows, a.Dc + rows, a.dq, a.dk, a.dv);
   else
     SSA_LAUNCH("slc_bwd_mma_kernel", slc_bwd_mma_kernel<8>, grid, 32 * kSlcWarps, smem, st, q, ksp, vsp, dO,
-               a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.hq, a.hkv, a.topk, qs2, a.scale,
+               a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
                a.lse + rows, a.Dc + rows, a.dq, a.dk, a.dv);
   return cudaGetLastError();
 }

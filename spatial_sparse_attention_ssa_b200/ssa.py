@@ -24,12 +24,12 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
                 4: "SSA_ERR_COORD_RANGE", 5: "SSA_ERR_CUDA", 6: "SSA_ERR_TIMEOUT"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 GATE_WEIGHTS, GATE_LOGITS = 0, 1
-OP_BIN, OP_FORWARD, OP_BACKWARD, OP_GEO_SELECT = 0, 1, 2, 3
+OP_BIN, OP_FORWARD, OP_BACKWARD, OP_GEO_SELECT, OP_CROSS_FORWARD, OP_CROSS_BACKWARD = 0, 1, 2, 3, 4, 5
 SEL_SCORES, SEL_GIVEN = 0, 1
 
 EXPORTS = ("ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size", "ssa_error_string",
            "ssa_get_device_status", "ssa_version", "ssa_launch_count", "ssa_profile_enable",
-           "ssa_profile_read", "ssa_geo_select")
+           "ssa_profile_read", "ssa_geo_select", "ssa_cross_forward", "ssa_cross_backward")
 
 
 class SSAError(RuntimeError):
@@ -76,6 +76,12 @@ def _lib():
         lib.ssa_backward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, pp, pp, vp, vp, vp, vp,
                                      ctypes.POINTER(Saved), vp, vp, vp, vp, vp, vp, sz, vp]
         lib.ssa_backward.restype = ctypes.c_int
+        lib.ssa_cross_forward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, i64, pp, vp, vp, vp, vp, vp,
+                                          ctypes.POINTER(Saved), vp, sz, vp]
+        lib.ssa_cross_forward.restype = ctypes.c_int
+        lib.ssa_cross_backward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, i64, pp, vp, vp, vp, vp,
+                                           ctypes.POINTER(Saved), vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.ssa_cross_backward.restype = ctypes.c_int
         lib.ssa_geo_select.argtypes = [vp, vp, i32, i64, i32, pp, i32, i32, i32, vp, vp, sz, vp]
         lib.ssa_geo_select.restype = ctypes.c_int
         lib.ssa_workspace_size.argtypes = [i32, ctypes.POINTER(Params), i32, i64, i64, i64]
@@ -253,6 +259,18 @@ class SavedTensors:
             torch.empty(3, n, p.hq, dtype=torch.float32, device=device),
             torch.empty(n, p.hkv, p.topk, dtype=torch.int32, device=device))
 
+    @staticmethod
+    def empty_cross(p: Params, nq: int, nkv: int, btot: int, dtype, device) -> "SavedTensors":
+        """Buffers of ssa_cross_forward: two branches, keys / values of the voxel tokens."""
+        return SavedTensors(
+            torch.empty(p.hkv, max(btot, 1), p.d, dtype=dtype, device=device),
+            torch.empty(p.hkv, max(btot, 1), p.d, dtype=dtype, device=device),
+            torch.empty(p.hkv, nkv, p.d, dtype=dtype, device=device),
+            torch.empty(p.hkv, nkv, p.d, dtype=dtype, device=device),
+            torch.empty(2, nq, p.hq, p.d, dtype=torch.float32, device=device),
+            torch.empty(2, nq, p.hq, dtype=torch.float32, device=device),
+            torch.empty(nq, p.hkv, p.topk, dtype=torch.int32, device=device))
+
     def c(self) -> Saved:
         return Saved(_ptr(self.kc), _ptr(self.vc), _ptr(self.ks), _ptr(self.vs), _ptr(self.o_branch),
                      _ptr(self.lse), _ptr(self.sel))
@@ -314,6 +332,61 @@ def ssa_backward(p: Params, cu_seqlens: torch.Tensor, blk: Bins, win: Bins, q, k
                              _ptr(q), _ptr(k), _ptr(v), _ptr(gates), ctypes.byref(sv), _ptr(dout), _ptr(dq),
                              _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ws), ws.numel(), _stream(dev))
     _check(st, "ssa_backward")
+    return dq, dk, dv, dg
+
+
+def ssa_cross_forward(p: Params, q_cu: torch.Tensor, blk: Bins, q: torch.Tensor, k: torch.Tensor,
+                      v: torch.Tensor, gates: torch.Tensor, out: torch.Tensor | None = None,
+                      saved: SavedTensors | None = None, workspace: torch.Tensor | None = None,
+                      sel: torch.Tensor | None = None):
+    """Cross-attention SSA: queries q [Nq, Hq, d] (sequence s = rows q_cu[s] ..
+    q_cu[s+1]-1) attend the voxel tokens k / v [Nkv, Hkv, d] binned into `blk`
+    through the compressed and selected branches; gates [Nq, Hq, 2].
+    Returns (out [Nq, Hq, d], saved)."""
+    _require_cuda(q_cu, q, k, v, gates)
+    nq, nkv = int(q.shape[0]), int(k.shape[0])
+    s = int(q_cu.shape[0]) - 1
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if saved is None:
+        saved = SavedTensors.empty_cross(p, nq, nkv, blk.count, q.dtype, dev)
+    if p.selection == SEL_GIVEN:
+        if sel is not None:
+            if sel.dtype != torch.int32 or not sel.is_contiguous() or tuple(sel.shape) != (nq, p.hkv, p.topk):
+                raise ValueError("sel must be a contiguous int32 tensor [Nq, Hkv, topk]")
+            saved = dataclasses.replace(saved, sel=sel)
+    elif sel is not None:
+        raise ValueError("sel is only read with selection=SEL_GIVEN")
+    need = workspace_size(OP_CROSS_FORWARD, p, s, nq, blk.count, 0)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb, sv = blk.c(), saved.c()
+    st = _lib().ssa_cross_forward(ctypes.byref(p), _ptr(q_cu), s, nq, nkv, ctypes.byref(pb), _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(gates), _ptr(out), ctypes.byref(sv), _ptr(ws), ws.numel(),
+                                  _stream(dev))
+    _check(st, "ssa_cross_forward")
+    return out, saved
+
+
+def ssa_cross_backward(p: Params, q_cu: torch.Tensor, blk: Bins, q, k, v, gates, saved: SavedTensors,
+                       dout: torch.Tensor, grads=None, workspace: torch.Tensor | None = None):
+    """Gradients of ssa_cross_forward: (dq, dk, dv, dgates), all fp32."""
+    _require_cuda(q_cu, q, k, v, gates, dout)
+    nq, nkv = int(q.shape[0]), int(k.shape[0])
+    s = int(q_cu.shape[0]) - 1
+    dev = q.device
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = (torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32),
+                 torch.empty(gates.shape, **f32))
+    dq, dk, dv, dg = grads
+    need = workspace_size(OP_CROSS_BACKWARD, p, s, nq, blk.count, 0)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb, sv = blk.c(), saved.c()
+    st = _lib().ssa_cross_backward(ctypes.byref(p), _ptr(q_cu), s, nq, nkv, ctypes.byref(pb), _ptr(q), _ptr(k),
+                                   _ptr(v), _ptr(gates), ctypes.byref(sv), _ptr(dout), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), _ptr(dg), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ssa_cross_backward")
     return dq, dk, dv, dg
 
 

@@ -333,6 +333,40 @@ def make_tensors(w: Workload, seed: int | None = None, with_do: bool | None = No
     return Tensors(q, k, v, gates, do, w.dtype)
 
 
+@dataclass
+class CrossQueries:
+    """Queries of another token set (image tokens in LSRM's cross attention) for
+    the voxel sequences of a workload: sequence s owns rows q_cu[s] .. q_cu[s+1]-1."""
+    q_cu: np.ndarray  # int64 [S + 1]
+    q: np.ndarray  # [Nq, Hq, d], bf16 bits or f32
+    gates: np.ndarray  # f32 [Nq, Hq, 2] (compressed, selected)
+    do: np.ndarray  # [Nq, Hq, d]
+    dtype: str
+
+    def as_f32(self, name: str) -> np.ndarray:
+        a = getattr(self, name)
+        if self.dtype == "bf16" and a.dtype == np.uint16:
+            return bf16_bits_to_f32(a)
+        return a.astype(np.float32, copy=False)
+
+
+def make_cross_queries(w: Workload, q_lens, seed: int = 0) -> CrossQueries:
+    """Q, dO ~ N(0,1) in the workload dtype for len(q_lens) == S sequences; gates as
+    in make_tensors (U(0,1) weights or N(0,1) logits), two columns."""
+    q_lens = np.asarray(q_lens, np.int64)
+    assert len(q_lens) == w.s
+    rng = np.random.default_rng(np.random.SeedSequence([w.seed, seed, 104729]))
+    nq = int(q_lens.sum())
+    q_cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int64)
+    q = _normal(rng, (nq, w.hq, w.d), w.dtype)
+    if w.gate_mode == 0:
+        gates = rng.uniform(0.0, 1.0, size=(nq, w.hq, 2)).astype(np.float32)
+    else:
+        gates = rng.standard_normal(size=(nq, w.hq, 2), dtype=np.float32)
+    do = _normal(rng, (nq, w.hq, w.d), w.dtype)
+    return CrossQueries(q_cu, q, gates, do, w.dtype)
+
+
 def permute_workload(w: Workload, t: Tensors, seed: int) -> tuple[Workload, Tensors, np.ndarray]:
     """Shuffle tokens inside each sequence (for permutation-equivariance checks).
     Returns the new workload, tensors and `src` with new[i] = old[src[i]]."""

@@ -8,6 +8,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from spatial_sparse_attention_ssa_b200 import ssa
 
@@ -90,3 +91,27 @@ def test_geo_select_argument_errors_are_found_on_the_host():
     assert call(R=40000) == 2                    # squared distances must fit 32 bits
     assert call(ws_bytes=100) == 3               # workspace too small
     assert call(N=0) == 0                        # nothing to do
+
+
+def test_cross_attention_argument_errors_are_found_on_the_host():
+    lib = ssa.lib()
+    p = ssa.make_params(16, 2, 64, 8, 8, 16, torch.bfloat16, 1)
+    part = ssa.Partition(1, 1, 1, 1, 1, 10)
+    sv = ssa.Saved(1, 1, 1, 1, 1, 1, 1)
+    need_f = ssa.workspace_size(ssa.OP_CROSS_FORWARD, p, 1, 1000, 10, 0)
+    need_b = ssa.workspace_size(ssa.OP_CROSS_BACKWARD, p, 1, 1000, 10, 0)
+    assert need_f > ssa.workspace_size(ssa.OP_FORWARD, p, 1, 1000, 10, 0) - 4096 and need_f > 3 * 1000 * 16 * 4
+    assert need_b > 3 * 1000 * 16 * 4
+
+    def fwd(S=1, nq=1000, nkv=500, ws_bytes=None, q=1):
+        return lib.ssa_cross_forward(ctypes.byref(p), 1, S, nq, nkv, ctypes.byref(part), q, 1, 1, 1, 1,
+                                     ctypes.byref(sv), 1, need_f if ws_bytes is None else ws_bytes, None)
+    assert fwd(S=0) == 1 and fwd(nq=-1) == 1 and fwd(q=None) == 1
+    assert fwd(nkv=5) == 1                       # fewer voxel tokens than blocks
+    assert fwd(ws_bytes=need_f - 1) == 3
+    assert fwd(nq=0) == 0                        # nothing to do
+    bad = ssa.make_params(16, 2, 64, 8, 8, 16, torch.bfloat16, 1, selection=7)
+    assert lib.ssa_cross_forward(ctypes.byref(bad), 1, 1, 10, 10, ctypes.byref(part), 1, 1, 1, 1, 1,
+                                 ctypes.byref(sv), 1, need_f, None) == 1
+    assert lib.ssa_cross_backward(ctypes.byref(p), 1, 1, 1000, 500, ctypes.byref(part), 1, 1, 1, 1,
+                                  ctypes.byref(sv), 1, 1, 1, 1, 1, 1, need_b - 1, None) == 3
