@@ -71,6 +71,7 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-geo", action="store_true", help="skip the separate timing of geometric block routing")
+    ap.add_argument("--no-cross", action="store_true", help="skip the separate timing of cross attention")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -473,6 +474,46 @@ def run_ours(a):
         geo = {"ms_per_call": g_ms, "tokens_per_s": n / (g_ms / 1e3), "blocks": int(blk.count),
                "topk": int(w.topk), "launches_per_call": 2}
 
+    # ---- cross attention (queries from another token set), timed on its own: the
+    # same voxel tokens as keys / values, Nq = n image-token queries, fwd + bwd
+    cross = None
+    if not a.no_cross:
+        cq = W.make_cross_queries(w, [n], seed=3)
+        q_cu = to_dev(cq.q_cu.astype(np.int32), False)
+        cq_q, cq_do = to_dev(cq.q), to_dev(cq.do)
+        cq_g = to_dev(cq.gates, False)
+        c_saved = ssa.SavedTensors.empty_cross(p, n, n, blk.count, torch.bfloat16, dev)
+        c_out = torch.empty_like(cq_q)
+        c_grads = (torch.empty(cq_q.shape, dtype=torch.float32, device=dev),
+                   torch.empty(k.shape, dtype=torch.float32, device=dev),
+                   torch.empty(v.shape, dtype=torch.float32, device=dev),
+                   torch.empty(cq_g.shape, dtype=torch.float32, device=dev))
+        c_wf = torch.empty(ssa.workspace_size(ssa.OP_CROSS_FORWARD, p, 1, n, blk.count, 0), dtype=torch.uint8,
+                           device=dev)
+        c_wb = torch.empty(ssa.workspace_size(ssa.OP_CROSS_BACKWARD, p, 1, n, blk.count, 0), dtype=torch.uint8,
+                           device=dev)
+
+        def cross_step():
+            ssa.ssa_cross_forward(p, q_cu, blk, cq_q, k, v, cq_g, out=c_out, saved=c_saved, workspace=c_wf)
+            ssa.ssa_cross_backward(p, q_cu, blk, cq_q, k, v, cq_g, c_saved, cq_do, grads=c_grads, workspace=c_wb)
+
+        for _ in range(3):
+            cross_step()
+        check_device("cross-attention warm-up")
+        ec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+        for i in range(a.steps):
+            flush.zero_()
+            ec[i][0].record()
+            cross_step()
+            ec[i][1].record()
+        torch.cuda.synchronize()
+        check_device("cross attention")
+        c_ms = sum(a_.elapsed_time(b_) for a_, b_ in ec) / a.steps
+        cross = {"ms_per_step": c_ms, "query_tokens_per_s": n / (c_ms / 1e3), "query_tokens": n, "voxel_tokens": n,
+                 "what": "ssa_cross_forward + ssa_cross_backward: N(0,1) bf16 image-token queries against the "
+                         "voxel tokens (compressed + selected branches, same heads, k, m_cmp)"}
+        del c_saved, c_grads, c_wf, c_wb
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -490,6 +531,7 @@ def run_ours(a):
                 "config": cfg, "roofline": roof, "roofline_exp": exp_roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(launches),
                 "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel, "geo_routing": geo,
+                "cross_attention": cross,
                 "peaks_source": peaks["_source"]}
         print(json.dumps(line), flush=True)
     if world > 1:
