@@ -114,6 +114,84 @@ def mean_pool(x: np.ndarray, blk: dict, pool_rounding: str) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
+# step 2, learned form: a sparse 3D convolution before the mean pool
+# ----------------------------------------------------------------------------
+
+# offsets of the 3^3 kernel; offset index (dx + 1) * 9 + (dy + 1) * 3 + (dz + 1)
+CONV_OFFSETS = [(dx, dy, dz) for dx in (-1, 0, 1) for dy in (-1, 0, 1) for dz in (-1, 0, 1)]
+
+
+def _neighbours(coords: np.ndarray, cu_seqlens: np.ndarray):
+    """For every token i and offset index o, the tokens of i's sequence at
+    coords_i + offset_o (all of them if coordinates repeat), as a list of lists."""
+    coords = np.asarray(coords, np.int64)
+    cu = np.asarray(cu_seqlens, np.int64)
+    nbr = [[None] * 27 for _ in range(len(coords))]
+    for s in range(len(cu) - 1):
+        where = {}
+        for t in range(cu[s], cu[s + 1]):
+            where.setdefault(tuple(coords[t]), []).append(t)
+        for t in range(cu[s], cu[s + 1]):
+            c = coords[t]
+            for o, off in enumerate(CONV_OFFSETS):
+                nbr[t][o] = where.get((c[0] + off[0], c[1] + off[1], c[2] + off[2]), [])
+    return nbr
+
+
+def sparse_conv3(coords, cu_seqlens, x, w, b, nbr=None) -> np.ndarray:
+    """Submanifold sparse 3D convolution with a 3^3 kernel (Direct3D-S2, "方法": the
+    sparse 3D compression may apply a sparse 3D convolution before pooling): at
+    every token i, out_i = b + sum_o W_o^T x_j over the tokens j of i's sequence at
+    coords_i + offset_o; empty voxels contribute nothing.
+    x [N, Hkv, d], w [Hkv, 27, d_in, d_out], b [Hkv, d] -> [N, Hkv, d] (float64)."""
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w, np.float64)
+    nbr = _neighbours(coords, cu_seqlens) if nbr is None else nbr
+    out = np.broadcast_to(np.asarray(b, np.float64), x.shape).copy()
+    for i in range(len(x)):
+        for o in range(27):
+            for j in nbr[i][o]:
+                out[i] += np.einsum("gc,gcd->gd", x[j], w[:, o])
+    return out
+
+
+def conv_pool(coords, cu_seqlens, x, w, b, blk: dict, rounding: str) -> np.ndarray:
+    """Learned compression: the block mean of the sparse convolution's output,
+    computed exactly and then rounded once to the storage type ("bf16", "f32",
+    or "none")."""
+    y = sparse_conv3(coords, cu_seqlens, x, w, b)
+    sums = np.zeros((blk["count"],) + y.shape[1:])
+    np.add.at(sums, blk["id"], y)
+    mean = sums / np.diff(blk["ptr"]).astype(np.float64)[:, None, None]
+    if rounding == "none":
+        return mean
+    if rounding == "f32":
+        return mean.astype(np.float32).astype(np.float64)
+    if rounding == "bf16":
+        return _round_bf16(mean.astype(np.float32))
+    raise ValueError(rounding)
+
+
+def conv_pool_backward(coords, cu_seqlens, x, w, blk: dict, dxc: np.ndarray):
+    """Gradients of the learned compression given dL/dXc [B, Hkv, d] (the rounding of
+    Xc passed straight through): each token's output receives dXc_b / n_b; then
+    dx_j = sum over (i, o) with j at coords_i + offset_o of W_o dout_i,
+    dW_o = sum over the same pairs of x_j dout_i^T, db = sum_i dout_i."""
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w, np.float64)
+    nbr = _neighbours(coords, cu_seqlens)
+    dout = dxc[blk["id"]] / np.diff(blk["ptr"]).astype(np.float64)[blk["id"]][:, None, None]
+    dx = np.zeros_like(x)
+    dw = np.zeros_like(w)
+    for i in range(len(x)):
+        for o in range(27):
+            for j in nbr[i][o]:
+                dx[j] += np.einsum("gcd,gd->gc", w[:, o], dout[i])
+                dw[:, o] += np.einsum("gc,gd->gcd", x[j], dout[i])
+    return dx, dw, dout.sum(axis=0)
+
+
+# ----------------------------------------------------------------------------
 # helpers
 # ----------------------------------------------------------------------------
 
@@ -192,9 +270,14 @@ class State(dict):
 
 
 def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
-            gate_mode, scale=None, pool_rounding="bf16", tokens=None, chunk=256, sel_given=None) -> State:
+            gate_mode, scale=None, pool_rounding="bf16", tokens=None, chunk=256, sel_given=None,
+            conv=None) -> State:
     """SSA forward.  q [N, Hq, d], k/v [N, Hkv, d] (any float type; converted to
     float64), gates [N, Hq, 3].
+
+    `conv` (a dict of wk, bk, wv, bv) makes the compression learned: Kc / Vc are the
+    block means of a sparse 3D convolution of K / V (`conv_pool`), rounded as
+    `pool_rounding` says.
 
     `sel_given` ([N, Hkv, topk] global block ids or -1) replaces the score top-k:
     the selected branch attends the tokens of those blocks instead (a routing by
@@ -214,8 +297,12 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
     cu_seqlens = np.asarray(cu_seqlens, dtype=np.int64)
     blk = bin_tokens(coords, cu_seqlens, m_cmp)
     win = bin_tokens(coords, cu_seqlens, m_win)
-    kc = mean_pool(k, blk, pool_rounding)
-    vc = mean_pool(v, blk, pool_rounding)
+    if conv is None:
+        kc = mean_pool(k, blk, pool_rounding)
+        vc = mean_pool(v, blk, pool_rounding)
+    else:
+        kc = conv_pool(coords, cu_seqlens, k, conv["wk"], conv["bk"], blk, pool_rounding)
+        vc = conv_pool(coords, cu_seqlens, v, conv["wv"], conv["bv"], blk, pool_rounding)
     seq = _seq_of_tokens(cu_seqlens, n)
     if tokens is None:
         tokens = np.arange(n)
@@ -271,7 +358,8 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
     out[tokens] = np.einsum("nhc,cnhd->nhd", gw, o[:, tokens])
     st = State(blk=blk, win=win, kc=kc, vc=vc, lse=lse, o=o, sel=sel, out=out, scale=scale,
                q=q, k=k, v=v, gates=np.asarray(gates, np.float64), gate_mode=gate_mode,
-               hq=hq, hkv=hkv, G=G, topk=topk, cu_seqlens=cu_seqlens, tokens=tokens)
+               hq=hq, hkv=hkv, G=G, topk=topk, cu_seqlens=cu_seqlens, tokens=tokens, conv=conv,
+               coords=np.asarray(coords, np.int64))
     return st
 
 
@@ -482,8 +570,16 @@ def backward(st: State, dout: np.ndarray, chunk: int = 256) -> dict:
                 dkc[b0:b1, g, :] += scale * np.einsum("ngb,ngd->bd", ds, qr)
                 dvc[b0:b1, g, :] += np.einsum("ngb,ngd->bd", p, dor)
     cnt = np.diff(blk["ptr"]).astype(np.float64)
-    dk["cmp"] = dkc[blk["id"]] / cnt[blk["id"]][:, None, None]
-    dv["cmp"] = dvc[blk["id"]] / cnt[blk["id"]][:, None, None]
+    conv = st.get("conv")
+    dconv = {}
+    if conv is None:
+        dk["cmp"] = dkc[blk["id"]] / cnt[blk["id"]][:, None, None]
+        dv["cmp"] = dvc[blk["id"]] / cnt[blk["id"]][:, None, None]
+    else:
+        dk["cmp"], dconv["dwk"], dconv["dbk"] = conv_pool_backward(st["coords"], st["cu_seqlens"], k, conv["wk"],
+                                                                   blk, dkc)
+        dv["cmp"], dconv["dwv"], dconv["dbv"] = conv_pool_backward(st["coords"], st["cu_seqlens"], v, conv["wv"],
+                                                                   blk, dvc)
 
     # selected-block and window branches
     for t in range(n):
@@ -509,6 +605,7 @@ def backward(st: State, dout: np.ndarray, chunk: int = 256) -> dict:
         "dv": dv["cmp"] + dv["slc"] + dv["win"],
         "dgates": dgates,
         "parts": {"dq": dq, "dk": dk, "dv": dv, "dkc": dkc, "dvc": dvc},
+        **dconv,
     }
 
 

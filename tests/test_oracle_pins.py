@@ -673,3 +673,104 @@ def test_cross_backward_matches_autograd():
         gr = O.cross_backward(st, do)
         for key, tt in (("dq", qt), ("dk", kt), ("dv", vt), ("dgates", gt)):
             np.testing.assert_allclose(gr[key], tt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# learned compression: sparse 3D convolution before the mean pool
+# ----------------------------------------------------------------------------
+
+
+def _conv_weights(seed, hkv, d, scale=0.2):
+    rng = np.random.default_rng(seed)
+    return {"wk": scale * rng.standard_normal((hkv, 27, d, d)), "bk": rng.standard_normal((hkv, d)),
+            "wv": scale * rng.standard_normal((hkv, 27, d, d)), "bv": rng.standard_normal((hkv, d))}
+
+
+def _dense_conv(coords, cu, x, w, b, R):
+    """torch conv3d (cross-correlation, padding 1, one group per KV head) on a dense
+    grid per sequence, read back at the tokens (duplicate voxels add up)."""
+    hkv, _, d, _ = w.shape
+    wt = torch.as_tensor(w, dtype=torch.float64)
+    wt = wt.reshape(hkv, 3, 3, 3, d, d).permute(0, 5, 4, 1, 2, 3).reshape(hkv * d, d, 3, 3, 3)
+    bt = torch.as_tensor(b, dtype=torch.float64).reshape(-1)
+    outs = []
+    xt = torch.as_tensor(x, dtype=torch.float64)
+    for s in range(len(cu) - 1):
+        a, e = int(cu[s]), int(cu[s + 1])
+        c = torch.from_numpy(np.asarray(coords[a:e], np.int64))
+        flat = (c[:, 0] * R + c[:, 1]) * R + c[:, 2]
+        grid = torch.zeros(hkv * d, R * R * R, dtype=torch.float64)
+        grid = grid.index_add(1, flat, xt[a:e].reshape(e - a, hkv * d).T)
+        y = torch.nn.functional.conv3d(grid.reshape(1, hkv * d, R, R, R), wt, bt, padding=1, groups=hkv)
+        outs.append(y.reshape(hkv * d, -1)[:, flat].T.reshape(e - a, hkv, d))
+    return torch.cat(outs)
+
+
+def test_sparse_conv_matches_dense_conv3d_with_duplicates_and_sequences():
+    coords, cu, _, k, _, _ = _rand_case(41, n_per_seq=(70, 0, 45), R=6, hq=4, hkv=2, d=5, unique=False)
+    cw = _conv_weights(1, 2, 5)
+    got = O.sparse_conv3(coords, cu, k, cw["wk"], cw["bk"])
+    want = _dense_conv(coords, cu, k, cw["wk"], cw["bk"], 6).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_identity_convolution_is_the_mean_pool():
+    coords, cu, _, k, _, _ = _rand_case(42, n_per_seq=(80, 33), R=8, hq=4, hkv=2, d=6)
+    w = np.zeros((2, 27, 6, 6))
+    w[:, 13] = np.eye(6)  # the centre offset (0, 0, 0)
+    blk = O.bin_tokens(coords, cu, 4)
+    got = O.conv_pool(coords, cu, k, w, np.zeros((2, 6)), blk, "none")
+    np.testing.assert_allclose(got, O.mean_pool(k, blk, "none"), rtol=1e-12, atol=1e-12)
+
+
+def test_conv_pool_backward_matches_autograd():
+    coords, cu, _, k, _, _ = _rand_case(43, n_per_seq=(50, 31), R=6, hq=4, hkv=2, d=4, unique=False)
+    cw = _conv_weights(2, 2, 4)
+    blk = O.bin_tokens(coords, cu, 2)
+    xt = torch.tensor(k, dtype=torch.float64, requires_grad=True)
+    wt = torch.tensor(cw["wk"], requires_grad=True)
+    bt = torch.tensor(cw["bk"], requires_grad=True)
+    y = _dense_conv(coords, cu, xt, wt, bt, 6)
+    onehot = torch.nn.functional.one_hot(torch.from_numpy(blk["id"]), int(blk["count"])).to(torch.float64)
+    xc = torch.einsum("nb,ngd->bgd", onehot, y) / onehot.sum(0)[:, None, None]
+    np.testing.assert_allclose(xc.detach().numpy(), O.conv_pool(coords, cu, k, cw["wk"], cw["bk"], blk, "none"),
+                               rtol=1e-12, atol=1e-12)
+    dxc = np.random.default_rng(9).standard_normal(xc.shape)
+    (xc * torch.from_numpy(dxc)).sum().backward()
+    dx, dw, db = O.conv_pool_backward(coords, cu, k, cw["wk"], blk, dxc)
+    np.testing.assert_allclose(dx, xt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dw, wt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(db, bt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_learned_compression_in_the_full_backward_by_central_differences():
+    coords, cu, q, k, v, gates = _rand_case(44, n_per_seq=(36,), R=6, hq=4, hkv=2, d=4)
+    cw = _conv_weights(3, 2, 4)
+    kw = dict(hq=4, hkv=2, m_cmp=2, m_win=3, topk=2, gate_mode=1, pool_rounding="none")
+    st = O.forward(coords, cu, q, k, v, gates, conv=cw, **kw)
+    do = np.random.default_rng(10).standard_normal(q.shape)
+    g = O.backward(st, do)
+    rng = np.random.default_rng(11)
+    for key, gkey in (("wk", "dwk"), ("bv", "dbv"), ("wv", "dwv")):
+        for _ in range(3):
+            idx = tuple(rng.integers(0, n) for n in cw[key].shape)
+            h = 1e-6
+            vals = []
+            for sgn in (1, -1):
+                c2 = {kk: vv.copy() for kk, vv in cw.items()}
+                c2[key][idx] += sgn * h
+                s2 = O.forward(coords, cu, q, k, v, gates, conv=c2, sel_given=st["sel"], **kw)
+                vals.append(np.sum(do * s2["out"]))
+            num = (vals[0] - vals[1]) / (2 * h)
+            assert abs(num - g[gkey][idx]) <= 1e-6 * max(1.0, abs(num)), (key, idx, num, g[gkey][idx])
+    # dK through the convolution as well
+    for _ in range(3):
+        idx = tuple(rng.integers(0, n) for n in k.shape)
+        vals = []
+        for sgn in (1, -1):
+            k2 = k.copy()
+            k2[idx] += sgn * 1e-6
+            s2 = O.forward(coords, cu, q, k2, v, gates, conv=cw, sel_given=st["sel"], **kw)
+            vals.append(np.sum(do * s2["out"]))
+        num = (vals[0] - vals[1]) / 2e-6
+        assert abs(num - g["dk"][idx]) <= 1e-6 * max(1.0, abs(num)), (idx, num, g["dk"][idx])
