@@ -43,7 +43,7 @@ FP32_LANES_PER_SM = 128
 # while the kernel's source file is byte-identical to the one profiled.
 NCU_TRAFFIC = {
     "cmp_bwd_dkv_tc_kernel": ("spatial_sparse_attention_ssa_b200/csrc/cmp_tc.cu",
-                              "1416e91a7431aecc7954f59276dc2ee191c71c97", 1.185e9,
+                              "7d0b4da601ee818c8ec43545aff7c214235d058e", 1.1887e9,
                               "profiles/cmp_bwd_dkv_dram_gigascale1024_131072.md"),
 }
 
