@@ -68,6 +68,28 @@ enum {
 };
 
 /* Shape and method parameters shared by forward and backward. */
+/*
+ * Learned compression (Direct3D-S2 "方法": the sparse 3D compression may apply a
+ * sparse 3D convolution before pooling): Kc_b, Vc_b are the block means of a
+ * submanifold sparse convolution with a 3x3x3 kernel of K and V,
+ *   y_i = b + sum_o W_o^T x_j over the tokens j of i's sequence at coords_i + offset_o
+ * (offset index o = (dx+1)*9 + (dy+1)*3 + (dz+1); empty voxels contribute nothing;
+ * repeated coordinates all count), evaluated in fp32 and rounded once to the
+ * storage type.  The selected and window branches keep the raw K and V.
+ * All pointers are device pointers owned by the caller.
+ */
+typedef struct ssa_conv {
+  const int32_t* coords; /* [N, 3] the token coordinates given to ssa_bin */
+  const float* wk;       /* [Hkv, 27, d, d] (offset, in, out): the convolution of K */
+  const float* bk;       /* [Hkv, d] its bias */
+  const float* wv;       /* [Hkv, 27, d, d]: the convolution of V */
+  const float* bv;       /* [Hkv, d] */
+  float* dwk;            /* backward outputs, same shapes, written (not accumulated) */
+  float* dbk;
+  float* dwv;
+  float* dbv;
+} ssa_conv;
+
 typedef struct ssa_params {
   int32_t hq;        /* query heads */
   int32_t hkv;       /* key/value heads; hq % hkv == 0, G = hq / hkv in {1,2,4,8,16} */
@@ -81,6 +103,8 @@ typedef struct ssa_params {
   int32_t selection; /* SSA_SEL_SCORES: the forward selects by compressed-attention score (top-k) and writes
                         saved->sel; SSA_SEL_GIVEN: saved->sel is an input the caller filled (for instance by
                         ssa_geo_select), read by the selected branch and the backward, see ssa_forward */
+  const ssa_conv* conv; /* NULL: mean-pool compression; else the learned compression (self attention only;
+                           Hkv * d <= 256); its workspace is included by ssa_workspace_size */
 } ssa_params;
 
 /*

@@ -41,12 +41,15 @@ ssa_status check_params(const ssa_params* p) {
   if (p->dtype != SSA_DTYPE_BF16 && p->dtype != SSA_DTYPE_F32) return SSA_ERR_INVALID_ARG;
   if (p->gate_mode != SSA_GATE_WEIGHTS && p->gate_mode != SSA_GATE_LOGITS) return SSA_ERR_INVALID_ARG;
   if (p->selection != SSA_SEL_SCORES && p->selection != SSA_SEL_GIVEN) return SSA_ERR_INVALID_ARG;
+  if (p->conv && (!p->conv->coords || !p->conv->wk || !p->conv->bk || !p->conv->wv || !p->conv->bv))
+    return SSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.f) || isinf(p->scale)) return SSA_ERR_INVALID_ARG;
   if (p->d != 32 && p->d != 64) return SSA_ERR_UNSUPPORTED;
   if (p->topk > 32) return SSA_ERR_UNSUPPORTED;
   const int G = p->hq / p->hkv;
   if (G & (G - 1)) return SSA_ERR_UNSUPPORTED;  // power of two
   if (G * (p->d / 32) > 32) return SSA_ERR_UNSUPPORTED;
+  if (p->conv && p->hkv * p->d > 256) return SSA_ERR_UNSUPPORTED;
   return SSA_OK;
 }
 
@@ -92,6 +95,37 @@ size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W
   if (wp) *wp = y1;
   if (wst) *wst = y2;
   return c.used;
+}
+
+// Learned-compression region after the regular workspace (0 without it).
+size_t conv_bytes(const ssa_params* p, int64_t N, int64_t B) {
+  return p->conv ? align256(sizeof(float) * ssa::conv_ws_floats(N, B, p->hkv, p->d)) + 256 : 0;
+}
+
+// Learned-compression arguments over the region at `base`.
+ssa::ConvArgs conv_args(const ssa_params* p, const ssa_partition* blk, int32_t S, int64_t N, void* base) {
+  ssa::ConvArgs c;
+  const ssa_conv* cv = p->conv;
+  c.coords = cv->coords;
+  c.blk = blk;
+  c.S = S;
+  c.N = N;
+  c.hkv = p->hkv;
+  c.d = p->d;
+  c.m = p->m_cmp;
+  c.wk = cv->wk;
+  c.bk = cv->bk;
+  c.wv = cv->wv;
+  c.bv = cv->bv;
+  c.dwk = cv->dwk;
+  c.dbk = cv->dbk;
+  c.dwv = cv->dwv;
+  c.dbv = cv->dbv;
+  char* b = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(base) + 255) & ~uintptr_t(255));
+  c.cs = reinterpret_cast<int4*>(b);
+  c.M = reinterpret_cast<float*>(b + align256(sizeof(int4) * (size_t)N));
+  c.dM = c.M + 2 * (size_t)blk->count * p->hkv * 27 * p->d;
+  return c;
 }
 
 // Cross-attention extras after the regular workspace: the gates widened to three
@@ -157,10 +191,10 @@ SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, in
   if (op == SSA_OP_BIN) return bin_bytes(S, N);
   if (op == SSA_OP_GEO_SELECT) return ssa::geo_ws_bytes(N);
   if (check_params(p) != SSA_OK) return 0;
-  if (op == SSA_OP_FORWARD) return fwd_bytes(p, S, N, B_tot, W_tot);
+  if (op == SSA_OP_FORWARD) return fwd_bytes(p, S, N, B_tot, W_tot) + conv_bytes(p, N, B_tot);
   if (op == SSA_OP_BACKWARD) {
     BwdWs w;
-    return carve_bwd(nullptr, p, S, N, B_tot, W_tot, &w);
+    return carve_bwd(nullptr, p, S, N, B_tot, W_tot, &w) + conv_bytes(p, N, B_tot);
   }
   // cross attention: N = query tokens, W_tot unused (no window branch)
   if (op == SSA_OP_CROSS_FORWARD) return fwd_bytes(p, S, N, B_tot, 0) + cross_extra_bytes(N, p->hq);
@@ -268,6 +302,11 @@ ssa_status forward_common(const ssa_params* p, const int32_t* cu, int32_t S, int
   cudaError_t e = ssa::launch_pool(p->dtype, k, v, blk, Nkv, p->hkv, p->d, saved->ks, saved->vs, saved->kc,
                                    saved->vc, st);
   if (e != cudaSuccess) return SSA_ERR_CUDA;
+  if (p->conv) {  // learned compression: Kc / Vc from the convolution instead of the plain mean
+    const ssa::ConvArgs c = conv_args(p, blk, S, Nkv, static_cast<char*>(ws) + fwd_bytes(p, S, N, blk->count,
+                                                                                           win ? win->count : 0));
+    if (ssa::conv_forward(c, p->dtype, k, v, saved->kc, saved->vc, st) != cudaSuccess) return SSA_ERR_CUDA;
+  }
   ssa::FwdArgs a;
   a.dtype = p->dtype;
   a.d = p->d;
@@ -314,8 +353,11 @@ ssa_status backward_common(const ssa_params* p, const int32_t* cu, int32_t S, in
                            const void* v, const float* gates, const ssa_saved* saved, const void* dout, float* dq,
                            float* dk, float* dv, float* dgates, void* ws, cudaStream_t st) {
   BwdWs w;
-  carve_bwd(ws, p, S, N, blk->count, win ? win->count : 0, &w);
+  const size_t used = carve_bwd(ws, p, S, N, blk->count, win ? win->count : 0, &w);
+  ssa::ConvArgs conv;
+  if (p->conv) conv = conv_args(p, blk, S, Nkv, static_cast<char*>(ws) + used);
   ssa::BwdArgs a;
+  a.conv = p->conv ? &conv : nullptr;
   a.dtype = p->dtype;
   a.d = p->d;
   a.hq = p->hq;
@@ -406,7 +448,7 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
   if (N == 0) return SSA_OK;
   if (!q || !k || !v || !gates || !out || !saved_ok(saved) || !ws) return SSA_ERR_INVALID_ARG;
   if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
-  if (ws_bytes < fwd_bytes(p, S, N, blk->count, win->count)) return SSA_ERR_WORKSPACE;
+  if (ws_bytes < fwd_bytes(p, S, N, blk->count, win->count) + conv_bytes(p, N, blk->count)) return SSA_ERR_WORKSPACE;
   return forward_common(p, cu_seqlens, S, N, N, 0, blk, win, q, k, v, gates, out, saved, ws,
                         static_cast<cudaStream_t>(stream));
 }
@@ -426,7 +468,9 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
   if (blk->count < 1 || blk->count > N || win->count < 1 || win->count > N) return SSA_ERR_INVALID_ARG;
   if ((int64_t)N * p->hkv * p->topk > INT32_MAX) return SSA_ERR_UNSUPPORTED;
   BwdWs w;
-  if (ws_bytes < carve_bwd(nullptr, p, S, N, blk->count, win->count, &w)) return SSA_ERR_WORKSPACE;
+  if (ws_bytes < carve_bwd(nullptr, p, S, N, blk->count, win->count, &w) + conv_bytes(p, N, blk->count))
+    return SSA_ERR_WORKSPACE;
+  if (p->conv && (!p->conv->dwk || !p->conv->dbk || !p->conv->dwv || !p->conv->dbv)) return SSA_ERR_INVALID_ARG;
   return backward_common(p, cu_seqlens, S, N, N, 0, blk, win, q, k, v, gates, saved, dout, dq, dk, dv, dgates, ws,
                          static_cast<cudaStream_t>(stream));
 }
@@ -440,6 +484,7 @@ SSA_API ssa_status ssa_cross_forward(const ssa_params* p, const int32_t* q_cu, i
   if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk) ||
       !saved)
     return SSA_ERR_INVALID_ARG;
+  if (p->conv) return SSA_ERR_UNSUPPORTED;  // the learned compression is built for self attention
   if (Nq == 0) return SSA_OK;
   if (Nkv < 1 || !q || !k || !v || !gates || !out || !saved_ok(saved) || !ws) return SSA_ERR_INVALID_ARG;
   if (blk->count < 1 || blk->count > Nkv) return SSA_ERR_INVALID_ARG;
@@ -462,6 +507,7 @@ SSA_API ssa_status ssa_cross_backward(const ssa_params* p, const int32_t* q_cu, 
   if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk) ||
       !saved)
     return SSA_ERR_INVALID_ARG;
+  if (p->conv) return SSA_ERR_UNSUPPORTED;
   if (Nkv > 0 && dk && dv && Nq == 0) {  // no queries: the key gradients are zero
     cudaStream_t st0 = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(dk, 0, sizeof(float) * Nkv * p->hkv * p->d, st0) != cudaSuccess ||

@@ -1339,6 +1339,8 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                                                  a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
                                                  a.Dc + 2 * rows, a.dk, a.dv);
   }
+  if (a.conv)  // the learned compression: dK, dV through the convolution, dW, db
+    return conv_backward(*a.conv, a.dtype, a.k, a.v, a.dkc, a.dvc, a.dk, a.dv, st);
   SSA_LAUNCH("cmp_scatter_kernel", cmp_scatter_kernel, grid_1d(a.Nkv * a.hkv * D / 4, 256, 148 * 32), 256, 0, st,
              a.dkc, a.dvc, a.blk->id, a.blk->ptr, a.Nkv, btot, a.hkv, D, a.dk, a.dv);
   return cudaGetLastError();

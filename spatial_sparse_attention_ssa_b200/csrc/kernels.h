@@ -40,10 +40,30 @@ struct FwdArgs {
   int32_t *win_cnt, *win_pre, *win_scan;  // [W + 1] window work plan
 };
 
+// Learned compression (sparse 3D convolution before the block mean), see conv.cu.
+struct ConvArgs {
+  const int32_t* coords;      // [N, 3] voxel coordinates
+  const ssa_partition* blk;
+  int S;
+  int64_t N;
+  int hkv, d, m;
+  const float *wk, *bk, *wv, *bv;  // [Hkv, 27, d, d], [Hkv, d]
+  float *dwk, *dbk, *dwv, *dbv;    // backward outputs
+  int4* cs;                   // workspace: [N] coordinates in block order
+  float* M;                   // workspace: [2][B][Hkv][27][d]
+  float* dM;                  // workspace: [2][B][Hkv][27][d] (backward)
+};
+size_t conv_ws_floats(int64_t N, int64_t B, int hkv, int d);
+cudaError_t conv_forward(const ConvArgs& c, int dtype, const void* k, const void* v, void* kc, void* vc,
+                         cudaStream_t st);
+cudaError_t conv_backward(const ConvArgs& c, int dtype, const void* k, const void* v, const float* dkc,
+                          const float* dvc, float* dk, float* dv, cudaStream_t st);
+
 struct BwdArgs {
   int dtype, d, hq, hkv, topk, gate_mode, m_cmp, m_win;
   int cross;    // as in FwdArgs
   int64_t Nkv;  // key / value tokens (= N unless cross)
+  const ConvArgs* conv;  // learned compression, or null (mean pool)
   int use_tc;
   int* status;
   float scale;

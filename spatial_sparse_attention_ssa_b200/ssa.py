@@ -39,11 +39,17 @@ class SSAError(RuntimeError):
                                                  _lib().ssa_error_string(status).decode()))
 
 
+class Conv(ctypes.Structure):
+    _fields_ = [("coords", ctypes.c_void_p), ("wk", ctypes.c_void_p), ("bk", ctypes.c_void_p),
+                ("wv", ctypes.c_void_p), ("bv", ctypes.c_void_p), ("dwk", ctypes.c_void_p),
+                ("dbk", ctypes.c_void_p), ("dwv", ctypes.c_void_p), ("dbv", ctypes.c_void_p)]
+
+
 class Params(ctypes.Structure):
     _fields_ = [("hq", ctypes.c_int32), ("hkv", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("m_cmp", ctypes.c_int32), ("m_win", ctypes.c_int32), ("topk", ctypes.c_int32),
                 ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("gate_mode", ctypes.c_int32),
-                ("selection", ctypes.c_int32)]
+                ("selection", ctypes.c_int32), ("conv", ctypes.POINTER(Conv))]
 
 
 class Partition(ctypes.Structure):
@@ -230,12 +236,38 @@ def ssa_bin_noalloc(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cm
 # ---------------------------------------------------------------------------
 
 
+@dataclass
+class ConvWeights:
+    """Learned compression: a sparse 3x3x3 convolution of K and V before the block
+    mean.  coords int32 [N, 3]; wk / wv fp32 [Hkv, 27, d, d] (offset, in, out); bk /
+    bv fp32 [Hkv, d]; the gradients dwk, dbk, dwv, dbv (same shapes) are written by
+    ssa_backward."""
+    coords: torch.Tensor
+    wk: torch.Tensor
+    bk: torch.Tensor
+    wv: torch.Tensor
+    bv: torch.Tensor
+    dwk: torch.Tensor | None = None
+    dbk: torch.Tensor | None = None
+    dwv: torch.Tensor | None = None
+    dbv: torch.Tensor | None = None
+
+    def __post_init__(self):
+        for name in ("dwk", "dbk", "dwv", "dbv"):
+            if getattr(self, name) is None:
+                setattr(self, name, torch.zeros_like(getattr(self, name[1:])))
+        self._c = Conv(*(_ptr(getattr(self, f)) for f, _ in Conv._fields_))
+
+
 def make_params(hq, hkv, d, m_cmp, m_win, topk, dtype: torch.dtype, gate_mode: int,
-                scale: float = 0.0, selection: int = SEL_SCORES) -> Params:
+                scale: float = 0.0, selection: int = SEL_SCORES, conv: ConvWeights | None = None) -> Params:
     dt = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32 if dtype == torch.float32 else None
     if dt is None:
         raise ValueError("dtype must be torch.bfloat16 or torch.float32")
-    return Params(hq, hkv, d, m_cmp, m_win, topk, scale, dt, gate_mode, selection)
+    prm = Params(hq, hkv, d, m_cmp, m_win, topk, scale, dt, gate_mode, selection,
+                 ctypes.pointer(conv._c) if conv is not None else None)
+    prm._conv = conv  # keeps the weights (and the struct the pointer refers to) alive
+    return prm
 
 
 @dataclass
