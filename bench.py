@@ -72,6 +72,7 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-geo", action="store_true", help="skip the separate timing of geometric block routing")
     ap.add_argument("--no-cross", action="store_true", help="skip the separate timing of cross attention")
+    ap.add_argument("--no-conv", action="store_true", help="skip the separate timing of the learned compression")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -514,6 +515,50 @@ def run_ours(a):
                          "voxel tokens (compressed + selected branches, same heads, k, m_cmp)"}
         del c_saved, c_grads, c_wf, c_wb
 
+    # ---- learned compression (sparse 3x3x3 convolution before the block mean), the
+    # same step with the convolution on; its own kernels' times from the library's events
+    learned = None
+    if not a.no_conv:
+        rng = np.random.default_rng(11)
+        std = 0.3 / np.sqrt(9 * w.d)
+        cw = [torch.from_numpy((std * rng.standard_normal((w.hkv, 27, w.d, w.d))).astype(np.float32)).to(dev),
+              torch.from_numpy((0.1 * rng.standard_normal((w.hkv, w.d))).astype(np.float32)).to(dev),
+              torch.from_numpy((std * rng.standard_normal((w.hkv, 27, w.d, w.d))).astype(np.float32)).to(dev),
+              torch.from_numpy((0.1 * rng.standard_normal((w.hkv, w.d))).astype(np.float32)).to(dev)]
+        conv = ssa.ConvWeights(coords, *cw)
+        pc = ssa.make_params(w.hq, w.hkv, w.d, w.m_cmp, w.m_win, w.topk, torch.bfloat16, w.gate_mode, conv=conv)
+        l_wf = torch.empty(ssa.workspace_size(ssa.OP_FORWARD, pc, s, n, blk.count, win.count), dtype=torch.uint8,
+                           device=dev)
+        l_wb = torch.empty(ssa.workspace_size(ssa.OP_BACKWARD, pc, s, n, blk.count, win.count), dtype=torch.uint8,
+                           device=dev)
+
+        def conv_step():
+            b_, w_ = ssa.ssa_bin(coords, cu, w.R, w.m_cmp, w.m_win, out=bins, workspace=ws_bin)
+            ssa.ssa_forward(pc, cu, b_, w_, q, k, v, gates, out=out, saved=saved, workspace=l_wf)
+            ssa.ssa_backward(pc, cu, b_, w_, q, k, v, gates, saved, do, grads=grads, workspace=l_wb)
+
+        for _ in range(3):
+            conv_step()
+        check_device("learned-compression warm-up")
+        el = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+        ssa.profile_read()
+        ssa.profile_enable(True)
+        for i in range(a.steps):
+            flush.zero_()
+            el[i][0].record()
+            conv_step()
+            el[i][1].record()
+        torch.cuda.synchronize()
+        ssa.profile_enable(False)
+        cprof = ssa.profile_read()
+        check_device("learned compression")
+        l_ms = sum(a_.elapsed_time(b_) for a_, b_ in el) / a.steps
+        conv_k = {nm: tot / a.steps for nm, (tot, cnt) in cprof.items() if nm.startswith("conv_")}
+        learned = {"ms_per_step": l_ms, "tokens_per_s": n / (l_ms / 1e3), "conv_kernels_ms_per_step": conv_k,
+                   "what": "the benchmark step with Kc / Vc from a sparse 3x3x3 convolution of K and V (random "
+                           "N(0, 0.3^2/(9d)) weights) before the block mean, gradients to the weights included"}
+        del l_wf, l_wb
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -531,7 +576,7 @@ def run_ours(a):
                 "config": cfg, "roofline": roof, "roofline_exp": exp_roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(launches),
                 "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel, "geo_routing": geo,
-                "cross_attention": cross,
+                "cross_attention": cross, "learned_compression": learned,
                 "peaks_source": peaks["_source"]}
         print(json.dumps(line), flush=True)
     if world > 1:
