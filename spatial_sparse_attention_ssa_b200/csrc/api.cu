@@ -99,7 +99,7 @@ size_t fwd_bytes(const ssa_params* p, int32_t S, int64_t N, int64_t B, int64_t W
 
 // Learned-compression region after the regular workspace (0 without it).
 size_t conv_bytes(const ssa_params* p, int64_t N, int64_t B) {
-  return p->conv ? align256(sizeof(float) * ssa::conv_ws_floats(N, B, p->hkv, p->d)) + 256 : 0;
+  return p->conv ? align256(sizeof(float) * ssa::conv_ws_floats(N, B, p->hkv, p->d, p->m_cmp)) + 256 : 0;
 }
 
 // Learned-compression arguments over the region at `base`.
@@ -125,6 +125,7 @@ ssa::ConvArgs conv_args(const ssa_params* p, const ssa_partition* blk, int32_t S
   c.cs = reinterpret_cast<int4*>(b);
   c.M = reinterpret_cast<float*>(b + align256(sizeof(int4) * (size_t)N));
   c.dM = c.M + 2 * (size_t)blk->count * p->hkv * 27 * p->d;
+  c.table = reinterpret_cast<int*>(c.dM + 2 * (size_t)blk->count * p->hkv * 27 * p->d);
   return c;
 }
 

@@ -11,8 +11,10 @@
 // no atomics).
 //
 // Neighbours of a token of block b lie in the 27 cells around b's cell; each CTA looks
-// their block ids up once (binary search over the sequence's sorted cell keys) and
-// then scans those blocks' members (coordinates in block order) for exact matches.
+// their block ids up once (binary search over the sequence's sorted cell keys).  For
+// m <= 8 a per-block table of the m^3 voxels of the cell (token, or -1 if empty, -2 if
+// several tokens share the voxel) answers a probe in one load; otherwise, and for
+// shared voxels, the block's members (coordinates in block order) are scanned.
 // Repeated coordinates are all matched, as a dense grid with summed duplicates would.
 #include "common.cuh"
 #include "kernels.h"
@@ -23,11 +25,22 @@ namespace {
 constexpr int kConvThreads = 256;
 constexpr int kConvWarps = kConvThreads / 32;
 
-__global__ void conv_prep_kernel(const int32_t* __restrict__ coords, const int32_t* __restrict__ perm, int64_t N,
-                                 int4* __restrict__ cs) {
+constexpr int kConvTableMaxM = 8;  // cells of up to 8^3 voxels get a lookup table
+
+__device__ __forceinline__ int local_voxel(int x, int y, int z, int m) { return ((x % m) * m + (y % m)) * m + (z % m); }
+
+// cs[p] = (x, y, z, token) of blk.perm[p]; with a table, table[b][voxel] = token (-2: shared)
+__global__ void conv_prep_kernel(const int32_t* __restrict__ coords, const int32_t* __restrict__ perm,
+                                 const int32_t* __restrict__ bid, int64_t N, int m, int4* __restrict__ cs,
+                                 int* __restrict__ table) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N; i += (int64_t)gridDim.x * blockDim.x) {
     const int32_t t = perm[i];
-    cs[i] = make_int4(coords[3 * (int64_t)t], coords[3 * (int64_t)t + 1], coords[3 * (int64_t)t + 2], t);
+    const int x = coords[3 * (int64_t)t], y = coords[3 * (int64_t)t + 1], z = coords[3 * (int64_t)t + 2];
+    cs[i] = make_int4(x, y, z, t);
+    if (table) {
+      int* slot = table + (int64_t)bid[t] * m * m * m + local_voxel(x, y, z, m);
+      if (atomicCAS(slot, -1, t) != -1) atomicExch(slot, -2);
+    }
   }
 }
 
@@ -69,12 +82,14 @@ struct Probe {
   int px, py, pz;  // the point
   int q, qend;     // remaining members of the block to scan
   int blk;         // that block
+  int direct;      // the token found in the table, returned first (-1: none)
 };
 __device__ __forceinline__ Probe make_probe(int4 c, int o, int sign, int m, const int* nb, const int32_t* bptr,
-                                            int kx, int ky, int kz) {
+                                            int kx, int ky, int kz, const int* __restrict__ table) {
   Probe pr;
   pr.q = pr.qend = 0;
   pr.blk = -1;
+  pr.direct = -1;
   pr.px = c.x + sign * (o / 9 - 1);
   pr.py = c.y + sign * ((o / 3) % 3 - 1);
   pr.pz = c.z + sign * (o % 3 - 1);
@@ -83,13 +98,23 @@ __device__ __forceinline__ Probe make_probe(int4 c, int o, int sign, int m, cons
     const int b = nb[(dx + 1) * 9 + (dy + 1) * 3 + (dz + 1)];
     if (b >= 0) {
       pr.blk = b;
-      pr.q = bptr[b];
-      pr.qend = bptr[b + 1];
+      const int tv = table ? table[(int64_t)b * m * m * m + local_voxel(pr.px, pr.py, pr.pz, m)] : -2;
+      if (tv >= 0) {
+        pr.direct = tv;
+      } else if (tv == -2) {  // no table, or several tokens on the voxel: scan the block
+        pr.q = bptr[b];
+        pr.qend = bptr[b + 1];
+      }
     }
   }
   return pr;
 }
 __device__ __forceinline__ int next_match(Probe& pr, const int4* __restrict__ cs) {
+  if (pr.direct >= 0) {
+    const int t = pr.direct;
+    pr.direct = -1;
+    return t;
+  }
   for (; pr.q < pr.qend; ++pr.q) {
     const int4 r = cs[pr.q];
     if (r.x == pr.px && r.y == pr.py && r.z == pr.pz) {
@@ -105,7 +130,7 @@ template <typename T>
 __global__ void __launch_bounds__(kConvThreads) conv_gather_kernel(
     const T* __restrict__ k, const T* __restrict__ v, const int4* __restrict__ cs, const int32_t* __restrict__ bptr,
     const int32_t* __restrict__ key, const int32_t* __restrict__ bcu, int S, int B, int hkv, int d, int m,
-    float* __restrict__ M) {
+    const int* __restrict__ table, float* __restrict__ M) {
   extern __shared__ float ms[];  // [2][hkv][27][d]
   __shared__ int nb[27];
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -118,7 +143,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_gather_kernel(
     const int* kb = key + 3 * (int64_t)b;
     const int p0 = bptr[b], p1 = bptr[b + 1];
     for (int p = p0 + w; p < p1; p += kConvWarps) {
-      Probe pr = make_probe(cs[p], lane, 1, m, nb, bptr, kb[0], kb[1], kb[2]);
+      Probe pr = make_probe(cs[p], lane, 1, m, nb, bptr, kb[0], kb[1], kb[2], table);
       for (;;) {
         const int j = next_match(pr, cs);
         unsigned bal = __ballot_sync(0xffffffffu, j >= 0);
@@ -149,7 +174,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_gather_kernel(
 __global__ void __launch_bounds__(kConvThreads) conv_dx_kernel(
     const float* __restrict__ dM, const int4* __restrict__ cs, const int32_t* __restrict__ bptr,
     const int32_t* __restrict__ key, const int32_t* __restrict__ bcu, int S, int B, int hkv, int d, int m,
-    float* __restrict__ dk, float* __restrict__ dv) {
+    const int* __restrict__ table, float* __restrict__ dk, float* __restrict__ dv) {
   __shared__ int nb[27];
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int row = hkv * d;
@@ -165,7 +190,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_dx_kernel(
       float ak[kMaxE], av[kMaxE];
 #pragma unroll
       for (int x = 0; x < kMaxE; ++x) ak[x] = av[x] = 0.f;
-      Probe pr = make_probe(c, lane, -1, m, nb, bptr, kb[0], kb[1], kb[2]);
+      Probe pr = make_probe(c, lane, -1, m, nb, bptr, kb[0], kb[1], kb[2], table);
       for (;;) {
         const int i = next_match(pr, cs);
         unsigned bal = __ballot_sync(0xffffffffu, i >= 0);
@@ -300,28 +325,34 @@ cudaError_t conv_gather(const ConvArgs& c, const void* k, const void* v, float* 
   }
   SSA_LAUNCH("conv_gather_kernel", conv_gather_kernel<T>, conv_grid(c.blk->count), kConvThreads, smem, st,
              static_cast<const T*>(k), static_cast<const T*>(v), c.cs, c.blk->ptr, c.blk->key, c.blk->cu, c.S,
-             (int)c.blk->count, c.hkv, c.d, c.m, M);
+             (int)c.blk->count, c.hkv, c.d, c.m, c.m <= kConvTableMaxM ? c.table : nullptr, M);
   return cudaGetLastError();
 }
 
-void launch_prep(const ConvArgs& c, cudaStream_t st) {
+cudaError_t launch_prep(const ConvArgs& c, cudaStream_t st) {
   const int64_t g = (c.N + 255) / 256;
+  int* table = c.m <= kConvTableMaxM ? c.table : nullptr;
+  if (table && cudaMemsetAsync(table, 0xff, sizeof(int) * (size_t)c.blk->count * c.m * c.m * c.m, st) != cudaSuccess)
+    return cudaErrorUnknown;
   SSA_LAUNCH("conv_prep_kernel", conv_prep_kernel, (int)(g < 148 * 32 ? (g > 0 ? g : 1) : 148 * 32), 256, 0, st,
-             c.coords, c.blk->perm, c.N, c.cs);
+             c.coords, c.blk->perm, c.blk->id, c.N, c.m, c.cs, table);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t conv_ws_floats(int64_t N, int64_t B, int hkv, int d) {
-  // cs (N int4), M [2][B][hkv][27][d], dM (the same)
-  return (size_t)N * 4 + 2 * (size_t)(2 * B * hkv * 27 * d) + 64;
+size_t conv_ws_floats(int64_t N, int64_t B, int hkv, int d, int m) {
+  // cs (N int4), M [2][B][hkv][27][d], dM (the same), the voxel table [B][m^3]
+  const size_t table = m <= kConvTableMaxM ? (size_t)B * m * m * m : 0;
+  return (size_t)N * 4 + 2 * (size_t)(2 * B * hkv * 27 * d) + table + 128;
 }
 
 cudaError_t conv_forward(const ConvArgs& c, int dtype, const void* k, const void* v, void* kc, void* vc,
                          cudaStream_t st) {
   const int64_t B = c.blk->count;
-  launch_prep(c, st);
-  cudaError_t e = dtype == SSA_DTYPE_BF16 ? conv_gather<__nv_bfloat16>(c, k, v, c.M, st) : conv_gather<float>(c, k, v, c.M, st);
+  cudaError_t e = launch_prep(c, st);
+  if (e != cudaSuccess) return e;
+  e = dtype == SSA_DTYPE_BF16 ? conv_gather<__nv_bfloat16>(c, k, v, c.M, st) : conv_gather<float>(c, k, v, c.M, st);
   if (e != cudaSuccess) return e;
   // Xc[g][b][n] = bias[g][n] + sum_K M[kv][b][g][K] W[g][K][n]
   const int per_g = 27 * c.d;
@@ -360,8 +391,9 @@ cudaError_t conv_backward(const ConvArgs& c, int dtype, const void* k, const voi
   const int64_t B = c.blk->count;
   const int per_g = 27 * c.d;
   const int64_t per_kv = B * c.hkv * per_g;
-  launch_prep(c, st);
-  cudaError_t e = dtype == SSA_DTYPE_BF16 ? conv_gather<__nv_bfloat16>(c, k, v, c.M, st) : conv_gather<float>(c, k, v, c.M, st);
+  cudaError_t e = launch_prep(c, st);
+  if (e != cudaSuccess) return e;
+  e = dtype == SSA_DTYPE_BF16 ? conv_gather<__nv_bfloat16>(c, k, v, c.M, st) : conv_gather<float>(c, k, v, c.M, st);
   if (e != cudaSuccess) return e;
   // dM[kv][b][g][K] = sum_n dXc[g][b][n] W[g][K][n]
   {
@@ -422,7 +454,7 @@ cudaError_t conv_backward(const ConvArgs& c, int dtype, const void* k, const voi
   SSA_LAUNCH("conv_db_kernel", conv_db_kernel, (2 * c.hkv * c.d + 255) / 256, 256, 0, st, dkc, dvc, (int)B, c.hkv,
              c.d, c.dbk, c.dbv);
   SSA_LAUNCH("conv_dx_kernel", conv_dx_kernel, conv_grid(B), kConvThreads, 0, st, c.dM, c.cs, c.blk->ptr,
-             c.blk->key, c.blk->cu, c.S, (int)B, c.hkv, c.d, c.m, dk, dv);
+             c.blk->key, c.blk->cu, c.S, (int)B, c.hkv, c.d, c.m, c.m <= kConvTableMaxM ? c.table : nullptr, dk, dv);
   return cudaGetLastError();
 }
 

@@ -52,8 +52,9 @@ struct ConvArgs {
   int4* cs;                   // workspace: [N] coordinates in block order
   float* M;                   // workspace: [2][B][Hkv][27][d]
   float* dM;                  // workspace: [2][B][Hkv][27][d] (backward)
+  int* table;                 // workspace: [B][m^3] voxel -> token (m <= 8)
 };
-size_t conv_ws_floats(int64_t N, int64_t B, int hkv, int d);
+size_t conv_ws_floats(int64_t N, int64_t B, int hkv, int d, int m);
 cudaError_t conv_forward(const ConvArgs& c, int dtype, const void* k, const void* v, void* kc, void* vc,
                          cudaStream_t st);
 cudaError_t conv_backward(const ConvArgs& c, int dtype, const void* k, const void* v, const float* dkc,

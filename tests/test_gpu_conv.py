@@ -6,7 +6,8 @@ sums of the neighbours first, then one product with the weights), so the stored
 Kc / Vc may differ from the oracle's by one unit in the last place of the storage
 type; everything downstream is compared with the usual tolerances, rows touched by a
 certified selection near-tie left out.  fp32 inputs (SIMT attention kernels) and
-bf16 inputs (tensor-core kernels); weight and bias gradients included.
+bf16 inputs (tensor-core kernels); weight and bias gradients included; the table and
+the scanning lookups of neighbours, repeated voxels included.
 """
 import numpy as np
 import pytest
@@ -28,10 +29,21 @@ def _weights(seed, hkv, d, std):
             "bv": (0.1 * rng.standard_normal((hkv, d))).astype(np.float32)}
 
 
-@pytest.mark.parametrize("hq,d,dtype", [(4, 32, "f32"), (16, 64, "bf16")])
-def test_learned_compression_forward_backward(hq, d, dtype):
+@pytest.mark.parametrize("hq,d,dtype,m,dup", [(4, 32, "f32", 4, False), (16, 64, "bf16", 4, False),
+                                               (4, 32, "f32", 4, True), (4, 32, "f32", 12, False)])
+def test_learned_compression_forward_backward(hq, d, dtype, m, dup):
+    """m = 4: the per-block voxel table answers the probes; dup: some voxels hold two
+    tokens (the table marks them and the probes scan); m = 12: no table, every probe
+    scans the neighbouring block."""
     w = W.small_shell(seed=53, R=40, n_prims=2, lo=4.0, hi=9.0, n_keep=700, n_seqs=2, hq=hq, hkv=2, d=d,
-                      m_cmp=4, m_win=4, topk=8, dtype=dtype)
+                      m_cmp=m, m_win=4, topk=8, dtype=dtype)
+    if dup:  # token i + 1 takes the voxel of token i, for every 7th i of each sequence
+        coords = w.coords.copy()
+        for s in range(w.s):
+            a, e = int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1])
+            for i in range(a, e - 1, 7):
+                coords[i + 1] = coords[i]
+        w = W.Workload(**{**w.__dict__, "coords": coords})
     t = W.make_tensors(w)
     cw = _weights(5, w.hkv, w.d, 0.3 / np.sqrt(9 * w.d))
     dev = "cuda"
