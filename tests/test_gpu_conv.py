@@ -78,7 +78,9 @@ def test_learned_compression_forward_backward(hq, d, dtype, m, dup):
 
     atol = ATOL[dtype]
     toks = np.arange(w.n)
-    flips = check_selection(saved.sel.cpu().numpy(), st, toks, tau=1e-6 if dtype == "f32" else 5e-2)
+    # bf16: a Kc element one ulp (<= 2^-7 relative) off moves a score by about |q| * ulp / sqrt(d)
+    # and a group's summed probability by well under 1e-3: a near-tie within that is certified
+    flips = check_selection(saved.sel.cpu().numpy(), st, toks, tau=1e-6 if dtype == "f32" else 1e-3)
     G = w.hq // w.hkv
     rows = np.ones((w.n, w.hq), bool)
     for tt, gg in flips:
