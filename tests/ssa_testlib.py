@@ -37,7 +37,7 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-class GpuRun:
+class DeviceRun:
     """Inputs on the device and the results of one bin/forward/backward pass."""
 
     def __init__(self, w: W.Workload, t: W.Tensors, backward: bool = True, dev: str = "cuda"):
@@ -116,7 +116,7 @@ def max_abs(a, b) -> float:
     return float(np.nanmax(d)) if d.size else 0.0
 
 
-def compare_forward(run: GpuRun, st: O.State, tokens, atol: float):
+def compare_forward(run: DeviceRun, st: O.State, tokens, atol: float):
     """Element-wise parity of Kc/Vc (bit-exact), selection (near-tie rule), the
     three branch outputs, their lse and the combined output on `tokens`."""
     w = run.w
@@ -152,7 +152,7 @@ def compare_forward(run: GpuRun, st: O.State, tokens, atol: float):
     return errs, flips
 
 
-def compare_backward(run: GpuRun, st: O.State, g: dict, atol: float, flips):
+def compare_backward(run: DeviceRun, st: O.State, g: dict, atol: float, flips):
     """Gradients; rows / keys touched by a certified selection flip are left out."""
     w = run.w
     dq, dk, dv, dg = (f64(x) for x in run.grads)

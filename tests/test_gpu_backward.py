@@ -5,13 +5,13 @@ import torch
 
 from oracle import ssa_oracle as O
 from spatial_sparse_attention_ssa_b200 import workloads as W
-from tests.ssa_testlib import ATOL, GpuRun, compare_backward, compare_forward, f64, run_oracle
+from tests.ssa_testlib import ATOL, DeviceRun, compare_backward, compare_forward, f64, run_oracle
 
 pytestmark = pytest.mark.gpu
 
 
 def _bwd_parity(w, t):
-    run = GpuRun(w, t).run()
+    run = DeviceRun(w, t).run()
     st = run_oracle(w, t)
     _, flips = compare_forward(run, st, np.arange(w.n), ATOL[w.dtype])
     g = O.backward(st, t.as_f32("do").astype(np.float64))
@@ -53,7 +53,7 @@ def test_zero_gates_give_zero_input_gradients():
     w = W.small_shell(seed=12, R=32, n_prims=2, lo=4.0, hi=9.0, n_keep=600, gate_mode=0)
     t = W.make_tensors(w)
     t.gates[:] = 0.0
-    run = GpuRun(w, t).run()
+    run = DeviceRun(w, t).run()
     dq, dk, dv, dg = run.grads
     assert not dq.abs().max().item() and not dk.abs().max().item() and not dv.abs().max().item()
     assert dg.abs().max().item() > 0
@@ -67,7 +67,7 @@ def test_gradient_sums():
     2e-2 + 1e-3 x (sum of the absolute values of the terms)."""
     w = W.small_shell(seed=13, R=40, n_prims=2, lo=5.0, hi=11.0, n_keep=1500)
     t = W.make_tensors(w)
-    run = GpuRun(w, t).run()
+    run = DeviceRun(w, t).run()
     dq, dk, dv, dg = (f64(x) for x in run.grads)
     gw = O.gate_weights(t.gates, w.gate_mode)
     do = t.as_f32("do").astype(np.float64)

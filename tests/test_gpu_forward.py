@@ -6,13 +6,13 @@ import torch
 
 from oracle import ssa_oracle as O
 from spatial_sparse_attention_ssa_b200 import workloads as W
-from tests.ssa_testlib import ATOL, GpuRun, compare_forward, f64, run_oracle
+from tests.ssa_testlib import ATOL, DeviceRun, compare_forward, f64, run_oracle
 
 pytestmark = pytest.mark.gpu
 
 
 def _parity(w, t, tokens=None):
-    run = GpuRun(w, t, backward=False).run(backward=False)
+    run = DeviceRun(w, t, backward=False).run(backward=False)
     st = run_oracle(w, t)
     toks = np.arange(w.n) if tokens is None else tokens
     errs, flips = compare_forward(run, st, toks, ATOL[w.dtype])
@@ -72,13 +72,13 @@ def test_varlen_with_empty_and_single_token_sequences():
 def test_batch_equals_separate_calls():
     w = W.small_shell(seed=7, R=32, n_prims=2, lo=4.0, hi=9.0, n_keep=800, n_seqs=3)
     t = W.make_tensors(w, with_do=False)
-    run = GpuRun(w, t, backward=False).run(backward=False)
+    run = DeviceRun(w, t, backward=False).run(backward=False)
     for s in range(w.s):
         a, b = int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1])
         ws = W.Workload("part", w.R, w.coords[a:b], np.array([0, b - a], np.int32), w.hq, w.hkv, w.d, w.m_cmp,
                         w.m_win, w.topk, w.dtype, w.gate_mode, w.seed)
         ts = W.Tensors(t.q[a:b], t.k[a:b], t.v[a:b], t.gates[a:b], None, t.dtype)
-        r2 = GpuRun(ws, ts, backward=False).run(backward=False)
+        r2 = DeviceRun(ws, ts, backward=False).run(backward=False)
         np.testing.assert_array_equal(f64(r2.out), f64(run.out[a:b]))
         off = run.blk.cu[s].item()
         sel = run.saved.sel[a:b].cpu().numpy()
@@ -88,9 +88,9 @@ def test_batch_equals_separate_calls():
 def test_token_permutation_equivariance():
     w = W.small_shell(seed=8, R=40, n_prims=2, lo=5.0, hi=11.0, n_keep=1200)
     t = W.make_tensors(w, with_do=False)
-    run = GpuRun(w, t, backward=False).run(backward=False)
+    run = DeviceRun(w, t, backward=False).run(backward=False)
     w2, t2, src = W.permute_workload(w, t, seed=1)
-    run2 = GpuRun(w2, t2, backward=False).run(backward=False)
+    run2 = DeviceRun(w2, t2, backward=False).run(backward=False)
     np.testing.assert_array_equal(run2.blk.id.cpu().numpy(), run.blk.id.cpu().numpy()[src])
     np.testing.assert_array_equal(run2.saved.sel.cpu().numpy(), run.saved.sel.cpu().numpy()[src])
     np.testing.assert_allclose(f64(run2.out), f64(run.out)[src], atol=1e-2)
@@ -102,8 +102,8 @@ def test_one_hot_gates_isolate_each_branch():
     for c in range(3):
         t.gates[:] = 0.0
         t.gates[:, :, c] = 1.0
-        run = GpuRun(w, t, backward=False).run(backward=False)
+        run = DeviceRun(w, t, backward=False).run(backward=False)
         assert torch.equal(run.out, run.saved.o_branch[c].to(run.out.dtype))
     t.gates[:] = 0.0
-    run = GpuRun(w, t, backward=False).run(backward=False)
+    run = DeviceRun(w, t, backward=False).run(backward=False)
     assert not run.out.float().abs().max().item()

@@ -18,7 +18,7 @@ import pytest
 
 from oracle import ssa_oracle as O
 from spatial_sparse_attention_ssa_b200 import workloads as W
-from tests.ssa_testlib import ATOL, GpuRun, compare_forward, f64, max_abs, run_oracle
+from tests.ssa_testlib import ATOL, DeviceRun, compare_forward, f64, max_abs, run_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -49,7 +49,7 @@ def _sample_tokens(w, n_per_seq: int, seed: int) -> np.ndarray:
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 def test_forward_sampled_rows_at_full_size(cfg):
     w, t = _load(cfg)
-    run = GpuRun(w, t, backward=False).run(backward=False)
+    run = DeviceRun(w, t, backward=False).run(backward=False)
     toks = _sample_tokens(w, 48 if w.s == 1 else 16, seed=cfg)
     st = run_oracle(w, t, tokens=toks)
     errs, flips = compare_forward(run, st, toks, ATOL[w.dtype])
@@ -58,7 +58,7 @@ def test_forward_sampled_rows_at_full_size(cfg):
 
 def test_backward_sampled_rows_and_sums_at_full_size():
     w, t = _load(5)
-    run = GpuRun(w, t).run()
+    run = DeviceRun(w, t).run()
     toks = _sample_tokens(w, 32, seed=55)
     st = run_oracle(w, t, tokens=toks)
     _, flips = compare_forward(run, st, toks, ATOL[w.dtype])
@@ -96,7 +96,7 @@ def test_window_gradients_of_sampled_windows_at_full_size():
     gates = np.zeros_like(t.gates)
     gates[:, :, 2] = 1.0  # window branch only: the other branches add exact zeros to dK / dV
     t = dataclasses.replace(t, gates=gates)
-    run = GpuRun(w, t).run()
+    run = DeviceRun(w, t).run()
     wb = O.bin_tokens(w.coords, w.cu_seqlens, w.m_win)
     sizes = np.diff(wb["ptr"])
     rng = np.random.default_rng(7)

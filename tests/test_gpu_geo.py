@@ -22,7 +22,7 @@ import torch
 from oracle import ssa_oracle as O
 from spatial_sparse_attention_ssa_b200 import ssa
 from spatial_sparse_attention_ssa_b200 import workloads as W
-from tests.ssa_testlib import ATOL, GpuRun, compare_backward, compare_forward, pool_rounding
+from tests.ssa_testlib import ATOL, DeviceRun, compare_backward, compare_forward, pool_rounding
 
 pytestmark = pytest.mark.gpu
 
@@ -107,7 +107,7 @@ def test_sampled_tokens_at_benchmark_size():
 
 def _run_given(w, t, sel=None):
     """bin -> geometric routing -> forward with the given selection -> backward."""
-    run = GpuRun(w, t)
+    run = DeviceRun(w, t)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     run.p = ssa.make_params(w.hq, w.hkv, w.d, w.m_cmp, w.m_win, w.topk, tdt, w.gate_mode,
                             selection=ssa.SEL_GIVEN)
