@@ -395,26 +395,58 @@ __global__ void __launch_bounds__(128) win_fwd_kernel(const T* __restrict__ q, c
 // ---------------------------------------------------------------------------
 // gated combine: out = sum_c w_c * o_c
 // ---------------------------------------------------------------------------
+// The combine streams the [3, rows, D] branch outputs as one contiguous range: a warp
+// takes 256 consecutive float4 slots (16 rows of 64 or 32 rows of 32), lane t the
+// slots t, t + 32, ..., so each load instruction of the warp reads 512 contiguous
+// bytes (a lane owning 128 contiguous bytes instead makes every instruction touch 32
+// lines, and the L1 wavefront rate, not HBM, sets the pace).  The branch outputs are
+// read once: streaming loads.
+constexpr int kSlotsPerWarp = 256;
+
+__device__ __forceinline__ float4 ldcs4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ void store4(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const float* v) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+
+// out = sum_c w_c o_c over the nbr branches (per row; w = gate weights)
 template <typename T, int D>
 __global__ void combine_kernel(const float* __restrict__ ob, const float* __restrict__ gates, int64_t rows, int mode,
                                int nbr, T* __restrict__ out) {
-  constexpr int NT = D / 32;
-  const int64_t total = rows * NT;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / NT;
-    const int sub = (int)(i % NT);
-    float acc[32], x[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+  const int64_t total4 = rows * (D / 4);
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t chunk = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; chunk * kSlotsPerWarp < total4;
+       chunk += nwarps) {
+    float4 x[3][8];
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
       if (c >= nbr) break;
-      const float w = gate_weight(gates, row * 3 + c, mode);
-      load32(ob + ((int64_t)c * rows + row) * D + sub * 32, x);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) acc[e] = fmaf(w, x[e], acc[e]);
+      for (int i = 0; i < 8; ++i) {
+        const int64_t sl = chunk * kSlotsPerWarp + i * 32 + lane;
+        x[c][i] = sl < total4 ? ldcs4(ob + ((int64_t)c * total4 + sl) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
-    store32(out + row * D + sub * 32, acc);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t sl = chunk * kSlotsPerWarp + i * 32 + lane;
+      if (sl >= total4) continue;
+      const int64_t row = sl / (D / 4);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        if (c >= nbr) break;
+        const float w = gate_weight(gates, row * 3 + c, mode);
+        acc[0] = fmaf(w, x[c][i].x, acc[0]);
+        acc[1] = fmaf(w, x[c][i].y, acc[1]);
+        acc[2] = fmaf(w, x[c][i].z, acc[2]);
+        acc[3] = fmaf(w, x[c][i].w, acc[3]);
+      }
+      store4(out + sl * 4, acc);
+    }
   }
 }
 
