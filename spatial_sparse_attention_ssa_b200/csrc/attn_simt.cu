@@ -455,28 +455,76 @@ __global__ void combine_kernel(const float* __restrict__ ob, const float* __rest
 // ---------------------------------------------------------------------------
 // Also writes the per-row constants of the tensor-core kernels (rc, [2][3][rows]):
 // for the compressed (c = 0) and window (c = 2) branches, -lse * log2(e), w and -D.
+// Access as in the combine, with 128 float4 slots per warp pass (4 per lane, to keep
+// the live registers low enough for 16+ warps per SM): a row's D / 4 slots sit in D / 4
+// consecutive lanes; their partial dot products are summed across those lanes, and
+// then lane L collects row L of the pass so that the per-row outputs are contiguous.
+constexpr int kPreSlots = 4;  // float4 slots per lane per pass
+
+__device__ __forceinline__ void load4s(const float* p, float* o) {
+  const float4 v = __ldcs(reinterpret_cast<const float4*>(p));
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+__device__ __forceinline__ void load4s(const __nv_bfloat16* p, float* o) {
+  const uint2 v = __ldcs(reinterpret_cast<const uint2*>(p));
+  o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xffff0000u);
+  o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xffff0000u);
+}
+
 template <typename T, int D>
 __global__ void bwd_pre_kernel(const float* __restrict__ ob, const T* __restrict__ dout, const float* __restrict__ gates,
                                const float* __restrict__ lse, int64_t rows, int mode, int nbr, float* __restrict__ Dc,
                                float* __restrict__ dgates, float* __restrict__ rc) {
-  constexpr int NT = D / 32;
-  const int64_t total = rows * NT;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t iters = (total + stride - 1) / stride;
-  for (int64_t it = 0; it < iters; ++it) {
-    const int64_t i = it * stride + blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    const bool valid = i < total;
-    const int64_t row = valid ? i / NT : 0;
-    const int sub = (int)(i % NT);
-    float dov[32], x[32];
-    load32(dout + row * D + sub * 32, dov);
+  constexpr int LPR = D / 4;      // lanes per row
+  constexpr int RPI = 32 / LPR;   // rows per slot index
+  constexpr int SPW = 32 * kPreSlots;  // slots per warp pass
+  const int64_t total4 = rows * LPR;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t chunk = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; chunk * SPW < total4; chunk += nwarps) {
+    float dov[kPreSlots][4];
+    float4 x[3][kPreSlots];
+#pragma unroll
+    for (int i = 0; i < kPreSlots; ++i) {
+      const int64_t sl = chunk * SPW + i * 32 + lane;
+      if (sl < total4) {
+        load4s(dout + sl * 4, dov[i]);
+      } else {
+        dov[i][0] = dov[i][1] = dov[i][2] = dov[i][3] = 0.f;
+      }
+    }
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
       if (c >= nbr) break;
-      load32(ob + ((int64_t)c * rows + row) * D + sub * 32, x);
-      const float dot = row_sum<NT>(dot32r(dov, x), 0xffffffffu);
-      if (valid && sub == 0) {
+#pragma unroll
+      for (int i = 0; i < kPreSlots; ++i) {
+        const int64_t sl = chunk * SPW + i * 32 + lane;
+        x[c][i] = sl < total4 ? __ldcs(reinterpret_cast<const float4*>(ob + ((int64_t)c * total4 + sl) * 4))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    const int my_i = lane / RPI, src = LPR * (lane % RPI);
+    float mine[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+#pragma unroll
+      for (int i = 0; i < kPreSlots; ++i) {
+        float dot = 0.f;
+        if (c < nbr)
+          dot = dov[i][0] * x[c][i].x + dov[i][1] * x[c][i].y + dov[i][2] * x[c][i].z + dov[i][3] * x[c][i].w;
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        const float t = __shfl_sync(0xffffffffu, dot, src);
+        if (i == my_i) mine[c] = t;
+      }
+    }
+    const int64_t row = chunk * (SPW / LPR) + lane;
+    if (lane < kPreSlots * RPI && row < rows) {
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        if (c >= nbr) break;
         const float w = gate_weight(gates, row * 3 + c, mode);
+        const float dot = mine[c];
         Dc[(int64_t)c * rows + row] = w * dot;
         dgates[row * nbr + c] = mode == SSA_GATE_LOGITS ? dot * w * (1.f - w) : dot;
         if (c != 1) {
