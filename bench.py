@@ -640,7 +640,7 @@ def run_reference(a):
     if rank != 0:
         return
     from spatial_sparse_attention_ssa_b200 import workloads as W
-    w = _workload(a.seed)
+    w = _workload(a.seed, a.tokens)
     t = W.make_tensors(w)
     budget = max(2.0, 150.0 / max(1, a.steps + a.warmup))  # whole run within a few minutes
     t0 = time.perf_counter()
