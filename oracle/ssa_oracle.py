@@ -369,7 +369,7 @@ def forward(coords, cu_seqlens, q, k, v, gates, *, hq, hkv, m_cmp, m_win, topk,
 
 
 def cross_forward(q_cu, kv_coords, kv_cu, q, k, v, gates, *, hq, hkv, m_cmp, topk, gate_mode, scale=None,
-                  pool_rounding="bf16", chunk=256, sel_given=None) -> State:
+                  pool_rounding="bf16", chunk=256, sel_given=None, tokens=None) -> State:
     """Cross-attention SSA (LSRM, shuwu5.cn/article/2502.html: the NSA attention is
     also used as cross attention between image tokens and voxel tokens).  The
     queries q [Nq, Hq, d] of sequence s are rows q_cu[s] .. q_cu[s+1]-1; the keys
@@ -378,7 +378,10 @@ def cross_forward(q_cu, kv_coords, kv_cu, q, k, v, gates, *, hq, hkv, m_cmp, top
     the self-attention path.  Two branches: compressed attention over all blocks
     of the sequence (with the group-summed top-k selection) and full attention
     over the tokens of the selected blocks.  The queries have no voxel, so there
-    is no window branch; gates [Nq, Hq, 2] weight (compressed, selected)."""
+    is no window branch; gates [Nq, Hq, 2] weight (compressed, selected).
+
+    `tokens` restricts the per-query outputs to a subset of query rows (the other
+    rows are left NaN / -1 / 0); compression is always complete."""
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     nq, _, d = q.shape
@@ -393,8 +396,9 @@ def cross_forward(q_cu, kv_coords, kv_cu, q, k, v, gates, *, hq, hkv, m_cmp, top
     lse = np.full((2, nq, hq), np.nan)
     o = np.zeros((2, nq, hq, d))
     sel = np.full((nq, hkv, topk), -1, dtype=np.int64)
+    rows = np.arange(nq) if tokens is None else np.asarray(tokens, np.int64)
     for s in range(len(q_cu) - 1):
-        toks = np.arange(q_cu[s], q_cu[s + 1])
+        toks = rows[(rows >= q_cu[s]) & (rows < q_cu[s + 1])]
         b0, b1 = int(blk["cu"][s]), int(blk["cu"][s + 1])
         if len(toks) == 0 or b1 == b0:
             continue
@@ -411,7 +415,7 @@ def cross_forward(q_cu, kv_coords, kv_cu, q, k, v, gates, *, hq, hkv, m_cmp, top
                     sel[tt, g, :] = np.where(loc >= 0, loc + b0, -1)
     if sel_given is not None:
         sel = np.asarray(sel_given, np.int64).copy()
-    for t in range(nq):
+    for t in rows:
         for g in range(hkv):
             hs = slice(g * G, (g + 1) * G)
             js = selected_tokens(sel[t, g], blk)
@@ -421,7 +425,8 @@ def cross_forward(q_cu, kv_coords, kv_cu, q, k, v, gates, *, hq, hkv, m_cmp, top
             lse[1, t, hs] = l_
             o[1, t, hs, :] = o_
     gw = gate_weights(gates, gate_mode)  # [Nq, Hq, 2]
-    out = np.einsum("nhc,cnhd->nhd", gw, o)
+    out = np.zeros((nq, hq, d))
+    out[rows] = np.einsum("nhc,cnhd->nhd", gw[rows], o[:, rows])
     return State(blk=blk, kc=kc, vc=vc, lse=lse, o=o, sel=sel, out=out, scale=scale, q=q, k=k, v=v,
                  gates=np.asarray(gates, np.float64), gate_mode=gate_mode, hq=hq, hkv=hkv, G=G, topk=topk,
                  q_cu=q_cu, kv_cu=kv_cu)

@@ -774,3 +774,14 @@ def test_learned_compression_in_the_full_backward_by_central_differences():
             vals.append(np.sum(do * s2["out"]))
         num = (vals[0] - vals[1]) / 2e-6
         assert abs(num - g["dk"][idx]) <= 1e-6 * max(1.0, abs(num)), (idx, num, g["dk"][idx])
+
+
+def test_cross_subset_of_query_rows_matches_full():
+    q_cu, coords, kv_cu, q, k, v, gates = _cross_case(35)
+    full = O.cross_forward(q_cu, coords, kv_cu, q, k, v, gates, hq=4, hkv=2, m_cmp=4, topk=3, gate_mode=1)
+    rows = np.array([0, 7, 39, 40, 62])
+    sub = O.cross_forward(q_cu, coords, kv_cu, q, k, v, gates, hq=4, hkv=2, m_cmp=4, topk=3, gate_mode=1,
+                          tokens=rows)
+    np.testing.assert_array_equal(sub["sel"][rows], full["sel"][rows])
+    np.testing.assert_array_equal(sub["o"][:, rows], full["o"][:, rows])
+    np.testing.assert_array_equal(sub["out"][rows], full["out"][rows])
