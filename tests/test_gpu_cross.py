@@ -127,3 +127,58 @@ def test_cross_rejects_a_sequence_with_queries_and_no_voxels():
     with pytest.raises(ssa.SSAError):
         _run(w2, t2, cq, backward=False)
     assert ssa.device_status() == 0
+
+
+def test_cross_at_benchmark_size_sampled_rows_and_sum_rules():
+    """131072 image-token queries against the 131072 voxel tokens of the benchmark
+    shell (the bench's cross-attention leg): sampled query rows element by element,
+    and over every row the sum rules of the key gradients (softmax rows sum to one in
+    both branches: sum_i dV_i = sum_rows (w_cmp + w_slc) dO, sum_i dK_i = 0 per KV
+    head; 4-sigma bound on independent bf16 rounding as in the self-attention test)."""
+    w = W.config(5)
+    assert w.s == 1
+    t = W.make_tensors(w)
+    cq = W.make_cross_queries(w, [w.n], seed=3)
+    out, saved, grads = _run(w, t, cq)
+    rng = np.random.default_rng(21)
+    toks = np.unique(np.concatenate([[0, w.n - 1], rng.choice(w.n, 62, replace=False)]))
+    st = O.cross_forward(cq.q_cu, w.coords, w.cu_seqlens, cq.as_f32("q"), t.as_f32("k"), t.as_f32("v"), cq.gates,
+                         hq=w.hq, hkv=w.hkv, m_cmp=w.m_cmp, topk=w.topk, gate_mode=w.gate_mode,
+                         pool_rounding=pool_rounding(w), tokens=toks)
+    atol = ATOL[w.dtype]
+    sel = saved.sel.cpu().numpy()
+    G = w.hq // w.hkv
+    b0, b1 = 0, int(st["blk"]["count"])
+    ob = f64(saved.o_branch)
+    lse = saved.lse.cpu().numpy().astype(np.float64)
+    o = f64(out)
+    flips = 0
+    for tt in toks:
+        np.testing.assert_allclose(ob[0, tt], st["o"][0, tt], rtol=0, atol=atol)
+        np.testing.assert_allclose(lse[0, tt], st["lse"][0, tt], rtol=0, atol=atol)
+        for g in range(w.hkv):
+            hs = slice(g * G, (g + 1) * G)
+            if not np.array_equal(sel[tt, g], st["sel"][tt, g]):  # must be a certified near-tie
+                _, _, p = O.cmp_attention(np.asarray(st["q"][tt:tt + 1, hs, :], np.float64), st["kc"][b0:b1, g, :],
+                                          st["vc"][b0:b1, g, :], st["scale"])
+                imp = p[0].sum(axis=0)
+                chosen = np.zeros(b1 - b0, bool)
+                chosen[sel[tt, g][sel[tt, g] >= 0]] = True
+                assert imp[chosen].min() >= imp[~chosen].max() - TAU_SEL, (tt, g)
+                flips += 1
+                continue
+            np.testing.assert_allclose(ob[1, tt, hs], st["o"][1, tt, hs], rtol=0, atol=atol)
+            np.testing.assert_allclose(lse[1, tt, hs], st["lse"][1, tt, hs], rtol=0, atol=atol)
+            np.testing.assert_allclose(o[tt, hs], st["out"][tt, hs], rtol=0, atol=atol)
+    dq, dk, dv, _ = (f64(x) for x in grads)
+    do = cq.as_f32("do").astype(np.float64)
+    gw = O.gate_weights(cq.gates, w.gate_mode)
+    for g in range(w.hkv):
+        hs = slice(g * G, (g + 1) * G)
+        wsum = gw[:, hs, :].sum(-1)
+        want = np.einsum("nh,nhd->d", wsum, do[:, hs, :])
+        noise = np.sqrt(np.einsum("nh,nhd->d", wsum ** 2, do[:, hs, :] ** 2))
+        assert (np.abs(dv[:, g, :].sum(0) - want) <= 2e-2 + 4 * 2.0 ** -9 / np.sqrt(3) * noise).all(), g
+        tol_k = 2e-2 + 4 * 2.0 ** -9 / np.sqrt(3) * np.sqrt((dk[:, g, :] ** 2).sum(0))
+        assert (np.abs(dk[:, g, :].sum(0)) <= tol_k).all(), g
+    print("flips", flips, "of", len(toks) * w.hkv)
