@@ -102,3 +102,78 @@ def gather_rows(local, plan: LocalPlan, n_total: int, group=None):
         ok = i >= 0
         out[i[ok]] = r[ok]
     return out
+
+
+# ---------------------------------------------------------------------------
+# One sequence across ranks (LSRM, "块感知序列并行与负载均衡"): whole blocks per rank
+# ---------------------------------------------------------------------------
+#
+# A rank owns a contiguous range of the sequence's blocks (blocks are numbered in
+# cell order, so a range is also spatially compact) and the tokens in them.  Its
+# queries attend (a) every compressed block and (b) the tokens of the selected
+# blocks, which needs the K / V of the whole sequence: the ranks all-gather K / V
+# (and could all-gather Kc / Vc instead of recomputing them); (c) the window
+# branch needs only the rank's own tokens when windows are whole blocks
+# (m_win = m_cmp).  In the backward, the key gradients of (a) and (b) are partial
+# sums over the rank's queries and go back to the owning ranks (a reduce-scatter).
+# Queries, outputs and gates never leave their rank.
+
+
+def block_ranges(counts, world: int) -> list[tuple[int, int]]:
+    """Split blocks 0 .. len(counts)-1, with counts[b] tokens each, into `world`
+    contiguous ranges [lo, hi) minimising the largest token count of a range (the
+    linear partition problem: the least feasible bound by binary search, each
+    range filled greedily).  Ranges may be empty when there are fewer blocks than
+    ranks; they cover the blocks in order."""
+    counts = np.asarray(counts, np.int64)
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    nb = len(counts)
+    if nb == 0:
+        return [(0, 0)] * world
+
+    def ranges_for(cap):
+        out, lo, acc = [], 0, 0
+        for b in range(nb):
+            if acc + counts[b] > cap and b > lo:
+                out.append((lo, b))
+                lo, acc = b, 0
+            acc += counts[b]
+        out.append((lo, nb))
+        return out
+
+    lo_c, hi_c = int(counts.max()), int(counts.sum())
+    while lo_c < hi_c:
+        mid = (lo_c + hi_c) // 2
+        if len(ranges_for(mid)) <= world:
+            hi_c = mid
+        else:
+            lo_c = mid + 1
+    r = ranges_for(lo_c)
+    return r + [(nb, nb)] * (world - len(r))
+
+
+def range_tokens(blk_perm, blk_ptr, lo: int, hi: int) -> np.ndarray:
+    """Tokens of blocks lo .. hi-1, in block order (global token indices)."""
+    blk_ptr = np.asarray(blk_ptr, np.int64)
+    return np.asarray(blk_perm, np.int64)[blk_ptr[lo]:blk_ptr[hi]]
+
+
+def all_gather_rows(local, tokens: np.ndarray, n_total: int, group=None):
+    """Every rank's rows (a torch tensor [len(tokens), ...] of the given global token
+    indices) placed at their token index in a [n_total, ...] tensor, on every rank:
+    the K / V exchange of the sequence-parallel forward."""
+    from types import SimpleNamespace
+    return gather_rows(local, SimpleNamespace(tokens=np.asarray(tokens, np.int64)), n_total, group)
+
+
+def reduce_to_owners(partial, tokens: np.ndarray, group=None):
+    """Sum the [n_total, ...] partial gradients of all ranks and keep this rank's
+    rows (`tokens`): the reduce-scatter of the key gradients.  Written as one
+    all-reduce for clarity; the rows are disjoint across ranks."""
+    import torch
+    import torch.distributed as dist
+
+    total = partial.clone()
+    dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
+    return total[torch.as_tensor(np.asarray(tokens, np.int64), device=total.device)]
