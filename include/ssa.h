@@ -14,13 +14,19 @@
  * GQA (several query heads per KV head) follows LSRM (shuwu5.cn/article/2502.html,
  * "阶段一": 32 query heads, 2 KV heads).
  *
+ * Entry points: ssa_bin (step 1), ssa_forward (steps 2-6), ssa_backward (step 7);
+ * ssa_geo_select (geometric block routing) and ssa_params.selection (a given
+ * selection); ssa_cross_forward / ssa_cross_backward (queries of another token
+ * set); ssa_params.conv (learned compression); ssa_bin_noalloc; workspace sizes,
+ * status, version and per-kernel timing.
+ *
  * Conventions for every entry point:
  *   - All array arguments are DEVICE pointers unless stated; the caller owns
  *     and allocates every buffer, including the workspace.  The library never
  *     allocates or frees device memory.
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
- *     legacy default stream).  Only ssa_bin and ssa_get_device_status
- *     synchronise that stream.
+ *     legacy default stream).  Only ssa_bin, ssa_bin_noalloc, ssa_cross_forward,
+ *     ssa_cross_backward and ssa_get_device_status synchronise that stream.
  *   - Errors are returned as ssa_status codes; nothing aborts or throws across
  *     the ABI.  Argument errors are detected on the host before any launch.
  *   - N = number of tokens (all sequences), S = number of sequences,
