@@ -115,3 +115,43 @@ def test_cross_attention_argument_errors_are_found_on_the_host():
                                  ctypes.byref(sv), 1, need_f, None) == 1
     assert lib.ssa_cross_backward(ctypes.byref(p), 1, 1, 1000, 500, ctypes.byref(part), 1, 1, 1, 1,
                                   ctypes.byref(sv), 1, 1, 1, 1, 1, 1, need_b - 1, None) == 3
+
+
+C_PROGRAM = r"""
+#include "ssa.h"
+#include <stdio.h>
+int main(void) {
+  ssa_params p = {0};
+  p.hq = 32; p.hkv = 2; p.d = 64; p.m_cmp = 8; p.m_win = 8; p.topk = 16;
+  p.dtype = SSA_DTYPE_BF16; p.gate_mode = SSA_GATE_LOGITS; p.selection = SSA_SEL_SCORES; p.conv = NULL;
+  size_t f = ssa_workspace_size(SSA_OP_FORWARD, &p, 1, 131072, 2322, 2322);
+  size_t c = ssa_workspace_size(SSA_OP_CROSS_FORWARD, &p, 1, 131072, 2322, 0);
+  ssa_status s = ssa_forward(&p, NULL, 1, 10, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL);
+  printf("%d %d %d %s\n", ssa_version(), f > 0 && c > f, (int)s, ssa_error_string(s));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as strict C99, a C program links
+    against libssa.so and makes host-side calls (no GPU needed)."""
+    import shutil
+    import subprocess
+
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.join(root, "spatial_sparse_attention_ssa_b200")
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(root, "include"),
+                        str(src), "-L", libdir, "-lssa", "-Wl,-rpath," + libdir, "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    version, sizes_ok, status, *msg = out.stdout.split()
+    assert int(version) == ssa.lib().ssa_version() and sizes_ok == "1"
+    assert int(status) == 1 and " ".join(msg) == "invalid argument"  # null cu_seqlens found on the host
