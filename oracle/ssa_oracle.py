@@ -23,9 +23,10 @@ Readings where the pages are silent (each is also listed in the design notes):
 * block / window ids: floor(coord / m), per sequence, numbered in
   lexicographic (x, y, z) order of the block coordinate, offset by the number
   of blocks of earlier sequences; members ordered by token index.
-* compression is the mean only (no learned convolution); the stored Kc/Vc is
-  computed as fp32(sum) / fp32(n), then rounded to the storage dtype (bf16
-  round-to-nearest-even) -- "pool_rounding".
+* compression is the mean by default; the stored Kc/Vc is computed as
+  fp32(sum) / fp32(n), then rounded to the storage dtype (bf16
+  round-to-nearest-even) -- "pool_rounding".  The learned form (a submanifold
+  sparse 3x3x3 convolution before the mean, weights as inputs) is `conv_pool`.
 * selection score: softmax probability over the sequence's compressed blocks,
   summed over the query heads of a GQA group; top-k with ties to the lower
   block id; k_eff = min(k, blocks in sequence); sel stored ascending, padded -1.
@@ -34,6 +35,12 @@ Readings where the pages are silent (each is also listed in the design notes):
   (mode 1).  softmax scale 1/sqrt(d) everywhere; no causal mask; a query's own
   token is in its window; selection is a constant for the backward; the
   rounding of Kc/Vc passes the gradient straight through (dKc/dK_i = 1/n_b).
+
+Beyond the self-attention path: `geo_topk` (selection by the shortest distance
+between voxel centres, LSRM "3D 感知空间块路由机制", voxel-only case), a given
+selection in `forward(sel_given=...)`, and `cross_forward` / `cross_backward`
+(queries of another token set, LSRM's cross attention between image and voxel
+tokens: compressed and selected branches, no window branch).
 
 Everything is computed in float64 from the exact input values.
 """
