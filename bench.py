@@ -17,7 +17,6 @@ the max over ranks.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import os
 import statistics
@@ -37,27 +36,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 SMS = 148
 FP32_LANES_PER_SM = 128
-
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch at the benchmark size
-# (131072 tokens, seed 0), from an ncu capture summarised under profiles/; reported only
-# while the kernel's source file is byte-identical to the one profiled.
-NCU_TRAFFIC = {
-    "cmp_bwd_dkv_tc_kernel": ("spatial_sparse_attention_ssa_b200/csrc/cmp_tc.cu",
-                              "7d0b4da601ee818c8ec43545aff7c214235d058e", 1.1887e9,
-                              "profiles/cmp_bwd_dkv_dram_gigascale1024_131072.md"),
-}
-
-
-def _traffic(kernel: str, tokens: int, seed: int):
-    entry = NCU_TRAFFIC.get(kernel)
-    if entry is None or tokens != 131072 or seed != 0:
-        return None, None
-    path, sha, nbytes, src = entry
-    with open(os.path.join(ROOT, path), "rb") as f:
-        if hashlib.sha1(f.read()).hexdigest() != sha:
-            return None, "kernel changed since " + src
-    return nbytes, src
-
 
 def _args():
     ap = argparse.ArgumentParser()
@@ -162,12 +140,20 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
-    """Per kernel name: (bound, algorithmic units per launch, unit).
+    """Algorithmic work per kernel and per stage (a stage is the kernels of one
+    branch and direction, e.g. the compressed backward = its dQ and dK/dV kernels;
+    a stage lists every kernel that may implement it, and the ones that ran count).
 
-    Scores: compressed = sum over sequences of n_s * Hq * B_s; selected = sum
-    over (token, group) of G * (tokens in the selected blocks); window = Hq *
-    sum over windows of n_w^2.  Contraction flops per score: 2d for each
-    q.k / p.v / dO.v / ds.k / ds^T.q / p^T.dO the kernel performs.
+    Scores: compressed = sum over sequences of n_s * Hq * B_s; selected = sum over
+    (token, group) of G * (tokens in the selected blocks); window = Hq * sum over
+    windows of n_w^2.  Flops per score are 2d for every contraction the method
+    needs, counted once per stage: forward 6d for the compressed branch (S for the
+    normaliser, S again for the selection's final probabilities, P.V) and 4d for
+    the others; backward 10d (S, dP, dQ, dK, dV).  Exponentials per score: 2 in the
+    compressed forward (lse pass, output pass), 1 elsewhere.  Per kernel the same
+    count covers the contractions that kernel performs; the bf16 low-part products,
+    masked tile padding and the backward's second S / dP are overhead, not work.
+    Memory kernels count the bytes they must move.
     """
     d, hq, hkv = w.d, w.hq, w.hkv
     G = hq // hkv
@@ -181,32 +167,34 @@ def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
     sc_win = float(hq * np.sum(wsize ** 2))
     e = 2  # bf16 bytes
     N, B = w.n, len(bsize)
+    # per kernel: (kind, contraction flops, exps) for attention, ("bytes", bytes) for memory kernels
     work = {
-        # tensor-core kernels: (kind, contraction flops, exps) -- the exps bound them at d = 64
         "cmp_lse_tc_kernel": ("tc", 2 * d * sc_cmp, sc_cmp),
         "cmp_out_tc_kernel": ("tc", 4 * d * sc_cmp, sc_cmp),
+        "cmp_fa_tc_kernel": ("tc", 4 * d * sc_cmp, sc_cmp),
+        "cmp_sel_tc_kernel": ("tc", 2 * d * sc_cmp, sc_cmp),
         "cmp_bwd_dq_tc_kernel": ("tc", 6 * d * sc_cmp, sc_cmp),
         "cmp_bwd_dkv_tc_kernel": ("tc", 8 * d * sc_cmp, sc_cmp),
-        "win_fwd_tc_kernel": ("tc", 4 * d * sc_win, 2 * sc_win),
+        "win_fwd_tc_kernel": ("tc", 4 * d * sc_win, sc_win),
         "win_bwd_dq_tc_kernel": ("tc", 6 * d * sc_win, sc_win),
         "win_bwd_dkv_tc_kernel": ("tc", 8 * d * sc_win, sc_win),
-        "slc_bwd_fused_kernel": ("flops", 10 * d * sc_slc),
-        "cmp_lse_kernel": ("flops", 2 * d * sc_cmp),
-        "cmp_out_topk_kernel": ("flops", 4 * d * sc_cmp),
-        "slc_fwd_kernel": ("flops", 4 * d * sc_slc),
-        "win_fwd_kernel": ("flops", 4 * d * sc_win),
-        "cmp_bwd_dq_kernel": ("flops", 6 * d * sc_cmp),
-        "cmp_bwd_dkv_kernel": ("flops", 8 * d * sc_cmp),
-        "slc_bwd_dq_kernel": ("flops", 6 * d * sc_slc),
-        "slc_bwd_dkv_kernel": ("flops", 8 * d * sc_slc),
-        "win_bwd_dq_kernel": ("flops", 6 * d * sc_win),
-        "win_bwd_dkv_kernel": ("flops", 8 * d * sc_win),
+        "slc_fwd_mma_kernel": ("tc", 4 * d * sc_slc, sc_slc),
+        "slc_bwd_mma_kernel": ("tc", 10 * d * sc_slc, sc_slc),
         "pool_kernel": ("bytes", 4.0 * N * hkv * d * e + 2.0 * B * hkv * d * e),
         "combine_kernel": ("bytes", 3.0 * N * hq * d * 4 + N * hq * 3 * 4 + N * hq * d * e),
         "bwd_pre_kernel": ("bytes", 3.0 * N * hq * d * 4 + N * hq * d * e + N * hq * 3 * 4 * 3),
     }
+    stages = {
+        "compressed forward": (("cmp_lse_tc_kernel", "cmp_out_tc_kernel", "cmp_fa_tc_kernel", "cmp_sel_tc_kernel"),
+                               6 * d * sc_cmp, 2 * sc_cmp),
+        "compressed backward": (("cmp_bwd_dq_tc_kernel", "cmp_bwd_dkv_tc_kernel"), 10 * d * sc_cmp, sc_cmp),
+        "window forward": (("win_fwd_tc_kernel",), 4 * d * sc_win, sc_win),
+        "window backward": (("win_bwd_dq_tc_kernel", "win_bwd_dkv_tc_kernel"), 10 * d * sc_win, sc_win),
+        "selected forward": (("slc_fwd_mma_kernel",), 4 * d * sc_slc, sc_slc),
+        "selected backward": (("slc_bwd_mma_kernel",), 10 * d * sc_slc, sc_slc),
+    }
     scores = {"cmp": sc_cmp, "slc": sc_slc, "win": sc_win}
-    return work, scores
+    return work, stages, scores
 
 
 # ---------------------------------------------------------------------------
@@ -411,48 +399,48 @@ def run_ours(a):
     blk_cu = blk.cu.cpu().numpy()
     win_ptr = win.ptr[:win.count + 1].cpu().numpy()
     sel = saved.sel.cpu().numpy()
-    work, scores = kernel_work(w, blk_ptr, blk_cu, win_ptr, sel)
+    work, stages, scores = kernel_work(w, blk_ptr, blk_cu, win_ptr, sel)
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    tc_peak = peaks.get("bf16_tflops")  # burst: the step is tens of ms, not a seconds-long loop
+    mufu_peak = SMS * 16 * mhz * 1e6 / 1e12  # Texp/s: 16 ex2 per clock per SM
     per_kernel = {}
-    step_ms_kernels = 0.0
     for name, (tot, cnt) in prof.items():
-        per_kernel[name] = {"ms_per_step": tot / a.steps, "launches": cnt, "ms_per_launch": tot / max(cnt, 1)}
-        step_ms_kernels += tot / a.steps
-    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
+        ms_l = tot / max(cnt, 1)
+        ent = {"ms_per_step": tot / a.steps, "launches": cnt, "ms_per_launch": ms_l}
+        wk = work.get(name)
+        if wk is not None and wk[0] == "tc":
+            ent["tflops"] = wk[1] / (ms_l / 1e3) / 1e12
+            ent["tensor_frac"] = ent["tflops"] / tc_peak
+            ent["mufu_frac"] = wk[2] / (ms_l / 1e3) / 1e12 / mufu_peak
+        elif wk is not None:
+            ent["gbs"] = wk[1] / (ms_l / 1e3) / 1e9
+            ent["hbm_frac"] = ent["gbs"] / peaks["hbm_gbs"]
+        per_kernel[name] = ent
+    stage_rows = {}
+    for sname, (cands, flops, exps) in stages.items():
+        kernels = [k_ for k_ in cands if k_ in prof]  # the stage's kernels that ran (one launch each per step)
+        if not kernels:
+            continue
+        ms_s = sum(prof[k_][0] / max(prof[k_][1], 1) for k_ in kernels)  # one launch of each per step
+        stage_rows[sname] = {"kernels": list(kernels), "ms": ms_s, "tflops": flops / (ms_s / 1e3) / 1e12,
+                             "tensor_frac": flops / (ms_s / 1e3) / 1e12 / tc_peak,
+                             "mufu_frac": exps / (ms_s / 1e3) / 1e12 / mufu_peak,
+                             "flops": flops, "exps": exps}
     roof = None
     exp_roof = None
-    if dom is not None:
-        avg_ms = prof[dom][0] / max(prof[dom][1], 1)
-        entry = work.get(dom, ("bytes", None))
-        kind, units = entry[0], entry[1]
-        mhz = peaks.get("sm_max_mhz", 1965.0)
-        if kind == "tc":
-            achieved = units / (avg_ms / 1e3) / 1e12
-            peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-            traffic, tsrc = _traffic(dom, a.tokens, a.seed)
-            roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": traffic, "traffic_source": tsrc,
-                    "peak_source": "%s bf16 dense, sustained (kernel timed inside the step)" % peaks["_source"],
-                    "algorithmic_per_launch": units, "ms_per_launch": avg_ms}
-            exps = entry[2]
-            mufu_peak = SMS * 16 * mhz * 1e6 / 1e12  # 16 ex2 per clock per SM
-            exp_roof = {"kernel": dom, "bound": "mufu", "achieved": exps / (avg_ms / 1e3) / 1e12,
-                        "peak": mufu_peak, "unit": "Texp/s", "frac": exps / (avg_ms / 1e3) / 1e12 / mufu_peak,
-                        "peak_source": "derived: %d SMs x 16 ex2/clock x %.0f MHz" % (SMS, mhz),
-                        "exps_per_launch": exps}
-        elif kind == "flops" and units is not None:
-            achieved = units / (avg_ms / 1e3) / 1e12
-            # the attention kernels in this build are fp32 SIMT (FFMA): ALU-bound
-            peak = SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
-            roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
-                    "peak_source": "derived: %d SMs x %d FP32 lanes x 2 flop x %.0f MHz" % (SMS, FP32_LANES_PER_SM, mhz),
-                    "algorithmic_per_launch": units, "ms_per_launch": avg_ms}
-        elif units is not None:
-            achieved = units / (avg_ms / 1e3) / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "traffic": None, "peak_source": peaks["_source"],
-                    "algorithmic_per_launch": units, "ms_per_launch": avg_ms}
+    if stage_rows:
+        dom = max(stage_rows, key=lambda k_: stage_rows[k_]["ms"])
+        r_ = stage_rows[dom]
+        roof = {"kernel": " + ".join(r_["kernels"]), "stage": dom, "bound": "tensor", "achieved": r_["tflops"],
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": r_["tensor_frac"], "traffic": None,
+                "peak_source": "%s bf16 dense, burst" % peaks["_source"],
+                "algorithmic_per_launch": r_["flops"], "ms_per_launch": r_["ms"],
+                "note": "the stage's kernels, one launch each, at its algorithmic flops (each contraction of "
+                        "the method once); DRAM traffic of these kernels is from ncu, not measured here"}
+        exp_roof = {"kernel": roof["kernel"], "bound": "mufu", "achieved": r_["exps"] / (r_["ms"] / 1e3) / 1e12,
+                    "peak": mufu_peak, "unit": "Texp/s", "frac": r_["mufu_frac"],
+                    "peak_source": "derived: %d SMs x 16 ex2/clock x %.0f MHz" % (SMS, mhz),
+                    "exps_per_launch": r_["exps"]}
 
     # ---- geometric block routing (selection by voxel distance), timed on its own
     geo = None
@@ -573,7 +561,8 @@ def run_ours(a):
                 "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded surface-shell voxels, N(0,1) bf16 Q/K/V/dO, N(0,1) gate logits)",
-                "config": cfg, "roofline": roof, "roofline_exp": exp_roof, "cpu_baseline": cpu, "e2e": e2e,
+                "config": cfg, "roofline": roof, "roofline_exp": exp_roof, "stages": stage_rows,
+                "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(launches),
                 "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel, "geo_routing": geo,
                 "cross_attention": cross, "learned_compression": learned,
@@ -600,11 +589,17 @@ def _blas_threads() -> int:
 
 
 def _oracle_sample(w, t, tokens):
+    """The oracle's forward of the sampled query tokens (binning and pooling of all
+    tokens, then the three branches of the sample), and the compressed branch's
+    backward of the sampled rows: their dQ and their contributions to dKc / dVc."""
     from oracle import ssa_oracle as O
-    st = O.forward(w.coords, w.cu_seqlens, t.as_f32("q"), t.as_f32("k"), t.as_f32("v"), t.gates, hq=w.hq,
+    q, do = t.as_f32("q"), t.as_f32("do")
+    st = O.forward(w.coords, w.cu_seqlens, q, t.as_f32("k"), t.as_f32("v"), t.gates, hq=w.hq,
                    hkv=w.hkv, m_cmp=w.m_cmp, m_win=w.m_win, topk=w.topk, gate_mode=w.gate_mode,
                    pool_rounding="bf16", tokens=tokens)
-    O.dq_rows(st, t.as_f32("do"), tokens)
+    for tok in tokens:
+        O.cmp_branch_range(q, st["kc"], st["vc"], st["blk"]["cu"], w.cu_seqlens, t.gates, hq=w.hq, hkv=w.hkv,
+                           topk=w.topk, gate_mode=w.gate_mode, t0=int(tok), t1=int(tok) + 1, dout=do)
 
 
 def _sample_tokens(w, n):
@@ -628,9 +623,10 @@ def cpu_baseline(w, t, seconds: float) -> dict:
     _oracle_sample(w, t, _sample_tokens(w, T))
     el = time.perf_counter() - t0
     return {"value": T / el, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": "numpy fp64 oracle: binning + mean pooling of all %d tokens, then compressed attention + "
-                      "top-k, selected and window attention and the dQ rows of %d evenly spaced query tokens "
-                      "(dK/dV, which need every query, not included); %.1f s" % (w.n, T, el),
+            "sample": "numpy fp64 oracle: binning + mean pooling of all %d tokens, then for %d evenly spaced "
+                      "query tokens the forward of all three branches and the compressed branch's backward (dQ "
+                      "and the rows' dKc / dVc sums; the selected and window backward, ~3%% of the flops, left "
+                      "out); %.1f s" % (w.n, T, el),
             "seconds": el}
 
 
@@ -639,9 +635,12 @@ def run_reference(a):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
+    from oracle import ssa_oracle as O
     from spatial_sparse_attention_ssa_b200 import workloads as W
     w = _workload(a.seed, a.tokens)
     t = W.make_tensors(w)
+    nb = int(O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)["count"])
+    nw = int(O.bin_tokens(w.coords, w.cu_seqlens, w.m_win)["count"])
     budget = max(2.0, 150.0 / max(1, a.steps + a.warmup))  # whole run within a few minutes
     t0 = time.perf_counter()
     _oracle_sample(w, t, _sample_tokens(w, 8))
@@ -660,10 +659,12 @@ def run_reference(a):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded workload as the GPU arm)",
-            "config": _workload_desc(w, None, None), "impl": "reference",
+            "config": dict(_workload_desc(w, nb, nw), global_batch=world, parallelism="dp%d" % world),
+            "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": "per step: binning + pooling of all tokens, then forward branches and dQ "
-                                       "rows of %d evenly spaced query tokens" % T},
+                             "sample": "per step: binning + pooling of all tokens, then the forward of all "
+                                       "branches and the compressed backward rows of %d evenly spaced query "
+                                       "tokens" % T},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

@@ -14,7 +14,8 @@
  * GQA (several query heads per KV head) follows LSRM (shuwu5.cn/article/2502.html,
  * "阶段一": 32 query heads, 2 KV heads).
  *
- * Entry points: ssa_bin (step 1), ssa_forward (steps 2-6), ssa_backward (step 7);
+ * Entry points: ssa_bin (step 1), ssa_pool (step 2 alone), ssa_forward (steps 2-6),
+ * ssa_backward (step 7);
  * ssa_geo_select (geometric block routing) and ssa_params.selection (a given
  * selection); ssa_cross_forward / ssa_cross_backward (queries of another token
  * set); ssa_params.conv (learned compression); ssa_bin_noalloc; workspace sizes,
@@ -169,9 +170,9 @@ SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int
  * every GPU that loads the library, held until the process exits), so:
  *   - N must be <= SSA_BIN_NOALLOC_MAX_TOKENS, else SSA_ERR_WORKSPACE and
  *     nothing is enqueued;
- *   - the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before capturing any stream into a CUDA graph;
+ *   - every call looks up the array's address on the current device
+ *     (cudaGetSymbolAddress), so call it with the device of the buffers current;
+ *   - like ssa_bin, it synchronises `stream` to return the counts;
  *   - all calls on a device share the array: calls whose GPU work overlaps
  *     (other streams, other host threads) race and corrupt each other; the
  *     array keeps the last call's contents, and each call clears the parts
@@ -183,6 +184,26 @@ SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int
 SSA_API ssa_status ssa_bin_noalloc(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N,
                                    int32_t R, int32_t m_cmp, int32_t m_win, ssa_partition* blk,
                                    ssa_partition* win, void* stream);
+
+/*
+ * ssa_pool -- step 2 alone, the sparse 3D compression (Direct3D-S2 "方法": each
+ * block's keys and values are mean-pooled; LSRM "空间块划分与键值压缩": in-block
+ * average pooling).  ssa_forward runs the same kernel first; this entry point is
+ * for callers that want only the compressed keys/values or time the step by itself.
+ *   dtype    SSA_DTYPE_BF16 or SSA_DTYPE_F32; hkv >= 1; d a multiple of 8 with
+ *            2 * hkv * d * sizeof(dtype) <= 16384 (SSA_ERR_UNSUPPORTED otherwise)
+ *   blk      the block partition from ssa_bin over the same N tokens (device arrays)
+ *   k, v     [N, Hkv, d] dtype, token-major
+ *   ks, vs   out [Hkv, N, d] dtype: rows gathered in blk.perm order (a block's tokens
+ *            are one contiguous range per head)
+ *   kc, vc   out [Hkv, blk.count, d] dtype: fp32(exact sum) / fp32(n), rounded to dtype
+ *            (bf16: round to nearest even)
+ * Every pointer must be 16-byte aligned.  Asynchronous; argument errors are found on
+ * the host before anything is enqueued.  Bit-exact for bf16 (fp64 sums of bf16
+ * values are exact).
+ */
+SSA_API ssa_status ssa_pool(int32_t dtype, int32_t hkv, int32_t d, int64_t N, const ssa_partition* blk,
+                            const void* k, const void* v, void* ks, void* vs, void* kc, void* vc, void* stream);
 
 /*
  * ssa_geo_select -- 3D-aware block routing (LSRM "3D 感知空间块路由机制", voxel-only

@@ -699,6 +699,98 @@ def window_kv_grads(st: State, dout: np.ndarray, windows) -> tuple:
 
 
 # ----------------------------------------------------------------------------
+# the compressed branch alone over a range of query tokens (full-size checks)
+# ----------------------------------------------------------------------------
+
+
+def cmp_branch_range(q, kc, vc, blk_cu, cu_seqlens, gates, *, hq, hkv, topk, gate_mode, t0, t1,
+                     dout=None, scale=None, chunk=256, sel_other=None) -> dict:
+    """Forward and backward of the compressed branch (Direct3D-S2 "方法": every
+    query attends to all compressed blocks of its sequence; the top-k blocks by
+    that score are selected) for the query tokens t0 .. t1-1 only.
+
+    The same definition as the compressed parts of `forward` and `backward`,
+    restricted to a token range so that a long sequence can be split over
+    processes: a query's lse, output, selection and dQ need only its own row, and
+    dKc / dVc are sums over query rows, so the per-range dkc / dvc returned here
+    add up to the full ones.  q, dout [N, Hq, d] (any float type, exact values);
+    kc, vc [B, Hkv, d] float64 (the stored, rounded block means); blk_cu [S+1]
+    block offsets per sequence; gates [N, Hq, 3] (only column 0 is used).
+
+    Returns lse [T, Hq], o [T, Hq, d], sel [T, Hkv, topk] (global ids ascending,
+    -1 padded), and with dout: dq [T, Hq, d] (this branch's part), dkc / dvc
+    [B, Hkv, d] (these rows' sums).  With `sel_other` (another selection of the
+    same rows, [T, Hkv, topk] global ids, -1 padded) also other_gap [T, Hkv]: the
+    lowest selection score among the blocks it chose minus the highest among the
+    blocks of the sequence it left out (+inf when it chose every block); a valid
+    top-k of these scores has other_gap >= 0, a near-tie choice >= -tau.
+    """
+    n, _, d = q.shape
+    G = hq // hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    cu_seqlens = np.asarray(cu_seqlens, np.int64)
+    blk_cu = np.asarray(blk_cu, np.int64)
+    T = t1 - t0
+    lse = np.full((T, hq), np.nan)
+    o = np.zeros((T, hq, d))
+    sel = np.full((T, hkv, topk), -1, dtype=np.int64)
+    res = {"lse": lse, "o": o, "sel": sel}
+    if sel_other is not None:
+        gap = np.full((T, hkv), np.inf)
+        res["other_gap"] = gap
+    if dout is not None:
+        dq = np.zeros((T, hq, d))
+        dkc = np.zeros(kc.shape)
+        dvc = np.zeros(vc.shape)
+        res.update(dq=dq, dkc=dkc, dvc=dvc)
+    for s in range(len(cu_seqlens) - 1):
+        a, b = max(t0, int(cu_seqlens[s])), min(t1, int(cu_seqlens[s + 1]))
+        if a >= b:
+            continue
+        b0, b1 = int(blk_cu[s]), int(blk_cu[s + 1])
+        for g in range(hkv):
+            hs = slice(g * G, (g + 1) * G)
+            kcg, vcg = kc[b0:b1, g, :], vc[b0:b1, g, :]
+            for c0 in range(a, b, chunk):
+                tt = np.arange(c0, min(b, c0 + chunk))
+                r = tt - t0
+                qr = np.asarray(q[tt, hs, :], np.float64)
+                l_, o_, p = cmp_attention(qr, kcg, vcg, scale)
+                lse[r, hs] = l_
+                o[r, hs, :] = o_
+                imp = p.sum(axis=1)  # [n, B_s]: probabilities summed over the group's heads
+                loc = topk_blocks(imp, topk)
+                sel[r, g, :] = np.where(loc >= 0, loc + b0, -1)
+                if sel_other is not None:
+                    chosen = np.zeros(imp.shape, bool)
+                    for i, row in enumerate(np.asarray(sel_other)[r, g]):
+                        ids = row[(row >= b0) & (row < b1)] - b0
+                        chosen[i, ids] = True
+                    lo = np.where(chosen, imp, np.inf).min(axis=1)
+                    hi = np.where(chosen, -np.inf, imp).max(axis=1)
+                    gap[r, g] = np.where(chosen.all(axis=1), np.inf, lo - hi)
+                if dout is None:
+                    continue
+                w = gate_weights(gates[tt, hs, 0], gate_mode)
+                dor = np.asarray(dout[tt, hs, :], np.float64) * w[..., None]
+                dp = dor @ vcg.T
+                ds = p * (dp - np.sum(p * dp, axis=-1, keepdims=True))
+                dq[r, hs, :] = scale * (ds @ kcg)
+                # sums over the chunk's (token, head) rows: [B_s, rows] x [rows, d]
+                dkc[b0:b1, g, :] += scale * (ds.reshape(-1, b1 - b0).T @ qr.reshape(-1, d))
+                dvc[b0:b1, g, :] += p.reshape(-1, b1 - b0).T @ dor.reshape(-1, d)
+    return res
+
+
+def cmp_token_grads(dkc: np.ndarray, dvc: np.ndarray, blk: dict):
+    """dK, dV [N, Hkv, d] of the compressed branch from dKc, dVc: each token gets
+    its block's gradient divided by the block size (the mean's derivative)."""
+    cnt = np.diff(blk["ptr"]).astype(np.float64)
+    return dkc[blk["id"]] / cnt[blk["id"]][:, None, None], dvc[blk["id"]] / cnt[blk["id"]][:, None, None]
+
+
+# ----------------------------------------------------------------------------
 # 3D-aware block routing (selection by geometric distance instead of scores)
 # ----------------------------------------------------------------------------
 

@@ -50,11 +50,14 @@ ssa_status check_params(const ssa_params* p) {
   if (G & (G - 1)) return SSA_ERR_UNSUPPORTED;  // power of two
   if (G * (p->d / 32) > 32) return SSA_ERR_UNSUPPORTED;
   if (p->conv && p->hkv * p->d > 256) return SSA_ERR_UNSUPPORTED;
+  if (!ssa::pool_supported(p->dtype, p->hkv, p->d)) return SSA_ERR_UNSUPPORTED;
   return SSA_OK;
 }
 
-bool partition_ok(const ssa_partition* x) {
-  return x && x->id && x->perm && x->ptr && x->cu && x->key && x->count >= 0;
+// The per-token arrays (id, perm) and the cell keys may be null when there are no
+// tokens: nothing is written to them then.  ptr and cu are always written.
+bool partition_ok(const ssa_partition* x, int64_t n) {
+  return x && x->ptr && x->cu && x->count >= 0 && (n == 0 || (x->id && x->perm && x->key));
 }
 
 float eff_scale(const ssa_params* p) { return p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->d); }
@@ -213,7 +216,7 @@ SSA_API ssa_status ssa_geo_select(const int32_t* coords, const int32_t* cu_seqle
     return SSA_ERR_INVALID_ARG;
   if (R > 32768) return SSA_ERR_UNSUPPORTED;  // squared distances must fit 32 bits
   if (N == 0) return SSA_OK;
-  if (!coords || !cu_seqlens || !partition_ok(blk) || !sel || !ws) return SSA_ERR_INVALID_ARG;
+  if (!coords || !cu_seqlens || !partition_ok(blk, N) || !sel || !ws) return SSA_ERR_INVALID_ARG;
   if (blk->count < 1 || blk->count > N) return SSA_ERR_INVALID_ARG;
   if (ws_bytes < ssa::geo_ws_bytes(N)) return SSA_ERR_WORKSPACE;
   return cuda_status(ssa::geo_select(coords, cu_seqlens, S, N, blk, m_cmp, topk, hkv, sel, ws,
@@ -237,12 +240,25 @@ SSA_API ssa_status ssa_get_device_status(void* stream) {
   return SSA_OK;
 }
 
+SSA_API ssa_status ssa_pool(int32_t dtype, int32_t hkv, int32_t d, int64_t N, const ssa_partition* blk,
+                            const void* k, const void* v, void* ks, void* vs, void* kc, void* vc, void* stream) {
+  if ((dtype != SSA_DTYPE_BF16 && dtype != SSA_DTYPE_F32) || hkv < 1 || d < 1 || N < 0 || N > INT32_MAX - 1)
+    return SSA_ERR_INVALID_ARG;
+  if (!ssa::pool_supported(dtype, hkv, d)) return SSA_ERR_UNSUPPORTED;
+  if (N == 0) return SSA_OK;
+  if (!partition_ok(blk, N) || blk->count < 1 || blk->count > N || !k || !v || !ks || !vs || !kc || !vc)
+    return SSA_ERR_INVALID_ARG;
+  for (const void* x : {k, v, (const void*)ks, (const void*)vs, (const void*)kc, (const void*)vc})
+    if (reinterpret_cast<uintptr_t>(x) % 16 != 0) return SSA_ERR_INVALID_ARG;
+  return cuda_status(ssa::launch_pool(dtype, k, v, blk, N, hkv, d, ks, vs, kc, vc, static_cast<cudaStream_t>(stream)));
+}
+
 SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N, int32_t R,
                            int32_t m_cmp, int32_t m_win, ssa_partition* blk, ssa_partition* win, void* ws,
                            size_t ws_bytes, void* stream) {
   if (S < 1 || N < 0 || N > INT32_MAX - 1 || R < 1 || R > (1 << 20) || m_cmp < 1 || m_win < 1)
     return SSA_ERR_INVALID_ARG;
-  if (!cu_seqlens || (N > 0 && !coords) || !partition_ok(blk) || !partition_ok(win) || !ws)
+  if (!cu_seqlens || (N > 0 && !coords) || !partition_ok(blk, N) || !partition_ok(win, N) || !ws)
     return SSA_ERR_INVALID_ARG;
   if (ws_bytes < bin_bytes(S, N)) return SSA_ERR_WORKSPACE;
   int sbits = 0;
@@ -444,7 +460,7 @@ SSA_API ssa_status ssa_forward(const ssa_params* p, const int32_t* cu_seqlens, i
                                size_t ws_bytes, void* stream) {
   ssa_status ps = check_params(p);
   if (ps != SSA_OK) return ps;
-  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk, N) || !partition_ok(win, N) || !saved)
     return SSA_ERR_INVALID_ARG;
   if (N == 0) return SSA_OK;
   if (!q || !k || !v || !gates || !out || !saved_ok(saved) || !ws) return SSA_ERR_INVALID_ARG;
@@ -461,7 +477,7 @@ SSA_API ssa_status ssa_backward(const ssa_params* p, const int32_t* cu_seqlens, 
                                 void* stream) {
   ssa_status ps = check_params(p);
   if (ps != SSA_OK) return ps;
-  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk) || !partition_ok(win) || !saved)
+  if (S < 1 || N < 0 || N > INT32_MAX - 1 || !cu_seqlens || !partition_ok(blk, N) || !partition_ok(win, N) || !saved)
     return SSA_ERR_INVALID_ARG;
   if (N == 0) return SSA_OK;
   if (!q || !k || !v || !gates || !dout || !dq || !dk || !dv || !dgates || !saved_ok(saved) || !ws)
@@ -482,7 +498,7 @@ SSA_API ssa_status ssa_cross_forward(const ssa_params* p, const int32_t* q_cu, i
                                      size_t ws_bytes, void* stream) {
   ssa_status ps = check_params(p);
   if (ps != SSA_OK) return ps;
-  if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk) ||
+  if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk, Nkv) ||
       !saved)
     return SSA_ERR_INVALID_ARG;
   if (p->conv) return SSA_ERR_UNSUPPORTED;  // the learned compression is built for self attention
@@ -505,7 +521,7 @@ SSA_API ssa_status ssa_cross_backward(const ssa_params* p, const int32_t* q_cu, 
                                       void* stream) {
   ssa_status ps = check_params(p);
   if (ps != SSA_OK) return ps;
-  if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk) ||
+  if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk, Nkv) ||
       !saved)
     return SSA_ERR_INVALID_ARG;
   if (p->conv) return SSA_ERR_UNSUPPORTED;

@@ -951,9 +951,249 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_out_tc_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// selection pass (transposed: thread = block): S^T = Kc Q^T in TMEM, double-
+// buffered; p = 2^(s qs2 - lse log2 e) with the final lse of the output pass; the
+// block's score for a token is the sum of its G heads' p, written to a per-CTA
+// scratch; a warpgroup picks each token's top-k of the previous row tile while the
+// compute warps work on the next one.  A quarter of each thread's exponentials are
+// evaluated on the FMA pipe (ex2_poly2) so that the MUFU and FMA pipes share them.
+// ---------------------------------------------------------------------------
+constexpr int kSelStages = 4;           // Kc ring depth
+constexpr int kSelPolyRows = 16;        // of the 64 rows a thread handles per key tile, rows on the FMA pipe
+
+struct SelSmem {
+  uint8_t q[2][kTile];
+  uint8_t kc[kSelStages][kTile];
+  __align__(16) float lse2[2][kRows];  // -lse log2(e) of the tile's rows, double-buffered by tile
+  float candv[kOutTopkWarps][kCandMax];
+  int candi[kOutTopkWarps][kCandMax];
+  uint64_t q_full[2], q_empty[2], mma_done, cw, imp_full[2], imp_empty[2];
+  uint64_t kc_full[kSelStages], kc_empty[kSelStages];
+  uint64_t s_full[2], s_empty[2];
+  uint32_t tmem;
+  int abort_flag;
+};
+
+template <int G>
+__global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap,
+    const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S,
+    int hq, int hkv, int btot, float qs2, const float* __restrict__ lse_in, int topk, int32_t* __restrict__ sel,
+    float* __restrict__ imp_scratch, int64_t imp_stride, int* status) {
+  constexpr int TPT = kRows / G;  // tokens per tile
+  extern __shared__ uint8_t smem_raw[];
+  SelSmem& sm = *reinterpret_cast<SelSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int ntiles = tpre[S];
+  const int total = ntiles * hkv;
+  float* imp_cta = imp_scratch + (int64_t)blockIdx.x * 2 * TPT * imp_stride;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+      mbar_init(&sm.imp_full[i], kComputeWarps);
+      mbar_init(&sm.imp_empty[i], kOutTopkWarps);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_empty[i], kComputeWarps);
+    }
+    mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.cw, kComputeWarps);
+    for (int i = 0; i < kSelStages; ++i) {
+      mbar_init(&sm.kc_full[i], 1);
+      mbar_init(&sm.kc_empty[i], 1);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;  // S^T buffers at columns [0,128) and [128,256)
+
+  if (warp == kOutTmaWarp) {
+    // ---------------- TMA producer: Q per tile; Kc per key tile
+    if (lane == 0) {
+      prefetch_tmap(&qmap);
+      prefetch_tmap(&kcmap);
+      uint32_t kc_count = 0, q_count = 0;
+      int last_par[kSelStages];
+      for (int i = 0; i < kSelStages; ++i) last_par[i] = -1;
+      for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+        mbar_expect_tx(&sm.q_full[qb], kTile);
+        tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        bool ok = true;
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kc_count % kSelStages;
+          const uint32_t ph = (kc_count / kSelStages) & 1;
+          if (!mbar_wait(&sm.kc_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); ok = false; break; }
+          mbar_expect_tx(&sm.kc_full[st], kTile);
+          tma_load_2d(sm.kc[st], &kcmap, &sm.kc_full[st], 0, ti.g * btot + ti.b0 + j * kBN);
+          last_par[st] = (int)ph;
+          ++kc_count;
+        }
+        if (!ok) break;
+      }
+      for (int i = 0; i < kSelStages; ++i)
+        if (last_par[i] >= 0) mbar_wait(&sm.kc_full[i], (uint32_t)last_par[i]);
+    }
+  } else if (warp == kOutMmaWarp) {
+    // ---------------- MMA issuer: S^T(j) into buffer j % 2 as soon as the compute warps released it
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(kBN, kRows);  // S^T[blocks, rows] = Kc Q^T
+      uint32_t kc_count = 0, q_count = 0, s_count = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
+        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const int qb = q_count % 2;
+        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
+        ++q_count;
+        const int nbt = (ti.nb + kBN - 1) / kBN;
+        for (int j = 0; j < nbt; ++j) {
+          const int st = kc_count % kSelStages;
+          const int sb = s_count % 2;
+          if (!mbar_wait(&sm.kc_full[st], (kc_count / kSelStages) & 1) ||
+              !mbar_wait(&sm.s_empty[sb], ((s_count / 2) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(tmem + sb * kBN, sdesc_kmajor_sw128(sm.kc[st], 32 * k), sdesc_kmajor_sw128(sm.q[qb], 32 * k),
+                        id_s, k > 0);
+          mma_commit(&sm.s_full[sb]);
+          mma_commit(&sm.kc_empty[st]);
+          ++kc_count;
+          ++s_count;
+        }
+        if (!ok) break;
+        mma_commit(&sm.q_empty[qb]);
+      }
+      if (!ok) record_timeout(status, &sm.abort_flag);
+      mma_commit(&sm.mma_done);
+      mbar_wait(&sm.mma_done, 0);
+    }
+  } else if (warp < kComputeWarps) {
+    // ---------------- compute warps (two warpgroups): thread = block of the key tile;
+    // warpgroup wg handles query rows [64 wg, 64 wg + 64) of the tile, in two passes of 32.
+    const int b = threadIdx.x % 128;
+    const int wg = warp / 4;
+    const int r0 = 64 * wg;
+    uint32_t s_count = 0, cw_phase = 0, n_tile = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x, ++n_tile) {
+      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+      const int lb = n_tile & 1;
+      if (wg == 0) {
+        const int r = threadIdx.x;
+        const int64_t t = min((int64_t)ti.t0 + r / G, (int64_t)ti.t_end - 1);
+        sm.lse2[lb][r] = -lse_in[t * hq + ti.g * G + r % G] * kLog2e;  // -lse log2(e)
+      }
+      if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
+      // the top-k warps have released this tile's importance buffer
+      if (!mbar_wait_warp(&sm.imp_empty[lb], ((n_tile >> 1) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+      float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
+      const int nbt = (ti.nb + kBN - 1) / kBN;
+      bool ok = true;
+      const float2 qs = make_float2(qs2, qs2);
+      for (int j = 0; j < nbt; ++j) {
+        const int sb = s_count % 2;
+        if (!mbar_wait_warp(&sm.s_full[sb], (s_count / 2) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const int bidx = j * kBN + b;  // block index inside the sequence
+        const bool bvalid = bidx < ti.nb;
+        const uint32_t taddr = tmem + sb * kBN + ((uint32_t)((warp % 4) * 32) << 16) + r0;
+        float p[2][32];
+        tmem_ld32(taddr, p[0]);
+        tmem_ld32(taddr + 32, p[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+        ++s_count;
+        if (bvalid) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+            for (int r = 0; r < 32; r += 4) {
+              const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[lb][r0 + 32 * hh + r]);
+              const float2 xa = ffma2(make_float2(p[hh][r], p[hh][r + 1]), qs, make_float2(l4.x, l4.y));
+              const float2 xb = ffma2(make_float2(p[hh][r + 2], p[hh][r + 3]), qs, make_float2(l4.z, l4.w));
+              const bool poly = 32 * hh + r < kSelPolyRows;
+              const float2 pa = poly ? ex2_poly2(xa) : ex2x2(xa);
+              const float2 pb = poly ? ex2_poly2(xb) : ex2x2(xb);
+              p[hh][r] = pa.x;
+              p[hh][r + 1] = pa.y;
+              p[hh][r + 2] = pb.x;
+              p[hh][r + 3] = pb.y;
+            }
+            // selection score of this block for the pass's tokens: probability summed over the group's heads
+#pragma unroll
+            for (int tl = 0; tl < 32 / G; ++tl) {
+              float2 acc = make_float2(p[hh][tl * G], p[hh][tl * G + 1]);
+#pragma unroll
+              for (int h2 = 2; h2 < G; h2 += 2) acc = fadd2(acc, make_float2(p[hh][tl * G + h2], p[hh][tl * G + h2 + 1]));
+              imp_base[(int64_t)((r0 + 32 * hh) / G + tl) * imp_stride + bidx] = acc.x + acc.y;
+            }
+          }
+        }
+      }
+      if (!ok) {
+        record_timeout(status, &sm.abort_flag);
+        break;
+      }
+      // this tile's scores are complete: hand them to the top-k warps
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.imp_full[lb]);
+    }
+  } else {
+    // ---------------- top-k warps: the selection of each tile's tokens (one warp per token)
+    const int tw = warp - kComputeWarps;
+    uint32_t n_tile = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x, ++n_tile) {
+      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+      const int lb = n_tile & 1;
+      if (!mbar_wait_warp(&sm.imp_full[lb], (n_tile >> 1) & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      const float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
+      for (int tk = tw; tk < TPT; tk += kOutTopkWarps) {
+        const int64_t t = ti.t0 + tk;
+        if (t < ti.t_end) {
+          const float* imp = imp_base + (int64_t)tk * imp_stride;
+          int32_t* dst = sel + (t * hkv + ti.g) * topk;
+          if (ti.nb <= 256 * kTopkRegF4) {
+            if (topk <= 16)
+              warp_topk_regs<kTopkRegF4, 16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+            else
+              warp_topk_regs<kTopkRegF4, kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+          } else if (topk <= 16) {
+            warp_topk_fast<16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+          } else {
+            warp_topk_fast<kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.imp_empty[lb]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
 // backward, dQ (thread = row): S = Q Kc^T, dP = dO Vc^T in TMEM over 64-block key
-// tiles; dS = P (w dP - D) in registers; dQ += dS Kc with dS (bf16 hi + lo) as the
-// TMEM A operand.  A CTA holds 256 TMEM columns and ~80 KB of shared memory, so two
+// tiles; dS = P (w dP - D) in registers; dQ += dS Kc with dS (bf16) as the TMEM A
+// operand.  A CTA holds 256 TMEM columns and ~80 KB of shared memory, so two
 // CTAs share an SM and one's exponentials overlap the other's MMAs.
 // ---------------------------------------------------------------------------
 constexpr int kBwdStages = 3;
@@ -1009,8 +1249,8 @@ __global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) cmp_bwd_dq_tc_kernel
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  // TMEM columns: S [0,64), dP [64,128), dS hi [128,160), dS lo [160,192), dQ [192,256)
-  const uint32_t tm_s = tmem, tm_dp = tmem + 64, tm_dsh = tmem + 128, tm_dsl = tmem + 160, tm_dq = tmem + 192;
+  // TMEM columns: S [0,64), dP [64,128), dS (bf16 pairs) [128,160), dQ [192,256)
+  const uint32_t tm_s = tmem, tm_dp = tmem + 64, tm_dsh = tmem + 128, tm_dq = tmem + 192;
 
   if (warp == 4) {
     // ---------------- TMA producer: (Q, dO) per row tile; (Kc, Vc) per key tile
@@ -1082,7 +1322,6 @@ __global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) cmp_bwd_dq_tc_kernel
           for (int k = 0; k < kDqBN / 16; ++k) {
             const uint64_t bdesc = sdesc_mnmajor_sw128(sm.kc[st], 2048 * k, kTile);
             mma_bf16_ts(tm_dq, tm_dsh + 8 * k, bdesc, id_q, j > 0 || k > 0);
-            mma_bf16_ts(tm_dq, tm_dsl + 8 * k, bdesc, id_q, true);
           }
           mma_commit(&sm.ds_empty);
           mma_commit(&sm.kv_empty[st]);
@@ -1136,13 +1375,15 @@ __global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) cmp_bwd_dq_tc_kernel
 #pragma unroll
             for (int c = 0; c < 32; ++c) sv[c] = c < nvh ? sv[c] : -CUDART_INF_F;
           }
-          // dS = p (w dP - D), p = 2^(s qs2 - lse log2 e)
-          uint32_t hi[16], lo[16];
+          // dS = p (w dP - D), p = 2^(s qs2 - lse log2 e), as one bf16 per entry: dQ of a
+          // row sums dS Kc over the row's own blocks, so the roundings of its terms are
+          // independent and stay far below the 2e-2 bound (unlike the dKc / dVc sums over
+          // up to millions of rows, which carry the low parts)
+          uint32_t hi[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
-            const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
-            split2(d, hi[c / 2], lo[c / 2]);
+            hi[c / 2] = pack2(fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2)));
           }
           if (hh == 0) {
             if (!mbar_wait_warp(&sm.ds_empty, (ds_count & 1) ^ 1)) {
@@ -1152,7 +1393,6 @@ __global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) cmp_bwd_dq_tc_kernel
             tc_fence_after();
           }
           tmem_st16(tm_dsh + lane_off + 16 * hh, hi);
-          tmem_st16(tm_dsl + lane_off + 16 * hh, lo);
         }
         if (!ok_half) {
           ok = false;

@@ -96,6 +96,7 @@ struct BwdArgs {
   int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
 };
 
+bool pool_supported(int dtype, int hkv, int d);
 cudaError_t launch_pool(int dtype, const void* k, const void* v, const ssa_partition* blk, int64_t N, int hkv,
                         int d, void* ks, void* vs, void* kc, void* vc, cudaStream_t st);
 cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st);

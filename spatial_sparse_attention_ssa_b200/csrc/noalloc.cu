@@ -13,8 +13,6 @@
 // SSA_BIN_NOALLOC_MAX_TOKENS tokens, and all calls on a device share the one
 // array -- calls whose work overlaps on the GPU (different streams, or host
 // threads racing) corrupt each other's results.
-#include <mutex>
-
 #include "common.cuh"
 
 namespace {
@@ -28,24 +26,16 @@ constexpr size_t kNoallocBytes = 11u << 20;  // 11 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
 
-// Device address of g_noalloc_scratch per device, looked up once per device.
-// In host code the array's name is only a stand-in for the symbol, never a
-// device address, so kernels must be given this looked-up pointer.
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
-
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a stand-in for the symbol, never a device address, so
+// kernels must be given this looked-up pointer.  It is looked up on every call
+// (a cheap runtime query): a cached address would go stale if the program reset
+// the device and the module were loaded again at another address.
 ssa_status scratch_for_current_device(unsigned char** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
-    void* ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || !ptr) return SSA_ERR_CUDA;
-    g_addr[dev] = ptr;
-  }
-  *out = static_cast<unsigned char*>(g_addr[dev]);
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess || !ptr) return SSA_ERR_CUDA;
+  *out = static_cast<unsigned char*>(ptr);
   return SSA_OK;
 }
 
@@ -56,8 +46,9 @@ extern "C" SSA_API ssa_status ssa_bin_noalloc(const int32_t* coords, const int32
                                               ssa_partition* blk, ssa_partition* win, void* stream) {
   if (S < 1 || N < 0 || R < 1 || R > (1 << 20) || m_cmp < 1 || m_win < 1) return SSA_ERR_INVALID_ARG;
   if (!cu_seqlens || (N > 0 && !coords) || !blk || !win) return SSA_ERR_INVALID_ARG;
-  if (!blk->id || !blk->perm || !blk->ptr || !blk->cu || !blk->key) return SSA_ERR_INVALID_ARG;
-  if (!win->id || !win->perm || !win->ptr || !win->cu || !win->key) return SSA_ERR_INVALID_ARG;
+  // per-token arrays and cell keys may be null when there are no tokens (nothing is written there)
+  if (!blk->ptr || !blk->cu || (N > 0 && (!blk->id || !blk->perm || !blk->key))) return SSA_ERR_INVALID_ARG;
+  if (!win->ptr || !win->cu || (N > 0 && (!win->id || !win->perm || !win->key))) return SSA_ERR_INVALID_ARG;
   // Inputs above the fixed scratch are refused before any work is enqueued.
   const size_t need = ssa::bin_ws_bytes(S, N);
   if (N > kNoallocTokens || need + 256 > kNoallocBytes) return SSA_ERR_WORKSPACE;

@@ -305,15 +305,15 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
 
 // x = hi + lo as two bf16 pairs, with integer and FMA-pipe instructions only (the
 // fp32 -> bf16 conversion instructions issue at a quarter of the FMA rate): hi is x
-// truncated to its upper 16 bits, lo = x - hi exactly in fp32, then rounded to bf16
-// (half away from zero, by adding 0x8000 to its bit pattern).  |x - hi - lo| is at
-// most 2^-15 |x| (|lo| < 2^-7 |x|, rounded to 8 significant bits).
+// truncated to its upper 16 bits, r = x - hi exactly in fp32, lo = r truncated the
+// same way.  |r| < 2^-7 |x| and the truncation of r loses less than 2^-7 |r|, so
+// |x - hi - lo| < 2^-14 |x|; five instructions per pair.
 __device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
   const uint32_t xa = __float_as_uint(x.x), xb = __float_as_uint(x.y);
   const float2 h = make_float2(__uint_as_float(xa & 0xffff0000u), __uint_as_float(xb & 0xffff0000u));
   const float2 r = ffma2(h, make_float2(-1.f, -1.f), x);
   hi = __byte_perm(xa, xb, 0x7632);
-  lo = __byte_perm(__float_as_uint(r.x) + 0x8000u, __float_as_uint(r.y) + 0x8000u, 0x7632);
+  lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
 }
 // x as one bf16 pair, rounded half away from zero (integer instructions only).
 __device__ __forceinline__ uint32_t pack2(float2 x) {

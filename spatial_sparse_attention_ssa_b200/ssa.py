@@ -29,7 +29,7 @@ SEL_SCORES, SEL_GIVEN = 0, 1
 
 EXPORTS = ("ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size", "ssa_error_string",
            "ssa_get_device_status", "ssa_version", "ssa_launch_count", "ssa_profile_enable",
-           "ssa_profile_read", "ssa_geo_select", "ssa_cross_forward", "ssa_cross_backward")
+           "ssa_profile_read", "ssa_geo_select", "ssa_cross_forward", "ssa_cross_backward", "ssa_pool")
 
 
 class SSAError(RuntimeError):
@@ -88,6 +88,8 @@ def _lib():
         lib.ssa_cross_backward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, i64, pp, vp, vp, vp, vp,
                                            ctypes.POINTER(Saved), vp, vp, vp, vp, vp, vp, sz, vp]
         lib.ssa_cross_backward.restype = ctypes.c_int
+        lib.ssa_pool.argtypes = [i32, i32, i32, i64, pp, vp, vp, vp, vp, vp, vp, vp]
+        lib.ssa_pool.restype = ctypes.c_int
         lib.ssa_geo_select.argtypes = [vp, vp, i32, i64, i32, pp, i32, i32, i32, vp, vp, sz, vp]
         lib.ssa_geo_select.restype = ctypes.c_int
         lib.ssa_workspace_size.argtypes = [i32, ctypes.POINTER(Params), i32, i64, i64, i64]
@@ -182,6 +184,23 @@ def ssa_bin(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, m_cmp: int, 
     blk.count = int(pb.count)
     win.count = int(pw.count)
     return blk, win
+
+
+def ssa_pool(blk: "Bins", k: torch.Tensor, v: torch.Tensor, out=None):
+    """Step 2 alone: (ks, vs, kc, vc) -- K and V gathered in block order, head-major
+    [Hkv, N, d], and the block means [Hkv, B, d], in the dtype of k."""
+    _require_cuda(k, v)
+    n, hkv, d = (int(x) for x in k.shape)
+    dt = DTYPE_BF16 if k.dtype == torch.bfloat16 else DTYPE_F32
+    if out is None:
+        e = lambda *shape: torch.empty(*shape, dtype=k.dtype, device=k.device)  # noqa: E731
+        out = (e(hkv, n, d), e(hkv, n, d), e(hkv, max(blk.count, 1), d), e(hkv, max(blk.count, 1), d))
+    ks, vs, kc, vc = out
+    pb = blk.c()
+    st = _lib().ssa_pool(dt, hkv, d, n, ctypes.byref(pb), _ptr(k), _ptr(v), _ptr(ks), _ptr(vs), _ptr(kc), _ptr(vc),
+                         _stream(k.device))
+    _check(st, "ssa_pool")
+    return ks, vs, kc, vc
 
 
 def ssa_geo_select(coords: torch.Tensor, cu_seqlens: torch.Tensor, R: int, blk: "Bins", m_cmp: int, topk: int,

@@ -47,7 +47,7 @@ def test_algorithmic_work_counts_scores_by_brute_force():
         for g in range(w.hkv):
             pick = rng.choice(np.arange(b0, b1), size=min(w.topk, b1 - b0), replace=False)
             sel[t, g, :len(pick)] = np.sort(pick)
-    work, scores = bench.kernel_work(w, blk["ptr"], blk["cu"], win["ptr"], sel)
+    work, stages, scores = bench.kernel_work(w, blk["ptr"], blk["cu"], win["ptr"], sel)
     G = w.hq // w.hkv
     cmp = slc = wnd = 0
     for t in range(w.n):
@@ -57,5 +57,12 @@ def test_algorithmic_work_counts_scores_by_brute_force():
             wnd += int((win["id"] == win["id"][t]).sum())  # every token of its window
     assert scores == {"cmp": float(cmp), "slc": float(slc), "win": float(wnd)}
     for name, per_score in (("cmp_lse_tc_kernel", 1), ("cmp_out_tc_kernel", 2), ("cmp_bwd_dq_tc_kernel", 3),
-                            ("cmp_bwd_dkv_tc_kernel", 4)):
+                            ("cmp_bwd_dkv_tc_kernel", 4), ("cmp_fa_tc_kernel", 2), ("cmp_sel_tc_kernel", 1)):
         assert work[name][1] == 2 * w.d * per_score * cmp, name
+    # stages count each contraction of the method once: the compressed forward needs S for the
+    # normaliser, S again for the selection's final probabilities and P V (6d); every backward
+    # needs S, dP, dQ, dK and dV (10d)
+    assert stages["compressed forward"][1:] == (6 * w.d * cmp, 2 * cmp)
+    assert stages["compressed backward"][1:] == (10 * w.d * cmp, cmp)
+    assert stages["window backward"][1] == 10 * w.d * wnd and stages["selected backward"][1] == 10 * w.d * slc
+    assert stages["window forward"][1] == 4 * w.d * wnd and stages["selected forward"][1] == 4 * w.d * slc

@@ -15,10 +15,11 @@ import functools
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import ssa_oracle as O
 from spatial_sparse_attention_ssa_b200 import workloads as W
-from tests.ssa_testlib import ATOL, DeviceRun, compare_forward, f64, max_abs, run_oracle
+from tests.ssa_testlib import ATOL, TAU_SEL, DeviceRun, compare_forward, f64, max_abs, run_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -111,3 +112,119 @@ def test_window_gradients_of_sampled_windows_at_full_size():
     print(len(wins), sizes[wins].max(), e)
     for key, val in e.items():
         assert val <= ATOL[w.dtype], (key, val)
+
+
+# ----------------------------------------------------------------------------
+# the compressed branch for every token at the benchmark size, and the selected
+# branch's key gradients of sampled blocks
+# ----------------------------------------------------------------------------
+
+
+def _one_hot(t, c):
+    gates = np.zeros_like(t.gates)
+    gates[:, :, c] = 1.0
+    return dataclasses.replace(t, gates=gates)
+
+
+@functools.lru_cache(maxsize=1)
+def _cmp_only_run():
+    """Config 5 with the compressed branch alone switched on (gate weights one-hot,
+    so the other branches add exact zeros to out, dQ, dK and dV): the GPU's
+    results and the oracle's compressed branch over all 131072 query tokens."""
+    from tests import cmp_full
+
+    w, t = _load(5)
+    w = dataclasses.replace(w, gate_mode=0)
+    t = _one_hot(t, 0)
+    run = DeviceRun(w, t).run()
+    blk = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)
+    kc = O.mean_pool(t.as_f32("k").astype(np.float64), blk, "bf16")
+    vc = O.mean_pool(t.as_f32("v").astype(np.float64), blk, "bf16")
+    dq, dk, dv, dg = (x.cpu().numpy() for x in run.grads)
+    arrays = {"q": t.q, "do": t.do, "gates": t.gates, "kc": kc, "vc": vc,
+              "sel_gpu": run.saved.sel.cpu().numpy(), "o_cmp_gpu": run.saved.o_branch[0].cpu().numpy(),
+              "lse_gpu": run.saved.lse[0].cpu().numpy(), "dq_gpu": dq, "dgates_gpu": dg,
+              "out_gpu": run.out.view(torch.int16).cpu().numpy().view(np.uint16)}
+    meta = {"blk_cu": blk["cu"], "cu": np.asarray(w.cu_seqlens, np.int64), "hq": w.hq, "hkv": w.hkv,
+            "topk": w.topk, "gate_mode": 0}
+    res = cmp_full.run(arrays, meta, w.n)
+    return w, t, blk, run, res, dk, dv
+
+
+def test_compressed_branch_every_token_at_full_size():
+    """Config 5 (131072 tokens, 2322 blocks, 9.7e9 compressed scores), compressed
+    branch only: lse, o_cmp, out, dQ and dgates of every query row, the selection of
+    every (token, group) (equal, or a certified near-tie), and dK / dV of every
+    token element by element against the oracle at 2e-2."""
+    w, t, blk, run, res, dk, dv = _cmp_only_run()
+    tol = ATOL[w.dtype]
+    flips = res["flips"]
+    assert res["bad_sel_rows"] == 0
+    assert all(gap >= -TAU_SEL for _, _, gap in flips), [f for f in flips if f[2] < -TAU_SEL][:5]
+    dk_ref, dv_ref = O.cmp_token_grads(res["dkc"], res["dvc"], blk)
+    errs = {key: res[key] for key in ("o", "lse", "out", "dq", "dgates_cmp")}
+    errs["dk"] = max_abs(dk, dk_ref)
+    errs["dv"] = max_abs(dv, dv_ref)
+    print("every token:", errs, "flips", len(flips), "of", w.n * w.hkv, "procs", res["procs"],
+          "max |dK|, |dV|", float(np.abs(dk_ref).max()), float(np.abs(dv_ref).max()))
+    for key, e in errs.items():
+        assert e <= tol, (key, e, tol)
+
+
+def test_selected_branch_key_gradients_of_sampled_blocks_at_full_size():
+    """Config 5 with the selected branch alone switched on: dK / dV of every token
+    of 16 blocks (the 4 most selected, 4 more that are selected, 8 at random, some of
+    them selected by nobody, whose gradient must be exactly zero), each against the
+    sum over all (token, group) rows whose selection holds the block.  The rows use
+    the GPU's selection, which the compressed-branch test certifies."""
+    w, t = _load(5)
+    w = dataclasses.replace(w, gate_mode=0)
+    t = _one_hot(t, 1)
+    run = DeviceRun(w, t).run()
+    sel = run.saved.sel.cpu().numpy()
+    blk = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)
+    counts = np.bincount(sel[sel >= 0], minlength=blk["count"])
+    rng = np.random.default_rng(9)
+    chosen = list(np.argsort(-counts, kind="stable")[:4])
+    used = np.nonzero(counts)[0]
+    chosen += list(rng.choice(used, 4, replace=False))
+    chosen += list(rng.choice(blk["count"], 8, replace=False))
+    chosen = sorted(set(int(b) for b in chosen))
+    q, k, v, do = (t.as_f32(x).astype(np.float64) for x in ("q", "k", "v", "do"))
+    G = w.hq // w.hkv
+    scale = 1.0 / np.sqrt(w.d)
+    dk_ref = {b: np.zeros((blk["ptr"][b + 1] - blk["ptr"][b], w.hkv, w.d)) for b in chosen}
+    dv_ref = {b: np.zeros_like(dk_ref[b]) for b in chosen}
+    want = set(chosen)
+    rows_seen = 0
+    tt_all, gg_all = np.nonzero(np.isin(sel, chosen).any(axis=2))
+    for tt, g in zip(tt_all, gg_all):
+        row = sel[tt, g]
+        js = O.selected_tokens(row, blk)
+        hs = slice(g * G, (g + 1) * G)
+        s_ = scale * (q[tt, hs] @ k[js, g].T)
+        p = np.exp(s_ - O._logsumexp(s_, -1)[:, None])
+        dp = do[tt, hs] @ v[js, g].T
+        ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+        dkj = scale * (ds.T @ q[tt, hs])
+        dvj = p.T @ do[tt, hs]
+        off = 0
+        for b in row:
+            if b < 0:
+                continue
+            nb = int(blk["ptr"][b + 1] - blk["ptr"][b])
+            if b in want:
+                dk_ref[b][:, g] += dkj[off:off + nb]
+                dv_ref[b][:, g] += dvj[off:off + nb]
+            off += nb
+        rows_seen += 1
+    dk, dv = (x.cpu().numpy() for x in run.grads[1:3])
+    errs = {}
+    for b in chosen:
+        members = blk["perm"][blk["ptr"][b]:blk["ptr"][b + 1]]
+        errs[b] = (max_abs(dk[members], dk_ref[b]), max_abs(dv[members], dv_ref[b]), int(counts[b]))
+        if counts[b] == 0:
+            assert not dk[members].any() and not dv[members].any(), b
+    print("selected blocks (dk err, dv err, rows):", errs, "rows", rows_seen)
+    for b, (ek, ev, _) in errs.items():
+        assert ek <= ATOL[w.dtype] and ev <= ATOL[w.dtype], (b, ek, ev)

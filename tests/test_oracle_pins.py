@@ -785,3 +785,137 @@ def test_cross_subset_of_query_rows_matches_full():
     np.testing.assert_array_equal(sub["sel"][rows], full["sel"][rows])
     np.testing.assert_array_equal(sub["o"][:, rows], full["o"][:, rows])
     np.testing.assert_array_equal(sub["out"][rows], full["out"][rows])
+
+
+# ----------------------------------------------------------------------------
+# the compressed branch over token ranges (used by the full-size GPU checks)
+# ----------------------------------------------------------------------------
+
+
+def _ranges_run(w, t, gates, gate_mode, bounds, sel_other=None):
+    st = O.forward(w.coords, w.cu_seqlens, t.as_f32("q"), t.as_f32("k"), t.as_f32("v"), gates, hq=w.hq,
+                   hkv=w.hkv, m_cmp=w.m_cmp, m_win=w.m_win, topk=w.topk, gate_mode=gate_mode)
+    parts = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        so = None if sel_other is None else sel_other[a:b]
+        parts.append(O.cmp_branch_range(t.as_f32("q"), st["kc"], st["vc"], st["blk"]["cu"], w.cu_seqlens, gates,
+                                        hq=w.hq, hkv=w.hkv, topk=w.topk, gate_mode=gate_mode, t0=a, t1=b,
+                                        dout=t.as_f32("do"), chunk=37, sel_other=so))
+    return st, parts
+
+
+def test_cmp_branch_ranges_match_the_full_forward_and_backward():
+    """Split at points inside sequences, the ranges reproduce the compressed branch
+    of `forward` / `backward`: lse, output, selection and dQ row by row, and dKc /
+    dVc (hence the tokens' dK / dV) as sums over the ranges."""
+    w, t = _small_workload(seed=4, n_seqs=3)
+    bounds = [0, 17, w.n // 2 + 3, w.n - 5, w.n]
+    st, parts = _ranges_run(w, t, t.gates, 1, bounds)
+    g = O.backward(st, t.as_f32("do"))
+    cat = lambda key: np.concatenate([p[key] for p in parts])  # noqa: E731
+    np.testing.assert_allclose(cat("lse"), st["lse"][0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(cat("o"), st["o"][0], rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(cat("sel"), st["sel"])
+    np.testing.assert_allclose(cat("dq"), g["parts"]["dq"]["cmp"], rtol=0, atol=1e-12)
+    dkc = sum(p["dkc"] for p in parts)
+    dvc = sum(p["dvc"] for p in parts)
+    np.testing.assert_allclose(dkc, g["parts"]["dkc"], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dvc, g["parts"]["dvc"], rtol=0, atol=1e-11)
+    dk, dv = O.cmp_token_grads(dkc, dvc, st["blk"])
+    np.testing.assert_allclose(dk, g["parts"]["dk"]["cmp"], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, g["parts"]["dv"]["cmp"], rtol=0, atol=1e-11)
+
+
+def test_cmp_branch_range_with_unit_blocks_is_full_attention_and_its_gradient():
+    """With one token per block (m_cmp = 1, unique coordinates) and the exact mean,
+    the compressed branch is textbook full attention: its output, and its dQ / dK /
+    dV against torch autograd of scaled_dot_product_attention (fp64)."""
+    coords, cu, q, k, v, gates = _rand_case(21)
+    hq, hkv, G = 4, 2, 2
+    k = k.astype(np.float32).astype(np.float64)  # fp32-representable: the f32 mean of one is itself
+    v = v.astype(np.float32).astype(np.float64)
+    blk = O.bin_tokens(coords, cu, 1)
+    kc, vc = O.mean_pool(k, blk, "f32"), O.mean_pool(v, blk, "f32")
+    rng = np.random.default_rng(5)
+    do = rng.standard_normal(q.shape)
+    gates = np.ones_like(gates)
+    r = O.cmp_branch_range(q, kc, vc, blk["cu"], cu, gates, hq=hq, hkv=hkv, topk=3, gate_mode=0, t0=0,
+                           t1=len(coords), dout=do)
+    np.testing.assert_allclose(r["o"], _sdpa_full(q, k, v, cu, hq, hkv), rtol=0, atol=1e-12)
+    dk, dv = O.cmp_token_grads(r["dkc"], r["dvc"], blk)
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        if a == b:
+            continue
+        qt = torch.from_numpy(q[a:b]).transpose(0, 1).requires_grad_()
+        kt = torch.from_numpy(k[a:b]).transpose(0, 1).requires_grad_()
+        vt = torch.from_numpy(v[a:b]).transpose(0, 1).requires_grad_()
+        o = torch.nn.functional.scaled_dot_product_attention(qt, kt.repeat_interleave(G, 0),
+                                                             vt.repeat_interleave(G, 0))
+        o.backward(torch.from_numpy(do[a:b]).transpose(0, 1))
+        np.testing.assert_allclose(r["dq"][a:b], qt.grad.transpose(0, 1).numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dk[a:b], kt.grad.transpose(0, 1).numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dv[a:b], vt.grad.transpose(0, 1).numpy(), rtol=0, atol=1e-11)
+
+
+def test_cmp_branch_gap_certifies_only_top_k_selections():
+    """other_gap of the oracle's own selection is >= 0; moving one pick to the best
+    block left out makes it exactly minus the score difference of the two blocks."""
+    w, t = _small_workload(seed=6, n_seqs=2)
+    st0, _ = _ranges_run(w, t, t.gates, 1, [0, w.n])
+    sel = st0["sel"].copy()
+    st, parts = _ranges_run(w, t, t.gates, 1, [0, w.n], sel_other=sel)
+    assert (parts[0]["other_gap"] >= 0).all()
+    moved = sel.copy()
+    rows = []
+    for tt in range(0, w.n, 7):
+        s = int(np.searchsorted(w.cu_seqlens, tt, side="right") - 1)
+        b0, b1 = int(st["blk"]["cu"][s]), int(st["blk"]["cu"][s + 1])
+        if b1 - b0 <= w.topk:
+            continue
+        imp = O.importance(st, tt, 0)
+        chosen = [int(x) for x in sel[tt, 0] if x >= 0]
+        rest = [b for b in range(b0, b1) if b not in chosen]
+        best = max(rest, key=lambda b: (imp[b - b0], -b))
+        worst = min(chosen, key=lambda b: (imp[b - b0], -b))
+        moved[tt, 0] = np.sort([b for b in chosen if b != worst] + [best])
+        rows.append((tt, imp[worst - b0] - imp[best - b0], imp))
+    _, parts2 = _ranges_run(w, t, t.gates, 1, [0, w.n], sel_other=moved)
+    for tt, diff, imp in rows:
+        gap = parts2[0]["other_gap"][tt, 0]
+        # the moved-in block is now the lowest chosen and the moved-out one the highest left out
+        assert gap <= 0 and abs(gap - (-(abs(diff)))) <= 1e-12, (tt, gap, diff)
+
+
+def test_attend_with_sel_equals_the_forward_given_that_selection():
+    """attend_with_sel (the check of rows whose selection flipped on the GPU) against
+    forward(sel_given=...) with a selection that differs from the score top-k, and
+    against textbook attention when the selection covers the sequence."""
+    w, t = _small_workload(seed=7, n_seqs=2)
+    st = _run(w, t)
+    rng = np.random.default_rng(3)
+    other = st["sel"].copy()
+    for tt in range(w.n):
+        s = int(np.searchsorted(w.cu_seqlens, tt, side="right") - 1)
+        b0, b1 = int(st["blk"]["cu"][s]), int(st["blk"]["cu"][s + 1])
+        k_eff = min(w.topk, b1 - b0)
+        for g in range(w.hkv):
+            other[tt, g, :k_eff] = np.sort(rng.choice(np.arange(b0, b1), size=k_eff, replace=False))
+    assert (other != st["sel"]).any()
+    st2 = _run(w, t, sel_given=other)
+    G = w.hq // w.hkv
+    for tt in range(0, w.n, 3):
+        for g in range(w.hkv):
+            l_, o_ = O.attend_with_sel(st, tt, g, other[tt, g])
+            np.testing.assert_allclose(o_, st2["o"][1][tt, g * G:(g + 1) * G], rtol=0, atol=1e-13)
+            np.testing.assert_allclose(l_, st2["lse"][1][tt, g * G:(g + 1) * G], rtol=0, atol=1e-13)
+    # every block of the sequence: the selected branch is full attention
+    coords, cu, q, k, v, gates = _rand_case(17)
+    stf = O.forward(coords, cu, q, k, v, gates, hq=4, hkv=2, m_cmp=4, m_win=4, topk=3, gate_mode=1)
+    full = _sdpa_full(q, k, v, cu, 4, 2)
+    for tt in (0, 45, 89, 90, 146):
+        s = int(np.searchsorted(cu, tt, side="right") - 1)
+        ids = np.arange(stf["blk"]["cu"][s], stf["blk"]["cu"][s + 1])
+        for g in range(2):
+            _, o_ = O.attend_with_sel(stf, tt, g, ids)
+            np.testing.assert_allclose(o_, full[tt, 2 * g:2 * g + 2], rtol=0, atol=1e-12)

@@ -77,3 +77,31 @@ def test_noalloc_refuses_inputs_above_its_fixed_scratch():
     status, blk, _ = _raw_noalloc(coords[:MAX_TOKENS].contiguous(),
                                   torch.tensor([0, MAX_TOKENS], dtype=torch.int32, device="cuda"), 64, 4, 4)
     assert status == 0 and blk.count == 1
+
+
+def test_noalloc_matches_the_oracle_and_recovers_after_a_failed_call():
+    """Against the oracle's binning directly; a call with a coordinate outside
+    [0, R) reports SSA_ERR_COORD_RANGE, and the next valid call still returns
+    SSA_OK with the right partition (the check word left in the shared scratch by
+    the failed call is cleared); N = 0 returns zero counts and all-zero offsets."""
+    from oracle import ssa_oracle as O
+    from tests.ssa_testlib import assert_bins_equal
+
+    w = W.small_shell(seed=12, R=40, n_prims=3, lo=4.0, hi=10.0, n_seqs=3)
+    coords, cu = _inputs(w)
+    bad = coords.clone()
+    bad[5, 1] = w.R  # one coordinate out of range
+    status, _, _ = _raw_noalloc(bad, cu, w.R, 4, 2)
+    torch.cuda.synchronize()
+    assert status == 4  # SSA_ERR_COORD_RANGE
+    status, blk, win = _raw_noalloc(coords, cu, w.R, 4, 2)
+    torch.cuda.synchronize()
+    assert status == 0, ssa.lib().ssa_error_string(status)
+    assert_bins_equal(blk, O.bin_tokens(w.coords, w.cu_seqlens, 4), "blk")
+    assert_bins_equal(win, O.bin_tokens(w.coords, w.cu_seqlens, 2), "win")
+    empty = torch.zeros(0, 3, dtype=torch.int32, device="cuda")
+    cu0 = torch.zeros(4, dtype=torch.int32, device="cuda")
+    status, blk0, win0 = _raw_noalloc(empty, cu0, 16, 4, 4)
+    torch.cuda.synchronize()
+    assert status == 0 and blk0.count == 0 and win0.count == 0
+    assert not blk0.cu.any() and not win0.cu.any()
