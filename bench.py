@@ -51,6 +51,10 @@ def _args():
     ap.add_argument("--no-geo", action="store_true", help="skip the separate timing of geometric block routing")
     ap.add_argument("--no-cross", action="store_true", help="skip the separate timing of cross attention")
     ap.add_argument("--no-conv", action="store_true", help="skip the separate timing of the learned compression")
+    ap.add_argument("--no-scaled", action="store_true",
+                    help="skip the timing of binning + compression at 16 * 2^20 tokens (HBM roofline)")
+    ap.add_argument("--scaled-copies", type=int, default=128,
+                    help="sequences of the scaled memory-bound leg (each a copy of the benchmark shell)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -547,6 +551,71 @@ def run_ours(a):
                            "N(0, 0.3^2/(9d)) weights) before the block mean, gradients to the weights included"}
         del l_wf, l_wb
 
+    # ---- the memory-bound steps at scale: binning (ssa_bin) and compression (ssa_pool) of
+    # 16 * 2^20 tokens, 128 sequences each holding a copy of the benchmark shell's coordinates,
+    # N(0,1) bf16 K / V drawn on the device.  At 131072 tokens these kernels are launch- and
+    # latency-bound (1.5 MB of coordinates); at this size their HBM rate shows.
+    scaled = None
+    if not a.no_scaled:
+        del bins, ws_bin
+        torch.cuda.empty_cache()
+        copies = a.scaled_copies
+        ns = copies * n
+        sc_coords = coords.repeat(copies, 1).contiguous()
+        sc_cu = (torch.arange(copies + 1, device=dev, dtype=torch.int64) * n).to(torch.int32)
+        gen = torch.Generator(device=dev).manual_seed(1234)
+        sk = torch.randn((ns, w.hkv, w.d), device=dev, generator=gen).to(torch.bfloat16)
+        sv = torch.randn((ns, w.hkv, w.d), device=dev, generator=gen).to(torch.bfloat16)
+        sbins = (ssa.Bins.empty(ns, copies, dev), ssa.Bins.empty(ns, copies, dev))
+        sws = torch.empty(ssa.lib().ssa_workspace_size(ssa.OP_BIN, None, copies, ns, ns, ns), dtype=torch.uint8,
+                          device=dev)
+        sb, sw = ssa.ssa_bin(sc_coords, sc_cu, w.R, w.m_cmp, w.m_win, out=sbins, workspace=sws)
+        pool_out = ssa.ssa_pool(sb, sk, sv)
+        torch.cuda.synchronize()
+        check_device("scaled warm-up")
+        reps = max(3, a.steps)
+        ssa.profile_read()
+        ssa.profile_enable(True)
+        eb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i in range(reps):
+            flush.zero_()
+            eb[i][0].record()
+            sb, sw = ssa.ssa_bin(sc_coords, sc_cu, w.R, w.m_cmp, w.m_win, out=sbins, workspace=sws)
+            eb[i][1].record()
+            flush.zero_()
+            ssa.ssa_pool(sb, sk, sv, out=pool_out)
+        torch.cuda.synchronize()
+        ssa.profile_enable(False)
+        sprof = ssa.profile_read()
+        check_device("scaled binning and compression")
+        bin_ms = sum(a_.elapsed_time(b_) for a_, b_ in eb) / reps
+        nb_s, nw_s = int(sb.count), int(sw.count)
+        # bytes the steps must move: binning reads the coordinates and writes, per partition, the
+        # token ids and permutation and, per cell, its pointer and key; compression reads K and V
+        # and writes their block-ordered copies and the block means
+        bin_bytes = 12.0 * ns + 2 * 8.0 * ns + 16.0 * (nb_s + nw_s)
+        pool_bytes = 4.0 * ns * w.hkv * w.d * 2 + 2.0 * nb_s * w.hkv * w.d * 2
+        pool_ms = sprof["pool_kernel"][0] / max(sprof["pool_kernel"][1], 1) if "pool_kernel" in sprof else None
+        bin_kernels = {k_: v_[0] / reps for k_, v_ in sprof.items() if k_ != "pool_kernel"}
+        bin_kernel_ms = sum(bin_kernels.values())
+        hbm = peaks["hbm_gbs"]
+        scaled = {"tokens": ns, "sequences": copies, "blocks": nb_s,
+                  "pool": {"ms": pool_ms, "bytes": pool_bytes,
+                           "gbs": pool_bytes / (pool_ms / 1e3) / 1e9 if pool_ms else None,
+                           "hbm_frac": pool_bytes / (pool_ms / 1e3) / 1e9 / hbm if pool_ms else None},
+                  "bin": {"ms_call": bin_ms, "ms_kernels": bin_kernel_ms, "bytes": bin_bytes,
+                          "gbs_call": bin_bytes / (bin_ms / 1e3) / 1e9,
+                          "hbm_frac_call": bin_bytes / (bin_ms / 1e3) / 1e9 / hbm,
+                          "gbs_kernels": bin_bytes / (bin_kernel_ms / 1e3) / 1e9,
+                          "hbm_frac_kernels": bin_bytes / (bin_kernel_ms / 1e3) / 1e9 / hbm,
+                          "kernels_ms": bin_kernels},
+                  "peak_gbs": hbm, "peak_source": peaks["_source"],
+                  "what": "ssa_bin (device events around the call, which synchronises once) and ssa_pool "
+                          "(pool_kernel events) at 16 * 2^20 tokens; algorithmic bytes: binning 12 B of "
+                          "coordinates + 2 x 8 B of ids / permutation per token + 16 B per cell; compression "
+                          "2 x 2 x Hkv x d x 2 B per token + 2 x Hkv x d x 2 B per block"}
+        del sk, sv, sbins, sws, pool_out, sc_coords
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -565,7 +634,7 @@ def run_ours(a):
                 "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(launches),
                 "clocks": clocks, "wall_s_timed": wall, "kernels": per_kernel, "geo_routing": geo,
-                "cross_attention": cross, "learned_compression": learned,
+                "cross_attention": cross, "learned_compression": learned, "memory_bound_scaled": scaled,
                 "peaks_source": peaks["_source"]}
         print(json.dumps(line), flush=True)
     if world > 1:

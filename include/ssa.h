@@ -71,7 +71,9 @@ enum {
   SSA_OP_BACKWARD = 2,
   SSA_OP_GEO_SELECT = 3,
   SSA_OP_CROSS_FORWARD = 4,
-  SSA_OP_CROSS_BACKWARD = 5
+  SSA_OP_CROSS_BACKWARD = 5,
+  SSA_OP_SP_FORWARD = 6,
+  SSA_OP_SP_BACKWARD = 7
 };
 
 /* Shape and method parameters shared by forward and backward. */
@@ -100,7 +102,7 @@ typedef struct ssa_conv {
 typedef struct ssa_params {
   int32_t hq;        /* query heads */
   int32_t hkv;       /* key/value heads; hq % hkv == 0, G = hq / hkv in {1,2,4,8,16} */
-  int32_t d;         /* head dim: 32 or 64 */
+  int32_t d;         /* head dim: 32, 64 or 128 (128: G * 4 <= 32, i.e. G <= 8; the fp32 CUDA-core kernels) */
   int32_t m_cmp;     /* compression block edge (voxels), >= 1 */
   int32_t m_win;     /* window edge (voxels), >= 1 */
   int32_t topk;      /* selected blocks per (token, KV head), 1..32 */
@@ -305,10 +307,58 @@ SSA_API ssa_status ssa_cross_backward(const ssa_params* p, const int32_t* q_cu, 
                                       void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * One rank's share of a batch whose sequences are split across ranks by whole blocks
+ * (LSRM, "块感知序列并行与负载均衡": a rank owns a contiguous range of a sequence's
+ * blocks and their tokens; compression and window attention stay local; the keys and
+ * values are exchanged; the key gradients go back to their owners).  The rank's query
+ * tokens attend every compressed block and the tokens of their selected blocks of the
+ * whole sequence (the K / V of all tokens, exchanged by the caller), and their windows,
+ * which lie inside the rank's blocks when m_cmp is a multiple of m_win.
+ */
+typedef struct ssa_sp_local {
+  int64_t n;                  /* Nr: this rank's tokens over all sequences */
+  const int32_t* cu_seqlens;  /* [S+1] device: this rank's tokens of sequence s are rows cu[s] .. cu[s+1]-1 */
+  const int32_t* tokens;      /* [Nr] device: the row of each of them in the all-token arrays (distinct) */
+  const ssa_partition* win;   /* ssa_bin of this rank's coordinates with this cu_seqlens, edge m_win */
+  const void* k;              /* [Nr, Hkv, d] dtype: this rank's K rows (the values of k[tokens]) */
+  const void* v;              /* [Nr, Hkv, d] dtype */
+  void* ks;                   /* [Hkv, Nr, d] dtype: their window-ordered copies, written by ssa_sp_forward */
+  void* vs;                   /*   and read by ssa_sp_backward */
+} ssa_sp_local;
+
+/*
+ * ssa_sp_forward -- the rank's forward: for its Nr query tokens q / gates [Nr, Hq, 3]
+ * (rows in the order of loc->tokens), out [Nr, Hq, d] = sum_c w_c o_c of the three
+ * branches, exactly as ssa_forward computes those rows on the whole batch.
+ *   blk: ssa_bin of all N tokens (every rank bins the same coordinates); k, v [N, Hkv, d]
+ *   all tokens.  saved: kc / vc [Hkv, B, d] and ks / vs [Hkv, N, d] of all tokens;
+ *   o_branch [3, Nr, Hq, d], lse [3, Nr, Hq], sel [Nr, Hkv, topk] of the rank's rows.
+ *   ws: ssa_workspace_size(SSA_OP_SP_FORWARD, p, S, Nr, B, loc->win->count) bytes.
+ * SSA_ERR_INVALID_ARG if m_cmp is not a multiple of m_win (a window would cross blocks)
+ * or params->conv is set.  Asynchronous.
+ *
+ * ssa_sp_backward -- the rank's backward: dq [Nr, Hq, d] and dgates [Nr, Hq, 3] of its
+ * rows, and dk, dv [N, Hkv, d] (all written): the contributions of its query rows to the
+ * gradient of every token's key and value.  Summed over the ranks they give the batch's
+ * dK, dV (each rank keeps the rows of its own tokens: a reduce-scatter).  `saved` and
+ * `loc` as left by ssa_sp_forward on the same inputs.
+ *   ws: ssa_workspace_size(SSA_OP_SP_BACKWARD, p, S, Nr, B, loc->win->count) bytes.
+ */
+SSA_API ssa_status ssa_sp_forward(const ssa_params* p, int32_t S, int64_t N, const ssa_partition* blk,
+                                  const ssa_sp_local* loc, const void* q, const void* k, const void* v,
+                                  const float* gates, void* out, const ssa_saved* saved, void* ws, size_t ws_bytes,
+                                  void* stream);
+SSA_API ssa_status ssa_sp_backward(const ssa_params* p, int32_t S, int64_t N, const ssa_partition* blk,
+                                   const ssa_sp_local* loc, const void* q, const void* k, const void* v,
+                                   const float* gates, const ssa_saved* saved, const void* dout, float* dq,
+                                   float* dk, float* dv, float* dgates, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Workspace bytes needed by `op` (SSA_OP_BIN / _FORWARD / _BACKWARD / _GEO_SELECT /
- * _CROSS_FORWARD / _CROSS_BACKWARD) for the given sizes; B_tot and W_tot are the
- * partition counts (pass N as an upper bound before binning); for the cross ops N
- * is the number of query tokens and W_tot is ignored.  The workspace must be
+ * _CROSS_FORWARD / _CROSS_BACKWARD / _SP_FORWARD / _SP_BACKWARD) for the given sizes;
+ * B_tot and W_tot are the partition counts (pass N as an upper bound before binning);
+ * for the cross ops N is the number of query tokens and W_tot is ignored; for the
+ * sequence-parallel ops N is the rank's token count and W_tot its window count.  The workspace must be
  * 256-byte aligned.  Returns 0 for invalid arguments.
  */
 SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, int64_t N,
@@ -338,6 +388,25 @@ SSA_API uint64_t ssa_launch_count(void);
 SSA_API void ssa_profile_enable(int32_t on);
 SSA_API int32_t ssa_profile_read(char* names, int32_t name_len, float* total_ms, int32_t* launches,
                                  int32_t max_entries);
+
+/*
+ * Diagnostics (no counterpart on the pages; for tests of the library itself).
+ *
+ * ssa_diag_wait_timeout: launches one warp that waits on an mbarrier nothing arrives
+ * at, with the same bounded waits the tensor-core kernels use (about one second of
+ * device time each): first one lane, then the whole warp.  Both give up, the kernel
+ * records the timeout in the device check word and returns; gave_up (device int32[2])
+ * receives 1 for each wait that gave up.  The following ssa_get_device_status then
+ * returns SSA_ERR_TIMEOUT, and the context stays usable.  Asynchronous.
+ *
+ * ssa_diag_ex2: y_poly[i] = 2^x[i] evaluated on the FMA pipe the way the kernels do
+ * for part of their exponentials (x clamped at -127; 2^x = 2^j * 2^f with j = round(x),
+ * 2^f a degree-5 polynomial interpolating at the Chebyshev nodes of [-1/2, 1/2]), and
+ * y_mufu[i] = the hardware approximation (ex2.approx.ftz.f32).  Device pointers, n
+ * values each.  Asynchronous.
+ */
+SSA_API ssa_status ssa_diag_wait_timeout(int32_t* gave_up, void* stream);
+SSA_API ssa_status ssa_diag_ex2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream);
 
 /* Library version as major*10000 + minor*100 + patch. */
 SSA_API int32_t ssa_version(void);

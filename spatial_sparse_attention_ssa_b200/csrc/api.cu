@@ -44,7 +44,7 @@ ssa_status check_params(const ssa_params* p) {
   if (p->conv && (!p->conv->coords || !p->conv->wk || !p->conv->bk || !p->conv->wv || !p->conv->bv))
     return SSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.f) || isinf(p->scale)) return SSA_ERR_INVALID_ARG;
-  if (p->d != 32 && p->d != 64) return SSA_ERR_UNSUPPORTED;
+  if (p->d != 32 && p->d != 64 && p->d != 128) return SSA_ERR_UNSUPPORTED;
   if (p->topk > 32) return SSA_ERR_UNSUPPORTED;
   const int G = p->hq / p->hkv;
   if (G & (G - 1)) return SSA_ERR_UNSUPPORTED;  // power of two
@@ -136,6 +136,16 @@ ssa::ConvArgs conv_args(const ssa_params* p, const ssa_partition* blk, int32_t S
 // columns (the kernels read gates with a row stride of 3) and one check word.
 size_t cross_extra_bytes(int64_t Nq, int hq) { return align256(sizeof(float) * 3 * (size_t)Nq * hq) + 256; }
 
+// Sequence-parallel extras after the regular workspace: the rank's window means
+// (forward; [Hkv, W, d] each for K and V) or its window key gradients (backward;
+// [Nr, Hkv, d] fp32 each).
+size_t sp_fwd_extra(const ssa_params* p, int64_t W) {
+  return 2 * align256((size_t)p->hkv * (W > 0 ? W : 1) * p->d * (p->dtype == SSA_DTYPE_BF16 ? 2 : 4)) + 256;
+}
+size_t sp_bwd_extra(const ssa_params* p, int64_t Nr) {
+  return 2 * align256(sizeof(float) * (size_t)(Nr > 0 ? Nr : 1) * p->hkv * p->d) + 256;
+}
+
 struct BwdWs {
   float* Dc;
   float* rc;
@@ -200,6 +210,12 @@ SSA_API size_t ssa_workspace_size(int32_t op, const ssa_params* p, int32_t S, in
     BwdWs w;
     return carve_bwd(nullptr, p, S, N, B_tot, W_tot, &w) + conv_bytes(p, N, B_tot);
   }
+  // a sequence-parallel rank: N = its tokens, W_tot = its windows
+  if (op == SSA_OP_SP_FORWARD) return fwd_bytes(p, S, N, B_tot, W_tot) + sp_fwd_extra(p, W_tot);
+  if (op == SSA_OP_SP_BACKWARD) {
+    BwdWs w;
+    return carve_bwd(nullptr, p, S, N, B_tot, W_tot, &w) + sp_bwd_extra(p, N);
+  }
   // cross attention: N = query tokens, W_tot unused (no window branch)
   if (op == SSA_OP_CROSS_FORWARD) return fwd_bytes(p, S, N, B_tot, 0) + cross_extra_bytes(N, p->hq);
   if (op == SSA_OP_CROSS_BACKWARD) {
@@ -221,6 +237,18 @@ SSA_API ssa_status ssa_geo_select(const int32_t* coords, const int32_t* cu_seqle
   if (ws_bytes < ssa::geo_ws_bytes(N)) return SSA_ERR_WORKSPACE;
   return cuda_status(ssa::geo_select(coords, cu_seqlens, S, N, blk, m_cmp, topk, hkv, sel, ws,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+SSA_API ssa_status ssa_diag_wait_timeout(int32_t* gave_up, void* stream) {
+  if (!gave_up) return SSA_ERR_INVALID_ARG;
+  int* sp = status_ptr();
+  if (!sp) return SSA_ERR_CUDA;
+  return cuda_status(ssa::diag_wait_timeout(sp, gave_up, static_cast<cudaStream_t>(stream)));
+}
+
+SSA_API ssa_status ssa_diag_ex2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_mufu))) return SSA_ERR_INVALID_ARG;
+  return cuda_status(ssa::diag_ex2(x, y_poly, y_mufu, n, static_cast<cudaStream_t>(stream)));
 }
 
 SSA_API ssa_status ssa_get_device_status(void* stream) {
@@ -315,7 +343,7 @@ namespace {
 ssa_status forward_common(const ssa_params* p, const int32_t* cu, int32_t S, int64_t N, int64_t Nkv, int cross,
                           const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
                           const void* v, const float* gates, void* out, const ssa_saved* saved, void* ws,
-                          cudaStream_t st) {
+                          cudaStream_t st, const ssa_sp_local* sp = nullptr) {
   cudaError_t e = ssa::launch_pool(p->dtype, k, v, blk, Nkv, p->hkv, p->d, saved->ks, saved->vs, saved->kc,
                                    saved->vc, st);
   if (e != cudaSuccess) return SSA_ERR_CUDA;
@@ -357,18 +385,38 @@ ssa_status forward_common(const ssa_params* p, const int32_t* cu, int32_t S, int
   a.o_branch = saved->o_branch;
   a.lse = saved->lse;
   a.sel = saved->sel;
+  a.has_win = !cross;
+  a.wk = k;
+  a.wv = v;
+  a.wks = saved->ks;
+  a.wvs = saved->vs;
   Carver c(ws);
   carve_plan(c, S, &a.tiles_cnt, &a.tiles_pre, &a.items_cnt, &a.items_pre, &a.scan_tmp);
   int32_t* win_scan = nullptr;
   fwd_bytes(p, S, N, blk->count, win ? win->count : 0, &a.imp_scratch, &a.win_cnt, &a.win_pre, &win_scan, ws);
   a.win_scan = win_scan;
+  if (sp) {  // a sequence-parallel rank: the window problem is its own tokens
+    a.has_win = 1;
+    a.win = sp->win;
+    a.wk = sp->k;
+    a.wv = sp->v;
+    a.wks = sp->ks;
+    a.wvs = sp->vs;
+    // their window-ordered copies (the window means land in the scratch after the workspace)
+    char* wsc = static_cast<char*>(ws) + fwd_bytes(p, S, N, blk->count, sp->win->count);
+    void* wkc = wsc;
+    void* wvc = wsc + align256((size_t)p->hkv * sp->win->count * p->d * (p->dtype == SSA_DTYPE_BF16 ? 2 : 4));
+    e = ssa::launch_pool(p->dtype, sp->k, sp->v, sp->win, N, p->hkv, p->d, sp->ks, sp->vs, wkc, wvc, st);
+    if (e != cudaSuccess) return SSA_ERR_CUDA;
+  }
   return cuda_status(ssa::simt_forward(a, st));
 }
 
 ssa_status backward_common(const ssa_params* p, const int32_t* cu, int32_t S, int64_t N, int64_t Nkv, int cross,
                            const ssa_partition* blk, const ssa_partition* win, const void* q, const void* k,
                            const void* v, const float* gates, const ssa_saved* saved, const void* dout, float* dq,
-                           float* dk, float* dv, float* dgates, void* ws, cudaStream_t st) {
+                           float* dk, float* dv, float* dgates, void* ws, cudaStream_t st,
+                           const ssa_sp_local* sp = nullptr, float* sp_wdk = nullptr, float* sp_wdv = nullptr) {
   BwdWs w;
   const size_t used = carve_bwd(ws, p, S, N, blk->count, win ? win->count : 0, &w);
   ssa::ConvArgs conv;
@@ -429,6 +477,25 @@ ssa_status backward_common(const ssa_params* p, const int32_t* cu, int32_t S, in
   a.items_cnt = w.ic;
   a.items_pre = w.ip;
   a.scan_tmp = w.st;
+  a.has_win = !cross;
+  a.wk = k;
+  a.wv = v;
+  a.wks = saved->ks;
+  a.wvs = saved->vs;
+  a.wdk = dk;
+  a.wdv = dv;
+  a.wtok = nullptr;
+  if (sp) {  // a sequence-parallel rank: the window problem is its own tokens
+    a.has_win = 1;
+    a.wk = sp->k;
+    a.wv = sp->v;
+    a.wks = sp->ks;
+    a.wvs = sp->vs;
+    a.win = sp->win;
+    a.wdk = sp_wdk;
+    a.wdv = sp_wdv;
+    a.wtok = sp->tokens;
+  }
   return cuda_status(ssa::simt_backward(a, st));
 }
 
@@ -546,6 +613,71 @@ SSA_API ssa_status ssa_cross_backward(const ssa_params* p, const int32_t* q_cu, 
   if (ps != SSA_OK) return ps;
   return backward_common(p, q_cu, S, Nq, Nkv, 1, blk, nullptr, q, k, v, gates3, saved, dout, dq, dk, dv, dgates,
                          ws, st);
+}
+
+
+}  // extern "C"
+
+namespace {
+
+ssa_status sp_check(const ssa_params* p, int32_t S, int64_t N, const ssa_partition* blk, const ssa_sp_local* loc) {
+  ssa_status ps = check_params(p);
+  if (ps != SSA_OK) return ps;
+  if (p->conv) return SSA_ERR_INVALID_ARG;  // the learned compression is built for the whole-sequence call
+  if (p->m_cmp % p->m_win != 0) return SSA_ERR_INVALID_ARG;  // a window must lie inside one block
+  if (S < 1 || N < 1 || N > INT32_MAX - 1 || !loc || loc->n < 0 || loc->n > N || !partition_ok(blk, N))
+    return SSA_ERR_INVALID_ARG;
+  if (!loc->cu_seqlens || !partition_ok(loc->win, loc->n)) return SSA_ERR_INVALID_ARG;
+  if (loc->n > 0 && (!loc->tokens || !loc->k || !loc->v || !loc->ks || !loc->vs)) return SSA_ERR_INVALID_ARG;
+  if (blk->count < 1 || blk->count > N || loc->win->count > loc->n) return SSA_ERR_INVALID_ARG;
+  return SSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+SSA_API ssa_status ssa_sp_forward(const ssa_params* p, int32_t S, int64_t N, const ssa_partition* blk,
+                                  const ssa_sp_local* loc, const void* q, const void* k, const void* v,
+                                  const float* gates, void* out, const ssa_saved* saved, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  ssa_status ps = sp_check(p, S, N, blk, loc);
+  if (ps != SSA_OK) return ps;
+  const int64_t nr = loc->n;
+  if (nr == 0) return SSA_OK;
+  if (!q || !k || !v || !gates || !out || !saved_ok(saved) || !ws) return SSA_ERR_INVALID_ARG;
+  if (ws_bytes < fwd_bytes(p, S, nr, blk->count, loc->win->count) + sp_fwd_extra(p, loc->win->count))
+    return SSA_ERR_WORKSPACE;
+  return forward_common(p, loc->cu_seqlens, S, nr, N, 1, blk, nullptr, q, k, v, gates, out, saved, ws,
+                        static_cast<cudaStream_t>(stream), loc);
+}
+
+SSA_API ssa_status ssa_sp_backward(const ssa_params* p, int32_t S, int64_t N, const ssa_partition* blk,
+                                   const ssa_sp_local* loc, const void* q, const void* k, const void* v,
+                                   const float* gates, const ssa_saved* saved, const void* dout, float* dq,
+                                   float* dk, float* dv, float* dgates, void* ws, size_t ws_bytes, void* stream) {
+  ssa_status ps = sp_check(p, S, N, blk, loc);
+  if (ps != SSA_OK) return ps;
+  const int64_t nr = loc->n;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (nr == 0) {  // no query rows here: this rank contributes nothing to any key gradient
+    if (!dk || !dv) return SSA_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(dk, 0, sizeof(float) * N * p->hkv * p->d, st) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, sizeof(float) * N * p->hkv * p->d, st) != cudaSuccess)
+      return SSA_ERR_CUDA;
+    return SSA_OK;
+  }
+  if (!q || !k || !v || !gates || !dout || !dq || !dk || !dv || !dgates || !saved_ok(saved) || !ws)
+    return SSA_ERR_INVALID_ARG;
+  if (nr * p->hkv * p->topk > INT32_MAX) return SSA_ERR_UNSUPPORTED;
+  BwdWs w;
+  const size_t base = carve_bwd(nullptr, p, S, nr, blk->count, loc->win->count, &w);
+  if (ws_bytes < base + sp_bwd_extra(p, nr)) return SSA_ERR_WORKSPACE;
+  char* extra = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + base + 255) & ~uintptr_t(255));
+  float* wdk = reinterpret_cast<float*>(extra);
+  float* wdv = reinterpret_cast<float*>(extra + align256(sizeof(float) * (size_t)nr * p->hkv * p->d));
+  return backward_common(p, loc->cu_seqlens, S, nr, N, 1, blk, nullptr, q, k, v, gates, saved, dout, dq, dk, dv,
+                         dgates, ws, st, loc, wdk, wdv);
 }
 
 }  // extern "C"

@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(128) win_fwd_kernel(const T* __restrict__ q, c
                                                       const int32_t* __restrict__ wptr, int64_t wtot, int hq, int hkv,
                                                       float qs2, float* __restrict__ o_out, float* __restrict__ lse_out) {
   using C = Cfg<D>;
-  constexpr int KT = 64;
+  constexpr int KT = D >= 128 ? 32 : 64;  // staged keys per chunk (two chunks of K and V fit 48 KB)
   __shared__ __align__(16) float sk[KT * C::KSTR];
   __shared__ __align__(16) float sv[KT * C::KSTR];
   const int g = blockIdx.y, G = hq / hkv;
@@ -771,14 +771,16 @@ __global__ void __launch_bounds__(128) slc_bwd_dq_kernel(
 // dk/dv are reduced over row slices in shared memory and added to dK/dV (zeroed
 // beforehand) with fp32 atomics.
 constexpr int kSlcRowChunk = 1024;
-constexpr int kSlcStageRows = 64;
+// staged query rows per pass (the q / dO stages of head dim 128 would not fit 48 KB at 64)
+template <int D>
+constexpr int slc_stage_rows() { return D >= 128 ? 32 : 64; }
 
 template <typename T, int D>
 struct SlcStage {
-  float q[kSlcStageRows * Cfg<D>::KSTR];
-  float dO[kSlcStageRows * Cfg<D>::KSTR];
-  float lse2[kSlcStageRows];
-  float Dr[kSlcStageRows];
+  float q[slc_stage_rows<D>() * Cfg<D>::KSTR];
+  float dO[slc_stage_rows<D>() * Cfg<D>::KSTR];
+  float lse2[slc_stage_rows<D>()];
+  float Dr[slc_stage_rows<D>()];
 };
 
 __global__ void slc_items_kernel(const int32_t* __restrict__ inv_ptr, int64_t nkeys, int G, int32_t* __restrict__ cnt) {
@@ -802,7 +804,8 @@ __global__ void __launch_bounds__(128) slc_bwd_dkv_kernel(
   constexpr int NT = D / 32;
   constexpr int SLOTS = 128 / NT;  // (key slot, row slice) pairs
   __shared__ __align__(16) SlcStage<T, D> st;
-  constexpr int KMAX = 64;  // key slots per pass (the reduction buffers hold KMAX * D floats each)
+  constexpr int kSlcStageRows = slc_stage_rows<D>();
+  constexpr int KMAX = D >= 128 ? 32 : 64;  // key slots per pass (the reduction buffers hold KMAX * D floats each)
   static_assert(kSlcStageRows * Cfg<D>::KSTR >= KMAX * D, "reduction buffers must fit in the staging area");
   const int G = hq / hkv;
   const int sub = threadIdx.x % NT;
@@ -1233,6 +1236,23 @@ __global__ void keys_to_ptr_kernel(const uint64_t* __restrict__ keys, int64_t n,
 }
 
 // per-sequence work counts for the tiled kernels
+// dst[rows[i]] += src[i] for rows of `w4` float4 (dK and dV at once); the rows are distinct.
+__global__ void rows_add_kernel(const float* __restrict__ srck, const float* __restrict__ srcv,
+                                const int32_t* __restrict__ rows, int64_t n, int w4, float* __restrict__ dstk,
+                                float* __restrict__ dstv) {
+  const int64_t total = n * w4;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / w4, c = i % w4;
+    const int64_t d = (int64_t)rows[r] * w4 + c;
+    const float4 a = reinterpret_cast<const float4*>(srck)[i], b = reinterpret_cast<const float4*>(srcv)[i];
+    float4 x = reinterpret_cast<float4*>(dstk)[d], y = reinterpret_cast<float4*>(dstv)[d];
+    x.x += a.x; x.y += a.y; x.z += a.z; x.w += a.w;
+    y.x += b.x; y.y += b.y; y.z += b.z; y.w += b.w;
+    reinterpret_cast<float4*>(dstk)[d] = x;
+    reinterpret_cast<float4*>(dstv)[d] = y;
+  }
+}
+
 __global__ void plan_counts_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, int S, int G,
                                    int rows_per_tile, int blocks_per_item, int rc_rows, int32_t* __restrict__ tiles,
                                    int32_t* __restrict__ items) {
@@ -1300,18 +1320,18 @@ cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
                q, static_cast<const T*>(a.ks), static_cast<const T*>(a.vs), a.blk->ptr, a.sel, a.N, a.Nkv, a.hq,
                a.hkv, a.topk, qs2, ob + rows * D, a.lse + rows);
   }
-  if (!a.cross) {  // cross attention has no window branch (the queries have no voxel)
+  if (a.has_win) {  // cross attention has no window branch (the queries have no voxel)
     const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
     if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
       e = win_fwd_tc(a, a.win_cnt, a.win_pre, a.win_scan, st);
       if (e != cudaSuccess) return e;
     } else
-      SSA_LAUNCH("win_fwd_kernel", (win_fwd_kernel<T, D>), gw, 128, 0, st, q, static_cast<const T*>(a.k),
-                 static_cast<const T*>(a.v), a.win->perm, a.win->ptr, a.win->count, a.hq, a.hkv, qs2,
+      SSA_LAUNCH("win_fwd_kernel", (win_fwd_kernel<T, D>), gw, 128, 0, st, q, static_cast<const T*>(a.wk),
+                 static_cast<const T*>(a.wv), a.win->perm, a.win->ptr, a.win->count, a.hq, a.hkv, qs2,
                  ob + 2 * rows * D, a.lse + 2 * rows);
   }
   SSA_LAUNCH("combine_kernel", (combine_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, a.gates,
-             rows, a.gate_mode, a.cross ? 2 : 3, static_cast<T*>(a.out));
+             rows, a.gate_mode, a.has_win ? 3 : 2, static_cast<T*>(a.out));
   return cudaGetLastError();
 }
 
@@ -1340,7 +1360,7 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
 
   SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout,
-             a.gates, a.lse, rows, a.gate_mode, a.cross ? 2 : 3, a.Dc, a.dgates, a.rc);
+             a.gates, a.lse, rows, a.gate_mode, a.has_win ? 3 : 2, a.Dc, a.dgates, a.rc);
   if (a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
     // 128-row tiles for the tensor-core kernels (tiles_cnt / tiles_pre are free again here)
     SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu,
@@ -1405,24 +1425,33 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                a.gate_mode, a.blk->ptr, a.blk->perm, a.inv_ptr, sv, a.slc_pre, a.Nkv, btot, a.hq, a.hkv, qs2, a.scale,
                a.lse + rows, a.Dc + rows, a.dk, a.dv);
   }
-  if (a.cross) {
-    // no window branch
-  } else if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
-    e = win_bwd_tc(a, a.win_cnt, a.win_pre, a.scan_tmp, st);
-    if (e != cudaSuccess) return e;
-  } else {
-    const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
-    SSA_LAUNCH("win_bwd_dq_kernel", (win_bwd_dq_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
-                                                a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
-                                                a.Dc + 2 * rows, a.dq);
-    SSA_LAUNCH("win_bwd_dkv_kernel", (win_bwd_dkv_kernel<T, D>), gw, 128, 0, st, q, k, v, dout, a.gates, a.gate_mode, a.win->perm, a.win->ptr,
-                                                 a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
-                                                 a.Dc + 2 * rows, a.dk, a.dv);
+  if (a.has_win) {
+    if (a.wtok) {  // a rank's window gradients go to a local buffer first
+      cudaMemsetAsync(a.wdk, 0, sizeof(float) * a.N * a.hkv * D, st);
+      cudaMemsetAsync(a.wdv, 0, sizeof(float) * a.N * a.hkv * D, st);
+    }
+    if (a.use_tc && D == 64 && win_tc_supported(a.dtype, D, a.hq, a.hkv, a.m_cmp, a.m_win)) {
+      e = win_bwd_tc(a, a.win_cnt, a.win_pre, a.scan_tmp, st);
+      if (e != cudaSuccess) return e;
+    } else {
+      const T* wk = static_cast<const T*>(a.wk);
+      const T* wv = static_cast<const T*>(a.wv);
+      const dim3 gw(grid_1d(a.win->count, 1, 148 * 16), a.hkv);
+      SSA_LAUNCH("win_bwd_dq_kernel", (win_bwd_dq_kernel<T, D>), gw, 128, 0, st, q, wk, wv, dout, a.gates,
+                 a.gate_mode, a.win->perm, a.win->ptr, a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
+                 a.Dc + 2 * rows, a.dq);
+      SSA_LAUNCH("win_bwd_dkv_kernel", (win_bwd_dkv_kernel<T, D>), gw, 128, 0, st, q, wk, wv, dout, a.gates,
+                 a.gate_mode, a.win->perm, a.win->ptr, a.win->count, a.hq, a.hkv, qs2, a.scale, a.lse + 2 * rows,
+                 a.Dc + 2 * rows, a.wdk, a.wdv);
+    }
   }
   if (a.conv)  // the learned compression: dK, dV through the convolution, dW, db
     return conv_backward(*a.conv, a.dtype, a.k, a.v, a.dkc, a.dvc, a.dk, a.dv, st);
   SSA_LAUNCH("cmp_scatter_kernel", cmp_scatter_kernel, grid_1d(a.Nkv * a.hkv * D / 4, 256, 148 * 32), 256, 0, st,
              a.dkc, a.dvc, a.blk->id, a.blk->ptr, a.Nkv, btot, a.hkv, D, a.dk, a.dv);
+  if (a.has_win && a.wtok)  // a rank's window gradients into the rows of its tokens
+    SSA_LAUNCH("rows_add_kernel", rows_add_kernel, grid_1d(a.N * a.hkv * D / 4, 256, 148 * 32), 256, 0, st, a.wdk,
+               a.wdv, a.wtok, a.N, a.hkv * D / 4, a.dk, a.dv);
   return cudaGetLastError();
 }
 
@@ -1439,9 +1468,11 @@ cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st) {
   if (a.dtype == SSA_DTYPE_BF16) {
     if (a.d == 32) return forward_impl<__nv_bfloat16, 32>(a, st);
     if (a.d == 64) return forward_impl<__nv_bfloat16, 64>(a, st);
+    if (a.d == 128) return forward_impl<__nv_bfloat16, 128>(a, st);
   } else {
     if (a.d == 32) return forward_impl<float, 32>(a, st);
     if (a.d == 64) return forward_impl<float, 64>(a, st);
+    if (a.d == 128) return forward_impl<float, 128>(a, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -1450,9 +1481,11 @@ cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st) {
   if (a.dtype == SSA_DTYPE_BF16) {
     if (a.d == 32) return backward_impl<__nv_bfloat16, 32>(a, st);
     if (a.d == 64) return backward_impl<__nv_bfloat16, 64>(a, st);
+    if (a.d == 128) return backward_impl<__nv_bfloat16, 128>(a, st);
   } else {
     if (a.d == 32) return backward_impl<float, 32>(a, st);
     if (a.d == 64) return backward_impl<float, 64>(a, st);
+    if (a.d == 128) return backward_impl<float, 128>(a, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -10,18 +10,17 @@
 // loaded by one 3D TMA box from Q [N, Hq, 64].  A key tile is 128 compressed
 // blocks of Kc/Vc [Hkv, B, 64] (2D TMA, 128-byte swizzle).
 //
-//   pass 1 (cmp_lse_tc):  S = Q Kc^T in TMEM, one thread per row keeps the
-//                         online max / sum of exp2 -> lse.
-//   pass 2 (cmp_out_tc):  S^T = Kc Q^T (one thread per block), p = exp2(s - lse)
-//                         with the final lse; the block's score for a token is
-//                         the sum of its G heads' p (registers); P^T goes to
-//                         shared memory as the MN-major A operand of
-//                         O += P Vc (TMEM accumulator); per-token top-k by
-//                         threshold filtering + insertion.
+//   output pass (cmp_fa_tc):     flash attention, thread = row: S = Q Kc^T, online
+//                                softmax, P (bf16 high + low) back into TMEM as the
+//                                operand of O += P Vc -> o_cmp and lse.
+//   selection pass (cmp_sel_tc): S^T = Kc Q^T, thread = block: p = exp2(s - lse)
+//                                with the final lse, summed over the G heads of a
+//                                token; a warpgroup picks each token's top-k.
+//   backward (cmp_bwd_dq_tc, cmp_bwd_dkv_tc): dQ by rows, dKc / dVc by blocks.
 //
-// Roles per CTA: warps 0-3 compute (thread i <-> TMEM lane i), warp 4 issues
-// TMA loads, warp 5 issues tcgen05.mma.  Every wait is bounded; on a timeout the
-// kernel records kStatusTimeout, drains what it issued (bounded) and exits.
+// Roles per CTA: compute warps (thread i <-> TMEM lane i), one warp issuing TMA
+// loads, one issuing tcgen05.mma.  Every wait is bounded; on a timeout the kernel
+// records kStatusTimeout, drains what it issued (bounded) and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -41,9 +40,6 @@ using namespace tch;
 
 constexpr int kBN = 128;             // compressed blocks per key tile
 constexpr int kTile = 128 * 128;     // bytes of a 128 x 64 bf16 tile
-constexpr int kStages = 4;           // key-tile ring depth
-constexpr int kPolyCols = 32;        // columns of a key tile whose exponentials pass 1 evaluates without the MUFU (1/4; measured best of 32-80)
-constexpr int kThreads = 192;        // 4 compute warps + TMA warp + MMA warp
 
 struct TileInfo {
   int g, s, t0, t_end, b0, nb;
@@ -72,180 +68,9 @@ __device__ __forceinline__ bool aborted(const int* abort_flag) {
 }
 
 // ---------------------------------------------------------------------------
-// pass 1: lse
-// ---------------------------------------------------------------------------
-struct LseSmem {
-  uint8_t q[2][kTile];
-  uint8_t kc[kStages][kTile];
-  uint64_t q_full[2], q_empty[2], mma_done;
-  uint64_t kc_full[kStages], kc_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
-  uint32_t tmem;
-  int abort_flag;
-};
-
-__global__ void __launch_bounds__(kThreads, 2) cmp_lse_tc_kernel(
-    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap, const int32_t* __restrict__ cu,
-    const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S, int hq, int hkv, int btot, float qs2,
-    float* __restrict__ lse_out, int* status) {
-  extern __shared__ uint8_t smem_raw[];
-  LseSmem& sm = *reinterpret_cast<LseSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int G = hq / hkv;
-  const int ntiles = tpre[S];
-  const int total = ntiles * hkv;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.q_full[i], 1);
-      mbar_init(&sm.q_empty[i], 1);
-    }
-    mbar_init(&sm.mma_done, 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sm.kc_full[i], 1);
-      mbar_init(&sm.kc_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_empty[i], 4);
-    }
-    sm.abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(&sm.tmem, 256);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm.tmem;
-
-  if (warp == 4) {
-    // ---------------- TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&qmap);
-      prefetch_tmap(&kcmap);
-      uint32_t kc_count = 0, q_count = 0;
-      int last_par[kStages];
-      for (int i = 0; i < kStages; ++i) last_par[i] = -1;
-      for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
-        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
-        const int qb = q_count % 2;
-        if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
-        mbar_expect_tx(&sm.q_full[qb], kTile);
-        tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
-        ++q_count;
-        const int nbt = (ti.nb + kBN - 1) / kBN;
-        for (int j = 0; j < nbt; ++j) {
-          const int st = kc_count % kStages;
-          const uint32_t ph = (kc_count / kStages) & 1;
-          if (!mbar_wait(&sm.kc_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
-          mbar_expect_tx(&sm.kc_full[st], kTile);
-          tma_load_2d(sm.kc[st], &kcmap, &sm.kc_full[st], 0, ti.g * btot + ti.b0 + j * kBN);
-          last_par[st] = (int)ph;
-          ++kc_count;
-        }
-      }
-      // drain: every issued load has landed before the CTA may exit
-      for (int i = 0; i < kStages; ++i)
-        if (last_par[i] >= 0) mbar_wait(&sm.kc_full[i], (uint32_t)last_par[i]);
-    }
-  } else if (warp == 5) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(kRows, kBN);
-      uint32_t kc_count = 0, q_count = 0, s_count = 0;
-      for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
-        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
-        const int qb = q_count % 2;
-        if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { record_timeout(status, &sm.abort_flag); break; }
-        ++q_count;
-        const int nbt = (ti.nb + kBN - 1) / kBN;
-        bool ok = true;
-        for (int j = 0; j < nbt; ++j) {
-          const int st = kc_count % kStages;
-          const int sb = s_count % 2;
-          if (!mbar_wait(&sm.kc_full[st], (kc_count / kStages) & 1) ||
-              !mbar_wait(&sm.s_empty[sb], ((s_count / 2) & 1) ^ 1)) {
-            record_timeout(status, &sm.abort_flag);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(tmem + sb * kBN, sdesc_kmajor_sw128(sm.q[qb], 32 * k), sdesc_kmajor_sw128(sm.kc[st], 32 * k),
-                        idesc, k > 0);
-          mma_commit(&sm.s_full[sb]);
-          mma_commit(&sm.kc_empty[st]);
-          ++kc_count;
-          ++s_count;
-        }
-        mma_commit(&sm.q_empty[qb]);
-        if (!ok) break;
-      }
-      mma_commit(&sm.mma_done);
-      mbar_wait(&sm.mma_done, 0);
-    }
-  } else {
-    // ---------------- compute warps: thread = row
-    const int r = threadIdx.x;  // 0..127
-    uint32_t s_count = 0;
-    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
-      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
-      const int64_t t = ti.t0 + r / G;
-      const int h = ti.g * G + r % G;
-      const bool valid = t < ti.t_end;
-      float m = -CUDART_INF_F, l = 0.f;
-      const int nbt = (ti.nb + kBN - 1) / kBN;
-      bool ok = true;
-      for (int j = 0; j < nbt; ++j) {
-        const int sb = s_count % 2;
-        if (!mbar_wait_warp(&sm.s_full[sb], (s_count / 2) & 1)) { record_timeout(status, &sm.abort_flag); ok = false; break; }
-        tc_fence_after();
-        float sv[kBN];
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + sb * kBN;
-#pragma unroll
-        for (int c = 0; c < kBN; c += 32) tmem_ld32(taddr + c, sv + c);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
-        ++s_count;
-        const int vc = min(kBN, ti.nb - j * kBN);
-        if (vc < kBN) {  // ragged last key tile
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) sv[c] = c < vc ? sv[c] : -CUDART_INF_F;
-        }
-        float cm = sv[0];
-#pragma unroll
-        for (int c = 1; c < kBN; ++c) cm = fmaxf(cm, sv[c]);
-        const float mn = fmaxf(m, cm * qs2);  // qs2 > 0
-        const float2 qs = make_float2(qs2, qs2), nm = make_float2(-mn, -mn);
-        // the MUFU bounds this pass: a quarter of the exponentials go to the FMA pipe
-        float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < kPolyCols; c += 2)
-          acc2 = fadd2(acc2, ex2_poly2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nm)));
-#pragma unroll
-        for (int c = kPolyCols; c < kBN; c += 2) acc = fadd2(acc, ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nm)));
-        l = l * ex2(m - mn) + ((acc.x + acc.y) + (acc2.x + acc2.y));
-        m = mn;
-      }
-      if (!ok) break;
-      if (valid) lse_out[t * hq + h] = (m + log2f(l)) * kLn2;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
-}
-
-// ---------------------------------------------------------------------------
 // pass 2: output + top-k (transposed: thread = block)
 // ---------------------------------------------------------------------------
 constexpr int kTopkMax = 32;
-constexpr int kOutStages = 3;
 constexpr int kCandMax = 128;  // top-k candidates per token kept for exact ranking
 constexpr int kComputeWarps = 8;  // pass 2: two warpgroups of compute warps
 // pass 2 adds a warpgroup that picks the top-k of the previous row tile while the
@@ -254,22 +79,6 @@ constexpr int kOutTopkWarps = 4;
 constexpr int kOutTmaWarp = kComputeWarps + kOutTopkWarps;
 constexpr int kOutMmaWarp = kOutTmaWarp + 1;
 constexpr int kOutThreadsTk = 32 * (kOutMmaWarp + 1);
-
-struct OutSmem {
-  uint8_t q[2][kTile];
-  uint8_t kc[kOutStages][kTile];
-  uint8_t vc[kOutStages][kTile];
-  uint8_t pt_hi[2 * kTile];  // P^T (bf16 high part) as the MN-major A operand: [2 row atoms][128 blocks][64 rows]
-  uint8_t pt_lo[2 * kTile];  // p - bf16(p), same layout: O += (P_hi + P_lo) Vc keeps fp32-level accuracy
-  __align__(16) float lse2[2][kRows];  // -lse log2(e) of the tile's rows, double-buffered by tile
-  float candv[kOutTopkWarps][kCandMax];
-  int candi[kOutTopkWarps][kCandMax];
-  uint64_t q_full[2], q_empty[2], mma_done, o_full, o_empty, cw, imp_full[2], imp_empty[2];
-  uint64_t kv_full[kOutStages], kv_empty[kOutStages];
-  uint64_t s_full, s_empty, pt_full, pt_empty;
-  uint32_t tmem;
-  int abort_flag;
-};
 
 // Store rows [8c, 8c+8) of block `b` into a P^T tile (MN-major A operand,
 // 128-byte swizzle): row atom a = row / 64 holds 64 rows of one block in a
@@ -531,45 +340,40 @@ __device__ void warp_topk_fast(const float* imp, int nb, int topk, int b0, int32
   __syncwarp();
 }
 
-// Exact top-k as warp_topk_fast for nb <= 256 * NF4, built for short dependency
-// chains: the scores are read in two batches of NF4 float4 per lane (each batch's
-// loads in flight together) for the lane bests, then read again (mostly L1 hits)
-// while candidates are compacted with warp votes, skipping the 4-entry groups that
-// hold none (typically all but a few).
-template <int NF4>
-__device__ __forceinline__ void load_batch(const float* imp, int nb, int base, int lane, float4* v) {
-#pragma unroll
-  for (int u = 0; u < NF4; ++u) {
-    const int i0 = base + 128 * u + 4 * lane;
-    if (i0 + 3 < nb) {
-      v[u] = *reinterpret_cast<const float4*>(imp + i0);
-    } else {
-      v[u].x = i0 + 0 < nb ? imp[i0 + 0] : -CUDART_INF_F;
-      v[u].y = i0 + 1 < nb ? imp[i0 + 1] : -CUDART_INF_F;
-      v[u].z = i0 + 2 < nb ? imp[i0 + 2] : -CUDART_INF_F;
-      v[u].w = -CUDART_INF_F;
-    }
-  }
-}
-template <int NF4, int KL>
-__device__ void warp_topk_regs(const float* imp, int nb, int topk, int b0, int32_t* __restrict__ out, float* cv,
-                               int* ci) {
+
+// Exact top-k of imp[0..nb) (the same result as warp_topk) from the scores and their
+// group maxima gm[0..ceil(nb/32)) (gm[i] = max of imp[32 i .. 32 i + 31]; scores are
+// sums of probabilities, never negative):
+//  1. each lane's best group maximum (lane l holds groups l, l + 32, ...);
+//  2. tau = the keff-th best of the 32 lane bests: they are scores of keff distinct
+//     blocks, so every top-keff score is >= tau;
+//  3. only groups whose maximum is >= tau can hold such scores: their members >= tau
+//     are collected (32 loads of a group in one coalesced access) and ranked exactly.
+// Falls back to warp_topk_fast over all scores for sequences of more than 4096 blocks,
+// when fewer than keff lanes hold a group, or when more than kCandMax scores reach tau.
+constexpr int kGrpPerLane = 4;
+constexpr int kGrpBatch = 8;  // candidate groups loaded together
+template <int KL>
+__device__ void warp_topk_groups(const float* imp, const float* gm, int nb, int topk, int b0,
+                                 int32_t* __restrict__ out, float* cv, int* ci, int* cg) {
   const int lane = threadIdx.x & 31;
   const int keff = min(topk, nb);
-  // 1. lane best (ties to the lower index); entries past nb are -inf and never win
-  float bv = -CUDART_INF_F;
+  const int ng = (nb + 31) / 32;
+  if (keff > 32 || ng > 32 * kGrpPerLane) {
+    warp_topk_fast<KL>(imp, nb, topk, b0, out, cv, ci);
+    return;
+  }
+  // 1. lane bests over the group maxima (absent groups read as -1, below every score)
+  float gv[kGrpPerLane];
+  float bv = -1.f;
   int bi = 0x7fffffff;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float4 v[NF4];
-    load_batch<NF4>(imp, nb, h * 128 * NF4, lane, v);
-#pragma unroll
-    for (int u = 0; u < NF4; ++u) {
-      const int i0 = h * 128 * NF4 + 128 * u + 4 * lane;
-      if (i0 < nb && v[u].x > bv) { bv = v[u].x; bi = i0; }
-      if (i0 + 1 < nb && v[u].y > bv) { bv = v[u].y; bi = i0 + 1; }
-      if (i0 + 2 < nb && v[u].z > bv) { bv = v[u].z; bi = i0 + 2; }
-      if (i0 + 3 < nb && v[u].w > bv) { bv = v[u].w; bi = i0 + 3; }
+  for (int u = 0; u < kGrpPerLane; ++u) {
+    const int i = lane + 32 * u;
+    gv[u] = i < ng ? gm[i] : -1.f;
+    if (gv[u] > bv) {
+      bv = gv[u];
+      bi = i;
     }
   }
   // 2. tau = the lane best of rank keff - 1 among the 32
@@ -580,46 +384,50 @@ __device__ void warp_topk_regs(const float* imp, int nb, int topk, int b0, int32
     const int i2 = __shfl_sync(0xffffffffu, bi, o);
     if (beats(v2, i2, bv, bi)) ++rank;
   }
-  const unsigned own = __ballot_sync(0xffffffffu, rank == keff - 1);
-  if (keff > 32 || own == 0u) {
-    warp_topk<KL>(imp, nb, topk, b0, out);
+  const unsigned own = __ballot_sync(0xffffffffu, rank == keff - 1 && bv >= 0.f);
+  if (own == 0u) {  // fewer than keff lanes hold a group
+    warp_topk_fast<KL>(imp, nb, topk, b0, out, cv, ci);
     return;
   }
-  const int src = __ffs(own) - 1;
-  const float tv = __shfl_sync(0xffffffffu, bv, src);
-  const int ti = __shfl_sync(0xffffffffu, bi, src);
-  // 3. entries at or above (tv, ti), compacted in index order by warp votes
+  const float tv = __shfl_sync(0xffffffffu, bv, __ffs(own) - 1);
+  // 3. candidate groups (maximum >= tau), compacted in index order
   const unsigned lt = (1u << lane) - 1u;
+  int ncg = 0;
+#pragma unroll
+  for (int u = 0; u < kGrpPerLane; ++u) {
+    const bool c = gv[u] >= tv;
+    const unsigned m = __ballot_sync(0xffffffffu, c);
+    if (c) cg[ncg + __popc(m & lt)] = lane + 32 * u;
+    ncg += __popc(m);
+  }
+  __syncwarp();
+  // their members >= tau, in index order
   int n = 0;
+  for (int c0 = 0; c0 < ncg; c0 += kGrpBatch) {
+    float x[kGrpBatch];
+    int id[kGrpBatch];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float4 v[NF4];
-    load_batch<NF4>(imp, nb, h * 128 * NF4, lane, v);
+    for (int k = 0; k < kGrpBatch; ++k) {
+      id[k] = c0 + k < ncg ? 32 * cg[c0 + k] + lane : nb;
+      x[k] = id[k] < nb ? imp[id[k]] : -1.f;
+    }
 #pragma unroll
-    for (int u = 0; u < NF4; ++u) {
-      const int i0 = h * 128 * NF4 + 128 * u + 4 * lane;
-      const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      bool tk[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) tk[e] = i0 + e < nb && (xs[e] == tv ? i0 + e <= ti : xs[e] > tv);
-      if (__ballot_sync(0xffffffffu, tk[0] || tk[1] || tk[2] || tk[3]) == 0u) continue;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const unsigned m = __ballot_sync(0xffffffffu, tk[e]);
-        if (tk[e]) {
-          const int slot = n + __popc(m & lt);
-          if (slot < kCandMax) {
-            cv[slot] = xs[e];
-            ci[slot] = i0 + e;
-          }
+    for (int k = 0; k < kGrpBatch; ++k) {
+      const bool keep = id[k] < nb && x[k] >= tv;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const int slot = n + __popc(m & lt);
+        if (slot < kCandMax) {
+          cv[slot] = x[k];
+          ci[slot] = id[k];
         }
-        n += __popc(m);
       }
+      n += __popc(m);
     }
   }
   if (n > kCandMax) {
     __syncwarp();
-    warp_topk<KL>(imp, nb, topk, b0, out);
+    warp_topk_fast<KL>(imp, nb, topk, b0, out, cv, ci);
     return;
   }
   __syncwarp();
@@ -632,12 +440,12 @@ __device__ void warp_topk_regs(const float* imp, int nb, int topk, int b0, int32
     picked[u] = false;
     picked_id[u] = 0x7fffffff;
     if (c < n) {
-      const float x = cv[c];
-      const int id = ci[c];
+      const float xv = cv[c];
+      const int xi = ci[c];
       int r = 0;
-      for (int j = 0; j < n; ++j) r += beats(cv[j], ci[j], x, id) ? 1 : 0;
+      for (int j = 0; j < n; ++j) r += beats(cv[j], ci[j], xv, xi) ? 1 : 0;
       picked[u] = r < keff;
-      picked_id[u] = id;
+      picked_id[u] = xi;
     }
   }
   __syncwarp();
@@ -658,305 +466,334 @@ __device__ void warp_topk_regs(const float* imp, int nb, int topk, int b0, int32
   for (int i = keff + lane; i < topk; i += 32) out[i] = -1;
   __syncwarp();
 }
-constexpr int kTopkRegF4 = 10;  // float4 per lane per batch: two batches cover sequences of up to 2560 blocks
 
+// ---------------------------------------------------------------------------
+// output pass (thread = row): flash attention of every query row over all compressed
+// blocks of its sequence, producing o_cmp and lse.  A work unit is a pair of 128-row
+// Q tiles (A, B) of the same (sequence, group), so each Kc / Vc tile is loaded once
+// for 256 rows.  One warpgroup per Q tile keeps its rows' running max m and sum l
+// (log2 domain, scale folded in); S of a key tile lands in TMEM, p = 2^(s qs2 - m)
+// is written back over S as bf16 high and low parts (quarter q of the tile's blocks:
+// high parts at columns 32q .. 32q+15, low parts at 32q+16 .. 32q+31) and consumed by
+// O += P Vc with P as the TMEM operand.  The next S of the same tile is issued into
+// the same columns after that product in the single MMA stream, which executes in
+// order.  O (TMEM) is rescaled only when a row's max grows by more than 2^8 since it
+// was last fixed, so p stays below 2^8 otherwise; a quarter of the exponentials run on
+// the FMA pipe.  The two tiles' softmax work and their MMAs interleave.
+// ---------------------------------------------------------------------------
+constexpr int kFaStages = 3;                 // Kc / Vc ring depth
+constexpr int kFaSoftmaxWarps = 8;           // warps 0-3: tile A, 4-7: tile B
+constexpr int kFaTmaWarp = kFaSoftmaxWarps;
+constexpr int kFaMmaWarp = kFaSoftmaxWarps + 1;
+constexpr int kFaThreads = 32 * (kFaSoftmaxWarps + 2);
+constexpr int kFaPolyCols = 0;               // columns of a key tile whose exponentials use the FMA pipe
+                                             // (0: this pass is issue-bound, 5.55 ms at 131072 tokens vs 6.19 with 32)
+constexpr float kFaRescaleLog2 = 8.f;
+
+struct FaSmem {
+  uint8_t q[2][2][kTile];  // [buffer][tile A / B]
+  uint8_t kc[kFaStages][kTile];
+  uint8_t vc[kFaStages][kTile];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t kv_full[kFaStages], kv_empty[kFaStages];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem;
+  int abort_flag;
+};
+
+struct PairInfo {
+  int g, s, t0, t_end, b0, nb;  // t0: first token of tile A; tile B starts 128/G tokens later
+};
+
+__device__ __forceinline__ PairInfo pair_info(int it, int npairs, const int32_t* ppre, int S, const int32_t* cu,
+                                              const int32_t* bcu, int G) {
+  PairInfo pi;
+  pi.g = it / npairs;
+  const int pr = it % npairs;
+  pi.s = find_segment(ppre, S, pr);
+  pi.t0 = cu[pi.s] + (pr - ppre[pi.s]) * (2 * kRows / G);
+  pi.t_end = cu[pi.s + 1];
+  pi.b0 = bcu[pi.s];
+  pi.nb = bcu[pi.s + 1] - pi.b0;
+  return pi;
+}
+
+// 320 threads x 200 registers fit the SM's register file
 template <int G>
-__global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_out_tc_kernel(
+__global__ void __maxnreg__(200) cmp_fa_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap,
     const __grid_constant__ CUtensorMap vcmap, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
-    const int32_t* __restrict__ tpre, int S, int hq, int hkv, int btot, float qs2, const float* __restrict__ lse_in,
-    float* __restrict__ o_out, int topk, int32_t* __restrict__ sel, float* __restrict__ imp_scratch,
-    int64_t imp_stride, int* status) {
-  constexpr int TPT = kRows / G;  // tokens per tile
+    const int32_t* __restrict__ ppre, int S, int64_t N, int hq, int hkv, int btot, float qs2,
+    float* __restrict__ o_out, float* __restrict__ lse_out, int* status) {
+  constexpr int TPT = kRows / G;  // tokens per Q tile
   extern __shared__ uint8_t smem_raw[];
-  OutSmem& sm = *reinterpret_cast<OutSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FaSmem& sm = *reinterpret_cast<FaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int ntiles = tpre[S];
-  const int total = ntiles * hkv;
-  // this CTA's scores, two buffers of [TPT tokens][imp_stride blocks]
-  float* imp_cta = imp_scratch + (int64_t)blockIdx.x * 2 * TPT * imp_stride;
+  const int npairs = ppre[S];
+  const int total = npairs * hkv;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.pv_done[i], 1);
+      mbar_init(&sm.o_full[i], 1);
+      mbar_init(&sm.o_empty[i], 4);
     }
-    mbar_init(&sm.mma_done, 1);
-    mbar_init(&sm.o_full, 1);
-    mbar_init(&sm.o_empty, kComputeWarps);
-    mbar_init(&sm.cw, kComputeWarps);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.imp_full[i], kComputeWarps);
-      mbar_init(&sm.imp_empty[i], kOutTopkWarps);
-    }
-    for (int i = 0; i < kOutStages; ++i) {
+    for (int i = 0; i < kFaStages; ++i) {
       mbar_init(&sm.kv_full[i], 1);
       mbar_init(&sm.kv_empty[i], 1);
     }
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_empty, kComputeWarps);
-    mbar_init(&sm.pt_full, kComputeWarps);
-    mbar_init(&sm.pt_empty, 1);
+    mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&sm.tmem, 256);
+    tmem_alloc(&sm.tmem, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  const uint32_t tm_s = tmem, tm_o = tmem + 128;  // S^T: columns [0,128); O: [128,192)
 
-  if (warp == kOutTmaWarp) {
-    // ---------------- TMA producer: Q per tile; (Kc, Vc) per key tile
+  if (warp == kFaTmaWarp) {
+    // ---------------- TMA producer: the pair's two Q tiles; (Kc, Vc) per key tile
     if (lane == 0) {
       prefetch_tmap(&qmap);
       prefetch_tmap(&kcmap);
       prefetch_tmap(&vcmap);
       uint32_t kv_count = 0, q_count = 0;
-      int last_par[kOutStages];
-      for (int i = 0; i < kOutStages; ++i) last_par[i] = -1;
+      int last_par[kFaStages];
+      for (int i = 0; i < kFaStages; ++i) last_par[i] = -1;
       for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
-        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const PairInfo pi = pair_info(it, npairs, ppre, S, cu, bcu, G);
         const int qb = q_count % 2;
         if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
-        mbar_expect_tx(&sm.q_full[qb], kTile);
-        tma_load_3d(sm.q[qb], &qmap, &sm.q_full[qb], 0, ti.g * G, ti.t0);
+        mbar_expect_tx(&sm.q_full[qb], 2 * kTile);
+        tma_load_3d(sm.q[qb][0], &qmap, &sm.q_full[qb], 0, pi.g * G, pi.t0);
+        // tile B: rows past the last token are never used; keep its box inside the tensor
+        const int tb = pi.t0 + TPT < N ? pi.t0 + TPT : pi.t0;
+        tma_load_3d(sm.q[qb][1], &qmap, &sm.q_full[qb], 0, pi.g * G, tb);
         ++q_count;
-        const int nbt = (ti.nb + kBN - 1) / kBN;
+        const int nbt = (pi.nb + kBN - 1) / kBN;
+        bool ok = true;
         for (int j = 0; j < nbt; ++j) {
-          const int st = kv_count % kOutStages;
-          const uint32_t ph = (kv_count / kOutStages) & 1;
-          if (!mbar_wait(&sm.kv_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
+          const int st = kv_count % kFaStages;
+          const uint32_t ph = (kv_count / kFaStages) & 1;
+          if (!mbar_wait(&sm.kv_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); ok = false; break; }
           mbar_expect_tx(&sm.kv_full[st], 2 * kTile);
-          const int row = ti.g * btot + ti.b0 + j * kBN;
+          const int row = pi.g * btot + pi.b0 + j * kBN;
           tma_load_2d(sm.kc[st], &kcmap, &sm.kv_full[st], 0, row);
           tma_load_2d(sm.vc[st], &vcmap, &sm.kv_full[st], 0, row);
           last_par[st] = (int)ph;
           ++kv_count;
         }
+        if (!ok) break;
       }
-      for (int i = 0; i < kOutStages; ++i)
+      for (int i = 0; i < kFaStages; ++i)
         if (last_par[i] >= 0) mbar_wait(&sm.kv_full[i], (uint32_t)last_par[i]);
     }
-  } else if (warp == kOutMmaWarp) {
-    // ---------------- MMA issuer: S^T(j+1) is issued as soon as S^T(j) has been read,
-    // so it overlaps with the exps of tile j; O += P(j) Vc(j) follows when P^T(j) is ready.
+  } else if (warp == kFaMmaWarp) {
+    // ---------------- MMA issuer: S_A(0), S_B(0); then per key tile j and side:
+    // O_side += P_side(j) Vc(j) once P_side(j) is in TMEM, then S_side(j+1) into the same columns
     if (lane == 0) {
-      const uint32_t id_s = idesc_bf16(kBN, kRows);            // S^T[blocks, rows] = Kc Q^T
-      const uint32_t id_o = idesc_bf16(kRows, 64, true, true);  // O[rows, 64] += P[rows, blocks] Vc
-      uint32_t kv_count = 0, q_count = 0, s_count = 0, pt_count = 0, o_count = 0;
+      const uint32_t id_s = idesc_bf16(kRows, kBN);             // S[rows, blocks] = Q Kc^T
+      const uint32_t id_o = idesc_bf16(kRows, 64, false, true);  // O[rows, 64] += P[rows, blocks] Vc
+      uint32_t kv_count = 0, q_count = 0, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
-        const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
+        const PairInfo pi = pair_info(it, npairs, ppre, S, cu, bcu, G);
         const int qb = q_count % 2;
         if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
         ++q_count;
-        const int nbt = (ti.nb + kBN - 1) / kBN;
-        auto issue_s = [&](uint32_t kv_idx) -> bool {
-          const int st = kv_idx % kOutStages;
-          if (!mbar_wait(&sm.kv_full[st], (kv_idx / kOutStages) & 1) || !mbar_wait(&sm.s_empty, (s_count & 1) ^ 1))
-            return false;
-          tc_fence_after();
+        const int nbt = (pi.nb + kBN - 1) / kBN;
+        auto issue_s = [&](int side, int st) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(tm_s, sdesc_kmajor_sw128(sm.kc[st], 32 * k), sdesc_kmajor_sw128(sm.q[qb], 32 * k), id_s,
-                        k > 0);
-          mma_commit(&sm.s_full);
-          ++s_count;
-          return true;
+            mma_bf16_ss(tmem + side * kBN, sdesc_kmajor_sw128(sm.q[qb][side], 32 * k),
+                        sdesc_kmajor_sw128(sm.kc[st], 32 * k), id_s, k > 0);
+          mma_commit(&sm.s_full[side]);
         };
-        if (nbt > 0 && !issue_s(kv_count)) { ok = false; break; }
-        for (int j = 0; j < nbt; ++j) {
-          const int st = kv_count % kOutStages;
-          if (j + 1 < nbt && !issue_s(kv_count + 1)) { ok = false; break; }
-          // O is overwritten by the first P Vc of a tile: the previous tile's O must have been read
-          if ((j == 0 && !mbar_wait(&sm.o_empty, (o_count & 1) ^ 1)) || !mbar_wait(&sm.pt_full, pt_count & 1)) {
-            ok = false;
-            break;
-          }
+        if (nbt > 0) {
+          const int st0 = kv_count % kFaStages;
+          if (!mbar_wait(&sm.kv_full[st0], (kv_count / kFaStages) & 1)) { ok = false; break; }
           tc_fence_after();
+          issue_s(0, st0);
+          issue_s(1, st0);
+        }
+        for (int j = 0; j < nbt && ok; ++j) {
+          const uint32_t kv_j = kv_count + j;
+          const int st = kv_j % kFaStages;
+          for (int side = 0; side < 2; ++side) {
+            if (!mbar_wait(&sm.p_full[side], p_cnt[side] & 1) ||
+                (j == 0 && !mbar_wait(&sm.o_empty[side], (o_cnt[side] & 1) ^ 1))) {
+              ok = false;
+              break;
+            }
+            ++p_cnt[side];
+            tc_fence_after();
+            const uint32_t tp = tmem + side * kBN, to = tmem + 2 * kBN + side * 64;
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {
-            const uint64_t bdesc = sdesc_mnmajor_sw128(sm.vc[st], 2048 * k, kTile);
-            mma_bf16_ss(tm_o, sdesc_mnmajor_sw128(sm.pt_hi, 2048 * k, kTile), bdesc, id_o, j > 0 || k > 0);
-            mma_bf16_ss(tm_o, sdesc_mnmajor_sw128(sm.pt_lo, 2048 * k, kTile), bdesc, id_o, true);
+            for (int k = 0; k < kBN / 16; ++k) {
+              const uint64_t bdesc = sdesc_mnmajor_sw128(sm.vc[st], 2048 * k, kTile);
+              const uint32_t col = 32 * (k / 2) + 8 * (k % 2);
+              mma_bf16_ts(to, tp + col, bdesc, id_o, j > 0 || k > 0);
+              mma_bf16_ts(to, tp + col + 16, bdesc, id_o, true);
+            }
+            mma_commit(&sm.pv_done[side]);
+            if (j + 1 < nbt) {
+              const int st1 = (kv_j + 1) % kFaStages;
+              if (side == 0 && !mbar_wait(&sm.kv_full[st1], ((kv_j + 1) / kFaStages) & 1)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_s(side, st1);
+            }
           }
-          mma_commit(&sm.pt_empty);
+          if (!ok) break;
           mma_commit(&sm.kv_empty[st]);
-          ++pt_count;
-          ++kv_count;
         }
         if (!ok) break;
+        kv_count += nbt;
+        for (int side = 0; side < 2; ++side) {
+          mma_commit(&sm.o_full[side]);
+          ++o_cnt[side];
+        }
         mma_commit(&sm.q_empty[qb]);
-        mma_commit(&sm.o_full);
-        ++o_count;
       }
       if (!ok) record_timeout(status, &sm.abort_flag);
       mma_commit(&sm.mma_done);
       mbar_wait(&sm.mma_done, 0);
     }
-  } else if (warp < kComputeWarps) {
-    // ---------------- compute warps (two warpgroups): thread = block of the key tile;
-    // warpgroup wg handles query rows [64 wg, 64 wg + 64) of the tile, in two passes of 32.
-    const int b = threadIdx.x % 128;
-    const int wg = warp / 4;
-    const int r0 = 64 * wg;
-    uint32_t s_count = 0, pt_count = 0, o_count = 0, cw_phase = 0, n_tile = 0;
-    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x, ++n_tile) {
-      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
-      const int lb = n_tile & 1;
-      if (wg == 0) {
-        const int r = threadIdx.x;
-        const int64_t t = min((int64_t)ti.t0 + r / G, (int64_t)ti.t_end - 1);
-        sm.lse2[lb][r] = -lse_in[t * hq + ti.g * G + r % G] * kLog2e;  // -lse log2(e)
-      }
-      if (!cw_sync(&sm.cw, cw_phase)) { record_timeout(status, &sm.abort_flag); break; }
-      // the top-k warps have released this tile's importance buffer
-      if (!mbar_wait_warp(&sm.imp_empty[lb], ((n_tile >> 1) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
-      float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
-      const int nbt = (ti.nb + kBN - 1) / kBN;
+  } else {
+    // ---------------- softmax warpgroups: thread = row of this side's Q tile
+    const int side = warp / 4;
+    const int r = threadIdx.x % 128;
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tm_s = tmem + side * kBN + lane_off, tm_o = tmem + 2 * kBN + side * 64 + lane_off;
+    const float2 qs = make_float2(qs2, qs2);
+    uint32_t s_cnt = 0, pv_base = 0, o_cnt = 0;
+    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+      const PairInfo pi = pair_info(it, npairs, ppre, S, cu, bcu, G);
+      const int64_t t = (int64_t)pi.t0 + side * TPT + r / G;
+      const int h = pi.g * G + r % G;
+      const bool valid = t < pi.t_end;
+      const int nbt = (pi.nb + kBN - 1) / kBN;
+      float m = -CUDART_INF_F, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
-        if (!mbar_wait_warp(&sm.s_full, s_count & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.s_full[side], s_cnt & 1)) { ok = false; break; }
+        ++s_cnt;
         tc_fence_after();
-        const int bidx = j * kBN + b;  // block index inside the sequence
-        const bool bvalid = bidx < ti.nb;
-        const uint32_t taddr = tm_s + ((uint32_t)((warp % 4) * 32) << 16) + r0;
-        const float2 qs = make_float2(qs2, qs2);
-        bool ok_half = true;
+        float sv[kBN];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float p[32];
-          tmem_ld32(taddr + 32 * hh, p);
-          tmem_ld_wait();
-          if (hh == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_empty);
-          }
-          if (!bvalid) {  // ragged last key tile: blocks past the sequence get p = 0
+        for (int c = 0; c < kBN; c += 32) tmem_ld32(tm_s + c, sv + c);
+        tmem_ld_wait();
+        const int vcols = min(kBN, pi.nb - j * kBN);
+        if (vcols < kBN) {  // ragged last key tile: blocks past the sequence get p = 0
 #pragma unroll
-            for (int r = 0; r < 32; ++r) p[r] = -CUDART_INF_F;
-          }
+          for (int c = 0; c < kBN; ++c) sv[c] = c < vcols ? sv[c] : -CUDART_INF_F;
+        }
+        // row max as 8 independent chains (a single chain of 127 dependent maxima would
+        // leave the two warps per scheduler waiting on its latency)
+        float mx[8];
 #pragma unroll
-          for (int r = 0; r < 32; r += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[lb][r0 + 32 * hh + r]);
-            const float2 pa = ex2x2(ffma2(make_float2(p[r], p[r + 1]), qs, make_float2(l4.x, l4.y)));
-            const float2 pb = ex2x2(ffma2(make_float2(p[r + 2], p[r + 3]), qs, make_float2(l4.z, l4.w)));
-            p[r] = pa.x;
-            p[r + 1] = pa.y;
-            p[r + 2] = pb.x;
-            p[r + 3] = pb.y;
-          }
-          if (hh == 0) {
-            if (!mbar_wait_warp(&sm.pt_empty, (pt_count & 1) ^ 1)) {
-              ok_half = false;
-              break;
-            }
-          }
+        for (int c = 0; c < 8; ++c) mx[c] = sv[c];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t hi[4], lo[4];
+        for (int c = 8; c < kBN; ++c) mx[c % 8] = fmaxf(mx[c % 8], sv[c]);
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * qs2;  // qs2 > 0
+        float alpha = 1.f;
+        bool resc = false;
+        if (j == 0) {
+          m = mt;
+        } else if (mt > m + kFaRescaleLog2) {
+          alpha = ex2(m - mt);
+          m = mt;
+          l *= alpha;
+          resc = true;
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          // O holds the sum of the products of tiles 0 .. j-1: wait for the last one, then scale
+          if (!mbar_wait_warp(&sm.pv_done[side], (pv_base + j - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) split2(make_float2(p[8 * c + 2 * e], p[8 * c + 2 * e + 1]), hi[e], lo[e]);
-            store_pt_chunk(sm.pt_hi, b, 8 * wg + 4 * hh + c, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-            store_pt_chunk(sm.pt_lo, b, 8 * wg + 4 * hh + c, make_uint4(lo[0], lo[1], lo[2], lo[3]));
-          }
-          // selection score of this block for the pass's tokens: probability summed over the group's heads
-          if (bvalid) {
+          for (int hh = 0; hh < 2; ++hh) {
+            float o[32];
+            tmem_ld32(tm_o + 32 * hh, o);
+            tmem_ld_wait();
+            uint32_t u[32];
 #pragma unroll
-            for (int tl = 0; tl < 32 / G; ++tl) {
-              float2 acc = make_float2(p[tl * G], p[tl * G + 1]);
-#pragma unroll
-              for (int hh2 = 2; hh2 < G; hh2 += 2) acc = fadd2(acc, make_float2(p[tl * G + hh2], p[tl * G + hh2 + 1]));
-              imp_base[(int64_t)((r0 + 32 * hh) / G + tl) * imp_stride + bidx] = acc.x + acc.y;
-            }
+            for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(o[c] * alpha);
+            tmem_st16(tm_o + 32 * hh, u);
+            tmem_st16(tm_o + 32 * hh + 16, u + 16);
           }
         }
-        if (!ok_half) {
-          ok = false;
-          break;
+        const float2 nm = make_float2(-m, -m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int qq = 0; qq < kBN / 32; ++qq) {
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 x = ffma2(make_float2(sv[32 * qq + c], sv[32 * qq + c + 1]), qs, nm);
+            const float2 p = 32 * qq < kFaPolyCols ? ex2_poly2(x) : ex2x2(x);
+            acc[(c / 2) % 4] = fadd2(acc[(c / 2) % 4], p);
+            split2(p, hi[c / 2], lo[c / 2]);
+          }
+          tmem_st16(tm_s + 32 * qq, hi);
+          tmem_st16(tm_s + 32 * qq + 16, lo);
         }
-        ++s_count;
-        fence_proxy_async_smem();
+        l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.pt_full);
-        ++pt_count;
+        if (lane == 0) mbar_arrive(&sm.p_full[side]);
       }
       if (!ok) {
         record_timeout(status, &sm.abort_flag);
         break;
       }
-      // this tile's importances are complete: hand them to the top-k warps
-      __threadfence_block();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.imp_full[lb]);
-      // O of this tile: wait for the last P Vc; warpgroup wg writes columns [32 wg, 32 wg + 32)
-      if (!mbar_wait_warp(&sm.o_full, o_count & 1)) { record_timeout(status, &sm.abort_flag); break; }
-      ++o_count;
+      pv_base += nbt;
+      // O of the pair: wait for the last product, normalise, write o_cmp and lse
+      if (!mbar_wait_warp(&sm.o_full[side], o_cnt & 1)) { record_timeout(status, &sm.abort_flag); break; }
+      ++o_cnt;
       tc_fence_after();
-      {
-        const int r = b;  // TMEM lane = query row
-        const int64_t t = ti.t0 + r / G;
-        const int h = ti.g * G + r % G;
-        float o[32];
-        tmem_ld32(tm_o + ((uint32_t)((warp % 4) * 32) << 16) + 32 * wg, o);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.o_empty);
-        if (t < ti.t_end) {
-          float4* dst = reinterpret_cast<float4*>(o_out + (t * hq + h) * 64 + 32 * wg);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        }
-      }
-    }
-  } else {
-    // ---------------- top-k warps: the selection of each tile's tokens (one warp per token)
-    const int tw = warp - kComputeWarps;
-    uint32_t n_tile = 0;
-    for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x, ++n_tile) {
-      const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
-      const int lb = n_tile & 1;
-      if (!mbar_wait_warp(&sm.imp_full[lb], (n_tile >> 1) & 1)) { record_timeout(status, &sm.abort_flag); break; }
-      const float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
-      for (int tk = tw; tk < TPT; tk += kOutTopkWarps) {
-        const int64_t t = ti.t0 + tk;
-        if (t < ti.t_end && sel) {  // no sel: the selection is given, only the protocol runs
-          const float* imp = imp_base + (int64_t)tk * imp_stride;
-          int32_t* dst = sel + (t * hkv + ti.g) * topk;
-          if (ti.nb <= 256 * kTopkRegF4) {
-            if (topk <= 16)
-              warp_topk_regs<kTopkRegF4, 16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-            else
-              warp_topk_regs<kTopkRegF4, kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-          } else if (topk <= 16) {
-            warp_topk_fast<16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-          } else {
-            warp_topk_fast<kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-          }
-        }
-      }
+      float o[64];
+      tmem_ld32(tm_o, o);
+      tmem_ld32(tm_o + 32, o + 32);
+      tmem_ld_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.imp_empty[lb]);
+      if (lane == 0) mbar_arrive(&sm.o_empty[side]);
+      if (valid) {
+        const float inv = 1.f / l;
+        float4* dst = reinterpret_cast<float4*>(o_out + (t * hq + h) * 64);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          dst[i] = make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+        lse_out[t * hq + h] = (m + log2f(l)) * kLn2;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
 // selection pass (transposed: thread = block): S^T = Kc Q^T in TMEM, double-
 // buffered; p = 2^(s qs2 - lse log2 e) with the final lse of the output pass; the
 // block's score for a token is the sum of its G heads' p, written to a per-CTA
-// scratch; a warpgroup picks each token's top-k of the previous row tile while the
-// compute warps work on the next one.  A quarter of each thread's exponentials are
-// evaluated on the FMA pipe (ex2_poly2) so that the MUFU and FMA pipes share them.
+// scratch together with the maximum of each group of 32 blocks (one warp-wide
+// reduction); a warpgroup picks each token's top-k of the previous row tile from
+// those (warp_topk_groups) while the compute warps work on the next one.  A quarter
+// of each thread's exponentials are evaluated on the FMA pipe (ex2_poly2) so that the
+// MUFU and FMA pipes share them.
 // ---------------------------------------------------------------------------
 constexpr int kSelStages = 4;           // Kc ring depth
 constexpr int kSelPolyRows = 16;        // of the 64 rows a thread handles per key tile, rows on the FMA pipe
@@ -967,6 +804,7 @@ struct SelSmem {
   __align__(16) float lse2[2][kRows];  // -lse log2(e) of the tile's rows, double-buffered by tile
   float candv[kOutTopkWarps][kCandMax];
   int candi[kOutTopkWarps][kCandMax];
+  int candg[kOutTopkWarps][32 * kGrpPerLane];
   uint64_t q_full[2], q_empty[2], mma_done, cw, imp_full[2], imp_empty[2];
   uint64_t kc_full[kSelStages], kc_empty[kSelStages];
   uint64_t s_full[2], s_empty[2];
@@ -974,19 +812,23 @@ struct SelSmem {
   int abort_flag;
 };
 
+// 448 threads x 144 registers fit the SM's register file
 template <int G>
-__global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
+__global__ void __maxnreg__(144) cmp_sel_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap,
     const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S,
     int hq, int hkv, int btot, float qs2, const float* __restrict__ lse_in, int topk, int32_t* __restrict__ sel,
-    float* __restrict__ imp_scratch, int64_t imp_stride, int* status) {
+    float* __restrict__ imp_scratch, int64_t imp_stride, int64_t gm_stride, int* status) {
   constexpr int TPT = kRows / G;  // tokens per tile
   extern __shared__ uint8_t smem_raw[];
   SelSmem& sm = *reinterpret_cast<SelSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntiles = tpre[S];
   const int total = ntiles * hkv;
-  float* imp_cta = imp_scratch + (int64_t)blockIdx.x * 2 * TPT * imp_stride;
+  // this CTA's scores, two buffers of [TPT tokens][imp_stride blocks], and their group
+  // maxima, two buffers of [TPT tokens][gm_stride groups of 32 blocks]
+  float* imp_cta = imp_scratch + (int64_t)blockIdx.x * 2 * TPT * (imp_stride + gm_stride);
+  float* gm_cta = imp_cta + 2 * TPT * imp_stride;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.q_full[i], 1);
@@ -1101,6 +943,7 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
       // the top-k warps have released this tile's importance buffer
       if (!mbar_wait_warp(&sm.imp_empty[lb], ((n_tile >> 1) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
       float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
+      float* gm_base = gm_cta + (int64_t)lb * TPT * gm_stride;
       const int nbt = (ti.nb + kBN - 1) / kBN;
       bool ok = true;
       const float2 qs = make_float2(qs2, qs2);
@@ -1119,9 +962,10 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
         ++s_count;
-        if (bvalid) {
+        const int grp = j * (kBN / 32) + (warp % 4);  // this warp's 32 blocks form one group
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < 2; ++hh) {
+          if (bvalid) {
 #pragma unroll
             for (int r = 0; r < 32; r += 4) {
               const float4 l4 = *reinterpret_cast<const float4*>(&sm.lse2[lb][r0 + 32 * hh + r]);
@@ -1135,14 +979,22 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
               p[hh][r + 2] = pb.x;
               p[hh][r + 3] = pb.y;
             }
-            // selection score of this block for the pass's tokens: probability summed over the group's heads
+          }
+          // selection score of this block for the pass's tokens: probability summed over the
+          // group's heads; and the maximum over the warp's 32 blocks (scores are >= 0, so their
+          // bit patterns order as unsigned integers; blocks past the sequence count as 0)
 #pragma unroll
-            for (int tl = 0; tl < 32 / G; ++tl) {
+          for (int tl = 0; tl < 32 / G; ++tl) {
+            float v = 0.f;
+            if (bvalid) {
               float2 acc = make_float2(p[hh][tl * G], p[hh][tl * G + 1]);
 #pragma unroll
               for (int h2 = 2; h2 < G; h2 += 2) acc = fadd2(acc, make_float2(p[hh][tl * G + h2], p[hh][tl * G + h2 + 1]));
-              imp_base[(int64_t)((r0 + 32 * hh) / G + tl) * imp_stride + bidx] = acc.x + acc.y;
+              v = acc.x + acc.y;
+              imp_base[(int64_t)((r0 + 32 * hh) / G + tl) * imp_stride + bidx] = v;
             }
+            const unsigned gmx = __reduce_max_sync(0xffffffffu, __float_as_uint(v));
+            if (lane == 0) gm_base[(int64_t)((r0 + 32 * hh) / G + tl) * gm_stride + grp] = __uint_as_float(gmx);
           }
         }
       }
@@ -1164,21 +1016,17 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
       const int lb = n_tile & 1;
       if (!mbar_wait_warp(&sm.imp_full[lb], (n_tile >> 1) & 1)) { record_timeout(status, &sm.abort_flag); break; }
       const float* imp_base = imp_cta + (int64_t)lb * TPT * imp_stride;
+      const float* gm_base = gm_cta + (int64_t)lb * TPT * gm_stride;
       for (int tk = tw; tk < TPT; tk += kOutTopkWarps) {
         const int64_t t = ti.t0 + tk;
         if (t < ti.t_end) {
           const float* imp = imp_base + (int64_t)tk * imp_stride;
+          const float* gm = gm_base + (int64_t)tk * gm_stride;
           int32_t* dst = sel + (t * hkv + ti.g) * topk;
-          if (ti.nb <= 256 * kTopkRegF4) {
-            if (topk <= 16)
-              warp_topk_regs<kTopkRegF4, 16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-            else
-              warp_topk_regs<kTopkRegF4, kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-          } else if (topk <= 16) {
-            warp_topk_fast<16>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-          } else {
-            warp_topk_fast<kTopkMax>(imp, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw]);
-          }
+          if (topk <= 16)
+            warp_topk_groups<16>(imp, gm, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw], sm.candg[tw]);
+          else
+            warp_topk_groups<kTopkMax>(imp, gm, ti.nb, topk, ti.b0, dst, sm.candv[tw], sm.candi[tw], sm.candg[tw]);
         }
       }
       __syncwarp();
@@ -1753,9 +1601,22 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t smem_bytes_lse() { return sizeof(LseSmem) + 1024; }
-size_t smem_bytes_out() { return sizeof(OutSmem) + 1024; }
 
+
+size_t smem_bytes_fa() { return sizeof(FaSmem) + 1024; }
+size_t smem_bytes_sel() { return sizeof(SelSmem) + 1024; }
+
+// Pairs of 128-row tiles per sequence (per group), for the output pass.
+__global__ void pair_plan_kernel(const int32_t* __restrict__ cu, int S, int G, int32_t* __restrict__ cnt) {
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s <= S; s += gridDim.x * blockDim.x) {
+    if (s == S) {
+      cnt[s] = 0;
+      continue;
+    }
+    const int64_t rows = (int64_t)(cu[s + 1] - cu[s]) * G;
+    cnt[s] = (int32_t)((rows + 2 * kRows - 1) / (2 * kRows));
+  }
+}
 
 template <int G>
 cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st) {
@@ -1767,20 +1628,31 @@ cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_ti
   const int btot = (int)a.blk->count;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaFuncSetAttribute(cmp_lse_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_lse());
-    cudaFuncSetAttribute(cmp_out_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_out());
-    cudaFuncSetAttribute(cmp_out_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_out());
+    cudaFuncSetAttribute(cmp_fa_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_fa());
+    cudaFuncSetAttribute(cmp_fa_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_fa());
+    cudaFuncSetAttribute(cmp_sel_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_sel());
+    cudaFuncSetAttribute(cmp_sel_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes_sel());
     attr_done = true;
   }
-  const int sms = num_sms() < kCmpOutCtas ? num_sms() : kCmpOutCtas;
-  const int64_t tiles = total_tiles_bound * a.hkv;
-  const int g1 = (int)(tiles < 2 * sms ? (tiles > 0 ? tiles : 1) : 2 * sms);
-  const int g2 = (int)(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);  // at most kCmpOutCtas (scratch size)
-  SSA_LAUNCH("cmp_lse_tc_kernel", cmp_lse_tc_kernel, g1, kThreads, smem_bytes_lse(), st, qm, km, a.cu_seqlens,
-             a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.status);
-  SSA_LAUNCH("cmp_out_tc_kernel", cmp_out_tc_kernel<G>, g2, kOutThreadsTk, smem_bytes_out(), st, qm, km, vm,
-             a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.o_branch, a.topk,
-             a.sel_given ? nullptr : a.sel, a.imp_scratch, (int64_t)((btot + 3) & ~3), a.status);
+  // output pass: pairs of row tiles (the per-sequence pair prefix goes to tiles_cnt / tiles_pre,
+  // which the tensor-core forward does not otherwise use)
+  SSA_LAUNCH("pair_plan_kernel", pair_plan_kernel, (a.S + 256) / 256, 256, 0, st, a.cu_seqlens, a.S, G,
+             a.tiles_cnt);
+  cudaError_t e = exclusive_scan(a.tiles_cnt, a.tiles_pre, a.S + 1, a.scan_tmp, st);
+  if (e != cudaSuccess) return e;
+  const int sms = num_sms();
+  const int64_t pairs = ((total_tiles_bound + 1) / 2 + a.S) * a.hkv;
+  const int g1 = (int)(pairs < sms ? (pairs > 0 ? pairs : 1) : sms);
+  SSA_LAUNCH("cmp_fa_tc_kernel", cmp_fa_tc_kernel<G>, g1, kFaThreads, smem_bytes_fa(), st, qm, km, vm, a.cu_seqlens,
+             a.blk->cu, a.tiles_pre, a.S, a.N, a.hq, a.hkv, btot, qs2, a.o_branch, a.lse, a.status);
+  if (!a.sel_given) {  // a given selection needs no scores
+    const int64_t tiles = total_tiles_bound * a.hkv;
+    const int smax = sms < kCmpOutCtas ? sms : kCmpOutCtas;  // the score scratch holds kCmpOutCtas CTAs
+    const int g2 = (int)(tiles < smax ? (tiles > 0 ? tiles : 1) : smax);
+    SSA_LAUNCH("cmp_sel_tc_kernel", cmp_sel_tc_kernel<G>, g2, kOutThreadsTk, smem_bytes_sel(), st, qm, km,
+               a.cu_seqlens, a.blk->cu, tpre, a.S, a.hq, a.hkv, btot, qs2, a.lse, a.topk, a.sel, a.imp_scratch,
+               (int64_t)((btot + 3) & ~3), (int64_t)(((btot + 31) / 32 + 3) & ~3), a.status);
+  }
   return cudaGetLastError();
 }
 
@@ -1851,7 +1723,8 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
 
 size_t cmp_tc_scratch_floats(int hq, int hkv, int64_t btot) {
   const int G = hkv > 0 ? hq / hkv : 1;
-  return (size_t)kCmpOutCtas * 2 * (kRows / (G > 0 ? G : 1)) * (size_t)((btot + 3) & ~int64_t(3)) + 4;
+  const size_t per_token = (size_t)((btot + 3) & ~int64_t(3)) + (size_t)(((btot + 31) / 32 + 3) & ~int64_t(3));
+  return (size_t)kCmpOutCtas * 2 * (kRows / (G > 0 ? G : 1)) * per_token + 4;
 }
 
 bool cmp_tc_supported(int dtype, int d, int hq, int hkv, int topk) {

@@ -38,6 +38,12 @@ struct FwdArgs {
   int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
   float* imp_scratch;  // [kCmpOutCtas, 128/G, B] selection scores (tensor-core path)
   int32_t *win_cnt, *win_pre, *win_scan;  // [W + 1] window work plan
+  // The window branch's problem: the queries' own tokens.  Self attention: has_win = 1,
+  // wk/wv = k/v, wks/wvs = ks/vs.  Cross attention: has_win = 0.  A sequence-parallel
+  // rank: its own tokens' K / V and their window-ordered copies.
+  int has_win;
+  const void *wk, *wv;  // [N, Hkv, d] K / V of the query tokens (SIMT window kernels)
+  void *wks, *wvs;      // [Hkv, N, d] the same in window order (tensor-core window kernels)
 };
 
 // Learned compression (sparse 3D convolution before the block mean), see conv.cu.
@@ -94,6 +100,13 @@ struct BwdArgs {
   int32_t* radix_tmp;
   int32_t *slc_cnt, *slc_pre;  // [Hkv * B + 1] work items of the selected-branch dK/dV kernel
   int32_t *tiles_cnt, *tiles_pre, *items_cnt, *items_pre, *scan_tmp;
+  // the window branch's problem, as in FwdArgs; its key gradients go to wdk / wdv
+  // ([N, Hkv, d]: dk / dv themselves unless the query rows are a rank's tokens, whose
+  // window gradients are then scatter-added into dk / dv at rows wtok[i])
+  int has_win;
+  const void *wk, *wv, *wks, *wvs;
+  float *wdk, *wdv;
+  const int32_t* wtok;
 };
 
 bool pool_supported(int dtype, int hkv, int d);
@@ -123,5 +136,9 @@ cudaError_t geo_select(const int32_t* coords, const int32_t* cu_seqlens, int S, 
 bool slc_mma_supported(int dtype, int d, int hq, int hkv, int topk);
 cudaError_t slc_fwd_mma(const FwdArgs& a, cudaStream_t st);
 cudaError_t slc_bwd_mma(const BwdArgs& a, cudaStream_t st);
+
+// Diagnostics (diag.cu): a bounded wait that runs out; the FMA-pipe exponential.
+cudaError_t diag_wait_timeout(int* status, int* out, cudaStream_t st);
+cudaError_t diag_ex2(const float* x, float* y_poly, float* y_mufu, int64_t n, cudaStream_t st);
 
 }  // namespace ssa

@@ -873,8 +873,8 @@ template <int G>
 cudaError_t win_fwd_tc_g(const FwdArgs& a, int32_t* cnt, int32_t* pre, int32_t* scan_tmp, cudaStream_t st) {
   const int64_t W = a.win->count, N = a.N;
   CUtensorMap qm, km, vm;
-  if (!map_q_token(&qm, a.q, N, a.hq, G) || !map_rows64(&km, a.ks, (int64_t)a.hkv * N) ||
-      !map_rows64(&vm, a.vs, (int64_t)a.hkv * N))
+  if (!map_q_token(&qm, a.q, N, a.hq, G) || !map_rows64(&km, a.wks, (int64_t)a.hkv * N) ||
+      !map_rows64(&vm, a.wvs, (int64_t)a.hkv * N))
     return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
@@ -897,7 +897,7 @@ cudaError_t win_bwd_tc_g(const BwdArgs& a, int32_t* cnt, int32_t* pre, int32_t* 
   const int64_t rows = N * a.hq;
   CUtensorMap qm, dm, km, vm, lm, cm, wm;
   if (!map_q_token(&qm, a.q, N, a.hq, G) || !map_q_token(&dm, a.dout, N, a.hq, G) ||
-      !map_rows64(&km, a.ks, (int64_t)a.hkv * N) || !map_rows64(&vm, a.vs, (int64_t)a.hkv * N) ||
+      !map_rows64(&km, a.wks, (int64_t)a.hkv * N) || !map_rows64(&vm, a.wvs, (int64_t)a.hkv * N) ||
       !map_rowscalars_token(&lm, a.rc + 3 * rows, N, a.hq, G) ||  // -lse log2(e) of the window branch
       !map_rowscalars_token(&cm, a.rc + 5 * rows, N, a.hq, G) ||  // -D
       !map_rowscalars_token(&wm, a.rc + 4 * rows, N, a.hq, G))    // w
@@ -920,8 +920,8 @@ cudaError_t win_bwd_tc_g(const BwdArgs& a, int32_t* cnt, int32_t* pre, int32_t* 
   e = exclusive_scan(cnt, pre, W + 1, scan_tmp, st);
   if (e != cudaSuccess) return e;
   SSA_LAUNCH("win_bwd_dkv_tc_kernel", win_bwd_dkv_tc_kernel<G>, num_sms(), 32 * (kCW + 2), sizeof(WinDkvSmem) + 1024,
-             st, qm, dm, km, vm, lm, cm, wm, a.win->perm, a.win->ptr, pre, W, N, a.hq, a.hkv, qs2, a.scale, a.dk,
-             a.dv, a.status);
+             st, qm, dm, km, vm, lm, cm, wm, a.win->perm, a.win->ptr, pre, W, N, a.hq, a.hkv, qs2, a.scale, a.wdk,
+             a.wdv, a.status);
   return cudaGetLastError();
 }
 

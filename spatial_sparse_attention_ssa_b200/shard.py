@@ -177,3 +177,21 @@ def reduce_to_owners(partial, tokens: np.ndarray, group=None):
     total = partial.clone()
     dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
     return total[torch.as_tensor(np.asarray(tokens, np.int64), device=total.device)]
+
+
+def sp_local_plan(blk_perm, blk_ptr, blk_cu, cu_seqlens, world: int, rank: int) -> LocalPlan:
+    """This rank's tokens when every sequence's blocks are split into `world` contiguous
+    ranges balanced by tokens (block_ranges) and rank r owns range r of each sequence:
+    `tokens` are global token indices in block order, `cu_seqlens` their per-sequence
+    offsets, `seqs` every sequence (a rank may own no block of a short one)."""
+    blk_ptr = np.asarray(blk_ptr, np.int64)
+    blk_cu = np.asarray(blk_cu, np.int64)
+    parts, cu = [], [0]
+    for s in range(len(cu_seqlens) - 1):
+        b0, b1 = int(blk_cu[s]), int(blk_cu[s + 1])
+        lo, hi = block_ranges(np.diff(blk_ptr[b0:b1 + 1]), world)[rank] if b1 > b0 else (0, 0)
+        toks = range_tokens(blk_perm, blk_ptr, b0 + lo, b0 + hi)
+        parts.append(toks)
+        cu.append(cu[-1] + len(toks))
+    tokens = np.concatenate(parts) if parts else np.zeros(0, np.int64)
+    return LocalPlan(np.arange(len(cu_seqlens) - 1), tokens.astype(np.int64), np.asarray(cu, np.int32))

@@ -25,11 +25,13 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
 DTYPE_BF16, DTYPE_F32 = 0, 1
 GATE_WEIGHTS, GATE_LOGITS = 0, 1
 OP_BIN, OP_FORWARD, OP_BACKWARD, OP_GEO_SELECT, OP_CROSS_FORWARD, OP_CROSS_BACKWARD = 0, 1, 2, 3, 4, 5
+OP_SP_FORWARD, OP_SP_BACKWARD = 6, 7
 SEL_SCORES, SEL_GIVEN = 0, 1
 
 EXPORTS = ("ssa_bin", "ssa_forward", "ssa_backward", "ssa_workspace_size", "ssa_error_string",
            "ssa_get_device_status", "ssa_version", "ssa_launch_count", "ssa_profile_enable",
-           "ssa_profile_read", "ssa_geo_select", "ssa_cross_forward", "ssa_cross_backward", "ssa_pool")
+           "ssa_profile_read", "ssa_geo_select", "ssa_cross_forward", "ssa_cross_backward", "ssa_pool",
+           "ssa_diag_wait_timeout", "ssa_diag_ex2", "ssa_sp_forward", "ssa_sp_backward")
 
 
 class SSAError(RuntimeError):
@@ -55,6 +57,12 @@ class Params(ctypes.Structure):
 class Partition(ctypes.Structure):
     _fields_ = [("id", ctypes.c_void_p), ("perm", ctypes.c_void_p), ("ptr", ctypes.c_void_p),
                 ("cu", ctypes.c_void_p), ("key", ctypes.c_void_p), ("count", ctypes.c_int64)]
+
+
+class SpLocalC(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("cu_seqlens", ctypes.c_void_p), ("tokens", ctypes.c_void_p),
+                ("win", ctypes.POINTER(Partition)), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("ks", ctypes.c_void_p), ("vs", ctypes.c_void_p)]
 
 
 class Saved(ctypes.Structure):
@@ -88,6 +96,17 @@ def _lib():
         lib.ssa_cross_backward.argtypes = [ctypes.POINTER(Params), vp, i32, i64, i64, pp, vp, vp, vp, vp,
                                            ctypes.POINTER(Saved), vp, vp, vp, vp, vp, vp, sz, vp]
         lib.ssa_cross_backward.restype = ctypes.c_int
+        spp = ctypes.POINTER(SpLocalC)
+        lib.ssa_sp_forward.argtypes = [ctypes.POINTER(Params), i32, i64, pp, spp, vp, vp, vp, vp, vp,
+                                       ctypes.POINTER(Saved), vp, sz, vp]
+        lib.ssa_sp_forward.restype = ctypes.c_int
+        lib.ssa_sp_backward.argtypes = [ctypes.POINTER(Params), i32, i64, pp, spp, vp, vp, vp, vp,
+                                        ctypes.POINTER(Saved), vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.ssa_sp_backward.restype = ctypes.c_int
+        lib.ssa_diag_wait_timeout.argtypes = [vp, vp]
+        lib.ssa_diag_wait_timeout.restype = ctypes.c_int
+        lib.ssa_diag_ex2.argtypes = [vp, vp, vp, i64, vp]
+        lib.ssa_diag_ex2.restype = ctypes.c_int
         lib.ssa_pool.argtypes = [i32, i32, i32, i64, pp, vp, vp, vp, vp, vp, vp, vp]
         lib.ssa_pool.restype = ctypes.c_int
         lib.ssa_geo_select.argtypes = [vp, vp, i32, i64, i32, pp, i32, i32, i32, vp, vp, sz, vp]
@@ -386,6 +405,80 @@ def ssa_backward(p: Params, cu_seqlens: torch.Tensor, blk: Bins, win: Bins, q, k
     return dq, dk, dv, dg
 
 
+@dataclass
+class SpLocal:
+    """One rank's tokens of a batch split by whole blocks (see ssa_sp_forward in
+    include/ssa.h): their per-sequence offsets, their rows among all tokens, their own
+    window partition and K / V, and room for their window-ordered K / V copies."""
+    cu_seqlens: torch.Tensor  # int32 [S+1]
+    tokens: torch.Tensor      # int32 [Nr]
+    win: Bins                 # ssa_bin of the rank's coordinates (edge m_win)
+    k: torch.Tensor           # [Nr, Hkv, d]
+    v: torch.Tensor
+    ks: torch.Tensor          # [Hkv, Nr, d]
+    vs: torch.Tensor
+
+    @staticmethod
+    def make(cu_seqlens, tokens, win: Bins, k, v) -> "SpLocal":
+        n, hkv, d = (int(x) for x in k.shape)
+        e = lambda: torch.empty(hkv, n, d, dtype=k.dtype, device=k.device)  # noqa: E731
+        return SpLocal(cu_seqlens, tokens, win, k, v, e(), e())
+
+    def c(self):
+        pw = self.win.c()
+        return SpLocalC(int(self.k.shape[0]), _ptr(self.cu_seqlens), _ptr(self.tokens), ctypes.pointer(pw),
+                        _ptr(self.k), _ptr(self.v), _ptr(self.ks), _ptr(self.vs)), pw
+
+
+def ssa_sp_forward(p: Params, blk: Bins, n_all: int, loc: SpLocal, q: torch.Tensor, k: torch.Tensor,
+                   v: torch.Tensor, gates: torch.Tensor, out: torch.Tensor | None = None,
+                   saved: SavedTensors | None = None, workspace: torch.Tensor | None = None):
+    """One rank's forward (sequences split by whole blocks): its query rows q / gates
+    [Nr, Hq, *] against all N tokens' k / v binned into `blk`; returns (out, saved)."""
+    _require_cuda(q, k, v, gates, loc.cu_seqlens, loc.tokens, loc.k, loc.v)
+    nr, s = int(q.shape[0]), int(loc.cu_seqlens.shape[0]) - 1
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if saved is None:  # the cross-attention buffers, with room for the third (window) branch
+        saved = dataclasses.replace(SavedTensors.empty_cross(p, nr, n_all, blk.count, q.dtype, dev),
+                                    o_branch=torch.empty(3, nr, p.hq, p.d, dtype=torch.float32, device=dev),
+                                    lse=torch.empty(3, nr, p.hq, dtype=torch.float32, device=dev))
+    need = workspace_size(OP_SP_FORWARD, p, s, nr, blk.count, loc.win.count)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb, sv = blk.c(), saved.c()
+    lc, _keep = loc.c()
+    st = _lib().ssa_sp_forward(ctypes.byref(p), s, int(n_all), ctypes.byref(pb), ctypes.byref(lc), _ptr(q), _ptr(k),
+                               _ptr(v), _ptr(gates), _ptr(out), ctypes.byref(sv), _ptr(ws), ws.numel(),
+                               _stream(dev))
+    _check(st, "ssa_sp_forward")
+    return out, saved
+
+
+def ssa_sp_backward(p: Params, blk: Bins, n_all: int, loc: SpLocal, q, k, v, gates, saved: SavedTensors,
+                    dout, grads=None, workspace: torch.Tensor | None = None):
+    """One rank's backward: (dq [Nr, Hq, d], dk, dv [N, Hkv, d] = its rows' contributions to every
+    token's key gradients, dgates [Nr, Hq, 3])."""
+    _require_cuda(q, k, v, gates, dout)
+    nr, s = int(q.shape[0]), int(loc.cu_seqlens.shape[0]) - 1
+    dev = q.device
+    if grads is None:
+        grads = (torch.empty(q.shape, dtype=torch.float32, device=dev),
+                 torch.empty(k.shape, dtype=torch.float32, device=dev),
+                 torch.empty(v.shape, dtype=torch.float32, device=dev),
+                 torch.empty(gates.shape, dtype=torch.float32, device=dev))
+    dq, dk, dv, dg = grads
+    need = workspace_size(OP_SP_BACKWARD, p, s, nr, blk.count, loc.win.count)
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, dev)
+    pb, sv = blk.c(), saved.c()
+    lc, _keep = loc.c()
+    st = _lib().ssa_sp_backward(ctypes.byref(p), s, int(n_all), ctypes.byref(pb), ctypes.byref(lc), _ptr(q), _ptr(k),
+                                _ptr(v), _ptr(gates), ctypes.byref(sv), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                _ptr(dg), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ssa_sp_backward")
+    return dq, dk, dv, dg
+
+
 def ssa_cross_forward(p: Params, q_cu: torch.Tensor, blk: Bins, q: torch.Tensor, k: torch.Tensor,
                       v: torch.Tensor, gates: torch.Tensor, out: torch.Tensor | None = None,
                       saved: SavedTensors | None = None, workspace: torch.Tensor | None = None,
@@ -467,6 +560,22 @@ def profile_read(max_entries: int = 128) -> dict:
         nm = names.raw[i * name_len:(i + 1) * name_len].split(b"\0", 1)[0].decode()
         out[nm] = (float(ms[i]), int(cnt[i]))
     return out
+
+
+def diag_wait_timeout(device=None) -> tuple[int, int]:
+    """Runs the bounded-wait diagnostic; returns (lane wait gave up, warp wait gave up)."""
+    out = torch.zeros(2, dtype=torch.int32, device=device or "cuda")
+    _check(_lib().ssa_diag_wait_timeout(_ptr(out), _stream(out.device)), "ssa_diag_wait_timeout")
+    o = out.cpu().tolist()
+    return int(o[0]), int(o[1])
+
+
+def diag_ex2(x: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """(2^x on the FMA pipe as the kernels evaluate it, 2^x from ex2.approx) for fp32 x."""
+    _require_cuda(x)
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    _check(_lib().ssa_diag_ex2(_ptr(x), _ptr(yp), _ptr(ym), x.numel(), _stream(x.device)), "ssa_diag_ex2")
+    return yp, ym
 
 
 def default_scale(d: int) -> float:

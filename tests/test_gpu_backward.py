@@ -24,6 +24,9 @@ def _bwd_parity(w, t):
     dict(hq=8, hkv=2, d=32, m_cmp=3, m_win=6, topk=5, dtype="bf16", gate_mode=0),
     dict(hq=4, hkv=2, d=64, m_cmp=4, m_win=4, topk=6, dtype="f32", gate_mode=1),
     dict(hq=2, hkv=1, d=32, m_cmp=4, m_win=4, topk=4, dtype="f32", gate_mode=0),
+    # head dim 128 (the fp32 CUDA-core kernels), bf16 and fp32
+    dict(hq=16, hkv=2, d=128, m_cmp=4, m_win=4, topk=6, dtype="bf16", gate_mode=1),
+    dict(hq=8, hkv=2, d=128, m_cmp=4, m_win=8, topk=4, dtype="f32", gate_mode=0),
 ])
 def test_small_shell_backward_parity(kw):
     w = W.small_shell(seed=11, R=32, n_prims=2, lo=4.0, hi=9.0, n_keep=900, n_seqs=2, **kw)

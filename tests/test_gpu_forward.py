@@ -33,6 +33,9 @@ def test_config1_fp32_full_parity():
     dict(hq=8, hkv=2, d=32, m_cmp=3, m_win=2, topk=5, dtype="bf16", gate_mode=0),
     dict(hq=16, hkv=1, d=64, m_cmp=4, m_win=4, topk=4, dtype="f32", gate_mode=1),
     dict(hq=2, hkv=2, d=64, m_cmp=8, m_win=4, topk=32, dtype="bf16", gate_mode=1),
+    # head dim 128 (the fp32 CUDA-core kernels), bf16 and fp32
+    dict(hq=16, hkv=2, d=128, m_cmp=4, m_win=4, topk=8, dtype="bf16", gate_mode=1),
+    dict(hq=4, hkv=1, d=128, m_cmp=4, m_win=8, topk=4, dtype="f32", gate_mode=0),
 ])
 def test_small_shell_parity(kw):
     w = W.small_shell(seed=3, R=40, n_prims=2, lo=5.0, hi=11.0, n_keep=1500, n_seqs=2, **kw)

@@ -58,8 +58,11 @@ def _rank_main(rank, world, port, result_q):
         q, k, v, do = (t.as_f32(x).astype(np.float64) for x in ("q", "k", "v", "do"))
         kw = dict(hq=w.hq, hkv=w.hkv, m_cmp=w.m_cmp, gate_mode=w.gate_mode, pool_rounding="none")
         blk = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)  # every rank bins the sequence the same way
+        # the plan the GPU path uses (ssa_sp_forward's callers): whole blocks per rank
+        plan = shard.sp_local_plan(blk["perm"], blk["ptr"], blk["cu"], w.cu_seqlens, world, rank)
+        mine = plan.tokens
         lo, hi = shard.block_ranges(np.diff(blk["ptr"]), world)[rank]
-        mine = shard.range_tokens(blk["perm"], blk["ptr"], lo, hi)
+        assert np.array_equal(mine, shard.range_tokens(blk["perm"], blk["ptr"], lo, hi))
         n, nr = w.n, len(mine)
 
         # all-gather of K / V: each rank contributes its own tokens' rows
@@ -119,3 +122,24 @@ def test_two_gloo_ranks_reproduce_one_sequence_forward_and_backward():
         assert e["sel"] == 0, e
         for key in ("out", "dq", "dk", "dv", "dgates"):
             assert e[key] <= 1e-12, (key, e)
+
+
+def test_sp_local_plan_partitions_every_sequence_by_whole_blocks():
+    w = W.small_shell(seed=62, R=32, n_prims=2, lo=4.0, hi=8.0, n_keep=300, n_seqs=3, hq=4, hkv=2, d=8,
+                      m_cmp=4, m_win=4, topk=3, dtype="f32")
+    blk = O.bin_tokens(w.coords, w.cu_seqlens, w.m_cmp)
+    for world in (1, 2, 3, 5):
+        seen = np.zeros(w.n, np.int64)
+        for r in range(world):
+            plan = shard.sp_local_plan(blk["perm"], blk["ptr"], blk["cu"], w.cu_seqlens, world, r)
+            seen[plan.tokens] += 1
+            assert plan.cu_seqlens[-1] == len(plan.tokens) and len(plan.cu_seqlens) == w.s + 1
+            for s_ in range(w.s):
+                toks = plan.tokens[plan.cu_seqlens[s_]:plan.cu_seqlens[s_ + 1]]
+                assert ((toks >= w.cu_seqlens[s_]) & (toks < w.cu_seqlens[s_ + 1])).all()
+                ids = blk["id"][toks]
+                # whole blocks, consecutive ids, members in block order
+                assert (np.diff(ids) >= 0).all() and (np.diff(np.unique(ids)) == 1).all()
+                for b in np.unique(ids):
+                    assert (ids == b).sum() == blk["ptr"][b + 1] - blk["ptr"][b]
+        assert (seen == 1).all()
