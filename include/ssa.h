@@ -114,6 +114,11 @@ typedef struct ssa_params {
                         ssa_geo_select), read by the selected branch and the backward, see ssa_forward */
   const ssa_conv* conv; /* NULL: mean-pool compression; else the learned compression (self attention only;
                            Hkv * d <= 256); its workspace is included by ssa_workspace_size */
+  int32_t deterministic; /* 0: the backward adds key gradients with fp32 atomics (bits may vary between
+                            runs); 1: it adds them as 64-bit fixed-point integers (2^-32 resolution, each
+                            accumulated component below 2^31 in magnitude), so every output is bitwise
+                            reproducible.  1 needs the tensor-core backward (bf16, d = 64, G in {8, 16},
+                            topk <= 32) and no conv, else SSA_ERR_UNSUPPORTED; its workspace is included */
 } ssa_params;
 
 /*

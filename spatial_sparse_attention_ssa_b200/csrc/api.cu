@@ -34,6 +34,16 @@ int* status_ptr() {
 
 ssa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
 
+// SSA_DISABLE_TC=1 selects the fp32 SIMT kernels for every shape (cross-checks).
+bool tc_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("SSA_DISABLE_TC");
+    v = (e && e[0] == '1') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 ssa_status check_params(const ssa_params* p) {
   if (!p) return SSA_ERR_INVALID_ARG;
   if (p->hq < 1 || p->hkv < 1 || p->hq % p->hkv != 0) return SSA_ERR_INVALID_ARG;
@@ -51,6 +61,11 @@ ssa_status check_params(const ssa_params* p) {
   if (G * (p->d / 32) > 32) return SSA_ERR_UNSUPPORTED;
   if (p->conv && p->hkv * p->d > 256) return SSA_ERR_UNSUPPORTED;
   if (!ssa::pool_supported(p->dtype, p->hkv, p->d)) return SSA_ERR_UNSUPPORTED;
+  if (p->deterministic != 0 && p->deterministic != 1) return SSA_ERR_INVALID_ARG;
+  if (p->deterministic &&
+      (p->conv || !tc_enabled() || !ssa::cmp_tc_supported(p->dtype, p->d, p->hq, p->hkv, p->topk) ||
+       !ssa::slc_mma_supported(p->dtype, p->d, p->hq, p->hkv, p->topk)))
+    return SSA_ERR_UNSUPPORTED;  // the fixed-point sums are built into the tensor-core backward
   return SSA_OK;
 }
 
@@ -61,16 +76,6 @@ bool partition_ok(const ssa_partition* x, int64_t n) {
 }
 
 float eff_scale(const ssa_params* p) { return p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->d); }
-
-// SSA_DISABLE_TC=1 selects the fp32 SIMT kernels for every shape (cross-checks).
-bool tc_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("SSA_DISABLE_TC");
-    v = (e && e[0] == '1') ? 0 : 1;
-  }
-  return v == 1;
-}
 
 // Workspace of the forward (after `ws` base): plan arrays.
 void carve_plan(Carver& c, int32_t S, int32_t** tc, int32_t** tp, int32_t** ic, int32_t** ip, int32_t** st) {
@@ -147,6 +152,7 @@ size_t sp_bwd_extra(const ssa_params* p, int64_t Nr) {
 }
 
 struct BwdWs {
+  unsigned long long *fx_kc, *fx_vc, *fx_k, *fx_v;
   float* Dc;
   float* rc;
   float *dkc, *dvc;
@@ -177,6 +183,14 @@ size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t 
   w->st = c.take<int32_t>(ssa::scan_tmp_ints(mx));
   int32_t* unused_st;
   carve_plan(c, S, &w->tc, &w->tp, &w->ic, &w->ip, &unused_st);
+  if (p->deterministic) {  // 64-bit fixed-point sums: dKc / dVc [Hkv, B, d], dK / dV [N, Hkv, d]
+    w->fx_kc = c.take<unsigned long long>(p->hkv * B * p->d);
+    w->fx_vc = c.take<unsigned long long>(p->hkv * B * p->d);
+    w->fx_k = c.take<unsigned long long>(N * p->hkv * p->d);
+    w->fx_v = c.take<unsigned long long>(N * p->hkv * p->d);
+  } else {
+    w->fx_kc = w->fx_vc = w->fx_k = w->fx_v = nullptr;
+  }
   return c.used;
 }
 
@@ -485,6 +499,10 @@ ssa_status backward_common(const ssa_params* p, const int32_t* cu, int32_t S, in
   a.wdk = dk;
   a.wdv = dv;
   a.wtok = nullptr;
+  a.fx_kc = w.fx_kc;
+  a.fx_vc = w.fx_vc;
+  a.fx_k = w.fx_k;
+  a.fx_v = w.fx_v;
   if (sp) {  // a sequence-parallel rank: the window problem is its own tokens
     a.has_win = 1;
     a.wk = sp->k;
@@ -591,7 +609,7 @@ SSA_API ssa_status ssa_cross_backward(const ssa_params* p, const int32_t* q_cu, 
   if (S < 1 || Nq < 0 || Nq > INT32_MAX - 1 || Nkv < 0 || Nkv > INT32_MAX - 1 || !q_cu || !partition_ok(blk, Nkv) ||
       !saved)
     return SSA_ERR_INVALID_ARG;
-  if (p->conv) return SSA_ERR_UNSUPPORTED;
+  if (p->conv || p->deterministic) return SSA_ERR_UNSUPPORTED;  // both are built for ssa_backward
   if (Nkv > 0 && dk && dv && Nq == 0) {  // no queries: the key gradients are zero
     cudaStream_t st0 = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(dk, 0, sizeof(float) * Nkv * p->hkv * p->d, st0) != cudaSuccess ||
@@ -624,6 +642,7 @@ ssa_status sp_check(const ssa_params* p, int32_t S, int64_t N, const ssa_partiti
   ssa_status ps = check_params(p);
   if (ps != SSA_OK) return ps;
   if (p->conv) return SSA_ERR_INVALID_ARG;  // the learned compression is built for the whole-sequence call
+  if (p->deterministic) return SSA_ERR_UNSUPPORTED;  // the fixed-point sums are built for ssa_backward
   if (p->m_cmp % p->m_win != 0) return SSA_ERR_INVALID_ARG;  // a window must lie inside one block
   if (S < 1 || N < 1 || N > INT32_MAX - 1 || !loc || loc->n < 0 || loc->n > N || !partition_ok(blk, N))
     return SSA_ERR_INVALID_ARG;

@@ -1236,6 +1236,13 @@ __global__ void keys_to_ptr_kernel(const uint64_t* __restrict__ keys, int64_t n,
 }
 
 // per-sequence work counts for the tiled kernels
+// dst[i] = src[i] * 2^-32: the deterministic fixed-point sums back to fp32 (through
+// fp64, which holds the 64-bit integer's leading bits exactly enough for one rounding).
+__global__ void fix_to_float_kernel(const unsigned long long* __restrict__ src, float* __restrict__ dst, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = (float)((double)(long long)src[i] * (1.0 / 4294967296.0));
+}
+
 // dst[rows[i]] += src[i] for rows of `w4` float4 (dK and dV at once); the rows are distinct.
 __global__ void rows_add_kernel(const float* __restrict__ srck, const float* __restrict__ srcv,
                                 const int32_t* __restrict__ rows, int64_t n, int w4, float* __restrict__ dstk,
@@ -1380,22 +1387,36 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
         a.scale, kCmpRowChunk, a.lse, a.Dc, a.dkc, a.dvc);
   }
   if (D == 64 && (G == 8 || G == 16)) {
-    cudaMemsetAsync(a.dk, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
-    cudaMemsetAsync(a.dv, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
     const int g_slc = grid_1d(a.N * a.hkv, 8, 148 * 16);
     if (a.use_tc && slc_mma_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
+      if (a.fx_k) {  // deterministic: fixed-point sums of the selected branch, then dK / dV = them
+        cudaMemsetAsync(a.fx_k, 0, sizeof(unsigned long long) * a.Nkv * a.hkv * D, st);
+        cudaMemsetAsync(a.fx_v, 0, sizeof(unsigned long long) * a.Nkv * a.hkv * D, st);
+      } else {
+        cudaMemsetAsync(a.dk, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
+        cudaMemsetAsync(a.dv, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
+      }
       e = slc_bwd_mma(a, st);
+      if (e == cudaSuccess && a.fx_k) {
+        e = fix_to_float(a.fx_k, a.dk, a.Nkv * a.hkv * D, st);
+        if (e == cudaSuccess) e = fix_to_float(a.fx_v, a.dv, a.Nkv * a.hkv * D, st);
+      }
       if (e != cudaSuccess) return e;
-    } else if (G == 16)
+    } else if (G == 16) {
+      cudaMemsetAsync(a.dk, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
+      cudaMemsetAsync(a.dv, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
       SSA_LAUNCH("slc_bwd_fused_kernel", (slc_bwd_fused_kernel<T, 16>), g_slc, 256, 0, st, q, ks, vs, dout, a.gates,
                  a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
                  a.lse + rows,
                  a.Dc + rows, a.dq, a.dk, a.dv);
-    else
+    } else {
+      cudaMemsetAsync(a.dk, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
+      cudaMemsetAsync(a.dv, 0, sizeof(float) * a.Nkv * a.hkv * D, st);
       SSA_LAUNCH("slc_bwd_fused_kernel", (slc_bwd_fused_kernel<T, 8>), g_slc, 256, 0, st, q, ks, vs, dout, a.gates,
                  a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
                  a.lse + rows,
                  a.Dc + rows, a.dq, a.dk, a.dv);
+    }
   } else {
     const int pairs_per_cta = 128 / (G * C::NT);
     SSA_LAUNCH("slc_bwd_dq_kernel", (slc_bwd_dq_kernel<T, D>), grid_1d(a.N * a.hkv, pairs_per_cta, 148 * 16), 128, 0, st, 
@@ -1475,6 +1496,12 @@ cudaError_t simt_forward(const FwdArgs& a, cudaStream_t st) {
     if (a.d == 128) return forward_impl<float, 128>(a, st);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t fix_to_float(const unsigned long long* src, float* dst, int64_t n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  SSA_LAUNCH("fix_to_float_kernel", fix_to_float_kernel, grid_1d(n, 256, 148 * 32), 256, 0, st, src, dst, n);
+  return cudaGetLastError();
 }
 
 cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st) {

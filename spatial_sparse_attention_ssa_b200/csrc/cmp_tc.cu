@@ -68,13 +68,16 @@ __device__ __forceinline__ bool aborted(const int* abort_flag) {
 }
 
 // ---------------------------------------------------------------------------
-// pass 2: output + top-k (transposed: thread = block)
+// top-k selection (the selection pass below runs it in a warpgroup of its own)
 // ---------------------------------------------------------------------------
 constexpr int kTopkMax = 32;
 constexpr int kCandMax = 128;  // top-k candidates per token kept for exact ranking
-constexpr int kComputeWarps = 8;  // pass 2: two warpgroups of compute warps
-// pass 2 adds a warpgroup that picks the top-k of the previous row tile while the
-// compute warps work on the next one (the importance scratch is double-buffered)
+// selection pass: warpgroups of compute warps (thread = block), each owning
+// kSelRowsPerWg of a row tile's 128 query rows, handled 32 at a time
+constexpr int kComputeWarps = 8;
+constexpr int kSelRowsPerWg = kRows / (kComputeWarps / 4);
+// a warpgroup picks the top-k of the previous row tile while the compute warps work
+// on the next one (the score scratch is double-buffered)
 constexpr int kOutTopkWarps = 4;
 constexpr int kOutTmaWarp = kComputeWarps + kOutTopkWarps;
 constexpr int kOutMmaWarp = kOutTmaWarp + 1;
@@ -519,9 +522,8 @@ __device__ __forceinline__ PairInfo pair_info(int it, int npairs, const int32_t*
   return pi;
 }
 
-// 320 threads x 200 registers fit the SM's register file
 template <int G>
-__global__ void __maxnreg__(200) cmp_fa_tc_kernel(
+__global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap,
     const __grid_constant__ CUtensorMap vcmap, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
     const int32_t* __restrict__ ppre, int S, int64_t N, int hq, int hkv, int btot, float qs2,
@@ -796,7 +798,7 @@ __global__ void __maxnreg__(200) cmp_fa_tc_kernel(
 // MUFU and FMA pipes share them.
 // ---------------------------------------------------------------------------
 constexpr int kSelStages = 4;           // Kc ring depth
-constexpr int kSelPolyRows = 16;        // of the 64 rows a thread handles per key tile, rows on the FMA pipe
+constexpr int kSelPolyRows = kSelRowsPerWg / 4;  // a quarter of a thread's rows of a key tile use the FMA pipe
 
 struct SelSmem {
   uint8_t q[2][kTile];
@@ -812,9 +814,8 @@ struct SelSmem {
   int abort_flag;
 };
 
-// 448 threads x 144 registers fit the SM's register file
 template <int G>
-__global__ void __maxnreg__(144) cmp_sel_tc_kernel(
+__global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kcmap,
     const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu, const int32_t* __restrict__ tpre, int S,
     int hq, int hkv, int btot, float qs2, const float* __restrict__ lse_in, int topk, int32_t* __restrict__ sel,
@@ -925,11 +926,12 @@ __global__ void __maxnreg__(144) cmp_sel_tc_kernel(
       mbar_wait(&sm.mma_done, 0);
     }
   } else if (warp < kComputeWarps) {
-    // ---------------- compute warps (two warpgroups): thread = block of the key tile;
-    // warpgroup wg handles query rows [64 wg, 64 wg + 64) of the tile, in two passes of 32.
+    // ---------------- compute warps: thread = block of the key tile; warpgroup wg handles
+    // query rows [kSelRowsPerWg wg, +kSelRowsPerWg) of the tile, 32 at a time.
+    constexpr int NH = kSelRowsPerWg / 32;
     const int b = threadIdx.x % 128;
     const int wg = warp / 4;
-    const int r0 = 64 * wg;
+    const int r0 = kSelRowsPerWg * wg;
     uint32_t s_count = 0, cw_phase = 0, n_tile = 0;
     for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x, ++n_tile) {
       const TileInfo ti = tile_info(it, ntiles, tpre, S, cu, bcu, G);
@@ -954,9 +956,9 @@ __global__ void __maxnreg__(144) cmp_sel_tc_kernel(
         const int bidx = j * kBN + b;  // block index inside the sequence
         const bool bvalid = bidx < ti.nb;
         const uint32_t taddr = tmem + sb * kBN + ((uint32_t)((warp % 4) * 32) << 16) + r0;
-        float p[2][32];
-        tmem_ld32(taddr, p[0]);
-        tmem_ld32(taddr + 32, p[1]);
+        float p[NH][32];
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) tmem_ld32(taddr + 32 * hh, p[hh]);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -964,7 +966,7 @@ __global__ void __maxnreg__(144) cmp_sel_tc_kernel(
         ++s_count;
         const int grp = j * (kBN / 32) + (warp % 4);  // this warp's 32 blocks form one group
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < NH; ++hh) {
           if (bvalid) {
 #pragma unroll
             for (int r = 0; r < 32; r += 4) {
@@ -1313,7 +1315,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
     const __grid_constant__ CUtensorMap lsemap, const __grid_constant__ CUtensorMap dcmap,
     const __grid_constant__ CUtensorMap wmap, const int32_t* __restrict__ cu, const int32_t* __restrict__ bcu,
     const int32_t* __restrict__ ipre, int S, int hq, int hkv, int btot, float qs2, float scale,
-    float* __restrict__ dkc, float* __restrict__ dvc, int* status) {
+    float* __restrict__ dkc, float* __restrict__ dvc, unsigned long long* __restrict__ fkc,
+    unsigned long long* __restrict__ fvc, int* status) {
   extern __shared__ uint8_t smem_raw[];
   DkvSmem& sm = *reinterpret_cast<DkvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -1584,12 +1587,20 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
       if (lane == 0) mbar_arrive(&sm.acc_empty);
       const int bidx = kt * kBN + b;
       if (bidx < nb && nrt > 0) {
-        float* dst = (wg < 2 ? dkc : dvc) + ((int64_t)g * btot + b0 + bidx) * 64 + 32 * (wg & 1);
+        const int64_t off = ((int64_t)g * btot + b0 + bidx) * 64 + 32 * (wg & 1);
         const float mul = wg < 2 ? scale : 1.f;
+        if (fkc) {  // deterministic: 64-bit fixed-point sums (integer addition is associative)
+          unsigned long long* dst = (wg < 2 ? fkc : fvc) + off;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          atomicAdd(reinterpret_cast<float4*>(dst) + i,
-                    make_float4(acc[4 * i] * mul, acc[4 * i + 1] * mul, acc[4 * i + 2] * mul, acc[4 * i + 3] * mul));
+          for (int i = 0; i < 32; ++i)
+            atomicAdd(dst + i, (unsigned long long)__float2ll_rn(acc[i] * mul * kFixScale));
+        } else {
+          float* dst = (wg < 2 ? dkc : dvc) + off;
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            atomicAdd(reinterpret_cast<float4*>(dst) + i,
+                      make_float4(acc[4 * i] * mul, acc[4 * i + 1] * mul, acc[4 * i + 2] * mul, acc[4 * i + 3] * mul));
+        }
       }
     }
   }
@@ -1707,8 +1718,13 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
              dkv_cnt);
   cudaError_t e = exclusive_scan(dkv_cnt, dkv_pre, a.S + 1, scan_tmp, st);
   if (e != cudaSuccess) return e;
-  cudaMemsetAsync(a.dkc, 0, sizeof(float) * rows_kv * 64, st);
-  cudaMemsetAsync(a.dvc, 0, sizeof(float) * rows_kv * 64, st);
+  if (a.fx_kc) {  // deterministic: the kernel adds fixed-point integers, converted below
+    cudaMemsetAsync(a.fx_kc, 0, sizeof(unsigned long long) * rows_kv * 64, st);
+    cudaMemsetAsync(a.fx_vc, 0, sizeof(unsigned long long) * rows_kv * 64, st);
+  } else {
+    cudaMemsetAsync(a.dkc, 0, sizeof(float) * rows_kv * 64, st);
+    cudaMemsetAsync(a.dvc, 0, sizeof(float) * rows_kv * 64, st);
+  }
   // row constants of the compressed branch: -lse log2(e), -D, w
   CUtensorMap lm, dcm, wm;
   if (!map_rowscalars(&lm, a.rc, a.N, a.hq, G) || !map_rowscalars(&dcm, a.rc + 2 * rows, a.N, a.hq, G) ||
@@ -1716,7 +1732,12 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
     return cudaErrorInvalidValue;
   SSA_LAUNCH("cmp_bwd_dkv_tc_kernel", cmp_bwd_dkv_tc_kernel<G>, sms, kDkvThreads, smem_bytes_dkv(), st, qm, dm, km,
              vm, lm, dcm, wm, a.cu_seqlens, a.blk->cu, dkv_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.dkc, a.dvc,
-             a.status);
+             a.fx_kc, a.fx_vc, a.status);
+  if (a.fx_kc) {
+    e = fix_to_float(a.fx_kc, a.dkc, rows_kv * 64, st);
+    if (e == cudaSuccess) e = fix_to_float(a.fx_vc, a.dvc, rows_kv * 64, st);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 }  // namespace

@@ -107,7 +107,14 @@ struct BwdArgs {
   const void *wk, *wv, *wks, *wvs;
   float *wdk, *wdv;
   const int32_t* wtok;
+  // deterministic mode: 64-bit fixed-point accumulators (2^-32 units) of the compressed
+  // dKc / dVc [Hkv, B, d] and of the selected branch's dK / dV [Nkv, Hkv, d]; null otherwise
+  unsigned long long *fx_kc, *fx_vc, *fx_k, *fx_v;
 };
+
+// Fixed-point unit of the deterministic accumulations: values are added as
+// round(x * 2^32) into 64-bit integers.
+constexpr float kFixScale = 4294967296.f;
 
 bool pool_supported(int dtype, int hkv, int d);
 cudaError_t launch_pool(int dtype, const void* k, const void* v, const ssa_partition* blk, int64_t N, int hkv,
@@ -126,6 +133,8 @@ cudaError_t win_bwd_tc(const BwdArgs& a, int32_t* cnt, int32_t* pre, int32_t* sc
 cudaError_t cmp_bwd_tc(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, int32_t* dkv_pre, int32_t* scan_tmp,
                        int64_t tiles_bound, cudaStream_t st);
 cudaError_t simt_backward(const BwdArgs& a, cudaStream_t st);
+// dst[i] = src[i] / 2^32 (the deterministic accumulators back to fp32)
+cudaError_t fix_to_float(const unsigned long long* src, float* dst, int64_t n, cudaStream_t st);
 
 // 3D-aware block routing: selection by the shortest distance to a block's voxels.
 size_t geo_ws_bytes(int64_t N);

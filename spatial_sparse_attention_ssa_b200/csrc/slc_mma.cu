@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(32 * kSlcWarps) slc_bwd_mma_kernel(
     const int32_t* __restrict__ bptr, const int32_t* __restrict__ bperm, const int32_t* __restrict__ sel, int64_t N,
     int64_t ldk, int hq, int hkv, int topk, float qs2, float scale, const float* __restrict__ lse_in,
     const float* __restrict__ Dc, float* __restrict__ dq_out, float* __restrict__ dk_out,
-    float* __restrict__ dv_out) {
+    float* __restrict__ dv_out, unsigned long long* __restrict__ fk, unsigned long long* __restrict__ fv) {
   extern __shared__ uint8_t smem_raw[];
   SlcBwdSmem& sm = *reinterpret_cast<SlcBwdSmem*>(smem_raw);
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -406,17 +406,27 @@ __global__ void __launch_bounds__(32 * kSlcWarps) slc_bwd_mma_kernel(
           else
             mma_keys_heads(acc, sm.ph[w], sm.pl[w], ds_t, mt, lane);
           float* dst = which == 0 ? dk_out : dv_out;
+          unsigned long long* fdst = which == 0 ? fk : fv;
           const float mul = which == 0 ? scale : 1.f;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const int kk = 16 * mt + gid + 8 * half;
             const int tok = sm.tok[w][kk];
             if (kk < nk) {
-              float* rowp = dst + ((int64_t)tok * hkv + g) * 64 + 2 * tig;
+              const int64_t off = ((int64_t)tok * hkv + g) * 64 + 2 * tig;
+              if (fdst) {  // deterministic: 64-bit fixed-point sums
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                atomicAdd(reinterpret_cast<float2*>(rowp + 8 * i),
-                          make_float2(acc[i][2 * half] * mul, acc[i][2 * half + 1] * mul));
+                for (int i = 0; i < 8; ++i) {
+                  atomicAdd(fdst + off + 8 * i, (unsigned long long)__float2ll_rn(acc[i][2 * half] * mul * kFixScale));
+                  atomicAdd(fdst + off + 8 * i + 1,
+                            (unsigned long long)__float2ll_rn(acc[i][2 * half + 1] * mul * kFixScale));
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  atomicAdd(reinterpret_cast<float2*>(dst + off + 8 * i),
+                            make_float2(acc[i][2 * half] * mul, acc[i][2 * half + 1] * mul));
+              }
             }
           }
         }
@@ -489,11 +499,11 @@ cudaError_t slc_bwd_mma(const BwdArgs& a, cudaStream_t st) {
   if (G == 16)
     SSA_LAUNCH("slc_bwd_mma_kernel", slc_bwd_mma_kernel<16>, grid, 32 * kSlcWarps, smem, st, q, ksp, vsp, dO,
                a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
-               a.lse + rows, a.Dc + rows, a.dq, a.dk, a.dv);
+               a.lse + rows, a.Dc + rows, a.dq, a.dk, a.dv, a.fx_k, a.fx_v);
   else
     SSA_LAUNCH("slc_bwd_mma_kernel", slc_bwd_mma_kernel<8>, grid, 32 * kSlcWarps, smem, st, q, ksp, vsp, dO,
                a.gates, a.gate_mode, a.blk->ptr, a.blk->perm, a.sel, a.N, a.Nkv, a.hq, a.hkv, a.topk, qs2, a.scale,
-               a.lse + rows, a.Dc + rows, a.dq, a.dk, a.dv);
+               a.lse + rows, a.Dc + rows, a.dq, a.dk, a.dv, a.fx_k, a.fx_v);
   return cudaGetLastError();
 }
 

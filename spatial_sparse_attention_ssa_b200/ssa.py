@@ -51,7 +51,7 @@ class Params(ctypes.Structure):
     _fields_ = [("hq", ctypes.c_int32), ("hkv", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("m_cmp", ctypes.c_int32), ("m_win", ctypes.c_int32), ("topk", ctypes.c_int32),
                 ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("gate_mode", ctypes.c_int32),
-                ("selection", ctypes.c_int32), ("conv", ctypes.POINTER(Conv))]
+                ("selection", ctypes.c_int32), ("conv", ctypes.POINTER(Conv)), ("deterministic", ctypes.c_int32)]
 
 
 class Partition(ctypes.Structure):
@@ -298,12 +298,13 @@ class ConvWeights:
 
 
 def make_params(hq, hkv, d, m_cmp, m_win, topk, dtype: torch.dtype, gate_mode: int,
-                scale: float = 0.0, selection: int = SEL_SCORES, conv: ConvWeights | None = None) -> Params:
+                scale: float = 0.0, selection: int = SEL_SCORES, conv: ConvWeights | None = None,
+                deterministic: bool = False) -> Params:
     dt = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32 if dtype == torch.float32 else None
     if dt is None:
         raise ValueError("dtype must be torch.bfloat16 or torch.float32")
     prm = Params(hq, hkv, d, m_cmp, m_win, topk, scale, dt, gate_mode, selection,
-                 ctypes.pointer(conv._c) if conv is not None else None)
+                 ctypes.pointer(conv._c) if conv is not None else None, 1 if deterministic else 0)
     prm._conv = conv  # keeps the weights (and the struct the pointer refers to) alive
     return prm
 
