@@ -17,6 +17,7 @@ the max over ranks.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -36,6 +37,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 SMS = 148
 FP32_LANES_PER_SM = 128
+# DRAM bytes per launch of the compressed backward's kernels at the 131072-token
+# benchmark, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass;
+# profiles/cmp_bwd_dram_gigascale1024_131072.md), valid while the kernels' source text
+# (the backward section of csrc/cmp_tc.cu) has the recorded sha1.
+BWD_TRAFFIC = {"source_sha1": "50ae9d262aa183ccce6e70e4331e8c1248f0bd01",
+               "bytes_per_launch": {"cmp_bwd_dq_tc_kernel": 1177.4e6 + 1023.4e6,
+                                    "cmp_bwd_dkv_tc_kernel": 1179.7e6 + 1.8e6}}
+
+
+def _backward_source_sha1() -> str:
+    path = os.path.join(ROOT, "spatial_sparse_attention_ssa_b200", "csrc", "cmp_tc.cu")
+    with open(path, encoding="utf-8") as f:
+        text = f.read()
+    a = text.index("// backward, dQ (thread = row)")
+    b = text.index("// host side", a)
+    return hashlib.sha1(text[a:b].encode()).hexdigest()
 
 def _args():
     ap = argparse.ArgumentParser()
@@ -142,6 +159,17 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # algorithmic work per kernel (flops / bytes per launch)
 # ---------------------------------------------------------------------------
+
+def _traffic(stage: str, n_tokens: int, row: dict):
+    """DRAM bytes per launch of the stage's kernels (ncu), or None when no capture of the
+    current source at this size exists."""
+    t = BWD_TRAFFIC
+    if stage != "compressed backward" or n_tokens != 131072 or not t["source_sha1"]:
+        return None
+    if _backward_source_sha1() != t["source_sha1"] or set(row["kernels"]) != set(t["bytes_per_launch"]):
+        return None
+    return float(sum(t["bytes_per_launch"].values()))
+
 
 def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
     """Algorithmic work per kernel and per stage (a stage is the kernels of one
@@ -436,11 +464,11 @@ def run_ours(a):
         dom = max(stage_rows, key=lambda k_: stage_rows[k_]["ms"])
         r_ = stage_rows[dom]
         roof = {"kernel": " + ".join(r_["kernels"]), "stage": dom, "bound": "tensor", "achieved": r_["tflops"],
-                "peak": tc_peak, "unit": "TFLOP/s", "frac": r_["tensor_frac"], "traffic": None,
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": r_["tensor_frac"], "traffic": _traffic(dom, n, r_),
                 "peak_source": "%s bf16 dense, burst" % peaks["_source"],
                 "algorithmic_per_launch": r_["flops"], "ms_per_launch": r_["ms"],
                 "note": "the stage's kernels, one launch each, at its algorithmic flops (each contraction of "
-                        "the method once); DRAM traffic of these kernels is from ncu, not measured here"}
+                        "the method once); traffic: ncu DRAM bytes per launch of these kernels (null unless captured on this source at this size)"}
         exp_roof = {"kernel": roof["kernel"], "bound": "mufu", "achieved": r_["exps"] / (r_["ms"] / 1e3) / 1e12,
                     "peak": mufu_peak, "unit": "Texp/s", "frac": r_["mufu_frac"],
                     "peak_source": "derived: %d SMs x 16 ex2/clock x %.0f MHz" % (SMS, mhz),

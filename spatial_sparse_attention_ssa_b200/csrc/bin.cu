@@ -103,6 +103,16 @@ __global__ void scan_sums_kernel(int32_t* sums, int64_t n) {
   }
 }
 
+// Single CTA: exclusive scan of a short array (at most kScanSmallChunks chunks) in one
+// launch; the plans' scans have S + 1 or W + 1 entries, where the launch gaps of the
+// three-kernel form would cost more than the scan.
+constexpr int64_t kScanSmallChunks = 8;
+__global__ void scan_small_kernel(const int32_t* in, int32_t* out, int64_t n) {
+  __shared__ int sh[kScanChunk + 8];
+  int carry = 0;
+  for (int64_t base = 0; base < n; base += kScanChunk) carry += block_scan_chunk(in, out, base, n, carry, sh);
+}
+
 __global__ void scan_apply_kernel(const int32_t* __restrict__ in, int32_t* __restrict__ out, int64_t n,
                                   const int32_t* __restrict__ sums) {
   __shared__ int sh[kScanChunk + 8];
@@ -269,6 +279,10 @@ size_t scan_tmp_ints(int64_t n) { return (size_t)cdiv(n, kScanChunk) + 64; }
 cudaError_t exclusive_scan(const int32_t* in, int32_t* out, int64_t n, int32_t* tmp, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const int64_t nc = cdiv(n, kScanChunk);
+  if (nc <= kScanSmallChunks) {
+    SSA_LAUNCH("scan_small_kernel", scan_small_kernel, 1, kScanThreads, 0, st, in, out, n);
+    return cudaGetLastError();
+  }
   SSA_LAUNCH("scan_reduce_kernel", scan_reduce_kernel, (unsigned)nc, kScanThreads, 0, st, in, n, tmp);
   SSA_LAUNCH("scan_sums_kernel", scan_sums_kernel, 1, kScanThreads, 0, st, tmp, nc);
   SSA_LAUNCH("scan_apply_kernel", scan_apply_kernel, (unsigned)nc, kScanThreads, 0, st, in, out, n, tmp);
