@@ -484,16 +484,17 @@ __device__ void warp_topk_groups(const float* imp, const float* gm, int nb, int 
 // need the high + low split.  The next S of the same tile is issued into the same
 // columns after that product in the single MMA stream, which executes in order.  O
 // (TMEM) is rescaled only when a row's max grows by more than 2^8 since it was last
-// fixed, so p stays below 2^8 otherwise.  The two tiles' softmax work and their MMAs
-// interleave.
+// fixed, so p stays below 2^8 otherwise.  The exponentials of a quarter of each key
+// tile's blocks run on the FMA pipe (ex2_poly2), the rest on the MUFU.  The two tiles'
+// softmax work and their MMAs interleave.
 // ---------------------------------------------------------------------------
 constexpr int kFaStages = 3;                 // Kc / Vc ring depth
 constexpr int kFaSoftmaxWarps = 8;           // warps 0-3: tile A, 4-7: tile B
 constexpr int kFaTmaWarp = kFaSoftmaxWarps;
 constexpr int kFaMmaWarp = kFaSoftmaxWarps + 1;
 constexpr int kFaThreads = 32 * (kFaSoftmaxWarps + 2);
-constexpr int kFaPolyCols = 0;               // columns of a key tile whose exponentials use the FMA pipe
-                                             // (0: this pass is issue-bound, 5.55 ms at 131072 tokens vs 6.19 with 32)
+constexpr int kFaPolyCols = 32;              // columns of a key tile whose exponentials use the FMA pipe
+                                             // (at 131072 tokens: 0 -> 5.04 ms, 32 -> 4.90, 64 -> 5.86)
 constexpr float kFaRescaleLog2 = 8.f;
 
 struct FaSmem {
@@ -791,12 +792,13 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
 // block's score for a token is the sum of its G heads' p, written to a per-CTA
 // scratch together with the maximum of each group of 32 blocks (one warp-wide
 // reduction); a warpgroup picks each token's top-k of the previous row tile from
-// those (warp_topk_groups) while the compute warps work on the next one.  A quarter
-// of each thread's exponentials are evaluated on the FMA pipe (ex2_poly2) so that the
-// MUFU and FMA pipes share them.
+// those (warp_topk_groups) while the compute warps work on the next one.  The
+// exponentials stay on the MUFU (kSelPolyRows = 0): moving a share to the FMA pipe
+// (ex2_poly2) measured slower here.
 // ---------------------------------------------------------------------------
 constexpr int kSelStages = 4;           // Kc ring depth
-constexpr int kSelPolyRows = kSelRowsPerWg / 4;  // a quarter of a thread's rows of a key tile use the FMA pipe
+constexpr int kSelPolyRows = 0;  // rows of a key tile whose exponentials use the FMA pipe (at 131072 tokens:
+                                  // 0 -> 4.87 ms, a quarter -> 5.12, a half -> 5.46)
 
 struct SelSmem {
   uint8_t q[2][kTile];
