@@ -37,13 +37,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 SMS = 148
 FP32_LANES_PER_SM = 128
-# DRAM bytes per launch of the compressed backward's kernels at the 131072-token
+# DRAM bytes per step of the compressed backward's kernels at the 131072-token
 # benchmark, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass;
 # profiles/cmp_bwd_dram_gigascale1024_131072.md), valid while the kernels' source text
 # (the backward section of csrc/cmp_tc.cu) has the recorded sha1.
-BWD_TRAFFIC = {"source_sha1": "50ae9d262aa183ccce6e70e4331e8c1248f0bd01",
-               "bytes_per_launch": {"cmp_bwd_dq_tc_kernel": 1177.4e6 + 1023.4e6,
-                                    "cmp_bwd_dkv_tc_kernel": 1179.7e6 + 1.8e6}}
+BWD_TRAFFIC = {"source_sha1": "aa754fc8a81eeaa6a56e449c60da54af21c20ae5",
+               "bytes_per_step": {"cmp_bwd_dq_tc_kernel": 1177.0e6 + 1024.0e6,
+                                  "to_f16_kernel": 1073.9e6 + 1014.3e6 + 1.2e6,
+                                  "cmp_bwd_dkv_tc_kernel": 1180.7e6 + 2.0e6}}
 
 
 def _backward_source_sha1() -> str:
@@ -166,9 +167,9 @@ def _traffic(stage: str, n_tokens: int, row: dict):
     t = BWD_TRAFFIC
     if stage != "compressed backward" or n_tokens != 131072 or not t["source_sha1"]:
         return None
-    if _backward_source_sha1() != t["source_sha1"] or set(row["kernels"]) != set(t["bytes_per_launch"]):
+    if _backward_source_sha1() != t["source_sha1"] or set(row["kernels"]) != set(t["bytes_per_step"]):
         return None
-    return float(sum(t["bytes_per_launch"].values()))
+    return float(sum(t["bytes_per_step"].values()))
 
 
 def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
@@ -201,8 +202,6 @@ def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
     N, B = w.n, len(bsize)
     # per kernel: (kind, contraction flops, exps) for attention, ("bytes", bytes) for memory kernels
     work = {
-        "cmp_lse_tc_kernel": ("tc", 2 * d * sc_cmp, sc_cmp),
-        "cmp_out_tc_kernel": ("tc", 4 * d * sc_cmp, sc_cmp),
         "cmp_fa_tc_kernel": ("tc", 4 * d * sc_cmp, sc_cmp),
         "cmp_sel_tc_kernel": ("tc", 2 * d * sc_cmp, sc_cmp),
         "cmp_bwd_dq_tc_kernel": ("tc", 6 * d * sc_cmp, sc_cmp),
@@ -215,11 +214,13 @@ def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
         "pool_kernel": ("bytes", 4.0 * N * hkv * d * e + 2.0 * B * hkv * d * e),
         "combine_kernel": ("bytes", 3.0 * N * hq * d * 4 + N * hq * 3 * 4 + N * hq * d * e),
         "bwd_pre_kernel": ("bytes", 3.0 * N * hq * d * 4 + N * hq * d * e + N * hq * 3 * 4 * 3),
+        # fp16 copies of Q, dO and of Kc, Vc for the compressed dK/dV kernel (two launches per step)
+        "to_f16_kernel": ("bytes", 2.0 * 2 * N * hq * d * e + 2.0 * 2 * B * hkv * d * e),
     }
     stages = {
-        "compressed forward": (("cmp_lse_tc_kernel", "cmp_out_tc_kernel", "cmp_fa_tc_kernel", "cmp_sel_tc_kernel"),
-                               6 * d * sc_cmp, 2 * sc_cmp),
-        "compressed backward": (("cmp_bwd_dq_tc_kernel", "cmp_bwd_dkv_tc_kernel"), 10 * d * sc_cmp, sc_cmp),
+        "compressed forward": (("cmp_fa_tc_kernel", "cmp_sel_tc_kernel"), 6 * d * sc_cmp, 2 * sc_cmp),
+        "compressed backward": (("cmp_bwd_dq_tc_kernel", "to_f16_kernel", "cmp_bwd_dkv_tc_kernel"), 10 * d * sc_cmp,
+                                sc_cmp),
         "window forward": (("win_fwd_tc_kernel",), 4 * d * sc_win, sc_win),
         "window backward": (("win_bwd_dq_tc_kernel", "win_bwd_dkv_tc_kernel"), 10 * d * sc_win, sc_win),
         "selected forward": (("slc_fwd_mma_kernel",), 4 * d * sc_slc, sc_slc),
@@ -438,22 +439,23 @@ def run_ours(a):
     per_kernel = {}
     for name, (tot, cnt) in prof.items():
         ms_l = tot / max(cnt, 1)
-        ent = {"ms_per_step": tot / a.steps, "launches": cnt, "ms_per_launch": ms_l}
+        ms_st = tot / a.steps  # the work figures are per step (to_f16_kernel runs twice a step)
+        ent = {"ms_per_step": ms_st, "launches": cnt, "ms_per_launch": ms_l}
         wk = work.get(name)
         if wk is not None and wk[0] == "tc":
-            ent["tflops"] = wk[1] / (ms_l / 1e3) / 1e12
+            ent["tflops"] = wk[1] / (ms_st / 1e3) / 1e12
             ent["tensor_frac"] = ent["tflops"] / tc_peak
-            ent["mufu_frac"] = wk[2] / (ms_l / 1e3) / 1e12 / mufu_peak
+            ent["mufu_frac"] = wk[2] / (ms_st / 1e3) / 1e12 / mufu_peak
         elif wk is not None:
-            ent["gbs"] = wk[1] / (ms_l / 1e3) / 1e9
+            ent["gbs"] = wk[1] / (ms_st / 1e3) / 1e9
             ent["hbm_frac"] = ent["gbs"] / peaks["hbm_gbs"]
         per_kernel[name] = ent
     stage_rows = {}
     for sname, (cands, flops, exps) in stages.items():
-        kernels = [k_ for k_ in cands if k_ in prof]  # the stage's kernels that ran (one launch each per step)
+        kernels = [k_ for k_ in cands if k_ in prof]  # the stage's kernels that ran
         if not kernels:
             continue
-        ms_s = sum(prof[k_][0] / max(prof[k_][1], 1) for k_ in kernels)  # one launch of each per step
+        ms_s = sum(prof[k_][0] / a.steps for k_ in kernels)  # device time of the stage per step
         stage_rows[sname] = {"kernels": list(kernels), "ms": ms_s, "tflops": flops / (ms_s / 1e3) / 1e12,
                              "tensor_frac": flops / (ms_s / 1e3) / 1e12 / tc_peak,
                              "mufu_frac": exps / (ms_s / 1e3) / 1e12 / mufu_peak,
@@ -467,8 +469,9 @@ def run_ours(a):
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": r_["tensor_frac"], "traffic": _traffic(dom, n, r_),
                 "peak_source": "%s bf16 dense, burst" % peaks["_source"],
                 "algorithmic_per_launch": r_["flops"], "ms_per_launch": r_["ms"],
-                "note": "the stage's kernels, one launch each, at its algorithmic flops (each contraction of "
-                        "the method once); traffic: ncu DRAM bytes per launch of these kernels (null unless captured on this source at this size)"}
+                "note": "one step's launches of the stage's kernels at its algorithmic flops (each contraction of "
+                        "the method once); traffic: ncu DRAM bytes of those launches (null unless captured on this "
+                        "source at this size)"}
         exp_roof = {"kernel": roof["kernel"], "bound": "mufu", "achieved": r_["exps"] / (r_["ms"] / 1e3) / 1e12,
                     "peak": mufu_peak, "unit": "Texp/s", "frac": r_["mufu_frac"],
                     "peak_source": "derived: %d SMs x 16 ex2/clock x %.0f MHz" % (SMS, mhz),

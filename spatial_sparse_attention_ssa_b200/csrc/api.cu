@@ -153,6 +153,7 @@ size_t sp_bwd_extra(const ssa_params* p, int64_t Nr) {
 
 struct BwdWs {
   unsigned long long *fx_kc, *fx_vc, *fx_k, *fx_v;
+  void *q16, *do16, *kc16, *vc16;
   float* Dc;
   float* rc;
   float *dkc, *dvc;
@@ -190,6 +191,15 @@ size_t carve_bwd(void* base, const ssa_params* p, int32_t S, int64_t N, int64_t 
     w->fx_v = c.take<unsigned long long>(N * p->hkv * p->d);
   } else {
     w->fx_kc = w->fx_vc = w->fx_k = w->fx_v = nullptr;
+  }
+  if (ssa::cmp_tc_supported(p->dtype, p->d, p->hq, p->hkv, p->topk)) {
+    // fp16 operands of the tensor-core dKc / dVc kernel: Q, dO [N, Hq, d], Kc, Vc [Hkv, B, d]
+    w->q16 = c.take<uint16_t>(N * p->hq * p->d);
+    w->do16 = c.take<uint16_t>(N * p->hq * p->d);
+    w->kc16 = c.take<uint16_t>(p->hkv * B * p->d);
+    w->vc16 = c.take<uint16_t>(p->hkv * B * p->d);
+  } else {
+    w->q16 = w->do16 = w->kc16 = w->vc16 = nullptr;
   }
   return c.used;
 }
@@ -491,6 +501,10 @@ ssa_status backward_common(const ssa_params* p, const int32_t* cu, int32_t S, in
   a.items_cnt = w.ic;
   a.items_pre = w.ip;
   a.scan_tmp = w.st;
+  a.q16 = w.q16;
+  a.do16 = w.do16;
+  a.kc16 = w.kc16;
+  a.vc16 = w.vc16;
   a.has_win = !cross;
   a.wk = k;
   a.wv = v;

@@ -1366,9 +1366,10 @@ cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   e = exclusive_scan(a.items_cnt, a.items_pre, a.S + 1, a.scan_tmp, st);
   if (e != cudaSuccess) return e;
 
+  const bool cmp_tc = a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk) && a.q16;
   SSA_LAUNCH("bwd_pre_kernel", (bwd_pre_kernel<T, D>), grid_1d(rows * C::NT, 256, 148 * 32), 256, 0, st, ob, dout,
              a.gates, a.lse, rows, a.gate_mode, a.has_win ? 3 : 2, a.Dc, a.dgates, a.rc);
-  if (a.use_tc && D == 64 && cmp_tc_supported(a.dtype, D, a.hq, a.hkv, a.topk)) {
+  if (cmp_tc) {
     // 128-row tiles for the tensor-core kernels (tiles_cnt / tiles_pre are free again here)
     SSA_LAUNCH("plan_counts_kernel", plan_counts_kernel, grid_1d(a.S + 1, 256), 256, 0, st, a.cu_seqlens, a.blk->cu,
                a.S, G, 128, 128, kCmpRowChunk, a.tiles_cnt, a.items_cnt);

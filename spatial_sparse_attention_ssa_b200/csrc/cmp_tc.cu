@@ -83,15 +83,6 @@ constexpr int kOutTmaWarp = kComputeWarps + kOutTopkWarps;
 constexpr int kOutMmaWarp = kOutTmaWarp + 1;
 constexpr int kOutThreadsTk = 32 * (kOutMmaWarp + 1);
 
-// Store rows [8c, 8c+8) of block `b` into a P^T tile (MN-major A operand,
-// 128-byte swizzle): row atom a = row / 64 holds 64 rows of one block in a
-// 128-byte line; the 16-byte chunks of line b are XOR-swizzled with b % 8.
-__device__ __forceinline__ void store_pt_chunk(uint8_t* pt, int b, int c, uint4 v) {
-  const int a = c / 8;
-  const int chunk = c % 8;
-  *reinterpret_cast<uint4*>(pt + a * kTile + b * 128 + ((chunk ^ (b & 7)) * 16)) = v;
-}
-
 // (v, id) ranks above (v2, id2): higher score, or equal score and lower id.
 __device__ __forceinline__ bool beats(float v, int id, float v2, int id2) { return v > v2 || (v == v2 && id < id2); }
 
@@ -1282,8 +1273,22 @@ __global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) cmp_bwd_dq_tc_kernel
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// ---------------------------------------------------------------------------
+// backward, dKc / dVc (thread = block): a work item is a 128-block key tile of one
+// (sequence, group) against a chunk of up to kDkvRowTilesPerItem row tiles of 128
+// query rows.  Per row tile: S^T = Kc Q^T and dP^T = Vc dO^T into TMEM; the compute
+// warps turn them into P^T w and dS^T = P^T (w dP - D) and store them back into TMEM
+// as fp16 (round to nearest even); dVc += (P^T w) dO and dKc += dS^T Q take them as
+// the TMEM operand.  Every operand of this kernel is fp16 (kind::f16 wants A and B of
+// one type): Q, dO, Kc and Vc come as exact fp16 copies of the bf16 inputs, made by
+// the backward preamble.  fp16's 11-bit significand is what keeps the key gradients
+// accurate: they sum P w dO and dS Q over millions of query rows, and a bf16 P (8
+// bits) carries a rounding error of about 2^-9 relative into sums of magnitude ~10
+// coherently, while fp16 brings it 8x lower (a fixed-point or high + low split costs
+// twice the products).
+// ---------------------------------------------------------------------------
 constexpr int kDkvRowTilesPerItem = 128;
-constexpr int kDkvQStages = 3;  // Q / dO / row-constant stages: each row tile is used once per item
+constexpr int kDkvQStages = 4;  // Q / dO / row-constant stages: each row tile is used once per item
 // four compute warpgroups of 32 rows each (thread = block): enough warps to hide
 // the latency of the per-score arithmetic
 constexpr int kDkvComputeWarps = 16;
@@ -1294,10 +1299,6 @@ struct DkvSmem {
   uint8_t vc[kTile];
   uint8_t q[kDkvQStages][kTile];
   uint8_t dout[kDkvQStages][kTile];
-  // low bf16 parts of P^T w and dS^T [blocks, 128 rows] (K-major A operands, two
-  // 64-row atoms each); the high parts are TMEM operands
-  uint8_t plo[2 * kTile];
-  uint8_t dslo[2 * kTile];
   // row constants, TMA destinations (128-byte aligned): -lse log2(e), -D, w
   __align__(128) float lse2[kDkvQStages][kRows];
   __align__(128) float Dr[kDkvQStages][kRows];
@@ -1416,8 +1417,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
   } else if (warp == kDkvComputeWarps + 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      const uint32_t id_s = idesc_bf16(kBN, kRows);              // S^T, dP^T [blocks, rows]
-      const uint32_t id_a = idesc_bf16(kBN, 64, false, true);     // dKc / dVc [blocks, 64] += X^T[blocks, rows] Y
+      const uint32_t id_s = idesc_bf16(kBN, kRows, false, false, true);  // S^T, dP^T [blocks, rows], fp16
+      const uint32_t id_a = idesc_bf16(kBN, 64, false, true, true);      // dKc / dVc [blocks, 64] += X^T Y, fp16
       uint32_t kv_count = 0, q_count = 0, sdp_count = 0, pds_count = 0, acc_count = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
@@ -1454,13 +1455,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kRows / 16; ++k) {
-            const uint64_t bdo = sdesc_mnmajor_sw128(sm.dout[qb], 2048 * k, kTile);
-            const uint64_t bq = sdesc_mnmajor_sw128(sm.q[qb], 2048 * k, kTile);
-            const uint32_t lo_off = (k / 4) * kTile;
-            mma_bf16_ts(tm_dv, tm_p + 8 * k, bdo, id_a, i > 0 || k > 0);
-            mma_bf16_ss(tm_dv, sdesc_kmajor_sw128(sm.plo + lo_off, 32 * (k % 4)), bdo, id_a, true);
-            mma_bf16_ts(tm_dk, tm_ds + 8 * k, bq, id_a, i > 0 || k > 0);
-            mma_bf16_ss(tm_dk, sdesc_kmajor_sw128(sm.dslo + lo_off, 32 * (k % 4)), bq, id_a, true);
+            mma_bf16_ts(tm_dv, tm_p + 8 * k, sdesc_mnmajor_sw128(sm.dout[qb], 2048 * k, kTile), id_a, i > 0 || k > 0);
+            mma_bf16_ts(tm_dk, tm_ds + 8 * k, sdesc_mnmajor_sw128(sm.q[qb], 2048 * k, kTile), id_a, i > 0 || k > 0);
           }
           mma_commit(&sm.pds_empty);
           mma_commit(&sm.q_empty[qb]);
@@ -1502,10 +1498,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
         const int nvr = (int)min((int64_t)kRows, (int64_t)(t_end - t_first) * G) - r0;  // valid rows of this warpgroup
         const float2 qs = make_float2(qs2, qs2);
         // the warpgroup's 32 rows in two passes of 16; S^T / dP^T are released after
-        // the second read, P^T w / dS^T written once the MMAs of the previous tile
-        // consumed them.  P^T w and dS^T go out as bf16 high + low parts: sums over
-        // many rows of near-equal probabilities would otherwise carry the bf16
-        // rounding of each term coherently (a 2^-9 relative bias).
+        // the second read, P^T w / dS^T (fp16) written once the MMAs of the previous
+        // tile consumed them.
         bool ok_half = true;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -1523,7 +1517,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
 #pragma unroll
             for (int c = 0; c < 16; ++c) sv[c] = c < nvh ? sv[c] : -CUDART_INF_F;
           }
-          uint32_t pw[8], dsv[8], pwl[8], dsl[8];
+          uint32_t pw[8], dsv[8];
 #pragma unroll
           for (int c = 0; c < 16; c += 4) {
             const int rr = r0 + 16 * hh + c;
@@ -1533,12 +1527,10 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
             const float2 wa = make_float2(w4.x, w4.y), wb = make_float2(w4.z, w4.w);
             const float2 pa = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, make_float2(l4.x, l4.y)));
             const float2 pb = ex2x2(ffma2(make_float2(sv[c + 2], sv[c + 3]), qs, make_float2(l4.z, l4.w)));
-            split2(fmul2(pa, wa), pw[c / 2], pwl[c / 2]);
-            split2(fmul2(pb, wb), pw[c / 2 + 1], pwl[c / 2 + 1]);
-            split2(fmul2(pa, ffma2(wa, make_float2(dp[c], dp[c + 1]), make_float2(d4.x, d4.y))), dsv[c / 2],
-                   dsl[c / 2]);
-            split2(fmul2(pb, ffma2(wb, make_float2(dp[c + 2], dp[c + 3]), make_float2(d4.z, d4.w))),
-                   dsv[c / 2 + 1], dsl[c / 2 + 1]);
+            pw[c / 2] = pack_f16x2(fmul2(pa, wa));
+            pw[c / 2 + 1] = pack_f16x2(fmul2(pb, wb));
+            dsv[c / 2] = pack_f16x2(fmul2(pa, ffma2(wa, make_float2(dp[c], dp[c + 1]), make_float2(d4.x, d4.y))));
+            dsv[c / 2 + 1] = pack_f16x2(fmul2(pb, ffma2(wb, make_float2(dp[c + 2], dp[c + 3]), make_float2(d4.z, d4.w))));
           }
           if (hh == 0) {
             if (!mbar_wait_warp(&sm.pds_empty, (pds_count & 1) ^ 1)) {
@@ -1547,22 +1539,15 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
             }
             tc_fence_after();
           }
-          // rows [r0 + 16 hh, +16): packed TMEM columns [r0/2 + 8 hh, +8), SMEM 8-row chunks 2 (r0/16 + hh) + {0, 1}
+          // rows [r0 + 16 hh, +16): packed TMEM columns [r0/2 + 8 hh, +8)
           tmem_st8(tm_p + lane_off + r0 / 2 + 8 * hh, pw);
           tmem_st8(tm_ds + lane_off + r0 / 2 + 8 * hh, dsv);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int ch = r0 / 8 + 2 * hh + c;
-            store_pt_chunk(sm.plo, b, ch, make_uint4(pwl[4 * c], pwl[4 * c + 1], pwl[4 * c + 2], pwl[4 * c + 3]));
-            store_pt_chunk(sm.dslo, b, ch, make_uint4(dsl[4 * c], dsl[4 * c + 1], dsl[4 * c + 2], dsl[4 * c + 3]));
-          }
         }
         if (!ok_half) {
           ok = false;
           break;
         }
         ++sdp_count;
-        fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -1607,6 +1592,29 @@ __global__ void __launch_bounds__(kDkvThreads, 1) cmp_bwd_dkv_tc_kernel(
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// Two bf16 arrays of n8 x 8 values -> fp16 copies (exact down to 2^-14, where fp16
+// turns subnormal), eight values per thread and step: the operands of the dKc / dVc
+// kernel (Q and dO; Kc and Vc).
+__global__ void to_f16_kernel(const uint4* __restrict__ a, const uint4* __restrict__ b, uint4* __restrict__ a16,
+                              uint4* __restrict__ b16, int64_t n8) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 2 * n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const bool second = i >= n8;
+    const int64_t j = second ? i - n8 : i;
+    const uint4 x = __ldcs((second ? b : a) + j);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      o[c] = pack_f16x2(make_float2(__uint_as_float(w[c] << 16), __uint_as_float(w[c] & 0xffff0000u)));
+    (second ? b16 : a16)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+int to_f16_grid(int64_t n8, int sms) {
+  const int64_t blocks = (2 * n8 + 255) / 256;
+  return (int)(blocks < 8 * (int64_t)sms ? (blocks > 0 ? blocks : 1) : 8 * (int64_t)sms);
 }
 
 // ---------------------------------------------------------------------------
@@ -1689,12 +1697,11 @@ size_t smem_bytes_dkv() { return sizeof(DkvSmem) + 1024; }
 template <int G>
 cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt, int32_t* dkv_pre,
                          int32_t* scan_tmp, int64_t tiles_bound, cudaStream_t st) {
-  CUtensorMap qm, dm, km, vm;
+  CUtensorMap qm, dm;
   const int64_t rows_kv = (int64_t)a.hkv * a.blk->count;
   CUtensorMap km64, vm64;  // 64-block key tiles of the dQ kernel
-  if (!map_q(&qm, a.q, a.N, a.hq, G) || !map_q(&dm, a.dout, a.N, a.hq, G) || !map_rows64(&km, a.kc, rows_kv) ||
-      !map_rows64(&vm, a.vc, rows_kv) || !map_rows64(&km64, a.kc, rows_kv, kDqBN) ||
-      !map_rows64(&vm64, a.vc, rows_kv, kDqBN))
+  if (!a.q16 || !map_q(&qm, a.q, a.N, a.hq, G) || !map_q(&dm, a.dout, a.N, a.hq, G) ||
+      !map_rows64(&km64, a.kc, rows_kv, kDqBN) || !map_rows64(&vm64, a.vc, rows_kv, kDqBN))
     return cudaErrorInvalidValue;
   static bool attr_done = false;
   if (!attr_done) {
@@ -1730,9 +1737,20 @@ cudaError_t cmp_bwd_tc_g(const BwdArgs& a, const int32_t* tpre, int32_t* dkv_cnt
   if (!map_rowscalars(&lm, a.rc, a.N, a.hq, G) || !map_rowscalars(&dcm, a.rc + 2 * rows, a.N, a.hq, G) ||
       !map_rowscalars(&wm, a.rc + rows, a.N, a.hq, G))
     return cudaErrorInvalidValue;
-  SSA_LAUNCH("cmp_bwd_dkv_tc_kernel", cmp_bwd_dkv_tc_kernel<G>, sms, kDkvThreads, smem_bytes_dkv(), st, qm, dm, km,
-             vm, lm, dcm, wm, a.cu_seqlens, a.blk->cu, dkv_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.dkc, a.dvc,
-             a.fx_kc, a.fx_vc, a.status);
+  // the fp16 operands: Q, dO [N, Hq, 64] and Kc, Vc [Hkv, B, 64].  The maps move
+  // 2-byte elements without conversion, so the bf16 map layout serves fp16.
+  const int64_t q8 = rows * 64 / 8, kv8 = rows_kv * 64 / 8;
+  SSA_LAUNCH("to_f16_kernel", to_f16_kernel, to_f16_grid(q8, sms), 256, 0, st, static_cast<const uint4*>(a.q),
+             static_cast<const uint4*>(a.dout), static_cast<uint4*>(a.q16), static_cast<uint4*>(a.do16), q8);
+  SSA_LAUNCH("to_f16_kernel", to_f16_kernel, to_f16_grid(kv8, sms), 256, 0, st, static_cast<const uint4*>(a.kc),
+             static_cast<const uint4*>(a.vc), static_cast<uint4*>(a.kc16), static_cast<uint4*>(a.vc16), kv8);
+  CUtensorMap q16m, d16m, k16m, v16m;
+  if (!map_q(&q16m, a.q16, a.N, a.hq, G) || !map_q(&d16m, a.do16, a.N, a.hq, G) || !map_rows64(&k16m, a.kc16, rows_kv) ||
+      !map_rows64(&v16m, a.vc16, rows_kv))
+    return cudaErrorInvalidValue;
+  SSA_LAUNCH("cmp_bwd_dkv_tc_kernel", cmp_bwd_dkv_tc_kernel<G>, sms, kDkvThreads, smem_bytes_dkv(), st, q16m, d16m,
+             k16m, v16m, lm, dcm, wm, a.cu_seqlens, a.blk->cu, dkv_pre, a.S, a.hq, a.hkv, btot, qs2, a.scale, a.dkc,
+             a.dvc, a.fx_kc, a.fx_vc, a.status);
   if (a.fx_kc) {
     e = fix_to_float(a.fx_kc, a.dkc, rows_kv * 64, st);
     if (e == cudaSuccess) e = fix_to_float(a.fx_vc, a.dvc, rows_kv * 64, st);

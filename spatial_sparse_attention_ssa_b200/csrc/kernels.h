@@ -110,6 +110,9 @@ struct BwdArgs {
   // deterministic mode: 64-bit fixed-point accumulators (2^-32 units) of the compressed
   // dKc / dVc [Hkv, B, d] and of the selected branch's dK / dV [Nkv, Hkv, d]; null otherwise
   unsigned long long *fx_kc, *fx_vc, *fx_k, *fx_v;
+  // fp16 copies of Q, dO [N, Hq, d] and Kc, Vc [Hkv, B, d] for the tensor-core dKc / dVc
+  // kernel (written by the backward preamble); null where that kernel does not run
+  void *q16, *do16, *kc16, *vc16;
 };
 
 // Fixed-point unit of the deterministic accumulations: values are added as

@@ -1,11 +1,12 @@
 // Blackwell (sm_100a) building blocks written from the PTX ISA: TMA tensor
-// loads, mbarriers with bounded waits, TMEM allocation, tcgen05.mma (bf16 in,
-// fp32 accumulate) with shared-memory matrix descriptors, and TMEM loads.
+// loads, mbarriers with bounded waits, TMEM allocation, tcgen05.mma (bf16 or fp16
+// in, fp32 accumulate) with shared-memory matrix descriptors, and TMEM loads.
 // Internal to libssa.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -228,11 +229,13 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(const void* tile, uint32
   return d;
 }
 
-// Instruction descriptor: D fp32, A/B bf16, both K-major unless stated, M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major = false, bool b_mn_major = false) {
+// Instruction descriptor of kind::f16: D fp32, A and B both bf16 (or both fp16 when
+// `fp16`), both K-major unless stated, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major = false, bool b_mn_major = false,
+                                                 bool fp16 = false) {
   return (1u << 4)                          // D format: f32
-         | (1u << 7)                        // A format: bf16
-         | (1u << 10)                       // B format: bf16
+         | ((fp16 ? 0u : 1u) << 7)          // A format: bf16 (1) or f16 (0)
+         | ((fp16 ? 0u : 1u) << 10)         // B format: the same as A
          | ((a_mn_major ? 1u : 0u) << 15)   // A major
          | ((b_mn_major ? 1u : 0u) << 16)   // B major
          | ((uint32_t)(N >> 3) << 17)       // N / 8
@@ -314,6 +317,11 @@ __device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
   const float2 r = ffma2(h, make_float2(-1.f, -1.f), x);
   hi = __byte_perm(xa, xb, 0x7632);
   lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+}
+// x as one fp16 pair (round to nearest even), x.x in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float2 x) {
+  const __half2 h = __floats2half2_rn(x.x, x.y);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 // x as one bf16 pair, rounded half away from zero (integer instructions only).
 __device__ __forceinline__ uint32_t pack2(float2 x) {

@@ -9,9 +9,10 @@
 // group); the tokens' Q (and dO) rows and per-row scalars are gathered by
 // per-token TMA boxes.  Key tiles are 128 rows of K_s / V_s.
 //   win_fwd_tc:     thread = row; S = Q K^T, online softmax across key tiles
-//                   (O in TMEM rescaled when the row max grows), P (bf16 hi+lo)
-//                   as the TMEM A operand of O += P V.
-//   win_bwd_dq_tc:  thread = row; S, dP = dO V^T; dS (hi+lo) -> dQ += dS K.
+//                   (O in TMEM rescaled when the row max grows), P (one bf16 per
+//                   key: a row's sum over its own window's keys) as the TMEM A
+//                   operand of O += P V.
+//   win_bwd_dq_tc:  thread = row; S, dP = dO V^T; dS (bf16) -> dQ += dS K.
 //   win_bwd_dkv_tc: thread = key; S^T = K Q^T, dP^T = V dO^T over the window's
 //                   row tiles; dV += (P^T w) dO, dK += dS^T Q; adds into dK/dV.
 // Roles: compute warps (thread <-> TMEM lane), one TMA warp, one MMA warp.
@@ -137,8 +138,8 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  // TMEM columns: S [0,128), P hi [128,192), P lo [192,256), O [256,320)
-  const uint32_t tm_s = tmem, tm_ph = tmem + 128, tm_pl = tmem + 192, tm_o = tmem + 256;
+  // TMEM columns: S [0,128), P [128,192), O [256,320)
+  const uint32_t tm_s = tmem, tm_ph = tmem + 128, tm_o = tmem + 256;
 
   if (warp == 4) {
     // ---------------- producer: gathered Q per item; (K, V) per key tile
@@ -214,7 +215,6 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
           for (int k = 0; k < nks; ++k) {
             const uint64_t bdesc = sdesc_mnmajor_sw128(sm.v[st], 2048 * k, kTile);
             mma_bf16_ts(tm_o, tm_ph + 8 * k, bdesc, id_o, kt > 0 || k > 0);
-            mma_bf16_ts(tm_o, tm_pl + 8 * k, bdesc, id_o, true);
           }
           mma_commit(&sm.pv_done);
           mma_commit(&sm.kv_empty[st]);
@@ -283,19 +283,18 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
         m = mn;
         const float2 qs = make_float2(qs2, qs2), nm = make_float2(-m, -m);
         float2 lsum = make_float2(0.f, 0.f);
-        uint32_t hi[64], lo[64];
+        uint32_t hi[64];
 #pragma unroll
         for (int c = 0; c < kKT; c += 2) {
           const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nm));
           lsum = fadd2(lsum, p);
-          split2(p, hi[c / 2], lo[c / 2]);
+          hi[c / 2] = pack2(p);
         }
         l += lsum.x + lsum.y;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 64; c += 16) {
           tmem_st16(tm_ph + lane_off + c, hi + c);
-          tmem_st16(tm_pl + lane_off + c, lo + c);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -393,8 +392,8 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  // TMEM columns: S [0,128), dP [128,256), dS hi [256,320), dS lo [320,384), dQ [384,448)
-  const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dsh = tmem + 256, tm_dsl = tmem + 320, tm_dq = tmem + 384;
+  // TMEM columns: S [0,128), dP [128,256), dS [256,320), dQ [384,448)
+  const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dsh = tmem + 256, tm_dq = tmem + 384;
 
   if (warp == 4) {
     // ---------------- producer: gathered Q, dO, row scalars per item; (K, V) per key tile
@@ -478,7 +477,6 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
           for (int k = 0; k < nks; ++k) {
             const uint64_t bdesc = sdesc_mnmajor_sw128(sm.k[st], 2048 * k, kTile);
             mma_bf16_ts(tm_dq, tm_dsh + 8 * k, bdesc, id_q, kt > 0 || k > 0);
-            mma_bf16_ts(tm_dq, tm_dsl + 8 * k, bdesc, id_q, true);
           }
           mma_commit(&sm.ds_empty);
           mma_commit(&sm.kv_empty[st]);
@@ -519,7 +517,7 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
         // only the 32-key chunks that hold keys of the window take part (vc keys)
         const int vc = min(kKT, x.nw - kt * kKT);
         const int nch = (vc + 31) / 32;
-        uint32_t hi[64], lo[64];
+        uint32_t hi[64];
 #pragma unroll
         for (int ch = 0; ch < kKT / 32; ++ch) {
           if (ch < nch) {
@@ -536,7 +534,7 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
             for (int c = 0; c < 32; c += 2) {
               const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nl2));
               const float2 d = fmul2(p, ffma2(w2, make_float2(dp[c], dp[c + 1]), nd2));
-              split2(d, hi[(32 * ch + c) / 2], lo[(32 * ch + c) / 2]);
+              hi[(32 * ch + c) / 2] = pack2(d);
             }
           }
         }
@@ -550,7 +548,6 @@ __global__ void __launch_bounds__(192, 1) win_bwd_dq_tc_kernel(
         for (int ch = 0; ch < kKT / 32; ++ch) {
           if (ch < nch) {
             tmem_st16(tm_dsh + lane_off + 16 * ch, hi + 16 * ch);
-            tmem_st16(tm_dsl + lane_off + 16 * ch, lo + 16 * ch);
           }
         }
         tmem_st_wait();

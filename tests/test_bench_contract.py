@@ -56,8 +56,8 @@ def test_algorithmic_work_counts_scores_by_brute_force():
             slc += sum(blk["ptr"][b + 1] - blk["ptr"][b] for b in sel[t, h // G] if b >= 0)
             wnd += int((win["id"] == win["id"][t]).sum())  # every token of its window
     assert scores == {"cmp": float(cmp), "slc": float(slc), "win": float(wnd)}
-    for name, per_score in (("cmp_lse_tc_kernel", 1), ("cmp_out_tc_kernel", 2), ("cmp_bwd_dq_tc_kernel", 3),
-                            ("cmp_bwd_dkv_tc_kernel", 4), ("cmp_fa_tc_kernel", 2), ("cmp_sel_tc_kernel", 1)):
+    for name, per_score in (("cmp_bwd_dq_tc_kernel", 3), ("cmp_bwd_dkv_tc_kernel", 4), ("cmp_fa_tc_kernel", 2),
+                            ("cmp_sel_tc_kernel", 1)):
         assert work[name][1] == 2 * w.d * per_score * cmp, name
     # stages count each contraction of the method once: the compressed forward needs S for the
     # normaliser, S again for the selection's final probabilities and P V (6d); every backward
