@@ -244,22 +244,29 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
       for (int kt = 0; kt < nkt; ++kt) {
         if (!mbar_wait_warp(&sm.s_full, s_count & 1)) { ok = false; break; }
         tc_fence_after();
+        // only the 32-key chunks that hold keys of the window are read and exponentiated
+        // (windows average ~56 tokens); nch is the same for the whole warp
+        const int vc = min(kKT, x.nw - kt * kKT);
+        const int nch = (vc + 31) / 32;
         float sv[kKT];
 #pragma unroll
-        for (int c = 0; c < kKT; c += 32) tmem_ld32(tm_s + lane_off + c, sv + c);
+        for (int ch = 0; ch < kKT / 32; ++ch)
+          if (ch < nch) tmem_ld32(tm_s + lane_off + 32 * ch, sv + 32 * ch);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_empty);
         ++s_count;
-        const int vc = min(kKT, x.nw - kt * kKT);
-        if (vc < kKT) {  // keys past the window
 #pragma unroll
-          for (int c = 0; c < kKT; ++c) sv[c] = c < vc ? sv[c] : -CUDART_INF_F;
-        }
-        float cm = sv[0];
+        for (int c = 0; c < kKT; ++c) sv[c] = c < vc ? sv[c] : -CUDART_INF_F;  // keys past the window
+        // row max as 8 independent chains
+        float mx8[8];
 #pragma unroll
-        for (int c = 1; c < kKT; ++c) cm = fmaxf(cm, sv[c]);
+        for (int c = 0; c < 8; ++c) mx8[c] = sv[c];
+#pragma unroll
+        for (int c = 8; c < kKT; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], sv[c]);
+        const float cm = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float mn = fmaxf(m, cm * qs2);  // qs2 > 0
         // the previous P V must be done before P is overwritten (and before O is rescaled)
         if (kt > 0 && !mbar_wait_warp(&sm.pv_done, (p_count - 1) & 1)) { ok = false; break; }
@@ -285,17 +292,21 @@ __global__ void __launch_bounds__(192, 1) win_fwd_tc_kernel(
         float2 lsum = make_float2(0.f, 0.f);
         uint32_t hi[64];
 #pragma unroll
-        for (int c = 0; c < kKT; c += 2) {
-          const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nm));
-          lsum = fadd2(lsum, p);
-          hi[c / 2] = pack2(p);
+        for (int ch = 0; ch < kKT / 32; ++ch) {
+          if (ch < nch) {
+#pragma unroll
+            for (int c = 32 * ch; c < 32 * ch + 32; c += 2) {
+              const float2 p = ex2x2(ffma2(make_float2(sv[c], sv[c + 1]), qs, nm));
+              lsum = fadd2(lsum, p);
+              hi[c / 2] = pack2(p);
+            }
+          }
         }
         l += lsum.x + lsum.y;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 64; c += 16) {
-          tmem_st16(tm_ph + lane_off + c, hi + c);
-        }
+        for (int ch = 0; ch < kKT / 32; ++ch)
+          if (ch < nch) tmem_st16(tm_ph + lane_off + 16 * ch, hi + 16 * ch);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
