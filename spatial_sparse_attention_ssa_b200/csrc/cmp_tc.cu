@@ -948,16 +948,24 @@ __global__ void __launch_bounds__(kOutThreadsTk, 1) cmp_sel_tc_kernel(
         const bool bvalid = bidx < ti.nb;
         const uint32_t taddr = tmem + sb * kBN + ((uint32_t)((warp % 4) * 32) << 16) + r0;
         float p[NH][32];
-#pragma unroll
-        for (int hh = 0; hh < NH; ++hh) tmem_ld32(taddr + 32 * hh, p[hh]);
+        tmem_ld32(taddr, p[0]);
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
         ++s_count;
         const int grp = j * (kBN / 32) + (warp % 4);  // this warp's 32 blocks form one group
 #pragma unroll
         for (int hh = 0; hh < NH; ++hh) {
+          // the next 32 rows land while this half is processed
+          if (hh > 0) {
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) asm volatile("" : "+f"(p[hh][i]));  // no use of p[hh] above the wait
+          }
+          if (hh == NH - 1) {  // every row of this S buffer is in registers: release it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+          }
+          if (hh + 1 < NH) tmem_ld32(taddr + 32 * (hh + 1), p[hh + 1]);
           if (bvalid) {
 #pragma unroll
             for (int r = 0; r < 32; r += 4) {
