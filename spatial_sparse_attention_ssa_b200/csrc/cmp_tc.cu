@@ -464,44 +464,50 @@ __device__ void warp_topk_groups(const float* imp, const float* gm, int nb, int 
 // ---------------------------------------------------------------------------
 // output pass (thread = row): flash attention of every query row over all compressed
 // blocks of its sequence, producing o_cmp and lse.  A work unit is a pair of 128-row
-// Q tiles (A, B) of the same (sequence, group), so each Kc / Vc tile is loaded once
-// for 256 rows.  One warpgroup per Q tile keeps its rows' running max m and sum l
-// (log2 domain, scale folded in); S of a key tile lands in TMEM, p = 2^(s qs2 - m)
-// is written back over S as one bf16 per block (blocks 16c .. 16c+15 packed in columns
-// 8c .. 8c+7) and consumed by O += P Vc with P as the TMEM operand.  A single bf16 is
-// enough here: each row's o_cmp is one sum over the blocks of its own sequence, and
-// the rounding (2^-9 relative per probability, unbiased) moves it by about 1e-4 at the
-// benchmark's sizes, against the sums over millions of rows in the key gradients that
-// need the high + low split.  The next S of the same tile is issued into the same
-// columns after that product in the single MMA stream, which executes in order.  O
-// (TMEM) is rescaled only when a row's max grows by more than 2^8 since it was last
-// fixed, so p stays below 2^8 otherwise.  The exponentials of a quarter of each key
-// tile's blocks run on the FMA pipe (ex2_poly2), the rest on the MUFU.  The two tiles'
-// softmax work and their MMAs interleave.
+// Q tiles (sides A, B) of the same (sequence, group), so each Kc / Vc tile of kFaBN
+// blocks is loaded once for 256 rows.  One warpgroup per side keeps its rows' running
+// max m and sum l (log2 domain, scale folded in).  Per side, S is double-buffered in
+// TMEM (two kFaBN-column buffers, then O: 2 x 96 + 64 = 256 columns, 512 for both
+// sides): the S of step g + 2 is issued into buffer g % 2 right after P V(g) has been
+// issued there (the MMA stream of one thread executes in order), so the tensor pipe
+// computes it while the softmax warps work on step g + 1.  p = 2^(s qs2 - m) goes back
+// into its S buffer as one bf16 per block (blocks 16c .. 16c+15 in columns 8c .. 8c+7)
+// and feeds O += P Vc as the TMEM operand.  A single bf16 is enough here: each row's
+// o_cmp is one sum over the blocks of its own sequence, and the rounding (2^-9 relative
+// per probability, unbiased) moves it by about 1e-4 at the benchmark's sizes, against
+// the sums over millions of rows in the key gradients.  O (TMEM) is rescaled only when
+// a row's max grows by more than 2^8 since it was last fixed, so p stays below 2^8
+// otherwise.  The exponentials of a quarter of each key tile's blocks run on the FMA
+// pipe (ex2_poly2), the rest on the MUFU.  Steps are counted per side across the
+// CTA's pairs (g), which sets the buffer (g % 2) and the barrier phases.
 // ---------------------------------------------------------------------------
-constexpr int kFaStages = 3;                 // Kc / Vc ring depth
-constexpr int kFaSoftmaxWarps = 8;           // warps 0-3: tile A, 4-7: tile B
+constexpr int kFaBN = 96;                    // compressed blocks per key tile
+constexpr int kFaStages = 4;                 // Kc / Vc ring depth (steps g, g + 1, g + 2 in use)
+constexpr int kFaSoftmaxWarps = 8;           // warps 0-3: side A, 4-7: side B
 constexpr int kFaTmaWarp = kFaSoftmaxWarps;
 constexpr int kFaMmaWarp = kFaSoftmaxWarps + 1;
 constexpr int kFaThreads = 32 * (kFaSoftmaxWarps + 2);
-constexpr int kFaPolyCols = 32;              // columns of a key tile whose exponentials use the FMA pipe
-                                             // (at 131072 tokens: 0 -> 5.04 ms, 32 -> 4.90, 64 -> 5.86)
+constexpr int kFaKvTile = kFaBN * 128;       // bytes of a [kFaBN, 64] bf16 tile
+constexpr int kFaSideCols = 2 * kFaBN + 64;  // TMEM per side: S buffers 0 and 1, O
+constexpr int kFaPolyCols = 24;              // blocks of a key tile whose exponentials use the FMA pipe
 constexpr float kFaRescaleLog2 = 8.f;
+static_assert(2 * kFaSideCols <= 512 && kFaBN % 32 == 0, "TMEM");
 
 struct FaSmem {
-  uint8_t q[2][2][kTile];  // [buffer][tile A / B]
-  uint8_t kc[kFaStages][kTile];
-  uint8_t vc[kFaStages][kTile];
+  uint8_t q[2][2][kTile];  // [buffer][side A / B]
+  uint8_t kc[kFaStages][kFaKvTile];
+  uint8_t vc[kFaStages][kFaKvTile];
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[kFaStages], kv_empty[kFaStages];
-  uint64_t s_full[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t s_full[2][2], p_full[2][2];  // [side][S buffer]
+  uint64_t pv_done[2], o_full[2], o_empty[2];
   uint64_t mma_done;
   uint32_t tmem;
   int abort_flag;
 };
 
 struct PairInfo {
-  int g, s, t0, t_end, b0, nb;  // t0: first token of tile A; tile B starts 128/G tokens later
+  int g, s, t0, t_end, b0, nb;  // t0: first token of side A; side B starts 128/G tokens later
 };
 
 __device__ __forceinline__ PairInfo pair_info(int it, int npairs, const int32_t* ppre, int S, const int32_t* cu,
@@ -533,11 +539,13 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], 4);
       mbar_init(&sm.pv_done[i], 1);
       mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.o_empty[i], 4);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&sm.s_full[i][b], 1);
+        mbar_init(&sm.p_full[i][b], 4);
+      }
     }
     for (int i = 0; i < kFaStages; ++i) {
       mbar_init(&sm.kv_full[i], 1);
@@ -571,18 +579,18 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
         if (!mbar_wait(&sm.q_empty[qb], ((q_count / 2) & 1) ^ 1)) { record_timeout(status, &sm.abort_flag); break; }
         mbar_expect_tx(&sm.q_full[qb], 2 * kTile);
         tma_load_3d(sm.q[qb][0], &qmap, &sm.q_full[qb], 0, pi.g * G, pi.t0);
-        // tile B: rows past the last token are never used; keep its box inside the tensor
+        // side B: rows past the last token are never used; keep its box inside the tensor
         const int tb = pi.t0 + TPT < N ? pi.t0 + TPT : pi.t0;
         tma_load_3d(sm.q[qb][1], &qmap, &sm.q_full[qb], 0, pi.g * G, tb);
         ++q_count;
-        const int nbt = (pi.nb + kBN - 1) / kBN;
+        const int nbt = (pi.nb + kFaBN - 1) / kFaBN;
         bool ok = true;
         for (int j = 0; j < nbt; ++j) {
           const int st = kv_count % kFaStages;
           const uint32_t ph = (kv_count / kFaStages) & 1;
           if (!mbar_wait(&sm.kv_empty[st], ph ^ 1)) { record_timeout(status, &sm.abort_flag); ok = false; break; }
-          mbar_expect_tx(&sm.kv_full[st], 2 * kTile);
-          const int row = pi.g * btot + pi.b0 + j * kBN;
+          mbar_expect_tx(&sm.kv_full[st], 2 * kFaKvTile);
+          const int row = pi.g * btot + pi.b0 + j * kFaBN;
           tma_load_2d(sm.kc[st], &kcmap, &sm.kv_full[st], 0, row);
           tma_load_2d(sm.vc[st], &vcmap, &sm.kv_full[st], 0, row);
           last_par[st] = (int)ph;
@@ -594,68 +602,65 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
         if (last_par[i] >= 0) mbar_wait(&sm.kv_full[i], (uint32_t)last_par[i]);
     }
   } else if (warp == kFaMmaWarp) {
-    // ---------------- MMA issuer: S_A(0), S_B(0); then per key tile j and side:
-    // O_side += P_side(j) Vc(j) once P_side(j) is in TMEM, then S_side(j+1) into the same columns
+    // ---------------- MMA issuer: S(0), S(1) of both sides; then per key tile j and
+    // side: O += P(j) Vc(j) once P(j) is in TMEM, then S(j + 2) into P(j)'s buffer
     if (lane == 0) {
-      const uint32_t id_s = idesc_bf16(kRows, kBN);             // S[rows, blocks] = Q Kc^T
+      const uint32_t id_s = idesc_bf16(kRows, kFaBN);            // S[rows, blocks] = Q Kc^T
       const uint32_t id_o = idesc_bf16(kRows, 64, false, true);  // O[rows, 64] += P[rows, blocks] Vc
-      uint32_t kv_count = 0, q_count = 0, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
+      uint32_t kv_count = 0, q_count = 0, g = 0, o_cnt = 0;  // g: steps of either side so far
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
         const PairInfo pi = pair_info(it, npairs, ppre, S, cu, bcu, G);
         const int qb = q_count % 2;
         if (!mbar_wait(&sm.q_full[qb], (q_count / 2) & 1)) { ok = false; break; }
         ++q_count;
-        const int nbt = (pi.nb + kBN - 1) / kBN;
-        auto issue_s = [&](int side, int st) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(tmem + side * kBN, sdesc_kmajor_sw128(sm.q[qb][side], 32 * k),
-                        sdesc_kmajor_sw128(sm.kc[st], 32 * k), id_s, k > 0);
-          mma_commit(&sm.s_full[side]);
-        };
-        if (nbt > 0) {
-          const int st0 = kv_count % kFaStages;
-          if (!mbar_wait(&sm.kv_full[st0], (kv_count / kFaStages) & 1)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(0, st0);
-          issue_s(1, st0);
-        }
-        for (int j = 0; j < nbt && ok; ++j) {
+        const int nbt = (pi.nb + kFaBN - 1) / kFaBN;
+        // S(j) of both sides from stage kv_count + j into buffer (g + j) % 2
+        auto issue_s = [&](int j) -> bool {
           const uint32_t kv_j = kv_count + j;
           const int st = kv_j % kFaStages;
+          if (!mbar_wait(&sm.kv_full[st], (kv_j / kFaStages) & 1)) return false;
+          tc_fence_after();
+          const int b = (g + j) & 1;
+#pragma unroll
           for (int side = 0; side < 2; ++side) {
-            if (!mbar_wait(&sm.p_full[side], p_cnt[side] & 1) ||
-                (j == 0 && !mbar_wait(&sm.o_empty[side], (o_cnt[side] & 1) ^ 1))) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ss(tmem + side * kFaSideCols + b * kFaBN, sdesc_kmajor_sw128(sm.q[qb][side], 32 * k),
+                          sdesc_kmajor_sw128(sm.kc[st], 32 * k), id_s, k > 0);
+            mma_commit(&sm.s_full[side][b]);
+          }
+          return true;
+        };
+        if (nbt > 0 && !issue_s(0)) { ok = false; break; }
+        if (nbt > 1 && !issue_s(1)) { ok = false; break; }
+        for (int j = 0; j < nbt && ok; ++j) {
+          const uint32_t gj = g + j;
+          const int b = gj & 1;
+          const int st = (kv_count + j) % kFaStages;
+#pragma unroll
+          for (int side = 0; side < 2; ++side) {
+            if (!mbar_wait(&sm.p_full[side][b], (gj >> 1) & 1) ||
+                (j == 0 && !mbar_wait(&sm.o_empty[side], (o_cnt & 1) ^ 1))) {
               ok = false;
               break;
             }
-            ++p_cnt[side];
             tc_fence_after();
-            const uint32_t tp = tmem + side * kBN, to = tmem + 2 * kBN + side * 64;
+            const uint32_t tp = tmem + side * kFaSideCols + b * kFaBN, to = tmem + side * kFaSideCols + 2 * kFaBN;
 #pragma unroll
-            for (int k = 0; k < kBN / 16; ++k)
-              mma_bf16_ts(to, tp + 8 * k, sdesc_mnmajor_sw128(sm.vc[st], 2048 * k, kTile), id_o, j > 0 || k > 0);
+            for (int k = 0; k < kFaBN / 16; ++k)
+              mma_bf16_ts(to, tp + 8 * k, sdesc_mnmajor_sw128(sm.vc[st], 2048 * k, kFaKvTile), id_o, j > 0 || k > 0);
             mma_commit(&sm.pv_done[side]);
-            if (j + 1 < nbt) {
-              const int st1 = (kv_j + 1) % kFaStages;
-              if (side == 0 && !mbar_wait(&sm.kv_full[st1], ((kv_j + 1) / kFaStages) & 1)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              issue_s(side, st1);
-            }
           }
           if (!ok) break;
           mma_commit(&sm.kv_empty[st]);
+          if (j + 2 < nbt && !issue_s(j + 2)) { ok = false; break; }
         }
         if (!ok) break;
         kv_count += nbt;
-        for (int side = 0; side < 2; ++side) {
-          mma_commit(&sm.o_full[side]);
-          ++o_cnt[side];
-        }
+        g += nbt;
+        for (int side = 0; side < 2; ++side) mma_commit(&sm.o_full[side]);
+        ++o_cnt;
         mma_commit(&sm.q_empty[qb]);
       }
       if (!ok) record_timeout(status, &sm.abort_flag);
@@ -667,37 +672,37 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
     const int side = warp / 4;
     const int r = threadIdx.x % 128;
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
-    const uint32_t tm_s = tmem + side * kBN + lane_off, tm_o = tmem + 2 * kBN + side * 64 + lane_off;
+    const uint32_t tbase = tmem + side * kFaSideCols + lane_off, tm_o = tbase + 2 * kFaBN;
     const float2 qs = make_float2(qs2, qs2);
-    uint32_t s_cnt = 0, pv_base = 0, o_cnt = 0;
+    uint32_t g = 0, o_cnt = 0;
     for (int it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
       const PairInfo pi = pair_info(it, npairs, ppre, S, cu, bcu, G);
       const int64_t t = (int64_t)pi.t0 + side * TPT + r / G;
       const int h = pi.g * G + r % G;
       const bool valid = t < pi.t_end;
-      const int nbt = (pi.nb + kBN - 1) / kBN;
+      const int nbt = (pi.nb + kFaBN - 1) / kFaBN;
       float m = -CUDART_INF_F, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nbt; ++j) {
-        if (!mbar_wait_warp(&sm.s_full[side], s_cnt & 1)) { ok = false; break; }
-        ++s_cnt;
+      for (int j = 0; j < nbt; ++j, ++g) {
+        const int b = g & 1;
+        if (!mbar_wait_warp(&sm.s_full[side][b], (g >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        float sv[kBN];
+        const uint32_t tm_s = tbase + b * kFaBN;
+        float sv[kFaBN];
 #pragma unroll
-        for (int c = 0; c < kBN; c += 32) tmem_ld32(tm_s + c, sv + c);
+        for (int c = 0; c < kFaBN; c += 32) tmem_ld32(tm_s + c, sv + c);
         tmem_ld_wait();
-        const int vcols = min(kBN, pi.nb - j * kBN);
-        if (vcols < kBN) {  // ragged last key tile: blocks past the sequence get p = 0
+        const int vcols = min(kFaBN, pi.nb - j * kFaBN);
+        if (vcols < kFaBN) {  // ragged last key tile: blocks past the sequence get p = 0
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) sv[c] = c < vcols ? sv[c] : -CUDART_INF_F;
+          for (int c = 0; c < kFaBN; ++c) sv[c] = c < vcols ? sv[c] : -CUDART_INF_F;
         }
-        // row max as 8 independent chains (a single chain of 127 dependent maxima would
-        // leave the two warps per scheduler waiting on its latency)
+        // row max as 8 independent chains
         float mx[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) mx[c] = sv[c];
 #pragma unroll
-        for (int c = 8; c < kBN; ++c) mx[c % 8] = fmaxf(mx[c % 8], sv[c]);
+        for (int c = 8; c < kFaBN; ++c) mx[c % 8] = fmaxf(mx[c % 8], sv[c]);
         const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * qs2;  // qs2 > 0
         float alpha = 1.f;
@@ -711,8 +716,8 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
           resc = true;
         }
         if (__any_sync(0xffffffffu, resc)) {
-          // O holds the sum of the products of tiles 0 .. j-1: wait for the last one, then scale
-          if (!mbar_wait_warp(&sm.pv_done[side], (pv_base + j - 1) & 1)) { ok = false; break; }
+          // O holds the sum of the products of steps .. g-1: wait for the last one, then scale
+          if (!mbar_wait_warp(&sm.pv_done[side], (g - 1) & 1)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
@@ -729,12 +734,12 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
         const float2 nm = make_float2(-m, -m);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int qq = 0; qq < kBN / 32; ++qq) {
+        for (int qq = 0; qq < kFaBN / 32; ++qq) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const float2 x = ffma2(make_float2(sv[32 * qq + c], sv[32 * qq + c + 1]), qs, nm);
-            const float2 p = 32 * qq < kFaPolyCols ? ex2_poly2(x) : ex2x2(x);
+            const float2 p = 32 * qq + c < kFaPolyCols ? ex2_poly2(x) : ex2x2(x);
             acc[(c / 2) % 4] = fadd2(acc[(c / 2) % 4], p);
             pk[c / 2] = pack2(p);
           }
@@ -744,13 +749,12 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[side]);
+        if (lane == 0) mbar_arrive(&sm.p_full[side][b]);
       }
       if (!ok) {
         record_timeout(status, &sm.abort_flag);
         break;
       }
-      pv_base += nbt;
       // O of the pair: wait for the last product, normalise, write o_cmp and lse
       if (!mbar_wait_warp(&sm.o_full[side], o_cnt & 1)) { record_timeout(status, &sm.abort_flag); break; }
       ++o_cnt;
@@ -1647,9 +1651,10 @@ __global__ void pair_plan_kernel(const int32_t* __restrict__ cu, int S, int G, i
 
 template <int G>
 cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_tiles_bound, cudaStream_t st) {
-  CUtensorMap qm, km, vm;
-  if (!map_q(&qm, a.q, a.N, a.hq, G) || !map_rows64(&km, a.kc, (int64_t)a.hkv * a.blk->count) ||
-      !map_rows64(&vm, a.vc, (int64_t)a.hkv * a.blk->count))
+  CUtensorMap qm, km, kmf, vmf;  // km: 128-block key tiles (selection pass); kmf, vmf: kFaBN (output pass)
+  const int64_t rows_kv = (int64_t)a.hkv * a.blk->count;
+  if (!map_q(&qm, a.q, a.N, a.hq, G) || !map_rows64(&km, a.kc, rows_kv) || !map_rows64(&kmf, a.kc, rows_kv, kFaBN) ||
+      !map_rows64(&vmf, a.vc, rows_kv, kFaBN))
     return cudaErrorInvalidValue;
   const float qs2 = a.scale * kLog2e;
   const int btot = (int)a.blk->count;
@@ -1670,7 +1675,7 @@ cudaError_t cmp_fwd_tc_g(const FwdArgs& a, const int32_t* tpre, int64_t total_ti
   const int sms = num_sms();
   const int64_t pairs = ((total_tiles_bound + 1) / 2 + a.S) * a.hkv;
   const int g1 = (int)(pairs < sms ? (pairs > 0 ? pairs : 1) : sms);
-  SSA_LAUNCH("cmp_fa_tc_kernel", cmp_fa_tc_kernel<G>, g1, kFaThreads, smem_bytes_fa(), st, qm, km, vm, a.cu_seqlens,
+  SSA_LAUNCH("cmp_fa_tc_kernel", cmp_fa_tc_kernel<G>, g1, kFaThreads, smem_bytes_fa(), st, qm, kmf, vmf, a.cu_seqlens,
              a.blk->cu, a.tiles_pre, a.S, a.N, a.hq, a.hkv, btot, qs2, a.o_branch, a.lse, a.status);
   if (!a.sel_given) {  // a given selection needs no scores
     const int64_t tiles = total_tiles_bound * a.hkv;
