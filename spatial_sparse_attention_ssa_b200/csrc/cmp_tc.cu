@@ -477,8 +477,9 @@ __device__ void warp_topk_groups(const float* imp, const float* gm, int nb, int 
 // per probability, unbiased) moves it by about 1e-4 at the benchmark's sizes, against
 // the sums over millions of rows in the key gradients.  O (TMEM) is rescaled only when
 // a row's max grows by more than 2^8 since it was last fixed, so p stays below 2^8
-// otherwise.  The exponentials of a quarter of each key tile's blocks run on the FMA
-// pipe (ex2_poly2), the rest on the MUFU.  Steps are counted per side across the
+// otherwise.  All exponentials run on the MUFU: with S double-buffered the softmax
+// warps are busy enough that moving a share to the FMA pipe (ex2_poly2) costs more
+// issue slots than it frees MUFU cycles.  Steps are counted per side across the
 // CTA's pairs (g), which sets the buffer (g % 2) and the barrier phases.
 // ---------------------------------------------------------------------------
 constexpr int kFaBN = 96;                    // compressed blocks per key tile
@@ -489,7 +490,8 @@ constexpr int kFaMmaWarp = kFaSoftmaxWarps + 1;
 constexpr int kFaThreads = 32 * (kFaSoftmaxWarps + 2);
 constexpr int kFaKvTile = kFaBN * 128;       // bytes of a [kFaBN, 64] bf16 tile
 constexpr int kFaSideCols = 2 * kFaBN + 64;  // TMEM per side: S buffers 0 and 1, O
-constexpr int kFaPolyCols = 24;              // blocks of a key tile whose exponentials use the FMA pipe
+constexpr int kFaPolyCols = 0;               // blocks of a key tile whose exponentials use the FMA pipe
+                                             // (at 131072 tokens: 0 -> 4.24 ms, 16 -> 4.42, 24 -> 4.49, 48 -> 4.76)
 constexpr float kFaRescaleLog2 = 8.f;
 static_assert(2 * kFaSideCols <= 512 && kFaBN % 32 == 0, "TMEM");
 
