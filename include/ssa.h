@@ -27,7 +27,11 @@
  *     allocates or frees device memory.
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
  *     legacy default stream).  Only ssa_bin, ssa_bin_noalloc, ssa_cross_forward,
- *     ssa_cross_backward and ssa_get_device_status synchronise that stream.
+ *     ssa_cross_backward and ssa_get_device_status synchronise that stream; they
+ *     read their few result ints through 64 bytes of pinned, mapped host memory
+ *     per calling thread (allocated on the thread's first such call, kept until
+ *     exit) that a one-thread kernel writes, so the read never waits in a copy
+ *     engine's queue behind other streams' bulk transfers.
  *   - Errors are returned as ssa_status codes; nothing aborts or throws across
  *     the ABI.  Argument errors are detected on the host before any launch.
  *   - N = number of tokens (all sequences), S = number of sequences,

@@ -279,9 +279,9 @@ SSA_API ssa_status ssa_get_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int* sp = status_ptr();
   if (!sp) return SSA_ERR_CUDA;
-  int h = 0;
-  if (cudaMemcpyAsync(&h, sp, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSA_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SSA_ERR_CUDA;
+  int32_t hv[3];
+  if (ssa::read_ints_to_host(sp, nullptr, nullptr, hv, st) != cudaSuccess) return SSA_ERR_CUDA;
+  const int h = hv[0];
   if (h) {
     cudaMemsetAsync(sp, 0, sizeof(int), st);
     cudaStreamSynchronize(st);
@@ -340,14 +340,11 @@ SSA_API ssa_status ssa_bin(const int32_t* coords, const int32_t* cu_seqlens, int
     e = ssa::bin_partition(coords, cu_seqlens, S, N, R, m_win, win, d_counts + 1, ws, sp, st);
   }
   if (e != cudaSuccess) return SSA_ERR_CUDA;
-  int32_t h_counts[2] = {0, 0};
-  int h_status = 0;
-  e = cudaMemcpyAsync(h_counts, d_counts, sizeof(h_counts), cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(&h_status, sp, sizeof(int), cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return SSA_ERR_CUDA;
-  blk->count = h_counts[0];
-  win->count = h_counts[1];
+  int32_t hv[3];
+  if (ssa::read_ints_to_host(d_counts, d_counts + 1, sp, hv, st) != cudaSuccess) return SSA_ERR_CUDA;
+  blk->count = hv[0];
+  win->count = hv[1];
+  const int h_status = hv[2];
   if (h_status) {
     cudaMemsetAsync(sp, 0, sizeof(int), st);
     cudaStreamSynchronize(st);
@@ -543,10 +540,9 @@ ssa_status cross_prepare(const ssa_params* p, const int32_t* q_cu, int32_t S, in
   int* bad = reinterpret_cast<int*>(static_cast<char*>(extra) + align256(sizeof(float) * 3 * (size_t)Nq * p->hq));
   if (cudaMemsetAsync(bad, 0, sizeof(int), st) != cudaSuccess) return SSA_ERR_CUDA;
   if (ssa::cross_prep(gates, Nq * p->hq, *gates3, q_cu, blk->cu, S, bad, st) != cudaSuccess) return SSA_ERR_CUDA;
-  int h = 0;
-  if (cudaMemcpyAsync(&h, bad, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSA_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SSA_ERR_CUDA;
-  return h ? SSA_ERR_INVALID_ARG : SSA_OK;
+  int32_t hv[3];
+  if (ssa::read_ints_to_host(bad, nullptr, nullptr, hv, st) != cudaSuccess) return SSA_ERR_CUDA;
+  return hv[0] ? SSA_ERR_INVALID_ARG : SSA_OK;
 }
 
 }  // namespace

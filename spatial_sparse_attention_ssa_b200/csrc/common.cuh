@@ -122,6 +122,11 @@ cudaError_t radix_sort_pairs(uint64_t* keys_a, int32_t* vals_a, uint64_t* keys_b
 
 // Binning of one partition (see ssa_bin).
 size_t bin_ws_bytes(int32_t S, int64_t N);
+// Synchronises `st` and reads up to three device ints (null sources read as 0) through
+// a pinned, mapped host buffer written by a kernel: no copy engine is involved.
+cudaError_t read_ints_to_host(const int32_t* s0, const int32_t* s1, const int32_t* s2, int32_t* out,
+                              cudaStream_t st);
+
 cudaError_t bin_partition(const int32_t* coords, const int32_t* cu_seqlens, int32_t S, int64_t N,
                           int32_t R, int32_t m, ssa_partition* out, int32_t* d_count, void* ws,
                           int* d_status, cudaStream_t st);

@@ -73,9 +73,8 @@ extern "C" SSA_API ssa_status ssa_bin_noalloc(const int32_t* coords, const int32
   if (e == cudaSuccess) e = ssa::bin_partition(coords, cu_seqlens, S, N, R, m_win, win, d_counts + 1, scratch, d_status, st);
   if (e != cudaSuccess) return SSA_ERR_CUDA;
   int32_t h[3] = {0, 0, 0};
-  e = cudaMemcpyAsync(h, d_counts, sizeof(h), cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return SSA_ERR_CUDA;
+  if (ssa::read_ints_to_host(d_counts, d_counts + 1, reinterpret_cast<const int32_t*>(d_status), h, st) != cudaSuccess)
+    return SSA_ERR_CUDA;
   blk->count = h[0];
   win->count = h[1];
   if (h[2] & ssa::kStatusTimeout) return SSA_ERR_TIMEOUT;
