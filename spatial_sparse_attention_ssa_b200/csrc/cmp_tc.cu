@@ -793,7 +793,7 @@ __global__ void __launch_bounds__(kFaThreads, 1) cmp_fa_tc_kernel(
 // exponentials stay on the MUFU (kSelPolyRows = 0): moving a share to the FMA pipe
 // (ex2_poly2) measured slower here.
 // ---------------------------------------------------------------------------
-constexpr int kSelStages = 4;           // Kc ring depth
+constexpr int kSelStages = 6;           // Kc ring depth (4.51 ms at 4, 4.38 at 6, at 131072 tokens)
 constexpr int kSelPolyRows = 0;  // rows of a key tile whose exponentials use the FMA pipe (at 131072 tokens:
                                   // 0 -> 4.87 ms, a quarter -> 5.12, a half -> 5.46)
 
