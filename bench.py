@@ -183,7 +183,7 @@ def kernel_work(w, blk_ptr, blk_cu, win_ptr, sel):
     needs, counted once per stage: forward 6d for the compressed branch (S for the
     normaliser, S again for the selection's final probabilities, P.V) and 4d for
     the others; backward 10d (S, dP, dQ, dK, dV).  Exponentials per score: 2 in the
-    compressed forward (lse pass, output pass), 1 elsewhere.  Per kernel the same
+    compressed forward (flash pass, selection pass), 1 elsewhere.  Per kernel the same
     count covers the contractions that kernel performs; the bf16 low-part products,
     masked tile padding and the backward's second S / dP are overhead, not work.
     Memory kernels count the bytes they must move.

@@ -7,16 +7,19 @@
 // heads of a GQA group (LSRM, shuwu5.cn, "阶段一").
 //
 // A row tile is 128 query rows = (128/G tokens) x (G heads of one KV group),
-// loaded by one 3D TMA box from Q [N, Hq, 64].  A key tile is 128 compressed
-// blocks of Kc/Vc [Hkv, B, 64] (2D TMA, 128-byte swizzle).
+// loaded by one 3D TMA box from Q [N, Hq, 64].  A key tile is a run of compressed
+// blocks of Kc/Vc [Hkv, B, 64] (2D TMA, 128-byte swizzle): 96 in the output pass,
+// 128 in the selection pass and the dK/dV kernel, 64 in the dQ kernel.
 //
-//   output pass (cmp_fa_tc):     flash attention, thread = row: S = Q Kc^T, online
-//                                softmax, P (bf16 high + low) back into TMEM as the
-//                                operand of O += P Vc -> o_cmp and lse.
+//   output pass (cmp_fa_tc):     flash attention, thread = row: S = Q Kc^T
+//                                (double-buffered), online softmax, P (one bf16 per
+//                                block) back into TMEM as the operand of O += P Vc
+//                                -> o_cmp and lse.
 //   selection pass (cmp_sel_tc): S^T = Kc Q^T, thread = block: p = exp2(s - lse)
 //                                with the final lse, summed over the G heads of a
 //                                token; a warpgroup picks each token's top-k.
-//   backward (cmp_bwd_dq_tc, cmp_bwd_dkv_tc): dQ by rows, dKc / dVc by blocks.
+//   backward (cmp_bwd_dq_tc, cmp_bwd_dkv_tc): dQ by rows (bf16), dKc / dVc by
+//                                blocks (fp16 operands, from to_f16_kernel).
 //
 // Roles per CTA: compute warps (thread i <-> TMEM lane i), one warp issuing TMA
 // loads, one issuing tcgen05.mma.  Every wait is bounded; on a timeout the kernel
